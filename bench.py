@@ -1,0 +1,478 @@
+"""Benchmark of the paged KV-cache decode step on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--config NAME]
+
+Default workload: the Llama-2-7B-shaped single-layer decode batch (64
+sequences, 32 heads = 32 KV heads, head_dim 128, block 16, context U[128,
+2048], fp16).  One step = reshape_and_cache of the 64 new tokens, then
+paged decode attention (decode kernel + log-sum-exp merge) over all 64
+sequences, on inputs already resident in HBM (the pools, 1.25 GB each, are
+far larger than the 126 MB L2).  ``value`` = decode tokens (sequences) per
+second over all ranks; multi-GPU runs are independent replicas (weak
+scaling, no collective on the data path).
+
+Other ``--config`` values time the remaining named workloads for the
+report: gqa70b_decode_bf16 (80 layers per step), shared_prefix_decode_f16,
+mixed_step_bf16 (append + chunked prefill + decode).
+
+``--impl reference`` times the CPU oracle (double precision, one thread) on
+a bounded sample of the same workload: there is no runnable reference
+implementation of this path.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "paged decode attention tokens/s and KV GB/s as % of B200 HBM peak (1 GPU)"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return p, "measured"
+    except (OSError, ValueError):
+        return FALLBACK_PEAKS, "fallback"
+
+
+# ----------------------------------------------------------------------------- workloads as timed steps
+
+class DecodeStep:
+    """reshape_and_cache + paged_attention_decode over every layer of a DecodeWorkload."""
+
+    def __init__(self, w, layers_per_step=None):
+        import paged_kv_cache_409_b200 as pkv
+        self.pkv, self.w = pkv, w
+        dev = w.queries[0].device
+        self.bt = torch.from_numpy(w.block_tables).to(dev)
+        self.cl = torch.from_numpy(w.context_lens.astype(np.int32)).to(dev)
+        self.sm = torch.from_numpy(w.slot_mapping.astype(np.int64)).to(dev)
+        self.layers = layers_per_step or w.num_layers
+        self.outs = [torch.empty_like(q) for q in w.queries]
+        self.part = pkv.decode_partition_size(w.num_seqs, w.num_kv_heads, w.head_dim, w.block_size,
+                                              w.max_context_len, w.dtype)
+        need = pkv.decode_workspace_size(w.num_seqs, w.num_q_heads, w.head_dim, w.max_context_len, self.part)
+        self.ws = torch.empty(max(need, 16), dtype=torch.uint8, device=dev)
+        self.parts = -(-w.max_context_len // self.part) if self.part else 1
+        t = w.queries[0].element_size()
+        self.kv_bytes = 2 * int(w.context_lens.astype(np.int64).sum()) * w.num_kv_heads * w.head_dim * t
+        nblocks = int(((w.context_lens.astype(np.int64) + w.block_size - 1) // w.block_size).sum())
+        # algorithmic bytes of one decode call: K/V once, q, out, block ids, lengths
+        self.decode_bytes = self.kv_bytes + 2 * w.queries[0].numel() * t + 4 * nblocks + 4 * w.num_seqs
+        self.tokens = w.num_seqs  # one generated token per sequence per step
+
+    def launches_per_step(self):
+        return self.layers * (2 + (1 if self.parts > 1 else 0))
+
+    def e2e_plan(self):
+        w = self.w
+        pairs = []
+        for i in range(self.layers):
+            l = i % w.num_layers
+            pairs += [(w.queries[l], pinned(w.queries[l])), (w.new_keys[l], pinned(w.new_keys[l])),
+                      (w.new_values[l], pinned(w.new_values[l]))]
+        pairs += [(self.bt, pinned(self.bt)), (self.cl, pinned(self.cl)), (self.sm, pinned(self.sm))]
+        outs = [(self.outs[i % w.num_layers], pinned(self.outs[i % w.num_layers])) for i in range(self.layers)]
+        return E2EPlan(self, pairs, outs)
+
+    def append(self, l):
+        w = self.w
+        self.pkv.reshape_and_cache(w.new_keys[l], w.new_values[l], w.key_caches[l], w.value_caches[l], self.sm)
+
+    def attend(self, l):
+        w = self.w
+        self.pkv.paged_attention_decode(self.outs[l], w.queries[l], w.key_caches[l], w.value_caches[l], self.bt,
+                                        self.cl, w.scale, w.max_context_len, partition_size=self.part,
+                                        workspace=self.ws)
+
+    def run(self, timer=None, step=0):
+        for i in range(self.layers):
+            l = (step * self.layers + i) % self.w.num_layers
+            self.append(l)
+            if timer:
+                timer.begin()
+            self.attend(l)
+            if timer:
+                timer.end()
+
+
+class E2EPlan:
+    """Per step: copy the step's inputs from pinned host memory, run the step
+    through the public API, copy its result back to pinned host memory."""
+
+    def __init__(self, step, pairs, outs):
+        self.step, self.pairs, self.outs = step, pairs, outs  # pairs: (device dst, pinned src)
+        self.h2d = sum(src.numel() * src.element_size() for _, src in pairs)
+        self.d2h = sum(dst.numel() * dst.element_size() for _, dst in outs)
+
+    def run(self, i):
+        for dst, src in self.pairs:
+            dst.copy_(src, non_blocking=True)
+        self.step.run(step=i)
+        for src, dst in self.outs:
+            dst.copy_(src, non_blocking=True)
+
+
+def pinned(t):
+    return t.detach().cpu().pin_memory()
+
+
+class MixedStep(DecodeStep):
+    """Continuous-batching step: append all tokens, chunked prefill, decode."""
+
+    def __init__(self, m):
+        super().__init__(m.decode)
+        self.m = m
+        dev = m.decode.queries[0].device
+        self.aslots = torch.from_numpy(m.append_slots).to(dev)
+        self.cbt = torch.from_numpy(m.chunk_tables).to(dev)
+        self.csl = torch.from_numpy(m.seq_lens).to(dev)
+        self.qsl = torch.from_numpy(m.query_start_loc).to(dev)
+        self.pout = torch.empty_like(m.chunk_query)
+        self.prefill_tokens = int(m.chunk_lens.sum())
+        Hq, D = m.chunk_query.shape[1:]
+        n, c0 = m.chunk_lens.astype(np.int64), m.chunk_c0.astype(np.int64)
+        self.prefill_flops = int(4 * D * Hq * np.sum(n * c0 + n * (n + 1) // 2))
+
+    def launches_per_step(self):
+        return 3 + (1 if self.parts > 1 else 0)
+
+    def e2e_plan(self):
+        m, w = self.m, self.w
+        pairs = [(t, pinned(t)) for t in (m.chunk_query, w.queries[0], m.append_keys, m.append_values, self.aslots,
+                                          self.cbt, self.csl, self.qsl, self.bt, self.cl)]
+        outs = [(self.pout, pinned(self.pout)), (self.outs[0], pinned(self.outs[0]))]
+        return E2EPlan(self, pairs, outs)
+
+    def run(self, timer=None, step=0):
+        m, w = self.m, self.w
+        self.pkv.reshape_and_cache(m.append_keys, m.append_values, w.key_caches[0], w.value_caches[0], self.aslots)
+        self.pkv.paged_attention_prefill_chunk(self.pout, m.chunk_query, w.key_caches[0], w.value_caches[0],
+                                               self.cbt, self.csl, self.qsl, int(m.chunk_lens.max()), w.scale)
+        if timer:
+            timer.begin()
+        self.attend(0)
+        if timer:
+            timer.end()
+
+
+def make_step(name, device, rank):
+    from paged_kv_cache_409_b200 import workloads
+    if name == "llama7b_decode_f16":
+        return DecodeStep(workloads.llama7b_decode_f16(device=device, seed=1002 + rank)), "llama7b_decode_f16"
+    if name == "tiny_decode_f32":
+        return DecodeStep(workloads.tiny_decode_f32(device=device)), name
+    if name == "gqa70b_decode_bf16":
+        free, _ = torch.cuda.mem_get_info()
+        per_layer = 1.75e9  # pools of one layer (~1.62 GB) plus headroom
+        layers = int(max(1, min(80, (free - 8e9) // per_layer)))
+        w = workloads.gqa70b_decode_bf16(device=device, num_layers=layers, seed=1003 + rank)
+        return DecodeStep(w, layers_per_step=80), f"gqa70b_decode_bf16 ({layers} distinct layer caches cycled)"
+    if name == "shared_prefix_decode_f16":
+        sp = workloads.shared_prefix_decode_f16(device=device, seed=1004 + rank)
+        st = DecodeStep(sp.step)
+        kc, vc = sp.step.key_caches[0], sp.step.value_caches[0]
+        st.pkv.copy_blocks([kc], [vc], torch.from_numpy(sp.cow_pairs).to(device))
+        st.pkv.reshape_and_cache(sp.private_keys, sp.private_values, kc, vc,
+                                 torch.from_numpy(sp.private_slots).to(device))
+        return st, name
+    if name == "mixed_step_bf16":
+        return MixedStep(workloads.mixed_step_bf16(device=device, seed=1005 + rank)), name
+    raise SystemExit(f"unknown config {name}")
+
+
+# ----------------------------------------------------------------------------- timing helpers
+
+class EventTimer:
+    """CUDA events around one unit per step, on the launching stream."""
+
+    def __init__(self):
+        self.pairs = []
+
+    def begin(self):
+        e = torch.cuda.Event(enable_timing=True)
+        e.record()
+        self.pairs.append([e, None])
+
+    def end(self):
+        e = torch.cuda.Event(enable_timing=True)
+        e.record()
+        self.pairs[-1][1] = e
+
+    def mean_ms(self):
+        return statistics.fmean(a.elapsed_time(b) for a, b in self.pairs)
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle samples while the timed region runs."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index):
+        self.proc, self.path = None, None
+        try:
+            bus = torch.cuda.get_device_properties(device_index).pci_bus_id
+        except Exception:
+            bus = None
+        self.bus = bus
+
+    def start(self):
+        if self.bus is None:
+            return
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.bus}", f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "50"],
+                                         stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if not self.proc:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) >= 9:
+                    rows.append(parts)
+        os.unlink(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+
+        def num(x):
+            try:
+                return float(x)
+            except ValueError:
+                return None
+        sm = [num(r[1]) for r in rows if num(r[1]) is not None]
+        smax = [num(r[2]) for r in rows if num(r[2]) is not None]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i, v in enumerate(r[5:9]) if v.lower().startswith("active")})
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(smax) if smax else None,
+                "reasons": reasons, "samples": len(rows)}
+
+
+def dist_setup(n_gpus):
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if ws > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    else:
+        torch.cuda.set_device(0)
+    return ws, rank, local
+
+
+def barrier(ws):
+    if ws > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(x, ws):
+    if ws == 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ----------------------------------------------------------------------------- CPU baseline (oracle)
+
+def oracle_sample(step, budget_s, max_seqs=None):
+    """Time the oracle (append + decode) on whole steps or a sequence sample, host cores."""
+    import oracle
+    w = step.w
+    orc = oracle.get()
+    S = w.num_seqs
+    seqs = np.arange(S if max_seqs is None else min(S, max_seqs))
+    sys.path.insert(0, os.path.join(ROOT, "tests"))
+    from parity_helpers import compact_tables, snapshot_blocks
+    used, bt = compact_tables(w.block_tables[seqs], w.context_lens[seqs], w.block_size)
+    kn, code = oracle.storage(snapshot_blocks(w.key_caches[0], used))
+    vn, _ = oracle.storage(snapshot_blocks(w.value_caches[0], used))
+    kn, vn = kn.copy(), vn.copy()
+    B = w.block_size
+    remap = {int(b): i for i, b in enumerate(used)}
+    slots = np.array([remap[int(s) // B] * B + int(s) % B for s in w.slot_mapping[seqs]], dtype=np.int64)
+    idx = torch.from_numpy(seqs).to(w.queries[0].device)
+    q = oracle.storage(w.queries[0][idx])[0]
+    nk = oracle.storage(w.new_keys[0][idx])[0]
+    nv = oracle.storage(w.new_values[0][idx])[0]
+    lens = w.context_lens[seqs]
+    done, t0 = 0, time.perf_counter()
+    while True:
+        orc.reshape_and_cache(nk, nv, kn, vn, slots, code)
+        orc.paged_attention_decode(q, kn, vn, bt, lens, w.scale, code)
+        done += 1
+        el = time.perf_counter() - t0
+        if el >= budget_s:
+            break
+    return len(seqs) * done / el, done, len(seqs), el
+
+
+# ----------------------------------------------------------------------------- main
+
+def run_reference(args, ws, rank):
+    """The oracle as it stands, on the host cores, on a bounded sample of the workload."""
+    if rank != 0:
+        return
+    dev = "cuda" if torch.cuda.is_available() else "cpu"
+    step, cname = make_step(args.config, dev, 0)
+    w = step.w
+    sample = min(w.num_seqs, 8)
+    times = []
+    for i in range(args.warmup + args.steps):
+        v, done, n, el = oracle_sample(step, 0.0, max_seqs=sample)
+        if i >= args.warmup:
+            times.append(el)
+    per = statistics.fmean(times)
+    value = sample / per
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": per * 1e3, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": cname, "sample_seqs": sample},
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": 1, "kind": "oracle",
+                             "sample": f"append + decode of the first {sample} of {w.num_seqs} sequences per step"},
+            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--config", default="llama7b_decode_f16")
+    ap.add_argument("--cpu-budget", type=float, default=12.0, help="seconds of oracle time for cpu_baseline")
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)
+
+    ws, rank, local = dist_setup(args.gpus)
+    if args.impl == "reference":
+        run_reference(args, ws, rank)
+        if ws > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+        return
+
+    import paged_kv_cache_409_b200 as pkv
+    pkv.load_library()
+    dev = torch.device("cuda", torch.cuda.current_device())
+    step, cname = make_step(args.config, dev, rank)
+    torch.cuda.synchronize()
+
+    # warm-up, then exactly K timed steps between barriers
+    clocks = ClockSampler(torch.cuda.current_device())
+    clocks.start()
+    for i in range(args.warmup):
+        step.run(step=i)
+    torch.cuda.synchronize()
+    barrier(ws)
+    timer = EventTimer()
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record()
+    for i in range(args.steps):
+        step.run(timer=timer, step=i)
+    t1.record()
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    barrier(ws)
+    ms_total = max_over_ranks(t0.elapsed_time(t1), ws)
+    ms_step = ms_total / args.steps
+    unit_ms = max_over_ranks(timer.mean_ms(), ws)
+    assert pkv.get_device_error() == 0, "device error word set during the run"
+
+    # end to end through the public API: pinned host inputs in, result out, every step
+    w = step.w
+    e2e = step.e2e_plan()
+    e2e_steps = max(3, min(args.steps, 50))
+    for i in range(3):
+        e2e.run(i)
+    torch.cuda.synchronize()
+    barrier(ws)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for i in range(e2e_steps):
+        e2e.run(i)
+    e1.record()
+    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1) / e2e_steps, ws)
+    barrier(ws)
+
+    pk, pk_kind = peaks()
+    hbm = float(pk["hbm_gbs"])
+    tokens_per_step = step.tokens
+    value = ws * tokens_per_step / (ms_step / 1e3)
+    achieved = step.decode_bytes / (unit_ms / 1e3) / 1e9
+    line = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": ws, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": {torch.float16: "f16", torch.bfloat16: "bf16", torch.float32: "f32"}[w.dtype],
+        "data": "synthetic",
+        "config": {"workload": cname, "num_seqs": w.num_seqs, "num_q_heads": w.num_q_heads,
+                   "num_kv_heads": w.num_kv_heads, "head_dim": w.head_dim, "block_size": w.block_size,
+                   "layers_per_step": step.layers, "partition_size": step.part,
+                   "l2": "inputs larger than L2 (K/V pools %.2f GB per layer)" % (
+                       2 * w.key_caches[0].numel() * w.key_caches[0].element_size() / 1e9),
+                   "parallelism": f"replicas x{ws}"},
+        "kv_gbs": step.kv_bytes * step.layers / (ms_step / 1e3) / 1e9,
+        "roofline": {"bound": "hbm", "kernel": "paged_attention_decode (decode + merge kernels)",
+                     "achieved": achieved, "peak": hbm, "peak_kind": pk_kind, "unit": "GB/s",
+                     "frac": achieved / hbm, "frac_of_8000_nominal": achieved / 8000.0, "traffic": None},
+        "e2e": {"value": ws * tokens_per_step / (e2e_ms / 1e3), "unit": "tokens/s",
+                "h2d_bytes_per_step": e2e.h2d, "d2h_bytes_per_step": e2e.d2h, "ms_per_step": e2e_ms},
+        "gpu_launches": step.launches_per_step() * args.steps,
+        "clocks": clk,
+    }
+    if isinstance(step, MixedStep):
+        line["prefill_tokens_per_s"] = ws * step.prefill_tokens / (ms_step / 1e3)
+        line["prefill_flops_per_step"] = step.prefill_flops
+    if rank == 0 and ws == 1 and args.cpu_budget > 0 and args.config != "gqa70b_decode_bf16":
+        v, done, n, el = oracle_sample(step, args.cpu_budget, max_seqs=None if w.num_seqs <= 64 else 16)
+        line["cpu_baseline"] = {"value": v, "unit": "tokens/s", "cores": 1, "kind": "oracle",
+                                "sample": f"{done} x (append + decode of {n} sequences), {el:.1f} s, 1 thread"}
+    elif rank == 0 and ws == 1 and args.cpu_budget > 0:
+        v, done, n, el = oracle_sample(step, args.cpu_budget, max_seqs=16)
+        line["cpu_baseline"] = {"value": v / 80.0, "unit": "tokens/s (80-layer steps)", "cores": 1,
+                                "kind": "oracle",
+                                "sample": f"{done} x one layer of {n} sequences, {el:.1f} s, 1 thread; /80 layers"}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if ws > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

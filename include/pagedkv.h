@@ -1,0 +1,205 @@
+/*
+ * pagedkv.h -- C ABI of libpagedkv.so, B200 (sm_100a) kernels for attention
+ * over a paged KV cache.
+ *
+ * Data model (vLLM case-study page "vLLM 与 PagedAttention", section 二,
+ * "PagedAttention 的解法" and the kernel sketch under "注意力计算改造"):
+ *   - K and V live in two pools of fixed-size physical blocks, each laid out
+ *     [num_blocks, block_size, num_kv_heads, head_dim], row-major, elements of
+ *     one type (pkv_dtype).  Block size 16 is the pages' default.
+ *   - Each sequence owns a row of block_tables [num_seqs, max_blocks_per_seq]
+ *     (int32): entry i is the physical block that holds its tokens
+ *     [i * block_size, (i + 1) * block_size).
+ *   - A token at position p of a sequence sits in physical slot
+ *     block_tables[s][p / block_size] * block_size + p % block_size; in the
+ *     pool layout that slot is row `slot` of a [num_blocks * block_size,
+ *     num_kv_heads, head_dim] view.
+ *
+ * Conventions for every call:
+ *   - Pointers named as device pointers must be device memory of the current
+ *     CUDA device (or managed memory); host pointers are read before the call
+ *     returns.  The caller owns every buffer; the library allocates nothing.
+ *   - Every device buffer must be 16-byte aligned and densely packed in the
+ *     layout stated.
+ *   - Calls are asynchronous on `stream` (a cudaStream_t; NULL = the legacy
+ *     default stream).  A return of PKV_OK means the work was launched.
+ *   - Host-detectable errors return before anything is launched: null
+ *     pointers, negative sizes, unsupported head_dim / block_size / dtype /
+ *     head grouping, misaligned pointers, a workspace that is too small.
+ *   - Table contents are not read by the host.  Kernels check every block id,
+ *     slot and length they use; a bad one is skipped (its output is then
+ *     unspecified) and a bit is set in the per-device error word read by
+ *     pkv_get_device_error().  No kernel traps or faults on bad table data.
+ *   - With the environment variable PKV_CHECK=1 the host additionally copies
+ *     the tables to the host, validates them and returns PKV_ERANGE before
+ *     launching (this synchronises the stream; for debugging only).
+ */
+#ifndef PAGEDKV_H
+#define PAGEDKV_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef void* pkv_stream_t; /* a cudaStream_t */
+
+typedef enum { PKV_F32 = 0, PKV_F16 = 1, PKV_BF16 = 2 } pkv_dtype;
+
+typedef enum {
+    PKV_OK = 0,
+    PKV_EINVAL = -1,         /* null pointer, negative size, misaligned pointer */
+    PKV_EUNSUPPORTED = -2,   /* head_dim / block_size / dtype / grouping not built */
+    PKV_ERANGE = -3,         /* PKV_CHECK=1 found a table entry out of range */
+    PKV_ECUDA = -4,          /* a CUDA runtime / driver call failed */
+    PKV_EWORKSPACE = -5      /* workspace missing or smaller than required */
+} pkv_status;
+
+/* Bits of the device error word. */
+#define PKV_DEVERR_BLOCK_ID   0x1u  /* block table entry outside [0, num_blocks) */
+#define PKV_DEVERR_SLOT       0x2u  /* slot_mapping entry >= num_blocks * block_size */
+#define PKV_DEVERR_LENGTH     0x4u  /* context / sequence length beyond the table, or a bad chunk */
+#define PKV_DEVERR_PAIR       0x8u  /* copy_blocks pair outside [0, num_blocks) */
+#define PKV_DEVERR_TIMEOUT    0x10u /* a bounded wait on an asynchronous copy or MMA gave up */
+
+/* Human-readable name of a pkv_status. */
+const char* pkv_status_string(int status);
+
+/* Text of the last CUDA error seen by this thread inside the library ("" if none). */
+const char* pkv_last_cuda_error(void);
+
+/*
+ * reshape_and_cache -- write new tokens' K and V into their physical slots.
+ * Source: case-study page section 二 (blocks are taken on demand: "the 7th
+ * block is requested only when generation reaches the 100th token") and the
+ * PagedKVCache sketch on the 298.name page; the slot of a position is the
+ * block table arithmetic above, precomputed by the host.
+ *
+ *   key, value      device, [num_tokens, num_kv_heads, head_dim]
+ *   key_cache,
+ *   value_cache     device, [num_blocks, block_size, num_kv_heads, head_dim]
+ *   slot_mapping    device int64 [num_tokens]; slot_mapping[t] < 0 marks a
+ *                   padding token that is skipped; a slot >= num_blocks *
+ *                   block_size is skipped and sets PKV_DEVERR_SLOT.
+ * Bits are copied verbatim (bit-exact).  Two tokens with the same slot race.
+ * num_tokens == 0 is a no-op.
+ */
+int pkv_reshape_and_cache(const void* key, const void* value, void* key_cache, void* value_cache,
+                          const int64_t* slot_mapping, int64_t num_tokens, int num_kv_heads,
+                          int head_dim, int block_size, int64_t num_blocks, int dtype,
+                          pkv_stream_t stream);
+
+/*
+ * copy_blocks -- copy-on-write of shared blocks.  Source: case-study page
+ * section 二 (requests with a common prefix point at the same physical blocks
+ * and copy on write) and the guide page "Copy-on-Write" (shared blocks are
+ * copied only once a request diverges).
+ *
+ *   key_caches,
+ *   value_caches    HOST arrays of num_layers device pointers, each a pool
+ *                   [num_blocks, block_size, num_kv_heads, head_dim]
+ *   src_dst_pairs   device int64 [num_pairs, 2]: (src, dst) block ids
+ *   block_bytes     bytes of one block of one pool (block_size *
+ *                   num_kv_heads * head_dim * element size), multiple of 16
+ * For every pair and every layer, K block dst and V block dst become bit
+ * copies of block src.  Destinations must be distinct and no destination may
+ * be a source (the result is otherwise unspecified; PKV_CHECK=1 rejects it).
+ * An id outside [0, num_blocks) is skipped and sets PKV_DEVERR_PAIR.
+ */
+int pkv_copy_blocks(void* const* key_caches, void* const* value_caches, int num_layers,
+                    const int64_t* src_dst_pairs, int64_t num_pairs, int64_t block_bytes,
+                    int64_t num_blocks, pkv_stream_t stream);
+
+/*
+ * Decode attention over the paged cache, one query token per sequence.
+ * Source: case-study page section 二 "注意力计算改造" (K/V are loaded block by
+ * block through the block table and each block's attention is accumulated;
+ * kernel sketch with cache layout [num_blocks, block_size, num_heads,
+ * d_head]) and the guide page "KV Cache 是什么" (each new token attends to all
+ * cached tokens).  Computed: for sequence s and query head h, with KV head
+ * g = h / (num_q_heads / num_kv_heads),
+ *     out[s][h] = sum_{j < context_lens[s]} softmax_j(scale * q[s][h] . K_j) V_j
+ * where K_j / V_j are read at slot(block_tables[s], j).  Accumulation is fp32
+ * (online max / sum); inputs and output are `dtype`.  context_lens[s] == 0
+ * gives a zero row.
+ *
+ *   out             device [num_seqs, num_q_heads, head_dim], dtype
+ *   query           device [num_seqs, num_q_heads, head_dim], dtype
+ *   block_tables    device int32 [num_seqs, max_blocks_per_seq]
+ *   context_lens    device int32 [num_seqs], each <= max_context_len and
+ *                   <= max_blocks_per_seq * block_size (else clamped and
+ *                   PKV_DEVERR_LENGTH)
+ *   max_context_len host bound on context_lens (sizes the launch)
+ *   partition_size  tokens per split-K partition: 0 = one partition per
+ *                   sequence (no workspace needed); otherwise a positive
+ *                   multiple of block_size.  Each partition's partial result
+ *                   (running max, running sum, normalised output) goes to the
+ *                   workspace and a log-sum-exp merge kernel combines them.
+ *   workspace       device, >= pkv_decode_workspace_size(...) bytes, 16-byte
+ *                   aligned; may be NULL when that size is 0.  Its contents
+ *                   need no initialisation and are scratch after the call.
+ * Supported: head_dim in {64, 128}; block_size in {8, 16, 32}; dtype in
+ * {F32, F16, BF16}; num_q_heads / num_kv_heads in {1, 2, 4, 8}.
+ */
+int pkv_paged_attention_decode(void* out, const void* query, const void* key_cache,
+                               const void* value_cache, const int32_t* block_tables,
+                               const int32_t* context_lens, float scale, int num_seqs,
+                               int num_q_heads, int num_kv_heads, int head_dim, int block_size,
+                               int max_blocks_per_seq, int64_t num_blocks, int max_context_len,
+                               int partition_size, int dtype, void* workspace,
+                               size_t workspace_bytes, pkv_stream_t stream);
+
+/* Workspace bytes pkv_paged_attention_decode needs for these sizes (0 when
+ * partition_size == 0 or max_context_len <= partition_size). */
+size_t pkv_decode_workspace_size(int num_seqs, int num_q_heads, int head_dim, int max_context_len,
+                                 int partition_size);
+
+/* Split-K partition size (tokens) the library recommends for a batch on the
+ * current device: 0 (no split) when the batch alone fills the GPU, else a
+ * multiple of block_size.  Returns a negative pkv_status on bad input. */
+int pkv_decode_partition_size(int num_seqs, int num_kv_heads, int head_dim, int block_size,
+                              int max_context_len, int dtype);
+
+/*
+ * Chunked prefill over the paged cache (guide page "Chunked Prefill": a long
+ * prompt's prefill is cut into chunks scheduled together with decode; case-
+ * study page section 六 "Chunked prefill").  Chunk r owns query rows
+ * [query_start_loc[r], query_start_loc[r + 1]) of the packed query; its
+ * sequence holds seq_lens[r] cached tokens of which the chunk's own n_r
+ * tokens are the last (written beforehand, e.g. by pkv_reshape_and_cache),
+ * so row i sits at absolute position c0 = seq_lens[r] - n_r plus i and
+ * attends causally to positions j <= c0 + i:
+ *     out[row][h] = sum_{j <= c0 + i} softmax_j(scale * q[row][h] . K_j) V_j.
+ * The Q.K^T and P.V products run on the tcgen05 tensor cores (fp32
+ * accumulation in tensor memory).
+ *
+ *   out, query      device [total_q_tokens, num_q_heads, head_dim], dtype
+ *   block_tables    device int32 [num_chunks, max_blocks_per_seq]
+ *   seq_lens        device int32 [num_chunks]
+ *   query_start_loc device int32 [num_chunks + 1], non-decreasing, last =
+ *                   total_q_tokens
+ *   max_q_len       host bound on the chunk lengths (sizes the launch)
+ * Supported: dtype in {F16, BF16}; head_dim in {64, 128}; block_size in
+ * {8, 16, 32}; num_q_heads / num_kv_heads in {1, 2, 4, 8}.  A chunk longer
+ * than its sequence, or a sequence beyond its table row, is skipped and sets
+ * PKV_DEVERR_LENGTH.
+ */
+int pkv_paged_attention_prefill_chunk(void* out, const void* query, const void* key_cache,
+                                      const void* value_cache, const int32_t* block_tables,
+                                      const int32_t* seq_lens, const int32_t* query_start_loc,
+                                      int num_chunks, int64_t total_q_tokens, int max_q_len,
+                                      float scale, int num_q_heads, int num_kv_heads, int head_dim,
+                                      int block_size, int max_blocks_per_seq, int64_t num_blocks,
+                                      int dtype, pkv_stream_t stream);
+
+/* Read, and reset to 0, the current device's error word (PKV_DEVERR_* bits)
+ * after all work queued on `stream` so far.  Synchronises `stream`. */
+int pkv_get_device_error(uint32_t* host_err, pkv_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* PAGEDKV_H */

@@ -1,0 +1,19 @@
+"""B200-native paged KV-cache attention: thin Python binding over ``libpagedkv.so``.
+
+The library (``csrc/``, declared in ``include/pagedkv.h``) holds every kernel
+of the path; this package only marshals torch tensors' device pointers and
+the current CUDA stream into its C-ABI calls.  Importing the package does not
+load the library; the first call does, and fails loudly if it is missing.
+"""
+from ._binding import (  # noqa: F401
+    PagedKVError,
+    copy_blocks,
+    decode_partition_size,
+    decode_workspace_size,
+    get_device_error,
+    library_path,
+    load_library,
+    paged_attention_decode,
+    paged_attention_prefill_chunk,
+    reshape_and_cache,
+)

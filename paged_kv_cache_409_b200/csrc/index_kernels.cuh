@@ -1,0 +1,85 @@
+// index_kernels.cuh -- the two indexing kernels of the paged cache:
+//   reshape_and_cache (write new tokens' K/V into their physical slots) and
+//   copy_blocks (copy-on-write of shared blocks).
+// Both are pure data movement: 16-byte vector loads and stores, several in
+// flight per thread, bounded by HBM bandwidth (or by launch latency when the
+// token count is small).
+#pragma once
+
+#include "ptx.cuh"
+
+namespace pkv {
+
+// One CTA per token (grid-stride over tokens).  A token's K row and V row are
+// each contiguous (num_kv_heads * head_dim elements) in the source and, in the
+// [num_blocks, block_size, num_kv_heads, head_dim] pool, at row `slot`.
+__global__ void __launch_bounds__(128) reshape_and_cache_kernel(const uint4* __restrict__ key,
+                                                                const uint4* __restrict__ value,
+                                                                uint4* __restrict__ key_cache,
+                                                                uint4* __restrict__ value_cache,
+                                                                const int64_t* __restrict__ slot_mapping,
+                                                                int64_t num_tokens, int row_vecs,
+                                                                int64_t num_slots) {
+    for (int64_t t = blockIdx.x; t < num_tokens; t += gridDim.x) {
+        const int64_t slot = slot_mapping[t];
+        if (slot < 0) continue;  // padding token
+        if (slot >= num_slots) {
+            if (threadIdx.x == 0) flag_error(PKV_DEVERR_SLOT);
+            continue;
+        }
+        const uint4* ks = key + t * row_vecs;
+        const uint4* vs = value + t * row_vecs;
+        uint4* kd = key_cache + slot * row_vecs;
+        uint4* vd = value_cache + slot * row_vecs;
+        for (int i = threadIdx.x; i < row_vecs; i += blockDim.x) {
+            const uint4 a = ks[i];
+            const uint4 b = vs[i];
+            kd[i] = a;
+            vd[i] = b;
+        }
+    }
+}
+
+constexpr int kMaxLayersPerLaunch = 32;
+
+struct LayerPools {
+    uint4* k[kMaxLayersPerLaunch];
+    uint4* v[kMaxLayersPerLaunch];
+};
+
+constexpr int kCopyThreads = 256;
+constexpr int kCopyUnroll = 4;
+
+// grid.x: chunks of one block (kCopyThreads * kCopyUnroll vectors each),
+// grid.y: pairs (grid-stride), grid.z: layer * 2 + (0 = K, 1 = V).
+__global__ void __launch_bounds__(kCopyThreads) copy_blocks_kernel(const LayerPools pools,
+                                                                   const int64_t* __restrict__ pairs,
+                                                                   int64_t num_pairs, int64_t block_vecs,
+                                                                   int64_t num_blocks) {
+    const int layer = blockIdx.z >> 1;
+    uint4* base = (blockIdx.z & 1) ? pools.v[layer] : pools.k[layer];
+    const int64_t first = static_cast<int64_t>(blockIdx.x) * kCopyThreads * kCopyUnroll + threadIdx.x;
+    for (int64_t p = blockIdx.y; p < num_pairs; p += gridDim.y) {
+        const int64_t src = pairs[2 * p];
+        const int64_t dst = pairs[2 * p + 1];
+        if (src < 0 || src >= num_blocks || dst < 0 || dst >= num_blocks) {
+            if (threadIdx.x == 0 && blockIdx.x == 0 && blockIdx.z == 0) flag_error(PKV_DEVERR_PAIR);
+            continue;
+        }
+        const uint4* s = base + src * block_vecs;
+        uint4* d = base + dst * block_vecs;
+        uint4 r[kCopyUnroll];
+#pragma unroll
+        for (int u = 0; u < kCopyUnroll; ++u) {
+            const int64_t i = first + u * kCopyThreads;
+            if (i < block_vecs) r[u] = s[i];
+        }
+#pragma unroll
+        for (int u = 0; u < kCopyUnroll; ++u) {
+            const int64_t i = first + u * kCopyThreads;
+            if (i < block_vecs) d[i] = r[u];
+        }
+    }
+}
+
+}  // namespace pkv

@@ -1,0 +1,576 @@
+// pagedkv.cu -- host side of libpagedkv.so: argument checks, TMA tensor maps,
+// kernel selection and launches behind the C ABI of include/pagedkv.h.
+//
+// The library is one translation unit (the kernels live in the .cuh files
+// included below) so that all kernels share the device error word.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdio>
+#include <cstdlib>
+#include <cstring>
+#include <mutex>
+#include <set>
+#include <vector>
+
+#include "pagedkv.h"
+#include "ptx.cuh"
+#include "index_kernels.cuh"
+#include "decode.cuh"
+#include "prefill.cuh"
+
+namespace {
+
+thread_local char g_last_cuda_error[256] = "";
+
+int cuda_fail(cudaError_t e, const char* where) {
+    snprintf(g_last_cuda_error, sizeof g_last_cuda_error, "%s: %s", where, cudaGetErrorString(e));
+    return PKV_ECUDA;
+}
+
+#define PKV_CUDA(call)                                      \
+    do {                                                    \
+        cudaError_t e__ = (call);                           \
+        if (e__ != cudaSuccess) return cuda_fail(e__, #call); \
+    } while (0)
+
+int elem_bytes(int dtype) {
+    switch (dtype) {
+        case PKV_F32: return 4;
+        case PKV_F16: return 2;
+        case PKV_BF16: return 2;
+        default: return 0;
+    }
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
+
+bool checked_mode() {
+    static const bool on = [] {
+        const char* v = getenv("PKV_CHECK");
+        return v && v[0] && strcmp(v, "0") != 0;
+    }();
+    return on;
+}
+
+// ------------------------------------------------------------ tensor maps
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    });
+    return fn;
+}
+
+CUtensorMapDataType cu_type(int dtype) {
+    switch (dtype) {
+        case PKV_F32: return CU_TENSOR_MAP_DATA_TYPE_FLOAT32;
+        case PKV_F16: return CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
+        default: return CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+    }
+}
+
+// Pool [num_blocks, block_size, num_kv_heads, head_dim] as a 4-D tensor
+// (head_dim innermost); one box = one block x one KV head x 128 bytes of
+// head_dim, 128-byte swizzled.
+int make_pool_map(CUtensorMap* map, const void* pool, int dtype, int64_t num_blocks, int block_size,
+                  int num_kv_heads, int head_dim) {
+    auto fn = encode_fn();
+    if (!fn) {
+        snprintf(g_last_cuda_error, sizeof g_last_cuda_error, "cuTensorMapEncodeTiled unavailable");
+        return PKV_ECUDA;
+    }
+    const int eb = elem_bytes(dtype);
+    cuuint64_t dims[4] = {(cuuint64_t)head_dim, (cuuint64_t)num_kv_heads, (cuuint64_t)block_size,
+                          (cuuint64_t)num_blocks};
+    cuuint64_t strides[3] = {(cuuint64_t)head_dim * eb, (cuuint64_t)num_kv_heads * head_dim * eb,
+                             (cuuint64_t)block_size * num_kv_heads * head_dim * eb};
+    cuuint32_t box[4] = {(cuuint32_t)(128 / eb), 1, (cuuint32_t)block_size, 1};
+    cuuint32_t estr[4] = {1, 1, 1, 1};
+    CUresult r = fn(map, cu_type(dtype), 4, const_cast<void*>(pool), dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) {
+        snprintf(g_last_cuda_error, sizeof g_last_cuda_error, "cuTensorMapEncodeTiled(pool) failed: %d", (int)r);
+        return PKV_ECUDA;
+    }
+    return PKV_OK;
+}
+
+// Packed query [tokens, num_q_heads, head_dim] as a 3-D tensor; one box =
+// 128 / group tokens x group heads x 128 bytes of head_dim.
+int make_query_map(CUtensorMap* map, const void* q, int dtype, int64_t tokens, int num_q_heads, int head_dim,
+                   int group) {
+    auto fn = encode_fn();
+    if (!fn) {
+        snprintf(g_last_cuda_error, sizeof g_last_cuda_error, "cuTensorMapEncodeTiled unavailable");
+        return PKV_ECUDA;
+    }
+    const int eb = elem_bytes(dtype);
+    cuuint64_t dims[3] = {(cuuint64_t)head_dim, (cuuint64_t)num_q_heads, (cuuint64_t)tokens};
+    cuuint64_t strides[2] = {(cuuint64_t)head_dim * eb, (cuuint64_t)num_q_heads * head_dim * eb};
+    cuuint32_t box[3] = {(cuuint32_t)(128 / eb), (cuuint32_t)group, (cuuint32_t)(128 / group)};
+    cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = fn(map, cu_type(dtype), 3, const_cast<void*>(q), dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) {
+        snprintf(g_last_cuda_error, sizeof g_last_cuda_error, "cuTensorMapEncodeTiled(query) failed: %d", (int)r);
+        return PKV_ECUDA;
+    }
+    return PKV_OK;
+}
+
+int sm_count() {
+    int dev = 0, n = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) return 148;
+    return n;
+}
+
+// ------------------------------------------------------------ checked mode
+template <typename I>
+int fetch(std::vector<I>& host, const I* dev, size_t n, cudaStream_t s) {
+    host.resize(n);
+    if (n == 0) return PKV_OK;
+    PKV_CUDA(cudaMemcpyAsync(host.data(), dev, n * sizeof(I), cudaMemcpyDeviceToHost, s));
+    PKV_CUDA(cudaStreamSynchronize(s));
+    return PKV_OK;
+}
+
+int check_tables(const int32_t* d_bt, const int32_t* d_lens, int num_seqs, int max_blocks, int block_size,
+                 int64_t num_blocks, int64_t max_len, cudaStream_t s) {
+    std::vector<int32_t> bt, lens;
+    int rc = fetch(lens, d_lens, num_seqs, s);
+    if (rc) return rc;
+    rc = fetch(bt, d_bt, (size_t)num_seqs * max_blocks, s);
+    if (rc) return rc;
+    for (int i = 0; i < num_seqs; ++i) {
+        const int64_t n = lens[i];
+        if (n < 0 || n > max_len || n > (int64_t)max_blocks * block_size) return PKV_ERANGE;
+        const int64_t nb = (n + block_size - 1) / block_size;
+        for (int64_t b = 0; b < nb; ++b) {
+            const int32_t id = bt[(size_t)i * max_blocks + b];
+            if (id < 0 || id >= num_blocks) return PKV_ERANGE;
+        }
+    }
+    return PKV_OK;
+}
+
+// ------------------------------------------------------------ decode dispatch
+constexpr int pick_stages(int stage_bytes) {
+    int n = 98304 / (pkv::kDecodeWarps * stage_bytes);
+    if (n < 2 && pkv::kDecodeWarps * 2 * stage_bytes <= 200 * 1024) n = 2;
+    if (n < 1) n = 1;
+    if (n > 4) n = 4;
+    return n;
+}
+
+template <typename T, int D, int B, int G>
+int launch_decode(const pkv::DecodeParams& prm, const CUtensorMap& tk, const CUtensorMap& tv, int grid,
+                  cudaStream_t s) {
+    constexpr int NST = pick_stages(2 * B * D * pkv::Elem<T>::kBytes);
+    using C = pkv::DecodeCfg<T, D, B, G, NST>;
+    const size_t smem = C::smem_bytes(prm.partition_blocks);
+    auto kern = pkv::paged_decode_kernel<T, D, B, G, NST>;
+    static size_t configured = 0;  // largest dynamic smem size set so far for this instantiation
+    if (smem > configured) {
+        PKV_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
+        configured = smem;
+    }
+    kern<<<grid, pkv::kDecodeThreads, smem, s>>>(prm, tk, tv);
+    PKV_CUDA(cudaGetLastError());
+    return PKV_OK;
+}
+
+template <typename T, int D, int B>
+int decode_by_group(int group, const pkv::DecodeParams& prm, const CUtensorMap& tk, const CUtensorMap& tv,
+                    int grid, cudaStream_t s) {
+    switch (group) {
+        case 1: return launch_decode<T, D, B, 1>(prm, tk, tv, grid, s);
+        case 2: return launch_decode<T, D, B, 2>(prm, tk, tv, grid, s);
+        case 4: return launch_decode<T, D, B, 4>(prm, tk, tv, grid, s);
+        case 8: return launch_decode<T, D, B, 8>(prm, tk, tv, grid, s);
+        default: return PKV_EUNSUPPORTED;
+    }
+}
+
+template <typename T, int D>
+int decode_by_block(int block_size, int group, const pkv::DecodeParams& prm, const CUtensorMap& tk,
+                    const CUtensorMap& tv, int grid, cudaStream_t s) {
+    switch (block_size) {
+        case 8: return decode_by_group<T, D, 8>(group, prm, tk, tv, grid, s);
+        case 16: return decode_by_group<T, D, 16>(group, prm, tk, tv, grid, s);
+        case 32: return decode_by_group<T, D, 32>(group, prm, tk, tv, grid, s);
+        default: return PKV_EUNSUPPORTED;
+    }
+}
+
+template <typename T>
+int decode_by_dim(int head_dim, int block_size, int group, const pkv::DecodeParams& prm, const CUtensorMap& tk,
+                  const CUtensorMap& tv, int grid, cudaStream_t s) {
+    switch (head_dim) {
+        case 64: return decode_by_block<T, 64>(block_size, group, prm, tk, tv, grid, s);
+        case 128: return decode_by_block<T, 128>(block_size, group, prm, tk, tv, grid, s);
+        default: return PKV_EUNSUPPORTED;
+    }
+}
+
+template <typename T>
+int launch_merge(int head_dim, const pkv::MergeParams& mp, cudaStream_t s) {
+    const int warps = mp.num_seqs * mp.num_q_heads;
+    const int grid = (warps + 3) / 4;
+    if (head_dim == 64)
+        pkv::paged_decode_merge_kernel<T, 64><<<grid, 128, 0, s>>>(mp);
+    else
+        pkv::paged_decode_merge_kernel<T, 128><<<grid, 128, 0, s>>>(mp);
+    PKV_CUDA(cudaGetLastError());
+    return PKV_OK;
+}
+
+bool supported_group(int g) { return g == 1 || g == 2 || g == 4 || g == 8; }
+
+int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
+
+// ------------------------------------------------------------ prefill dispatch
+template <typename T, int D, int G>
+int launch_prefill(const pkv::PrefillParams& prm, const CUtensorMap& tq, const CUtensorMap& tk,
+                   const CUtensorMap& tv, int grid, cudaStream_t s) {
+    using C = pkv::PrefillCfg<T, D, G>;
+    auto kern = pkv::paged_prefill_kernel<T, D, G>;
+    static bool configured = false;
+    if (!configured) {
+        PKV_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM));
+        configured = true;
+    }
+    kern<<<grid, pkv::kPrefillThreads, C::SMEM, s>>>(prm, tq, tk, tv);
+    PKV_CUDA(cudaGetLastError());
+    return PKV_OK;
+}
+
+template <typename T, int D>
+int prefill_by_group(int group, const pkv::PrefillParams& prm, const CUtensorMap& tq, const CUtensorMap& tk,
+                     const CUtensorMap& tv, int grid, cudaStream_t s) {
+    switch (group) {
+        case 1: return launch_prefill<T, D, 1>(prm, tq, tk, tv, grid, s);
+        case 2: return launch_prefill<T, D, 2>(prm, tq, tk, tv, grid, s);
+        case 4: return launch_prefill<T, D, 4>(prm, tq, tk, tv, grid, s);
+        case 8: return launch_prefill<T, D, 8>(prm, tq, tk, tv, grid, s);
+        default: return PKV_EUNSUPPORTED;
+    }
+}
+
+}  // namespace
+
+// ============================================================ C ABI
+extern "C" {
+
+const char* pkv_status_string(int status) {
+    switch (status) {
+        case PKV_OK: return "ok";
+        case PKV_EINVAL: return "invalid argument";
+        case PKV_EUNSUPPORTED: return "unsupported shape or dtype";
+        case PKV_ERANGE: return "table entry out of range";
+        case PKV_ECUDA: return "CUDA error";
+        case PKV_EWORKSPACE: return "workspace missing or too small";
+        default: return "unknown status";
+    }
+}
+
+const char* pkv_last_cuda_error(void) { return g_last_cuda_error; }
+
+int pkv_reshape_and_cache(const void* key, const void* value, void* key_cache, void* value_cache,
+                          const int64_t* slot_mapping, int64_t num_tokens, int num_kv_heads, int head_dim,
+                          int block_size, int64_t num_blocks, int dtype, pkv_stream_t stream) {
+    const int eb = elem_bytes(dtype);
+    if (!eb) return PKV_EUNSUPPORTED;
+    if (num_tokens < 0 || num_kv_heads <= 0 || head_dim <= 0 || block_size <= 0 || num_blocks <= 0)
+        return PKV_EINVAL;
+    const int64_t row_bytes = (int64_t)num_kv_heads * head_dim * eb;
+    if (row_bytes % 16 != 0) return PKV_EUNSUPPORTED;
+    if (num_tokens == 0) return PKV_OK;
+    if (!key || !value || !key_cache || !value_cache || !slot_mapping) return PKV_EINVAL;
+    if (!aligned16(key) || !aligned16(value) || !aligned16(key_cache) || !aligned16(value_cache) ||
+        (reinterpret_cast<uintptr_t>(slot_mapping) & 7))
+        return PKV_EINVAL;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const int64_t num_slots = num_blocks * block_size;
+    if (checked_mode()) {
+        std::vector<int64_t> sm;
+        int rc = fetch(sm, slot_mapping, (size_t)num_tokens, s);
+        if (rc) return rc;
+        for (int64_t v : sm)
+            if (v >= num_slots) return PKV_ERANGE;
+    }
+    const int grid = (int)std::min<int64_t>(num_tokens, 65535);
+    pkv::reshape_and_cache_kernel<<<grid, 128, 0, s>>>(
+        static_cast<const uint4*>(key), static_cast<const uint4*>(value), static_cast<uint4*>(key_cache),
+        static_cast<uint4*>(value_cache), slot_mapping, num_tokens, (int)(row_bytes / 16), num_slots);
+    PKV_CUDA(cudaGetLastError());
+    return PKV_OK;
+}
+
+int pkv_copy_blocks(void* const* key_caches, void* const* value_caches, int num_layers,
+                    const int64_t* src_dst_pairs, int64_t num_pairs, int64_t block_bytes, int64_t num_blocks,
+                    pkv_stream_t stream) {
+    if (num_layers < 0 || num_pairs < 0 || block_bytes <= 0 || num_blocks <= 0) return PKV_EINVAL;
+    if (block_bytes % 16 != 0) return PKV_EUNSUPPORTED;
+    if (num_layers == 0 || num_pairs == 0) return PKV_OK;
+    if (!key_caches || !value_caches || !src_dst_pairs || (reinterpret_cast<uintptr_t>(src_dst_pairs) & 7))
+        return PKV_EINVAL;
+    for (int l = 0; l < num_layers; ++l)
+        if (!key_caches[l] || !value_caches[l] || !aligned16(key_caches[l]) || !aligned16(value_caches[l]))
+            return PKV_EINVAL;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (checked_mode()) {
+        std::vector<int64_t> pr;
+        int rc = fetch(pr, src_dst_pairs, (size_t)num_pairs * 2, s);
+        if (rc) return rc;
+        std::set<int64_t> srcs, dsts;
+        for (int64_t i = 0; i < num_pairs; ++i) {
+            const int64_t a = pr[2 * i], b = pr[2 * i + 1];
+            if (a < 0 || a >= num_blocks || b < 0 || b >= num_blocks) return PKV_ERANGE;
+            if (!dsts.insert(b).second) return PKV_ERANGE;
+            srcs.insert(a);
+        }
+        for (int64_t d : dsts)
+            if (srcs.count(d)) return PKV_ERANGE;
+    }
+    const int64_t block_vecs = block_bytes / 16;
+    const int64_t per_cta = (int64_t)pkv::kCopyThreads * pkv::kCopyUnroll;
+    const unsigned gx = (unsigned)ceil_div(block_vecs, per_cta);
+    const unsigned gy = (unsigned)std::min<int64_t>(num_pairs, 65535);
+    for (int l0 = 0; l0 < num_layers; l0 += pkv::kMaxLayersPerLaunch) {
+        const int nl = std::min(pkv::kMaxLayersPerLaunch, num_layers - l0);
+        pkv::LayerPools pools;
+        memset(&pools, 0, sizeof pools);
+        for (int l = 0; l < nl; ++l) {
+            pools.k[l] = static_cast<uint4*>(key_caches[l0 + l]);
+            pools.v[l] = static_cast<uint4*>(value_caches[l0 + l]);
+        }
+        dim3 grid(gx, gy, 2 * nl);
+        pkv::copy_blocks_kernel<<<grid, pkv::kCopyThreads, 0, s>>>(pools, src_dst_pairs, num_pairs, block_vecs,
+                                                                    num_blocks);
+        PKV_CUDA(cudaGetLastError());
+    }
+    return PKV_OK;
+}
+
+size_t pkv_decode_workspace_size(int num_seqs, int num_q_heads, int head_dim, int max_context_len,
+                                 int partition_size) {
+    if (num_seqs <= 0 || num_q_heads <= 0 || head_dim <= 0 || partition_size <= 0 || max_context_len <= 0)
+        return 0;
+    const int64_t parts = ceil_div(max_context_len, partition_size);
+    if (parts <= 1) return 0;
+    const int64_t rows = (int64_t)num_seqs * num_q_heads * parts;
+    // max and sum (rounded up to 16 bytes each), then the partial outputs
+    const int64_t ml = ((rows * 4 + 15) / 16) * 16;
+    return (size_t)(2 * ml + rows * head_dim * 4);
+}
+
+int pkv_decode_partition_size(int num_seqs, int num_kv_heads, int head_dim, int block_size, int max_context_len,
+                              int dtype) {
+    if (num_seqs < 0 || num_kv_heads <= 0 || head_dim <= 0 || block_size <= 0 || max_context_len < 0 ||
+        !elem_bytes(dtype))
+        return PKV_EINVAL;
+    // One partition per sequence when the (sequence, KV head) pairs alone make
+    // several waves of short CTAs; otherwise split long contexts into runs of
+    // 512 tokens (a multiple of every supported block size) so that the
+    // longest CTA stays short against the whole step.
+    (void)head_dim;
+    const int split = 512;
+    if (max_context_len <= split) return 0;
+    const int64_t pairs = (int64_t)num_seqs * num_kv_heads;
+    if (pairs >= (int64_t)sm_count() * 64) return 0;
+    return ((split + block_size - 1) / block_size) * block_size;
+}
+
+int pkv_paged_attention_decode(void* out, const void* query, const void* key_cache, const void* value_cache,
+                               const int32_t* block_tables, const int32_t* context_lens, float scale, int num_seqs,
+                               int num_q_heads, int num_kv_heads, int head_dim, int block_size,
+                               int max_blocks_per_seq, int64_t num_blocks, int max_context_len, int partition_size,
+                               int dtype, void* workspace, size_t workspace_bytes, pkv_stream_t stream) {
+    if (!elem_bytes(dtype)) return PKV_EUNSUPPORTED;
+    if (num_seqs < 0 || num_q_heads <= 0 || num_kv_heads <= 0 || max_blocks_per_seq <= 0 || num_blocks <= 0 ||
+        max_context_len < 0 || partition_size < 0 || !std::isfinite(scale))
+        return PKV_EINVAL;
+    if (num_q_heads % num_kv_heads) return PKV_EINVAL;
+    const int group = num_q_heads / num_kv_heads;
+    if (!supported_group(group) || (head_dim != 64 && head_dim != 128) ||
+        (block_size != 8 && block_size != 16 && block_size != 32))
+        return PKV_EUNSUPPORTED;
+    if (partition_size % block_size) return PKV_EINVAL;
+    if (num_blocks >= (int64_t)INT32_MAX || (int64_t)max_blocks_per_seq * block_size > INT32_MAX) return PKV_EINVAL;
+    if (num_seqs == 0) return PKV_OK;
+    if (!out || !query || !key_cache || !value_cache || !block_tables || !context_lens) return PKV_EINVAL;
+    if (!aligned16(out) || !aligned16(query) || !aligned16(key_cache) || !aligned16(value_cache) ||
+        (reinterpret_cast<uintptr_t>(block_tables) & 3) || (reinterpret_cast<uintptr_t>(context_lens) & 3))
+        return PKV_EINVAL;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+
+    const int64_t max_blocks_needed = std::max<int64_t>(1, ceil_div(std::max(max_context_len, 1), block_size));
+    int64_t pb = partition_size > 0 ? partition_size / block_size : max_blocks_needed;
+    pb = std::min(pb, max_blocks_needed);
+    const int64_t parts = ceil_div(max_blocks_needed, pb);
+    if (pb > 4096) return PKV_EUNSUPPORTED;  // per-CTA block list lives in shared memory
+    const size_t need = parts > 1 ? pkv_decode_workspace_size(num_seqs, num_q_heads, head_dim, max_context_len,
+                                                              (int)(pb * block_size))
+                                  : 0;
+    if (need > 0 && (!workspace || workspace_bytes < need || !aligned16(workspace))) return PKV_EWORKSPACE;
+    const int64_t grid = (int64_t)num_seqs * parts * num_kv_heads;
+    if (grid > INT32_MAX) return PKV_EUNSUPPORTED;
+
+    if (checked_mode()) {
+        int rc = check_tables(block_tables, context_lens, num_seqs, max_blocks_per_seq, block_size, num_blocks,
+                              max_context_len, s);
+        if (rc) return rc;
+    }
+
+    CUtensorMap tk, tv;
+    int rc = make_pool_map(&tk, key_cache, dtype, num_blocks, block_size, num_kv_heads, head_dim);
+    if (rc) return rc;
+    rc = make_pool_map(&tv, value_cache, dtype, num_blocks, block_size, num_kv_heads, head_dim);
+    if (rc) return rc;
+
+    pkv::DecodeParams prm;
+    prm.out = out;
+    prm.query = query;
+    prm.block_tables = block_tables;
+    prm.context_lens = context_lens;
+    const int64_t rows = (int64_t)num_seqs * num_q_heads * parts;
+    const int64_t ml = ((rows * 4 + 15) / 16) * 16;
+    prm.ws_max = need ? reinterpret_cast<float*>(workspace) : nullptr;
+    prm.ws_sum = need ? reinterpret_cast<float*>(static_cast<char*>(workspace) + ml) : nullptr;
+    prm.ws_out = need ? reinterpret_cast<float*>(static_cast<char*>(workspace) + 2 * ml) : nullptr;
+    prm.scale_log2 = scale * 1.4426950408889634f;
+    prm.num_seqs = num_seqs;
+    prm.num_q_heads = num_q_heads;
+    prm.num_kv_heads = num_kv_heads;
+    prm.max_blocks_per_seq = max_blocks_per_seq;
+    prm.num_blocks = num_blocks;
+    prm.partition_blocks = (int)pb;
+    prm.num_partitions = (int)parts;
+
+    switch (dtype) {
+        case PKV_F32: rc = decode_by_dim<float>(head_dim, block_size, group, prm, tk, tv, (int)grid, s); break;
+        case PKV_F16: rc = decode_by_dim<__half>(head_dim, block_size, group, prm, tk, tv, (int)grid, s); break;
+        default: rc = decode_by_dim<__nv_bfloat16>(head_dim, block_size, group, prm, tk, tv, (int)grid, s); break;
+    }
+    if (rc || parts <= 1) return rc;
+
+    pkv::MergeParams mp;
+    mp.out = out;
+    mp.context_lens = context_lens;
+    mp.ws_max = prm.ws_max;
+    mp.ws_sum = prm.ws_sum;
+    mp.ws_out = prm.ws_out;
+    mp.num_seqs = num_seqs;
+    mp.num_q_heads = num_q_heads;
+    mp.block_size = block_size;
+    mp.max_blocks_per_seq = max_blocks_per_seq;
+    mp.partition_blocks = (int)pb;
+    mp.num_partitions = (int)parts;
+    switch (dtype) {
+        case PKV_F32: return launch_merge<float>(head_dim, mp, s);
+        case PKV_F16: return launch_merge<__half>(head_dim, mp, s);
+        default: return launch_merge<__nv_bfloat16>(head_dim, mp, s);
+    }
+}
+
+int pkv_paged_attention_prefill_chunk(void* out, const void* query, const void* key_cache, const void* value_cache,
+                                      const int32_t* block_tables, const int32_t* seq_lens,
+                                      const int32_t* query_start_loc, int num_chunks, int64_t total_q_tokens,
+                                      int max_q_len, float scale, int num_q_heads, int num_kv_heads, int head_dim,
+                                      int block_size, int max_blocks_per_seq, int64_t num_blocks, int dtype,
+                                      pkv_stream_t stream) {
+    if (dtype != PKV_F16 && dtype != PKV_BF16) return elem_bytes(dtype) ? PKV_EUNSUPPORTED : PKV_EUNSUPPORTED;
+    if (num_chunks < 0 || total_q_tokens < 0 || max_q_len < 0 || num_q_heads <= 0 || num_kv_heads <= 0 ||
+        max_blocks_per_seq <= 0 || num_blocks <= 0 || !std::isfinite(scale))
+        return PKV_EINVAL;
+    if (num_q_heads % num_kv_heads) return PKV_EINVAL;
+    const int group = num_q_heads / num_kv_heads;
+    if (!supported_group(group) || (head_dim != 64 && head_dim != 128) ||
+        (block_size != 8 && block_size != 16 && block_size != 32))
+        return PKV_EUNSUPPORTED;
+    if (num_blocks >= (int64_t)INT32_MAX || (int64_t)max_blocks_per_seq * block_size > INT32_MAX ||
+        total_q_tokens > INT32_MAX)
+        return PKV_EINVAL;
+    if (num_chunks == 0 || total_q_tokens == 0 || max_q_len == 0) return PKV_OK;
+    if (!out || !query || !key_cache || !value_cache || !block_tables || !seq_lens || !query_start_loc)
+        return PKV_EINVAL;
+    if (!aligned16(out) || !aligned16(query) || !aligned16(key_cache) || !aligned16(value_cache) ||
+        (reinterpret_cast<uintptr_t>(block_tables) & 3) || (reinterpret_cast<uintptr_t>(seq_lens) & 3) ||
+        (reinterpret_cast<uintptr_t>(query_start_loc) & 3))
+        return PKV_EINVAL;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+
+    if (checked_mode()) {
+        std::vector<int32_t> qsl, lens;
+        int rc = fetch(qsl, query_start_loc, (size_t)num_chunks + 1, s);
+        if (rc) return rc;
+        rc = fetch(lens, seq_lens, (size_t)num_chunks, s);
+        if (rc) return rc;
+        if (qsl[0] < 0 || qsl[num_chunks] > total_q_tokens) return PKV_ERANGE;
+        for (int r = 0; r < num_chunks; ++r) {
+            const int n = qsl[r + 1] - qsl[r];
+            if (n < 0 || n > max_q_len || lens[r] < n) return PKV_ERANGE;
+        }
+        rc = check_tables(block_tables, seq_lens, num_chunks, max_blocks_per_seq, block_size, num_blocks,
+                          (int64_t)max_blocks_per_seq * block_size, s);
+        if (rc) return rc;
+    }
+
+    CUtensorMap tq, tk, tv;
+    int rc = make_query_map(&tq, query, dtype, total_q_tokens, num_q_heads, head_dim, group);
+    if (rc) return rc;
+    rc = make_pool_map(&tk, key_cache, dtype, num_blocks, block_size, num_kv_heads, head_dim);
+    if (rc) return rc;
+    rc = make_pool_map(&tv, value_cache, dtype, num_blocks, block_size, num_kv_heads, head_dim);
+    if (rc) return rc;
+
+    const int tile_tokens = 128 / group;
+    const int64_t q_tiles = ceil_div(max_q_len, tile_tokens);
+    const int64_t grid = (int64_t)num_chunks * q_tiles * num_kv_heads;
+    if (grid > INT32_MAX) return PKV_EUNSUPPORTED;
+
+    pkv::PrefillParams prm;
+    prm.out = out;
+    prm.block_tables = block_tables;
+    prm.seq_lens = seq_lens;
+    prm.query_start_loc = query_start_loc;
+    prm.scale_log2 = scale * 1.4426950408889634f;
+    prm.num_chunks = num_chunks;
+    prm.num_q_heads = num_q_heads;
+    prm.num_kv_heads = num_kv_heads;
+    prm.max_blocks_per_seq = max_blocks_per_seq;
+    prm.block_size = block_size;
+    prm.num_blocks = num_blocks;
+    prm.q_tiles = (int)q_tiles;
+    const bool bf16 = dtype == PKV_BF16;
+    if (head_dim == 64)
+        return bf16 ? prefill_by_group<__nv_bfloat16, 64>(group, prm, tq, tk, tv, (int)grid, s)
+                    : prefill_by_group<__half, 64>(group, prm, tq, tk, tv, (int)grid, s);
+    return bf16 ? prefill_by_group<__nv_bfloat16, 128>(group, prm, tq, tk, tv, (int)grid, s)
+                : prefill_by_group<__half, 128>(group, prm, tq, tk, tv, (int)grid, s);
+}
+
+int pkv_get_device_error(uint32_t* host_err, pkv_stream_t stream) {
+    if (!host_err) return PKV_EINVAL;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    unsigned int v = 0;
+    PKV_CUDA(cudaMemcpyFromSymbolAsync(&v, pkv::g_device_error, sizeof v, 0, cudaMemcpyDeviceToHost, s));
+    const unsigned int zero = 0;
+    PKV_CUDA(cudaMemcpyToSymbolAsync(pkv::g_device_error, &zero, sizeof zero, 0, cudaMemcpyHostToDevice, s));
+    PKV_CUDA(cudaStreamSynchronize(s));
+    *host_err = v;
+    return PKV_OK;
+}
+
+}  // extern "C"

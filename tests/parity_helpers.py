@@ -1,0 +1,113 @@
+"""Shared pieces of the GPU parity tests: run a workload through the CUDA
+library and through the CPU oracle on the same seeded inputs.
+
+Inputs for the oracle are always snapshots taken BEFORE the CUDA path runs
+(or host copies of generator output); nothing the kernels write feeds the
+oracle.  Sampled checks on large pools copy only the blocks the sampled
+sequences use and renumber them densely -- the oracle's own pins show that
+physical placement does not change its result.
+"""
+from __future__ import annotations
+
+import numpy as np
+import torch
+
+import oracle
+import paged_kv_cache_409_b200 as pkv
+
+TOL = {torch.float32: (1e-5, 0.0), torch.float16: (2e-3, 1e-2), torch.bfloat16: (2e-3, 1e-2)}
+
+
+def assert_close(gpu: torch.Tensor, ref: np.ndarray, dtype, what=""):
+    """|gpu - ref| <= atol + rtol |ref| element-wise (fp32: max-abs 1e-5)."""
+    atol, rtol = TOL[dtype]
+    g = gpu.detach().float().cpu().double().numpy()
+    assert g.shape == ref.shape, (g.shape, ref.shape)
+    assert np.all(np.isfinite(g)), f"{what}: non-finite output"
+    err = np.abs(g - ref)
+    bound = atol + rtol * np.abs(ref)
+    bad = err > bound
+    if bad.any():
+        i = np.unravel_index(np.argmax(err - bound), err.shape)
+        raise AssertionError(f"{what}: {bad.sum()} of {bad.size} elements out of tolerance; worst at {i}: "
+                             f"gpu {g[i]!r} ref {ref[i]!r} (atol {atol}, rtol {rtol})")
+    return float(err.max())
+
+
+def bits(t: torch.Tensor) -> np.ndarray:
+    """Raw element bits of a tensor, for bit-exact comparisons (NaN payloads included)."""
+    t = t.detach().cpu().contiguous()
+    if t.element_size() == 4:
+        return t.view(torch.int32).numpy()
+    return t.view(torch.int16).numpy()
+
+
+def snapshot_blocks(cache: torch.Tensor, ids: np.ndarray) -> torch.Tensor:
+    """Host copy of the listed physical blocks of a pool."""
+    return cache[torch.from_numpy(ids.astype(np.int64)).to(cache.device)].cpu().clone()
+
+
+def compact_tables(tables: np.ndarray, lens, block_size: int):
+    """Blocks used by these sequences, and their tables renumbered densely."""
+    need = [(int(n) + block_size - 1) // block_size for n in lens]
+    used = np.unique(np.concatenate([tables[i, :k] for i, k in enumerate(need)] + [np.zeros(0, np.int32)]))
+    remap = {int(b): i for i, b in enumerate(used)}
+    out = np.full_like(tables, -1)
+    for i, k in enumerate(need):
+        out[i, :k] = [remap[int(b)] for b in tables[i, :k]]
+    return used.astype(np.int64), out.astype(np.int32)
+
+
+def oracle_decode_step(w, seqs=None, layer=0, pre_k=None, pre_v=None):
+    """Oracle of append-then-attend for sequences ``seqs`` of a DecodeWorkload.
+
+    ``pre_k``/``pre_v``: host snapshots of the whole pools taken before the
+    CUDA path ran (else the workload's own pools, which must still be
+    untouched).  Returns (out float64 [len(seqs), Hq, D], k_after, v_after,
+    used block ids) where *_after are the compacted pools after the append.
+    """
+    S = w.num_seqs
+    seqs = np.arange(S) if seqs is None else np.asarray(seqs)
+    lens = w.context_lens[seqs]
+    used, bt = compact_tables(w.block_tables[seqs], lens, w.block_size)
+    src_k = pre_k if pre_k is not None else w.key_caches[layer]
+    src_v = pre_v if pre_v is not None else w.value_caches[layer]
+    kc, code = oracle.storage(snapshot_blocks(src_k, used))
+    vc, _ = oracle.storage(snapshot_blocks(src_v, used))
+    kc, vc = kc.copy(), vc.copy()
+    nk, _ = oracle.storage(w.new_keys[layer][torch.from_numpy(seqs).to(w.new_keys[layer].device)])
+    nv, _ = oracle.storage(w.new_values[layer][torch.from_numpy(seqs).to(w.new_values[layer].device)])
+    B = w.block_size
+    remap = {int(b): i for i, b in enumerate(used)}
+    slots = np.array([remap[int(s) // B] * B + int(s) % B for s in w.slot_mapping[seqs]], dtype=np.int64)
+    orc = oracle.get()
+    orc.reshape_and_cache(nk, nv, kc, vc, slots, code)
+    q, _ = oracle.storage(w.queries[layer][torch.from_numpy(seqs).to(w.queries[layer].device)])
+    out = orc.paged_attention_decode(q, kc, vc, bt, lens, w.scale, code)
+    return out, kc, vc, used
+
+
+def gpu_tables(w, device="cuda"):
+    bt = torch.from_numpy(w.block_tables).to(device)
+    cl = torch.from_numpy(w.context_lens.astype(np.int32)).to(device)
+    sm = torch.from_numpy(w.slot_mapping.astype(np.int64)).to(device)
+    return bt, cl, sm
+
+
+def to_device(w, device="cuda"):
+    """Move a CPU-generated DecodeWorkload's tensors to the GPU (in place)."""
+    for name in ("key_caches", "value_caches", "queries", "new_keys", "new_values"):
+        setattr(w, name, [t.to(device) for t in getattr(w, name)])
+    return w
+
+
+def gpu_decode_step(w, layer=0, partition_size=None, out=None, tables=None):
+    """reshape_and_cache then paged_attention_decode on the GPU."""
+    bt, cl, sm = tables if tables is not None else gpu_tables(w, w.queries[layer].device)
+    kc, vc = w.key_caches[layer], w.value_caches[layer]
+    pkv.reshape_and_cache(w.new_keys[layer], w.new_values[layer], kc, vc, sm)
+    if out is None:
+        out = torch.empty_like(w.queries[layer])
+    pkv.paged_attention_decode(out, w.queries[layer], kc, vc, bt, cl, w.scale, w.max_context_len,
+                               partition_size=partition_size)
+    return out

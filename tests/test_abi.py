@@ -1,0 +1,77 @@
+"""The C-ABI library loads without a GPU and exports every entry point its header declares."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import paged_kv_cache_409_b200 as pkv
+from paged_kv_cache_409_b200 import _binding
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def declared():
+    src = open(os.path.join(ROOT, "include", "pagedkv.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(pkv_[a-z_]+)\s*\(", src)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from paged_kv_cache_409_b200 import build
+    build.build()
+    return pkv.load_library()
+
+
+def test_every_declared_symbol_is_exported(lib):
+    names = declared()
+    assert len(names) >= 9
+    for n in names:
+        assert hasattr(lib, n), f"{n} declared in include/pagedkv.h but not exported"
+    assert set(names) == set(_binding.EXPORTED) | (set(names) - set(_binding.EXPORTED))
+    for n in _binding.EXPORTED:
+        assert n in names, f"binding names {n} which the header does not declare"
+
+
+def test_status_strings(lib):
+    assert lib.pkv_status_string(0) == b"ok"
+    assert lib.pkv_status_string(-5).startswith(b"workspace")
+
+
+def test_workspace_size_arithmetic(lib):
+    # no split -> no workspace
+    assert pkv.decode_workspace_size(64, 32, 128, 2048, 0) == 0
+    assert pkv.decode_workspace_size(64, 32, 128, 512, 512) == 0
+    # 64 x 32 heads x 4 partitions: max + sum (16-byte rounded) + outputs
+    rows = 64 * 32 * 4
+    assert pkv.decode_workspace_size(64, 32, 128, 2048, 512) == 2 * rows * 4 + rows * 128 * 4
+
+
+def test_partition_heuristic_is_block_multiple(lib):
+    for B in (8, 16, 32):
+        p = pkv.decode_partition_size(64, 32, 128, B, 2048, 1)
+        assert p == 0 or p % B == 0
+    assert pkv.decode_partition_size(64, 32, 128, 16, 300, 1) == 0
+
+
+def test_host_rejections_before_launch(lib):
+    # unsupported dtype and bad sizes are refused before any device work
+    assert lib.pkv_paged_attention_decode(None, None, None, None, None, None, 0.1, 1, 4, 2, 128, 16, 1, 1, 16, 0, 7,
+                                          None, 0, None) == -2
+    assert lib.pkv_paged_attention_decode(None, None, None, None, None, None, 0.1, 1, 4, 3, 128, 16, 1, 1, 16, 0, 1,
+                                          None, 0, None) == -1
+    assert lib.pkv_paged_attention_decode(None, None, None, None, None, None, 0.1, 1, 4, 2, 128, 16, 1, 1, 16, 0, 1,
+                                          None, 0, None) == -1  # null pointers
+    assert lib.pkv_reshape_and_cache(None, None, None, None, None, 0, 2, 64, 16, 4, 1, None) == 0  # empty: no-op
+    assert lib.pkv_copy_blocks(None, None, 0, None, 0, 4096, 4, None) == 0
+    assert lib.pkv_paged_attention_prefill_chunk(None, None, None, None, None, None, None, 1, 4, 4, 0.1, 2, 2, 64,
+                                                 16, 1, 4, 0, None) == -2  # fp32 prefill
+    assert lib.pkv_get_device_error(None, None) == -1
+
+
+def test_missing_library_fails_loudly(monkeypatch, tmp_path):
+    monkeypatch.setattr(_binding, "_lib", None)
+    monkeypatch.setattr(_binding, "LIB", str(tmp_path / "nope.so"))
+    with pytest.raises(RuntimeError):
+        _binding.load_library()
