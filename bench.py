@@ -65,7 +65,8 @@ class DecodeStep:
         self.layers = layers_per_step or w.num_layers
         self.outs = [torch.empty_like(q) for q in w.queries]
         self.part = pkv.decode_partition_size(w.num_seqs, w.num_kv_heads, w.head_dim, w.block_size,
-                                              w.max_context_len, w.dtype)
+                                              w.max_context_len, w.dtype,
+                                              int(w.context_lens.astype(np.int64).sum()))
         need = pkv.decode_workspace_size(w.num_seqs, w.num_q_heads, w.head_dim, w.max_context_len, self.part)
         self.ws = torch.empty(max(need, 16), dtype=torch.uint8, device=dev)
         self.parts = -(-w.max_context_len // self.part) if self.part else 1
@@ -171,10 +172,11 @@ class MixedStep(DecodeStep):
             timer.end()
 
 
-def make_step(name, device, rank):
+def make_step(name, device, rank, seqs=None):
     from paged_kv_cache_409_b200 import workloads
     if name == "llama7b_decode_f16":
-        return DecodeStep(workloads.llama7b_decode_f16(device=device, seed=1002 + rank)), "llama7b_decode_f16"
+        w = workloads.llama7b_decode_f16(device=device, seed=1002 + rank, num_seqs=seqs or 64)
+        return DecodeStep(w), "llama7b_decode_f16" + (f" ({seqs} sequences)" if seqs else "")
     if name == "tiny_decode_f32":
         return DecodeStep(workloads.tiny_decode_f32(device=device)), name
     if name == "gqa70b_decode_bf16":
@@ -219,74 +221,84 @@ class EventTimer:
 
 
 class ClockSampler:
-    """nvidia-smi clock / throttle samples while the timed region runs."""
+    """SM clock and throttle reasons sampled through NVML (read-only queries)
+    from a background thread every ~2 ms; ``window`` keeps the samples taken
+    inside the timed region."""
 
-    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    REASONS = {"hw_slowdown": 0x8, "sw_thermal_slowdown": 0x20, "hw_thermal_slowdown": 0x40,
+               "sw_power_cap": 0x4}
 
     def __init__(self, device_index):
-        self.proc, self.path = None, None
+        import threading
+        self.samples, self.t_lo, self.t_hi = [], None, None
+        self.stop_evt = threading.Event()
+        self.thread = None
+        self.nvml = None
         try:
-            bus = torch.cuda.get_device_properties(device_index).pci_bus_id
+            import pynvml
+            pynvml.nvmlInit()
+            props = torch.cuda.get_device_properties(device_index)
+            want = (int(props.pci_domain_id), int(props.pci_bus_id), int(props.pci_device_id))
+            for i in range(pynvml.nvmlDeviceGetCount()):
+                h = pynvml.nvmlDeviceGetHandleByIndex(i)
+                pci = pynvml.nvmlDeviceGetPciInfo(h)
+                if (int(pci.domain), int(pci.bus), int(pci.device)) == want:
+                    self.nvml, self.h = pynvml, h
+                    self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM)
+                    break
         except Exception:
-            bus = None
-        self.bus = bus
+            self.nvml = None
+
+    def _loop(self):
+        n = self.nvml
+        while not self.stop_evt.is_set():
+            try:
+                sm = n.nvmlDeviceGetClockInfo(self.h, n.NVML_CLOCK_SM)
+                rs = n.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                self.samples.append((time.perf_counter(), sm, rs))
+            except Exception:
+                pass
+            time.sleep(0.002)
 
     def start(self):
-        if self.bus is None:
-            return
-        fd, self.path = tempfile.mkstemp(suffix=".csv")
-        os.close(fd)
-        try:
-            self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.bus}", f"--query-gpu={self.FIELDS}",
-                                          "--format=csv,noheader,nounits", "-lms", "50"],
-                                         stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
-        except OSError:
-            self.proc = None
+        import threading
+        if self.nvml:
+            self.thread = threading.Thread(target=self._loop, daemon=True)
+            self.thread.start()
+
+    def mark(self, lo, hi):
+        self.t_lo, self.t_hi = lo, hi
 
     def stop(self):
-        if not self.proc:
-            return None
-        self.proc.terminate()
-        try:
-            self.proc.wait(timeout=5)
-        except subprocess.TimeoutExpired:
-            self.proc.kill()
-        rows = []
-        with open(self.path) as f:
-            for line in f:
-                parts = [p.strip() for p in line.split(",")]
-                if len(parts) >= 9:
-                    rows.append(parts)
-        os.unlink(self.path)
-        if not rows:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
-
-        def num(x):
-            try:
-                return float(x)
-            except ValueError:
-                return None
-        sm = [num(r[1]) for r in rows if num(r[1]) is not None]
-        smax = [num(r[2]) for r in rows if num(r[2]) is not None]
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        reasons = sorted({names[i] for r in rows for i, v in enumerate(r[5:9]) if v.lower().startswith("active")})
-        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(smax) if smax else None,
-                "reasons": reasons, "samples": len(rows)}
+        if not self.thread:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvml unavailable"]}
+        self.stop_evt.set()
+        self.thread.join(timeout=2)
+        win = [x for x in self.samples if self.t_lo is not None and self.t_lo <= x[0] <= self.t_hi]
+        use = win if win else self.samples
+        if not use:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": ["no samples"]}
+        reasons = sorted({k for _, _, r in use for k, bit in self.REASONS.items() if r & bit})
+        return {"sm_mhz": statistics.median(x[1] for x in use), "sm_max_mhz": self.max_mhz, "reasons": reasons,
+                "samples": len(use), "in_timed_region": bool(win)}
 
 
-def dist_setup(n_gpus):
+def dist_setup(n_gpus, backend=None):
+    """Rank / world size from the torchrun environment; one process per GPU."""
     ws = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
     if ws > 1:
         import datetime
         import torch.distributed as dist
-        torch.cuda.set_device(local)
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                device_id=torch.device("cuda", local))
-    else:
+        backend = backend or ("nccl" if torch.cuda.is_available() else "gloo")
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+            dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                    device_id=torch.device("cuda", local))
+        else:
+            dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+    elif torch.cuda.is_available():
         torch.cuda.set_device(0)
     return ws, rank, local
 
@@ -297,13 +309,20 @@ def barrier(ws):
         dist.barrier()
 
 
-def max_over_ranks(x, ws):
+def max_over_ranks(x, ws, device=None):
+    """Max of a per-rank float over all ranks (the slowest rank sets the time)."""
     if ws == 1:
         return x
     import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dev = device or ("cuda" if dist.get_backend() == "nccl" else "cpu")
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def weak_scaling_value(ws, units_per_rank, max_ms_per_step):
+    """Whole-job throughput: units all ranks processed / the slowest rank's time."""
+    return ws * units_per_rank / (max_ms_per_step / 1e3)
 
 
 # ----------------------------------------------------------------------------- CPU baseline (oracle)
@@ -370,11 +389,13 @@ def run_reference(args, ws, rank):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--steps", type=int, default=500)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--config", default="llama7b_decode_f16")
     ap.add_argument("--cpu-budget", type=float, default=12.0, help="seconds of oracle time for cpu_baseline")
+    ap.add_argument("--seqs", type=int, default=None,
+                    help="fewer sequences of the named workload (small profiling cases)")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
 
@@ -389,7 +410,7 @@ def main():
     import paged_kv_cache_409_b200 as pkv
     pkv.load_library()
     dev = torch.device("cuda", torch.cuda.current_device())
-    step, cname = make_step(args.config, dev, rank)
+    step, cname = make_step(args.config, dev, rank, args.seqs)
     torch.cuda.synchronize()
 
     # warm-up, then exactly K timed steps between barriers
@@ -401,11 +422,15 @@ def main():
     barrier(ws)
     timer = EventTimer()
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    h0 = time.perf_counter()
+    torch.cuda.nvtx.range_push("timed")
     t0.record()
     for i in range(args.steps):
         step.run(timer=timer, step=i)
     t1.record()
+    torch.cuda.nvtx.range_pop()
     torch.cuda.synchronize()
+    clocks.mark(h0, time.perf_counter())
     clk = clocks.stop()
     barrier(ws)
     ms_total = max_over_ranks(t0.elapsed_time(t1), ws)
@@ -433,7 +458,7 @@ def main():
     pk, pk_kind = peaks()
     hbm = float(pk["hbm_gbs"])
     tokens_per_step = step.tokens
-    value = ws * tokens_per_step / (ms_step / 1e3)
+    value = weak_scaling_value(ws, tokens_per_step, ms_step)
     achieved = step.decode_bytes / (unit_ms / 1e3) / 1e9
     line = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": ws, "steps": args.steps,
@@ -450,7 +475,7 @@ def main():
         "roofline": {"bound": "hbm", "kernel": "paged_attention_decode (decode + merge kernels)",
                      "achieved": achieved, "peak": hbm, "peak_kind": pk_kind, "unit": "GB/s",
                      "frac": achieved / hbm, "frac_of_8000_nominal": achieved / 8000.0, "traffic": None},
-        "e2e": {"value": ws * tokens_per_step / (e2e_ms / 1e3), "unit": "tokens/s",
+        "e2e": {"value": weak_scaling_value(ws, tokens_per_step, e2e_ms), "unit": "tokens/s",
                 "h2d_bytes_per_step": e2e.h2d, "d2h_bytes_per_step": e2e.d2h, "ms_per_step": e2e_ms},
         "gpu_launches": step.launches_per_step() * args.steps,
         "clocks": clk,

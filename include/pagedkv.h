@@ -157,10 +157,12 @@ size_t pkv_decode_workspace_size(int num_seqs, int num_q_heads, int head_dim, in
                                  int partition_size);
 
 /* Split-K partition size (tokens) the library recommends for a batch on the
- * current device: 0 (no split) when the batch alone fills the GPU, else a
- * multiple of block_size.  Returns a negative pkv_status on bad input. */
+ * current device: 0 (no split) when the (sequence, KV head) pairs alone fill
+ * the GPU and no context is far longer than the mean, else a multiple of
+ * block_size.  total_context_tokens (sum of context_lens, 0 = unknown) lets
+ * it see a long tail.  Returns a negative pkv_status on bad input. */
 int pkv_decode_partition_size(int num_seqs, int num_kv_heads, int head_dim, int block_size,
-                              int max_context_len, int dtype);
+                              int max_context_len, int64_t total_context_tokens, int dtype);
 
 /*
  * Chunked prefill over the paged cache (guide page "Chunked Prefill": a long

@@ -69,7 +69,7 @@ def load_library():
     lib.pkv_paged_attention_decode.argtypes = [P, P, P, P, P, P, F, I, I, I, I, I, I, I64, I, I, I, P, SZ, P]
     lib.pkv_decode_workspace_size.argtypes = [I, I, I, I, I]
     lib.pkv_decode_workspace_size.restype = SZ
-    lib.pkv_decode_partition_size.argtypes = [I, I, I, I, I, I]
+    lib.pkv_decode_partition_size.argtypes = [I, I, I, I, I, I64, I]
     lib.pkv_paged_attention_prefill_chunk.argtypes = [P, P, P, P, P, P, P, I, I64, I, F, I, I, I, I, I, I64, I, P]
     lib.pkv_get_device_error.argtypes = [ctypes.POINTER(ctypes.c_uint32), P]
     for name in ("pkv_reshape_and_cache", "pkv_copy_blocks", "pkv_paged_attention_decode",
@@ -145,21 +145,23 @@ def decode_workspace_size(num_seqs, num_q_heads, head_dim, max_context_len, part
                                                          partition_size))
 
 
-def decode_partition_size(num_seqs, num_kv_heads, head_dim, block_size, max_context_len, dtype) -> int:
+def decode_partition_size(num_seqs, num_kv_heads, head_dim, block_size, max_context_len, dtype,
+                          total_context_tokens=0) -> int:
     code = DTYPE_CODE[dtype] if isinstance(dtype, torch.dtype) else int(dtype)
     rc = load_library().pkv_decode_partition_size(num_seqs, num_kv_heads, head_dim, block_size, max_context_len,
-                                                  code)
+                                                  int(total_context_tokens), code)
     if rc < 0:
         raise PagedKVError("decode_partition_size", rc)
     return rc
 
 
 def paged_attention_decode(out, query, key_cache, value_cache, block_tables, context_lens, scale, max_context_len,
-                           partition_size=None, workspace=None, stream=None):
+                           partition_size=None, workspace=None, stream=None, total_context_tokens=0):
     """Decode attention; ``out``/``query`` ``[S, Hq, D]``, pools ``[NB, B, Hkv, D]``.
 
-    ``partition_size`` None picks the library's recommendation; a workspace
-    is allocated here when one is needed and none is given.
+    ``partition_size`` None picks the library's recommendation (given the
+    optional host-side ``total_context_tokens``); a workspace is allocated
+    here when one is needed and none is given.
     """
     lib = load_library()
     S, Hq, D = query.shape
@@ -168,7 +170,7 @@ def paged_attention_decode(out, query, key_cache, value_cache, block_tables, con
     if block_tables.dtype != torch.int32 or context_lens.dtype != torch.int32:
         raise ValueError("block_tables and context_lens must be int32")
     if partition_size is None:
-        partition_size = decode_partition_size(S, Hkv, D, B, max_context_len, query.dtype)
+        partition_size = decode_partition_size(S, Hkv, D, B, max_context_len, query.dtype, total_context_tokens)
     need = decode_workspace_size(S, Hq, D, max_context_len, partition_size) if partition_size else 0
     if need and (workspace is None or workspace.numel() * workspace.element_size() < need):
         workspace = torch.empty(need, dtype=torch.uint8, device=query.device)

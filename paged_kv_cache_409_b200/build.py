@@ -14,7 +14,7 @@ CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libpagedkv.so")
 SOURCES = ["pagedkv.cu"]
-DEPENDS = ["pagedkv.cu", "ptx.cuh", "index_kernels.cuh", "decode.cuh", "prefill.cuh"]
+DEPENDS = ["pagedkv.cu", "ptx.cuh", "index_kernels.cuh", "decode.cuh", "decode_mma.cuh", "prefill.cuh"]
 
 
 def nvcc() -> str:

@@ -38,11 +38,10 @@ struct DecodeParams {
     int num_partitions;    // P (grid extent)
 };
 
-constexpr int kDecodeWarps = 4;
-constexpr int kDecodeThreads = kDecodeWarps * 32;
-
-template <typename T, int D, int B, int G, int NST>
+template <typename T, int D, int B, int G, int NST, int NW>
 struct DecodeCfg {
+    static constexpr int WARPS = NW;
+    static constexpr int THREADS = NW * 32;
     static constexpr int TB = Elem<T>::kBytes;
     static constexpr int PANEL = 128 / TB;              // elements per 128-byte swizzle row
     static constexpr int NP = D * TB / 128;             // panels per row
@@ -53,15 +52,15 @@ struct DecodeCfg {
     static constexpr int LPT = 32 / B;                  // lanes per token in Q.K
     static constexpr int CPL = NCH / LPT;               // chunks per lane in Q.K
     static constexpr int DPL = D / 32;                  // output dims per lane in P.V
-    static constexpr int STAGES_BYTES = kDecodeWarps * NST * STAGE;
+    static constexpr int STAGES_BYTES = NW * NST * STAGE;
     static constexpr int Q_OFF = STAGES_BYTES;
     static constexpr int BT_OFF = Q_OFF + G * D * 4;
-    static constexpr int RED_BYTES = kDecodeWarps * G * (D + 2) * 4;
+    static constexpr int RED_BYTES = NW * G * (D + 2) * 4;
     static_assert(TILE % 1024 == 0, "tiles must keep 1024-byte alignment for the 128-byte swizzle");
     static_assert(NCH % LPT == 0 && D % 32 == 0 && B <= 32, "unsupported decode shape");
     static_assert(RED_BYTES <= STAGES_BYTES, "merge scratch must fit in the stage buffers");
     static size_t smem_bytes(int pb) {
-        return 1024 + BT_OFF + static_cast<size_t>(pb) * 4 + 16 + kDecodeWarps * NST * 8;
+        return 1024 + BT_OFF + static_cast<size_t>(pb) * 4 + 16 + NW * NST * 8;
     }
 };
 
@@ -78,11 +77,53 @@ __device__ __forceinline__ int decode_seq_blocks(int ctx, int block_size, int ma
     return nb;
 }
 
-template <typename T, int D, int B, int G, int NST>
-__global__ void __launch_bounds__(kDecodeThreads) paged_decode_kernel(const DecodeParams p,
+// Combine the NW warps' (max, sum, output) states of one CTA, left in
+// shared memory as red_m[w][h], red_l[w][h], red_o[w][h][D], and write the
+// output row (single partition) or the partition's partial to the workspace.
+template <typename T, int D, int G, int NW>
+__device__ __forceinline__ void decode_finish(const DecodeParams& p, const float* red_m, int s, int g, int part,
+                                              bool direct) {
+    const float* red_l = red_m + NW * G;
+    const float* red_o = red_l + NW * G;
+    const int64_t row0 = static_cast<int64_t>(s) * p.num_q_heads + static_cast<int64_t>(g) * G;
+    for (int i = threadIdx.x; i < G * D; i += NW * 32) {
+        const int h = i / D, d = i - h * D;
+        float mx = -INFINITY;
+#pragma unroll
+        for (int w = 0; w < NW; ++w) mx = fmaxf(mx, red_m[w * G + h]);
+        float sum = 0.f, o = 0.f;
+        if (mx != -INFINITY) {
+#pragma unroll
+            for (int w = 0; w < NW; ++w) {
+                const float mw = red_m[w * G + h];
+                if (mw != -INFINITY) {
+                    const float f = exp2f(mw - mx);
+                    sum += red_l[w * G + h] * f;
+                    o += red_o[(w * G + h) * D + d] * f;
+                }
+            }
+        }
+        const float val = mx != -INFINITY ? o / sum : 0.f;
+        if (direct) {
+            reinterpret_cast<T*>(p.out)[(row0 + h) * D + d] = Elem<T>::from_f(val);
+        } else {
+            const int64_t pi = (row0 + h) * p.num_partitions + part;
+            p.ws_out[pi * D + d] = val;
+            if (d == 0) {
+                p.ws_max[pi] = mx;
+                p.ws_sum[pi] = sum;
+            }
+        }
+    }
+}
+
+template <typename T, int D, int B, int G, int NST, int NW>
+__global__ void __launch_bounds__(NW * 32) paged_decode_kernel(const DecodeParams p,
                                                                       const __grid_constant__ CUtensorMap tm_k,
                                                                       const __grid_constant__ CUtensorMap tm_v) {
-    using C = DecodeCfg<T, D, B, G, NST>;
+    using C = DecodeCfg<T, D, B, G, NST, NW>;
+    constexpr int kDecodeWarps = NW;
+    constexpr int kDecodeThreads = NW * 32;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = align_1024(smem_raw);
 
@@ -292,36 +333,7 @@ __global__ void __launch_bounds__(kDecodeThreads) paged_decode_kernel(const Deco
         for (int j = 0; j < C::DPL; ++j) red_o[(warp * G + h) * D + pd0 + j] = acc[h][j];
     __syncthreads();
 
-    const int64_t row0 = static_cast<int64_t>(s) * p.num_q_heads + static_cast<int64_t>(g) * G;
-    for (int i = threadIdx.x; i < G * D; i += kDecodeThreads) {
-        const int h = i / D, d = i - h * D;
-        float mx = -INFINITY;
-#pragma unroll
-        for (int w = 0; w < kDecodeWarps; ++w) mx = fmaxf(mx, red_m[w * G + h]);
-        float sum = 0.f, o = 0.f;
-        if (mx != -INFINITY) {
-#pragma unroll
-            for (int w = 0; w < kDecodeWarps; ++w) {
-                const float mw = red_m[w * G + h];
-                if (mw != -INFINITY) {
-                    const float f = exp2f(mw - mx);
-                    sum += red_l[w * G + h] * f;
-                    o += red_o[(w * G + h) * D + d] * f;
-                }
-            }
-        }
-        const float val = mx != -INFINITY ? o / sum : 0.f;
-        if (direct) {
-            reinterpret_cast<T*>(p.out)[(row0 + h) * D + d] = Elem<T>::from_f(val);
-        } else {
-            const int64_t pi = (row0 + h) * p.num_partitions + part;
-            p.ws_out[pi * D + d] = val;
-            if (d == 0) {
-                p.ws_max[pi] = mx;
-                p.ws_sum[pi] = sum;
-            }
-        }
-    }
+    decode_finish<T, D, G, NW>(p, red_m, s, g, part, direct);
 }
 
 // ---- log-sum-exp merge of the partitions: one warp per (sequence, q head).

@@ -13,7 +13,8 @@
 //                        (input dtype) into shared memory in the 128-byte
 //                        swizzled K-major layout;
 //   O_t = P . V          tcgen05.mma, A = P (K-major), B = V tile (MN-major),
-//                        N = head_dim, into a second tensor-memory region;
+//                        N = head_dim, into a second tensor-memory region
+//                        (bf16: P as hi + lo terms, two MMAs per K step);
 //   O  = O * alpha + O_t kept in registers (one row per thread).
 // K/V tiles are double-buffered: the TMA for tile j+2 is issued as soon as
 // the P.V product of tile j has consumed its buffer.
@@ -51,10 +52,15 @@ struct PrefillCfg {
     static constexpr int KT_BYTES = NP * BN * 128;
     static constexpr int STAGE = 2 * KT_BYTES;
     static constexpr int P_BYTES = (BN / 64) * BM * 128;
+    // bf16 keeps only 8 significant bits: P goes to the tensor cores as two
+    // bf16 terms (P = hi + lo, |lo| <= 2^-8 |P|), which brings the rounding of
+    // the attention weights below the output tolerance.  fp16 P is one term.
+    static constexpr bool SPLIT_P = Elem<T>::kCuType == CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
     static constexpr int Q_OFF = 0;
     static constexpr int ST_OFF = Q_OFF + Q_BYTES;
     static constexpr int P_OFF = ST_OFF + 2 * STAGE;
-    static constexpr int BAR_OFF = P_OFF + P_BYTES;
+    static constexpr int PLO_OFF = P_OFF + P_BYTES;
+    static constexpr int BAR_OFF = PLO_OFF + (SPLIT_P ? P_BYTES : 0);
     static constexpr int SMEM = 1024 + BAR_OFF + 64;
     static constexpr uint32_t TMEM_COLS = 256;
     static constexpr uint32_t S_COL = 0;
@@ -73,6 +79,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1) paged_prefill_kernel(const
     uint8_t* smem = align_1024(smem_raw);
     uint8_t* q_s = smem + C::Q_OFF;
     uint8_t* p_s = smem + C::P_OFF;
+    uint8_t* plo_s = smem + C::PLO_OFF;
     uint64_t* bar_q = reinterpret_cast<uint64_t*>(smem + C::BAR_OFF);
     uint64_t* bar_kv = bar_q + 1;  // [2]
     uint64_t* bar_s = bar_q + 3;
@@ -162,6 +169,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1) paged_prefill_kernel(const
     constexpr uint32_t IDESC_O = umma_idesc_f16(128, D, kBf16, false, true);
     const uint32_t q_addr = smem_u32(q_s);
     const uint32_t p_addr = smem_u32(p_s);
+    const uint32_t plo_addr = smem_u32(plo_s);
 
     float o[D];
 #pragma unroll
@@ -236,7 +244,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1) paged_prefill_kernel(const
 #pragma unroll
         for (int c = 0; c < C::BN / 32; ++c) {
             tmem_ld32(t_s + c * 32, v);
-            uint32_t packed[16];
+            uint32_t packed[16], packed_lo[16];
 #pragma unroll
             for (int i = 0; i < 32; i += 2) {
                 const int key = tile_k0 + c * 32 + i;
@@ -244,13 +252,21 @@ __global__ void __launch_bounds__(kPrefillThreads, 1) paged_prefill_kernel(const
                 const float p1 = key + 1 <= qpos ? exp2f(v[i + 1] * p.scale_log2 - mnew) : 0.f;
                 tsum += p0 + p1;
                 packed[i / 2] = Elem<T>::pack(p0, p1);
+                if constexpr (C::SPLIT_P) {
+                    const float2 hi = Elem<T>::pair(packed[i / 2]);
+                    packed_lo[i / 2] = Elem<T>::pack(p0 - hi.x, p1 - hi.y);
+                }
             }
             // keys c*32 .. c*32+31 -> panel c/2, 16-byte chunks 4*(c%2) .. +3
 #pragma unroll
             for (int q = 0; q < 4; ++q) {
                 const int cc = 4 * (c % 2) + q;
-                *reinterpret_cast<uint4*>(p_s + (c / 2) * (C::BM * 128) + row * 128 + ((cc ^ (row & 7)) << 4)) =
+                const int off = (c / 2) * (C::BM * 128) + row * 128 + ((cc ^ (row & 7)) << 4);
+                *reinterpret_cast<uint4*>(p_s + off) =
                     make_uint4(packed[4 * q], packed[4 * q + 1], packed[4 * q + 2], packed[4 * q + 3]);
+                if constexpr (C::SPLIT_P)
+                    *reinterpret_cast<uint4*>(plo_s + off) = make_uint4(packed_lo[4 * q], packed_lo[4 * q + 1],
+                                                                        packed_lo[4 * q + 2], packed_lo[4 * q + 3]);
             }
         }
         lsum = lsum * alpha + tsum;
@@ -264,8 +280,10 @@ __global__ void __launch_bounds__(kPrefillThreads, 1) paged_prefill_kernel(const
 #pragma unroll
             for (int kk = 0; kk < C::BN / 16; ++kk) {
                 const uint32_t poff = (kk / 4) * (C::BM * 128) + (kk % 4) * 32;
-                umma_f16_ss(t_o - lane_base, smem_desc_sw128(p_addr + poff, 16, 1024),
-                            smem_desc_sw128(v_addr + kk * 16 * 128, C::BN * 128, 1024), IDESC_O, kk > 0);
+                const uint64_t vdesc = smem_desc_sw128(v_addr + kk * 16 * 128, C::BN * 128, 1024);
+                umma_f16_ss(t_o - lane_base, smem_desc_sw128(p_addr + poff, 16, 1024), vdesc, IDESC_O, kk > 0);
+                if constexpr (C::SPLIT_P)
+                    umma_f16_ss(t_o - lane_base, smem_desc_sw128(plo_addr + poff, 16, 1024), vdesc, IDESC_O, 1);
             }
             umma_commit(bar_o);
         }

@@ -48,11 +48,19 @@ def test_workspace_size_arithmetic(lib):
     assert pkv.decode_workspace_size(64, 32, 128, 2048, 512) == 2 * rows * 4 + rows * 128 * 4
 
 
-def test_partition_heuristic_is_block_multiple(lib):
+def test_partition_heuristic(lib):
+    # large batches: one CTA per (sequence, KV head), no split
+    assert pkv.decode_partition_size(64, 32, 128, 16, 2048, 1) == 0
+    assert pkv.decode_partition_size(192, 8, 128, 32, 32768, 2) == 0
+    # small batches: block-multiple partitions of at least 256 tokens, shorter than the context
     for B in (8, 16, 32):
-        p = pkv.decode_partition_size(64, 32, 128, B, 2048, 1)
-        assert p == 0 or p % B == 0
-    assert pkv.decode_partition_size(64, 32, 128, 16, 300, 1) == 0
+        p = pkv.decode_partition_size(2, 2, 128, B, 10000, 1)
+        assert p % B == 0 and 256 <= p < 10000
+    assert pkv.decode_partition_size(1, 1, 128, 16, 200, 1) == 0
+    # a long tail (max far above the mean) is cut at 1.5x the mean
+    p = pkv.decode_partition_size(256, 8, 128, 16, 4096, 2, total_context_tokens=256 * 1436)
+    assert p == 2160
+    assert pkv.decode_partition_size(192, 8, 128, 32, 32768, 2, total_context_tokens=192 * 16500) == 0
 
 
 def test_host_rejections_before_launch(lib):
