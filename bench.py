@@ -172,7 +172,7 @@ class MixedStep(DecodeStep):
             timer.end()
 
 
-def make_step(name, device, rank, seqs=None):
+def make_step(name, device, rank, seqs=None, layers=None):
     from paged_kv_cache_409_b200 import workloads
     if name == "llama7b_decode_f16":
         w = workloads.llama7b_decode_f16(device=device, seed=1002 + rank, num_seqs=seqs or 64)
@@ -181,10 +181,12 @@ def make_step(name, device, rank, seqs=None):
         return DecodeStep(workloads.tiny_decode_f32(device=device)), name
     if name == "gqa70b_decode_bf16":
         free, _ = torch.cuda.mem_get_info()
-        per_layer = 1.75e9  # pools of one layer (~1.62 GB) plus headroom
-        layers = int(max(1, min(80, (free - 8e9) // per_layer)))
-        w = workloads.gqa70b_decode_bf16(device=device, num_layers=layers, seed=1003 + rank)
-        return DecodeStep(w, layers_per_step=80), f"gqa70b_decode_bf16 ({layers} distinct layer caches cycled)"
+        per_layer = 1.75e9 * (seqs or 256) / 256  # pools of one layer (~1.62 GB at 256 sequences) plus headroom
+        fit = int(max(1, min(80, (free - 8e9) // per_layer)))
+        layers = min(fit, layers) if layers else fit
+        w = workloads.gqa70b_decode_bf16(device=device, num_layers=layers, seed=1003 + rank, num_seqs=seqs or 256)
+        note = "" if layers == 80 else f", {layers} distinct layer pools cycled"
+        return DecodeStep(w, layers_per_step=80), f"gqa70b_decode_bf16 (80 layers per step{note})"
     if name == "shared_prefix_decode_f16":
         sp = workloads.shared_prefix_decode_f16(device=device, seed=1004 + rank)
         st = DecodeStep(sp.step)
@@ -194,7 +196,8 @@ def make_step(name, device, rank, seqs=None):
                                  torch.from_numpy(sp.private_slots).to(device))
         return st, name
     if name == "mixed_step_bf16":
-        return MixedStep(workloads.mixed_step_bf16(device=device, seed=1005 + rank)), name
+        m = workloads.mixed_step_bf16(device=device, seed=1005 + rank, num_decode=seqs or 192)
+        return MixedStep(m), name + (f" ({seqs} decode sequences)" if seqs else "")
     raise SystemExit(f"unknown config {name}")
 
 
@@ -396,6 +399,7 @@ def main():
     ap.add_argument("--cpu-budget", type=float, default=12.0, help="seconds of oracle time for cpu_baseline")
     ap.add_argument("--seqs", type=int, default=None,
                     help="fewer sequences of the named workload (small profiling cases)")
+    ap.add_argument("--layers", type=int, default=None, help="cap on distinct layer pools (gqa70b_decode_bf16)")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
 
@@ -410,7 +414,7 @@ def main():
     import paged_kv_cache_409_b200 as pkv
     pkv.load_library()
     dev = torch.device("cuda", torch.cuda.current_device())
-    step, cname = make_step(args.config, dev, rank, args.seqs)
+    step, cname = make_step(args.config, dev, rank, args.seqs, args.layers)
     torch.cuda.synchronize()
 
     # warm-up, then exactly K timed steps between barriers
