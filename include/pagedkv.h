@@ -196,6 +196,38 @@ int pkv_paged_attention_prefill_chunk(void* out, const void* query, const void* 
                                       int block_size, int max_blocks_per_seq, int64_t num_blocks,
                                       int dtype, pkv_stream_t stream);
 
+/*
+ * pkv_paged_attention_decode_static_scratch -- the same decode attention as
+ * pkv_paged_attention_decode, for callers that cannot allocate device memory
+ * at the call site (code running inside another framework's allocator, a
+ * plugin that only receives the operation's own tensors, a serving loop that
+ * must not call the allocator between steps).  The vLLM pages have no
+ * counterpart: this is a library convenience.
+ *
+ * Arguments are those of pkv_paged_attention_decode without the workspace:
+ * the caller still passes every input and output buffer.  The split-K scratch
+ * is a library-owned device array of PKV_STATIC_DECODE_SCRATCH_BYTES bytes,
+ * present on every GPU that loads the library until the process exits.  The
+ * call allocates nothing and calls no allocating routine.
+ *   - A request that needs more scratch than that (see
+ *     pkv_decode_workspace_size) returns PKV_EWORKSPACE before any device work;
+ *     partition_size == 0 needs none.
+ *   - The first call on a device looks up the array's device address
+ *     (cudaGetSymbolAddress) with that device current; make that first call
+ *     before any stream capture.
+ *   - All calls share the one array, which keeps the last call's contents.
+ *     The decode writes every partial it later reads, so nothing needs to
+ *     start at zero.  Calls whose executions overlap on the GPU (different
+ *     streams, or host threads) race on the array: serialise them.
+ */
+#define PKV_STATIC_DECODE_SCRATCH_BYTES (32u << 20)
+int pkv_paged_attention_decode_static_scratch(void* out, const void* query, const void* key_cache,
+                                              const void* value_cache, const int32_t* block_tables,
+                                              const int32_t* context_lens, float scale, int num_seqs,
+                                              int num_q_heads, int num_kv_heads, int head_dim, int block_size,
+                                              int max_blocks_per_seq, int64_t num_blocks, int max_context_len,
+                                              int partition_size, int dtype, pkv_stream_t stream);
+
 /* Read, and reset to 0, the current device's error word (PKV_DEVERR_* bits)
  * after all work queued on `stream` so far.  Synchronises `stream`. */
 int pkv_get_device_error(uint32_t* host_err, pkv_stream_t stream);

@@ -621,3 +621,73 @@ int pkv_get_device_error(uint32_t* host_err, pkv_stream_t stream) {
 }
 
 }  // extern "C"
+
+// ============================================================ decode without caller-provided scratch
+// Some callers cannot allocate device memory when they call decode: code that
+// runs inside another framework's allocator-controlled region, plugins that are
+// handed only the tensors of one operation, or a serving loop that must not
+// touch the allocator between steps.  For them the split-K scratch lives in a
+// file-scope device array owned by the library.  The name below is a host-side
+// stand-in in host code, so its device address is looked up once per device
+// with cudaGetSymbolAddress and passed to the kernels as an ordinary pointer.
+static __device__ __align__(256) unsigned char g_static_decode_scratch[PKV_STATIC_DECODE_SCRATCH_BYTES];
+
+namespace {
+
+// Device address of the scratch array on the current device, looked up once
+// per device (with that device current) and cached.
+void* static_scratch_address(int* rc) {
+    static std::mutex mu;
+    static void* addr[64] = {};
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) {
+        *rc = cuda_fail(e, "cudaGetDevice");
+        return nullptr;
+    }
+    if (dev < 0 || dev >= 64) {
+        *rc = PKV_EUNSUPPORTED;
+        return nullptr;
+    }
+    std::lock_guard<std::mutex> lock(mu);
+    if (!addr[dev]) {
+        void* p = nullptr;
+        e = cudaGetSymbolAddress(&p, g_static_decode_scratch);
+        if (e != cudaSuccess || !p) {
+            *rc = cuda_fail(e != cudaSuccess ? e : cudaErrorInvalidSymbol, "cudaGetSymbolAddress(scratch)");
+            return nullptr;
+        }
+        addr[dev] = p;
+    }
+    *rc = PKV_OK;
+    return addr[dev];
+}
+
+}  // namespace
+
+extern "C" int pkv_paged_attention_decode_static_scratch(
+    void* out, const void* query, const void* key_cache, const void* value_cache, const int32_t* block_tables,
+    const int32_t* context_lens, float scale, int num_seqs, int num_q_heads, int num_kv_heads, int head_dim,
+    int block_size, int max_blocks_per_seq, int64_t num_blocks, int max_context_len, int partition_size, int dtype,
+    pkv_stream_t stream) {
+    // Size check first: a request that needs more scratch than the array holds
+    // is refused before any device work.
+    int64_t ps = partition_size;
+    if (ps > 0 && block_size > 0 && max_context_len > 0) {
+        const int64_t max_blocks = ceil_div(max_context_len, block_size);
+        ps = std::min<int64_t>(ps, max_blocks * block_size);  // the clamp the decode applies
+    }
+    const size_t need = ps > 0 ? pkv_decode_workspace_size(num_seqs, num_q_heads, head_dim, max_context_len, (int)ps)
+                               : 0;
+    if (need > (size_t)PKV_STATIC_DECODE_SCRATCH_BYTES) return PKV_EWORKSPACE;
+    void* scratch = nullptr;
+    if (need > 0) {
+        int rc = PKV_OK;
+        scratch = static_scratch_address(&rc);
+        if (rc) return rc;
+    }
+    return pkv_paged_attention_decode(out, query, key_cache, value_cache, block_tables, context_lens, scale, num_seqs,
+                                      num_q_heads, num_kv_heads, head_dim, block_size, max_blocks_per_seq,
+                                      num_blocks, max_context_len, partition_size, dtype, scratch,
+                                      need > 0 ? (size_t)PKV_STATIC_DECODE_SCRATCH_BYTES : 0, stream);
+}
