@@ -1,23 +1,32 @@
 // prefill.cuh -- causal chunked-prefill attention over the paged cache on the
-// tcgen05 tensor cores.
+// tcgen05 tensor cores, warp-specialised.
 //
-// One CTA (128 threads) per (chunk, query tile, KV head).  A query tile is
-// 128 rows = 128/G query tokens x the G query heads that share the KV head, so
-// every K/V tile staged in shared memory serves all of them.  Per key tile of
-// 128 keys (128/B physical blocks, each fetched by its own TMA box through the
-// block table):
-//   S  = Q . K^T        tcgen05.mma, A = Q (K-major), B = K tile (K-major),
-//                        M = 128, N = 128, accumulator in tensor memory;
-//   P  = exp2(S*scale*log2e - m)   one thread per row reads its row of S from
-//                        tensor memory, keeps the running max / sum, writes P
-//                        (input dtype) into shared memory in the 128-byte
-//                        swizzled K-major layout;
-//   O_t = P . V          tcgen05.mma, A = P (K-major), B = V tile (MN-major),
-//                        N = head_dim, into a second tensor-memory region
-//                        (bf16: P as hi + lo terms, two MMAs per K step);
-//   O  = O * alpha + O_t kept in registers (one row per thread).
-// K/V tiles are double-buffered: the TMA for tile j+2 is issued as soon as
-// the P.V product of tile j has consumed its buffer.
+// One CTA per (query tile, chunk, KV head).  A query tile is 128 rows = 128/G
+// query tokens x the G query heads that share the KV head, so every K/V tile
+// staged in shared memory serves all of them.  Key tiles are 128 keys =
+// 128/B physical blocks, each fetched by its own TMA box through the block
+// table.
+//
+// Roles (160 threads):
+//  * warp 4 -- producer.  A loop that polls the pipeline's mbarriers
+//    (test_wait, which never suspends) issues, from lane 0,, whenever its inputs are ready and its target buffer is
+//    free: the TMA loads of K and V tiles (two stages each; K of tile j+2
+//    as soon as Q.K^T of tile j is done, V of tile j+2 as soon as P.V of tile
+//    j is done), S_j = Q . K_j^T (tcgen05.mma, M = N = 128, into one of two
+//    S buffers in tensor memory), and O_j = P_j . V_j (N = head_dim, into one
+//    of two O buffers; bf16 P goes in as hi + lo terms).  The warp's lanes
+//    prefetch the next tiles' block ids (one per lane) so that table reads
+//    overlap the pipeline.
+//  * warps 0-3 -- one query row per thread.  For tile j: read S_j from tensor
+//    memory (row max), fold the finished P.V product of tile j-1 into the
+//    register accumulator (online-softmax rescale), write P_j = exp2(S_j *
+//    scale * log2 e - m) to shared memory in the 128-byte-swizzled K-major
+//    layout, and release the S buffer.  The Q.K^T product of tile j+1 runs
+//    on the tensor cores meanwhile, and P.V of tile j-1 during the max pass.
+// Every wait is bounded; a wait that gives up raises a CTA-wide abort flag
+// that ends the other roles' waits too.  In the softmax warps every wait
+// outcome is agreed by the whole warp (the tcgen05.ld that follow are
+// warp-collective).
 #pragma once
 
 #include "ptx.cuh"
@@ -39,7 +48,8 @@ struct PrefillParams {
     int q_tiles;  // query tiles per chunk in the grid
 };
 
-constexpr int kPrefillThreads = 128;
+constexpr int kPrefillSoftmaxWarps = 4;
+constexpr int kPrefillThreads = (kPrefillSoftmaxWarps + 1) * 32;
 
 template <typename T, int D, int G>
 struct PrefillCfg {
@@ -49,22 +59,23 @@ struct PrefillCfg {
     static constexpr int NP = D / 64;      // 128-byte panels per row (16-bit types)
     static constexpr int PANEL = 64;
     static constexpr int Q_BYTES = NP * BM * 128;
-    static constexpr int KT_BYTES = NP * BN * 128;
-    static constexpr int STAGE = 2 * KT_BYTES;
+    static constexpr int KT_BYTES = NP * BN * 128;  // one K (or V) tile
     static constexpr int P_BYTES = (BN / 64) * BM * 128;
     // bf16 keeps only 8 significant bits: P goes to the tensor cores as two
-    // bf16 terms (P = hi + lo, |lo| <= 2^-8 |P|), which brings the rounding of
-    // the attention weights below the output tolerance.  fp16 P is one term.
+    // bf16 terms (P = hi + lo: hi the top 16 bits of P, lo the remainder
+    // rounded, |lo| < 2^-7 |P|), which brings the rounding of the attention
+    // weights far below the output tolerance.  fp16 P is one term.
     static constexpr bool SPLIT_P = Elem<T>::kCuType == CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
     static constexpr int Q_OFF = 0;
-    static constexpr int ST_OFF = Q_OFF + Q_BYTES;
-    static constexpr int P_OFF = ST_OFF + 2 * STAGE;
+    static constexpr int K_OFF = Q_OFF + Q_BYTES;
+    static constexpr int V_OFF = K_OFF + 2 * KT_BYTES;
+    static constexpr int P_OFF = V_OFF + 2 * KT_BYTES;
     static constexpr int PLO_OFF = P_OFF + P_BYTES;
     static constexpr int BAR_OFF = PLO_OFF + (SPLIT_P ? P_BYTES : 0);
-    static constexpr int SMEM = 1024 + BAR_OFF + 64;
-    static constexpr uint32_t TMEM_COLS = 256;
-    static constexpr uint32_t S_COL = 0;
-    static constexpr uint32_t O_COL = 128;
+    static constexpr int NBAR = 16;
+    static constexpr int SMEM = 1024 + BAR_OFF + NBAR * 8;
+    static constexpr uint32_t TMEM_COLS = 512;
+    static constexpr uint32_t S_COL0 = 0, O_COL0 = 256;  // S buffers at 0 / 128, O buffers at 256 / 384
     static_assert(D == 64 || D == 128, "head_dim");
 };
 
@@ -77,20 +88,26 @@ __global__ void __launch_bounds__(kPrefillThreads, 1) paged_prefill_kernel(const
     const int B = p.block_size;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = align_1024(smem_raw);
-    uint8_t* q_s = smem + C::Q_OFF;
-    uint8_t* p_s = smem + C::P_OFF;
-    uint8_t* plo_s = smem + C::PLO_OFF;
-    uint64_t* bar_q = reinterpret_cast<uint64_t*>(smem + C::BAR_OFF);
-    uint64_t* bar_kv = bar_q + 1;  // [2]
-    uint64_t* bar_s = bar_q + 3;
-    uint64_t* bar_o = bar_q + 4;
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar_q + 5);
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::BAR_OFF);
+    uint64_t* q_full = bars + 0;
+    uint64_t* k_full = bars + 1;   // [2]
+    uint64_t* v_full = bars + 3;   // [2]
+    uint64_t* s_full = bars + 5;   // [2]  Q.K^T done (tcgen05.commit)
+    uint64_t* s_free = bars + 7;   // [2]  softmax finished reading S
+    uint64_t* p_full = bars + 9;   //      P of the current tile written
+    uint64_t* o_full = bars + 10;  // [2]  P.V done (tcgen05.commit)
+    uint64_t* o_free = bars + 12;  // [2]  softmax folded O into registers
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 14);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + 15);
 
-    const int per_chunk = p.q_tiles * p.num_kv_heads;
-    const int r = blockIdx.x / per_chunk;
-    const int rem = blockIdx.x - r * per_chunk;
-    const int qt = rem / p.num_kv_heads;
-    const int g = rem - qt * p.num_kv_heads;
+    // Launch order: query tile outermost, last tile first -- later tiles of a
+    // chunk attend to more keys, so the longest CTAs start in the first wave
+    // and the short ones fill the tail.
+    const int ctas_per_qtile = p.num_chunks * p.num_kv_heads;
+    const int qt = p.q_tiles - 1 - static_cast<int>(blockIdx.x) / ctas_per_qtile;
+    const int rem = static_cast<int>(blockIdx.x) % ctas_per_qtile;
+    const int r = rem / p.num_kv_heads;
+    const int g = rem % p.num_kv_heads;
     const int tid = threadIdx.x;
     const int warp = tid >> 5;
 
@@ -114,196 +131,316 @@ __global__ void __launch_bounds__(kPrefillThreads, 1) paged_prefill_kernel(const
         tmem_relinquish();
     }
     if (tid == 0) {
-        mbar_init(bar_q, 1);
-        mbar_init(&bar_kv[0], 1);
-        mbar_init(&bar_kv[1], 1);
-        mbar_init(bar_s, 1);
-        mbar_init(bar_o, 1);
+        mbar_init(q_full, 1);
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&k_full[i], 1);
+            mbar_init(&v_full[i], 1);
+            mbar_init(&s_full[i], 1);
+            mbar_init(&s_free[i], kPrefillSoftmaxWarps * 32);
+            mbar_init(&o_full[i], 1);
+            mbar_init(&o_free[i], kPrefillSoftmaxWarps * 32);
+        }
+        mbar_init(p_full, kPrefillSoftmaxWarps * 32);
+        *abort_flag = 0;
         fence_mbar_init();
     }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
-    const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
-    const uint32_t t_s = tmem + lane_base + C::S_COL;
-    const uint32_t t_o = tmem + lane_base + C::O_COL;
+    constexpr bool kBf16 = Elem<T>::kCuType == CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
 
-    auto issue_kv = [&](int j) {  // thread 0 only
-        const int st = j & 1;
-        uint8_t* kd = smem + C::ST_OFF + st * C::STAGE;
-        uint8_t* vd = kd + C::KT_BYTES;
-        mbar_arrive_expect_tx(&bar_kv[st], C::STAGE);
-#pragma unroll 1
-        for (int i = 0; i < C::BN / B; ++i) {
-            const int lb = j * (C::BN / B) + i;
-            int id = lb < nblk ? bt_row[lb] : -1;
-            if (lb < nblk && (id < 0 || id >= p.num_blocks)) {
+    if (warp == kPrefillSoftmaxWarps) {
+        // ================================================================ producer (whole warp, lane 0 issues)
+        const int lane = tid & 31;
+        const bool leader = lane == 0;
+        constexpr uint32_t IDESC_S = umma_idesc_f16(128, C::BN, kBf16, false, false);
+        constexpr uint32_t IDESC_O = umma_idesc_f16(128, D, kBf16, false, true);
+        const uint32_t q_addr = smem_u32(smem + C::Q_OFF);
+        const uint32_t p_addr = smem_u32(smem + C::P_OFF);
+        const uint32_t plo_addr = smem_u32(smem + C::PLO_OFF);
+        const int per_tile = C::BN / B;  // blocks per key tile (4..16)
+        // Block ids of key tile j, one per lane (lane < per_tile), fetched ahead
+        // of use so that the table read overlaps the pipeline.
+        // (the load is only issued here; its value is first used, and checked,
+        // when the tile is loaded, so the read overlaps the pipeline)
+        auto fetch_ids = [&](int j) -> int {
+            const int lb = j * per_tile + lane;
+            return (lane < per_tile && lb < nblk) ? bt_row[lb] : -1;
+        };
+        auto load_tile = [&](const CUtensorMap* map, int off, uint64_t* full, int j, int ids) {
+            const int st = j & 1;
+            uint8_t* dst = smem + off + st * C::KT_BYTES;
+            const int lb = j * per_tile + lane;
+            if (lane < per_tile && lb < nblk && (ids < 0 || ids >= p.num_blocks)) {
                 flag_error(PKV_DEVERR_BLOCK_ID);
-                id = -1;
+                ids = -1;
             }
-            const int coord = id >= 0 ? id : static_cast<int>(p.num_blocks);  // out of range: zero fill
+            if (leader) mbar_arrive_expect_tx(&full[st], C::KT_BYTES);
+            for (int i = 0; i < per_tile; ++i) {
+                const int id = __shfl_sync(0xffffffffu, ids, i);
+                const int coord = id >= 0 ? id : static_cast<int>(p.num_blocks);  // out of range: zero fill
+                if (leader) {
 #pragma unroll
-            for (int pn = 0; pn < C::NP; ++pn) {
-                tma_load_4d(kd + pn * C::BN * 128 + i * B * 128, &tm_k, pn * C::PANEL, g, 0, coord, &bar_kv[st]);
-                tma_load_4d(vd + pn * C::BN * 128 + i * B * 128, &tm_v, pn * C::PANEL, g, 0, coord, &bar_kv[st]);
-            }
-        }
-    };
-
-    if (tid == 0) {
-        mbar_arrive_expect_tx(bar_q, C::Q_BYTES);
-#pragma unroll
-        for (int pn = 0; pn < C::NP; ++pn)
-            tma_load_3d(q_s + pn * C::BM * 128, &tm_q, pn * C::PANEL, g * G, q0 + qt * C::TT, bar_q);
-        issue_kv(0);
-        if (nkt > 1) issue_kv(1);
-    }
-
-    // this thread's row
-    const int row = tid;
-    const int tok = qt * C::TT + row / G;
-    const int qpos = c0 + tok;  // absolute position of the row's query
-    constexpr bool kBf16 = sizeof(T) == 2 && Elem<T>::kCuType == CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
-    constexpr uint32_t IDESC_S = umma_idesc_f16(128, C::BN, kBf16, false, false);
-    constexpr uint32_t IDESC_O = umma_idesc_f16(128, D, kBf16, false, true);
-    const uint32_t q_addr = smem_u32(q_s);
-    const uint32_t p_addr = smem_u32(p_s);
-    const uint32_t plo_addr = smem_u32(plo_s);
-
-    float o[D];
-#pragma unroll
-    for (int d = 0; d < D; ++d) o[d] = 0.f;
-    float m = -INFINITY, lsum = 0.f;
-
-    // Every wait below is bounded; its outcome is made CTA-uniform so that all
-    // threads leave the loop together.  `pending` records an MMA still in
-    // flight when a wait gave up (1: Q.K^T, 2: P.V).
-    bool ok = !__syncthreads_or(!mbar_wait(bar_q, 0));
-    int pending = 0;
-    int j = 0;
-    for (; ok && j < nkt; ++j) {
-        const int st = j & 1;
-        uint8_t* ks = smem + C::ST_OFF + st * C::STAGE;
-        uint8_t* vs = ks + C::KT_BYTES;
-        if (__syncthreads_or(!mbar_wait(&bar_kv[st], (j >> 1) & 1))) {
-            ok = false;
-            break;
-        }
-        // Keys at or past L inside the last live block hold no token: zero
-        // their V rows so that 0-weighted garbage cannot reach the output.
-        const int tile_k0 = j * C::BN;
-        const int dead_lo = max(L, tile_k0), dead_hi = min(nblk * B, tile_k0 + C::BN);
-        if (dead_lo < dead_hi) {
-            const int rows = dead_hi - dead_lo;
-            for (int i = tid; i < rows * C::NP * 8; i += kPrefillThreads) {
-                const int rr = (dead_lo - tile_k0) + i / (C::NP * 8);
-                const int rest = i % (C::NP * 8);
-                *reinterpret_cast<uint4*>(vs + (rest / 8) * C::BN * 128 + rr * 128 + (rest % 8) * 16) =
-                    make_uint4(0, 0, 0, 0);
-            }
-            fence_proxy_async();
-        }
-        tc_fence_before();
-        __syncthreads();
-        if (tid == 0) {
-            tc_fence_after();
-            const uint32_t k_addr = smem_u32(ks);
-#pragma unroll
-            for (int kk = 0; kk < D / 16; ++kk) {
-                const uint32_t off = (kk / 4) * (C::BM * 128) + (kk % 4) * 32;
-                const uint32_t koff = (kk / 4) * (C::BN * 128) + (kk % 4) * 32;
-                umma_f16_ss(t_s - lane_base, smem_desc_sw128(q_addr + off, 16, 1024),
-                            smem_desc_sw128(k_addr + koff, 16, 1024), IDESC_S, kk > 0);
-            }
-            umma_commit(bar_s);
-        }
-        if (__syncthreads_or(!mbar_wait(bar_s, j & 1))) {
-            ok = false;
-            pending = 1;
-            break;
-        }
-        tc_fence_after();
-
-        // ---- softmax on this thread's row of S (two passes over tensor memory)
-        float v[32];
-        float mloc = -INFINITY;
-#pragma unroll
-        for (int c = 0; c < C::BN / 32; ++c) {
-            tmem_ld32(t_s + c * 32, v);
-#pragma unroll
-            for (int i = 0; i < 32; ++i) {
-                const int key = tile_k0 + c * 32 + i;
-                const float sv = key <= qpos ? v[i] * p.scale_log2 : -INFINITY;
-                mloc = fmaxf(mloc, sv);
-            }
-        }
-        const float mnew = fmaxf(m, mloc);
-        const float alpha = exp2f(m - mnew);
-        float tsum = 0.f;
-#pragma unroll
-        for (int c = 0; c < C::BN / 32; ++c) {
-            tmem_ld32(t_s + c * 32, v);
-            uint32_t packed[16], packed_lo[16];
-#pragma unroll
-            for (int i = 0; i < 32; i += 2) {
-                const int key = tile_k0 + c * 32 + i;
-                const float p0 = key <= qpos ? exp2f(v[i] * p.scale_log2 - mnew) : 0.f;
-                const float p1 = key + 1 <= qpos ? exp2f(v[i + 1] * p.scale_log2 - mnew) : 0.f;
-                tsum += p0 + p1;
-                packed[i / 2] = Elem<T>::pack(p0, p1);
-                if constexpr (C::SPLIT_P) {
-                    const float2 hi = Elem<T>::pair(packed[i / 2]);
-                    packed_lo[i / 2] = Elem<T>::pack(p0 - hi.x, p1 - hi.y);
+                    for (int pn = 0; pn < C::NP; ++pn)
+                        tma_load_4d(dst + pn * C::BN * 128 + i * B * 128, map, pn * C::PANEL, g, 0, coord, &full[st]);
                 }
             }
-            // keys c*32 .. c*32+31 -> panel c/2, 16-byte chunks 4*(c%2) .. +3
+        };
+        auto poll = [&](uint64_t* bar, uint32_t parity) -> bool {  // lane 0 probes, the warp agrees
+            return __shfl_sync(0xffffffffu, leader ? (int)mbar_poll(bar, parity) : 0, 0) != 0;
+        };
+        if (leader) {
+            mbar_arrive_expect_tx(q_full, C::Q_BYTES);
 #pragma unroll
-            for (int q = 0; q < 4; ++q) {
-                const int cc = 4 * (c % 2) + q;
-                const int off = (c / 2) * (C::BM * 128) + row * 128 + ((cc ^ (row & 7)) << 4);
-                *reinterpret_cast<uint4*>(p_s + off) =
-                    make_uint4(packed[4 * q], packed[4 * q + 1], packed[4 * q + 2], packed[4 * q + 3]);
-                if constexpr (C::SPLIT_P)
-                    *reinterpret_cast<uint4*>(plo_s + off) = make_uint4(packed_lo[4 * q], packed_lo[4 * q + 1],
-                                                                        packed_lo[4 * q + 2], packed_lo[4 * q + 3]);
+            for (int pn = 0; pn < C::NP; ++pn)
+                tma_load_3d(smem + C::Q_OFF + pn * C::BM * 128, &tm_q, pn * C::PANEL, g * G, q0 + qt * C::TT, q_full);
+        }
+        int nk = 0, nv = 0;
+        int ids_k = fetch_ids(0), ids_v = ids_k;
+        for (; nk < min(nkt, 2); ++nk) {
+            load_tile(&tm_k, C::K_OFF, k_full, nk, ids_k);
+            load_tile(&tm_v, C::V_OFF, v_full, nk, ids_k);
+            ids_k = fetch_ids(nk + 1);
+        }
+        nv = nk;
+        ids_v = ids_k;
+        int ns = 0, npv = 0;
+        bool q_ready = false;
+        uint64_t t_last = global_timer_ns();
+        while (npv < nkt) {
+            bool progress = false;
+            if (__shfl_sync(0xffffffffu, leader ? *abort_flag : 0, 0)) break;
+            if (!q_ready) q_ready = poll(q_full, 0);
+            // S_ns = Q . K_ns^T into S buffer ns % 2 (free once the softmax read S_{ns-2})
+            if (q_ready && ns < nkt) {
+                const int st = ns & 1;
+                if (poll(&k_full[st], (ns >> 1) & 1) && (ns < 2 || poll(&s_free[st], ((ns - 2) >> 1) & 1))) {
+                    if (leader) {
+                        tc_fence_after();
+                        const uint32_t k_addr = smem_u32(smem + C::K_OFF + st * C::KT_BYTES);
+#pragma unroll
+                        for (int kk = 0; kk < D / 16; ++kk) {
+                            const uint32_t qoff = (kk / 4) * (C::BM * 128) + (kk % 4) * 32;
+                            const uint32_t koff = (kk / 4) * (C::BN * 128) + (kk % 4) * 32;
+                            umma_f16_ss(tmem + C::S_COL0 + st * 128, smem_desc_sw128(q_addr + qoff, 16, 1024),
+                                        smem_desc_sw128(k_addr + koff, 16, 1024), IDESC_S, kk > 0);
+                        }
+                        umma_commit(&s_full[st]);
+                    }
+                    __syncwarp();
+                    ++ns;
+                    progress = true;
+                }
+            }
+            // K of tile nk into stage nk % 2 once Q.K^T of tile nk - 2 is done
+            if (nk < nkt && nk - 2 < ns && poll(&s_full[nk & 1], ((nk - 2) >> 1) & 1)) {
+                load_tile(&tm_k, C::K_OFF, k_full, nk, ids_k);
+                ++nk;
+                ids_k = fetch_ids(nk);
+                progress = true;
+            }
+            // O_npv = P_npv . V_npv into O buffer npv % 2 (free once the softmax folded O_{npv-2})
+            if (npv < ns) {
+                const int st = npv & 1;
+                if (poll(p_full, npv & 1) && poll(&v_full[st], (npv >> 1) & 1) &&
+                    (npv < 2 || poll(&o_free[st], ((npv - 2) >> 1) & 1))) {
+                    if (leader) {
+                        tc_fence_after();
+                        const uint32_t v_addr = smem_u32(smem + C::V_OFF + st * C::KT_BYTES);
+#pragma unroll
+                        for (int kk = 0; kk < C::BN / 16; ++kk) {
+                            const uint32_t poff = (kk / 4) * (C::BM * 128) + (kk % 4) * 32;
+                            const uint64_t vdesc = smem_desc_sw128(v_addr + kk * 16 * 128, C::BN * 128, 1024);
+                            umma_f16_ss(tmem + C::O_COL0 + st * 128, smem_desc_sw128(p_addr + poff, 16, 1024), vdesc,
+                                        IDESC_O, kk > 0);
+                            if constexpr (C::SPLIT_P)
+                                umma_f16_ss(tmem + C::O_COL0 + st * 128, smem_desc_sw128(plo_addr + poff, 16, 1024),
+                                            vdesc, IDESC_O, 1);
+                        }
+                        umma_commit(&o_full[st]);
+                    }
+                    __syncwarp();
+                    ++npv;
+                    progress = true;
+                }
+            }
+            // V of tile nv into stage nv % 2 once P.V of tile nv - 2 is done
+            if (nv < nkt && nv - 2 < npv && poll(&o_full[nv & 1], ((nv - 2) >> 1) & 1)) {
+                load_tile(&tm_v, C::V_OFF, v_full, nv, ids_v);
+                ++nv;
+                ids_v = fetch_ids(nv);
+                progress = true;
+            }
+            if (progress) {
+                t_last = global_timer_ns();
+            } else {
+                __nanosleep(32);  // leave issue slots to the softmax warp sharing this scheduler
+                if (__shfl_sync(0xffffffffu, (int)(global_timer_ns() - t_last > kWaitLimitNs), 0)) {
+                    if (leader) {
+                        flag_error(PKV_DEVERR_TIMEOUT);
+                        *abort_flag = 1;
+                    }
+                    break;
+                }
             }
         }
-        lsum = lsum * alpha + tsum;
-        m = mnew;
-        fence_proxy_async();
-        tc_fence_before();
-        __syncthreads();
-        if (tid == 0) {
+        if (leader && *abort_flag) {
+            // Wait (bounded) for the last MMAs and copies this warp issued
+            // before tensor and shared memory are released.
+            if (ns > 0) mbar_wait(&s_full[(ns - 1) & 1], ((ns - 1) >> 1) & 1);
+            if (npv > 0) mbar_wait(&o_full[(npv - 1) & 1], ((npv - 1) >> 1) & 1);
+            for (int j = max(0, nk - 2); j < nk; ++j) mbar_wait(&k_full[j & 1], (j >> 1) & 1);
+            for (int j = max(0, nv - 2); j < nv; ++j) mbar_wait(&v_full[j & 1], (j >> 1) & 1);
+        }
+    } else {
+        // ================================================================ softmax rows
+        const int row = tid;
+        const int tok = qt * C::TT + row / G;
+        const int qpos = c0 + tok;  // absolute position of the row's query
+        const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
+        uint8_t* p_s = smem + C::P_OFF;
+        uint8_t* plo_s = smem + C::PLO_OFF;
+        const float sl2 = p.scale_log2;
+        float o[D];
+#pragma unroll
+        for (int d = 0; d < D; ++d) o[d] = 0.f;
+        float m = -INFINITY, lsum = 0.f, alpha_prev = 1.f;
+        bool ok = true;
+        float v[32];
+        for (int j = 0; j < nkt; ++j) {
+            const int st = j & 1;
+            if (!__all_sync(0xffffffffu, mbar_wait_or_abort(&s_full[st], (j >> 1) & 1, abort_flag))) {
+                ok = false;
+                break;
+            }
             tc_fence_after();
-            const uint32_t v_addr = smem_u32(vs);
+            const uint32_t ts = tmem + lane_base + C::S_COL0 + st * 128;
+            const int k0 = j * C::BN;
+            const bool all_vis = k0 + C::BN - 1 <= qpos;
+            const bool none_vis = k0 > qpos;
+            // ---- pass 1: row max of the visible scores (scale sign handled by max / min)
+            // (tcgen05.ld is warp-collective: every lane loads, masking is per row in registers)
+            float hi_raw = -INFINITY, lo_raw = INFINITY;
 #pragma unroll
-            for (int kk = 0; kk < C::BN / 16; ++kk) {
-                const uint32_t poff = (kk / 4) * (C::BM * 128) + (kk % 4) * 32;
-                const uint64_t vdesc = smem_desc_sw128(v_addr + kk * 16 * 128, C::BN * 128, 1024);
-                umma_f16_ss(t_o - lane_base, smem_desc_sw128(p_addr + poff, 16, 1024), vdesc, IDESC_O, kk > 0);
-                if constexpr (C::SPLIT_P)
-                    umma_f16_ss(t_o - lane_base, smem_desc_sw128(plo_addr + poff, 16, 1024), vdesc, IDESC_O, 1);
+            for (int c = 0; c < C::BN / 32; ++c) {
+                tmem_ld32(ts + c * 32, v);
+                if (all_vis) {
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) hi_raw = fmaxf(hi_raw, v[i]), lo_raw = fminf(lo_raw, v[i]);
+                } else if (!none_vis) {
+#pragma unroll
+                    for (int i = 0; i < 32; ++i)
+                        if (k0 + c * 32 + i <= qpos) hi_raw = fmaxf(hi_raw, v[i]), lo_raw = fminf(lo_raw, v[i]);
+                }
             }
-            umma_commit(bar_o);
-        }
-        if (__syncthreads_or(!mbar_wait(bar_o, j & 1))) {
-            ok = false;
-            pending = 2;
-            break;
-        }
-        tc_fence_after();
-        if (tid == 0 && j + 2 < nkt) issue_kv(j + 2);
+            const float mloc = none_vis ? -INFINITY : (sl2 >= 0.f ? hi_raw * sl2 : lo_raw * sl2);
+            const float mnew = fmaxf(m, mloc);
+            const float alpha = ex2_approx(m - mnew);
+            // ---- fold P.V of the previous tile into the accumulator
+            if (j >= 1) {
+                const int jp = j - 1;
+                if (!__all_sync(0xffffffffu, mbar_wait_or_abort(&o_full[jp & 1], (jp >> 1) & 1, abort_flag))) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                const uint32_t to = tmem + lane_base + C::O_COL0 + (jp & 1) * 128;
 #pragma unroll
-        for (int c = 0; c < D / 32; ++c) {
-            tmem_ld32(t_o + c * 32, v);
+                for (int c = 0; c < D / 32; ++c) {
+                    tmem_ld32(to + c * 32, v);
 #pragma unroll
-            for (int i = 0; i < 32; ++i) o[c * 32 + i] = fmaf(o[c * 32 + i], alpha, v[i]);
+                    for (int i = 0; i < 32; ++i) o[c * 32 + i] = fmaf(o[c * 32 + i], alpha_prev, v[i]);
+                }
+                tc_fence_before();
+                mbar_arrive(&o_free[jp & 1]);
+            }
+            // ---- the last tile may hold the dead tail of the sequence's last
+            // block: zero those V rows (0 * NaN must not reach the output)
+            if (j == nkt - 1) {
+                const int dead_lo = max(L, k0), dead_hi = min(nblk * B, k0 + C::BN);
+                if (dead_lo < dead_hi) {
+                    if (!__all_sync(0xffffffffu, mbar_wait_or_abort(&v_full[st], (j >> 1) & 1, abort_flag))) {
+                        ok = false;
+                        break;
+                    }
+                    uint8_t* vs = smem + C::V_OFF + st * C::KT_BYTES;
+                    const int rows = dead_hi - dead_lo;
+                    for (int i = tid; i < rows * C::NP * 8; i += kPrefillSoftmaxWarps * 32) {
+                        const int rr = (dead_lo - k0) + i / (C::NP * 8);
+                        const int rest = i % (C::NP * 8);
+                        *reinterpret_cast<uint4*>(vs + (rest / 8) * C::BN * 128 + rr * 128 + (rest % 8) * 16) =
+                            make_uint4(0, 0, 0, 0);
+                    }
+                }
+            }
+            // ---- pass 2: P = exp2(S * scale * log2 e - m), K-major swizzled rows
+            float tsum = 0.f;
+#pragma unroll
+            for (int c = 0; c < C::BN / 32; ++c) {
+                uint32_t hi[16], lo[16];
+                tmem_ld32(ts + c * 32, v);
+                if (none_vis) {
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) hi[i] = lo[i] = 0u;
+                } else {
+#pragma unroll
+                    for (int i = 0; i < 32; i += 2) {
+                        const int key = k0 + c * 32 + i;
+                        float p0 = ex2_approx(fmaf(v[i], sl2, -mnew));
+                        float p1 = ex2_approx(fmaf(v[i + 1], sl2, -mnew));
+                        if (!all_vis) {
+                            p0 = key <= qpos ? p0 : 0.f;
+                            p1 = key + 1 <= qpos ? p1 : 0.f;
+                        }
+                        tsum += p0 + p1;
+                        if constexpr (C::SPLIT_P) {
+                            // hi = p truncated to bf16 (its top 16 bits, one byte permute for the
+                            // pair); lo = the exact remainder rounded to bf16, |lo| < 2^-7 |p|
+                            const uint32_t b0 = __float_as_uint(p0), b1 = __float_as_uint(p1);
+                            hi[i / 2] = __byte_perm(b0, b1, 0x7632);
+                            lo[i / 2] = Elem<T>::pack(p0 - __uint_as_float(b0 & 0xFFFF0000u),
+                                                      p1 - __uint_as_float(b1 & 0xFFFF0000u));
+                        } else {
+                            hi[i / 2] = Elem<T>::pack(p0, p1);
+                        }
+                    }
+                }
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    const int cc = 4 * (c % 2) + q;
+                    const int off = (c / 2) * (C::BM * 128) + row * 128 + ((cc ^ (row & 7)) << 4);
+                    *reinterpret_cast<uint4*>(p_s + off) =
+                        make_uint4(hi[4 * q], hi[4 * q + 1], hi[4 * q + 2], hi[4 * q + 3]);
+                    if constexpr (C::SPLIT_P)
+                        *reinterpret_cast<uint4*>(plo_s + off) =
+                            make_uint4(lo[4 * q], lo[4 * q + 1], lo[4 * q + 2], lo[4 * q + 3]);
+                }
+            }
+            tc_fence_before();
+            mbar_arrive(&s_free[st]);
+            fence_proxy_async();
+            mbar_arrive(p_full);
+            lsum = lsum * alpha + tsum;
+            m = mnew;
+            alpha_prev = alpha;
         }
-    }
-
-    if (ok) {
-        if (tok < n) {
+        if (ok) {
+            const int jl = nkt - 1;
+            if (__all_sync(0xffffffffu, mbar_wait_or_abort(&o_full[jl & 1], (jl >> 1) & 1, abort_flag))) {
+                tc_fence_after();
+                const uint32_t to = tmem + lane_base + C::O_COL0 + (jl & 1) * 128;
+#pragma unroll
+                for (int c = 0; c < D / 32; ++c) {
+                    tmem_ld32(to + c * 32, v);
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) o[c * 32 + i] = fmaf(o[c * 32 + i], alpha_prev, v[i]);
+                }
+            } else {
+                ok = false;
+            }
+        }
+        if (ok && !*abort_flag && tok < n) {
             const float inv = 1.f / lsum;
             T* dst = reinterpret_cast<T*>(p.out) +
                      (static_cast<int64_t>(q0 + tok) * p.num_q_heads + static_cast<int64_t>(g) * G + row % G) * D;
@@ -317,12 +454,6 @@ __global__ void __launch_bounds__(kPrefillThreads, 1) paged_prefill_kernel(const
                 *reinterpret_cast<uint4*>(dst + d) = w;
             }
         }
-    } else if (tid == 0) {
-        // A wait gave up: wait (bounded) for whatever is still in flight
-        // before tensor memory and shared memory are released.
-        if (pending == 1) mbar_wait(bar_s, j & 1);
-        if (pending == 2) mbar_wait(bar_o, j & 1);
-        for (int jj = pending ? j + 1 : j; jj < min(nkt, j + 2); ++jj) mbar_wait(&bar_kv[jj & 1], (jj >> 1) & 1);
     }
     tc_fence_before();
     __syncthreads();
