@@ -7,7 +7,9 @@ sequences, 32 heads = 32 KV heads, head_dim 128, block 16, context U[128,
 2048], fp16).  One step = reshape_and_cache of the 64 new tokens, then
 paged decode attention (decode kernel + log-sum-exp merge) over all 64
 sequences, on inputs already resident in HBM (the pools, 1.25 GB each, are
-far larger than the 126 MB L2).  ``value`` = decode tokens (sequences) per
+far larger than the 126 MB L2).  The step's launches are captured once in a
+CUDA graph and replayed (``--no-graph`` launches them one by one); the
+decode-call duration for the roofline comes from a plain launch loop.  ``value`` = decode tokens (sequences) per
 second over all ranks; multi-GPU runs are independent replicas (weak
 scaling, no collective on the data path).
 
@@ -389,6 +391,49 @@ def run_reference(args, ws, rank):
     print(json.dumps(line), flush=True)
 
 
+def run_swap(args, ws, rank):
+    """Pre-emption swap: every block of the llama7b-shaped batch to page-locked
+    host memory and back (swap_blocks), GB/s per direction."""
+    import paged_kv_cache_409_b200 as pkv
+    from paged_kv_cache_409_b200 import workloads
+    w = workloads.llama7b_decode_f16(device="cuda", seed=1002 + rank)
+    B = w.block_size
+    nblk = ((w.context_lens.astype(np.int64) + B - 1) // B)
+    used = np.concatenate([w.block_tables[s, :nblk[s]] for s in range(w.num_seqs)]).astype(np.int64)
+    n = len(used)
+    kc, vc = w.key_caches[0], w.value_caches[0]
+    hk = torch.empty((n,) + tuple(kc.shape[1:]), dtype=kc.dtype).pin_memory()
+    hv = torch.empty_like(hk).pin_memory()
+    out_pairs = torch.from_numpy(np.stack([used, np.arange(n)], 1)).cuda()
+    in_pairs = torch.from_numpy(np.stack([np.arange(n), used], 1)).cuda()
+    nbytes = 2 * n * kc[0].numel() * kc.element_size()
+    for _ in range(args.warmup):
+        pkv.swap_blocks(kc, vc, hk, hv, out_pairs)
+        pkv.swap_blocks(hk, hv, kc, vc, in_pairs)
+    torch.cuda.synchronize()
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+    t_out = t_in = 0.0
+    for _ in range(args.steps):
+        ev[0].record()
+        pkv.swap_blocks(kc, vc, hk, hv, out_pairs)
+        ev[1].record()
+        pkv.swap_blocks(hk, hv, kc, vc, in_pairs)
+        ev[2].record()
+        torch.cuda.synchronize()
+        t_out += ev[0].elapsed_time(ev[1])
+        t_in += ev[1].elapsed_time(ev[2])
+    assert pkv.get_device_error() == 0
+    line = {"metric": "swap_blocks GB/s (device pool <-> page-locked host pool)", "value":
+            nbytes / (t_out / args.steps / 1e3) / 1e9, "unit": "GB/s", "n_gpus": ws, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": (t_out + t_in) / args.steps, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f16", "data": "synthetic",
+            "config": {"workload": "llama7b_decode_f16: all blocks in use", "blocks": int(n), "bytes": int(nbytes)},
+            "swap_out_gbs": nbytes / (t_out / args.steps / 1e3) / 1e9,
+            "swap_in_gbs": nbytes / (t_in / args.steps / 1e3) / 1e9, "gpu_launches": 2 * args.steps}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -400,6 +445,8 @@ def main():
     ap.add_argument("--seqs", type=int, default=None,
                     help="fewer sequences of the named workload (small profiling cases)")
     ap.add_argument("--layers", type=int, default=None, help="cap on distinct layer pools (gqa70b_decode_bf16)")
+    ap.add_argument("--no-graph", dest="graph", action="store_false",
+                    help="launch every kernel of every step instead of replaying one captured CUDA graph")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
 
@@ -413,6 +460,9 @@ def main():
 
     import paged_kv_cache_409_b200 as pkv
     pkv.load_library()
+    if args.config == "swap_llama7b_f16":
+        run_swap(args, ws, rank)
+        return
     dev = torch.device("cuda", torch.cuda.current_device())
     step, cname = make_step(args.config, dev, rank, args.seqs, args.layers)
     torch.cuda.synchronize()
@@ -425,12 +475,28 @@ def main():
     torch.cuda.synchronize()
     barrier(ws)
     timer = EventTimer()
+    graph = None
+    if args.graph:
+        # one whole step (every layer) per graph; layers cycle within it
+        side = torch.cuda.Stream()
+        side.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(side):
+            step.run(step=0)
+        torch.cuda.current_stream().wait_stream(side)
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph):
+            step.run(step=0)
+        graph.replay()
+        torch.cuda.synchronize()
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     h0 = time.perf_counter()
     torch.cuda.nvtx.range_push("timed")
     t0.record()
     for i in range(args.steps):
-        step.run(timer=timer, step=i)
+        if graph is not None:
+            graph.replay()
+        else:
+            step.run(timer=timer, step=i)
     t1.record()
     torch.cuda.nvtx.range_pop()
     torch.cuda.synchronize()
@@ -439,6 +505,12 @@ def main():
     barrier(ws)
     ms_total = max_over_ranks(t0.elapsed_time(t1), ws)
     ms_step = ms_total / args.steps
+    if graph is not None:
+        # the decode-call duration for the roofline, from a short plain loop
+        for i in range(min(args.steps, 50)):
+            step.run(timer=timer, step=i)
+        torch.cuda.synchronize()
+        del graph
     unit_ms = max_over_ranks(timer.mean_ms(), ws)
     assert pkv.get_device_error() == 0, "device error word set during the run"
 
@@ -471,7 +543,7 @@ def main():
         "data": "synthetic",
         "config": {"workload": cname, "num_seqs": w.num_seqs, "num_q_heads": w.num_q_heads,
                    "num_kv_heads": w.num_kv_heads, "head_dim": w.head_dim, "block_size": w.block_size,
-                   "layers_per_step": step.layers, "partition_size": step.part,
+                   "layers_per_step": step.layers, "partition_size": step.part, "cuda_graph": bool(args.graph),
                    "l2": "inputs larger than L2 (K/V pools %.2f GB per layer)" % (
                        2 * w.key_caches[0].numel() * w.key_caches[0].element_size() / 1e9),
                    "parallelism": f"replicas x{ws}"},

@@ -113,6 +113,27 @@ int pkv_copy_blocks(void* const* key_caches, void* const* value_caches, int num_
                     int64_t num_blocks, pkv_stream_t stream);
 
 /*
+ * swap_blocks -- move whole blocks between two pools, e.g. from the device pool
+ * to a pool in page-locked host memory and back.  Source: case-study page
+ * section 三 (under memory pressure the scheduler pre-empts a request by
+ * swapping its KV out to CPU memory and brings it back later) and the tutorial
+ * page, 4.3 (pre-emption and resumption).
+ *
+ *   src_key_pool, src_value_pool   [src_num_blocks, block_size, Hkv, D]
+ *   dst_key_pool, dst_value_pool   [dst_num_blocks, block_size, Hkv, D]
+ *                  each device, managed or page-locked host memory (reached
+ *                  through unified addressing); pageable host memory -> PKV_EINVAL
+ *   src_dst_pairs  int64 [num_pairs, 2] (src block, dst block), device or
+ *                  page-locked host memory
+ * Bit copies, one kernel launch for all pairs, K and V.  An id outside its pool
+ * is skipped and sets PKV_DEVERR_PAIR.  Destinations must be distinct.
+ */
+int pkv_swap_blocks(const void* src_key_pool, const void* src_value_pool, void* dst_key_pool,
+                    void* dst_value_pool, const int64_t* src_dst_pairs, int64_t num_pairs,
+                    int64_t block_bytes, int64_t src_num_blocks, int64_t dst_num_blocks,
+                    pkv_stream_t stream);
+
+/*
  * Decode attention over the paged cache, one query token per sequence.
  * Source: case-study page section 二 "注意力计算改造" (K/V are loaded block by
  * block through the block table and each block's attention is accumulated;

@@ -1,0 +1,137 @@
+"""Plain model of the host block manager's policy (test infrastructure).
+
+It restates, with Python lists and dicts, the policy written in
+``include/pagedkv_block_manager.h``: a free stack with block 0 on top, blocks
+taken on demand, reference counts, copy-on-write of a shared partial last
+block, and a prefix cache of full blocks keyed by their exact content chain
+(parent block's key, token ids) -- no hashing -- whose unreferenced blocks sit
+in an LRU list, oldest evicted first.  The data model it follows is that of the
+vLLM case-study page ("vLLM 与 PagedAttention", sections 二 and 四) and the
+298.name page's ``PagedKVCache`` sketch.  The tests compare the C++ manager to
+this model operation by operation.
+"""
+from __future__ import annotations
+
+
+class NoSpace(Exception):
+    pass
+
+
+class BlockManagerModel:
+    def __init__(self, num_blocks, block_size, prefix_caching=True):
+        self.B = block_size
+        self.prefix_caching = prefix_caching
+        self.free_stack = list(range(num_blocks - 1, -1, -1))  # block 0 on top (end of the list)
+        self.ref = [0] * num_blocks
+        self.key_of = [None] * num_blocks
+        self.cache = {}
+        self.lru = []  # oldest first
+        self.seqs = {}
+        self.hits = self.evictions = self.cows = 0
+
+    # -- blocks
+    def _take(self):
+        if self.free_stack:
+            b = self.free_stack.pop()
+        elif self.lru:
+            b = self.lru.pop(0)
+            del self.cache[self.key_of[b]]
+            self.key_of[b] = None
+            self.evictions += 1
+        else:
+            raise NoSpace()
+        self.ref[b] = 1
+        return b
+
+    def _release(self, b):
+        self.ref[b] -= 1
+        if self.ref[b] == 0:
+            (self.lru if self.key_of[b] is not None else self.free_stack).append(b)
+
+    def _register_full(self, seq, b, toks):
+        key = (seq["last_key"], tuple(toks))
+        if self.prefix_caching and self.key_of[b] is None and key not in self.cache:
+            self.cache[key] = b
+            self.key_of[b] = key
+        seq["last_key"] = key
+
+    def _available(self):
+        return len(self.free_stack) + len(self.lru)
+
+    # -- operations
+    def add_sequence(self, sid, tokens):
+        tokens = list(tokens)
+        assert sid not in self.seqs
+        B = self.B
+        full, need = len(tokens) // B, -(-len(tokens) // B)
+        hits, parent = [], None
+        if self.prefix_caching:
+            for i in range(full):
+                key = (parent, tuple(tokens[i * B:(i + 1) * B]))
+                if key not in self.cache:
+                    break
+                hits.append(self.cache[key])
+                parent = key
+        if need - len(hits) > self._available() - sum(1 for b in hits if b in self.lru):
+            raise NoSpace()
+        seq = {"blocks": [], "last_key": parent, "tail": [], "n": len(tokens)}
+        for b in hits:
+            if self.ref[b] == 0 and b in self.lru:
+                self.lru.remove(b)
+            self.ref[b] += 1
+            seq["blocks"].append(b)
+        self.hits += len(hits)
+        for i in range(len(hits), need):
+            b = self._take()
+            seq["blocks"].append(b)
+            if i < full:
+                self._register_full(seq, b, tokens[i * B:(i + 1) * B])
+        seq["tail"] = tokens[full * B:]
+        self.seqs[sid] = seq
+        return len(hits) * B
+
+    def append(self, sid, tokens):
+        seq, B = self.seqs[sid], self.B
+        tokens = list(tokens)
+        off0 = seq["n"] % B
+        cow = bool(tokens) and off0 != 0 and self.ref[seq["blocks"][-1]] > 1
+        new_blocks = -(-(off0 + len(tokens)) // B) - (1 if off0 else 0)
+        if new_blocks + (1 if cow else 0) > self._available():
+            raise NoSpace()
+        pairs = []
+        if cow:
+            src = seq["blocks"][-1]
+            dst = self._take()
+            self._release(src)
+            seq["blocks"][-1] = dst
+            pairs.append((src, dst))
+            self.cows += 1
+        slots = []
+        for t in tokens:
+            if seq["n"] % B == 0:
+                seq["blocks"].append(self._take())
+            slots.append(seq["blocks"][-1] * B + seq["n"] % B)
+            seq["tail"].append(t)
+            seq["n"] += 1
+            if seq["n"] % B == 0:
+                self._register_full(seq, seq["blocks"][-1], seq["tail"])
+                seq["tail"] = []
+        return slots, pairs
+
+    def fork(self, parent, child):
+        p = self.seqs[parent]
+        self.seqs[child] = {"blocks": list(p["blocks"]), "last_key": p["last_key"], "tail": list(p["tail"]),
+                            "n": p["n"]}
+        for b in p["blocks"]:
+            self.ref[b] += 1
+
+    def free(self, sid):
+        for b in reversed(self.seqs.pop(sid)["blocks"]):
+            self._release(b)
+
+    def block_table(self, sid):
+        return list(self.seqs[sid]["blocks"])
+
+    def stats(self):
+        return {"free": len(self.free_stack), "evictable": len(self.lru), "cached": len(self.cache),
+                "hits": self.hits, "evictions": self.evictions, "cow_copies": self.cows, "sequences": len(self.seqs)}

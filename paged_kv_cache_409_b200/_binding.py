@@ -30,6 +30,7 @@ EXPORTED = (
     "pkv_last_cuda_error",
     "pkv_reshape_and_cache",
     "pkv_copy_blocks",
+    "pkv_swap_blocks",
     "pkv_paged_attention_decode",
     "pkv_decode_workspace_size",
     "pkv_decode_partition_size",
@@ -66,13 +67,14 @@ def load_library():
     lib.pkv_last_cuda_error.restype = ctypes.c_char_p
     lib.pkv_reshape_and_cache.argtypes = [P, P, P, P, P, I64, I, I, I, I64, I, P]
     lib.pkv_copy_blocks.argtypes = [P, P, I, P, I64, I64, I64, P]
+    lib.pkv_swap_blocks.argtypes = [P, P, P, P, P, I64, I64, I64, I64, P]
     lib.pkv_paged_attention_decode.argtypes = [P, P, P, P, P, P, F, I, I, I, I, I, I, I64, I, I, I, P, SZ, P]
     lib.pkv_decode_workspace_size.argtypes = [I, I, I, I, I]
     lib.pkv_decode_workspace_size.restype = SZ
     lib.pkv_decode_partition_size.argtypes = [I, I, I, I, I, I64, I]
     lib.pkv_paged_attention_prefill_chunk.argtypes = [P, P, P, P, P, P, P, I, I64, I, F, I, I, I, I, I, I64, I, P]
     lib.pkv_get_device_error.argtypes = [ctypes.POINTER(ctypes.c_uint32), P]
-    for name in ("pkv_reshape_and_cache", "pkv_copy_blocks", "pkv_paged_attention_decode",
+    for name in ("pkv_reshape_and_cache", "pkv_copy_blocks", "pkv_swap_blocks", "pkv_paged_attention_decode",
                  "pkv_decode_partition_size", "pkv_paged_attention_prefill_chunk", "pkv_get_device_error"):
         getattr(lib, name).restype = I
     _lib = lib
@@ -138,6 +140,26 @@ def copy_blocks(key_caches, value_caches, src_dst_pairs, stream=None):
     rc = lib.pkv_copy_blocks(kp, vp, L, _dev(src_dst_pairs, "src_dst_pairs") if npairs else None, npairs,
                              block_bytes, NB, _stream(stream))
     _ok(rc, "copy_blocks")
+
+
+def swap_blocks(src_key, src_value, dst_key, dst_value, src_dst_pairs, stream=None):
+    """Move blocks ``src -> dst`` between two pools (device and/or pinned host tensors)."""
+    lib = load_library()
+    for t, name in ((src_key, "src_key"), (src_value, "src_value"), (dst_key, "dst_key"), (dst_value, "dst_value"),
+                    (src_dst_pairs, "src_dst_pairs")):
+        if not t.is_contiguous():
+            raise ValueError(f"{name} must be contiguous")
+        if not (t.is_cuda or t.is_pinned()):
+            raise ValueError(f"{name} must be a CUDA tensor or pinned host memory")
+    if src_dst_pairs.dtype != torch.int64:
+        raise ValueError("src_dst_pairs must be int64")
+    block_bytes = src_key[0].numel() * src_key.element_size()
+    if dst_key[0].numel() * dst_key.element_size() != block_bytes:
+        raise ValueError("pools differ in block size")
+    rc = lib.pkv_swap_blocks(src_key.data_ptr(), src_value.data_ptr(), dst_key.data_ptr(), dst_value.data_ptr(),
+                             src_dst_pairs.data_ptr(), src_dst_pairs.numel() // 2, block_bytes, src_key.shape[0],
+                             dst_key.shape[0], _stream(stream))
+    _ok(rc, "swap_blocks")
 
 
 def decode_workspace_size(num_seqs, num_q_heads, head_dim, max_context_len, partition_size) -> int:

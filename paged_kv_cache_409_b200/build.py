@@ -13,8 +13,8 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libpagedkv.so")
-SOURCES = ["pagedkv.cu"]
-DEPENDS = ["pagedkv.cu", "ptx.cuh", "index_kernels.cuh", "decode.cuh", "decode_mma.cuh", "prefill.cuh"]
+SOURCES = ["pagedkv.cu", "block_manager.cpp"]
+DEPENDS = ["pagedkv.cu", "block_manager.cpp", "ptx.cuh", "index_kernels.cuh", "decode.cuh", "decode_mma.cuh", "prefill.cuh"]
 
 
 def nvcc() -> str:
@@ -34,7 +34,7 @@ def stale() -> bool:
     if not os.path.exists(LIB):
         return True
     t = os.path.getmtime(LIB)
-    deps = [os.path.join(CSRC, d) for d in DEPENDS] + [os.path.join(INCLUDE, "pagedkv.h")]
+    deps = [os.path.join(CSRC, d) for d in DEPENDS] + [os.path.join(INCLUDE, h) for h in ("pagedkv.h", "pagedkv_block_manager.h")]
     return any(os.path.getmtime(d) > t for d in deps)
 
 

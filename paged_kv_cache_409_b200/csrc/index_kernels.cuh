@@ -82,4 +82,39 @@ __global__ void __launch_bounds__(kCopyThreads) copy_blocks_kernel(const LayerPo
     }
 }
 
+// Block moves between two pools (device HBM and/or page-locked host memory,
+// reached through unified addressing): grid.x chunks of a block, grid.y pairs
+// (grid-stride), grid.z 0 = K, 1 = V.
+__global__ void __launch_bounds__(kCopyThreads) swap_blocks_kernel(const uint4* __restrict__ src_k,
+                                                                   const uint4* __restrict__ src_v,
+                                                                   uint4* __restrict__ dst_k, uint4* __restrict__ dst_v,
+                                                                   const int64_t* __restrict__ pairs, int64_t num_pairs,
+                                                                   int64_t block_vecs, int64_t src_blocks,
+                                                                   int64_t dst_blocks) {
+    const uint4* sbase = blockIdx.z ? src_v : src_k;
+    uint4* dbase = blockIdx.z ? dst_v : dst_k;
+    const int64_t first = static_cast<int64_t>(blockIdx.x) * kCopyThreads * kCopyUnroll + threadIdx.x;
+    for (int64_t p = blockIdx.y; p < num_pairs; p += gridDim.y) {
+        const int64_t src = pairs[2 * p];
+        const int64_t dst = pairs[2 * p + 1];
+        if (src < 0 || src >= src_blocks || dst < 0 || dst >= dst_blocks) {
+            if (threadIdx.x == 0 && blockIdx.x == 0 && blockIdx.z == 0) flag_error(PKV_DEVERR_PAIR);
+            continue;
+        }
+        const uint4* s = sbase + src * block_vecs;
+        uint4* d = dbase + dst * block_vecs;
+        uint4 r[kCopyUnroll];
+#pragma unroll
+        for (int u = 0; u < kCopyUnroll; ++u) {
+            const int64_t i = first + u * kCopyThreads;
+            if (i < block_vecs) r[u] = s[i];
+        }
+#pragma unroll
+        for (int u = 0; u < kCopyUnroll; ++u) {
+            const int64_t i = first + u * kCopyThreads;
+            if (i < block_vecs) d[i] = r[u];
+        }
+    }
+}
+
 }  // namespace pkv

@@ -396,6 +396,36 @@ int pkv_copy_blocks(void* const* key_caches, void* const* value_caches, int num_
     return PKV_OK;
 }
 
+int pkv_swap_blocks(const void* src_key_pool, const void* src_value_pool, void* dst_key_pool, void* dst_value_pool,
+                    const int64_t* src_dst_pairs, int64_t num_pairs, int64_t block_bytes, int64_t src_num_blocks,
+                    int64_t dst_num_blocks, pkv_stream_t stream) {
+    if (num_pairs < 0 || block_bytes <= 0 || src_num_blocks <= 0 || dst_num_blocks <= 0) return PKV_EINVAL;
+    if (block_bytes % 16 != 0) return PKV_EUNSUPPORTED;
+    if (num_pairs == 0) return PKV_OK;
+    const void* ptrs[5] = {src_key_pool, src_value_pool, dst_key_pool, dst_value_pool, src_dst_pairs};
+    for (const void* q : ptrs) {
+        if (!q || (q != src_dst_pairs && !aligned16(q))) return PKV_EINVAL;
+        // every buffer must be reachable by the GPU: device, managed or page-locked host memory
+        cudaPointerAttributes a;
+        if (cudaPointerGetAttributes(&a, q) != cudaSuccess) {
+            cudaGetLastError();
+            return PKV_EINVAL;
+        }
+        if (a.type == cudaMemoryTypeUnregistered) return PKV_EINVAL;
+    }
+    if (reinterpret_cast<uintptr_t>(src_dst_pairs) & 7) return PKV_EINVAL;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const int64_t block_vecs = block_bytes / 16;
+    const int64_t per_cta = (int64_t)pkv::kCopyThreads * pkv::kCopyUnroll;
+    dim3 grid((unsigned)ceil_div(block_vecs, per_cta), (unsigned)std::min<int64_t>(num_pairs, 65535), 2);
+    pkv::swap_blocks_kernel<<<grid, pkv::kCopyThreads, 0, s>>>(
+        static_cast<const uint4*>(src_key_pool), static_cast<const uint4*>(src_value_pool),
+        static_cast<uint4*>(dst_key_pool), static_cast<uint4*>(dst_value_pool), src_dst_pairs, num_pairs, block_vecs,
+        src_num_blocks, dst_num_blocks);
+    PKV_CUDA(cudaGetLastError());
+    return PKV_OK;
+}
+
 size_t pkv_decode_workspace_size(int num_seqs, int num_q_heads, int head_dim, int max_context_len,
                                  int partition_size) {
     if (num_seqs <= 0 || num_q_heads <= 0 || head_dim <= 0 || partition_size <= 0 || max_context_len <= 0)

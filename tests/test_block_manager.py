@@ -1,0 +1,207 @@
+"""Host block manager (C++, in libpagedkv.so) against the pages' statements and
+against a plain model of the same policy, operation by operation (no GPU)."""
+import numpy as np
+import pytest
+
+from oracle.block_manager_model import BlockManagerModel, NoSpace
+from oracle_pins import golden
+from paged_kv_cache_409_b200.block_manager import BlockManager, NoSpaceError
+
+
+@pytest.fixture(autouse=True)
+def _built():
+    from paged_kv_cache_409_b200 import build
+    build.build()
+
+
+def test_on_demand_allocation_matches_pages_examples():
+    g = golden()
+    for e in g["blocks_needed"]:
+        bm = BlockManager(64, e["block_size"], prefix_caching=False)
+        bm.add_sequence(1, np.arange(e["tokens"]))
+        assert len(bm.block_table(1)) == e["blocks"], e["source"]
+    # generation one token at a time: the 7th block is only taken once the
+    # sequence passes 96 tokens; at the 100th token 7 blocks are held
+    bm = BlockManager(64, 16, prefix_caching=False)
+    bm.add_sequence(1, [])
+    held = []
+    for t in range(100):
+        bm.append(1, [t])
+        held.append(len(bm.block_table(1)))
+    assert held[95] == 6 and held[96] == 7 and held[99] == 7
+
+
+def test_fragmentation_below_one_block():
+    rng = np.random.default_rng(3)
+    bm = BlockManager(4096, 16)
+    for s in range(50):
+        n = int(rng.integers(0, 400))
+        bm.add_sequence(s, rng.integers(0, 1000, n))
+        assert len(bm.block_table(s)) * 16 - n < 16
+
+
+def test_slots_follow_the_block_table():
+    bm = BlockManager(100, 16)
+    bm.add_sequence(7, np.arange(40))
+    bt = bm.block_table(7)
+    slots = bm.slots(7, 0, 40)
+    assert slots.tolist() == [bt[p // 16] * 16 + p % 16 for p in range(40)]
+    s, pairs = bm.append(7, [1, 2, 3])
+    assert s.tolist() == [bt[2] * 16 + 8, bt[2] * 16 + 9, bt[2] * 16 + 10] and len(pairs) == 0
+
+
+def test_prefix_caching_reuses_the_system_prompt():
+    """Case-study page, section 四: a 1500-token system prompt prefilled once is
+    reused by later requests, which prefill only their own query."""
+    rng = np.random.default_rng(4)
+    system = rng.integers(0, 32000, 1500)
+    bm = BlockManager(1000, 16)
+    assert bm.add_sequence(1, np.concatenate([system, rng.integers(0, 32000, 8)])) == 0
+    cached = bm.add_sequence(2, np.concatenate([system, rng.integers(0, 32000, 8)]))
+    assert cached == 93 * 16                     # every full block of the shared prefix
+    assert cached / 1508 >= 0.80                 # the page's "80-95% of prefill saved" at least
+    assert bm.block_table(1)[:93].tolist() == bm.block_table(2)[:93].tolist()
+    assert bm.block_table(1)[93] != bm.block_table(2)[93]   # the partial block is private
+    assert bm.stats()["hits"] == 93
+
+
+def test_cached_blocks_survive_free_and_evict_lru_first():
+    bm = BlockManager(8, 4)
+    bm.add_sequence(1, [1, 2, 3, 4, 5, 6, 7, 8])        # two full blocks: 0, 1 (cached)
+    bm.free(1)
+    st = bm.stats()
+    assert st["free"] == 6 and st["evictable"] == 2 and st["cached"] == 2
+    assert bm.add_sequence(2, [1, 2, 3, 4, 9]) == 4      # first block hits the cache
+    assert bm.block_table(2)[0] == 0
+    bm.free(2)
+    bm.add_sequence(3, list(range(100, 128)))            # 7 blocks: all free ones, then an eviction
+    assert bm.stats()["evictions"] >= 1
+
+
+def test_fork_then_append_copies_the_shared_partial_block():
+    bm = BlockManager(32, 16)
+    bm.add_sequence(1, np.arange(20))                    # blocks: 1 full + 1 partial
+    bm.fork(1, 2)
+    last = bm.block_table(1)[1]
+    assert bm.ref_count(last) == 2
+    slots, pairs = bm.append(2, [99])
+    assert len(pairs) == 1 and pairs[0, 0] == last
+    new = bm.block_table(2)[1]
+    assert pairs[0, 1] == new and new != last
+    assert slots[0] == new * 16 + 4
+    assert bm.ref_count(last) == 1 and bm.block_table(1)[1] == last
+    assert bm.block_table(2)[0] == bm.block_table(1)[0]  # the full block stays shared
+
+
+def test_out_of_space_changes_nothing():
+    bm = BlockManager(4, 4)
+    bm.add_sequence(1, range(12))
+    before = (bm.stats(), bm.block_table(1).tolist())
+    with pytest.raises(NoSpaceError):
+        bm.add_sequence(2, range(100, 108))
+    with pytest.raises(NoSpaceError):
+        bm.append(1, range(5))
+    assert (bm.stats(), bm.block_table(1).tolist()) == before
+
+
+def _run_both(ops, num_blocks, B, caching):
+    cpp, model = BlockManager(num_blocks, B, caching), BlockManagerModel(num_blocks, B, caching)
+    for op in ops:
+        kind = op[0]
+        try:
+            if kind == "add":
+                a = cpp.add_sequence(op[1], op[2])
+            elif kind == "append":
+                s, p = cpp.append(op[1], op[2])
+                a = (s.tolist(), [tuple(x) for x in p.tolist()])
+            elif kind == "fork":
+                a = cpp.fork(op[1], op[2])
+            else:
+                a = cpp.free(op[1])
+        except NoSpaceError:
+            a = "nospace"
+        try:
+            if kind == "add":
+                b = model.add_sequence(op[1], op[2])
+            elif kind == "append":
+                b = model.append(op[1], op[2])
+            elif kind == "fork":
+                b = model.fork(op[1], op[2])
+            else:
+                b = model.free(op[1])
+        except NoSpace:
+            b = "nospace"
+        assert a == b, (op, a, b)
+        assert cpp.stats() == model.stats(), op
+        for sid in model.seqs:
+            assert cpp.block_table(sid).tolist() == model.block_table(sid), (op, sid)
+            assert cpp.num_tokens(sid) == model.seqs[sid]["n"]
+
+
+@pytest.mark.parametrize("seed", range(6))
+@pytest.mark.parametrize("caching", [True, False])
+def test_matches_plain_model_on_random_operations(seed, caching):
+    rng = np.random.default_rng(100 + seed)
+    B = int(rng.choice([4, 8, 16]))
+    prefixes = [rng.integers(0, 50, int(rng.integers(0, 6 * B))).tolist() for _ in range(3)]
+    live, next_id, ops = [], 0, []
+    for _ in range(400):
+        r = rng.random()
+        if r < 0.3 or not live:
+            toks = prefixes[int(rng.integers(0, 3))] + rng.integers(0, 50, int(rng.integers(0, 3 * B))).tolist()
+            ops.append(("add", next_id, toks))
+            live.append(next_id)
+            next_id += 1
+        elif r < 0.7:
+            ops.append(("append", live[int(rng.integers(0, len(live)))],
+                        rng.integers(0, 50, int(rng.integers(1, 2 * B))).tolist()))
+        elif r < 0.8:
+            ops.append(("fork", live[int(rng.integers(0, len(live)))], next_id))
+            live.append(next_id)
+            next_id += 1
+        else:
+            sid = live.pop(int(rng.integers(0, len(live))))
+            ops.append(("free", sid))
+    # replay against both, dropping ops on sequences a failed add never created
+    cpp_live = set()
+    filtered = []
+    model = BlockManagerModel(40, B, caching)
+    for op in ops:
+        if op[0] in ("append", "free", "fork") and op[1] not in cpp_live:
+            continue
+        filtered.append(op)
+        try:
+            if op[0] == "add":
+                model.add_sequence(op[1], op[2])
+                cpp_live.add(op[1])
+            elif op[0] == "append":
+                model.append(op[1], op[2])
+            elif op[0] == "fork":
+                model.fork(op[1], op[2])
+                cpp_live.add(op[2])
+            else:
+                model.free(op[1])
+                cpp_live.discard(op[1])
+        except NoSpace:
+            pass
+    _run_both(filtered, 40, B, caching)
+
+
+def test_append_batch_equals_one_by_one():
+    rng = np.random.default_rng(9)
+    a, b = BlockManager(200, 8), BlockManager(200, 8)
+    for bm in (a, b):
+        for s in range(6):
+            bm.add_sequence(s, np.arange(5 * s + 3))
+        bm.fork(2, 10)
+    ids = np.array([0, 1, 2, 3, 4, 5, 10])
+    for step in range(12):
+        toks = rng.integers(0, 99, ids.size)
+        sb, pb = b.append_batch(ids, toks)
+        sa, pa = [], []
+        for sid, t in zip(ids, toks):
+            s1, p1 = a.append(sid, [t])
+            sa += s1.tolist()
+            pa += [tuple(x) for x in p1.tolist()]
+        assert sb.tolist() == sa and [tuple(x) for x in pb.tolist()] == pa
+    assert a.stats() == b.stats()

@@ -1,0 +1,87 @@
+"""Decode steps driven by the host block manager on the GPU, checked against the oracle.
+
+Requests share a system prompt through the prefix cache (the second request
+prefills only its own tokens and attends to K/V the first one wrote), one
+request is forked mid-generation (its first append copies the shared partial
+block), and every step the manager's slots, copy-on-write pairs and tables
+drive reshape_and_cache, copy_blocks and paged_attention_decode.  A host
+mirror of the pools runs the same operations through the oracle.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import paged_kv_cache_409_b200 as pkv
+from paged_kv_cache_409_b200.block_manager import BlockManager
+from parity_helpers import assert_close
+
+pytestmark = pytest.mark.gpu
+
+B, Hq, Hkv, D, NB, VOCAB = 16, 8, 2, 128, 256, 512
+DT = torch.float16
+
+
+def kv_of(tokens, positions, table):
+    """K or V rows of tokens at positions: a fixed per-token vector, scaled by position."""
+    t = torch.as_tensor(np.asarray(tokens), dtype=torch.long)
+    p = torch.as_tensor(np.asarray(positions), dtype=torch.float32)
+    return (table[t] * (1.0 + 0.05 * (p % 11)).view(-1, 1, 1)).to(DT)
+
+
+def test_block_manager_drives_decode_steps():
+    rng = np.random.default_rng(21)
+    g = torch.Generator().manual_seed(21)
+    ek = torch.randn(VOCAB, Hkv, D, generator=g)
+    ev = torch.randn(VOCAB, Hkv, D, generator=g)
+    bm = BlockManager(NB, B, prefix_caching=True)
+    kc = torch.zeros(NB, B, Hkv, D, dtype=DT, device="cuda")
+    vc = torch.zeros_like(kc)
+    kn = np.zeros((NB, B, Hkv, D), dtype=np.float16)  # host mirror for the oracle
+    vn = np.zeros_like(kn)
+    orc = oracle.get()
+    tokens = {}
+
+    def write(sid, start, toks, slots):
+        pos = np.arange(start, start + len(toks))
+        k, v = kv_of(toks, pos, ek), kv_of(toks, pos, ev)
+        sl = torch.from_numpy(np.asarray(slots, dtype=np.int64))
+        pkv.reshape_and_cache(k.cuda(), v.cuda(), kc, vc, sl.cuda())
+        orc.reshape_and_cache(k.numpy(), v.numpy(), kn, vn, sl.numpy(), oracle.F16)
+
+    system = rng.integers(0, VOCAB, 40).tolist()
+    prompts = {0: system + rng.integers(0, VOCAB, 5).tolist(), 1: system + rng.integers(0, VOCAB, 7).tolist(),
+               2: rng.integers(0, VOCAB, 23).tolist()}
+    for sid, pr in prompts.items():
+        cached = bm.add_sequence(sid, pr)
+        assert cached == (32 if sid == 1 else 0)   # two full blocks of the system prompt
+        write(sid, cached, pr[cached:], bm.slots(sid, cached, len(pr) - cached))
+        tokens[sid] = list(pr)
+    live = [0, 1, 2]
+    cows = 0
+    for step in range(20):
+        if step == 5:
+            bm.fork(0, 3)
+            tokens[3] = list(tokens[0])
+            live.append(3)
+        new = rng.integers(0, VOCAB, len(live))
+        slots, pairs = bm.append_batch(live, new)
+        if len(pairs):
+            cows += len(pairs)
+            pkv.copy_blocks([kc], [vc], torch.from_numpy(pairs).cuda())
+            orc.copy_blocks([kn], [vn], pairs)
+        for i, sid in enumerate(live):
+            write(sid, len(tokens[sid]), [int(new[i])], [slots[i]])
+            tokens[sid].append(int(new[i]))
+        lens = np.array([bm.num_tokens(s) for s in live], dtype=np.int32)
+        mb = int(-(-lens.max() // B))
+        bt = bm.tables(live, mb)
+        q = torch.randn(len(live), Hq, D, generator=g).to(DT)
+        out = torch.empty(len(live), Hq, D, dtype=DT, device="cuda")
+        pkv.paged_attention_decode(out, q.cuda(), kc, vc, torch.from_numpy(bt).cuda(), torch.from_numpy(lens).cuda(),
+                                   D ** -0.5, int(lens.max()))
+        ref = orc.paged_attention_decode(q.numpy(), kn, vn, bt, lens, float(np.float32(D ** -0.5)), oracle.F16)
+        assert_close(out, ref, DT, f"step {step}")
+    assert cows == 1                                 # the fork's first append copied the shared partial block
+    assert pkv.get_device_error() == 0
+    assert np.array_equal(kc.cpu().numpy().view(np.int16), kn.view(np.int16))
