@@ -7,8 +7,8 @@
 // 128/B physical blocks, each fetched by its own TMA box through the block
 // table.
 //
-// Roles (160 threads):
-//  * warp 4 -- producer.  A loop that polls the pipeline's mbarriers
+// Roles (288 threads):
+//  * warp 8 -- producer.  A loop that polls the pipeline's mbarriers
 //    (test_wait, which never suspends) issues, from lane 0,, whenever its inputs are ready and its target buffer is
 //    free: the TMA loads of K and V tiles (two stages each; K of tile j+2
 //    as soon as Q.K^T of tile j is done, V of tile j+2 as soon as P.V of tile
@@ -17,7 +17,10 @@
 //    of two O buffers; bf16 P goes in as hi + lo terms).  The warp's lanes
 //    prefetch the next tiles' block ids (one per lane) so that table reads
 //    overlap the pipeline.
-//  * warps 0-3 -- one query row per thread.  For tile j: read S_j from tensor
+//  * warps 0-7 -- two threads per query row (warps w and w + 4 share TMEM lane
+//    quadrant w, each takes half of the 128 key columns and half of the
+//    head_dim output columns; the row max is exchanged through shared memory
+//    under a pair of mbarriers per quadrant).  For tile j: read S_j from tensor
 //    memory (row max), fold the finished P.V product of tile j-1 into the
 //    register accumulator (online-softmax rescale), write P_j = exp2(S_j *
 //    scale * log2 e - m) to shared memory in the 128-byte-swizzled K-major
@@ -48,8 +51,10 @@ struct PrefillParams {
     int q_tiles;  // query tiles per chunk in the grid
 };
 
-constexpr int kPrefillSoftmaxWarps = 4;
-constexpr int kPrefillThreads = (kPrefillSoftmaxWarps + 1) * 32;
+constexpr int kPrefillSoftmaxWarps = 8;  // two per TMEM lane quadrant: each row split in two column halves
+constexpr int kPrefillLoadWarp = kPrefillSoftmaxWarps;      // TMA loads of K / V tiles
+constexpr int kPrefillMmaWarp = kPrefillSoftmaxWarps + 1;   // tcgen05.mma issue
+constexpr int kPrefillThreads = (kPrefillSoftmaxWarps + 2) * 32;
 
 template <typename T, int D, int G>
 struct PrefillCfg {
@@ -72,8 +77,9 @@ struct PrefillCfg {
     static constexpr int P_OFF = V_OFF + 2 * KT_BYTES;
     static constexpr int PLO_OFF = P_OFF + P_BYTES;
     static constexpr int BAR_OFF = PLO_OFF + (SPLIT_P ? P_BYTES : 0);
-    static constexpr int NBAR = 16;
-    static constexpr int SMEM = 1024 + BAR_OFF + NBAR * 8;
+    static constexpr int NBAR = 24;
+    static constexpr int XCH_OFF = BAR_OFF + NBAR * 8;      // [128 rows][2 halves] floats
+    static constexpr int SMEM = 1024 + XCH_OFF + BM * 2 * 4;
     static constexpr uint32_t TMEM_COLS = 512;
     static constexpr uint32_t S_COL0 = 0, O_COL0 = 256;  // S buffers at 0 / 128, O buffers at 256 / 384
     static_assert(D == 64 || D == 128, "head_dim");
@@ -99,6 +105,8 @@ __global__ void __launch_bounds__(kPrefillThreads, 1) paged_prefill_kernel(const
     uint64_t* o_free = bars + 12;  // [2]  softmax folded O into registers
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 14);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + 15);
+    uint64_t* xch_full = bars + 16;  // [4]  both halves of a quadrant's rows posted a value
+    uint64_t* xch_read = bars + 20;  // [4]  both halves read their partner's value
 
     // Launch order: query tile outermost, last tile first -- later tiles of a
     // chunk attend to more keys, so the longest CTAs start in the first wave
@@ -141,6 +149,10 @@ __global__ void __launch_bounds__(kPrefillThreads, 1) paged_prefill_kernel(const
             mbar_init(&o_free[i], kPrefillSoftmaxWarps * 32);
         }
         mbar_init(p_full, kPrefillSoftmaxWarps * 32);
+        for (int i = 0; i < 4; ++i) {
+            mbar_init(&xch_full[i], 64);
+            mbar_init(&xch_read[i], 64);
+        }
         *abort_flag = 0;
         fence_mbar_init();
     }
@@ -150,20 +162,14 @@ __global__ void __launch_bounds__(kPrefillThreads, 1) paged_prefill_kernel(const
     const uint32_t tmem = *tmem_slot;
     constexpr bool kBf16 = Elem<T>::kCuType == CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
 
-    if (warp == kPrefillSoftmaxWarps) {
-        // ================================================================ producer (whole warp, lane 0 issues)
+    if (warp == kPrefillLoadWarp) {
+        // ================================================================ loader (whole warp, lane 0 issues)
         const int lane = tid & 31;
         const bool leader = lane == 0;
-        constexpr uint32_t IDESC_S = umma_idesc_f16(128, C::BN, kBf16, false, false);
-        constexpr uint32_t IDESC_O = umma_idesc_f16(128, D, kBf16, false, true);
-        const uint32_t q_addr = smem_u32(smem + C::Q_OFF);
-        const uint32_t p_addr = smem_u32(smem + C::P_OFF);
-        const uint32_t plo_addr = smem_u32(smem + C::PLO_OFF);
         const int per_tile = C::BN / B;  // blocks per key tile (4..16)
-        // Block ids of key tile j, one per lane (lane < per_tile), fetched ahead
-        // of use so that the table read overlaps the pipeline.
-        // (the load is only issued here; its value is first used, and checked,
-        // when the tile is loaded, so the read overlaps the pipeline)
+        // Block ids of key tile j, one per lane (lane < per_tile).  The load is
+        // only issued here; its value is first used, and checked, when the tile
+        // is loaded, so the table read overlaps the pipeline.
         auto fetch_ids = [&](int j) -> int {
             const int lb = j * per_tile + lane;
             return (lane < per_tile && lb < nblk) ? bt_row[lb] : -1;
@@ -187,127 +193,128 @@ __global__ void __launch_bounds__(kPrefillThreads, 1) paged_prefill_kernel(const
                 }
             }
         };
-        auto poll = [&](uint64_t* bar, uint32_t parity) -> bool {  // lane 0 probes, the warp agrees
-            return __shfl_sync(0xffffffffu, leader ? (int)mbar_poll(bar, parity) : 0, 0) != 0;
-        };
         if (leader) {
             mbar_arrive_expect_tx(q_full, C::Q_BYTES);
 #pragma unroll
             for (int pn = 0; pn < C::NP; ++pn)
                 tma_load_3d(smem + C::Q_OFF + pn * C::BM * 128, &tm_q, pn * C::PANEL, g * G, q0 + qt * C::TT, q_full);
         }
-        int nk = 0, nv = 0;
-        int ids_k = fetch_ids(0), ids_v = ids_k;
-        for (; nk < min(nkt, 2); ++nk) {
-            load_tile(&tm_k, C::K_OFF, k_full, nk, ids_k);
-            load_tile(&tm_v, C::V_OFF, v_full, nk, ids_k);
-            ids_k = fetch_ids(nk + 1);
+        int ids = fetch_ids(0);
+        int j = 0;
+        for (; j < min(nkt, 2); ++j) {
+            load_tile(&tm_k, C::K_OFF, k_full, j, ids);
+            load_tile(&tm_v, C::V_OFF, v_full, j, ids);
+            ids = fetch_ids(j + 1);
         }
-        nv = nk;
-        ids_v = ids_k;
-        int ns = 0, npv = 0;
-        bool q_ready = false;
-        uint64_t t_last = global_timer_ns();
-        while (npv < nkt) {
-            bool progress = false;
-            if (__shfl_sync(0xffffffffu, leader ? *abort_flag : 0, 0)) break;
-            if (!q_ready) q_ready = poll(q_full, 0);
-            // S_ns = Q . K_ns^T into S buffer ns % 2 (free once the softmax read S_{ns-2})
-            if (q_ready && ns < nkt) {
-                const int st = ns & 1;
-                if (poll(&k_full[st], (ns >> 1) & 1) && (ns < 2 || poll(&s_free[st], ((ns - 2) >> 1) & 1))) {
-                    if (leader) {
-                        tc_fence_after();
-                        const uint32_t k_addr = smem_u32(smem + C::K_OFF + st * C::KT_BYTES);
-#pragma unroll
-                        for (int kk = 0; kk < D / 16; ++kk) {
-                            const uint32_t qoff = (kk / 4) * (C::BM * 128) + (kk % 4) * 32;
-                            const uint32_t koff = (kk / 4) * (C::BN * 128) + (kk % 4) * 32;
-                            umma_f16_ss(tmem + C::S_COL0 + st * 128, smem_desc_sw128(q_addr + qoff, 16, 1024),
-                                        smem_desc_sw128(k_addr + koff, 16, 1024), IDESC_S, kk > 0);
-                        }
-                        umma_commit(&s_full[st]);
-                    }
-                    __syncwarp();
-                    ++ns;
-                    progress = true;
-                }
-            }
-            // K of tile nk into stage nk % 2 once Q.K^T of tile nk - 2 is done
-            if (nk < nkt && nk - 2 < ns && poll(&s_full[nk & 1], ((nk - 2) >> 1) & 1)) {
-                load_tile(&tm_k, C::K_OFF, k_full, nk, ids_k);
-                ++nk;
-                ids_k = fetch_ids(nk);
-                progress = true;
-            }
-            // O_npv = P_npv . V_npv into O buffer npv % 2 (free once the softmax folded O_{npv-2})
-            if (npv < ns) {
-                const int st = npv & 1;
-                if (poll(p_full, npv & 1) && poll(&v_full[st], (npv >> 1) & 1) &&
-                    (npv < 2 || poll(&o_free[st], ((npv - 2) >> 1) & 1))) {
-                    if (leader) {
-                        tc_fence_after();
-                        const uint32_t v_addr = smem_u32(smem + C::V_OFF + st * C::KT_BYTES);
-#pragma unroll
-                        for (int kk = 0; kk < C::BN / 16; ++kk) {
-                            const uint32_t poff = (kk / 4) * (C::BM * 128) + (kk % 4) * 32;
-                            const uint64_t vdesc = smem_desc_sw128(v_addr + kk * 16 * 128, C::BN * 128, 1024);
-                            umma_f16_ss(tmem + C::O_COL0 + st * 128, smem_desc_sw128(p_addr + poff, 16, 1024), vdesc,
-                                        IDESC_O, kk > 0);
-                            if constexpr (C::SPLIT_P)
-                                umma_f16_ss(tmem + C::O_COL0 + st * 128, smem_desc_sw128(plo_addr + poff, 16, 1024),
-                                            vdesc, IDESC_O, 1);
-                        }
-                        umma_commit(&o_full[st]);
-                    }
-                    __syncwarp();
-                    ++npv;
-                    progress = true;
-                }
-            }
-            // V of tile nv into stage nv % 2 once P.V of tile nv - 2 is done
-            if (nv < nkt && nv - 2 < npv && poll(&o_full[nv & 1], ((nv - 2) >> 1) & 1)) {
-                load_tile(&tm_v, C::V_OFF, v_full, nv, ids_v);
-                ++nv;
-                ids_v = fetch_ids(nv);
-                progress = true;
-            }
-            if (progress) {
-                t_last = global_timer_ns();
-            } else {
-                __nanosleep(32);  // leave issue slots to the softmax warp sharing this scheduler
-                if (__shfl_sync(0xffffffffu, (int)(global_timer_ns() - t_last > kWaitLimitNs), 0)) {
-                    if (leader) {
-                        flag_error(PKV_DEVERR_TIMEOUT);
-                        *abort_flag = 1;
-                    }
-                    break;
-                }
-            }
+        // K of tile j once Q.K^T of tile j - 2 freed its stage; V of tile j once P.V of tile j - 2 did.
+        int loaded_k = j, loaded_v = j;
+        for (; j < nkt; ++j) {
+            const int ids_next = fetch_ids(j + 1);
+            if (!__all_sync(0xffffffffu, mbar_wait_or_abort(&s_full[j & 1], ((j - 2) >> 1) & 1, abort_flag))) break;
+            load_tile(&tm_k, C::K_OFF, k_full, j, ids);
+            loaded_k = j + 1;
+            if (!__all_sync(0xffffffffu, mbar_wait_or_abort(&o_full[j & 1], ((j - 2) >> 1) & 1, abort_flag))) break;
+            load_tile(&tm_v, C::V_OFF, v_full, j, ids);
+            loaded_v = j + 1;
+            ids = ids_next;
         }
         if (leader && *abort_flag) {
-            // Wait (bounded) for the last MMAs and copies this warp issued
-            // before tensor and shared memory are released.
-            if (ns > 0) mbar_wait(&s_full[(ns - 1) & 1], ((ns - 1) >> 1) & 1);
-            if (npv > 0) mbar_wait(&o_full[(npv - 1) & 1], ((npv - 1) >> 1) & 1);
-            for (int j = max(0, nk - 2); j < nk; ++j) mbar_wait(&k_full[j & 1], (j >> 1) & 1);
-            for (int j = max(0, nv - 2); j < nv; ++j) mbar_wait(&v_full[j & 1], (j >> 1) & 1);
+            // wait (bounded) for this warp's copies still in flight
+            for (int t = max(0, loaded_k - 2); t < loaded_k; ++t) mbar_wait(&k_full[t & 1], (t >> 1) & 1);
+            for (int t = max(0, loaded_v - 2); t < loaded_v; ++t) mbar_wait(&v_full[t & 1], (t >> 1) & 1);
+        }
+    } else if (warp == kPrefillMmaWarp) {
+        // ================================================================ MMA issue (lane 0)
+        // Order: S_0, S_1, O_0, S_2, O_1, ... -- the next tile's Q.K^T is always
+        // queued ahead of the current tile's P.V.
+        if ((tid & 31) == 0) {
+            constexpr uint32_t IDESC_S = umma_idesc_f16(128, C::BN, kBf16, false, false);
+            constexpr uint32_t IDESC_O = umma_idesc_f16(128, D, kBf16, false, true);
+            const uint32_t q_addr = smem_u32(smem + C::Q_OFF);
+            const uint32_t p_addr = smem_u32(smem + C::P_OFF);
+            const uint32_t plo_addr = smem_u32(smem + C::PLO_OFF);
+            int ns = 0, npv = 0;
+            auto issue_s = [&](int t) -> bool {
+                const int st = t & 1;
+                if (!mbar_wait_or_abort(&k_full[st], (t >> 1) & 1, abort_flag)) return false;
+                if (t >= 2 && !mbar_wait_or_abort(&s_free[st], ((t - 2) >> 1) & 1, abort_flag)) return false;
+                tc_fence_after();
+                const uint32_t k_addr = smem_u32(smem + C::K_OFF + st * C::KT_BYTES);
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk) {
+                    const uint32_t qoff = (kk / 4) * (C::BM * 128) + (kk % 4) * 32;
+                    const uint32_t koff = (kk / 4) * (C::BN * 128) + (kk % 4) * 32;
+                    umma_f16_ss(tmem + C::S_COL0 + st * 128, smem_desc_sw128(q_addr + qoff, 16, 1024),
+                                smem_desc_sw128(k_addr + koff, 16, 1024), IDESC_S, kk > 0);
+                }
+                umma_commit(&s_full[st]);
+                ns = t + 1;
+                return true;
+            };
+            auto issue_pv = [&](int t) -> bool {
+                const int st = t & 1;
+                if (!mbar_wait_or_abort(p_full, t & 1, abort_flag)) return false;
+                if (!mbar_wait_or_abort(&v_full[st], (t >> 1) & 1, abort_flag)) return false;
+                if (t >= 2 && !mbar_wait_or_abort(&o_free[st], ((t - 2) >> 1) & 1, abort_flag)) return false;
+                tc_fence_after();
+                const uint32_t v_addr = smem_u32(smem + C::V_OFF + st * C::KT_BYTES);
+#pragma unroll
+                for (int kk = 0; kk < C::BN / 16; ++kk) {
+                    const uint32_t poff = (kk / 4) * (C::BM * 128) + (kk % 4) * 32;
+                    const uint64_t vdesc = smem_desc_sw128(v_addr + kk * 16 * 128, C::BN * 128, 1024);
+                    umma_f16_ss(tmem + C::O_COL0 + st * 128, smem_desc_sw128(p_addr + poff, 16, 1024), vdesc, IDESC_O,
+                                kk > 0);
+                    if constexpr (C::SPLIT_P)
+                        umma_f16_ss(tmem + C::O_COL0 + st * 128, smem_desc_sw128(plo_addr + poff, 16, 1024), vdesc,
+                                    IDESC_O, 1);
+                }
+                umma_commit(&o_full[st]);
+                npv = t + 1;
+                return true;
+            };
+            bool ok = mbar_wait_or_abort(q_full, 0, abort_flag) && issue_s(0);
+            for (int t = 0; ok && t < nkt; ++t) {
+                if (t + 1 < nkt) ok = issue_s(t + 1);
+                if (ok) ok = issue_pv(t);
+            }
+            if (*abort_flag) {
+                // wait (bounded) for the MMAs this thread issued before tensor memory is released
+                if (ns > 0) mbar_wait(&s_full[(ns - 1) & 1], ((ns - 1) >> 1) & 1);
+                if (npv > 0) mbar_wait(&o_full[(npv - 1) & 1], ((npv - 1) >> 1) & 1);
+            }
         }
     } else {
         // ================================================================ softmax rows
-        const int row = tid;
+        const int quad = warp & 3, half = warp >> 2;
+        const int row = quad * 32 + (tid & 31);
         const int tok = qt * C::TT + row / G;
         const int qpos = c0 + tok;  // absolute position of the row's query
-        const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
+        const uint32_t lane_base = static_cast<uint32_t>(quad * 32) << 16;
+        constexpr int HC = C::BN / 2;  // key columns of this thread
+        constexpr int HD = D / 2;      // output columns of this thread
         uint8_t* p_s = smem + C::P_OFF;
         uint8_t* plo_s = smem + C::PLO_OFF;
+        float* xch = reinterpret_cast<float*>(smem + C::XCH_OFF);
         const float sl2 = p.scale_log2;
-        float o[D];
+        float o[HD];
 #pragma unroll
-        for (int d = 0; d < D; ++d) o[d] = 0.f;
+        for (int d = 0; d < HD; ++d) o[d] = 0.f;
         float m = -INFINITY, lsum = 0.f, alpha_prev = 1.f;
         bool ok = true;
         float v[32];
+        // Post this half's value for the row, return the partner half's (exchange
+        // number e; the slot is reused once the partner read the previous one).
+        auto exchange = [&](float mine, int e, float& theirs) -> bool {
+            if (e > 0 &&
+                !__all_sync(0xffffffffu, mbar_wait_or_abort(&xch_read[quad], (e - 1) & 1, abort_flag)))
+                return false;
+            xch[row * 2 + half] = mine;
+            mbar_arrive(&xch_full[quad]);
+            if (!__all_sync(0xffffffffu, mbar_wait_or_abort(&xch_full[quad], e & 1, abort_flag))) return false;
+            theirs = xch[row * 2 + (half ^ 1)];
+            mbar_arrive(&xch_read[quad]);
+            return true;
+        };
         for (int j = 0; j < nkt; ++j) {
             const int st = j & 1;
             if (!__all_sync(0xffffffffu, mbar_wait_or_abort(&s_full[st], (j >> 1) & 1, abort_flag))) {
@@ -315,15 +322,15 @@ __global__ void __launch_bounds__(kPrefillThreads, 1) paged_prefill_kernel(const
                 break;
             }
             tc_fence_after();
-            const uint32_t ts = tmem + lane_base + C::S_COL0 + st * 128;
-            const int k0 = j * C::BN;
-            const bool all_vis = k0 + C::BN - 1 <= qpos;
+            const uint32_t ts = tmem + lane_base + C::S_COL0 + st * 128 + half * HC;
+            const int k0 = j * C::BN + half * HC;  // first key of this thread's columns
+            const bool all_vis = k0 + HC - 1 <= qpos;
             const bool none_vis = k0 > qpos;
-            // ---- pass 1: row max of the visible scores (scale sign handled by max / min)
+            // ---- pass 1: max of the visible scores of this half row (scale sign via max / min)
             // (tcgen05.ld is warp-collective: every lane loads, masking is per row in registers)
             float hi_raw = -INFINITY, lo_raw = INFINITY;
 #pragma unroll
-            for (int c = 0; c < C::BN / 32; ++c) {
+            for (int c = 0; c < HC / 32; ++c) {
                 tmem_ld32(ts + c * 32, v);
                 if (all_vis) {
 #pragma unroll
@@ -334,31 +341,56 @@ __global__ void __launch_bounds__(kPrefillThreads, 1) paged_prefill_kernel(const
                         if (k0 + c * 32 + i <= qpos) hi_raw = fmaxf(hi_raw, v[i]), lo_raw = fminf(lo_raw, v[i]);
                 }
             }
-            const float mloc = none_vis ? -INFINITY : (sl2 >= 0.f ? hi_raw * sl2 : lo_raw * sl2);
-            const float mnew = fmaxf(m, mloc);
+            const float mhalf = none_vis ? -INFINITY : (sl2 >= 0.f ? hi_raw * sl2 : lo_raw * sl2);
+            float mother = -INFINITY;
+            if (!exchange(mhalf, j, mother)) {
+                ok = false;
+                break;
+            }
+            const float mnew = fmaxf(m, fmaxf(mhalf, mother));
             const float alpha = ex2_approx(m - mnew);
-            // ---- fold P.V of the previous tile into the accumulator
-            if (j >= 1) {
-                const int jp = j - 1;
-                if (!__all_sync(0xffffffffu, mbar_wait_or_abort(&o_full[jp & 1], (jp >> 1) & 1, abort_flag))) {
-                    ok = false;
-                    break;
-                }
-                tc_fence_after();
-                const uint32_t to = tmem + lane_base + C::O_COL0 + (jp & 1) * 128;
+            // ---- pass 2: P = exp2(S * scale * log2 e - m) for this half (= P panel `half`), into registers
+            float tsum = 0.f;
+            uint32_t hi[HC / 2], lo[C::SPLIT_P ? HC / 2 : 1];
 #pragma unroll
-                for (int c = 0; c < D / 32; ++c) {
-                    tmem_ld32(to + c * 32, v);
+            for (int c = 0; c < HC / 32; ++c) {
+                tmem_ld32(ts + c * 32, v);
 #pragma unroll
-                    for (int i = 0; i < 32; ++i) o[c * 32 + i] = fmaf(o[c * 32 + i], alpha_prev, v[i]);
+                for (int i = 0; i < 32; i += 2) {
+                    const int key = k0 + c * 32 + i;
+                    float p0 = ex2_approx(fmaf(v[i], sl2, -mnew));
+                    float p1 = ex2_approx(fmaf(v[i + 1], sl2, -mnew));
+                    if (!all_vis) {
+                        p0 = key <= qpos ? p0 : 0.f;
+                        p1 = key + 1 <= qpos ? p1 : 0.f;
+                    }
+                    tsum += p0 + p1;
+                    const int w = c * 16 + i / 2;
+                    if constexpr (C::SPLIT_P) {
+                        // hi = p truncated to bf16 (its top 16 bits, one byte permute for the
+                        // pair); lo = the exact remainder rounded to bf16, |lo| < 2^-7 |p|
+                        const uint32_t b0 = __float_as_uint(p0), b1 = __float_as_uint(p1);
+                        hi[w] = __byte_perm(b0, b1, 0x7632);
+                        lo[w] = Elem<T>::pack(p0 - __uint_as_float(b0 & 0xFFFF0000u),
+                                              p1 - __uint_as_float(b1 & 0xFFFF0000u));
+                    } else {
+                        hi[w] = Elem<T>::pack(p0, p1);
+                    }
                 }
-                tc_fence_before();
-                mbar_arrive(&o_free[jp & 1]);
+            }
+            tc_fence_before();
+            mbar_arrive(&s_free[st]);  // S_j fully read: its buffer may take S_{j+2}
+            // ---- P.V of the previous tile must be done before P is overwritten
+            if (j >= 1 &&
+                !__all_sync(0xffffffffu, mbar_wait_or_abort(&o_full[(j - 1) & 1], ((j - 1) >> 1) & 1, abort_flag))) {
+                ok = false;
+                break;
             }
             // ---- the last tile may hold the dead tail of the sequence's last
             // block: zero those V rows (0 * NaN must not reach the output)
             if (j == nkt - 1) {
-                const int dead_lo = max(L, k0), dead_hi = min(nblk * B, k0 + C::BN);
+                const int tk0 = j * C::BN;
+                const int dead_lo = max(L, tk0), dead_hi = min(nblk * B, tk0 + C::BN);
                 if (dead_lo < dead_hi) {
                     if (!__all_sync(0xffffffffu, mbar_wait_or_abort(&v_full[st], (j >> 1) & 1, abort_flag))) {
                         ok = false;
@@ -367,61 +399,37 @@ __global__ void __launch_bounds__(kPrefillThreads, 1) paged_prefill_kernel(const
                     uint8_t* vs = smem + C::V_OFF + st * C::KT_BYTES;
                     const int rows = dead_hi - dead_lo;
                     for (int i = tid; i < rows * C::NP * 8; i += kPrefillSoftmaxWarps * 32) {
-                        const int rr = (dead_lo - k0) + i / (C::NP * 8);
+                        const int rr = (dead_lo - tk0) + i / (C::NP * 8);
                         const int rest = i % (C::NP * 8);
                         *reinterpret_cast<uint4*>(vs + (rest / 8) * C::BN * 128 + rr * 128 + (rest % 8) * 16) =
                             make_uint4(0, 0, 0, 0);
                     }
                 }
             }
-            // ---- pass 2: P = exp2(S * scale * log2 e - m), K-major swizzled rows
-            float tsum = 0.f;
 #pragma unroll
-            for (int c = 0; c < C::BN / 32; ++c) {
-                uint32_t hi[16], lo[16];
-                tmem_ld32(ts + c * 32, v);
-                if (none_vis) {
-#pragma unroll
-                    for (int i = 0; i < 16; ++i) hi[i] = lo[i] = 0u;
-                } else {
-#pragma unroll
-                    for (int i = 0; i < 32; i += 2) {
-                        const int key = k0 + c * 32 + i;
-                        float p0 = ex2_approx(fmaf(v[i], sl2, -mnew));
-                        float p1 = ex2_approx(fmaf(v[i + 1], sl2, -mnew));
-                        if (!all_vis) {
-                            p0 = key <= qpos ? p0 : 0.f;
-                            p1 = key + 1 <= qpos ? p1 : 0.f;
-                        }
-                        tsum += p0 + p1;
-                        if constexpr (C::SPLIT_P) {
-                            // hi = p truncated to bf16 (its top 16 bits, one byte permute for the
-                            // pair); lo = the exact remainder rounded to bf16, |lo| < 2^-7 |p|
-                            const uint32_t b0 = __float_as_uint(p0), b1 = __float_as_uint(p1);
-                            hi[i / 2] = __byte_perm(b0, b1, 0x7632);
-                            lo[i / 2] = Elem<T>::pack(p0 - __uint_as_float(b0 & 0xFFFF0000u),
-                                                      p1 - __uint_as_float(b1 & 0xFFFF0000u));
-                        } else {
-                            hi[i / 2] = Elem<T>::pack(p0, p1);
-                        }
-                    }
-                }
-#pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                    const int cc = 4 * (c % 2) + q;
-                    const int off = (c / 2) * (C::BM * 128) + row * 128 + ((cc ^ (row & 7)) << 4);
-                    *reinterpret_cast<uint4*>(p_s + off) =
-                        make_uint4(hi[4 * q], hi[4 * q + 1], hi[4 * q + 2], hi[4 * q + 3]);
-                    if constexpr (C::SPLIT_P)
-                        *reinterpret_cast<uint4*>(plo_s + off) =
-                            make_uint4(lo[4 * q], lo[4 * q + 1], lo[4 * q + 2], lo[4 * q + 3]);
-                }
+            for (int q = 0; q < HC / 8; ++q) {  // 16-byte chunks of this half row
+                const int off = half * (C::BM * 128) + row * 128 + ((q ^ (row & 7)) << 4);
+                *reinterpret_cast<uint4*>(p_s + off) = make_uint4(hi[4 * q], hi[4 * q + 1], hi[4 * q + 2], hi[4 * q + 3]);
+                if constexpr (C::SPLIT_P)
+                    *reinterpret_cast<uint4*>(plo_s + off) =
+                        make_uint4(lo[4 * q], lo[4 * q + 1], lo[4 * q + 2], lo[4 * q + 3]);
             }
-            tc_fence_before();
-            mbar_arrive(&s_free[st]);
             fence_proxy_async();
             mbar_arrive(p_full);
-            lsum = lsum * alpha + tsum;
+            // ---- fold P.V of the previous tile into this half of the accumulator
+            if (j >= 1) {
+                tc_fence_after();
+                const uint32_t to = tmem + lane_base + C::O_COL0 + ((j - 1) & 1) * 128 + half * HD;
+#pragma unroll
+                for (int c = 0; c < HD / 32; ++c) {
+                    tmem_ld32(to + c * 32, v);
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) o[c * 32 + i] = fmaf(o[c * 32 + i], alpha_prev, v[i]);
+                }
+                tc_fence_before();
+                mbar_arrive(&o_free[(j - 1) & 1]);
+            }
+            lsum = lsum * alpha + tsum;  // this half's share of the row sum
             m = mnew;
             alpha_prev = alpha;
         }
@@ -429,9 +437,9 @@ __global__ void __launch_bounds__(kPrefillThreads, 1) paged_prefill_kernel(const
             const int jl = nkt - 1;
             if (__all_sync(0xffffffffu, mbar_wait_or_abort(&o_full[jl & 1], (jl >> 1) & 1, abort_flag))) {
                 tc_fence_after();
-                const uint32_t to = tmem + lane_base + C::O_COL0 + (jl & 1) * 128;
+                const uint32_t to = tmem + lane_base + C::O_COL0 + (jl & 1) * 128 + half * HD;
 #pragma unroll
-                for (int c = 0; c < D / 32; ++c) {
+                for (int c = 0; c < HD / 32; ++c) {
                     tmem_ld32(to + c * 32, v);
 #pragma unroll
                     for (int i = 0; i < 32; ++i) o[c * 32 + i] = fmaf(o[c * 32 + i], alpha_prev, v[i]);
@@ -440,12 +448,15 @@ __global__ void __launch_bounds__(kPrefillThreads, 1) paged_prefill_kernel(const
                 ok = false;
             }
         }
+        float lother = 0.f;
+        if (ok && !exchange(lsum, nkt, lother)) ok = false;
         if (ok && !*abort_flag && tok < n) {
-            const float inv = 1.f / lsum;
+            const float inv = 1.f / (lsum + lother);
             T* dst = reinterpret_cast<T*>(p.out) +
-                     (static_cast<int64_t>(q0 + tok) * p.num_q_heads + static_cast<int64_t>(g) * G + row % G) * D;
+                     (static_cast<int64_t>(q0 + tok) * p.num_q_heads + static_cast<int64_t>(g) * G + row % G) * D +
+                     half * HD;
 #pragma unroll
-            for (int d = 0; d < D; d += 8) {
+            for (int d = 0; d < HD; d += 8) {
                 uint4 w;
                 w.x = Elem<T>::pack(o[d] * inv, o[d + 1] * inv);
                 w.y = Elem<T>::pack(o[d + 2] * inv, o[d + 3] * inv);
