@@ -174,6 +174,73 @@ class MixedStep(DecodeStep):
             timer.end()
 
 
+class MultiTokenStep:
+    """Multi-token decode (speculative verification): append each sequence's
+    draft tokens, then the causal attention of all of them over the cache in
+    one chunked-prefill call."""
+
+    def __init__(self, m):
+        import paged_kv_cache_409_b200 as pkv
+        self.pkv, self.m, self.w = pkv, m, m.decode
+        dev = m.chunk_query.device
+        self.aslots = torch.from_numpy(m.append_slots).to(dev)
+        self.cbt = torch.from_numpy(m.chunk_tables).to(dev)
+        self.csl = torch.from_numpy(m.seq_lens).to(dev)
+        self.qsl = torch.from_numpy(m.query_start_loc).to(dev)
+        self.out = torch.empty_like(m.chunk_query)
+        self.max_q = int(m.chunk_lens.max())
+        self.layers, self.part = 1, 0
+        w = m.decode
+        t = m.chunk_query.element_size()
+        self.kv_bytes = 2 * int(m.seq_lens.astype(np.int64).sum()) * w.num_kv_heads * w.head_dim * t
+        nblocks = int(((m.seq_lens.astype(np.int64) + w.block_size - 1) // w.block_size).sum())
+        self.decode_bytes = self.kv_bytes + 2 * m.chunk_query.numel() * t + 4 * nblocks + 8 * len(m.seq_lens)
+        self.tokens = int(m.chunk_lens.sum())
+        self.kernel = "paged_attention_prefill_chunk (tcgen05)"
+
+    def config(self):
+        m = self.m
+        return {"num_seqs": len(m.chunk_lens), "draft_tokens": self.tokens,
+                "draft_len_range": [int(m.chunk_lens.min()), int(m.chunk_lens.max())],
+                "context_range": [int(m.chunk_c0.min()), int(m.chunk_c0.max())]}
+
+    def oracle_sample(self, budget_s, max_seqs=8):
+        """Oracle append + causal attention of the first sequences' drafts."""
+        sys.path.insert(0, os.path.join(ROOT, "tests"))
+        from parity_helpers import oracle_prefill_chunks
+        m, w = self.m, self.w
+        chunks = np.arange(min(max_seqs, len(m.chunk_lens)))
+        pre_k, pre_v = w.key_caches[0].cpu(), w.value_caches[0].cpu()
+        done, t0 = 0, time.perf_counter()
+        while True:
+            oracle_prefill_chunks(m, pre_k, pre_v, chunks)
+            done += 1
+            el = time.perf_counter() - t0
+            if el >= budget_s:
+                break
+        ntok = int(m.chunk_lens[chunks].sum())
+        return ntok * done / el, done, f"{len(chunks)} sequences ({ntok} draft tokens)", el
+
+    def launches_per_step(self):
+        return 2
+
+    def e2e_plan(self):
+        m = self.m
+        pairs = [(t, pinned(t)) for t in (m.chunk_query, m.append_keys, m.append_values, self.aslots, self.cbt,
+                                          self.csl, self.qsl)]
+        return E2EPlan(self, pairs, [(self.out, pinned(self.out))])
+
+    def run(self, timer=None, step=0):
+        m, w = self.m, self.w
+        self.pkv.reshape_and_cache(m.append_keys, m.append_values, w.key_caches[0], w.value_caches[0], self.aslots)
+        if timer:
+            timer.begin()
+        self.pkv.paged_attention_prefill_chunk(self.out, m.chunk_query, w.key_caches[0], w.value_caches[0],
+                                               self.cbt, self.csl, self.qsl, self.max_q, w.scale)
+        if timer:
+            timer.end()
+
+
 def make_step(name, device, rank, seqs=None, layers=None):
     from paged_kv_cache_409_b200 import workloads
     if name == "llama7b_decode_f16":
@@ -200,6 +267,9 @@ def make_step(name, device, rank, seqs=None, layers=None):
     if name == "mixed_step_bf16":
         m = workloads.mixed_step_bf16(device=device, seed=1005 + rank, num_decode=seqs or 192)
         return MixedStep(m), name + (f" ({seqs} decode sequences)" if seqs else "")
+    if name == "multi_token_decode_bf16":
+        m = workloads.multi_token_decode_bf16(device=device, seed=1006 + rank, num_seqs=seqs or 64)
+        return MultiTokenStep(m), name + (f" ({seqs} sequences)" if seqs else "")
     raise SystemExit(f"unknown config {name}")
 
 
@@ -373,20 +443,29 @@ def run_reference(args, ws, rank):
     dev = "cuda" if torch.cuda.is_available() else "cpu"
     step, cname = make_step(args.config, dev, 0)
     w = step.w
-    sample = min(w.num_seqs, 8)
     times = []
-    for i in range(args.warmup + args.steps):
-        v, done, n, el = oracle_sample(step, 0.0, max_seqs=sample)
-        if i >= args.warmup:
-            times.append(el)
-    per = statistics.fmean(times)
-    value = sample / per
+    if hasattr(step, "oracle_sample"):
+        for i in range(args.warmup + args.steps):
+            v, done, what, el = step.oracle_sample(0.0)
+            if i >= args.warmup:
+                times.append(el)
+        per = statistics.fmean(times)
+        value, sample_text = v * el / per, f"append + causal attention of {what} per step"
+        sample = what
+    else:
+        sample = min(w.num_seqs, 8)
+        for i in range(args.warmup + args.steps):
+            v, done, n, el = oracle_sample(step, 0.0, max_seqs=sample)
+            if i >= args.warmup:
+                times.append(el)
+        per = statistics.fmean(times)
+        value = sample / per
+        sample_text = f"append + decode of the first {sample} of {w.num_seqs} sequences per step"
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": args.gpus,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": per * 1e3, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": cname, "sample_seqs": sample},
-            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": 1, "kind": "oracle",
-                             "sample": f"append + decode of the first {sample} of {w.num_seqs} sequences per step"},
+            "config": {"workload": cname, "sample": sample},
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": 1, "kind": "oracle", "sample": sample_text},
             "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
 
@@ -548,7 +627,7 @@ def main():
                        2 * w.key_caches[0].numel() * w.key_caches[0].element_size() / 1e9),
                    "parallelism": f"replicas x{ws}"},
         "kv_gbs": step.kv_bytes * step.layers / (ms_step / 1e3) / 1e9,
-        "roofline": {"bound": "hbm", "kernel": "paged_attention_decode (decode + merge kernels)",
+        "roofline": {"bound": "hbm", "kernel": getattr(step, "kernel", "paged_attention_decode (decode + merge kernels)"),
                      "achieved": achieved, "peak": hbm, "peak_kind": pk_kind, "unit": "GB/s",
                      "frac": achieved / hbm, "frac_of_8000_nominal": achieved / 8000.0, "traffic": None},
         "e2e": {"value": weak_scaling_value(ws, tokens_per_step, e2e_ms), "unit": "tokens/s",
@@ -556,10 +635,16 @@ def main():
         "gpu_launches": step.launches_per_step() * args.steps,
         "clocks": clk,
     }
+    if hasattr(step, "config"):
+        line["config"].update(step.config())
     if isinstance(step, MixedStep):
         line["prefill_tokens_per_s"] = ws * step.prefill_tokens / (ms_step / 1e3)
         line["prefill_flops_per_step"] = step.prefill_flops
-    if rank == 0 and ws == 1 and args.cpu_budget > 0 and args.config != "gqa70b_decode_bf16":
+    if rank == 0 and ws == 1 and args.cpu_budget > 0 and hasattr(step, "oracle_sample"):
+        v, done, what, el = step.oracle_sample(args.cpu_budget)
+        line["cpu_baseline"] = {"value": v, "unit": "tokens/s", "cores": 1, "kind": "oracle",
+                                "sample": f"{done} x (append + causal attention of {what}), {el:.1f} s, 1 thread"}
+    elif rank == 0 and ws == 1 and args.cpu_budget > 0 and args.config != "gqa70b_decode_bf16":
         v, done, n, el = oracle_sample(step, args.cpu_budget, max_seqs=None if w.num_seqs <= 64 else 16)
         line["cpu_baseline"] = {"value": v, "unit": "tokens/s", "cores": 1, "kind": "oracle",
                                 "sample": f"{done} x (append + decode of {n} sequences), {el:.1f} s, 1 thread"}

@@ -354,10 +354,24 @@ def mixed_step_bf16(device="cpu", num_decode=192, num_chunks=4, chunk_len=512, p
                           poison=poison)
 
 
+def multi_token_decode_bf16(device="cpu", num_seqs=64, draft_lo=2, draft_hi=6, c0_lo=256, c0_hi=4096,
+                            poison=False, seed=1006):
+    """Multi-token decode (speculative verification): each of 64 sequences
+    appends n ~ U{2..6} draft tokens after a context of U[256, 4096] tokens and
+    attends causally over the whole cache; 32 q heads over 8 KV heads, d 128,
+    block 32, bf16."""
+    rng = np.random.default_rng(seed)
+    c0 = rng.integers(c0_lo, c0_hi + 1, size=num_seqs)
+    n = rng.integers(draft_lo, draft_hi + 1, size=num_seqs)
+    return mixed_workload("multi_token_decode_bf16", [], c0, n, 32, 8, 128, 32, torch.bfloat16, seed=seed,
+                          device=device, poison=poison)
+
+
 CONFIGS = {
     "tiny_decode_f32": tiny_decode_f32,
     "llama7b_decode_f16": llama7b_decode_f16,
     "gqa70b_decode_bf16": gqa70b_decode_bf16,
     "shared_prefix_decode_f16": shared_prefix_decode_f16,
     "mixed_step_bf16": mixed_step_bf16,
+    "multi_token_decode_bf16": multi_token_decode_bf16,
 }

@@ -111,3 +111,36 @@ def gpu_decode_step(w, layer=0, partition_size=None, out=None, tables=None):
     pkv.paged_attention_decode(out, w.queries[layer], kc, vc, bt, cl, w.scale, w.max_context_len,
                                partition_size=partition_size)
     return out
+
+
+def oracle_prefill_chunks(m, pre_k, pre_v, chunks=None, row_select=None):
+    """Oracle of append-then-prefill for chunks ``chunks`` of a MixedWorkload.
+
+    ``pre_k``/``pre_v`` are host snapshots of the pools taken before the CUDA
+    path ran.  Only the blocks of the selected chunks are copied (renumbered
+    densely).  Returns float64 [sum of the selected chunk lengths, Hq, D].
+    """
+    R = len(m.chunk_lens)
+    chunks = np.arange(R) if chunks is None else np.asarray(chunks)
+    S = m.decode.num_seqs
+    B = m.decode.block_size
+    lens = m.seq_lens[chunks]
+    used, bt = compact_tables(m.chunk_tables[chunks], lens, B)
+    kn, code = oracle.storage(snapshot_blocks(pre_k, used))
+    vn, _ = oracle.storage(snapshot_blocks(pre_v, used))
+    kn, vn = kn.copy(), vn.copy()
+    remap = {int(b): i for i, b in enumerate(used)}
+    qsl = m.query_start_loc
+    rows = np.concatenate([np.arange(qsl[r], qsl[r + 1]) for r in chunks]).astype(np.int64)
+    src = S + rows  # the chunk tokens follow the decode tokens in append_*
+    cslots = m.append_slots[src]
+    slots = np.array([remap[int(x) // B] * B + int(x) % B for x in cslots], dtype=np.int64)
+    orc = oracle.get()
+    idx = torch.from_numpy(src)
+    orc.reshape_and_cache(oracle.storage(m.append_keys.cpu()[idx])[0], oracle.storage(m.append_values.cpu()[idx])[0],
+                          kn, vn, slots, code)
+    n = m.chunk_lens[chunks].astype(np.int64)
+    new_qsl = np.concatenate([[0], np.cumsum(n)]).astype(np.int32)
+    q = oracle.storage(m.chunk_query.cpu()[torch.from_numpy(rows)])[0]
+    return orc.paged_attention_prefill_chunk(q, kn, vn, bt, lens, new_qsl, m.decode.scale, code,
+                                             row_select=row_select)
