@@ -27,7 +27,7 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 SOURCE = os.path.join(_HERE, "pagedkv_oracle.c")
 _LIB_PATH = os.path.join(_HERE, "liboracle.so")
 
-F32, F16, BF16 = 0, 1, 2
+F32, F16, BF16, E4M3 = 0, 1, 2, 3
 
 
 def compile_source(src: str, out: str) -> str:
@@ -84,8 +84,15 @@ class Oracle:
         lib.oracle_copy_blocks.argtypes = [P, P, I, P, L, L, L]
         lib.oracle_paged_attention_decode.argtypes = [P, P, P, P, I, P, P, D, L, I, I, I, I, I, L]
         lib.oracle_paged_attention_prefill_chunk.argtypes = [P, P, P, P, I, P, P, P, I, D, I, I, I, I, I, L, P]
+        lib.oracle_e4m3_encode.argtypes = [P, P, L]
+        lib.oracle_reshape_and_cache_fp8.argtypes = [P, P, P, P, P, L, I, I, I, L, I, D, D]
+        lib.oracle_paged_attention_decode_kv.argtypes = [P, P, I, P, P, I, D, D, P, P, D, L, I, I, I, I, I, L]
+        lib.oracle_paged_attention_prefill_chunk_kv.argtypes = [P, P, I, P, P, I, D, D, P, P, P, I, D, I, I, I, I,
+                                                                I, L, P]
         for f in (lib.oracle_to_double, lib.oracle_reshape_and_cache, lib.oracle_copy_blocks,
-                  lib.oracle_paged_attention_decode, lib.oracle_paged_attention_prefill_chunk):
+                  lib.oracle_paged_attention_decode, lib.oracle_paged_attention_prefill_chunk,
+                  lib.oracle_e4m3_encode, lib.oracle_reshape_and_cache_fp8, lib.oracle_paged_attention_decode_kv,
+                  lib.oracle_paged_attention_prefill_chunk_kv):
             f.restype = ctypes.c_int
         self.lib = lib
         self.path = path
@@ -156,6 +163,61 @@ class Oracle:
             _ptr(sl), _ptr(qsl), len(sl), float(scale), Hq, Hkv, D, B, bt.shape[1], NB,
             _ptr(sel) if sel is not None else None)
         _check(rc, "paged_attention_prefill_chunk")
+        return out
+
+
+    # ---------------------------------------------------------------- FP8 (E4M3) pools
+    def e4m3_encode(self, x) -> np.ndarray:
+        """uint8 E4M3 codes of float64 values (nearest, ties to even, clamp at 448)."""
+        x = np.ascontiguousarray(x, dtype=np.float64)
+        out = np.empty(x.shape, dtype=np.uint8)
+        _check(self.lib.oracle_e4m3_encode(_ptr(out), _ptr(x), x.size), "e4m3_encode")
+        return out
+
+    def reshape_and_cache_fp8(self, key, value, key_cache, value_cache, slot_mapping, src_dtype, k_scale, v_scale):
+        """In place on uint8 pools ``[NB, B, Hkv, D]``: codes of key / k_scale and value / v_scale."""
+        T, Hkv, D = key.shape
+        NB, B = key_cache.shape[:2]
+        assert key_cache.dtype == np.uint8 and value_cache.dtype == np.uint8
+        sm = np.ascontiguousarray(slot_mapping, dtype=np.int64)
+        rc = self.lib.oracle_reshape_and_cache_fp8(_ptr(np.ascontiguousarray(key)), _ptr(np.ascontiguousarray(value)),
+                                                   _ptr(key_cache), _ptr(value_cache), _ptr(sm), T, Hkv, D, B, NB,
+                                                   src_dtype, float(k_scale), float(v_scale))
+        _check(rc, "reshape_and_cache_fp8")
+
+    def paged_attention_decode_kv(self, query, q_dtype, key_cache, value_cache, kv_dtype, k_scale, v_scale,
+                                  block_tables, context_lens, scale):
+        """Decode with the pools in their own type and scales: float64 ``[S, Hq, D]``."""
+        S, Hq, D = query.shape
+        NB, B, Hkv, D2 = key_cache.shape
+        assert D2 == D
+        bt = np.ascontiguousarray(block_tables, dtype=np.int32).reshape(S, -1)
+        cl = np.ascontiguousarray(context_lens, dtype=np.int32)
+        out = np.zeros((S, Hq, D), dtype=np.float64)
+        rc = self.lib.oracle_paged_attention_decode_kv(
+            _ptr(out), _ptr(np.ascontiguousarray(query)), q_dtype, _ptr(key_cache), _ptr(value_cache), kv_dtype,
+            float(k_scale), float(v_scale), _ptr(bt), _ptr(cl), float(scale), S, Hq, Hkv, D, B, bt.shape[1], NB)
+        _check(rc, "paged_attention_decode_kv")
+        return out
+
+    def paged_attention_prefill_chunk_kv(self, query, q_dtype, key_cache, value_cache, kv_dtype, k_scale, v_scale,
+                                         block_tables, seq_lens, query_start_loc, scale, row_select=None):
+        """Chunked prefill with the pools in their own type and scales."""
+        Tq, Hq, D = query.shape
+        NB, B, Hkv, _ = key_cache.shape
+        sl = np.ascontiguousarray(seq_lens, dtype=np.int32)
+        bt = np.ascontiguousarray(block_tables, dtype=np.int32).reshape(len(sl), -1)
+        qsl = np.ascontiguousarray(query_start_loc, dtype=np.int32)
+        out = np.full((Tq, Hq, D), np.nan, dtype=np.float64)
+        sel = None
+        if row_select is not None:
+            sel = np.ascontiguousarray(row_select, dtype=np.uint8)
+            assert sel.shape == (Tq,)
+        rc = self.lib.oracle_paged_attention_prefill_chunk_kv(
+            _ptr(out), _ptr(np.ascontiguousarray(query)), q_dtype, _ptr(key_cache), _ptr(value_cache), kv_dtype,
+            float(k_scale), float(v_scale), _ptr(bt), _ptr(sl), _ptr(qsl), len(sl), float(scale), Hq, Hkv, D, B,
+            bt.shape[1], NB, _ptr(sel) if sel is not None else None)
+        _check(rc, "paged_attention_prefill_chunk_kv")
         return out
 
 

@@ -35,23 +35,81 @@
  * (max subtraction only guards exp() against overflow; it does not change the
  * mathematical value).
  *
- * Element types: 0 = fp32, 1 = fp16 (IEEE binary16), 2 = bf16.  Every stored
- * element is converted exactly to double before any arithmetic.
+ * Element types: 0 = fp32, 1 = fp16 (IEEE binary16), 2 = bf16, 3 = FP8 E4M3
+ * (cache pools only).  Every stored element is converted exactly to double
+ * before any arithmetic.
+ *
+ * FP8 KV cache.  Both pages list FP8 (E4M3) among vLLM's quantisation modes
+ * (case-study page, section 五 "量化支持", table row "FP8 (E4M3)"; guide page,
+ * "量化": 8 bits, half the memory of FP16, close to lossless, native on Hopper)
+ * but only for weights and activations and without a scaling rule.  Reading
+ * used here for the cache: one scale per pool (k_scale, v_scale); a stored
+ * code is the E4M3 value nearest to x / scale (ties to even, magnitudes above
+ * the largest finite value 448 clamped to 448, NaN kept NaN); the value a
+ * code stands for is scale * e4m3(code).  E4M3 itself is the OCP 8-bit
+ * floating-point format: 1 sign bit, 4 exponent bits with bias 7, 3 mantissa
+ * bits, subnormals at exponent field 0, no infinities, and the single NaN
+ * pattern S.1111.111 per sign.
  */
 #include <math.h>
 #include <stdint.h>
 #include <stdlib.h>
 #include <string.h>
 
-enum { ORC_F32 = 0, ORC_F16 = 1, ORC_BF16 = 2 };
+enum { ORC_F32 = 0, ORC_F16 = 1, ORC_BF16 = 2, ORC_E4M3 = 3 };
 
 static int elem_bytes(int dtype) {
     switch (dtype) {
         case ORC_F32: return 4;
         case ORC_F16: return 2;
         case ORC_BF16: return 2;
+        case ORC_E4M3: return 1;
         default: return 0;
     }
+}
+
+/* E4M3 code -> double, by the format's definition (exact). */
+static double e4m3_bits_to_double(uint8_t c) {
+    int sign = (c >> 7) & 1;
+    int expo = (c >> 3) & 0xf;
+    int mant = c & 0x7;
+    double v;
+    if (expo == 15 && mant == 7) {
+        v = NAN;
+    } else if (expo == 0) {
+        v = ldexp((double)mant, -9);                /* 0.mant * 2^(1-7) = mant/8 * 2^-6 */
+    } else {
+        v = ldexp((double)(8 + mant), expo - 10);   /* 1.mant * 2^(e-7) */
+    }
+    return sign ? -v : v;
+}
+
+/* double -> E4M3 code: the nearest of the 127 non-negative finite values to
+ * |x| (found by trying them all), ties to the even code (adjacent values have
+ * adjacent codes, so this is ties-to-even-mantissa); magnitudes above 448 thus
+ * go to 448, infinities included; the sign bit is the sign of x (so -0 and
+ * negative values that round to zero give 0x80); NaN gives 0x7F. */
+static uint8_t double_to_e4m3(double x) {
+    if (isnan(x)) return 0x7F;
+    uint8_t sign = signbit(x) ? 0x80 : 0x00;
+    double a = fabs(x);
+    int best = 0;
+    double best_err = INFINITY;
+    for (int c = 0; c <= 0x7E; ++c) {
+        double err = fabs(e4m3_bits_to_double((uint8_t)c) - a);
+        if (err < best_err || (err == best_err && (c & 1) == 0)) {
+            best = c;
+            best_err = err;
+        }
+    }
+    return (uint8_t)(sign | best);
+}
+
+/* Exposed for the pins: codes of n doubles. */
+int oracle_e4m3_encode(uint8_t* dst, const double* src, int64_t n) {
+    if (n < 0) return -1;
+    for (int64_t i = 0; i < n; ++i) dst[i] = double_to_e4m3(src[i]);
+    return 0;
 }
 
 /* IEEE binary16 -> double, exact (every binary16 value is a double). */
@@ -84,6 +142,7 @@ static double load_elem(const void* base, int64_t idx, int dtype) {
         memcpy(&f, (const char*)base + idx * 4, 4);
         return (double)f;
     }
+    if (dtype == ORC_E4M3) return e4m3_bits_to_double(((const uint8_t*)base)[idx]);
     uint16_t h;
     memcpy(&h, (const char*)base + idx * 2, 2);
     return dtype == ORC_F16 ? half_bits_to_double(h) : bf16_bits_to_double(h);
@@ -153,6 +212,36 @@ int oracle_reshape_and_cache(const void* key, const void* value, void* key_cache
 }
 
 /* ---------------------------------------------------------------------------
+ * reshape_and_cache into FP8 pools: as above, but each element x of token t's
+ * K (V) row is stored as the E4M3 code of x / k_scale (x / v_scale); the
+ * quotient is formed in double.  key/value are in src_dtype (fp32/fp16/bf16),
+ * the pools hold one byte per element.
+ * ------------------------------------------------------------------------- */
+int oracle_reshape_and_cache_fp8(const void* key, const void* value, uint8_t* key_cache, uint8_t* value_cache,
+                                 const int64_t* slot_mapping, int64_t num_tokens, int num_kv_heads,
+                                 int head_dim, int block_size, int64_t num_blocks, int src_dtype,
+                                 double k_scale, double v_scale) {
+    if (src_dtype == ORC_E4M3 || !elem_bytes(src_dtype) || !(k_scale > 0.0) || !(v_scale > 0.0)) return -1;
+    int64_t row_elems = (int64_t)num_kv_heads * head_dim;
+    for (int64_t t = 0; t < num_tokens; ++t) {
+        int64_t slot = slot_mapping[t];
+        if (slot < 0) continue;
+        if (slot >= num_blocks * block_size) return -1;
+        int64_t block = slot / block_size;
+        int64_t offset = slot % block_size;
+        for (int h = 0; h < num_kv_heads; ++h) {
+            for (int d = 0; d < head_dim; ++d) {
+                int64_t src = t * row_elems + (int64_t)h * head_dim + d;
+                int64_t dst = ((block * block_size + offset) * num_kv_heads + h) * (int64_t)head_dim + d;
+                key_cache[dst] = double_to_e4m3(load_elem(key, src, src_dtype) / k_scale);
+                value_cache[dst] = double_to_e4m3(load_elem(value, src, src_dtype) / v_scale);
+            }
+        }
+    }
+    return 0;
+}
+
+/* ---------------------------------------------------------------------------
  * copy_blocks (copy-on-write of a shared block): for every pair (src, dst)
  * in order, and for every layer's K and V pool, copy the whole physical block
  * src (block_bytes bytes) over block dst.  Returns -1 on an id outside the
@@ -176,10 +265,13 @@ int oracle_copy_blocks(void* const* key_caches, void* const* value_caches, int n
 }
 
 /* Gather positions [0, n) of one sequence's KV head g into contiguous
- * K[n][head_dim], V[n][head_dim] (double), following the block table. */
+ * K[n][head_dim], V[n][head_dim] (double), following the block table; each
+ * element is its stored value times the pool's scale (1 for 16/32-bit
+ * pools, which is exact). */
 static int gather_sequence(double* Kc, double* Vc, const void* key_cache, const void* value_cache,
-                           int dtype, const int32_t* bt_row, int64_t n, int g, int num_kv_heads,
-                           int head_dim, int block_size, int max_blocks_per_seq, int64_t num_blocks) {
+                           int dtype, double k_scale, double v_scale, const int32_t* bt_row, int64_t n, int g,
+                           int num_kv_heads, int head_dim, int block_size, int max_blocks_per_seq,
+                           int64_t num_blocks) {
     for (int64_t j = 0; j < n; ++j) {
         int64_t logical_block = j / block_size;
         int64_t offset = j % block_size;
@@ -188,8 +280,8 @@ static int gather_sequence(double* Kc, double* Vc, const void* key_cache, const 
         if (physical < 0 || physical >= num_blocks) return -1;
         int64_t row = ((physical * block_size + offset) * num_kv_heads + g) * (int64_t)head_dim;
         for (int d = 0; d < head_dim; ++d) {
-            Kc[j * head_dim + d] = load_elem(key_cache, row + d, dtype);
-            Vc[j * head_dim + d] = load_elem(value_cache, row + d, dtype);
+            Kc[j * head_dim + d] = k_scale * load_elem(key_cache, row + d, dtype);
+            Vc[j * head_dim + d] = v_scale * load_elem(value_cache, row + d, dtype);
         }
     }
     return 0;
@@ -223,16 +315,17 @@ static void attend(double* o, const double* q, const double* Kc, const double* V
  * Decode: one query token per sequence.  out[s][h][:] for query head h uses
  * KV head h / (num_q_heads / num_kv_heads) and attends over positions
  * j < context_lens[s] read through block_tables[s][:].
- * query [num_seqs, num_q_heads, head_dim] in dtype; out double, same shape.
+ * query [num_seqs, num_q_heads, head_dim] in q_dtype; pools in kv_dtype with
+ * scales k_scale / v_scale (see gather_sequence); out double, query's shape.
  * Returns 0, or -1 on a malformed argument / table entry.
  * ------------------------------------------------------------------------- */
-int oracle_paged_attention_decode(double* out, const void* query, const void* key_cache,
-                                  const void* value_cache, int dtype, const int32_t* block_tables,
-                                  const int32_t* context_lens, double scale, int64_t num_seqs,
-                                  int num_q_heads, int num_kv_heads, int head_dim, int block_size,
-                                  int max_blocks_per_seq, int64_t num_blocks) {
-    if (!elem_bytes(dtype) || num_kv_heads <= 0 || num_q_heads % num_kv_heads != 0 || head_dim <= 0 ||
-        block_size <= 0)
+int oracle_paged_attention_decode_kv(double* out, const void* query, int q_dtype, const void* key_cache,
+                                     const void* value_cache, int kv_dtype, double k_scale, double v_scale,
+                                     const int32_t* block_tables, const int32_t* context_lens, double scale,
+                                     int64_t num_seqs, int num_q_heads, int num_kv_heads, int head_dim,
+                                     int block_size, int max_blocks_per_seq, int64_t num_blocks) {
+    if (!elem_bytes(q_dtype) || q_dtype == ORC_E4M3 || !elem_bytes(kv_dtype) || num_kv_heads <= 0 ||
+        num_q_heads % num_kv_heads != 0 || head_dim <= 0 || block_size <= 0)
         return -1;
     int group = num_q_heads / num_kv_heads;
     int rc = 0;
@@ -249,19 +342,31 @@ int oracle_paged_attention_decode(double* out, const void* query, const void* ke
             return -1;
         }
         for (int g = 0; g < num_kv_heads && rc == 0; ++g) {
-            rc = gather_sequence(Kc, Vc, key_cache, value_cache, dtype,
+            rc = gather_sequence(Kc, Vc, key_cache, value_cache, kv_dtype, k_scale, v_scale,
                                  block_tables + s * max_blocks_per_seq, n, g, num_kv_heads, head_dim,
                                  block_size, max_blocks_per_seq, num_blocks);
             for (int hh = 0; hh < group && rc == 0; ++hh) {
                 int h = g * group + hh;
                 for (int d = 0; d < head_dim; ++d)
-                    qv[d] = load_elem(query, (s * num_q_heads + h) * (int64_t)head_dim + d, dtype);
+                    qv[d] = load_elem(query, (s * num_q_heads + h) * (int64_t)head_dim + d, q_dtype);
                 attend(out + (s * num_q_heads + h) * (int64_t)head_dim, qv, Kc, Vc, n, head_dim, scale, x);
             }
         }
         free(Kc); free(Vc); free(x); free(qv);
     }
     return rc;
+}
+
+/* Decode with query and pools of one type (no scaling). */
+int oracle_paged_attention_decode(double* out, const void* query, const void* key_cache,
+                                  const void* value_cache, int dtype, const int32_t* block_tables,
+                                  const int32_t* context_lens, double scale, int64_t num_seqs,
+                                  int num_q_heads, int num_kv_heads, int head_dim, int block_size,
+                                  int max_blocks_per_seq, int64_t num_blocks) {
+    if (dtype == ORC_E4M3) return -1;
+    return oracle_paged_attention_decode_kv(out, query, dtype, key_cache, value_cache, dtype, 1.0, 1.0,
+                                            block_tables, context_lens, scale, num_seqs, num_q_heads,
+                                            num_kv_heads, head_dim, block_size, max_blocks_per_seq, num_blocks);
 }
 
 /* ---------------------------------------------------------------------------
@@ -275,14 +380,14 @@ int oracle_paged_attention_decode(double* out, const void* query, const void* ke
  * row_select (may be NULL = all rows) lets a caller evaluate a sample of rows;
  * unselected output rows are left untouched.
  * ------------------------------------------------------------------------- */
-int oracle_paged_attention_prefill_chunk(double* out, const void* query, const void* key_cache,
-                                         const void* value_cache, int dtype, const int32_t* block_tables,
-                                         const int32_t* seq_lens, const int32_t* query_start_loc,
-                                         int num_chunks, double scale, int num_q_heads, int num_kv_heads,
-                                         int head_dim, int block_size, int max_blocks_per_seq,
-                                         int64_t num_blocks, const uint8_t* row_select) {
-    if (!elem_bytes(dtype) || num_kv_heads <= 0 || num_q_heads % num_kv_heads != 0 || head_dim <= 0 ||
-        block_size <= 0)
+int oracle_paged_attention_prefill_chunk_kv(double* out, const void* query, int q_dtype, const void* key_cache,
+                                            const void* value_cache, int kv_dtype, double k_scale, double v_scale,
+                                            const int32_t* block_tables, const int32_t* seq_lens,
+                                            const int32_t* query_start_loc, int num_chunks, double scale,
+                                            int num_q_heads, int num_kv_heads, int head_dim, int block_size,
+                                            int max_blocks_per_seq, int64_t num_blocks, const uint8_t* row_select) {
+    if (!elem_bytes(q_dtype) || q_dtype == ORC_E4M3 || !elem_bytes(kv_dtype) || num_kv_heads <= 0 ||
+        num_q_heads % num_kv_heads != 0 || head_dim <= 0 || block_size <= 0)
         return -1;
     int group = num_q_heads / num_kv_heads;
     int rc = 0;
@@ -302,7 +407,7 @@ int oracle_paged_attention_prefill_chunk(double* out, const void* query, const v
             return -1;
         }
         for (int g = 0; g < num_kv_heads && rc == 0; ++g) {
-            rc = gather_sequence(Kc, Vc, key_cache, value_cache, dtype,
+            rc = gather_sequence(Kc, Vc, key_cache, value_cache, kv_dtype, k_scale, v_scale,
                                  block_tables + (int64_t)r * max_blocks_per_seq, len, g, num_kv_heads,
                                  head_dim, block_size, max_blocks_per_seq, num_blocks);
             for (int64_t i = 0; i < nq && rc == 0; ++i) {
@@ -311,7 +416,7 @@ int oracle_paged_attention_prefill_chunk(double* out, const void* query, const v
                 for (int hh = 0; hh < group; ++hh) {
                     int h = g * group + hh;
                     for (int d = 0; d < head_dim; ++d)
-                        qv[d] = load_elem(query, (row * num_q_heads + h) * (int64_t)head_dim + d, dtype);
+                        qv[d] = load_elem(query, (row * num_q_heads + h) * (int64_t)head_dim + d, q_dtype);
                     /* causal key set: positions 0 .. c0 + i inclusive */
                     attend(out + (row * num_q_heads + h) * (int64_t)head_dim, qv, Kc, Vc, c0 + i + 1,
                            head_dim, scale, x);
@@ -321,4 +426,18 @@ int oracle_paged_attention_prefill_chunk(double* out, const void* query, const v
         free(Kc); free(Vc); free(x); free(qv);
     }
     return rc;
+}
+
+/* Prefill with query and pools of one type (no scaling). */
+int oracle_paged_attention_prefill_chunk(double* out, const void* query, const void* key_cache,
+                                         const void* value_cache, int dtype, const int32_t* block_tables,
+                                         const int32_t* seq_lens, const int32_t* query_start_loc,
+                                         int num_chunks, double scale, int num_q_heads, int num_kv_heads,
+                                         int head_dim, int block_size, int max_blocks_per_seq,
+                                         int64_t num_blocks, const uint8_t* row_select) {
+    if (dtype == ORC_E4M3) return -1;
+    return oracle_paged_attention_prefill_chunk_kv(out, query, dtype, key_cache, value_cache, dtype, 1.0, 1.0,
+                                                   block_tables, seq_lens, query_start_loc, num_chunks, scale,
+                                                   num_q_heads, num_kv_heads, head_dim, block_size,
+                                                   max_blocks_per_seq, num_blocks, row_select);
 }

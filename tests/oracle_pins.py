@@ -310,4 +310,159 @@ def pin_index_examples(orc: oracle.Oracle):
     assert (slot // h["block_size"], slot % h["block_size"]) == (h["logical_block"], h["offset"])
 
 
+# ---------------------------------------------------------------------------
+# FP8 (E4M3) pools
+# ---------------------------------------------------------------------------
+
+def _torch_e4m3_values(codes: np.ndarray) -> np.ndarray:
+    return torch.from_numpy(codes.astype(np.uint8)).view(torch.float8_e4m3fn).to(torch.float64).numpy()
+
+
+def _torch_e4m3_codes(x32: np.ndarray) -> np.ndarray:
+    """torch's float32 -> float8_e4m3fn cast (round to nearest even; only used for |x| <= 448)."""
+    return torch.from_numpy(np.ascontiguousarray(x32, dtype=np.float32)).to(torch.float8_e4m3fn).view(
+        torch.uint8).numpy()
+
+
+def pin_e4m3_decodes_like_torch(orc: oracle.Oracle):
+    """Every one of the 256 codes decodes to torch's float8_e4m3fn value (NaN where torch has NaN)."""
+    codes = np.arange(256, dtype=np.uint8)
+    got = orc.to_double(codes, oracle.E4M3)
+    ref = _torch_e4m3_values(codes)
+    assert np.array_equal(np.isnan(got), np.isnan(ref))
+    ok = ~np.isnan(ref)
+    assert np.array_equal(got[ok], ref[ok])
+    assert np.array_equal(np.signbit(got[ok]), np.signbit(ref[ok]))
+
+
+def pin_e4m3_closed_forms(orc: oracle.Oracle):
+    """Values fixed by the format: bias 7, 3 mantissa bits, subnormals, 448 max, S.1111.111 NaN."""
+    want = {0x38: 1.0, 0x39: 1.125, 0x40: 2.0, 0x7E: 448.0, 0x08: 2.0 ** -6, 0x07: 7 * 2.0 ** -9,
+            0x01: 2.0 ** -9, 0x00: 0.0, 0xB8: -1.0, 0xFE: -448.0, 0x30: 0.5, 0x77: 240.0}
+    codes = np.array(list(want), dtype=np.uint8)
+    got = orc.to_double(codes, oracle.E4M3)
+    np.testing.assert_array_equal(got, np.array(list(want.values())))
+    nan = orc.to_double(np.array([0x7F, 0xFF], dtype=np.uint8), oracle.E4M3)
+    assert np.isnan(nan).all()
+    neg0 = orc.to_double(np.array([0x80], dtype=np.uint8), oracle.E4M3)
+    assert neg0[0] == 0.0 and np.signbit(neg0[0])
+
+
+def pin_e4m3_encode_rounding(orc: oracle.Oracle):
+    """Encoding: every finite code round-trips; in range it equals torch's round-to-nearest-even cast;
+    exact midpoints go to the even code; beyond 448 it saturates; the sign survives rounding to zero."""
+    codes = np.arange(256, dtype=np.uint8)
+    vals = orc.to_double(codes, oracle.E4M3)
+    fin = ~np.isnan(vals)
+    back = orc.e4m3_encode(vals[fin])
+    assert np.array_equal(back, codes[fin])
+    # every finite fp16 value within range, and random fp32 values
+    h = np.arange(1 << 16, dtype=np.uint16).view(np.float16).astype(np.float32)
+    h = h[np.isfinite(h) & (np.abs(h) <= 448)]
+    r = (np.random.default_rng(31).standard_normal(20000) * np.exp2(np.random.default_rng(32).integers(
+        -12, 9, 20000))).astype(np.float32)
+    r = r[np.abs(r) <= 448]
+    for x in (h, r):
+        assert np.array_equal(orc.e4m3_encode(x.astype(np.float64)), _torch_e4m3_codes(x))
+    # midpoints of adjacent non-negative codes: ties to the even code
+    pos = vals[:0x7F]
+    mids = (pos[:-1] + pos[1:]) / 2
+    got = orc.e4m3_encode(mids)
+    lo = np.arange(0x7E, dtype=np.uint8)
+    want = np.where(lo % 2 == 0, lo, lo + 1).astype(np.uint8)
+    assert np.array_equal(got, want)
+    assert orc.e4m3_encode(np.array([1.0625]))[0] == 0x38 and orc.e4m3_encode(np.array([1.1875]))[0] == 0x3A
+    sat = orc.e4m3_encode(np.array([448.0, 449.0, 464.0, 1e30, np.inf, -500.0, -np.inf]))
+    assert list(sat) == [0x7E, 0x7E, 0x7E, 0x7E, 0x7E, 0xFE, 0xFE]
+    special = orc.e4m3_encode(np.array([np.nan, -0.0, -1e-9, 1e-9, 2.0 ** -10, 2.0 ** -10 * 1.0001]))
+    assert list(special) == [0x7F, 0x80, 0x80, 0x00, 0x00, 0x01]
+
+
+def pin_fp8_reshape_quantises_each_element(orc: oracle.Oracle):
+    """FP8 append: slot t gets the codes of key[t] / k_scale (value / v_scale); -1 skipped; nothing else moves.
+    Power-of-two scales keep x / scale exact in fp32, so torch's cast gives the expected codes."""
+    rng = np.random.default_rng(33)
+    NB, B, Hkv, D, T = 6, 4, 2, 16, 7
+    kc = rng.integers(0, 256, (NB, B, Hkv, D), dtype=np.uint8)
+    vc = rng.integers(0, 256, (NB, B, Hkv, D), dtype=np.uint8)
+    k = (rng.standard_normal((T, Hkv, D)) * 3).astype(np.float16)
+    v = (rng.standard_normal((T, Hkv, D)) * 300).astype(np.float16)   # some beyond 448 * v_scale
+    k_scale, v_scale = 2.0 ** -4, 0.5
+    slots = rng.choice(NB * B, size=T, replace=False).astype(np.int64)
+    slots[3] = -1
+    ek, ev = kc.copy(), vc.copy()
+    ok = slots >= 0
+    qk = np.clip(k.astype(np.float32) / np.float32(k_scale), -448, 448)
+    qv = np.clip(v.astype(np.float32) / np.float32(v_scale), -448, 448)
+    ek.reshape(NB * B, Hkv, D)[slots[ok]] = _torch_e4m3_codes(qk[ok])
+    ev.reshape(NB * B, Hkv, D)[slots[ok]] = _torch_e4m3_codes(qv[ok])
+    orc.reshape_and_cache_fp8(k, v, kc, vc, slots, oracle.F16, k_scale, v_scale)
+    assert np.array_equal(kc, ek)
+    assert np.array_equal(vc, ev)
+
+
+def _fp8_case(rng, lens, Hq, Hkv, D, B, extra_blocks=2):
+    """Random codes in randomly placed pools (no NaN codes in used slots)."""
+    S = len(lens)
+    need = [(n + B - 1) // B for n in lens]
+    nb = sum(need) + extra_blocks
+    kc = rng.integers(0, 0x7F, (nb, B, Hkv, D), dtype=np.uint8) | (rng.integers(0, 2, (nb, B, Hkv, D),
+                                                                               dtype=np.uint8) << 7)
+    vc = rng.integers(0, 0x7F, (nb, B, Hkv, D), dtype=np.uint8) | (rng.integers(0, 2, (nb, B, Hkv, D),
+                                                                               dtype=np.uint8) << 7)
+    perm = rng.permutation(nb)
+    bt = np.full((S, max(need)), -1, dtype=np.int32)
+    k = 0
+    for s, m in enumerate(need):
+        bt[s, :m] = perm[k:k + m]
+        k += m
+    return kc.astype(np.uint8), vc.astype(np.uint8), bt
+
+
+def _dense(cache, bt, s, n, B):
+    rows = [cache[bt[s, j // B], j % B] for j in range(n)]  # [n, Hkv, D]
+    return np.stack(rows)
+
+
+def pin_fp8_decode_matches_sdpa_on_dequantised(orc: oracle.Oracle):
+    """Decode over E4M3 pools == SDPA over k_scale * torch(codes), v_scale * torch(codes)."""
+    rng = np.random.default_rng(34)
+    lens = [1, 9, 20]
+    Hq, Hkv, D, B = 4, 2, 8, 4
+    kc, vc, bt = _fp8_case(rng, lens, Hq, Hkv, D, B)
+    q = rng.standard_normal((len(lens), Hq, D)).astype(np.float32)
+    k_scale, v_scale, scale = 0.013, 2.5, 0.4
+    out = orc.paged_attention_decode_kv(q, oracle.F32, kc, vc, oracle.E4M3, k_scale, v_scale, bt, np.array(lens),
+                                        scale)
+    G = Hq // Hkv
+    for s, n in enumerate(lens):
+        k = k_scale * _torch_e4m3_values(_dense(kc, bt, s, n, B))
+        v = v_scale * _torch_e4m3_values(_dense(vc, bt, s, n, B))
+        k = np.repeat(k.transpose(1, 0, 2), G, axis=0)
+        v = np.repeat(v.transpose(1, 0, 2), G, axis=0)
+        ref = sdpa_reference(q[s][:, None, :], k, v, scale)[:, 0, :]
+        np.testing.assert_allclose(out[s], ref, rtol=0, atol=1e-12 * max(1.0, np.abs(ref).max()))
+
+
+def pin_fp8_prefill_matches_masked_sdpa(orc: oracle.Oracle):
+    """Chunked prefill over E4M3 pools == causal SDPA over the dequantised K/V."""
+    rng = np.random.default_rng(35)
+    c0s, ns = [3, 0], [5, 7]
+    lens = [c + n for c, n in zip(c0s, ns)]
+    Hq, Hkv, D, B = 4, 4, 8, 4
+    kc, vc, bt = _fp8_case(rng, lens, Hq, Hkv, D, B)
+    qsl = np.concatenate([[0], np.cumsum(ns)]).astype(np.int32)
+    q = rng.standard_normal((int(qsl[-1]), Hq, D)).astype(np.float16)
+    k_scale, v_scale, scale = 0.02, 0.7, 0.3
+    out = orc.paged_attention_prefill_chunk_kv(q, oracle.F16, kc, vc, oracle.E4M3, k_scale, v_scale, bt,
+                                               np.array(lens), qsl, scale)
+    for r, (c0, n) in enumerate(zip(c0s, ns)):
+        L = c0 + n
+        k = (k_scale * _torch_e4m3_values(_dense(kc, bt, r, L, B))).transpose(1, 0, 2)
+        v = (v_scale * _torch_e4m3_values(_dense(vc, bt, r, L, B))).transpose(1, 0, 2)
+        mask = np.arange(L)[None, :] <= (c0 + np.arange(n))[:, None]
+        ref = sdpa_reference(q[qsl[r]:qsl[r + 1]].astype(np.float64).transpose(1, 0, 2), k, v, scale, mask)
+        np.testing.assert_allclose(out[qsl[r]:qsl[r + 1]], ref.transpose(1, 0, 2), rtol=0, atol=1e-12)
+
+
 ALL_PINS = [v for k, v in sorted(globals().items()) if k.startswith("pin_")]
