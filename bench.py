@@ -67,13 +67,14 @@ class DecodeStep:
         self.layers = layers_per_step or w.num_layers
         self.outs = [torch.empty_like(q) for q in w.queries]
         self.part = pkv.decode_partition_size(w.num_seqs, w.num_kv_heads, w.head_dim, w.block_size,
-                                              w.max_context_len, w.dtype,
+                                              w.max_context_len, 3 if w.fp8 else w.dtype,
                                               int(w.context_lens.astype(np.int64).sum()))
         need = pkv.decode_workspace_size(w.num_seqs, w.num_q_heads, w.head_dim, w.max_context_len, self.part)
         self.ws = torch.empty(max(need, 16), dtype=torch.uint8, device=dev)
         self.parts = -(-w.max_context_len // self.part) if self.part else 1
         t = w.queries[0].element_size()
-        self.kv_bytes = 2 * int(w.context_lens.astype(np.int64).sum()) * w.num_kv_heads * w.head_dim * t
+        tkv = w.key_caches[0].element_size()
+        self.kv_bytes = 2 * int(w.context_lens.astype(np.int64).sum()) * w.num_kv_heads * w.head_dim * tkv
         nblocks = int(((w.context_lens.astype(np.int64) + w.block_size - 1) // w.block_size).sum())
         # algorithmic bytes of one decode call: K/V once, q, out, block ids, lengths
         self.decode_bytes = self.kv_bytes + 2 * w.queries[0].numel() * t + 4 * nblocks + 4 * w.num_seqs
@@ -95,13 +96,22 @@ class DecodeStep:
 
     def append(self, l):
         w = self.w
-        self.pkv.reshape_and_cache(w.new_keys[l], w.new_values[l], w.key_caches[l], w.value_caches[l], self.sm)
+        if w.fp8:
+            self.pkv.reshape_and_cache_fp8(w.new_keys[l], w.new_values[l], w.key_caches[l], w.value_caches[l],
+                                           self.sm, w.extra["k_scale"], w.extra["v_scale"])
+        else:
+            self.pkv.reshape_and_cache(w.new_keys[l], w.new_values[l], w.key_caches[l], w.value_caches[l], self.sm)
 
     def attend(self, l):
         w = self.w
-        self.pkv.paged_attention_decode(self.outs[l], w.queries[l], w.key_caches[l], w.value_caches[l], self.bt,
-                                        self.cl, w.scale, w.max_context_len, partition_size=self.part,
-                                        workspace=self.ws)
+        if w.fp8:
+            self.pkv.paged_attention_decode_fp8(self.outs[l], w.queries[l], w.key_caches[l], w.value_caches[l],
+                                                self.bt, self.cl, w.scale, w.extra["k_scale"], w.extra["v_scale"],
+                                                w.max_context_len, partition_size=self.part, workspace=self.ws)
+        else:
+            self.pkv.paged_attention_decode(self.outs[l], w.queries[l], w.key_caches[l], w.value_caches[l], self.bt,
+                                            self.cl, w.scale, w.max_context_len, partition_size=self.part,
+                                            workspace=self.ws)
 
     def run(self, timer=None, step=0):
         for i in range(self.layers):
@@ -246,6 +256,17 @@ def make_step(name, device, rank, seqs=None, layers=None):
     if name == "llama7b_decode_f16":
         w = workloads.llama7b_decode_f16(device=device, seed=1002 + rank, num_seqs=seqs or 64)
         return DecodeStep(w), "llama7b_decode_f16" + (f" ({seqs} sequences)" if seqs else "")
+    if name == "llama7b_decode_fp8":
+        w = workloads.llama7b_decode_fp8(device=device, seed=1002 + rank, num_seqs=seqs or 64)
+        return DecodeStep(w), "llama7b_decode_fp8" + (f" ({seqs} sequences)" if seqs else "")
+    if name == "gqa70b_decode_fp8":
+        free, _ = torch.cuda.mem_get_info()
+        per_layer = 0.9e9 * (seqs or 256) / 256  # FP8 pools of one layer (~0.81 GB at 256 sequences) plus headroom
+        fit = int(max(1, min(80, (free - 8e9) // per_layer)))
+        layers = min(fit, layers) if layers else fit
+        w = workloads.gqa70b_decode_fp8(device=device, num_layers=layers, seed=1003 + rank, num_seqs=seqs or 256)
+        note = "" if layers == 80 else f", {layers} distinct layer pools cycled"
+        return DecodeStep(w, layers_per_step=80), f"gqa70b_decode_fp8 (80 layers per step{note})"
     if name == "tiny_decode_f32":
         return DecodeStep(workloads.tiny_decode_f32(device=device)), name
     if name == "gqa70b_decode_bf16":
@@ -419,14 +440,19 @@ def oracle_sample(step, budget_s, max_seqs=None):
     remap = {int(b): i for i, b in enumerate(used)}
     slots = np.array([remap[int(s) // B] * B + int(s) % B for s in w.slot_mapping[seqs]], dtype=np.int64)
     idx = torch.from_numpy(seqs).to(w.queries[0].device)
-    q = oracle.storage(w.queries[0][idx])[0]
+    q, qcode = oracle.storage(w.queries[0][idx])
     nk = oracle.storage(w.new_keys[0][idx])[0]
     nv = oracle.storage(w.new_values[0][idx])[0]
     lens = w.context_lens[seqs]
     done, t0 = 0, time.perf_counter()
     while True:
-        orc.reshape_and_cache(nk, nv, kn, vn, slots, code)
-        orc.paged_attention_decode(q, kn, vn, bt, lens, w.scale, code)
+        if w.fp8:
+            ks, vs = w.extra["k_scale"], w.extra["v_scale"]
+            orc.reshape_and_cache_fp8(nk, nv, kn, vn, slots, qcode, ks, vs)
+            orc.paged_attention_decode_kv(q, qcode, kn, vn, oracle.E4M3, ks, vs, bt, lens, w.scale)
+        else:
+            orc.reshape_and_cache(nk, nv, kn, vn, slots, code)
+            orc.paged_attention_decode(q, kn, vn, bt, lens, w.scale, code)
         done += 1
         el = time.perf_counter() - t0
         if el >= budget_s:
@@ -618,7 +644,9 @@ def main():
     line = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": ws, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": {torch.float16: "f16", torch.bfloat16: "bf16", torch.float32: "f32"}[w.dtype],
+        "vs_baseline": None,
+        "dtype": {torch.float16: "f16", torch.bfloat16: "bf16", torch.float32: "f32"}[w.dtype] + (
+            " (e4m3 KV pools)" if getattr(w, "fp8", False) else ""),
         "data": "synthetic",
         "config": {"workload": cname, "num_seqs": w.num_seqs, "num_q_heads": w.num_q_heads,
                    "num_kv_heads": w.num_kv_heads, "head_dim": w.head_dim, "block_size": w.block_size,
@@ -644,7 +672,7 @@ def main():
         v, done, what, el = step.oracle_sample(args.cpu_budget)
         line["cpu_baseline"] = {"value": v, "unit": "tokens/s", "cores": 1, "kind": "oracle",
                                 "sample": f"{done} x (append + causal attention of {what}), {el:.1f} s, 1 thread"}
-    elif rank == 0 and ws == 1 and args.cpu_budget > 0 and args.config != "gqa70b_decode_bf16":
+    elif rank == 0 and ws == 1 and args.cpu_budget > 0 and not args.config.startswith("gqa70b"):
         v, done, n, el = oracle_sample(step, args.cpu_budget, max_seqs=None if w.num_seqs <= 64 else 16)
         line["cpu_baseline"] = {"value": v, "unit": "tokens/s", "cores": 1, "kind": "oracle",
                                 "sample": f"{done} x (append + decode of {n} sequences), {el:.1f} s, 1 thread"}

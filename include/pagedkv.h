@@ -46,7 +46,10 @@ extern "C" {
 
 typedef void* pkv_stream_t; /* a cudaStream_t */
 
-typedef enum { PKV_F32 = 0, PKV_F16 = 1, PKV_BF16 = 2 } pkv_dtype;
+/* Element types.  PKV_FP8_E4M3 is a pool type only (one byte per element,
+ * the OCP 8-bit float E4M3: bias 7, 3 mantissa bits, max 448, no
+ * infinities); queries and outputs are F32, F16 or BF16. */
+typedef enum { PKV_F32 = 0, PKV_F16 = 1, PKV_BF16 = 2, PKV_FP8_E4M3 = 3 } pkv_dtype;
 
 typedef enum {
     PKV_OK = 0,
@@ -83,13 +86,38 @@ const char* pkv_last_cuda_error(void);
  *   slot_mapping    device int64 [num_tokens]; slot_mapping[t] < 0 marks a
  *                   padding token that is skipped; a slot >= num_blocks *
  *                   block_size is skipped and sets PKV_DEVERR_SLOT.
- * Bits are copied verbatim (bit-exact).  Two tokens with the same slot race.
- * num_tokens == 0 is a no-op.
+ * Bits are copied verbatim (bit-exact); dtype may be any pkv_dtype (FP8
+ * codes that are already quantised are copied as bytes).  Two tokens with the
+ * same slot race.  num_tokens == 0 is a no-op.
  */
 int pkv_reshape_and_cache(const void* key, const void* value, void* key_cache, void* value_cache,
                           const int64_t* slot_mapping, int64_t num_tokens, int num_kv_heads,
                           int head_dim, int block_size, int64_t num_blocks, int dtype,
                           pkv_stream_t stream);
+
+/*
+ * reshape_and_cache_fp8 -- write new tokens' K and V into FP8 (E4M3) pools,
+ * quantising on the way.  The pages list FP8 E4M3 among vLLM's quantisation
+ * modes (case-study page, section 五 "量化支持"; guide page, "量化": half the
+ * memory of FP16, near lossless) without a rule for the KV cache; this library
+ * keeps one scale per pool.  Element x of a K row is stored as the E4M3 code
+ * nearest to the exact quotient x / k_scale (ties to even; magnitudes beyond
+ * 448 saturate to +-448; NaN is stored as 0x7F); V likewise with v_scale.
+ *
+ *   key, value      device, [num_tokens, num_kv_heads, head_dim] in src_dtype
+ *                   (F32, F16 or BF16)
+ *   key_cache,
+ *   value_cache     device, [num_blocks, block_size, num_kv_heads, head_dim],
+ *                   one byte per element
+ *   slot_mapping    as for pkv_reshape_and_cache
+ *   k_scale, v_scale  finite and > 0
+ * num_kv_heads * head_dim must be a multiple of 16.  The codes are bit-exact
+ * (correctly rounded).
+ */
+int pkv_reshape_and_cache_fp8(const void* key, const void* value, void* key_cache, void* value_cache,
+                              const int64_t* slot_mapping, int64_t num_tokens, int num_kv_heads, int head_dim,
+                              int block_size, int64_t num_blocks, int src_dtype, float k_scale, float v_scale,
+                              pkv_stream_t stream);
 
 /*
  * copy_blocks -- copy-on-write of shared blocks.  Source: case-study page
@@ -171,6 +199,30 @@ int pkv_paged_attention_decode(void* out, const void* query, const void* key_cac
                                int max_blocks_per_seq, int64_t num_blocks, int max_context_len,
                                int partition_size, int dtype, void* workspace,
                                size_t workspace_bytes, pkv_stream_t stream);
+
+/*
+ * Decode attention over FP8 (E4M3) pools written by pkv_reshape_and_cache_fp8:
+ * the same result as pkv_paged_attention_decode with every pool element read
+ * as k_scale * e4m3(code) (K) or v_scale * e4m3(code) (V).  The pools stream
+ * half the bytes of fp16 pools.  Both products run on warp tensor-core MMAs
+ * with f16 inputs (every E4M3 value is exact in f16; the query is rounded to
+ * f16, so |query| must stay below 65504) and fp32 accumulation.
+ *
+ *   query, out      device [num_seqs, num_q_heads, head_dim], dtype F16 or BF16
+ *   key_cache,
+ *   value_cache     device, one byte per element, layout as above
+ *   k_scale, v_scale  the pools' scales, finite and > 0
+ * Every other argument, the workspace (pkv_decode_workspace_size) and the
+ * error behaviour are those of pkv_paged_attention_decode.
+ * Supported: head_dim 128; block_size in {8, 16, 32}; num_q_heads /
+ * num_kv_heads in {1, 2, 4, 8}.
+ */
+int pkv_paged_attention_decode_fp8(void* out, const void* query, const void* key_cache, const void* value_cache,
+                                   const int32_t* block_tables, const int32_t* context_lens, float scale,
+                                   float k_scale, float v_scale, int num_seqs, int num_q_heads, int num_kv_heads,
+                                   int head_dim, int block_size, int max_blocks_per_seq, int64_t num_blocks,
+                                   int max_context_len, int partition_size, int dtype, void* workspace,
+                                   size_t workspace_bytes, pkv_stream_t stream);
 
 /* Workspace bytes pkv_paged_attention_decode needs for these sizes (0 when
  * partition_size == 0 or max_context_len <= partition_size). */

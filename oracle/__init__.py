@@ -47,7 +47,7 @@ def build(force: bool = False) -> str:
 
 
 def storage(t) -> tuple:
-    """(numpy storage array, dtype code) of a CPU torch tensor."""
+    """(numpy storage array, dtype code) of a CPU torch tensor (uint8 = E4M3 codes)."""
     import torch
     t = t.detach().cpu().contiguous()
     if t.dtype == torch.float32:
@@ -56,6 +56,8 @@ def storage(t) -> tuple:
         return t.numpy(), F16
     if t.dtype == torch.bfloat16:
         return t.view(torch.int16).numpy().view(np.uint16), BF16
+    if t.dtype in (torch.uint8, torch.float8_e4m3fn):   # pools of E4M3 codes
+        return t.view(torch.uint8).numpy(), E4M3
     raise TypeError(f"unsupported oracle dtype {t.dtype}")
 
 

@@ -14,7 +14,9 @@ from ._binding import (  # noqa: F401
     library_path,
     load_library,
     paged_attention_decode,
+    paged_attention_decode_fp8,
     paged_attention_prefill_chunk,
     reshape_and_cache,
+    reshape_and_cache_fp8,
     swap_blocks,
 )

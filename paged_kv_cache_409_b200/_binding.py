@@ -18,6 +18,8 @@ from .build import LIB
 _lib = None
 
 DTYPE_CODE = {torch.float32: 0, torch.float16: 1, torch.bfloat16: 2}
+FP8_E4M3 = 3
+FP8_POOL_DTYPES = (torch.uint8, torch.float8_e4m3fn)  # one E4M3 code per element
 
 DEVERR_BLOCK_ID = 0x1
 DEVERR_SLOT = 0x2
@@ -29,9 +31,12 @@ EXPORTED = (
     "pkv_status_string",
     "pkv_last_cuda_error",
     "pkv_reshape_and_cache",
+    "pkv_reshape_and_cache_fp8",
     "pkv_copy_blocks",
     "pkv_swap_blocks",
     "pkv_paged_attention_decode",
+    "pkv_paged_attention_decode_fp8",
+    "pkv_paged_attention_decode_static_scratch",
     "pkv_decode_workspace_size",
     "pkv_decode_partition_size",
     "pkv_paged_attention_prefill_chunk",
@@ -66,6 +71,9 @@ def load_library():
     lib.pkv_last_cuda_error.argtypes = []
     lib.pkv_last_cuda_error.restype = ctypes.c_char_p
     lib.pkv_reshape_and_cache.argtypes = [P, P, P, P, P, I64, I, I, I, I64, I, P]
+    lib.pkv_reshape_and_cache_fp8.argtypes = [P, P, P, P, P, I64, I, I, I, I64, I, F, F, P]
+    lib.pkv_paged_attention_decode_fp8.argtypes = [P, P, P, P, P, P, F, F, F, I, I, I, I, I, I, I64, I, I, I, P, SZ,
+                                                   P]
     lib.pkv_copy_blocks.argtypes = [P, P, I, P, I64, I64, I64, P]
     lib.pkv_swap_blocks.argtypes = [P, P, P, P, P, I64, I64, I64, I64, P]
     lib.pkv_paged_attention_decode.argtypes = [P, P, P, P, P, P, F, I, I, I, I, I, I, I64, I, I, I, P, SZ, P]
@@ -74,7 +82,8 @@ def load_library():
     lib.pkv_decode_partition_size.argtypes = [I, I, I, I, I, I64, I]
     lib.pkv_paged_attention_prefill_chunk.argtypes = [P, P, P, P, P, P, P, I, I64, I, F, I, I, I, I, I, I64, I, P]
     lib.pkv_get_device_error.argtypes = [ctypes.POINTER(ctypes.c_uint32), P]
-    for name in ("pkv_reshape_and_cache", "pkv_copy_blocks", "pkv_swap_blocks", "pkv_paged_attention_decode",
+    for name in ("pkv_reshape_and_cache", "pkv_reshape_and_cache_fp8", "pkv_paged_attention_decode_fp8",
+                 "pkv_copy_blocks", "pkv_swap_blocks", "pkv_paged_attention_decode",
                  "pkv_decode_partition_size", "pkv_paged_attention_prefill_chunk", "pkv_get_device_error"):
         getattr(lib, name).restype = I
     _lib = lib
@@ -120,6 +129,26 @@ def reshape_and_cache(key, value, key_cache, value_cache, slot_mapping, stream=N
                                    _dev(value_cache, "value_cache"), _dev(slot_mapping, "slot_mapping"), T, Hkv,
                                    D, B, NB, _code(key), _stream(stream))
     _ok(rc, "reshape_and_cache")
+
+
+def _fp8_pool(t: torch.Tensor, name: str) -> int:
+    if t.dtype not in FP8_POOL_DTYPES:
+        raise ValueError(f"{name} must be a uint8 or float8_e4m3fn pool of E4M3 codes")
+    return _dev(t, name)
+
+
+def reshape_and_cache_fp8(key, value, key_cache, value_cache, slot_mapping, k_scale, v_scale, stream=None):
+    """Quantise ``key``/``value`` ``[T, Hkv, D]`` (fp32/fp16/bf16) by ``1/k_scale``, ``1/v_scale`` into the
+    E4M3 pools' slots ``slot_mapping`` (int64, -1 = skip)."""
+    lib = load_library()
+    T, Hkv, D = key.shape
+    NB, B = key_cache.shape[:2]
+    if slot_mapping.dtype != torch.int64:
+        raise ValueError("slot_mapping must be int64")
+    rc = lib.pkv_reshape_and_cache_fp8(_dev(key, "key"), _dev(value, "value"), _fp8_pool(key_cache, "key_cache"),
+                                       _fp8_pool(value_cache, "value_cache"), _dev(slot_mapping, "slot_mapping"), T,
+                                       Hkv, D, B, NB, _code(key), float(k_scale), float(v_scale), _stream(stream))
+    _ok(rc, "reshape_and_cache_fp8")
 
 
 def copy_blocks(key_caches, value_caches, src_dst_pairs, stream=None):
@@ -204,6 +233,33 @@ def paged_attention_decode(out, query, key_cache, value_cache, block_tables, con
                                         int(max_context_len), int(partition_size), _code(query), ws_ptr, ws_bytes,
                                         _stream(stream))
     _ok(rc, "paged_attention_decode")
+    return out
+
+
+def paged_attention_decode_fp8(out, query, key_cache, value_cache, block_tables, context_lens, scale, k_scale,
+                               v_scale, max_context_len, partition_size=None, workspace=None, stream=None,
+                               total_context_tokens=0):
+    """Decode attention over E4M3 pools (values ``k_scale * code``, ``v_scale * code``); ``out``/``query``
+    ``[S, Hq, D]`` in fp16 or bf16."""
+    lib = load_library()
+    S, Hq, D = query.shape
+    NB, B, Hkv, _ = key_cache.shape
+    MB = block_tables.shape[1] if block_tables.dim() == 2 else 1
+    if block_tables.dtype != torch.int32 or context_lens.dtype != torch.int32:
+        raise ValueError("block_tables and context_lens must be int32")
+    if partition_size is None:
+        partition_size = decode_partition_size(S, Hkv, D, B, max_context_len, FP8_E4M3, total_context_tokens)
+    need = decode_workspace_size(S, Hq, D, max_context_len, partition_size) if partition_size else 0
+    if need and (workspace is None or workspace.numel() * workspace.element_size() < need):
+        workspace = torch.empty(need, dtype=torch.uint8, device=query.device)
+    ws_ptr = _dev(workspace, "workspace") if (need and workspace is not None) else None
+    ws_bytes = workspace.numel() * workspace.element_size() if ws_ptr else 0
+    rc = lib.pkv_paged_attention_decode_fp8(_dev(out, "out"), _dev(query, "query"), _fp8_pool(key_cache, "key_cache"),
+                                            _fp8_pool(value_cache, "value_cache"), _dev(block_tables, "block_tables"),
+                                            _dev(context_lens, "context_lens"), float(scale), float(k_scale),
+                                            float(v_scale), S, Hq, Hkv, D, B, MB, NB, int(max_context_len),
+                                            int(partition_size), _code(query), ws_ptr, ws_bytes, _stream(stream))
+    _ok(rc, "paged_attention_decode_fp8")
     return out
 
 

@@ -28,7 +28,8 @@ struct DecodeParams {
     float* ws_max;    // [num_seqs, Hq, P]   (log2 domain)
     float* ws_sum;    // [num_seqs, Hq, P]
     float* ws_out;    // [num_seqs, Hq, P, D]
-    float scale_log2; // scale * log2(e)
+    float scale_log2; // scale * log2(e) (times the K pool's scale for FP8 pools)
+    float out_scale;  // the V pool's scale for FP8 pools, else 1
     int num_seqs;
     int num_q_heads;
     int num_kv_heads;
@@ -103,7 +104,7 @@ __device__ __forceinline__ void decode_finish(const DecodeParams& p, const float
                 }
             }
         }
-        const float val = mx != -INFINITY ? o / sum : 0.f;
+        const float val = mx != -INFINITY ? o / sum * p.out_scale : 0.f;
         if (direct) {
             reinterpret_cast<T*>(p.out)[(row0 + h) * D + d] = Elem<T>::from_f(val);
         } else {

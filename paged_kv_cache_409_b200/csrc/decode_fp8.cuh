@@ -1,0 +1,309 @@
+// decode_fp8.cuh -- paged decode attention over FP8 (E4M3) K/V pools, head
+// dim 128, query and output in fp16 or bf16, 1 to 8 query heads per KV head.
+//
+// An FP8 pool halves the bytes decode streams from HBM, so at HBM speed each
+// SM has twice as many K/V elements per second to turn into products as with
+// 16-bit pools.  Both products therefore run on warp MMAs (mma.sync m16n8k16,
+// f16 inputs, fp32 accumulation) for every grouping, one head included:
+//   S^T [16 tokens x 8 heads] = K_tile . Q^T,   O^T [16 dims x 8 heads] += V^T . P^T.
+// Every E4M3 value is exactly an f16 value, so K and V are widened with
+// cvt.f16x2.e4m3x2 straight out of ldmatrix fragments:
+//   * K: ldmatrix of the FP8 tile read as 16-bit pairs gives a lane four
+//     consecutive dims (4c .. 4c+3) of one token.  The MMA contracts over any
+//     fixed order of the dims, so those four become the lane's k slots
+//     (2c, 2c+1, 2c+8, 2c+9) and the query fragment is loaded in the same
+//     order.
+//   * V: ldmatrix.trans of the same pairs gives a lane two tokens x two
+//     adjacent dims; a byte permute regroups them per dim, and the two dims
+//     become rows g and g + 8 of the lane's A fragment (row g = dim 2g, row
+//     g + 8 = dim 2g + 1 of the 16-dim chunk) -- the output rows come back in
+//     that order.
+// The query is rounded to f16 once (a bf16 query keeps its 8 significant bits
+// unless |q| < 2^-14; |q| must stay below 65504), the weights P go in as f16
+// (11 significant bits, one MMA term).  The pools' scales fold into the
+// score scale (k_scale) and the final normalisation (v_scale).  Partitions,
+// per-warp TMA pipelines and the CTA merge are those of decode.cuh.
+#pragma once
+
+#include "decode.cuh"
+
+namespace pkv {
+
+template <int B, int G, int NST, int NW>
+struct DecodeFp8Cfg {
+    static constexpr int D = 128;
+    static constexpr int TILE = B * D;       // one block-head of K (or V): B rows of 128 bytes
+    static constexpr int STAGE = 2 * TILE;
+    static constexpr int STAGES_BYTES = NW * NST * STAGE;
+    static constexpr int RED_BYTES = NW * G * (D + 2) * 4;  // the merge reuses the stage buffers
+    static constexpr int BT_OFF = STAGES_BYTES > RED_BYTES ? STAGES_BYTES : RED_BYTES;
+    static_assert(TILE % 1024 == 0, "tiles must keep 1024-byte alignment for the 128-byte swizzle");
+    static size_t smem_bytes(int pb) { return 1024 + BT_OFF + static_cast<size_t>(pb) * 4 + 16 + NW * NST * 8; }
+};
+
+template <typename T, int B, int G, int NST, int NW>
+__global__ void __launch_bounds__(NW * 32) paged_decode_fp8_kernel(const DecodeParams p,
+                                                                   const __grid_constant__ CUtensorMap tm_k,
+                                                                   const __grid_constant__ CUtensorMap tm_v) {
+    using C = DecodeFp8Cfg<B, G, NST, NW>;
+    constexpr int D = C::D;
+    constexpr int kThreads = NW * 32;
+    constexpr int KS = D / 16;         // 16-dim chunks
+    constexpr int MT = (B + 15) / 16;  // 16-token tiles per block
+    static_assert(sizeof(T) == 2 && G >= 1 && G <= 8, "FP8 decode takes a 16-bit query and 1..8 heads");
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = align_1024(smem_raw);
+
+    const int per_seq = p.num_partitions * p.num_kv_heads;
+    const int s = blockIdx.x / per_seq;
+    const int rem = blockIdx.x - s * per_seq;
+    const int part = rem / p.num_kv_heads;
+    const int g = rem - part * p.num_kv_heads;
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+
+    const int ctx_raw = p.context_lens[s];
+    const int nblk = decode_seq_blocks(ctx_raw, B, p.max_blocks_per_seq, p.num_partitions * p.partition_blocks,
+                                       threadIdx.x == 0 && part == 0 && g == 0);
+    const int ctx = min(max(ctx_raw, 0), nblk * B);
+    const int nparts = nblk > 0 ? (nblk + p.partition_blocks - 1) / p.partition_blocks : 1;
+    if (part >= nparts) return;
+    const int b0 = part * p.partition_blocks;
+    const int nb = max(0, min(nblk - b0, p.partition_blocks));
+    const bool direct = nparts == 1;
+
+    int* bt_s = reinterpret_cast<int*>(smem + C::BT_OFF);
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + ((C::BT_OFF + p.partition_blocks * 4 + 15) & ~15));
+    const int32_t* bt_row = p.block_tables + static_cast<int64_t>(s) * p.max_blocks_per_seq + b0;
+    for (int i = threadIdx.x; i < nb; i += kThreads) {
+        int id = bt_row[i];
+        if (id < 0 || id >= p.num_blocks) {
+            flag_error(PKV_DEVERR_BLOCK_ID);
+            id = -1;
+        }
+        bt_s[i] = id;
+    }
+    if (lane == 0) {
+#pragma unroll
+        for (int st = 0; st < NST; ++st) mbar_init(&bars[warp * NST + st], 1);
+        fence_mbar_init();
+    }
+
+    // Q^T fragments (B operand, f16): head lane/4, dims 16 ks + 4 (lane%4) + {0,1} | {2,3}.
+    uint32_t qf[KS][2];
+    {
+        const int hq = lane >> 2, k4 = 4 * (lane & 3);
+        const T* qrow = reinterpret_cast<const T*>(p.query) +
+                        (static_cast<int64_t>(s) * p.num_q_heads + static_cast<int64_t>(g) * G + hq) * D;
+#pragma unroll
+        for (int ks = 0; ks < KS; ++ks) {
+            if (hq < G) {
+                const uint2 raw = *reinterpret_cast<const uint2*>(qrow + 16 * ks + k4);
+                const float2 a = Elem<T>::pair(raw.x), b = Elem<T>::pair(raw.y);
+                qf[ks][0] = pack_half2(a.x, a.y);
+                qf[ks][1] = pack_half2(b.x, b.y);
+            } else {
+                qf[ks][0] = qf[ks][1] = 0u;
+            }
+        }
+    }
+    __syncthreads();
+
+    const int nw = nb > warp ? (nb - warp + NW - 1) / NW : 0;
+    uint8_t* wstage = smem + warp * NST * C::STAGE;
+    uint64_t* wbar = bars + warp * NST;
+#ifndef PKV_FP8_EVICT_NORMAL
+    const uint64_t policy = l2_policy_evict_first();
+#else
+    const uint64_t policy = l2_policy_evict_normal();
+#endif
+
+    auto issue = [&](int k) {  // lane 0 only
+        const int st = k % NST;
+        const int id = bt_s[warp + k * NW];
+        const int coord = id >= 0 ? id : static_cast<int>(p.num_blocks);  // out of range: zero fill
+        uint8_t* kd = wstage + st * C::STAGE;
+        mbar_arrive_expect_tx(&wbar[st], C::STAGE);
+        tma_load_4d_hint(kd, &tm_k, 0, g, 0, coord, &wbar[st], policy);
+        tma_load_4d_hint(kd + C::TILE, &tm_v, 0, g, 0, coord, &wbar[st], policy);
+    };
+    if (lane == 0) {
+        for (int k = 0; k < NST && k < nw; ++k) issue(k);
+    }
+    __syncwarp();
+
+    float mA = -INFINITY, mB = -INFINITY, lA = 0.f, lB = 0.f;
+    // O^T: [chunk t][c0: (dim 16t + 2(lane/4), hA), c1: (same dim, hB), c2: (dim + 1, hA), c3: (dim + 1, hB)]
+    float o[KS][4];
+#pragma unroll
+    for (int t = 0; t < KS; ++t) o[t][0] = o[t][1] = o[t][2] = o[t][3] = 0.f;
+
+    const int lr = lane & 7, lm = lane >> 3;
+
+    int k = 0;
+    for (; k < nw; ++k) {
+        const int st = k % NST;
+        const bool ok = mbar_wait(&wbar[st], (k / NST) & 1);
+        if (!__all_sync(0xffffffffu, ok)) break;
+        const int lb = b0 + warp + k * NW;
+        const int valid = min(B, ctx - lb * B);
+        if (bt_s[warp + k * NW] >= 0) {
+            const uint8_t* Ks = wstage + st * C::STAGE;
+            const uint8_t* Vs = Ks + C::TILE;
+            // ---- S^T = K . Q^T
+            float sc[MT][4];
+#pragma unroll
+            for (int mt = 0; mt < MT; ++mt) {
+                sc[mt][0] = sc[mt][1] = sc[mt][2] = sc[mt][3] = 0.f;
+#pragma unroll
+                for (int kp = 0; kp < KS / 2; ++kp) {
+                    // r[0]: token g, chunk 2kp; r[1]: token g + 8, chunk 2kp; r[2], r[3]: chunk 2kp + 1
+                    uint32_t r[4];
+                    if constexpr (B >= 16) {
+                        const int tok = 16 * mt + lr + 8 * (lm & 1);
+                        const int ch = 2 * kp + (lm >> 1);
+                        ldsm_x4(r, Ks + tok * 128 + ((ch ^ (tok & 7)) << 4));
+                    } else {
+                        const int tok = lr;
+                        const int ch = 2 * kp + (lm & 1);
+                        ldsm_x2(r[0], r[2], Ks + tok * 128 + ((ch ^ (tok & 7)) << 4));
+                        r[1] = r[3] = 0u;
+                    }
+#pragma unroll
+                    for (int h = 0; h < 2; ++h) {
+                        const uint32_t top = r[2 * h], bot = r[2 * h + 1];
+                        const uint32_t a[4] = {f16x2_from_e4m3x2(static_cast<uint16_t>(top)),
+                                               f16x2_from_e4m3x2(static_cast<uint16_t>(bot)),
+                                               f16x2_from_e4m3x2(static_cast<uint16_t>(top >> 16)),
+                                               f16x2_from_e4m3x2(static_cast<uint16_t>(bot >> 16))};
+                        mma_16816<false>(sc[mt], a, qf[2 * kp + h][0], qf[2 * kp + h][1]);
+                    }
+                }
+            }
+            // ---- online softmax per head column (log2 domain)
+            float bmA = -INFINITY, bmB = -INFINITY;
+#pragma unroll
+            for (int mt = 0; mt < MT; ++mt) {
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    const int tok = 16 * mt + (lane >> 2) + (j >= 2 ? 8 : 0);
+                    sc[mt][j] = tok < valid ? sc[mt][j] * p.scale_log2 : -INFINITY;
+                }
+                bmA = fmaxf(bmA, fmaxf(sc[mt][0], sc[mt][2]));
+                bmB = fmaxf(bmB, fmaxf(sc[mt][1], sc[mt][3]));
+            }
+#pragma unroll
+            for (int off = 4; off < 32; off <<= 1) {
+                bmA = fmaxf(bmA, __shfl_xor_sync(0xffffffffu, bmA, off));
+                bmB = fmaxf(bmB, __shfl_xor_sync(0xffffffffu, bmB, off));
+            }
+            const float mnA = fmaxf(mA, bmA), mnB = fmaxf(mB, bmB);
+            const float alA = exp2f(mA - mnA), alB = exp2f(mB - mnB);
+            float sA = 0.f, sB = 0.f;
+#pragma unroll
+            for (int mt = 0; mt < MT; ++mt) {
+                sc[mt][0] = exp2f(sc[mt][0] - mnA);
+                sc[mt][1] = exp2f(sc[mt][1] - mnB);
+                sc[mt][2] = exp2f(sc[mt][2] - mnA);
+                sc[mt][3] = exp2f(sc[mt][3] - mnB);
+                sA += sc[mt][0] + sc[mt][2];
+                sB += sc[mt][1] + sc[mt][3];
+            }
+#pragma unroll
+            for (int off = 4; off < 32; off <<= 1) {
+                sA += __shfl_xor_sync(0xffffffffu, sA, off);
+                sB += __shfl_xor_sync(0xffffffffu, sB, off);
+            }
+            lA = lA * alA + sA;
+            lB = lB * alB + sB;
+            mA = mnA;
+            mB = mnB;
+#pragma unroll
+            for (int t = 0; t < KS; ++t) {
+                o[t][0] *= alA;
+                o[t][1] *= alB;
+                o[t][2] *= alA;
+                o[t][3] *= alB;
+            }
+            // ---- O^T += V^T . P^T
+#pragma unroll
+            for (int kt = 0; kt < MT; ++kt) {
+                const uint32_t bh0 = movmatrix_trans(pack_half2(sc[kt][0], sc[kt][1]));
+                const uint32_t bh1 = movmatrix_trans(pack_half2(sc[kt][2], sc[kt][3]));
+                const int t0 = 16 * kt + 2 * (lane & 3);
+                const bool partial = valid < 16 * kt + 16;
+                const uint32_t m0 = (t0 < valid ? 0x0000FFFFu : 0u) | (t0 + 1 < valid ? 0xFFFF0000u : 0u);
+                const uint32_t m1 = (t0 + 8 < valid ? 0x0000FFFFu : 0u) | (t0 + 9 < valid ? 0xFFFF0000u : 0u);
+#pragma unroll
+                for (int jp = 0; jp < KS / 2; ++jp) {
+                    // r[0]: tokens 2c, 2c+1 x dims 2g, 2g+1 of chunk 2jp; r[1]: tokens + 8; r[2], r[3]: chunk 2jp + 1
+                    uint32_t r[4];
+                    if constexpr (B >= 16) {
+                        const int tok = 16 * kt + lr + 8 * (lm & 1);
+                        const int ch = 2 * jp + (lm >> 1);
+                        ldsm_x4_trans(r, Vs + tok * 128 + ((ch ^ (tok & 7)) << 4));
+                    } else {
+                        const int tok = lr;
+                        const int ch = 2 * jp + (lm & 1);
+                        ldsm_x2_trans(r[0], r[2], Vs + tok * 128 + ((ch ^ (tok & 7)) << 4));
+                        r[1] = r[3] = 0u;
+                    }
+#pragma unroll
+                    for (int h = 0; h < 2; ++h) {
+                        // bytes (tok 2c, dim 2g) (tok 2c, dim 2g+1) (tok 2c+1, dim 2g) (tok 2c+1, dim 2g+1)
+                        // -> dim 2g: (tok 2c, tok 2c+1) in the low half, dim 2g+1 in the high half
+                        const uint32_t lo = __byte_perm(r[2 * h], 0u, 0x3120);
+                        const uint32_t hi = __byte_perm(r[2 * h + 1], 0u, 0x3120);
+                        uint32_t a[4] = {f16x2_from_e4m3x2(static_cast<uint16_t>(lo)),
+                                         f16x2_from_e4m3x2(static_cast<uint16_t>(lo >> 16)),
+                                         f16x2_from_e4m3x2(static_cast<uint16_t>(hi)),
+                                         f16x2_from_e4m3x2(static_cast<uint16_t>(hi >> 16))};
+                        if (partial) {  // rows past the context may hold anything: 0 * NaN must not reach O
+                            a[0] &= m0;
+                            a[1] &= m0;
+                            a[2] &= m1;
+                            a[3] &= m1;
+                        }
+                        mma_16816<false>(o[2 * jp + h], a, bh0, bh1);
+                    }
+                }
+            }
+        }
+        __syncwarp();
+        if (lane == 0 && k + NST < nw) {
+            fence_proxy_async();
+            issue(k + NST);
+        }
+    }
+    if (k < nw && lane == 0) {
+        for (int kk = k + 1; kk < min(nw, k + NST); ++kk) mbar_wait(&wbar[kk % NST], (kk / NST) & 1);
+    }
+    if (k < nw) mA = mB = -INFINITY, lA = lB = 0.f;
+
+    // ---- hand this warp's state to the CTA merge
+    __syncthreads();
+    float* red_m = reinterpret_cast<float*>(smem);
+    float* red_l = red_m + NW * G;
+    float* red_o = red_l + NW * G;
+    const int hA = 2 * (lane & 3), hB = hA + 1;
+    if (lane < 4) {
+        if (hA < G) red_m[warp * G + hA] = mA, red_l[warp * G + hA] = lA;
+        if (hB < G) red_m[warp * G + hB] = mB, red_l[warp * G + hB] = lB;
+    }
+#pragma unroll
+    for (int t = 0; t < KS; ++t) {
+        const int d = 16 * t + 2 * (lane >> 2);
+        if (hA < G) {
+            red_o[(warp * G + hA) * D + d] = o[t][0];
+            red_o[(warp * G + hA) * D + d + 1] = o[t][2];
+        }
+        if (hB < G) {
+            red_o[(warp * G + hB) * D + d] = o[t][1];
+            red_o[(warp * G + hB) * D + d + 1] = o[t][3];
+        }
+    }
+    __syncthreads();
+    decode_finish<T, D, G, NW>(p, red_m, s, g, part, direct);
+}
+
+}  // namespace pkv

@@ -40,6 +40,72 @@ __global__ void __launch_bounds__(128) reshape_and_cache_kernel(const uint4* __r
     }
 }
 
+// ---- reshape_and_cache into FP8 (E4M3) pools.
+// A stored code is the E4M3 value nearest to x / scale (ties to even,
+// saturated at 448).  The quotient is formed in fp32 with rounding to odd --
+// the truncated quotient with its last bit set when the division was inexact
+// (Boldo and Melquiond, "Emulation of FMA and correctly rounded sums: proved
+// algorithms using rounding to odd", 2008) -- so that the one rounding to
+// E4M3 that follows gives the nearest value to the EXACT quotient: with 24
+// significant bits against E4M3's 4, round-to-odd followed by round-to-nearest
+// is a single correct rounding.  NaN is stored as 0x7F.
+__device__ __forceinline__ float quotient_round_to_odd(float x, float scale) {
+    float q = __fdiv_rz(x, scale);
+    if (isfinite(q)) {
+        const float r = fmaf(-q, scale, x);  // exact remainder of the truncated quotient
+        if (r != 0.f) q = __uint_as_float(__float_as_uint(q) | 1u);
+    } else if (isnan(q)) {
+        q = __uint_as_float(0x7fc00000u);
+    }
+    return q;
+}
+
+template <typename TS>
+__device__ __forceinline__ void load8(const TS* p, float (&f)[8]) {
+    if constexpr (sizeof(TS) == 4) {
+        const float4 a = reinterpret_cast<const float4*>(p)[0], b = reinterpret_cast<const float4*>(p)[1];
+        f[0] = a.x, f[1] = a.y, f[2] = a.z, f[3] = a.w, f[4] = b.x, f[5] = b.y, f[6] = b.z, f[7] = b.w;
+    } else {
+        Elem<TS>::unpack16(*reinterpret_cast<const uint4*>(p), f);
+    }
+}
+
+__device__ __forceinline__ uint2 quantise8(const float (&f)[8], float scale) {
+    uint32_t w[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+        w[i] = e4m3x2_from_f32(quotient_round_to_odd(f[2 * i + 1], scale), quotient_round_to_odd(f[2 * i], scale));
+    return make_uint2(w[0] | (w[1] << 16), w[2] | (w[3] << 16));
+}
+
+// One CTA per token (grid-stride); each thread quantises 8 consecutive
+// elements of the token's K row and of its V row.
+template <typename TS>
+__global__ void __launch_bounds__(128) reshape_and_cache_fp8_kernel(const TS* __restrict__ key,
+                                                                    const TS* __restrict__ value,
+                                                                    uint2* __restrict__ key_cache,
+                                                                    uint2* __restrict__ value_cache,
+                                                                    const int64_t* __restrict__ slot_mapping,
+                                                                    int64_t num_tokens, int row_elems,
+                                                                    int64_t num_slots, float k_scale, float v_scale) {
+    const int groups = row_elems / 8;
+    for (int64_t t = blockIdx.x; t < num_tokens; t += gridDim.x) {
+        const int64_t slot = slot_mapping[t];
+        if (slot < 0) continue;
+        if (slot >= num_slots) {
+            if (threadIdx.x == 0) flag_error(PKV_DEVERR_SLOT);
+            continue;
+        }
+        for (int i = threadIdx.x; i < groups; i += blockDim.x) {
+            float kf[8], vf[8];
+            load8(key + t * row_elems + 8 * i, kf);
+            load8(value + t * row_elems + 8 * i, vf);
+            key_cache[slot * groups + i] = quantise8(kf, k_scale);
+            value_cache[slot * groups + i] = quantise8(vf, v_scale);
+        }
+    }
+}
+
 constexpr int kMaxLayersPerLaunch = 32;
 
 struct LayerPools {

@@ -20,6 +20,7 @@
 #include "index_kernels.cuh"
 #include "decode.cuh"
 #include "decode_mma.cuh"
+#include "decode_fp8.cuh"
 #include "prefill.cuh"
 
 namespace {
@@ -42,9 +43,13 @@ int elem_bytes(int dtype) {
         case PKV_F32: return 4;
         case PKV_F16: return 2;
         case PKV_BF16: return 2;
+        case PKV_FP8_E4M3: return 1;
         default: return 0;
     }
 }
+
+// Types a query / output may have (FP8 is a pool type only).
+bool query_type(int dtype) { return dtype == PKV_F32 || dtype == PKV_F16 || dtype == PKV_BF16; }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
 
@@ -74,6 +79,7 @@ CUtensorMapDataType cu_type(int dtype) {
     switch (dtype) {
         case PKV_F32: return CU_TENSOR_MAP_DATA_TYPE_FLOAT32;
         case PKV_F16: return CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
+        case PKV_FP8_E4M3: return CU_TENSOR_MAP_DATA_TYPE_UINT8;
         default: return CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
     }
 }
@@ -81,6 +87,10 @@ CUtensorMapDataType cu_type(int dtype) {
 // Pool [num_blocks, block_size, num_kv_heads, head_dim] as a 4-D tensor
 // (head_dim innermost); one box = one block x one KV head x 128 bytes of
 // head_dim, 128-byte swizzled.
+#ifndef PKV_FP8_L2_PROMOTION
+#define PKV_FP8_L2_PROMOTION CU_TENSOR_MAP_L2_PROMOTION_L2_256B
+#endif
+
 int make_pool_map(CUtensorMap* map, const void* pool, int dtype, int64_t num_blocks, int block_size,
                   int num_kv_heads, int head_dim) {
     auto fn = encode_fn();
@@ -95,8 +105,10 @@ int make_pool_map(CUtensorMap* map, const void* pool, int dtype, int64_t num_blo
                              (cuuint64_t)block_size * num_kv_heads * head_dim * eb};
     cuuint32_t box[4] = {(cuuint32_t)(128 / eb), 1, (cuuint32_t)block_size, 1};
     cuuint32_t estr[4] = {1, 1, 1, 1};
+    const CUtensorMapL2promotion promo =
+        dtype == PKV_FP8_E4M3 ? PKV_FP8_L2_PROMOTION : CU_TENSOR_MAP_L2_PROMOTION_L2_256B;
     CUresult r = fn(map, cu_type(dtype), 4, const_cast<void*>(pool), dims, strides, box, estr,
-                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, promo,
                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     if (r != CUDA_SUCCESS) {
         snprintf(g_last_cuda_error, sizeof g_last_cuda_error, "cuTensorMapEncodeTiled(pool) failed: %d", (int)r);
@@ -254,6 +266,48 @@ int decode_by_dim(int head_dim, int block_size, int group, const pkv::DecodePara
     }
 }
 
+#ifndef PKV_FP8_WARPS
+#define PKV_FP8_WARPS 4
+#endif
+#ifndef PKV_FP8_STAGE_BUDGET
+#define PKV_FP8_STAGE_BUDGET 32768  // bytes of K/V stages per FP8 decode CTA
+#endif
+
+template <typename T, int B, int G>
+int launch_decode_fp8(const pkv::DecodeParams& prm, const CUtensorMap& tk, const CUtensorMap& tv, int grid,
+                      cudaStream_t s) {
+    constexpr int STAGE = 2 * B * 128;
+    constexpr int NW = PKV_FP8_WARPS;
+    constexpr int NST = std::max(1, std::min(8, PKV_FP8_STAGE_BUDGET / (NW * STAGE)));
+    using C = pkv::DecodeFp8Cfg<B, G, NST, NW>;
+    static size_t configured[64] = {};
+    return launch_decode_kernel(pkv::paged_decode_fp8_kernel<T, B, G, NST, NW>, C::smem_bytes(prm.partition_blocks),
+                                NW * 32, prm, tk, tv, grid, s, configured);
+}
+
+template <typename T, int B>
+int decode_fp8_by_group(int group, const pkv::DecodeParams& prm, const CUtensorMap& tk, const CUtensorMap& tv,
+                        int grid, cudaStream_t s) {
+    switch (group) {
+        case 1: return launch_decode_fp8<T, B, 1>(prm, tk, tv, grid, s);
+        case 2: return launch_decode_fp8<T, B, 2>(prm, tk, tv, grid, s);
+        case 4: return launch_decode_fp8<T, B, 4>(prm, tk, tv, grid, s);
+        case 8: return launch_decode_fp8<T, B, 8>(prm, tk, tv, grid, s);
+        default: return PKV_EUNSUPPORTED;
+    }
+}
+
+template <typename T>
+int decode_fp8_by_block(int block_size, int group, const pkv::DecodeParams& prm, const CUtensorMap& tk,
+                        const CUtensorMap& tv, int grid, cudaStream_t s) {
+    switch (block_size) {
+        case 8: return decode_fp8_by_group<T, 8>(group, prm, tk, tv, grid, s);
+        case 16: return decode_fp8_by_group<T, 16>(group, prm, tk, tv, grid, s);
+        case 32: return decode_fp8_by_group<T, 32>(group, prm, tk, tv, grid, s);
+        default: return PKV_EUNSUPPORTED;
+    }
+}
+
 template <typename T>
 int launch_merge(int head_dim, const pkv::MergeParams& mp, cudaStream_t s) {
     const int warps = mp.num_seqs * mp.num_q_heads;
@@ -297,6 +351,110 @@ int prefill_by_group(int group, const pkv::PrefillParams& prm, const CUtensorMap
         case 4: return launch_prefill<T, D, 4>(prm, tq, tk, tv, grid, s);
         case 8: return launch_prefill<T, D, 8>(prm, tq, tk, tv, grid, s);
         default: return PKV_EUNSUPPORTED;
+    }
+}
+
+// Decode with the query / output in `dtype` and the pools in `kv_dtype`
+// (the same 16/32-bit type, or FP8 E4M3 with its two scales).
+int decode_impl(void* out, const void* query, const void* key_cache, const void* value_cache,
+                const int32_t* block_tables, const int32_t* context_lens, float scale, int num_seqs, int num_q_heads,
+                int num_kv_heads, int head_dim, int block_size, int max_blocks_per_seq, int64_t num_blocks,
+                int max_context_len, int partition_size, int dtype, int kv_dtype, float k_scale, float v_scale,
+                void* workspace, size_t workspace_bytes, pkv_stream_t stream) {
+    const bool fp8 = kv_dtype == PKV_FP8_E4M3;
+    if (!query_type(dtype) || (kv_dtype != dtype && !fp8)) return PKV_EUNSUPPORTED;
+    if (fp8 && (dtype == PKV_F32 || head_dim != 128)) return PKV_EUNSUPPORTED;
+    if (num_seqs < 0 || num_q_heads <= 0 || num_kv_heads <= 0 || max_blocks_per_seq <= 0 || num_blocks <= 0 ||
+        max_context_len < 0 || partition_size < 0 || !std::isfinite(scale))
+        return PKV_EINVAL;
+    if (num_q_heads % num_kv_heads) return PKV_EINVAL;
+    const int group = num_q_heads / num_kv_heads;
+    if (!supported_group(group) || (head_dim != 64 && head_dim != 128) ||
+        (block_size != 8 && block_size != 16 && block_size != 32))
+        return PKV_EUNSUPPORTED;
+    if (partition_size % block_size) return PKV_EINVAL;
+    if (num_blocks >= (int64_t)INT32_MAX || (int64_t)max_blocks_per_seq * block_size > INT32_MAX) return PKV_EINVAL;
+    if (num_seqs == 0) return PKV_OK;
+    if (!out || !query || !key_cache || !value_cache || !block_tables || !context_lens) return PKV_EINVAL;
+    if (!aligned16(out) || !aligned16(query) || !aligned16(key_cache) || !aligned16(value_cache) ||
+        (reinterpret_cast<uintptr_t>(block_tables) & 3) || (reinterpret_cast<uintptr_t>(context_lens) & 3))
+        return PKV_EINVAL;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+
+    const int64_t max_blocks_needed = std::max<int64_t>(1, ceil_div(std::max(max_context_len, 1), block_size));
+    int64_t pb = partition_size > 0 ? partition_size / block_size : max_blocks_needed;
+    pb = std::min(pb, max_blocks_needed);
+    const int64_t parts = ceil_div(max_blocks_needed, pb);
+    if (pb > 4096) return PKV_EUNSUPPORTED;  // per-CTA block list lives in shared memory
+    const size_t need = parts > 1 ? pkv_decode_workspace_size(num_seqs, num_q_heads, head_dim, max_context_len,
+                                                              (int)(pb * block_size))
+                                  : 0;
+    if (need > 0 && (!workspace || workspace_bytes < need || !aligned16(workspace))) return PKV_EWORKSPACE;
+    const int64_t grid = (int64_t)num_seqs * parts * num_kv_heads;
+    if (grid > INT32_MAX) return PKV_EUNSUPPORTED;
+
+    if (checked_mode()) {
+        int rc = check_tables(block_tables, context_lens, num_seqs, max_blocks_per_seq, block_size, num_blocks,
+                              max_context_len, s);
+        if (rc) return rc;
+    }
+
+    CUtensorMap tk, tv;
+    int rc = make_pool_map(&tk, key_cache, kv_dtype, num_blocks, block_size, num_kv_heads, head_dim);
+    if (rc) return rc;
+    rc = make_pool_map(&tv, value_cache, kv_dtype, num_blocks, block_size, num_kv_heads, head_dim);
+    if (rc) return rc;
+
+    pkv::DecodeParams prm;
+    prm.out = out;
+    prm.query = query;
+    prm.block_tables = block_tables;
+    prm.context_lens = context_lens;
+    const int64_t rows = (int64_t)num_seqs * num_q_heads * parts;
+    const int64_t ml = ((rows * 4 + 15) / 16) * 16;
+    prm.ws_max = need ? reinterpret_cast<float*>(workspace) : nullptr;
+    prm.ws_sum = need ? reinterpret_cast<float*>(static_cast<char*>(workspace) + ml) : nullptr;
+    prm.ws_out = need ? reinterpret_cast<float*>(static_cast<char*>(workspace) + 2 * ml) : nullptr;
+    prm.scale_log2 = scale * 1.4426950408889634f * k_scale;
+    prm.out_scale = v_scale;
+    prm.num_seqs = num_seqs;
+    prm.num_q_heads = num_q_heads;
+    prm.num_kv_heads = num_kv_heads;
+    prm.max_blocks_per_seq = max_blocks_per_seq;
+    prm.num_blocks = num_blocks;
+    prm.partition_blocks = (int)pb;
+    prm.num_partitions = (int)parts;
+
+    if (fp8) {
+        rc = dtype == PKV_F16 ? decode_fp8_by_block<__half>(block_size, group, prm, tk, tv, (int)grid, s)
+                              : decode_fp8_by_block<__nv_bfloat16>(block_size, group, prm, tk, tv, (int)grid, s);
+    } else {
+        switch (dtype) {
+            case PKV_F32: rc = decode_by_dim<float>(head_dim, block_size, group, prm, tk, tv, (int)grid, s); break;
+            case PKV_F16: rc = decode_by_dim<__half>(head_dim, block_size, group, prm, tk, tv, (int)grid, s); break;
+            default:
+                rc = decode_by_dim<__nv_bfloat16>(head_dim, block_size, group, prm, tk, tv, (int)grid, s);
+                break;
+        }
+    }
+    if (rc || parts <= 1) return rc;
+
+    pkv::MergeParams mp;
+    mp.out = out;
+    mp.context_lens = context_lens;
+    mp.ws_max = prm.ws_max;
+    mp.ws_sum = prm.ws_sum;
+    mp.ws_out = prm.ws_out;
+    mp.num_seqs = num_seqs;
+    mp.num_q_heads = num_q_heads;
+    mp.block_size = block_size;
+    mp.max_blocks_per_seq = max_blocks_per_seq;
+    mp.partition_blocks = (int)pb;
+    mp.num_partitions = (int)parts;
+    switch (dtype) {
+        case PKV_F32: return launch_merge<float>(head_dim, mp, s);
+        case PKV_F16: return launch_merge<__half>(head_dim, mp, s);
+        default: return launch_merge<__nv_bfloat16>(head_dim, mp, s);
     }
 }
 
@@ -346,6 +504,54 @@ int pkv_reshape_and_cache(const void* key, const void* value, void* key_cache, v
     pkv::reshape_and_cache_kernel<<<grid, 128, 0, s>>>(
         static_cast<const uint4*>(key), static_cast<const uint4*>(value), static_cast<uint4*>(key_cache),
         static_cast<uint4*>(value_cache), slot_mapping, num_tokens, (int)(row_bytes / 16), num_slots);
+    PKV_CUDA(cudaGetLastError());
+    return PKV_OK;
+}
+
+int pkv_reshape_and_cache_fp8(const void* key, const void* value, void* key_cache, void* value_cache,
+                              const int64_t* slot_mapping, int64_t num_tokens, int num_kv_heads, int head_dim,
+                              int block_size, int64_t num_blocks, int src_dtype, float k_scale, float v_scale,
+                              pkv_stream_t stream) {
+    if (!query_type(src_dtype)) return PKV_EUNSUPPORTED;
+    if (num_tokens < 0 || num_kv_heads <= 0 || head_dim <= 0 || block_size <= 0 || num_blocks <= 0)
+        return PKV_EINVAL;
+    if (!(std::isfinite(k_scale) && k_scale > 0.f && std::isfinite(v_scale) && v_scale > 0.f)) return PKV_EINVAL;
+    const int64_t row_elems = (int64_t)num_kv_heads * head_dim;
+    if (row_elems % 16 != 0 || row_elems > INT32_MAX) return PKV_EUNSUPPORTED;
+    if (num_tokens == 0) return PKV_OK;
+    if (!key || !value || !key_cache || !value_cache || !slot_mapping) return PKV_EINVAL;
+    if (!aligned16(key) || !aligned16(value) || !aligned16(key_cache) || !aligned16(value_cache) ||
+        (reinterpret_cast<uintptr_t>(slot_mapping) & 7))
+        return PKV_EINVAL;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const int64_t num_slots = num_blocks * block_size;
+    if (checked_mode()) {
+        std::vector<int64_t> sm;
+        int rc = fetch(sm, slot_mapping, (size_t)num_tokens, s);
+        if (rc) return rc;
+        for (int64_t v : sm)
+            if (v >= num_slots) return PKV_ERANGE;
+    }
+    const int grid = (int)std::min<int64_t>(num_tokens, 65535);
+    uint2* kc = static_cast<uint2*>(key_cache);
+    uint2* vc = static_cast<uint2*>(value_cache);
+    switch (src_dtype) {
+        case PKV_F32:
+            pkv::reshape_and_cache_fp8_kernel<float><<<grid, 128, 0, s>>>(
+                static_cast<const float*>(key), static_cast<const float*>(value), kc, vc, slot_mapping, num_tokens,
+                (int)row_elems, num_slots, k_scale, v_scale);
+            break;
+        case PKV_F16:
+            pkv::reshape_and_cache_fp8_kernel<__half><<<grid, 128, 0, s>>>(
+                static_cast<const __half*>(key), static_cast<const __half*>(value), kc, vc, slot_mapping, num_tokens,
+                (int)row_elems, num_slots, k_scale, v_scale);
+            break;
+        default:
+            pkv::reshape_and_cache_fp8_kernel<__nv_bfloat16><<<grid, 128, 0, s>>>(
+                static_cast<const __nv_bfloat16*>(key), static_cast<const __nv_bfloat16*>(value), kc, vc, slot_mapping,
+                num_tokens, (int)row_elems, num_slots, k_scale, v_scale);
+            break;
+    }
     PKV_CUDA(cudaGetLastError());
     return PKV_OK;
 }
@@ -474,91 +680,21 @@ int pkv_paged_attention_decode(void* out, const void* query, const void* key_cac
                                int num_q_heads, int num_kv_heads, int head_dim, int block_size,
                                int max_blocks_per_seq, int64_t num_blocks, int max_context_len, int partition_size,
                                int dtype, void* workspace, size_t workspace_bytes, pkv_stream_t stream) {
-    if (!elem_bytes(dtype)) return PKV_EUNSUPPORTED;
-    if (num_seqs < 0 || num_q_heads <= 0 || num_kv_heads <= 0 || max_blocks_per_seq <= 0 || num_blocks <= 0 ||
-        max_context_len < 0 || partition_size < 0 || !std::isfinite(scale))
-        return PKV_EINVAL;
-    if (num_q_heads % num_kv_heads) return PKV_EINVAL;
-    const int group = num_q_heads / num_kv_heads;
-    if (!supported_group(group) || (head_dim != 64 && head_dim != 128) ||
-        (block_size != 8 && block_size != 16 && block_size != 32))
-        return PKV_EUNSUPPORTED;
-    if (partition_size % block_size) return PKV_EINVAL;
-    if (num_blocks >= (int64_t)INT32_MAX || (int64_t)max_blocks_per_seq * block_size > INT32_MAX) return PKV_EINVAL;
-    if (num_seqs == 0) return PKV_OK;
-    if (!out || !query || !key_cache || !value_cache || !block_tables || !context_lens) return PKV_EINVAL;
-    if (!aligned16(out) || !aligned16(query) || !aligned16(key_cache) || !aligned16(value_cache) ||
-        (reinterpret_cast<uintptr_t>(block_tables) & 3) || (reinterpret_cast<uintptr_t>(context_lens) & 3))
-        return PKV_EINVAL;
-    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    return decode_impl(out, query, key_cache, value_cache, block_tables, context_lens, scale, num_seqs, num_q_heads,
+                       num_kv_heads, head_dim, block_size, max_blocks_per_seq, num_blocks, max_context_len,
+                       partition_size, dtype, dtype, 1.f, 1.f, workspace, workspace_bytes, stream);
+}
 
-    const int64_t max_blocks_needed = std::max<int64_t>(1, ceil_div(std::max(max_context_len, 1), block_size));
-    int64_t pb = partition_size > 0 ? partition_size / block_size : max_blocks_needed;
-    pb = std::min(pb, max_blocks_needed);
-    const int64_t parts = ceil_div(max_blocks_needed, pb);
-    if (pb > 4096) return PKV_EUNSUPPORTED;  // per-CTA block list lives in shared memory
-    const size_t need = parts > 1 ? pkv_decode_workspace_size(num_seqs, num_q_heads, head_dim, max_context_len,
-                                                              (int)(pb * block_size))
-                                  : 0;
-    if (need > 0 && (!workspace || workspace_bytes < need || !aligned16(workspace))) return PKV_EWORKSPACE;
-    const int64_t grid = (int64_t)num_seqs * parts * num_kv_heads;
-    if (grid > INT32_MAX) return PKV_EUNSUPPORTED;
-
-    if (checked_mode()) {
-        int rc = check_tables(block_tables, context_lens, num_seqs, max_blocks_per_seq, block_size, num_blocks,
-                              max_context_len, s);
-        if (rc) return rc;
-    }
-
-    CUtensorMap tk, tv;
-    int rc = make_pool_map(&tk, key_cache, dtype, num_blocks, block_size, num_kv_heads, head_dim);
-    if (rc) return rc;
-    rc = make_pool_map(&tv, value_cache, dtype, num_blocks, block_size, num_kv_heads, head_dim);
-    if (rc) return rc;
-
-    pkv::DecodeParams prm;
-    prm.out = out;
-    prm.query = query;
-    prm.block_tables = block_tables;
-    prm.context_lens = context_lens;
-    const int64_t rows = (int64_t)num_seqs * num_q_heads * parts;
-    const int64_t ml = ((rows * 4 + 15) / 16) * 16;
-    prm.ws_max = need ? reinterpret_cast<float*>(workspace) : nullptr;
-    prm.ws_sum = need ? reinterpret_cast<float*>(static_cast<char*>(workspace) + ml) : nullptr;
-    prm.ws_out = need ? reinterpret_cast<float*>(static_cast<char*>(workspace) + 2 * ml) : nullptr;
-    prm.scale_log2 = scale * 1.4426950408889634f;
-    prm.num_seqs = num_seqs;
-    prm.num_q_heads = num_q_heads;
-    prm.num_kv_heads = num_kv_heads;
-    prm.max_blocks_per_seq = max_blocks_per_seq;
-    prm.num_blocks = num_blocks;
-    prm.partition_blocks = (int)pb;
-    prm.num_partitions = (int)parts;
-
-    switch (dtype) {
-        case PKV_F32: rc = decode_by_dim<float>(head_dim, block_size, group, prm, tk, tv, (int)grid, s); break;
-        case PKV_F16: rc = decode_by_dim<__half>(head_dim, block_size, group, prm, tk, tv, (int)grid, s); break;
-        default: rc = decode_by_dim<__nv_bfloat16>(head_dim, block_size, group, prm, tk, tv, (int)grid, s); break;
-    }
-    if (rc || parts <= 1) return rc;
-
-    pkv::MergeParams mp;
-    mp.out = out;
-    mp.context_lens = context_lens;
-    mp.ws_max = prm.ws_max;
-    mp.ws_sum = prm.ws_sum;
-    mp.ws_out = prm.ws_out;
-    mp.num_seqs = num_seqs;
-    mp.num_q_heads = num_q_heads;
-    mp.block_size = block_size;
-    mp.max_blocks_per_seq = max_blocks_per_seq;
-    mp.partition_blocks = (int)pb;
-    mp.num_partitions = (int)parts;
-    switch (dtype) {
-        case PKV_F32: return launch_merge<float>(head_dim, mp, s);
-        case PKV_F16: return launch_merge<__half>(head_dim, mp, s);
-        default: return launch_merge<__nv_bfloat16>(head_dim, mp, s);
-    }
+int pkv_paged_attention_decode_fp8(void* out, const void* query, const void* key_cache, const void* value_cache,
+                                   const int32_t* block_tables, const int32_t* context_lens, float scale,
+                                   float k_scale, float v_scale, int num_seqs, int num_q_heads, int num_kv_heads,
+                                   int head_dim, int block_size, int max_blocks_per_seq, int64_t num_blocks,
+                                   int max_context_len, int partition_size, int dtype, void* workspace,
+                                   size_t workspace_bytes, pkv_stream_t stream) {
+    if (!(std::isfinite(k_scale) && k_scale > 0.f && std::isfinite(v_scale) && v_scale > 0.f)) return PKV_EINVAL;
+    return decode_impl(out, query, key_cache, value_cache, block_tables, context_lens, scale, num_seqs, num_q_heads,
+                       num_kv_heads, head_dim, block_size, max_blocks_per_seq, num_blocks, max_context_len,
+                       partition_size, dtype, PKV_FP8_E4M3, k_scale, v_scale, workspace, workspace_bytes, stream);
 }
 
 int pkv_paged_attention_prefill_chunk(void* out, const void* query, const void* key_cache, const void* value_cache,

@@ -158,6 +158,11 @@ __device__ __forceinline__ uint64_t l2_policy_evict_first() {
     asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
     return p;
 }
+__device__ __forceinline__ uint64_t l2_policy_evict_normal() {
+    uint64_t p;
+    asm volatile("createpolicy.fractional.L2::evict_normal.b64 %0, 1.0;" : "=l"(p));
+    return p;
+}
 
 // ---------------------------------------------------------------- tcgen05
 // Allocate `ncols` tensor-memory columns (power of two >= 32); the address is
@@ -284,6 +289,25 @@ __device__ __forceinline__ void mma_16816(float (&c)[4], const uint32_t (&a)[4],
 }
 
 // ---------------------------------------------------------------- element types
+// ---- FP8 E4M3 (OCP 8-bit float: bias 7, 3 mantissa bits, max 448, no infinities)
+// Two fp32 values to two E4M3 codes, round to nearest even, magnitudes beyond
+// 448 saturated; `hi` goes to bits 15:8, `lo` to bits 7:0.
+__device__ __forceinline__ uint16_t e4m3x2_from_f32(float hi, float lo) {
+    uint16_t d;
+    asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(d) : "f"(hi), "f"(lo));
+    return d;
+}
+// Two E4M3 codes (bits 15:8, 7:0) to an f16x2 (upper, lower half); exact.
+__device__ __forceinline__ uint32_t f16x2_from_e4m3x2(uint16_t v) {
+    uint32_t d;
+    asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(d) : "h"(v));
+    return d;
+}
+__device__ __forceinline__ uint32_t pack_half2(float lo, float hi) {
+    const __half2 h = __floats2half2_rn(lo, hi);
+    return *reinterpret_cast<const uint32_t*>(&h);
+}
+
 template <typename T>
 struct Elem;
 

@@ -58,6 +58,18 @@ def randn(shape, dtype, gen, device) -> torch.Tensor:
     return fill_normal(torch.empty(shape, dtype=dtype, device=device), gen)
 
 
+def randn_e4m3(shape, scale: float, gen, device, chunk: int = 1 << 26) -> torch.Tensor:
+    """uint8 E4M3 codes of N(0, 1) values drawn in fp32 and divided by ``scale``
+    (torch's float8_e4m3fn cast, magnitudes clamped to 448 first)."""
+    out = torch.empty(shape, dtype=torch.uint8, device=device)
+    flat = out.view(-1)
+    for i in range(0, flat.numel(), chunk):
+        n = min(chunk, flat.numel() - i)
+        x = torch.randn(n, generator=gen, device=device, dtype=torch.float32) / scale
+        flat[i:i + n] = x.clamp_(-448.0, 448.0).to(torch.float8_e4m3fn).view(torch.uint8)
+    return out
+
+
 def pool_size(blocks_in_use: int, free_fraction: float = 0.1) -> int:
     """Pool of the blocks in use plus ``free_fraction`` free blocks (rounded up)."""
     tenths = int(round(free_fraction * 10))
@@ -92,12 +104,13 @@ def live_slots(block_tables: np.ndarray, lens, block_size: int) -> np.ndarray:
 
 
 def poison_pool(cache: torch.Tensor, keep_slots: np.ndarray):
-    """Set every slot of ``cache`` ([NB, B, Hkv, D]) outside ``keep_slots`` to NaN."""
+    """Set every slot of ``cache`` ([NB, B, Hkv, D]) outside ``keep_slots`` to NaN
+    (code 0x7F in a uint8 E4M3 pool)."""
     nb, b = cache.shape[:2]
     mask = torch.ones(nb * b, dtype=torch.bool)
     mask[torch.from_numpy(np.asarray(keep_slots, dtype=np.int64))] = False
     rows = cache.view(nb * b, -1)
-    rows[mask.to(cache.device)] = float("nan")
+    rows[mask.to(cache.device)] = 0x7F if cache.dtype == torch.uint8 else float("nan")
 
 
 @dataclass
@@ -139,16 +152,23 @@ class DecodeWorkload:
     def max_context_len(self):
         return int(self.context_lens.max()) if len(self.context_lens) else 0
 
+    @property
+    def fp8(self) -> bool:
+        """Pools of uint8 E4M3 codes (scales in ``extra``) instead of ``dtype`` elements."""
+        return self.key_caches[0].dtype == torch.uint8
+
     def kv_bytes(self) -> int:
         """Bytes of K and V the attention must read once: sum_s 2 c_s Hkv D T, all layers."""
-        t = torch.tensor([], dtype=self.dtype).element_size()
+        t = self.key_caches[0].element_size()
         return int(2 * int(self.context_lens.astype(np.int64).sum()) * self.num_kv_heads * self.head_dim * t
                    * self.num_layers)
 
 
 def decode_workload(name, context_lens, num_q_heads, num_kv_heads, head_dim, block_size, dtype, *,
                     seed, device="cpu", num_blocks=None, num_layers=1, poison=False,
-                    max_blocks_per_seq=None, scale=None) -> DecodeWorkload:
+                    max_blocks_per_seq=None, scale=None, fp8_scales=None) -> DecodeWorkload:
+    """``fp8_scales=(k_scale, v_scale)`` makes the pools uint8 E4M3 codes of
+    N(0, 1) / scale; queries and new tokens stay in ``dtype``."""
     rng = np.random.default_rng(seed)
     gen = _gen(seed, device)
     lens = np.asarray(context_lens, dtype=np.int32)
@@ -161,8 +181,12 @@ def decode_workload(name, context_lens, num_q_heads, num_kv_heads, head_dim, blo
         np.zeros(0, np.int64)
     kc, vc, qs, nk, nv = [], [], [], [], []
     for _ in range(num_layers):
-        kc.append(randn((nb, block_size, num_kv_heads, head_dim), dtype, gen, device))
-        vc.append(randn((nb, block_size, num_kv_heads, head_dim), dtype, gen, device))
+        if fp8_scales is None:
+            kc.append(randn((nb, block_size, num_kv_heads, head_dim), dtype, gen, device))
+            vc.append(randn((nb, block_size, num_kv_heads, head_dim), dtype, gen, device))
+        else:
+            kc.append(randn_e4m3((nb, block_size, num_kv_heads, head_dim), fp8_scales[0], gen, device))
+            vc.append(randn_e4m3((nb, block_size, num_kv_heads, head_dim), fp8_scales[1], gen, device))
         qs.append(randn((S, num_q_heads, head_dim), dtype, gen, device))
         nk.append(randn((S, num_kv_heads, head_dim), dtype, gen, device))
         nv.append(randn((S, num_kv_heads, head_dim), dtype, gen, device))
@@ -171,8 +195,10 @@ def decode_workload(name, context_lens, num_q_heads, num_kv_heads, head_dim, blo
         for c in kc + vc:
             poison_pool(c, keep)
     sc = float(np.float32(1.0 / math.sqrt(head_dim))) if scale is None else float(np.float32(scale))
+    extra = {} if fp8_scales is None else {"k_scale": float(np.float32(fp8_scales[0])),
+                                           "v_scale": float(np.float32(fp8_scales[1]))}
     return DecodeWorkload(name, S, num_q_heads, num_kv_heads, head_dim, block_size, dtype, sc, nb, lens, bt,
-                          slots, kc, vc, qs, nk, nv)
+                          slots, kc, vc, qs, nk, nv, extra)
 
 
 # --------------------------------------------------------------------------
@@ -191,6 +217,30 @@ def llama7b_decode_f16(device="cpu", num_seqs=64, poison=False, seed=1002):
     lens = rng.integers(128, 2048 + 1, size=num_seqs)
     return decode_workload("llama7b_decode_f16", lens, 32, 32, 128, 16, torch.float16, seed=seed,
                            device=device, poison=poison)
+
+
+# FP8 pools: a scale that maps 4 standard deviations of N(0, 1) to E4M3's 448
+# for K, and a different one for V, neither a power of two.
+FP8_K_SCALE = 4.0 / 448.0
+FP8_V_SCALE = 5.0 / 448.0
+
+
+def llama7b_decode_fp8(device="cpu", num_seqs=64, poison=False, seed=1002):
+    """The llama7b batch (64 sequences, context U[128, 2048], 32 = 32 KV heads,
+    d 128, block 16) with FP8 E4M3 pools and an fp16 query."""
+    rng = np.random.default_rng(seed)
+    lens = rng.integers(128, 2048 + 1, size=num_seqs)
+    return decode_workload("llama7b_decode_fp8", lens, 32, 32, 128, 16, torch.float16, seed=seed, device=device,
+                           poison=poison, fp8_scales=(FP8_K_SCALE, FP8_V_SCALE))
+
+
+def gqa70b_decode_fp8(device="cpu", num_seqs=256, num_layers=80, poison=False, seed=1003):
+    """The gqa70b batch (256 sequences, lognormal context, 64 q heads over 8 KV
+    heads, d 128, block 16, 80 layers) with FP8 E4M3 pools and a bf16 query."""
+    rng = np.random.default_rng(seed)
+    lens = np.clip(np.rint(np.exp(rng.normal(math.log(1024.0), 1.0, size=num_seqs))), 16, 4096).astype(np.int64)
+    return decode_workload("gqa70b_decode_fp8", lens, 64, 8, 128, 16, torch.bfloat16, seed=seed, device=device,
+                           num_layers=num_layers, poison=poison, fp8_scales=(FP8_K_SCALE, FP8_V_SCALE))
 
 
 def gqa70b_decode_bf16(device="cpu", num_seqs=256, num_layers=80, poison=False, seed=1003):
@@ -374,4 +424,6 @@ CONFIGS = {
     "shared_prefix_decode_f16": shared_prefix_decode_f16,
     "mixed_step_bf16": mixed_step_bf16,
     "multi_token_decode_bf16": multi_token_decode_bf16,
+    "llama7b_decode_fp8": llama7b_decode_fp8,
+    "gqa70b_decode_fp8": gqa70b_decode_fp8,
 }

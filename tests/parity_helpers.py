@@ -81,9 +81,14 @@ def oracle_decode_step(w, seqs=None, layer=0, pre_k=None, pre_v=None):
     remap = {int(b): i for i, b in enumerate(used)}
     slots = np.array([remap[int(s) // B] * B + int(s) % B for s in w.slot_mapping[seqs]], dtype=np.int64)
     orc = oracle.get()
-    orc.reshape_and_cache(nk, nv, kc, vc, slots, code)
-    q, _ = oracle.storage(w.queries[layer][torch.from_numpy(seqs).to(w.queries[layer].device)])
-    out = orc.paged_attention_decode(q, kc, vc, bt, lens, w.scale, code)
+    q, qcode = oracle.storage(w.queries[layer][torch.from_numpy(seqs).to(w.queries[layer].device)])
+    if w.fp8:
+        ks, vs = w.extra["k_scale"], w.extra["v_scale"]
+        orc.reshape_and_cache_fp8(nk, nv, kc, vc, slots, qcode, ks, vs)
+        out = orc.paged_attention_decode_kv(q, qcode, kc, vc, oracle.E4M3, ks, vs, bt, lens, w.scale)
+    else:
+        orc.reshape_and_cache(nk, nv, kc, vc, slots, code)
+        out = orc.paged_attention_decode(q, kc, vc, bt, lens, w.scale, code)
     return out, kc, vc, used
 
 
@@ -105,9 +110,15 @@ def gpu_decode_step(w, layer=0, partition_size=None, out=None, tables=None):
     """reshape_and_cache then paged_attention_decode on the GPU."""
     bt, cl, sm = tables if tables is not None else gpu_tables(w, w.queries[layer].device)
     kc, vc = w.key_caches[layer], w.value_caches[layer]
-    pkv.reshape_and_cache(w.new_keys[layer], w.new_values[layer], kc, vc, sm)
     if out is None:
         out = torch.empty_like(w.queries[layer])
+    if w.fp8:
+        ks, vs = w.extra["k_scale"], w.extra["v_scale"]
+        pkv.reshape_and_cache_fp8(w.new_keys[layer], w.new_values[layer], kc, vc, sm, ks, vs)
+        pkv.paged_attention_decode_fp8(out, w.queries[layer], kc, vc, bt, cl, w.scale, ks, vs, w.max_context_len,
+                                       partition_size=partition_size)
+        return out
+    pkv.reshape_and_cache(w.new_keys[layer], w.new_values[layer], kc, vc, sm)
     pkv.paged_attention_decode(out, w.queries[layer], kc, vc, bt, cl, w.scale, w.max_context_len,
                                partition_size=partition_size)
     return out
