@@ -186,12 +186,14 @@ class MixedStep(DecodeStep):
 
 class MultiTokenStep:
     """Multi-token decode (speculative verification): append each sequence's
-    draft tokens, then the causal attention of all of them over the cache in
-    one chunked-prefill call."""
+    draft tokens, then the causal attention of all of them over the cache
+    (``paged_attention_decode_multi``; ``via_prefill`` times the chunked-prefill
+    call on the same step instead)."""
 
-    def __init__(self, m):
+    def __init__(self, m, via_prefill=False):
         import paged_kv_cache_409_b200 as pkv
         self.pkv, self.m, self.w = pkv, m, m.decode
+        self.via_prefill = via_prefill
         dev = m.chunk_query.device
         self.aslots = torch.from_numpy(m.append_slots).to(dev)
         self.cbt = torch.from_numpy(m.chunk_tables).to(dev)
@@ -199,20 +201,29 @@ class MultiTokenStep:
         self.qsl = torch.from_numpy(m.query_start_loc).to(dev)
         self.out = torch.empty_like(m.chunk_query)
         self.max_q = int(m.chunk_lens.max())
-        self.layers, self.part = 1, 0
+        self.max_len = int(m.seq_lens.max())
         w = m.decode
+        R, Hkv, B = len(m.seq_lens), w.num_kv_heads, w.block_size
+        self.layers = 1
+        self.part = 0 if via_prefill else pkv.decode_multi_partition_size(R, Hkv, B, self.max_len)
+        Tq, Hq, D = m.chunk_query.shape
+        need = pkv.decode_workspace_size(Tq, Hq, D, self.max_len, self.part) if self.part else 0
+        self.ws = torch.empty(max(need, 16), dtype=torch.uint8, device=dev)
+        self.parts = -(-self.max_len // self.part) if self.part else 1
         t = m.chunk_query.element_size()
         self.kv_bytes = 2 * int(m.seq_lens.astype(np.int64).sum()) * w.num_kv_heads * w.head_dim * t
         nblocks = int(((m.seq_lens.astype(np.int64) + w.block_size - 1) // w.block_size).sum())
         self.decode_bytes = self.kv_bytes + 2 * m.chunk_query.numel() * t + 4 * nblocks + 8 * len(m.seq_lens)
         self.tokens = int(m.chunk_lens.sum())
-        self.kernel = "paged_attention_prefill_chunk (tcgen05)"
+        self.kernel = ("paged_attention_prefill_chunk (tcgen05)" if via_prefill else
+                       "paged_attention_decode_multi (multi-token decode + merge kernels)")
 
     def config(self):
         m = self.m
         return {"num_seqs": len(m.chunk_lens), "draft_tokens": self.tokens,
                 "draft_len_range": [int(m.chunk_lens.min()), int(m.chunk_lens.max())],
-                "context_range": [int(m.chunk_c0.min()), int(m.chunk_c0.max())]}
+                "context_range": [int(m.chunk_c0.min()), int(m.chunk_c0.max())],
+                "partition_size": self.part, "call": "prefill_chunk" if self.via_prefill else "decode_multi"}
 
     def oracle_sample(self, budget_s, max_seqs=8):
         """Oracle append + causal attention of the first sequences' drafts."""
@@ -232,7 +243,7 @@ class MultiTokenStep:
         return ntok * done / el, done, f"{len(chunks)} sequences ({ntok} draft tokens)", el
 
     def launches_per_step(self):
-        return 2
+        return 2 + (1 if self.parts > 1 else 0)
 
     def e2e_plan(self):
         m = self.m
@@ -245,8 +256,13 @@ class MultiTokenStep:
         self.pkv.reshape_and_cache(m.append_keys, m.append_values, w.key_caches[0], w.value_caches[0], self.aslots)
         if timer:
             timer.begin()
-        self.pkv.paged_attention_prefill_chunk(self.out, m.chunk_query, w.key_caches[0], w.value_caches[0],
-                                               self.cbt, self.csl, self.qsl, self.max_q, w.scale)
+        if self.via_prefill:
+            self.pkv.paged_attention_prefill_chunk(self.out, m.chunk_query, w.key_caches[0], w.value_caches[0],
+                                                   self.cbt, self.csl, self.qsl, self.max_q, w.scale)
+        else:
+            self.pkv.paged_attention_decode_multi(self.out, m.chunk_query, w.key_caches[0], w.value_caches[0],
+                                                  self.cbt, self.csl, self.qsl, self.max_q, self.max_len, w.scale,
+                                                  partition_size=self.part, workspace=self.ws)
         if timer:
             timer.end()
 
@@ -288,9 +304,10 @@ def make_step(name, device, rank, seqs=None, layers=None):
     if name == "mixed_step_bf16":
         m = workloads.mixed_step_bf16(device=device, seed=1005 + rank, num_decode=seqs or 192)
         return MixedStep(m), name + (f" ({seqs} decode sequences)" if seqs else "")
-    if name == "multi_token_decode_bf16":
+    if name in ("multi_token_decode_bf16", "multi_token_decode_bf16_via_prefill"):
         m = workloads.multi_token_decode_bf16(device=device, seed=1006 + rank, num_seqs=seqs or 64)
-        return MultiTokenStep(m), name + (f" ({seqs} sequences)" if seqs else "")
+        return MultiTokenStep(m, via_prefill=name.endswith("via_prefill")), name + (
+            f" ({seqs} sequences)" if seqs else "")
     raise SystemExit(f"unknown config {name}")
 
 

@@ -270,6 +270,43 @@ int pkv_paged_attention_prefill_chunk(void* out, const void* query, const void* 
                                       int dtype, pkv_stream_t stream);
 
 /*
+ * Multi-token decode: the chunked-prefill computation above for chunks of a
+ * few tokens -- a sequence that verifies n draft tokens in one pass (guide
+ * page "Speculative Decoding": a small draft model proposes the next tokens,
+ * e.g. --num-speculative-tokens 5, and the large model checks them at once).
+ * Row i of chunk r (its n_r tokens are the last of its seq_lens[r] cached
+ * tokens, written beforehand) attends causally to positions
+ * j <= seq_lens[r] - n_r + i, exactly as pkv_paged_attention_prefill_chunk.
+ * The n_r * G query rows that share a KV head go to the M side of warp
+ * tensor-core MMAs (16 rows per warp) and the K/V stream in 16-token units,
+ * split into partitions like decode (partials merged by a log-sum-exp kernel).
+ *
+ *   out, query, block_tables, seq_lens, query_start_loc   as for prefill_chunk
+ *   max_q_len       host bound on n_r; max_q_len * (num_q_heads / num_kv_heads)
+ *                   must be <= 32
+ *   max_seq_len     host bound on seq_lens (sizes the partitions)
+ *   partition_size  0 = one partition per chunk, else a multiple of block_size
+ *                   (pkv_decode_multi_partition_size recommends one)
+ *   workspace       >= pkv_decode_workspace_size(total_q_tokens, num_q_heads,
+ *                   head_dim, max_seq_len, partition_size) bytes
+ * Supported: dtype in {F16, BF16}; head_dim in {64, 128}; block_size in
+ * {8, 16, 32}; num_q_heads / num_kv_heads in {1, 2, 4, 8}.  A chunk whose n_r
+ * exceeds the row limit or its sequence is skipped and sets PKV_DEVERR_LENGTH.
+ */
+int pkv_paged_attention_decode_multi(void* out, const void* query, const void* key_cache, const void* value_cache,
+                                     const int32_t* block_tables, const int32_t* seq_lens,
+                                     const int32_t* query_start_loc, int num_chunks, int64_t total_q_tokens,
+                                     int max_q_len, int max_seq_len, float scale, int num_q_heads, int num_kv_heads,
+                                     int head_dim, int block_size, int max_blocks_per_seq, int64_t num_blocks,
+                                     int partition_size, int dtype, void* workspace, size_t workspace_bytes,
+                                     pkv_stream_t stream);
+
+/* Partition size (tokens) recommended for pkv_paged_attention_decode_multi:
+ * enough partitions for about eight CTAs per SM, at least 256 tokens each, a
+ * multiple of block_size; 0 = no split.  Negative pkv_status on bad input. */
+int pkv_decode_multi_partition_size(int num_chunks, int num_kv_heads, int block_size, int max_seq_len);
+
+/*
  * pkv_paged_attention_decode_static_scratch -- the same decode attention as
  * pkv_paged_attention_decode, for callers that cannot allocate device memory
  * at the call site (code running inside another framework's allocator, a

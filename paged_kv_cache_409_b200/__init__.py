@@ -8,6 +8,7 @@ load the library; the first call does, and fails loudly if it is missing.
 from ._binding import (  # noqa: F401
     PagedKVError,
     copy_blocks,
+    decode_multi_partition_size,
     decode_partition_size,
     decode_workspace_size,
     get_device_error,
@@ -15,6 +16,7 @@ from ._binding import (  # noqa: F401
     load_library,
     paged_attention_decode,
     paged_attention_decode_fp8,
+    paged_attention_decode_multi,
     paged_attention_prefill_chunk,
     reshape_and_cache,
     reshape_and_cache_fp8,

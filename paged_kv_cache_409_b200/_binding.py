@@ -40,6 +40,8 @@ EXPORTED = (
     "pkv_decode_workspace_size",
     "pkv_decode_partition_size",
     "pkv_paged_attention_prefill_chunk",
+    "pkv_paged_attention_decode_multi",
+    "pkv_decode_multi_partition_size",
     "pkv_get_device_error",
 )
 
@@ -81,10 +83,14 @@ def load_library():
     lib.pkv_decode_workspace_size.restype = SZ
     lib.pkv_decode_partition_size.argtypes = [I, I, I, I, I, I64, I]
     lib.pkv_paged_attention_prefill_chunk.argtypes = [P, P, P, P, P, P, P, I, I64, I, F, I, I, I, I, I, I64, I, P]
+    lib.pkv_paged_attention_decode_multi.argtypes = [P, P, P, P, P, P, P, I, I64, I, I, F, I, I, I, I, I, I64, I, I,
+                                                     P, SZ, P]
+    lib.pkv_decode_multi_partition_size.argtypes = [I, I, I, I]
     lib.pkv_get_device_error.argtypes = [ctypes.POINTER(ctypes.c_uint32), P]
     for name in ("pkv_reshape_and_cache", "pkv_reshape_and_cache_fp8", "pkv_paged_attention_decode_fp8",
                  "pkv_copy_blocks", "pkv_swap_blocks", "pkv_paged_attention_decode",
-                 "pkv_decode_partition_size", "pkv_paged_attention_prefill_chunk", "pkv_get_device_error"):
+                 "pkv_decode_partition_size", "pkv_paged_attention_prefill_chunk", "pkv_get_device_error",
+                 "pkv_paged_attention_decode_multi", "pkv_decode_multi_partition_size"):
         getattr(lib, name).restype = I
     _lib = lib
     return lib
@@ -280,6 +286,42 @@ def paged_attention_prefill_chunk(out, query, key_cache, value_cache, block_tabl
                                                R, Tq, int(max_q_len), float(scale), Hq, Hkv, D, B, MB, NB,
                                                _code(query), _stream(stream))
     _ok(rc, "paged_attention_prefill_chunk")
+    return out
+
+
+def decode_multi_partition_size(num_chunks, num_kv_heads, block_size, max_seq_len) -> int:
+    rc = load_library().pkv_decode_multi_partition_size(num_chunks, num_kv_heads, block_size, max_seq_len)
+    if rc < 0:
+        raise PagedKVError("decode_multi_partition_size", rc)
+    return rc
+
+
+def paged_attention_decode_multi(out, query, key_cache, value_cache, block_tables, seq_lens, query_start_loc,
+                                 max_q_len, max_seq_len, scale, partition_size=None, workspace=None, stream=None):
+    """Multi-token decode (a few causal query tokens per sequence); arguments as for
+    :func:`paged_attention_prefill_chunk` plus the host bound ``max_seq_len``."""
+    lib = load_library()
+    Tq, Hq, D = query.shape
+    NB, B, Hkv, _ = key_cache.shape
+    R = seq_lens.numel()
+    MB = block_tables.shape[1]
+    for t, name in ((block_tables, "block_tables"), (seq_lens, "seq_lens"), (query_start_loc, "query_start_loc")):
+        if t.dtype != torch.int32:
+            raise ValueError(f"{name} must be int32")
+    if partition_size is None:
+        partition_size = decode_multi_partition_size(R, Hkv, B, max_seq_len)
+    need = decode_workspace_size(Tq, Hq, D, max_seq_len, partition_size) if partition_size else 0
+    if need and (workspace is None or workspace.numel() * workspace.element_size() < need):
+        workspace = torch.empty(need, dtype=torch.uint8, device=query.device)
+    ws_ptr = _dev(workspace, "workspace") if (need and workspace is not None) else None
+    ws_bytes = workspace.numel() * workspace.element_size() if ws_ptr else 0
+    rc = lib.pkv_paged_attention_decode_multi(_dev(out, "out"), _dev(query, "query"), _dev(key_cache, "key_cache"),
+                                              _dev(value_cache, "value_cache"), _dev(block_tables, "block_tables"),
+                                              _dev(seq_lens, "seq_lens"), _dev(query_start_loc, "query_start_loc"),
+                                              R, Tq, int(max_q_len), int(max_seq_len), float(scale), Hq, Hkv, D, B,
+                                              MB, NB, int(partition_size), _code(query), ws_ptr, ws_bytes,
+                                              _stream(stream))
+    _ok(rc, "paged_attention_decode_multi")
     return out
 
 

@@ -21,6 +21,7 @@
 #include "decode.cuh"
 #include "decode_mma.cuh"
 #include "decode_fp8.cuh"
+#include "decode_multi.cuh"
 #include "prefill.cuh"
 
 namespace {
@@ -91,8 +92,9 @@ CUtensorMapDataType cu_type(int dtype) {
 #define PKV_FP8_L2_PROMOTION CU_TENSOR_MAP_L2_PROMOTION_L2_256B
 #endif
 
+// box_rows: tokens per box (the whole block by default).
 int make_pool_map(CUtensorMap* map, const void* pool, int dtype, int64_t num_blocks, int block_size,
-                  int num_kv_heads, int head_dim) {
+                  int num_kv_heads, int head_dim, int box_rows = 0) {
     auto fn = encode_fn();
     if (!fn) {
         snprintf(g_last_cuda_error, sizeof g_last_cuda_error, "cuTensorMapEncodeTiled unavailable");
@@ -103,7 +105,7 @@ int make_pool_map(CUtensorMap* map, const void* pool, int dtype, int64_t num_blo
                           (cuuint64_t)num_blocks};
     cuuint64_t strides[3] = {(cuuint64_t)head_dim * eb, (cuuint64_t)num_kv_heads * head_dim * eb,
                              (cuuint64_t)block_size * num_kv_heads * head_dim * eb};
-    cuuint32_t box[4] = {(cuuint32_t)(128 / eb), 1, (cuuint32_t)block_size, 1};
+    cuuint32_t box[4] = {(cuuint32_t)(128 / eb), 1, (cuuint32_t)(box_rows > 0 ? box_rows : block_size), 1};
     cuuint32_t estr[4] = {1, 1, 1, 1};
     const CUtensorMapL2promotion promo =
         dtype == PKV_FP8_E4M3 ? PKV_FP8_L2_PROMOTION : CU_TENSOR_MAP_L2_PROMOTION_L2_256B;
@@ -304,6 +306,52 @@ int decode_fp8_by_block(int block_size, int group, const pkv::DecodeParams& prm,
         case 8: return decode_fp8_by_group<T, 8>(group, prm, tk, tv, grid, s);
         case 16: return decode_fp8_by_group<T, 16>(group, prm, tk, tv, grid, s);
         case 32: return decode_fp8_by_group<T, 32>(group, prm, tk, tv, grid, s);
+        default: return PKV_EUNSUPPORTED;
+    }
+}
+
+// ------------------------------------------------------------ multi-token decode dispatch
+constexpr int kMultiWarps = 4;
+#ifndef PKV_MULTI_STAGE_BUDGET
+#define PKV_MULTI_STAGE_BUDGET 65536
+#endif
+
+template <typename T, int D, int B, int RG>
+int launch_multi(const pkv::MultiParams& prm, int group, const CUtensorMap& tk, const CUtensorMap& tv, int grid,
+                 cudaStream_t s) {
+    constexpr int UT = B < 16 ? B : 16;
+    constexpr int STAGE = 2 * UT * D * 2;
+    constexpr int NST = std::max(1, std::min(4, PKV_MULTI_STAGE_BUDGET / (kMultiWarps * STAGE)));
+    using C = pkv::MultiCfg<T, D, B, NST, kMultiWarps, RG>;
+    auto kern = pkv::paged_decode_multi_kernel<T, D, B, NST, kMultiWarps, RG>;
+    const size_t smem = C::smem_bytes(prm.partition_blocks);
+    int dev = 0;
+    PKV_CUDA(cudaGetDevice(&dev));
+    static size_t configured[64] = {};
+    size_t& have = configured[dev & 63];
+    if (smem > have) {
+        PKV_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
+        have = smem;
+    }
+    kern<<<grid, kMultiWarps * 32, smem, s>>>(prm, group, tk, tv);
+    PKV_CUDA(cudaGetLastError());
+    return PKV_OK;
+}
+
+template <typename T, int D, int B>
+int multi_by_rows(int row_groups, const pkv::MultiParams& prm, int group, const CUtensorMap& tk,
+                  const CUtensorMap& tv, int grid, cudaStream_t s) {
+    return row_groups == 1 ? launch_multi<T, D, B, 1>(prm, group, tk, tv, grid, s)
+                           : launch_multi<T, D, B, 2>(prm, group, tk, tv, grid, s);
+}
+
+template <typename T, int D>
+int multi_by_block(int block_size, int row_groups, const pkv::MultiParams& prm, int group, const CUtensorMap& tk,
+                   const CUtensorMap& tv, int grid, cudaStream_t s) {
+    switch (block_size) {
+        case 8: return multi_by_rows<T, D, 8>(row_groups, prm, group, tk, tv, grid, s);
+        case 16: return multi_by_rows<T, D, 16>(row_groups, prm, group, tk, tv, grid, s);
+        case 32: return multi_by_rows<T, D, 32>(row_groups, prm, group, tk, tv, grid, s);
         default: return PKV_EUNSUPPORTED;
     }
 }
@@ -772,6 +820,142 @@ int pkv_paged_attention_prefill_chunk(void* out, const void* query, const void* 
                     : prefill_by_group<__half, 64>(group, prm, tq, tk, tv, (int)grid, s);
     return bf16 ? prefill_by_group<__nv_bfloat16, 128>(group, prm, tq, tk, tv, (int)grid, s)
                 : prefill_by_group<__half, 128>(group, prm, tq, tk, tv, (int)grid, s);
+}
+
+int pkv_paged_attention_decode_multi(void* out, const void* query, const void* key_cache, const void* value_cache,
+                                     const int32_t* block_tables, const int32_t* seq_lens,
+                                     const int32_t* query_start_loc, int num_chunks, int64_t total_q_tokens,
+                                     int max_q_len, int max_seq_len, float scale, int num_q_heads, int num_kv_heads,
+                                     int head_dim, int block_size, int max_blocks_per_seq, int64_t num_blocks,
+                                     int partition_size, int dtype, void* workspace, size_t workspace_bytes,
+                                     pkv_stream_t stream) {
+    if (dtype != PKV_F16 && dtype != PKV_BF16) return PKV_EUNSUPPORTED;
+    if (num_chunks < 0 || total_q_tokens < 0 || max_q_len < 0 || max_seq_len < 0 || num_q_heads <= 0 ||
+        num_kv_heads <= 0 || max_blocks_per_seq <= 0 || num_blocks <= 0 || partition_size < 0 ||
+        !std::isfinite(scale))
+        return PKV_EINVAL;
+    if (num_q_heads % num_kv_heads) return PKV_EINVAL;
+    const int group = num_q_heads / num_kv_heads;
+    if (!supported_group(group) || (head_dim != 64 && head_dim != 128) ||
+        (block_size != 8 && block_size != 16 && block_size != 32))
+        return PKV_EUNSUPPORTED;
+    if ((int64_t)max_q_len * group > 32) return PKV_EUNSUPPORTED;  // at most two 16-row groups per KV head
+    if (partition_size % block_size) return PKV_EINVAL;
+    if (num_blocks >= (int64_t)INT32_MAX || (int64_t)max_blocks_per_seq * block_size > INT32_MAX ||
+        total_q_tokens > INT32_MAX)
+        return PKV_EINVAL;
+    if (num_chunks == 0 || total_q_tokens == 0 || max_q_len == 0) return PKV_OK;
+    if (!out || !query || !key_cache || !value_cache || !block_tables || !seq_lens || !query_start_loc)
+        return PKV_EINVAL;
+    if (!aligned16(out) || !aligned16(query) || !aligned16(key_cache) || !aligned16(value_cache) ||
+        (reinterpret_cast<uintptr_t>(block_tables) & 3) || (reinterpret_cast<uintptr_t>(seq_lens) & 3) ||
+        (reinterpret_cast<uintptr_t>(query_start_loc) & 3))
+        return PKV_EINVAL;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+
+    const int64_t max_blocks_needed = std::max<int64_t>(1, ceil_div(std::max(max_seq_len, 1), block_size));
+    int64_t pb = partition_size > 0 ? partition_size / block_size : max_blocks_needed;
+    pb = std::min(pb, max_blocks_needed);
+    const int64_t parts = ceil_div(max_blocks_needed, pb);
+    if (pb > 4096) return PKV_EUNSUPPORTED;
+    const size_t need = parts > 1 ? pkv_decode_workspace_size((int)total_q_tokens, num_q_heads, head_dim,
+                                                              max_seq_len, (int)(pb * block_size))
+                                  : 0;
+    if (need > 0 && (!workspace || workspace_bytes < need || !aligned16(workspace))) return PKV_EWORKSPACE;
+    const int64_t grid = (int64_t)num_chunks * parts * num_kv_heads;
+    if (grid > INT32_MAX) return PKV_EUNSUPPORTED;
+
+    if (checked_mode()) {
+        std::vector<int32_t> qsl, lens;
+        int rc = fetch(qsl, query_start_loc, (size_t)num_chunks + 1, s);
+        if (rc) return rc;
+        rc = fetch(lens, seq_lens, (size_t)num_chunks, s);
+        if (rc) return rc;
+        if (qsl[0] < 0 || qsl[num_chunks] > total_q_tokens) return PKV_ERANGE;
+        for (int r = 0; r < num_chunks; ++r) {
+            const int n = qsl[r + 1] - qsl[r];
+            if (n < 0 || n > max_q_len || lens[r] < n) return PKV_ERANGE;
+        }
+        rc = check_tables(block_tables, seq_lens, num_chunks, max_blocks_per_seq, block_size, num_blocks,
+                          max_seq_len, s);
+        if (rc) return rc;
+    }
+
+    const int unit_rows = block_size < 16 ? block_size : 16;
+    CUtensorMap tk, tv;
+    int rc = make_pool_map(&tk, key_cache, dtype, num_blocks, block_size, num_kv_heads, head_dim, unit_rows);
+    if (rc) return rc;
+    rc = make_pool_map(&tv, value_cache, dtype, num_blocks, block_size, num_kv_heads, head_dim, unit_rows);
+    if (rc) return rc;
+
+    pkv::MultiParams prm;
+    prm.out = out;
+    prm.query = query;
+    prm.block_tables = block_tables;
+    prm.seq_lens = seq_lens;
+    prm.query_start_loc = query_start_loc;
+    const int64_t rows = total_q_tokens * num_q_heads * parts;
+    const int64_t ml = ((rows * 4 + 15) / 16) * 16;
+    prm.ws_max = need ? reinterpret_cast<float*>(workspace) : nullptr;
+    prm.ws_sum = need ? reinterpret_cast<float*>(static_cast<char*>(workspace) + ml) : nullptr;
+    prm.ws_out = need ? reinterpret_cast<float*>(static_cast<char*>(workspace) + 2 * ml) : nullptr;
+    prm.scale_log2 = scale * 1.4426950408889634f;
+    prm.num_chunks = num_chunks;
+    prm.num_q_heads = num_q_heads;
+    prm.num_kv_heads = num_kv_heads;
+    prm.max_blocks_per_seq = max_blocks_per_seq;
+    prm.num_blocks = num_blocks;
+    prm.partition_blocks = (int)pb;
+    prm.num_partitions = (int)parts;
+    prm.total_q_tokens = total_q_tokens;
+    const int row_groups = max_q_len * group > 16 ? 2 : 1;
+    const bool bf16 = dtype == PKV_BF16;
+    if (head_dim == 64)
+        rc = bf16 ? multi_by_block<__nv_bfloat16, 64>(block_size, row_groups, prm, group, tk, tv, (int)grid, s)
+                  : multi_by_block<__half, 64>(block_size, row_groups, prm, group, tk, tv, (int)grid, s);
+    else
+        rc = bf16 ? multi_by_block<__nv_bfloat16, 128>(block_size, row_groups, prm, group, tk, tv, (int)grid, s)
+                  : multi_by_block<__half, 128>(block_size, row_groups, prm, group, tk, tv, (int)grid, s);
+    if (rc || parts <= 1) return rc;
+
+    pkv::MultiMergeParams mp;
+    mp.out = out;
+    mp.seq_lens = seq_lens;
+    mp.query_start_loc = query_start_loc;
+    mp.ws_max = prm.ws_max;
+    mp.ws_sum = prm.ws_sum;
+    mp.ws_out = prm.ws_out;
+    mp.num_chunks = num_chunks;
+    mp.num_q_heads = num_q_heads;
+    mp.total_q_tokens = total_q_tokens;
+    mp.block_size = block_size;
+    mp.max_blocks_per_seq = max_blocks_per_seq;
+    mp.partition_blocks = (int)pb;
+    mp.num_partitions = (int)parts;
+    const int64_t warps = total_q_tokens * num_q_heads;
+    const int mgrid = (int)ceil_div(warps, 4);
+    if (head_dim == 64) {
+        if (bf16) pkv::paged_decode_multi_merge_kernel<__nv_bfloat16, 64><<<mgrid, 128, 0, s>>>(mp);
+        else pkv::paged_decode_multi_merge_kernel<__half, 64><<<mgrid, 128, 0, s>>>(mp);
+    } else {
+        if (bf16) pkv::paged_decode_multi_merge_kernel<__nv_bfloat16, 128><<<mgrid, 128, 0, s>>>(mp);
+        else pkv::paged_decode_multi_merge_kernel<__half, 128><<<mgrid, 128, 0, s>>>(mp);
+    }
+    PKV_CUDA(cudaGetLastError());
+    return PKV_OK;
+}
+
+int pkv_decode_multi_partition_size(int num_chunks, int num_kv_heads, int block_size, int max_seq_len) {
+    if (num_chunks < 0 || num_kv_heads <= 0 || block_size <= 0 || max_seq_len < 0) return PKV_EINVAL;
+    const int64_t pairs = (int64_t)num_chunks * num_kv_heads;
+    if (max_seq_len <= 0 || pairs == 0) return 0;
+    // About eight CTAs per SM over the whole launch, so that CTAs of uneven
+    // length even out; partitions of at least 256 tokens.
+    const int64_t target = 8 * (int64_t)sm_count();
+    const int64_t parts = std::max<int64_t>(1, ceil_div(target, pairs));
+    int64_t ps = std::max<int64_t>(256, ceil_div(max_seq_len, parts));
+    ps = ceil_div(ps, block_size) * block_size;
+    return ps >= max_seq_len ? 0 : (int)ps;
 }
 
 int pkv_get_device_error(uint32_t* host_err, pkv_stream_t stream) {

@@ -1,6 +1,7 @@
 """Multi-token decode (speculative verification): every sequence appends a few
-draft tokens and each of them attends causally over the whole cache -- the
-chunked-prefill call with short chunks over long prior contexts."""
+draft tokens and each of them attends causally over the whole cache.  Both
+calls that compute it are checked: the chunked-prefill call (tcgen05) and the
+multi-token decode call (warp MMAs, split-K partitions)."""
 import numpy as np
 import pytest
 import torch
@@ -12,16 +13,19 @@ from parity_helpers import assert_close, oracle_prefill_chunks
 pytestmark = pytest.mark.gpu
 
 
-def run_gpu(m, dev="cuda"):
+def run_gpu(m, dev="cuda", call="prefill", partition_size=None):
     """Append every draft token, then the causal attention of all of them."""
     kc, vc = m.decode.key_caches[0].to(dev), m.decode.value_caches[0].to(dev)
     pkv.reshape_and_cache(m.append_keys.to(dev), m.append_values.to(dev), kc, vc,
                           torch.from_numpy(m.append_slots).to(dev))
     out = torch.empty_like(m.chunk_query, device=dev)
-    pkv.paged_attention_prefill_chunk(out, m.chunk_query.to(dev), kc, vc, torch.from_numpy(m.chunk_tables).to(dev),
-                                      torch.from_numpy(m.seq_lens).to(dev),
-                                      torch.from_numpy(m.query_start_loc).to(dev), int(m.chunk_lens.max()),
-                                      m.decode.scale)
+    args = (out, m.chunk_query.to(dev), kc, vc, torch.from_numpy(m.chunk_tables).to(dev),
+            torch.from_numpy(m.seq_lens).to(dev), torch.from_numpy(m.query_start_loc).to(dev),
+            int(m.chunk_lens.max()))
+    if call == "prefill":
+        pkv.paged_attention_prefill_chunk(*args, m.decode.scale)
+    else:
+        pkv.paged_attention_decode_multi(*args, int(m.seq_lens.max()), m.decode.scale, partition_size=partition_size)
     return out, kc, vc
 
 
@@ -30,43 +34,81 @@ CASES = [
     (torch.bfloat16, 128, 32, 32, 8, [0, 31, 32, 1000, 4093], [2, 3, 6, 5, 4]),
     (torch.float16, 128, 16, 8, 2, [15, 16, 17, 700], [6, 6, 2, 3]),
     (torch.bfloat16, 64, 8, 16, 16, [1, 63, 300], [2, 4, 6]),
-    (torch.float16, 64, 32, 8, 1, [129, 2048], [5, 2]),
+    (torch.float16, 64, 32, 8, 1, [129, 2048], [4, 2]),
 ]
 
 
+@pytest.mark.parametrize("call", ["prefill", "multi"])
 @pytest.mark.parametrize("case", CASES, ids=[f"case{i}" for i in range(len(CASES))])
-def test_multi_token_matches_oracle(case):
+def test_multi_token_matches_oracle(case, call):
     dtype, D, B, Hq, Hkv, c0s, ns = case
     m = workloads.mixed_workload("mt", [], c0s, ns, Hq, Hkv, D, B, dtype, seed=7 + sum(c0s) + D, poison=True)
     pre_k, pre_v = m.decode.key_caches[0].clone(), m.decode.value_caches[0].clone()
-    out, _, _ = run_gpu(m)
-    torch.cuda.synchronize()
-    assert pkv.get_device_error() == 0
     ref = oracle_prefill_chunks(m, pre_k, pre_v)
-    assert_close(out, ref, dtype, f"multi-token {case}")
+    parts = [None] if call == "prefill" else [0, B, 4 * B, None]
+    for part in parts:
+        out, _, _ = run_gpu(m, call=call, partition_size=part)
+        torch.cuda.synchronize()
+        assert pkv.get_device_error() == 0
+        assert_close(out, ref, dtype, f"multi-token {call} {case} partition {part}")
 
 
-def test_multi_token_full_size_sampled():
-    """The 64-sequence bf16 batch (drafts of 2..6 tokens, contexts 256..4096):
-    every row of six sampled sequences against the oracle."""
+# more rows than one warp's 16: two row groups (n * G up to 32), and one head per KV head with 16-token drafts
+ROW_CASES = [
+    (torch.bfloat16, 128, 16, 32, 8, [40, 1000, 3], [8, 5, 7]),
+    (torch.float16, 64, 32, 16, 16, [100, 31], [16, 9]),
+    (torch.bfloat16, 128, 8, 64, 8, [77, 500], [4, 3]),
+]
+
+
+@pytest.mark.parametrize("case", ROW_CASES, ids=[f"rows{i}" for i in range(len(ROW_CASES))])
+def test_multi_token_row_groups(case):
+    dtype, D, B, Hq, Hkv, c0s, ns = case
+    m = workloads.mixed_workload("mtr", [], c0s, ns, Hq, Hkv, D, B, dtype, seed=3 + sum(ns), poison=True)
+    pre_k, pre_v = m.decode.key_caches[0].clone(), m.decode.value_caches[0].clone()
+    ref = oracle_prefill_chunks(m, pre_k, pre_v)
+    for part in (0, 2 * B):
+        out, _, _ = run_gpu(m, call="multi", partition_size=part)
+        torch.cuda.synchronize()
+        assert pkv.get_device_error() == 0
+        assert_close(out, ref, dtype, f"multi-token rows {case} partition {part}")
+
+
+def test_multi_token_call_rejects_too_many_rows():
+    q = torch.zeros(9, 32, 128, device="cuda", dtype=torch.float16)  # 9 tokens x G 4 = 36 rows > 32
+    kc = torch.zeros(4, 16, 8, 128, device="cuda", dtype=torch.float16)
+    bt = torch.zeros(1, 4, dtype=torch.int32, device="cuda")
+    sl = torch.tensor([20], dtype=torch.int32, device="cuda")
+    qsl = torch.tensor([0, 9], dtype=torch.int32, device="cuda")
+    with pytest.raises(pkv.PagedKVError) as e:
+        pkv.paged_attention_decode_multi(torch.empty_like(q), q, kc, kc, bt, sl, qsl, 9, 20, 0.1)
+    assert e.value.status == -2
+
+
+@pytest.mark.parametrize("call", ["prefill", "multi"])
+def test_multi_token_full_size_sampled(call):
+    """The 64-sequence bf16 batch (drafts of 2..6 tokens, contexts 256..4096) in the
+    launch configuration the benchmark times: every row of six sampled sequences
+    against the oracle."""
     m = workloads.multi_token_decode_bf16(poison=True)
     pre_k, pre_v = m.decode.key_caches[0].clone(), m.decode.value_caches[0].clone()
-    out, _, _ = run_gpu(m)
+    out, _, _ = run_gpu(m, call=call)
     torch.cuda.synchronize()
     assert pkv.get_device_error() == 0
     chunks = np.array([0, 9, 21, 40, 52, 63])
     ref = oracle_prefill_chunks(m, pre_k, pre_v, chunks)
     qsl = m.query_start_loc
     rows = np.concatenate([np.arange(qsl[r], qsl[r + 1]) for r in chunks])
-    assert_close(out[torch.from_numpy(rows).cuda()], ref, torch.bfloat16, "multi-token 64 sequences")
+    assert_close(out[torch.from_numpy(rows).cuda()], ref, torch.bfloat16, f"multi-token 64 sequences ({call})")
 
 
-def test_multi_token_rows_equal_single_token_decode():
+@pytest.mark.parametrize("call", ["prefill", "multi"])
+def test_multi_token_rows_equal_single_token_decode(call):
     """Draft token i of a sequence sees exactly the first c0 + i + 1 tokens:
-    its row equals the one-token decode over that prefix (tensor-core prefill
-    path against the decode path, every row of the full-size batch)."""
+    its row equals the one-token decode over that prefix (every row of the
+    full-size batch, against the single-token decode path)."""
     m = workloads.multi_token_decode_bf16()
-    out, kc, vc = run_gpu(m)
+    out, kc, vc = run_gpu(m, call=call)
     R = len(m.chunk_lens)
     seq = np.repeat(np.arange(R), m.chunk_lens)
     pos = np.concatenate([m.chunk_c0[r] + np.arange(m.chunk_lens[r]) for r in range(R)])
