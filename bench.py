@@ -161,8 +161,16 @@ class MixedStep(DecodeStep):
         Hq, D = m.chunk_query.shape[1:]
         n, c0 = m.chunk_lens.astype(np.int64), m.chunk_c0.astype(np.int64)
         self.prefill_flops = int(4 * D * Hq * np.sum(n * c0 + n * (n + 1) // 2))
+        self.pws = None
+        if m.decode.fp8:
+            w = m.decode
+            need = self.pkv.prefill_fp8_workspace_size(len(n), m.chunk_tables.shape[1], w.block_size,
+                                                       w.num_kv_heads, D, m.chunk_query.shape[0], Hq, w.dtype)
+            self.pws = torch.empty(need, dtype=torch.uint8, device=dev)
 
     def launches_per_step(self):
+        if self.w.fp8:
+            return self.launches_per_step_fp8()
         return 3 + (1 if self.parts > 1 else 0)
 
     def e2e_plan(self):
@@ -172,11 +180,23 @@ class MixedStep(DecodeStep):
         outs = [(self.pout, pinned(self.pout)), (self.outs[0], pinned(self.outs[0]))]
         return E2EPlan(self, pairs, outs)
 
+    def launches_per_step_fp8(self):
+        return 4 + (1 if self.parts > 1 else 0)  # append, widen, query to f16, prefill, decode (+ merge)
+
     def run(self, timer=None, step=0):
         m, w = self.m, self.w
-        self.pkv.reshape_and_cache(m.append_keys, m.append_values, w.key_caches[0], w.value_caches[0], self.aslots)
-        self.pkv.paged_attention_prefill_chunk(self.pout, m.chunk_query, w.key_caches[0], w.value_caches[0],
-                                               self.cbt, self.csl, self.qsl, int(m.chunk_lens.max()), w.scale)
+        if w.fp8:
+            ks, vs = w.extra["k_scale"], w.extra["v_scale"]
+            self.pkv.reshape_and_cache_fp8(m.append_keys, m.append_values, w.key_caches[0], w.value_caches[0],
+                                           self.aslots, ks, vs)
+            self.pkv.paged_attention_prefill_chunk_fp8(self.pout, m.chunk_query, w.key_caches[0], w.value_caches[0],
+                                                       self.cbt, self.csl, self.qsl, int(m.chunk_lens.max()), w.scale,
+                                                       ks, vs, workspace=self.pws)
+        else:
+            self.pkv.reshape_and_cache(m.append_keys, m.append_values, w.key_caches[0], w.value_caches[0],
+                                       self.aslots)
+            self.pkv.paged_attention_prefill_chunk(self.pout, m.chunk_query, w.key_caches[0], w.value_caches[0],
+                                                   self.cbt, self.csl, self.qsl, int(m.chunk_lens.max()), w.scale)
         if timer:
             timer.begin()
         self.attend(0)
@@ -301,8 +321,9 @@ def make_step(name, device, rank, seqs=None, layers=None):
         st.pkv.reshape_and_cache(sp.private_keys, sp.private_values, kc, vc,
                                  torch.from_numpy(sp.private_slots).to(device))
         return st, name
-    if name == "mixed_step_bf16":
-        m = workloads.mixed_step_bf16(device=device, seed=1005 + rank, num_decode=seqs or 192)
+    if name in ("mixed_step_bf16", "mixed_step_fp8"):
+        make = workloads.mixed_step_bf16 if name == "mixed_step_bf16" else workloads.mixed_step_fp8
+        m = make(device=device, seed=1005 + rank, num_decode=seqs or 192)
         return MixedStep(m), name + (f" ({seqs} decode sequences)" if seqs else "")
     if name in ("multi_token_decode_bf16", "multi_token_decode_bf16_via_prefill"):
         m = workloads.multi_token_decode_bf16(device=device, seed=1006 + rank, num_seqs=seqs or 64)

@@ -270,6 +270,39 @@ int pkv_paged_attention_prefill_chunk(void* out, const void* query, const void* 
                                       int dtype, pkv_stream_t stream);
 
 /*
+ * Chunked prefill over FP8 (E4M3) pools: the computation of
+ * pkv_paged_attention_prefill_chunk with every pool element read as
+ * k_scale * e4m3(code) (K) or v_scale * e4m3(code) (V).  The prefill is bound
+ * by the tensor cores, not by HBM, so the blocks the chunks' tables name are
+ * first widened to f16 (exactly: every E4M3 value is an f16 value) into
+ * scratch pools in the workspace, a bf16 query is rounded to f16 there too
+ * (|query| must stay below 65504), and the tcgen05 prefill then runs in f16
+ * (weights P as one f16 term) with the scales folded into the score scale and
+ * the final normalisation; the output is written in dtype.
+ *
+ *   query, out      device, dtype F16 or BF16, layouts as for prefill_chunk
+ *   key_cache,
+ *   value_cache     device, one byte per element
+ *   workspace       >= pkv_prefill_fp8_workspace_size(...) bytes, 256-byte
+ *                   aligned; scratch after the call
+ * Every other argument and the supported shapes are those of
+ * pkv_paged_attention_prefill_chunk.
+ */
+int pkv_paged_attention_prefill_chunk_fp8(void* out, const void* query, const void* key_cache, const void* value_cache,
+                                          const int32_t* block_tables, const int32_t* seq_lens,
+                                          const int32_t* query_start_loc, int num_chunks, int64_t total_q_tokens,
+                                          int max_q_len, float scale, float k_scale, float v_scale, int num_q_heads,
+                                          int num_kv_heads, int head_dim, int block_size, int max_blocks_per_seq,
+                                          int64_t num_blocks, int dtype, void* workspace, size_t workspace_bytes,
+                                          pkv_stream_t stream);
+
+/* Workspace bytes of pkv_paged_attention_prefill_chunk_fp8: two f16 scratch
+ * pools of num_chunks * max_blocks_per_seq blocks, their table, and (bf16
+ * queries) the f16 query. */
+size_t pkv_prefill_fp8_workspace_size(int num_chunks, int max_blocks_per_seq, int block_size, int num_kv_heads,
+                                      int head_dim, int64_t total_q_tokens, int num_q_heads, int dtype);
+
+/*
  * Multi-token decode: the chunked-prefill computation above for chunks of a
  * few tokens -- a sequence that verifies n draft tokens in one pass (guide
  * page "Speculative Decoding": a small draft model proposes the next tokens,

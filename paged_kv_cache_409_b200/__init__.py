@@ -11,6 +11,7 @@ from ._binding import (  # noqa: F401
     decode_multi_partition_size,
     decode_partition_size,
     decode_workspace_size,
+    prefill_fp8_workspace_size,
     get_device_error,
     library_path,
     load_library,
@@ -18,6 +19,7 @@ from ._binding import (  # noqa: F401
     paged_attention_decode_fp8,
     paged_attention_decode_multi,
     paged_attention_prefill_chunk,
+    paged_attention_prefill_chunk_fp8,
     reshape_and_cache,
     reshape_and_cache_fp8,
     swap_blocks,

@@ -40,6 +40,8 @@ EXPORTED = (
     "pkv_decode_workspace_size",
     "pkv_decode_partition_size",
     "pkv_paged_attention_prefill_chunk",
+    "pkv_paged_attention_prefill_chunk_fp8",
+    "pkv_prefill_fp8_workspace_size",
     "pkv_paged_attention_decode_multi",
     "pkv_decode_multi_partition_size",
     "pkv_get_device_error",
@@ -86,11 +88,17 @@ def load_library():
     lib.pkv_paged_attention_decode_multi.argtypes = [P, P, P, P, P, P, P, I, I64, I, I, F, I, I, I, I, I, I64, I, I,
                                                      P, SZ, P]
     lib.pkv_decode_multi_partition_size.argtypes = [I, I, I, I]
+    lib.pkv_paged_attention_prefill_chunk_fp8.argtypes = [P, P, P, P, P, P, P, I, I64, I, F, F, F, I, I, I, I, I,
+                                                          I64, I, P, SZ, P]
+    lib.pkv_prefill_fp8_workspace_size.argtypes = [I, I, I, I, I, I64, I, I]
+    lib.pkv_prefill_fp8_workspace_size.restype = SZ
     lib.pkv_get_device_error.argtypes = [ctypes.POINTER(ctypes.c_uint32), P]
     for name in ("pkv_reshape_and_cache", "pkv_reshape_and_cache_fp8", "pkv_paged_attention_decode_fp8",
                  "pkv_copy_blocks", "pkv_swap_blocks", "pkv_paged_attention_decode",
                  "pkv_decode_partition_size", "pkv_paged_attention_prefill_chunk", "pkv_get_device_error",
-                 "pkv_paged_attention_decode_multi", "pkv_decode_multi_partition_size"):
+                 "pkv_paged_attention_prefill_chunk_fp8",
+    "pkv_prefill_fp8_workspace_size",
+    "pkv_paged_attention_decode_multi", "pkv_decode_multi_partition_size"):
         getattr(lib, name).restype = I
     _lib = lib
     return lib
@@ -286,6 +294,38 @@ def paged_attention_prefill_chunk(out, query, key_cache, value_cache, block_tabl
                                                R, Tq, int(max_q_len), float(scale), Hq, Hkv, D, B, MB, NB,
                                                _code(query), _stream(stream))
     _ok(rc, "paged_attention_prefill_chunk")
+    return out
+
+
+def prefill_fp8_workspace_size(num_chunks, max_blocks_per_seq, block_size, num_kv_heads, head_dim, total_q_tokens,
+                               num_q_heads, dtype) -> int:
+    code = DTYPE_CODE[dtype] if isinstance(dtype, torch.dtype) else int(dtype)
+    return int(load_library().pkv_prefill_fp8_workspace_size(num_chunks, max_blocks_per_seq, block_size,
+                                                             num_kv_heads, head_dim, int(total_q_tokens),
+                                                             num_q_heads, code))
+
+
+def paged_attention_prefill_chunk_fp8(out, query, key_cache, value_cache, block_tables, seq_lens, query_start_loc,
+                                      max_q_len, scale, k_scale, v_scale, workspace=None, stream=None):
+    """Causal chunked prefill over E4M3 pools (values ``k_scale * code``, ``v_scale * code``)."""
+    lib = load_library()
+    Tq, Hq, D = query.shape
+    NB, B, Hkv, _ = key_cache.shape
+    R = seq_lens.numel()
+    MB = block_tables.shape[1]
+    for t, name in ((block_tables, "block_tables"), (seq_lens, "seq_lens"), (query_start_loc, "query_start_loc")):
+        if t.dtype != torch.int32:
+            raise ValueError(f"{name} must be int32")
+    need = prefill_fp8_workspace_size(R, MB, B, Hkv, D, Tq, Hq, query.dtype)
+    if workspace is None or workspace.numel() * workspace.element_size() < need or workspace.data_ptr() % 256:
+        workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=query.device)
+    rc = lib.pkv_paged_attention_prefill_chunk_fp8(
+        _dev(out, "out"), _dev(query, "query"), _fp8_pool(key_cache, "key_cache"),
+        _fp8_pool(value_cache, "value_cache"), _dev(block_tables, "block_tables"), _dev(seq_lens, "seq_lens"),
+        _dev(query_start_loc, "query_start_loc"), R, Tq, int(max_q_len), float(scale), float(k_scale),
+        float(v_scale), Hq, Hkv, D, B, MB, NB, _code(query), _dev(workspace, "workspace"),
+        workspace.numel() * workspace.element_size(), _stream(stream))
+    _ok(rc, "paged_attention_prefill_chunk_fp8")
     return out
 
 

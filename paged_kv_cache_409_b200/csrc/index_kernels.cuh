@@ -106,6 +106,71 @@ __global__ void __launch_bounds__(128) reshape_and_cache_fp8_kernel(const TS* __
     }
 }
 
+// ---- widening of FP8 pools for the chunked prefill.
+// One CTA per block-table entry (chunk r, logical block b): the E4M3 codes of
+// that physical block's K and V are written as f16 (exact: every E4M3 value is
+// an f16 value) to block r * max_blocks + b of two f16 scratch pools, and the
+// scratch table entry is that index (-1 for blocks past the sequence or with
+// an id outside the pool, which also sets PKV_DEVERR_BLOCK_ID).
+__device__ __forceinline__ void widen16(const uint4 x, uint4& lo, uint4& hi) {
+    lo.x = f16x2_from_e4m3x2(static_cast<uint16_t>(x.x));
+    lo.y = f16x2_from_e4m3x2(static_cast<uint16_t>(x.x >> 16));
+    lo.z = f16x2_from_e4m3x2(static_cast<uint16_t>(x.y));
+    lo.w = f16x2_from_e4m3x2(static_cast<uint16_t>(x.y >> 16));
+    hi.x = f16x2_from_e4m3x2(static_cast<uint16_t>(x.z));
+    hi.y = f16x2_from_e4m3x2(static_cast<uint16_t>(x.z >> 16));
+    hi.z = f16x2_from_e4m3x2(static_cast<uint16_t>(x.w));
+    hi.w = f16x2_from_e4m3x2(static_cast<uint16_t>(x.w >> 16));
+}
+
+__global__ void __launch_bounds__(256) widen_fp8_blocks_kernel(const uint4* __restrict__ kc8,
+                                                               const uint4* __restrict__ vc8,
+                                                               uint4* __restrict__ kc16, uint4* __restrict__ vc16,
+                                                               const int32_t* __restrict__ block_tables,
+                                                               const int32_t* __restrict__ seq_lens,
+                                                               int32_t* __restrict__ tables_out, int max_blocks,
+                                                               int block_size, int64_t num_blocks, int block_vecs) {
+    const int64_t e = blockIdx.x;
+    const int64_t r = e / max_blocks;
+    const int b = static_cast<int>(e - r * max_blocks);
+    const int len = max(seq_lens[r], 0);
+    const int nblk = min((len + block_size - 1) / block_size, max_blocks);
+    int id = -1;
+    if (b < nblk) {
+        id = block_tables[e];
+        if (id < 0 || id >= num_blocks) {
+            if (threadIdx.x == 0) flag_error(PKV_DEVERR_BLOCK_ID);
+            id = -1;
+        }
+    }
+    if (threadIdx.x == 0) tables_out[e] = id >= 0 ? static_cast<int32_t>(e) : -1;
+    if (id < 0) return;
+    const uint4* ks = kc8 + static_cast<int64_t>(id) * block_vecs;
+    const uint4* vs = vc8 + static_cast<int64_t>(id) * block_vecs;
+    uint4* kd = kc16 + e * 2 * block_vecs;
+    uint4* vd = vc16 + e * 2 * block_vecs;
+    for (int i = threadIdx.x; i < block_vecs; i += blockDim.x) {
+        const uint4 a = ks[i], c = vs[i];
+        uint4 lo, hi;
+        widen16(a, lo, hi);
+        kd[2 * i] = lo;
+        kd[2 * i + 1] = hi;
+        widen16(c, lo, hi);
+        vd[2 * i] = lo;
+        vd[2 * i + 1] = hi;
+    }
+}
+
+// bf16 -> f16, round to nearest even (grid-stride over pairs).
+__global__ void __launch_bounds__(256) bf16_to_f16_kernel(const uint32_t* __restrict__ src, uint32_t* __restrict__ dst,
+                                                          int64_t pairs) {
+    for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < pairs;
+         i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+        const float2 f = Elem<__nv_bfloat16>::pair(src[i]);
+        dst[i] = pack_half2(f.x, f.y);
+    }
+}
+
 constexpr int kMaxLayersPerLaunch = 32;
 
 struct LayerPools {

@@ -373,11 +373,11 @@ bool supported_group(int g) { return g == 1 || g == 2 || g == 4 || g == 8; }
 int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
 
 // ------------------------------------------------------------ prefill dispatch
-template <typename T, int D, int G>
+template <typename T, int D, int G, typename TO = T>
 int launch_prefill(const pkv::PrefillParams& prm, const CUtensorMap& tq, const CUtensorMap& tk,
                    const CUtensorMap& tv, int grid, cudaStream_t s) {
     using C = pkv::PrefillCfg<T, D, G>;
-    auto kern = pkv::paged_prefill_kernel<T, D, G>;
+    auto kern = pkv::paged_prefill_kernel<T, D, G, TO>;
     int dev = 0;
     PKV_CUDA(cudaGetDevice(&dev));
     static bool configured[64] = {};
@@ -390,14 +390,14 @@ int launch_prefill(const pkv::PrefillParams& prm, const CUtensorMap& tq, const C
     return PKV_OK;
 }
 
-template <typename T, int D>
+template <typename T, int D, typename TO = T>
 int prefill_by_group(int group, const pkv::PrefillParams& prm, const CUtensorMap& tq, const CUtensorMap& tk,
                      const CUtensorMap& tv, int grid, cudaStream_t s) {
     switch (group) {
-        case 1: return launch_prefill<T, D, 1>(prm, tq, tk, tv, grid, s);
-        case 2: return launch_prefill<T, D, 2>(prm, tq, tk, tv, grid, s);
-        case 4: return launch_prefill<T, D, 4>(prm, tq, tk, tv, grid, s);
-        case 8: return launch_prefill<T, D, 8>(prm, tq, tk, tv, grid, s);
+        case 1: return launch_prefill<T, D, 1, TO>(prm, tq, tk, tv, grid, s);
+        case 2: return launch_prefill<T, D, 2, TO>(prm, tq, tk, tv, grid, s);
+        case 4: return launch_prefill<T, D, 4, TO>(prm, tq, tk, tv, grid, s);
+        case 8: return launch_prefill<T, D, 8, TO>(prm, tq, tk, tv, grid, s);
         default: return PKV_EUNSUPPORTED;
     }
 }
@@ -814,6 +814,7 @@ int pkv_paged_attention_prefill_chunk(void* out, const void* query, const void* 
     prm.block_size = block_size;
     prm.num_blocks = num_blocks;
     prm.q_tiles = (int)q_tiles;
+    prm.out_scale = 1.f;
     const bool bf16 = dtype == PKV_BF16;
     if (head_dim == 64)
         return bf16 ? prefill_by_group<__nv_bfloat16, 64>(group, prm, tq, tk, tv, (int)grid, s)
@@ -956,6 +957,123 @@ int pkv_decode_multi_partition_size(int num_chunks, int num_kv_heads, int block_
     int64_t ps = std::max<int64_t>(256, ceil_div(max_seq_len, parts));
     ps = ceil_div(ps, block_size) * block_size;
     return ps >= max_seq_len ? 0 : (int)ps;
+}
+
+size_t pkv_prefill_fp8_workspace_size(int num_chunks, int max_blocks_per_seq, int block_size, int num_kv_heads,
+                                      int head_dim, int64_t total_q_tokens, int num_q_heads, int dtype) {
+    if (num_chunks <= 0 || max_blocks_per_seq <= 0 || block_size <= 0 || num_kv_heads <= 0 || head_dim <= 0 ||
+        total_q_tokens < 0 || num_q_heads <= 0)
+        return 0;
+    auto al = [](int64_t x) { return ((x + 1023) / 1024) * 1024; };
+    const int64_t entries = (int64_t)num_chunks * max_blocks_per_seq;
+    const int64_t pool = entries * block_size * num_kv_heads * head_dim * 2;
+    const int64_t q = dtype == PKV_BF16 ? total_q_tokens * num_q_heads * head_dim * 2 : 0;
+    return (size_t)(al(q) + 2 * al(pool) + al(entries * 4));
+}
+
+int pkv_paged_attention_prefill_chunk_fp8(void* out, const void* query, const void* key_cache, const void* value_cache,
+                                          const int32_t* block_tables, const int32_t* seq_lens,
+                                          const int32_t* query_start_loc, int num_chunks, int64_t total_q_tokens,
+                                          int max_q_len, float scale, float k_scale, float v_scale, int num_q_heads,
+                                          int num_kv_heads, int head_dim, int block_size, int max_blocks_per_seq,
+                                          int64_t num_blocks, int dtype, void* workspace, size_t workspace_bytes,
+                                          pkv_stream_t stream) {
+    if (dtype != PKV_F16 && dtype != PKV_BF16) return PKV_EUNSUPPORTED;
+    if (num_chunks < 0 || total_q_tokens < 0 || max_q_len < 0 || num_q_heads <= 0 || num_kv_heads <= 0 ||
+        max_blocks_per_seq <= 0 || num_blocks <= 0 || !std::isfinite(scale))
+        return PKV_EINVAL;
+    if (!(std::isfinite(k_scale) && k_scale > 0.f && std::isfinite(v_scale) && v_scale > 0.f)) return PKV_EINVAL;
+    if (num_q_heads % num_kv_heads) return PKV_EINVAL;
+    const int group = num_q_heads / num_kv_heads;
+    if (!supported_group(group) || (head_dim != 64 && head_dim != 128) ||
+        (block_size != 8 && block_size != 16 && block_size != 32))
+        return PKV_EUNSUPPORTED;
+    const int64_t entries = (int64_t)num_chunks * max_blocks_per_seq;
+    if (entries >= (int64_t)INT32_MAX || (int64_t)max_blocks_per_seq * block_size > INT32_MAX ||
+        total_q_tokens > INT32_MAX || num_blocks >= (int64_t)INT32_MAX)
+        return PKV_EINVAL;
+    if (num_chunks == 0 || total_q_tokens == 0 || max_q_len == 0) return PKV_OK;
+    if (!out || !query || !key_cache || !value_cache || !block_tables || !seq_lens || !query_start_loc)
+        return PKV_EINVAL;
+    if (!aligned16(out) || !aligned16(query) || !aligned16(key_cache) || !aligned16(value_cache) ||
+        (reinterpret_cast<uintptr_t>(block_tables) & 3) || (reinterpret_cast<uintptr_t>(seq_lens) & 3) ||
+        (reinterpret_cast<uintptr_t>(query_start_loc) & 3))
+        return PKV_EINVAL;
+    const size_t need = pkv_prefill_fp8_workspace_size(num_chunks, max_blocks_per_seq, block_size, num_kv_heads,
+                                                       head_dim, total_q_tokens, num_q_heads, dtype);
+    if (!workspace || workspace_bytes < need || (reinterpret_cast<uintptr_t>(workspace) & 255))
+        return PKV_EWORKSPACE;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (checked_mode()) {
+        std::vector<int32_t> qsl, lens;
+        int rc = fetch(qsl, query_start_loc, (size_t)num_chunks + 1, s);
+        if (rc) return rc;
+        rc = fetch(lens, seq_lens, (size_t)num_chunks, s);
+        if (rc) return rc;
+        if (qsl[0] < 0 || qsl[num_chunks] > total_q_tokens) return PKV_ERANGE;
+        for (int r = 0; r < num_chunks; ++r) {
+            const int n = qsl[r + 1] - qsl[r];
+            if (n < 0 || n > max_q_len || lens[r] < n) return PKV_ERANGE;
+        }
+        rc = check_tables(block_tables, seq_lens, num_chunks, max_blocks_per_seq, block_size, num_blocks,
+                          (int64_t)max_blocks_per_seq * block_size, s);
+        if (rc) return rc;
+    }
+    // workspace: [f16 query (bf16 input only)] [f16 K scratch pool] [f16 V scratch pool] [scratch tables]
+    auto al = [](int64_t x) { return ((x + 1023) / 1024) * 1024; };
+    const int64_t pool = entries * block_size * num_kv_heads * head_dim * 2;
+    const int64_t qbytes = dtype == PKV_BF16 ? total_q_tokens * num_q_heads * head_dim * 2 : 0;
+    char* ws = static_cast<char*>(workspace);
+    void* q16 = dtype == PKV_BF16 ? (void*)ws : const_cast<void*>(query);
+    void* k16 = ws + al(qbytes);
+    void* v16 = ws + al(qbytes) + al(pool);
+    int32_t* bt16 = reinterpret_cast<int32_t*>(ws + al(qbytes) + 2 * al(pool));
+    const int block_vecs = block_size * num_kv_heads * head_dim / 16;  // 16-byte vectors of codes per block
+    pkv::widen_fp8_blocks_kernel<<<(unsigned)entries, 256, 0, s>>>(
+        static_cast<const uint4*>(key_cache), static_cast<const uint4*>(value_cache), static_cast<uint4*>(k16),
+        static_cast<uint4*>(v16), block_tables, seq_lens, bt16, max_blocks_per_seq, block_size, num_blocks,
+        block_vecs);
+    PKV_CUDA(cudaGetLastError());
+    if (dtype == PKV_BF16) {
+        const int64_t pairs = total_q_tokens * num_q_heads * head_dim / 2;
+        const unsigned g = (unsigned)std::min<int64_t>(ceil_div(pairs, 256), 4 * (int64_t)sm_count());
+        pkv::bf16_to_f16_kernel<<<g, 256, 0, s>>>(static_cast<const uint32_t*>(query), static_cast<uint32_t*>(q16),
+                                                   pairs);
+        PKV_CUDA(cudaGetLastError());
+    }
+
+    CUtensorMap tq, tk, tv;
+    int rc = make_query_map(&tq, q16, PKV_F16, total_q_tokens, num_q_heads, head_dim, group);
+    if (rc) return rc;
+    rc = make_pool_map(&tk, k16, PKV_F16, entries, block_size, num_kv_heads, head_dim);
+    if (rc) return rc;
+    rc = make_pool_map(&tv, v16, PKV_F16, entries, block_size, num_kv_heads, head_dim);
+    if (rc) return rc;
+
+    const int tile_tokens = 128 / group;
+    const int64_t q_tiles = ceil_div(max_q_len, tile_tokens);
+    const int64_t grid = (int64_t)num_chunks * q_tiles * num_kv_heads;
+    if (grid > INT32_MAX) return PKV_EUNSUPPORTED;
+    pkv::PrefillParams prm;
+    prm.out = out;
+    prm.block_tables = bt16;
+    prm.seq_lens = seq_lens;
+    prm.query_start_loc = query_start_loc;
+    prm.scale_log2 = scale * 1.4426950408889634f * k_scale;
+    prm.out_scale = v_scale;
+    prm.num_chunks = num_chunks;
+    prm.num_q_heads = num_q_heads;
+    prm.num_kv_heads = num_kv_heads;
+    prm.max_blocks_per_seq = max_blocks_per_seq;
+    prm.block_size = block_size;
+    prm.num_blocks = entries;
+    prm.q_tiles = (int)q_tiles;
+    const bool bf16 = dtype == PKV_BF16;
+    if (head_dim == 64)
+        return bf16 ? prefill_by_group<__half, 64, __nv_bfloat16>(group, prm, tq, tk, tv, (int)grid, s)
+                    : prefill_by_group<__half, 64>(group, prm, tq, tk, tv, (int)grid, s);
+    return bf16 ? prefill_by_group<__half, 128, __nv_bfloat16>(group, prm, tq, tk, tv, (int)grid, s)
+                : prefill_by_group<__half, 128>(group, prm, tq, tk, tv, (int)grid, s);
 }
 
 int pkv_get_device_error(uint32_t* host_err, pkv_stream_t stream) {

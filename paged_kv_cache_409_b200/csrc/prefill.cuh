@@ -41,7 +41,8 @@ struct PrefillParams {
     const int32_t* block_tables;
     const int32_t* seq_lens;
     const int32_t* query_start_loc;
-    float scale_log2;
+    float scale_log2;  // scale * log2(e) (times the K pool's scale for widened FP8 pools)
+    float out_scale;   // the V pool's scale for widened FP8 pools, else 1
     int num_chunks;
     int num_q_heads;
     int num_kv_heads;
@@ -85,7 +86,8 @@ struct PrefillCfg {
     static_assert(D == 64 || D == 128, "head_dim");
 };
 
-template <typename T, int D, int G>
+// T: the type of the query and the K/V tiles the MMAs read; TO: the output's.
+template <typename T, int D, int G, typename TO = T>
 __global__ void __launch_bounds__(kPrefillThreads, 1) paged_prefill_kernel(const PrefillParams p,
                                                                          const __grid_constant__ CUtensorMap tm_q,
                                                                          const __grid_constant__ CUtensorMap tm_k,
@@ -451,17 +453,17 @@ __global__ void __launch_bounds__(kPrefillThreads, 1) paged_prefill_kernel(const
         float lother = 0.f;
         if (ok && !exchange(lsum, nkt, lother)) ok = false;
         if (ok && !*abort_flag && tok < n) {
-            const float inv = 1.f / (lsum + lother);
-            T* dst = reinterpret_cast<T*>(p.out) +
+            const float inv = p.out_scale / (lsum + lother);
+            TO* dst = reinterpret_cast<TO*>(p.out) +
                      (static_cast<int64_t>(q0 + tok) * p.num_q_heads + static_cast<int64_t>(g) * G + row % G) * D +
                      half * HD;
 #pragma unroll
             for (int d = 0; d < HD; d += 8) {
                 uint4 w;
-                w.x = Elem<T>::pack(o[d] * inv, o[d + 1] * inv);
-                w.y = Elem<T>::pack(o[d + 2] * inv, o[d + 3] * inv);
-                w.z = Elem<T>::pack(o[d + 4] * inv, o[d + 5] * inv);
-                w.w = Elem<T>::pack(o[d + 6] * inv, o[d + 7] * inv);
+                w.x = Elem<TO>::pack(o[d] * inv, o[d + 1] * inv);
+                w.y = Elem<TO>::pack(o[d + 2] * inv, o[d + 3] * inv);
+                w.z = Elem<TO>::pack(o[d + 4] * inv, o[d + 5] * inv);
+                w.w = Elem<TO>::pack(o[d + 6] * inv, o[d + 7] * inv);
                 *reinterpret_cast<uint4*>(dst + d) = w;
             }
         }

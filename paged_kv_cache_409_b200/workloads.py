@@ -356,7 +356,9 @@ class MixedWorkload:
 
 
 def mixed_workload(name, decode_lens, chunk_c0, chunk_lens, num_q_heads, num_kv_heads, head_dim, block_size,
-                   dtype, *, seed, device="cpu", poison=False):
+                   dtype, *, seed, device="cpu", poison=False, fp8_scales=None):
+    """``fp8_scales=(k_scale, v_scale)`` makes the pools uint8 E4M3 codes of
+    N(0, 1) / scale; queries and appended tokens stay in ``dtype``."""
     rng = np.random.default_rng(seed)
     gen = _gen(seed, device)
     B = block_size
@@ -370,8 +372,12 @@ def mixed_workload(name, decode_lens, chunk_c0, chunk_lens, num_q_heads, num_kv_
     bt_all, _ = place_blocks(rng, bps, nb)
     dbt, cbt = bt_all[:S].copy(), bt_all[S:].copy()
     Hkv, D = num_kv_heads, head_dim
-    kc = randn((nb, B, Hkv, D), dtype, gen, device)
-    vc = randn((nb, B, Hkv, D), dtype, gen, device)
+    if fp8_scales is None:
+        kc = randn((nb, B, Hkv, D), dtype, gen, device)
+        vc = randn((nb, B, Hkv, D), dtype, gen, device)
+    else:
+        kc = randn_e4m3((nb, B, Hkv, D), fp8_scales[0], gen, device)
+        vc = randn_e4m3((nb, B, Hkv, D), fp8_scales[1], gen, device)
     dq = randn((S, num_q_heads, D), dtype, gen, device)
     cq = randn((int(n.sum()), num_q_heads, D), dtype, gen, device)
     ak = randn((S + int(n.sum()), Hkv, D), dtype, gen, device)
@@ -385,8 +391,10 @@ def mixed_workload(name, decode_lens, chunk_c0, chunk_lens, num_q_heads, num_kv_
         for c in (kc, vc):
             poison_pool(c, keep)
     qsl = np.concatenate([[0], np.cumsum(n)]).astype(np.int32)
+    extra = {} if fp8_scales is None else {"k_scale": float(np.float32(fp8_scales[0])),
+                                           "v_scale": float(np.float32(fp8_scales[1]))}
     dec = DecodeWorkload(name, S, num_q_heads, Hkv, D, B, dtype, float(np.float32(1.0 / math.sqrt(D))), nb,
-                         dl.astype(np.int32), dbt, dslots, [kc], [vc], [dq], [ak[:S]], [av[:S]])
+                         dl.astype(np.int32), dbt, dslots, [kc], [vc], [dq], [ak[:S]], [av[:S]], extra)
     return MixedWorkload(dec, n.astype(np.int32), c0.astype(np.int32), cbt, cq, qsl, sl.astype(np.int32), ak, av,
                          np.concatenate([dslots, cslots]).astype(np.int64))
 
@@ -402,6 +410,18 @@ def mixed_step_bf16(device="cpu", num_decode=192, num_chunks=4, chunk_len=512, p
     n = np.full(num_chunks, chunk_len)
     return mixed_workload("mixed_step_bf16", dl, c0, n, 32, 8, 128, 32, torch.bfloat16, seed=seed, device=device,
                           poison=poison)
+
+
+def mixed_step_fp8(device="cpu", num_decode=192, num_chunks=4, chunk_len=512, poison=False, seed=1005,
+                   decode_lo=256, decode_hi=32768, c0_hi=8192):
+    """The mixed step (192 decode sequences + 4 prefill chunks of 512, 32 q
+    heads over 8 KV heads, d 128, block 32, bf16 queries) on E4M3 pools."""
+    rng = np.random.default_rng(seed)
+    dl = rng.integers(decode_lo, decode_hi + 1, size=num_decode)
+    c0 = rng.integers(0, c0_hi + 1, size=num_chunks)
+    n = np.full(num_chunks, chunk_len)
+    return mixed_workload("mixed_step_fp8", dl, c0, n, 32, 8, 128, 32, torch.bfloat16, seed=seed, device=device,
+                          poison=poison, fp8_scales=(FP8_K_SCALE, FP8_V_SCALE))
 
 
 def multi_token_decode_bf16(device="cpu", num_seqs=64, draft_lo=2, draft_hi=6, c0_lo=256, c0_hi=4096,
@@ -425,5 +445,6 @@ CONFIGS = {
     "mixed_step_bf16": mixed_step_bf16,
     "multi_token_decode_bf16": multi_token_decode_bf16,
     "llama7b_decode_fp8": llama7b_decode_fp8,
+    "mixed_step_fp8": mixed_step_fp8,
     "gqa70b_decode_fp8": gqa70b_decode_fp8,
 }

@@ -148,10 +148,16 @@ def oracle_prefill_chunks(m, pre_k, pre_v, chunks=None, row_select=None):
     slots = np.array([remap[int(x) // B] * B + int(x) % B for x in cslots], dtype=np.int64)
     orc = oracle.get()
     idx = torch.from_numpy(src)
-    orc.reshape_and_cache(oracle.storage(m.append_keys.cpu()[idx])[0], oracle.storage(m.append_values.cpu()[idx])[0],
-                          kn, vn, slots, code)
+    ak, acode = oracle.storage(m.append_keys.cpu()[idx])
+    av, _ = oracle.storage(m.append_values.cpu()[idx])
     n = m.chunk_lens[chunks].astype(np.int64)
     new_qsl = np.concatenate([[0], np.cumsum(n)]).astype(np.int32)
-    q = oracle.storage(m.chunk_query.cpu()[torch.from_numpy(rows)])[0]
+    q, qcode = oracle.storage(m.chunk_query.cpu()[torch.from_numpy(rows)])
+    if m.decode.fp8:
+        ks, vs = m.decode.extra["k_scale"], m.decode.extra["v_scale"]
+        orc.reshape_and_cache_fp8(ak, av, kn, vn, slots, acode, ks, vs)
+        return orc.paged_attention_prefill_chunk_kv(q, qcode, kn, vn, oracle.E4M3, ks, vs, bt, lens, new_qsl,
+                                                    m.decode.scale, row_select=row_select)
+    orc.reshape_and_cache(ak, av, kn, vn, slots, code)
     return orc.paged_attention_prefill_chunk(q, kn, vn, bt, lens, new_qsl, m.decode.scale, code,
                                              row_select=row_select)

@@ -8,7 +8,8 @@ import torch
 import oracle
 import paged_kv_cache_409_b200 as pkv
 from paged_kv_cache_409_b200 import workloads
-from parity_helpers import assert_close, gpu_decode_step, gpu_tables, oracle_decode_step, to_device
+from parity_helpers import assert_close, gpu_decode_step, gpu_tables, oracle_decode_step, oracle_prefill_chunks, \
+    to_device
 
 pytestmark = pytest.mark.gpu
 
@@ -153,3 +154,50 @@ def test_gqa70b_decode_fp8_one_layer_sampled():
     seqs = np.concatenate([order[:3], order[-3:], [100, 200]])
     ref, _, _, _ = oracle_decode_step(w, seqs=seqs, pre_k=pre_k.cpu(), pre_v=pre_v.cpu())
     assert_close(out[torch.from_numpy(seqs).cuda()], ref, torch.bfloat16, "gqa70b fp8")
+
+
+PREFILL_CASES = [
+    # dtype, D, B, Hq, Hkv, c0s, ns
+    (torch.bfloat16, 128, 32, 32, 8, [0, 300], [512, 77]),
+    (torch.float16, 128, 16, 8, 8, [5, 0, 129], [1, 130, 128]),
+    (torch.bfloat16, 64, 8, 16, 2, [1000, 0], [33, 257]),
+    (torch.float16, 64, 16, 4, 2, [17], [300]),
+    (torch.bfloat16, 128, 16, 16, 2, [255, 64], [200, 16]),
+]
+
+
+@pytest.mark.parametrize("case", PREFILL_CASES, ids=[f"case{i}" for i in range(len(PREFILL_CASES))])
+def test_fp8_prefill_matches_oracle(case):
+    """Quantising append of every chunk token, then chunked prefill over the E4M3 pools."""
+    dtype, D, B, Hq, Hkv, c0s, ns = case
+    m = workloads.mixed_workload("p8", [], c0s, ns, Hq, Hkv, D, B, dtype, seed=sum(c0s) + sum(ns) + D + B,
+                                 poison=True, fp8_scales=(0.0119, 0.0143))
+    w = m.decode
+    pre_k, pre_v = w.key_caches[0].clone(), w.value_caches[0].clone()
+    ref = oracle_prefill_chunks(m, pre_k, pre_v)
+    dev = "cuda"
+    kc, vc = pre_k.to(dev), pre_v.to(dev)
+    ks, vs = w.extra["k_scale"], w.extra["v_scale"]
+    pkv.reshape_and_cache_fp8(m.append_keys.to(dev), m.append_values.to(dev), kc, vc,
+                              torch.from_numpy(m.append_slots).to(dev), ks, vs)
+    out = torch.empty_like(m.chunk_query, device=dev)
+    pkv.paged_attention_prefill_chunk_fp8(out, m.chunk_query.to(dev), kc, vc, torch.from_numpy(m.chunk_tables).to(dev),
+                                          torch.from_numpy(m.seq_lens).to(dev),
+                                          torch.from_numpy(m.query_start_loc).to(dev), int(m.chunk_lens.max()),
+                                          w.scale, ks, vs)
+    torch.cuda.synchronize()
+    assert pkv.get_device_error() == 0
+    assert_close(out, ref, dtype, f"fp8 prefill {case}")
+
+
+def test_fp8_prefill_rejects_small_workspace():
+    q = torch.zeros(4, 2, 64, device="cuda", dtype=torch.float16)
+    kc = torch.zeros(2, 16, 2, 64, device="cuda", dtype=torch.uint8)
+    i32 = torch.zeros(2, dtype=torch.int32, device="cuda")
+    ws = torch.empty(1024, dtype=torch.uint8, device="cuda")
+    lib = pkv.load_library()
+    rc = lib.pkv_paged_attention_prefill_chunk_fp8(
+        q.data_ptr(), q.data_ptr(), kc.data_ptr(), kc.data_ptr(), i32.data_ptr(), (i32[:1] + 4).data_ptr(),
+        torch.tensor([0, 4], dtype=torch.int32, device="cuda").data_ptr(), 1, 4, 4, 0.1, 1.0, 1.0, 2, 2, 64, 16, 2,
+        2, 1, ws.data_ptr(), 16, torch.cuda.current_stream().cuda_stream)
+    assert rc == -5
