@@ -5,6 +5,10 @@
 // context is read once per KV head, and all G query heads that share that KV
 // head (grouped-query attention) are served from the same bytes.
 //
+// The kernel below computes on the CUDA cores and serves fp32 pools; fp16 and
+// bf16 pools use the tensor-core variant in decode_mma.cuh, which shares the
+// parameters, the partitioning, the merge and decode_finish defined here.
+//
 // Work decomposition: one CTA per (sequence, partition, KV head), KV head
 // fastest so that CTAs running together read neighbouring bytes of the same
 // physical blocks.  A partition is a run of `PB` logical blocks; its four warps

@@ -78,6 +78,44 @@ def test_host_rejections_before_launch(lib):
     assert lib.pkv_get_device_error(None, None) == -1
 
 
+def test_host_rejections_fp8_and_multi_token(lib):
+    # FP8 pools: fp32 query, head_dim 64, non-positive or non-finite scales, an fp8 query type
+    dec8 = lib.pkv_paged_attention_decode_fp8
+    assert dec8(None, None, None, None, None, None, 0.1, 1.0, 1.0, 1, 4, 2, 128, 16, 1, 1, 16, 0, 0, None, 0,
+                None) == -2
+    assert dec8(None, None, None, None, None, None, 0.1, 1.0, 1.0, 1, 4, 2, 64, 16, 1, 1, 16, 0, 1, None, 0,
+                None) == -2
+    assert dec8(None, None, None, None, None, None, 0.1, 0.0, 1.0, 1, 4, 2, 128, 16, 1, 1, 16, 0, 1, None, 0,
+                None) == -1
+    assert dec8(None, None, None, None, None, None, 0.1, 1.0, float("inf"), 1, 4, 2, 128, 16, 1, 1, 16, 0, 1,
+                None, 0, None) == -1
+    assert lib.pkv_paged_attention_decode(None, None, None, None, None, None, 0.1, 1, 4, 2, 128, 16, 1, 1, 16, 0, 3,
+                                          None, 0, None) == -2  # an FP8 query is not a query type
+    assert lib.pkv_reshape_and_cache_fp8(None, None, None, None, None, 4, 2, 64, 16, 4, 3, 1.0, 1.0, None) == -2
+    assert lib.pkv_reshape_and_cache_fp8(None, None, None, None, None, 4, 2, 64, 16, 4, 1, -1.0, 1.0, None) == -1
+    assert lib.pkv_reshape_and_cache_fp8(None, None, None, None, None, 0, 2, 64, 16, 4, 1, 1.0, 1.0, None) == 0
+    assert lib.pkv_reshape_and_cache_fp8(None, None, None, None, None, 4, 1, 8, 16, 4, 1, 1.0, 1.0, None) == -2
+    # FP8 prefill: workspace is checked before any device work
+    pf8 = lib.pkv_paged_attention_prefill_chunk_fp8
+    assert pf8(None, None, None, None, None, None, None, 1, 4, 4, 0.1, 1.0, 1.0, 2, 2, 64, 16, 1, 4, 0, None, 0,
+               None) == -2  # fp32 query
+    assert lib.pkv_prefill_fp8_workspace_size(2, 10, 16, 8, 128, 100, 32, 2) == \
+        100 * 32 * 128 * 2 + 2 * (2 * 10 * 16 * 8 * 128 * 2) + 1024
+    assert lib.pkv_prefill_fp8_workspace_size(2, 10, 16, 8, 128, 100, 32, 1) == \
+        2 * (2 * 10 * 16 * 8 * 128 * 2) + 1024
+    # multi-token decode: more than 32 rows per KV head, bad partition size
+    mt = lib.pkv_paged_attention_decode_multi
+    assert mt(None, None, None, None, None, None, None, 1, 9, 9, 100, 0.1, 32, 8, 128, 16, 8, 16, 0, 1, None, 0,
+              None) == -2
+    assert mt(None, None, None, None, None, None, None, 1, 6, 6, 100, 0.1, 32, 8, 128, 16, 8, 16, 24, 1, None, 0,
+              None) == -1
+    assert mt(None, None, None, None, None, None, None, 0, 0, 6, 100, 0.1, 32, 8, 128, 16, 8, 16, 0, 1, None, 0,
+              None) == 0
+    assert pkv.decode_multi_partition_size(64, 8, 32, 4039) % 32 == 0
+    assert pkv.decode_multi_partition_size(1000, 32, 16, 2048) == 0  # enough pairs: no split
+    assert pkv.decode_multi_partition_size(1, 1, 16, 200) == 0       # short: no split
+
+
 def test_missing_library_fails_loudly(monkeypatch, tmp_path):
     monkeypatch.setattr(_binding, "_lib", None)
     monkeypatch.setattr(_binding, "LIB", str(tmp_path / "nope.so"))
