@@ -201,3 +201,41 @@ def test_fp8_prefill_rejects_small_workspace():
         torch.tensor([0, 4], dtype=torch.int32, device="cuda").data_ptr(), 1, 4, 4, 0.1, 1.0, 1.0, 2, 2, 64, 16, 2,
         2, 1, ws.data_ptr(), 16, torch.cuda.current_stream().cuda_stream)
     assert rc == -5
+
+
+def test_mixed_step_fp8_sampled():
+    """The mixed step on E4M3 pools in the benchmark's launch configuration (quantising append of
+    every token, FP8 chunked prefill, FP8 decode with the recommended split): sampled decode
+    sequences and prefill rows against the oracle."""
+    m = workloads.mixed_step_fp8(device="cuda")
+    w = m.decode
+    kc, vc = w.key_caches[0], w.value_caches[0]
+    pre_k, pre_v = kc.clone(), vc.clone()
+    ks, vs = w.extra["k_scale"], w.extra["v_scale"]
+    pkv.reshape_and_cache_fp8(m.append_keys, m.append_values, kc, vc, torch.from_numpy(m.append_slots).cuda(), ks, vs)
+    pout = torch.empty_like(m.chunk_query)
+    pkv.paged_attention_prefill_chunk_fp8(pout, m.chunk_query, kc, vc, torch.from_numpy(m.chunk_tables).cuda(),
+                                          torch.from_numpy(m.seq_lens).cuda(),
+                                          torch.from_numpy(m.query_start_loc).cuda(), int(m.chunk_lens.max()),
+                                          w.scale, ks, vs)
+    bt, cl, _ = gpu_tables(w)
+    part = pkv.decode_partition_size(w.num_seqs, w.num_kv_heads, w.head_dim, w.block_size, w.max_context_len, 3,
+                                     int(w.context_lens.sum()))
+    dout = torch.empty_like(w.queries[0])
+    pkv.paged_attention_decode_fp8(dout, w.queries[0], kc, vc, bt, cl, w.scale, ks, vs, w.max_context_len,
+                                   partition_size=part)
+    torch.cuda.synchronize()
+    assert pkv.get_device_error() == 0
+    order = np.argsort(w.context_lens)
+    dsample = np.unique(np.concatenate([order[:2], order[-3:], np.arange(7, w.num_seqs, 47)]))
+    ref, _, _, _ = oracle_decode_step(w, seqs=dsample, pre_k=pre_k, pre_v=pre_v)
+    assert_close(dout[torch.from_numpy(dsample).cuda()], ref, torch.bfloat16, "fp8 mixed decode sample")
+    sel = np.zeros(int(m.query_start_loc[-1]), dtype=np.uint8)
+    for r in range(len(m.chunk_lens)):
+        q0, n = int(m.query_start_loc[r]), int(m.chunk_lens[r])
+        for i in (0, 1, 31, 32, 127, 128, 255, 256, n - 1):
+            if 0 <= i < n:
+                sel[q0 + i] = 1
+    ref = oracle_prefill_chunks(m, pre_k, pre_v, row_select=sel)
+    rows = np.nonzero(sel)[0]
+    assert_close(pout[torch.from_numpy(rows).cuda()], ref[rows], torch.bfloat16, "fp8 mixed prefill sample")
