@@ -82,7 +82,7 @@ struct PrefillCfg {
     static constexpr int XCH_OFF = BAR_OFF + NBAR * 8;      // [128 rows][2 halves] floats
     static constexpr int SMEM = 1024 + XCH_OFF + BM * 2 * 4;
     static constexpr uint32_t TMEM_COLS = 512;
-    static constexpr uint32_t S_COL0 = 0, O_COL0 = 256;  // S buffers at 0 / 128, O buffers at 256 / 384
+    static constexpr uint32_t S_COL0 = 0, O_COL0 = 256;  // S buffers at 0 / 128, the O accumulator at 256
     static_assert(D == 64 || D == 128, "head_dim");
 };
 
@@ -103,8 +103,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1) paged_prefill_kernel(const
     uint64_t* s_full = bars + 5;   // [2]  Q.K^T done (tcgen05.commit)
     uint64_t* s_free = bars + 7;   // [2]  softmax finished reading S
     uint64_t* p_full = bars + 9;   //      P of the current tile written
-    uint64_t* o_full = bars + 10;  // [2]  P.V done (tcgen05.commit)
-    uint64_t* o_free = bars + 12;  // [2]  softmax folded O into registers
+    uint64_t* o_full = bars + 10;  // [2]  P.V of tile t done (tcgen05.commit), barrier t & 1
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 14);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + 15);
     uint64_t* xch_full = bars + 16;  // [4]  both halves of a quadrant's rows posted a value
@@ -148,7 +147,6 @@ __global__ void __launch_bounds__(kPrefillThreads, 1) paged_prefill_kernel(const
             mbar_init(&s_full[i], 1);
             mbar_init(&s_free[i], kPrefillSoftmaxWarps * 32);
             mbar_init(&o_full[i], 1);
-            mbar_init(&o_free[i], kPrefillSoftmaxWarps * 32);
         }
         mbar_init(p_full, kPrefillSoftmaxWarps * 32);
         for (int i = 0; i < 4; ++i) {
@@ -253,22 +251,22 @@ __global__ void __launch_bounds__(kPrefillThreads, 1) paged_prefill_kernel(const
                 ns = t + 1;
                 return true;
             };
+            // O accumulates over all key tiles in one TMEM buffer; the softmax
+            // rescales it (rarely) before it posts P of the next tile.
             auto issue_pv = [&](int t) -> bool {
                 const int st = t & 1;
                 if (!mbar_wait_or_abort(p_full, t & 1, abort_flag)) return false;
                 if (!mbar_wait_or_abort(&v_full[st], (t >> 1) & 1, abort_flag)) return false;
-                if (t >= 2 && !mbar_wait_or_abort(&o_free[st], ((t - 2) >> 1) & 1, abort_flag)) return false;
                 tc_fence_after();
                 const uint32_t v_addr = smem_u32(smem + C::V_OFF + st * C::KT_BYTES);
 #pragma unroll
                 for (int kk = 0; kk < C::BN / 16; ++kk) {
                     const uint32_t poff = (kk / 4) * (C::BM * 128) + (kk % 4) * 32;
                     const uint64_t vdesc = smem_desc_sw128(v_addr + kk * 16 * 128, C::BN * 128, 1024);
-                    umma_f16_ss(tmem + C::O_COL0 + st * 128, smem_desc_sw128(p_addr + poff, 16, 1024), vdesc, IDESC_O,
-                                kk > 0);
+                    umma_f16_ss(tmem + C::O_COL0, smem_desc_sw128(p_addr + poff, 16, 1024), vdesc, IDESC_O,
+                                t > 0 || kk > 0);
                     if constexpr (C::SPLIT_P)
-                        umma_f16_ss(tmem + C::O_COL0 + st * 128, smem_desc_sw128(plo_addr + poff, 16, 1024), vdesc,
-                                    IDESC_O, 1);
+                        umma_f16_ss(tmem + C::O_COL0, smem_desc_sw128(plo_addr + poff, 16, 1024), vdesc, IDESC_O, 1);
                 }
                 umma_commit(&o_full[st]);
                 npv = t + 1;
@@ -298,11 +296,14 @@ __global__ void __launch_bounds__(kPrefillThreads, 1) paged_prefill_kernel(const
         uint8_t* plo_s = smem + C::PLO_OFF;
         float* xch = reinterpret_cast<float*>(smem + C::XCH_OFF);
         const float sl2 = p.scale_log2;
-        float o[HD];
-#pragma unroll
-        for (int d = 0; d < HD; ++d) o[d] = 0.f;
-        float m = -INFINITY, lsum = 0.f, alpha_prev = 1.f;
+        // Lazy rescaling: the exponent base m_used moves (and O, lsum are
+        // rescaled) only when a tile's row max exceeds it by more than
+        // kRescaleLog2; until then the weights exp2(s - m_used) stay below
+        // 2^kRescaleLog2, far inside fp32 and the 16-bit P range.
+        constexpr float kRescaleLog2 = 8.f;
+        float m_used = -INFINITY, lsum = 0.f;
         bool ok = true;
+        float sv[HC];  // this thread's half row of S for the current tile
         float v[32];
         // Post this half's value for the row, return the partner half's (exchange
         // number e; the slot is reused once the partner read the previous one).
@@ -317,6 +318,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1) paged_prefill_kernel(const
             mbar_arrive(&xch_read[quad]);
             return true;
         };
+        const uint32_t to = tmem + lane_base + C::O_COL0 + half * HD;  // this half row of O
         for (int j = 0; j < nkt; ++j) {
             const int st = j & 1;
             if (!__all_sync(0xffffffffu, mbar_wait_or_abort(&s_full[st], (j >> 1) & 1, abort_flag))) {
@@ -328,65 +330,72 @@ __global__ void __launch_bounds__(kPrefillThreads, 1) paged_prefill_kernel(const
             const int k0 = j * C::BN + half * HC;  // first key of this thread's columns
             const bool all_vis = k0 + HC - 1 <= qpos;
             const bool none_vis = k0 > qpos;
-            // ---- pass 1: max of the visible scores of this half row (scale sign via max / min)
+            // ---- S into registers (scaled to the log2 domain, hidden keys at -inf), half-row max
             // (tcgen05.ld is warp-collective: every lane loads, masking is per row in registers)
-            float hi_raw = -INFINITY, lo_raw = INFINITY;
+            float mhalf = -INFINITY;
 #pragma unroll
             for (int c = 0; c < HC / 32; ++c) {
                 tmem_ld32(ts + c * 32, v);
-                if (all_vis) {
 #pragma unroll
-                    for (int i = 0; i < 32; ++i) hi_raw = fmaxf(hi_raw, v[i]), lo_raw = fminf(lo_raw, v[i]);
-                } else if (!none_vis) {
-#pragma unroll
-                    for (int i = 0; i < 32; ++i)
-                        if (k0 + c * 32 + i <= qpos) hi_raw = fmaxf(hi_raw, v[i]), lo_raw = fminf(lo_raw, v[i]);
+                for (int i = 0; i < 32; ++i) {
+                    const float x = v[i] * sl2;
+                    sv[c * 32 + i] = (all_vis || k0 + c * 32 + i <= qpos) ? x : -INFINITY;
+                    mhalf = fmaxf(mhalf, sv[c * 32 + i]);
                 }
             }
-            const float mhalf = none_vis ? -INFINITY : (sl2 >= 0.f ? hi_raw * sl2 : lo_raw * sl2);
+            tc_fence_before();
+            mbar_arrive(&s_free[st]);  // S_j is in registers: its buffer may take S_{j+2}
+            if (none_vis) mhalf = -INFINITY;
             float mother = -INFINITY;
             if (!exchange(mhalf, j, mother)) {
                 ok = false;
                 break;
             }
-            const float mnew = fmaxf(m, fmaxf(mhalf, mother));
-            const float alpha = ex2_approx(m - mnew);
-            // ---- pass 2: P = exp2(S * scale * log2 e - m) for this half (= P panel `half`), into registers
+            const float mrow = fmaxf(mhalf, mother);
+            // both halves of a row see the same (m_used, mrow) and take the same decision
+            const bool rescale = mrow > m_used + kRescaleLog2 || (m_used == -INFINITY && mrow != -INFINITY);
+            float alpha = 1.f;
+            if (rescale) {
+                alpha = ex2_approx(m_used - mrow);  // 0 when m_used is -inf
+                m_used = mrow;
+            }
+            const float mexp = m_used == -INFINITY ? 0.f : m_used;
+            // ---- P = exp2(S - m_used) for this half (= P panel `half`), into registers
             float tsum = 0.f;
             uint32_t hi[HC / 2], lo[C::SPLIT_P ? HC / 2 : 1];
 #pragma unroll
-            for (int c = 0; c < HC / 32; ++c) {
-                tmem_ld32(ts + c * 32, v);
-#pragma unroll
-                for (int i = 0; i < 32; i += 2) {
-                    const int key = k0 + c * 32 + i;
-                    float p0 = ex2_approx(fmaf(v[i], sl2, -mnew));
-                    float p1 = ex2_approx(fmaf(v[i + 1], sl2, -mnew));
-                    if (!all_vis) {
-                        p0 = key <= qpos ? p0 : 0.f;
-                        p1 = key + 1 <= qpos ? p1 : 0.f;
-                    }
-                    tsum += p0 + p1;
-                    const int w = c * 16 + i / 2;
-                    if constexpr (C::SPLIT_P) {
-                        // hi = p truncated to bf16 (its top 16 bits, one byte permute for the
-                        // pair); lo = the exact remainder rounded to bf16, |lo| < 2^-7 |p|
-                        const uint32_t b0 = __float_as_uint(p0), b1 = __float_as_uint(p1);
-                        hi[w] = __byte_perm(b0, b1, 0x7632);
-                        lo[w] = Elem<T>::pack(p0 - __uint_as_float(b0 & 0xFFFF0000u),
-                                              p1 - __uint_as_float(b1 & 0xFFFF0000u));
-                    } else {
-                        hi[w] = Elem<T>::pack(p0, p1);
-                    }
+            for (int i = 0; i < HC; i += 2) {
+                const float p0 = ex2_approx(sv[i] - mexp);
+                const float p1 = ex2_approx(sv[i + 1] - mexp);
+                tsum += p0 + p1;
+                const int w = i / 2;
+                if constexpr (C::SPLIT_P) {
+                    // hi = p truncated to bf16 (its top 16 bits, one byte permute for the
+                    // pair); lo = the exact remainder rounded to bf16, |lo| < 2^-7 |p|
+                    const uint32_t b0 = __float_as_uint(p0), b1 = __float_as_uint(p1);
+                    hi[w] = __byte_perm(b0, b1, 0x7632);
+                    lo[w] = Elem<T>::pack(p0 - __uint_as_float(b0 & 0xFFFF0000u),
+                                          p1 - __uint_as_float(b1 & 0xFFFF0000u));
+                } else {
+                    hi[w] = Elem<T>::pack(p0, p1);
                 }
             }
-            tc_fence_before();
-            mbar_arrive(&s_free[st]);  // S_j fully read: its buffer may take S_{j+2}
-            // ---- P.V of the previous tile must be done before P is overwritten
+            lsum = lsum * alpha + tsum;  // this half's share of the row sum
+            // ---- P.V of the previous tile must be done before P is overwritten (and O rescaled)
             if (j >= 1 &&
                 !__all_sync(0xffffffffu, mbar_wait_or_abort(&o_full[(j - 1) & 1], ((j - 1) >> 1) & 1, abort_flag))) {
                 ok = false;
                 break;
+            }
+            if (j >= 1 && __any_sync(0xffffffffu, rescale && alpha != 1.f)) {
+                tc_fence_after();
+#pragma unroll
+                for (int c = 0; c < HD / 32; ++c) {  // warp-collective: lanes without a rescale store O back as is
+                    tmem_ld32(to + c * 32, v);
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) v[i] *= alpha;
+                    tmem_st32(to + c * 32, v);
+                }
             }
             // ---- the last tile may hold the dead tail of the sequence's last
             // block: zero those V rows (0 * NaN must not reach the output)
@@ -417,34 +426,19 @@ __global__ void __launch_bounds__(kPrefillThreads, 1) paged_prefill_kernel(const
                         make_uint4(lo[4 * q], lo[4 * q + 1], lo[4 * q + 2], lo[4 * q + 3]);
             }
             fence_proxy_async();
+            tc_fence_before();
             mbar_arrive(p_full);
-            // ---- fold P.V of the previous tile into this half of the accumulator
-            if (j >= 1) {
-                tc_fence_after();
-                const uint32_t to = tmem + lane_base + C::O_COL0 + ((j - 1) & 1) * 128 + half * HD;
-#pragma unroll
-                for (int c = 0; c < HD / 32; ++c) {
-                    tmem_ld32(to + c * 32, v);
-#pragma unroll
-                    for (int i = 0; i < 32; ++i) o[c * 32 + i] = fmaf(o[c * 32 + i], alpha_prev, v[i]);
-                }
-                tc_fence_before();
-                mbar_arrive(&o_free[(j - 1) & 1]);
-            }
-            lsum = lsum * alpha + tsum;  // this half's share of the row sum
-            m = mnew;
-            alpha_prev = alpha;
         }
+        float o[HD];
         if (ok) {
             const int jl = nkt - 1;
             if (__all_sync(0xffffffffu, mbar_wait_or_abort(&o_full[jl & 1], (jl >> 1) & 1, abort_flag))) {
                 tc_fence_after();
-                const uint32_t to = tmem + lane_base + C::O_COL0 + (jl & 1) * 128 + half * HD;
 #pragma unroll
                 for (int c = 0; c < HD / 32; ++c) {
                     tmem_ld32(to + c * 32, v);
 #pragma unroll
-                    for (int i = 0; i < 32; ++i) o[c * 32 + i] = fmaf(o[c * 32 + i], alpha_prev, v[i]);
+                    for (int i = 0; i < 32; ++i) o[c * 32 + i] = v[i];
                 }
             } else {
                 ok = false;
