@@ -332,17 +332,29 @@ __global__ void __launch_bounds__(kPrefillThreads, 1) paged_prefill_kernel(const
             const bool none_vis = k0 > qpos;
             // ---- S into registers (scaled to the log2 domain, hidden keys at -inf), half-row max
             // (tcgen05.ld is warp-collective: every lane loads, masking is per row in registers)
+            // A fully visible half row keeps the raw scores (the scale goes into the
+            // exponent's FMA); a diagonal one holds scaled scores with -inf masks.
             float mhalf = -INFINITY;
 #pragma unroll
-            for (int c = 0; c < HC / 32; ++c) {
-                tmem_ld32(ts + c * 32, v);
+            for (int c = 0; c < HC / 32; ++c) tmem_ld32(ts + c * 32, *reinterpret_cast<float(*)[32]>(&sv[c * 32]));
+            if (all_vis) {
+                float r = sv[0];
+                if (sl2 >= 0.f) {
 #pragma unroll
-                for (int i = 0; i < 32; ++i) {
-                    const float x = v[i] * sl2;
-                    sv[c * 32 + i] = (all_vis || k0 + c * 32 + i <= qpos) ? x : -INFINITY;
-                    mhalf = fmaxf(mhalf, sv[c * 32 + i]);
+                    for (int i = 1; i < HC; ++i) r = fmaxf(r, sv[i]);
+                } else {
+#pragma unroll
+                    for (int i = 1; i < HC; ++i) r = fminf(r, sv[i]);
+                }
+                mhalf = r * sl2;
+            } else {
+#pragma unroll
+                for (int i = 0; i < HC; ++i) {
+                    sv[i] = k0 + i <= qpos ? sv[i] * sl2 : -INFINITY;
+                    mhalf = fmaxf(mhalf, sv[i]);
                 }
             }
+            const float smul = all_vis ? sl2 : 1.f;  // the exponent is sv * smul - m
             tc_fence_before();
             mbar_arrive(&s_free[st]);  // S_j is in registers: its buffer may take S_{j+2}
             if (none_vis) mhalf = -INFINITY;
@@ -365,8 +377,8 @@ __global__ void __launch_bounds__(kPrefillThreads, 1) paged_prefill_kernel(const
             uint32_t hi[HC / 2], lo[C::SPLIT_P ? HC / 2 : 1];
 #pragma unroll
             for (int i = 0; i < HC; i += 2) {
-                const float p0 = ex2_approx(sv[i] - mexp);
-                const float p1 = ex2_approx(sv[i + 1] - mexp);
+                const float p0 = ex2_approx(fmaf(sv[i], smul, -mexp));
+                const float p1 = ex2_approx(fmaf(sv[i + 1], smul, -mexp));
                 tsum += p0 + p1;
                 const int w = i / 2;
                 if constexpr (C::SPLIT_P) {
