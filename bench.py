@@ -287,6 +287,19 @@ class MultiTokenStep:
             timer.end()
 
 
+# DRAM bytes (read + write) per algorithmic byte of the decode call, from one
+# ncu capture of the same kernel on a smaller case of the workload (traffic
+# grows with the blocks read, so it scales to the full launch by the
+# algorithmic bytes).  A workload is listed only while its kernel is unchanged
+# since the capture.
+TRAFFIC_PER_ALGORITHMIC_BYTE = {
+    "llama7b_decode_f16": ((287.471104 + 3.418624) / 285.38096,
+                           "profiles/paged_decode_mma_kernel_llama7b_16seq_full.md"),
+    "llama7b_decode_fp8": ((305.048832 + 4.018688) / 303.293524,
+                           "profiles/paged_decode_fp8_kernel_llama7b_fp8_32seq.md"),
+}
+
+
 def make_step(name, device, rank, seqs=None, layers=None):
     from paged_kv_cache_409_b200 import workloads
     if name == "llama7b_decode_f16":
@@ -703,6 +716,11 @@ def main():
     }
     if hasattr(step, "config"):
         line["config"].update(step.config())
+    if args.config in TRAFFIC_PER_ALGORITHMIC_BYTE and not args.seqs:
+        ratio, source = TRAFFIC_PER_ALGORITHMIC_BYTE[args.config]
+        line["roofline"]["traffic"] = ratio * step.decode_bytes  # DRAM bytes per decode call
+        line["roofline"]["traffic_unit"] = "bytes per launch"
+        line["roofline"]["traffic_source"] = source + " (smaller case, scaled by algorithmic bytes)"
     if isinstance(step, MixedStep):
         line["prefill_tokens_per_s"] = ws * step.prefill_tokens / (ms_step / 1e3)
         line["prefill_flops_per_step"] = step.prefill_flops
