@@ -322,9 +322,11 @@ size_t pkv_prefill_fp8_workspace_size(int num_chunks, int max_blocks_per_seq, in
  *                   (pkv_decode_multi_partition_size recommends one)
  *   workspace       >= pkv_decode_workspace_size(total_q_tokens, num_q_heads,
  *                   head_dim, max_seq_len, partition_size) bytes
- * Supported: dtype in {F16, BF16}; head_dim in {64, 128}; block_size in
- * {8, 16, 32}; num_q_heads / num_kv_heads in {1, 2, 4, 8}.  A chunk whose n_r
- * exceeds the row limit or its sequence is skipped and sets PKV_DEVERR_LENGTH.
+ * Supported: dtype in {F16, BF16} (16-bit pools; over FP8 pools the same
+ * computation is pkv_paged_attention_prefill_chunk_fp8); head_dim in {64,
+ * 128}; block_size in {8, 16, 32}; num_q_heads / num_kv_heads in {1, 2, 4, 8}.
+ * A chunk whose n_r exceeds the row limit or its sequence is skipped and sets
+ * PKV_DEVERR_LENGTH.
  */
 int pkv_paged_attention_decode_multi(void* out, const void* query, const void* key_cache, const void* value_cache,
                                      const int32_t* block_tables, const int32_t* seq_lens,
