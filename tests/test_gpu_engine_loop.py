@@ -29,15 +29,19 @@ def kv_of(tokens, positions, table):
     return (table[t] * (1.0 + 0.05 * (p % 11)).view(-1, 1, 1)).to(DT)
 
 
-def test_block_manager_drives_decode_steps():
+@pytest.mark.parametrize("pools", ["fp16", "e4m3"])
+def test_block_manager_drives_decode_steps(pools):
+    fp8 = pools == "e4m3"
+    KS, VS = 0.0131, 0.0157  # E4M3 pool scales
     rng = np.random.default_rng(21)
     g = torch.Generator().manual_seed(21)
     ek = torch.randn(VOCAB, Hkv, D, generator=g)
     ev = torch.randn(VOCAB, Hkv, D, generator=g)
     bm = BlockManager(NB, B, prefix_caching=True)
-    kc = torch.zeros(NB, B, Hkv, D, dtype=DT, device="cuda")
+    pool_dt = torch.uint8 if fp8 else DT
+    kc = torch.zeros(NB, B, Hkv, D, dtype=pool_dt, device="cuda")
     vc = torch.zeros_like(kc)
-    kn = np.zeros((NB, B, Hkv, D), dtype=np.float16)  # host mirror for the oracle
+    kn = np.zeros((NB, B, Hkv, D), dtype=np.uint8 if fp8 else np.float16)  # host mirror for the oracle
     vn = np.zeros_like(kn)
     orc = oracle.get()
     tokens = {}
@@ -46,8 +50,13 @@ def test_block_manager_drives_decode_steps():
         pos = np.arange(start, start + len(toks))
         k, v = kv_of(toks, pos, ek), kv_of(toks, pos, ev)
         sl = torch.from_numpy(np.asarray(slots, dtype=np.int64))
-        pkv.reshape_and_cache(k.cuda(), v.cuda(), kc, vc, sl.cuda())
-        orc.reshape_and_cache(k.numpy(), v.numpy(), kn, vn, sl.numpy(), oracle.F16)
+        if fp8:
+            pkv.reshape_and_cache_fp8(k.cuda(), v.cuda(), kc, vc, sl.cuda(), KS, VS)
+            orc.reshape_and_cache_fp8(k.numpy(), v.numpy(), kn, vn, sl.numpy(), oracle.F16,
+                                      float(np.float32(KS)), float(np.float32(VS)))
+        else:
+            pkv.reshape_and_cache(k.cuda(), v.cuda(), kc, vc, sl.cuda())
+            orc.reshape_and_cache(k.numpy(), v.numpy(), kn, vn, sl.numpy(), oracle.F16)
 
     system = rng.integers(0, VOCAB, 40).tolist()
     prompts = {0: system + rng.integers(0, VOCAB, 5).tolist(), 1: system + rng.integers(0, VOCAB, 7).tolist(),
@@ -78,10 +87,17 @@ def test_block_manager_drives_decode_steps():
         bt = bm.tables(live, mb)
         q = torch.randn(len(live), Hq, D, generator=g).to(DT)
         out = torch.empty(len(live), Hq, D, dtype=DT, device="cuda")
-        pkv.paged_attention_decode(out, q.cuda(), kc, vc, torch.from_numpy(bt).cuda(), torch.from_numpy(lens).cuda(),
-                                   D ** -0.5, int(lens.max()))
-        ref = orc.paged_attention_decode(q.numpy(), kn, vn, bt, lens, float(np.float32(D ** -0.5)), oracle.F16)
+        scale = float(np.float32(D ** -0.5))
+        if fp8:
+            pkv.paged_attention_decode_fp8(out, q.cuda(), kc, vc, torch.from_numpy(bt).cuda(),
+                                           torch.from_numpy(lens).cuda(), scale, KS, VS, int(lens.max()))
+            ref = orc.paged_attention_decode_kv(q.numpy(), oracle.F16, kn, vn, oracle.E4M3, float(np.float32(KS)),
+                                                float(np.float32(VS)), bt, lens, scale)
+        else:
+            pkv.paged_attention_decode(out, q.cuda(), kc, vc, torch.from_numpy(bt).cuda(),
+                                       torch.from_numpy(lens).cuda(), scale, int(lens.max()))
+            ref = orc.paged_attention_decode(q.numpy(), kn, vn, bt, lens, scale, oracle.F16)
         assert_close(out, ref, DT, f"step {step}")
     assert cows == 1                                 # the fork's first append copied the shared partial block
     assert pkv.get_device_error() == 0
-    assert np.array_equal(kc.cpu().numpy().view(np.int16), kn.view(np.int16))
+    assert np.array_equal(kc.cpu().numpy().view(np.uint8), kn.view(np.uint8))
