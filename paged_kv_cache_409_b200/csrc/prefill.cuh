@@ -338,15 +338,21 @@ __global__ void __launch_bounds__(kPrefillThreads, 1) paged_prefill_kernel(const
 #pragma unroll
             for (int c = 0; c < HC / 32; ++c) tmem_ld32(ts + c * 32, *reinterpret_cast<float(*)[32]>(&sv[c * 32]));
             if (all_vis) {
-                float r = sv[0];
+                // four independent chains (max and min are exact in any order)
+                float r0 = sv[0], r1 = sv[1], r2 = sv[2], r3 = sv[3];
                 if (sl2 >= 0.f) {
 #pragma unroll
-                    for (int i = 1; i < HC; ++i) r = fmaxf(r, sv[i]);
+                    for (int i = 4; i < HC; i += 4)
+                        r0 = fmaxf(r0, sv[i]), r1 = fmaxf(r1, sv[i + 1]), r2 = fmaxf(r2, sv[i + 2]),
+                        r3 = fmaxf(r3, sv[i + 3]);
+                    mhalf = fmaxf(fmaxf(r0, r1), fmaxf(r2, r3)) * sl2;
                 } else {
 #pragma unroll
-                    for (int i = 1; i < HC; ++i) r = fminf(r, sv[i]);
+                    for (int i = 4; i < HC; i += 4)
+                        r0 = fminf(r0, sv[i]), r1 = fminf(r1, sv[i + 1]), r2 = fminf(r2, sv[i + 2]),
+                        r3 = fminf(r3, sv[i + 3]);
+                    mhalf = fminf(fminf(r0, r1), fminf(r2, r3)) * sl2;
                 }
-                mhalf = r * sl2;
             } else {
 #pragma unroll
                 for (int i = 0; i < HC; ++i) {
@@ -373,13 +379,13 @@ __global__ void __launch_bounds__(kPrefillThreads, 1) paged_prefill_kernel(const
             }
             const float mexp = m_used == -INFINITY ? 0.f : m_used;
             // ---- P = exp2(S - m_used) for this half (= P panel `half`), into registers
-            float tsum = 0.f;
+            float ts4[4] = {0.f, 0.f, 0.f, 0.f};  // partial sums: four independent chains
             uint32_t hi[HC / 2], lo[C::SPLIT_P ? HC / 2 : 1];
 #pragma unroll
             for (int i = 0; i < HC; i += 2) {
                 const float p0 = ex2_approx(fmaf(sv[i], smul, -mexp));
                 const float p1 = ex2_approx(fmaf(sv[i + 1], smul, -mexp));
-                tsum += p0 + p1;
+                ts4[(i / 2) & 3] += p0 + p1;
                 const int w = i / 2;
                 if constexpr (C::SPLIT_P) {
                     // hi = p truncated to bf16 (its top 16 bits, one byte permute for the
@@ -392,6 +398,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1) paged_prefill_kernel(const
                     hi[w] = Elem<T>::pack(p0, p1);
                 }
             }
+            const float tsum = (ts4[0] + ts4[1]) + (ts4[2] + ts4[3]);
             lsum = lsum * alpha + tsum;  // this half's share of the row sum
             // ---- P.V of the previous tile must be done before P is overwritten (and O rescaled)
             if (j >= 1 &&
