@@ -112,11 +112,7 @@ __global__ void __launch_bounds__(NW * 32) paged_decode_fp8_kernel(const DecodeP
     const int nw = nb > warp ? (nb - warp + NW - 1) / NW : 0;
     uint8_t* wstage = smem + warp * NST * C::STAGE;
     uint64_t* wbar = bars + warp * NST;
-#ifndef PKV_FP8_EVICT_NORMAL
     const uint64_t policy = l2_policy_evict_first();
-#else
-    const uint64_t policy = l2_policy_evict_normal();
-#endif
 
     auto issue = [&](int k) {  // lane 0 only
         const int st = k % NST;

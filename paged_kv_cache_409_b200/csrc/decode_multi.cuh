@@ -15,9 +15,10 @@
 //   O [16 rows x D]       += P [16 x 16 keys] . V   (A: S accumulators reused,
 //                                                     B: ldmatrix.trans of V)
 // Rows are (token, head) pairs, token-major: row r = i * G + hh.  A CTA serves
-// one (chunk, partition, KV head); its warps form RG row groups of 16 rows and
-// SW = NW / RG streams, each warp with its own TMA pipeline over the 16-token
-// units (sub-blocks) of its stream, and its own online-softmax state.  Warps of
+// one (chunk, partition, KV head); its warps form one row group of 16 rows per
+// 16 live rows (at most RG) and NW / groups streams, each warp with its own
+// TMA pipeline over the 16-token units (sub-blocks) of its stream, and its own
+// online-softmax state.  Warps of
 // one row group merge in shared memory; the CTA writes output rows (one
 // partition) or partials for the merge kernel, which combines partitions as
 // the decode merge does.
@@ -63,12 +64,8 @@ struct MultiCfg {
     static size_t smem_bytes(int pb) { return 1024 + BT_OFF + static_cast<size_t>(pb) * 4 + 16 + NW * NST * 8; }
 };
 
-#ifndef PKV_MULTI_MIN_BLOCKS
-#define PKV_MULTI_MIN_BLOCKS 1
-#endif
-
 template <typename T, int D, int B, int NST, int NW, int RG>
-__global__ void __launch_bounds__(NW * 32, PKV_MULTI_MIN_BLOCKS) paged_decode_multi_kernel(const MultiParams p, const int G,
+__global__ void __launch_bounds__(NW * 32) paged_decode_multi_kernel(const MultiParams p, const int G,
                                                                      const __grid_constant__ CUtensorMap tm_k,
                                                                      const __grid_constant__ CUtensorMap tm_v) {
     using C = MultiCfg<T, D, B, NST, NW, RG>;

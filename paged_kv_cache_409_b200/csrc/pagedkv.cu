@@ -88,10 +88,6 @@ CUtensorMapDataType cu_type(int dtype) {
 // Pool [num_blocks, block_size, num_kv_heads, head_dim] as a 4-D tensor
 // (head_dim innermost); one box = one block x one KV head x 128 bytes of
 // head_dim, 128-byte swizzled.
-#ifndef PKV_FP8_L2_PROMOTION
-#define PKV_FP8_L2_PROMOTION CU_TENSOR_MAP_L2_PROMOTION_L2_256B
-#endif
-
 // box_rows: tokens per box (the whole block by default).
 int make_pool_map(CUtensorMap* map, const void* pool, int dtype, int64_t num_blocks, int block_size,
                   int num_kv_heads, int head_dim, int box_rows = 0) {
@@ -107,10 +103,8 @@ int make_pool_map(CUtensorMap* map, const void* pool, int dtype, int64_t num_blo
                              (cuuint64_t)block_size * num_kv_heads * head_dim * eb};
     cuuint32_t box[4] = {(cuuint32_t)(128 / eb), 1, (cuuint32_t)(box_rows > 0 ? box_rows : block_size), 1};
     cuuint32_t estr[4] = {1, 1, 1, 1};
-    const CUtensorMapL2promotion promo =
-        dtype == PKV_FP8_E4M3 ? PKV_FP8_L2_PROMOTION : CU_TENSOR_MAP_L2_PROMOTION_L2_256B;
     CUresult r = fn(map, cu_type(dtype), 4, const_cast<void*>(pool), dims, strides, box, estr,
-                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, promo,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     if (r != CUDA_SUCCESS) {
         snprintf(g_last_cuda_error, sizeof g_last_cuda_error, "cuTensorMapEncodeTiled(pool) failed: %d", (int)r);
