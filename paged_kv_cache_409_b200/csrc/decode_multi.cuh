@@ -61,7 +61,8 @@ struct MultiCfg {
     static constexpr int BT_OFF = STAGES_BYTES > RED_BYTES ? STAGES_BYTES : RED_BYTES;
     static_assert(TILE % 1024 == 0, "tiles must keep 1024-byte alignment for the 128-byte swizzle");
     static_assert(NW % RG == 0, "warps must split evenly into row groups");
-    static size_t smem_bytes(int pb) { return 1024 + BT_OFF + static_cast<size_t>(pb) * 4 + 16 + NW * NST * 8; }
+    // per warp: NST full barriers, then NST empty barriers (used when two row groups share a stream's stages)
+    static size_t smem_bytes(int pb) { return 1024 + BT_OFF + static_cast<size_t>(pb) * 4 + 16 + 2 * NW * NST * 8; }
 };
 
 template <typename T, int D, int B, int NST, int NW, int RG>
@@ -113,17 +114,25 @@ __global__ void __launch_bounds__(NW * 32) paged_decode_multi_kernel(const Multi
         }
         bt_s[i] = id;
     }
-    if (lane == 0) {
-#pragma unroll
-        for (int st = 0; st < NST; ++st) mbar_init(&bars[warp * NST + st], 1);
-        fence_mbar_init();
-    }
-
     // ---- this warp's 16 rows: the lane holds rows rq and rq + 8 (rq = lane / 4).
     // A chunk with at most 16 rows uses one row group: every warp is a stream.
+    // With two row groups the two warps of a stream share its stages: the
+    // first issues each unit's copy once into a ring of 2 * NST stages, both
+    // read it, and each releases it on the stage's empty barrier.
     const int nrg = n * G > 16 ? RG : 1;
     const int nsw = NW / nrg;
     const int rg = warp % nrg, stream = warp / nrg;
+    const int ring = nrg * NST;
+    uint64_t* fbar = bars + stream * ring;            // full: the unit's bytes arrived
+    uint64_t* ebar = bars + NW * NST + stream * ring;  // empty: every reader of the stage is done
+    if (lane == 0) {
+#pragma unroll
+        for (int st = 0; st < NST; ++st) {
+            mbar_init(&bars[warp * NST + st], 1);
+            mbar_init(&bars[NW * NST + warp * NST + st], nrg);
+        }
+        fence_mbar_init();
+    }
     const int gq = lane >> 2, cq = lane & 3;
     int lim[2];  // last key position each of the lane's two rows may see
     uint32_t qa[KS][4];
@@ -148,27 +157,28 @@ __global__ void __launch_bounds__(NW * 32) paged_decode_multi_kernel(const Multi
     const int span = max(0, min(len, (b0 + nb) * B) - b0 * B);
     const int units = (span + UT - 1) / UT;
     const int nw = units > stream ? (units - stream + nsw - 1) / nsw : 0;
-    uint8_t* wstage = smem + warp * NST * C::STAGE;
-    uint64_t* wbar = bars + warp * NST;
+    uint8_t* wstage = smem + stream * ring * C::STAGE;  // the stream's ring of stages
+    const bool producer = rg == 0;
     const uint64_t policy = l2_policy_evict_first();
 
-    auto issue = [&](int k) {  // lane 0 only
-        const int st = k % NST;
+    auto issue = [&](int k) {  // lane 0 of the producer only
+        const int st = k % ring;
         const int u = stream + k * nsw;
         const int id = bt_s[u / C::UPB];
         const int coord = id >= 0 ? id : static_cast<int>(p.num_blocks);  // out of range: zero fill
         const int row0 = (u % C::UPB) * UT;
         uint8_t* kd = wstage + st * C::STAGE;
         uint8_t* vd = kd + C::TILE;
-        mbar_arrive_expect_tx(&wbar[st], C::STAGE);
+        mbar_arrive_expect_tx(&fbar[st], C::STAGE);
 #pragma unroll
         for (int pn = 0; pn < C::NP; ++pn) {
-            tma_load_4d_hint(kd + pn * UT * 128, &tm_k, pn * 64, g, row0, coord, &wbar[st], policy);
-            tma_load_4d_hint(vd + pn * UT * 128, &tm_v, pn * 64, g, row0, coord, &wbar[st], policy);
+            tma_load_4d_hint(kd + pn * UT * 128, &tm_k, pn * 64, g, row0, coord, &fbar[st], policy);
+            tma_load_4d_hint(vd + pn * UT * 128, &tm_v, pn * 64, g, row0, coord, &fbar[st], policy);
         }
     };
-    if (lane == 0) {
-        for (int k = 0; k < NST && k < nw; ++k) issue(k);
+    int issued = 0;
+    if (lane == 0 && producer) {
+        for (; issued < ring && issued < nw; ++issued) issue(issued);
     }
     __syncwarp();
 
@@ -180,8 +190,8 @@ __global__ void __launch_bounds__(NW * 32) paged_decode_multi_kernel(const Multi
 
     int k = 0;
     for (; k < nw; ++k) {
-        const int st = k % NST;
-        const bool ok = mbar_wait(&wbar[st], (k / NST) & 1);
+        const int st = k % ring;
+        const bool ok = mbar_wait(&fbar[st], (k / ring) & 1);
         if (!__all_sync(0xffffffffu, ok)) break;
         const int u = stream + k * nsw;
         const int pos0 = (b0 + u / C::UPB) * B + (u % C::UPB) * UT;  // key position of the unit's first token
@@ -308,13 +318,27 @@ __global__ void __launch_bounds__(NW * 32) paged_decode_multi_kernel(const Multi
             }
         }
         __syncwarp();
-        if (lane == 0 && k + NST < nw) {
-            fence_proxy_async();
-            issue(k + NST);
+        bool go = true;
+        if (lane == 0) {
+            if (nrg > 1) mbar_arrive(&ebar[st]);
+            if (producer && k + ring < nw) {
+                // the stage is refilled once every reader released unit k
+                go = nrg == 1 || mbar_wait(&ebar[st], (k / ring) & 1);
+                if (go) {
+                    fence_proxy_async();
+                    issue(k + ring);
+                    issued = k + ring + 1;
+                }
+            }
+        }
+        if (!__shfl_sync(0xffffffffu, go, 0)) {
+            ++k;
+            break;
         }
     }
-    if (k < nw && lane == 0) {
-        for (int kk = k + 1; kk < min(nw, k + NST); ++kk) mbar_wait(&wbar[kk % NST], (kk / NST) & 1);
+    if (k < nw && lane == 0 && producer) {
+        // a wait gave up: wait (bounded) for this warp's copies still in flight
+        for (int kk = k; kk < issued; ++kk) mbar_wait(&fbar[kk % ring], (kk / ring) & 1);
     }
     if (k < nw) m[0] = m[1] = -INFINITY, l[0] = l[1] = 0.f;
 #pragma unroll
