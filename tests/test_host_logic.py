@@ -117,3 +117,21 @@ def test_poison_marks_only_dead_slots():
     dead = np.setdiff1d(np.arange(kc.shape[0]), live)
     assert torch.isfinite(kc[torch.from_numpy(live)]).all()
     assert torch.isnan(kc[torch.from_numpy(dead)]).all()
+
+
+def test_fp8_workload_codes():
+    """E4M3 pools hold finite codes of N(0,1)/scale in live slots and the NaN code 0x7F in dead ones."""
+    w = workloads.decode_workload("f8", [5, 33, 70], 8, 2, 128, 16, torch.float16, seed=3, poison=True,
+                                  fp8_scales=(0.02, 0.03))
+    assert w.fp8 and w.key_caches[0].dtype == torch.uint8
+    assert w.extra["k_scale"] == float(np.float32(0.02)) and w.extra["v_scale"] == float(np.float32(0.03))
+    live = workloads.live_slots(w.block_tables, w.context_lens, w.block_size)
+    rows = w.key_caches[0].view(-1, 2 * 128)
+    mask = np.zeros(rows.shape[0], dtype=bool)
+    mask[live] = True
+    codes_live = rows[torch.from_numpy(mask)].numpy()
+    assert not np.isin(codes_live, [0x7F, 0xFF]).any()           # no NaN codes where tokens live
+    assert (rows[torch.from_numpy(~mask)].numpy() == 0x7F).all()  # dead slots poisoned
+    vals = torch.from_numpy(codes_live).view(torch.float8_e4m3fn).float() * 0.02
+    assert abs(vals.std().item() - 1.0) < 0.1                     # N(0,1) after the scale
+    assert w.kv_bytes() == 2 * int(w.context_lens.sum()) * 2 * 128  # one byte per element
