@@ -66,7 +66,7 @@ class DecodeStep:
         self.sm = torch.from_numpy(w.slot_mapping.astype(np.int64)).to(dev)
         self.layers = layers_per_step or w.num_layers
         self.outs = [torch.empty_like(q) for q in w.queries]
-        self.part = pkv.decode_partition_size(w.num_seqs, w.num_kv_heads, w.head_dim, w.block_size,
+        self.part = pkv.decode_partition_size(w.num_seqs, w.num_q_heads, w.num_kv_heads, w.head_dim, w.block_size,
                                               w.max_context_len, 3 if w.fp8 else w.dtype,
                                               int(w.context_lens.astype(np.int64).sum()))
         need = pkv.decode_workspace_size(w.num_seqs, w.num_q_heads, w.head_dim, w.max_context_len, self.part)

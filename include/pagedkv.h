@@ -233,8 +233,11 @@ size_t pkv_decode_workspace_size(int num_seqs, int num_q_heads, int head_dim, in
  * current device: 0 (no split) when the (sequence, KV head) pairs alone fill
  * the GPU and no context is far longer than the mean, else a multiple of
  * block_size.  total_context_tokens (sum of context_lens, 0 = unknown) lets
- * it see a long tail.  Returns a negative pkv_status on bad input. */
-int pkv_decode_partition_size(int num_seqs, int num_kv_heads, int head_dim, int block_size,
+ * it see a long tail and, for E4M3 pools (dtype PKV_FP8_E4M3) with one query
+ * head per KV head, size parts so that the CTAs fill whole waves.
+ * num_q_heads must be a multiple of num_kv_heads.  Returns a negative
+ * pkv_status on bad input. */
+int pkv_decode_partition_size(int num_seqs, int num_q_heads, int num_kv_heads, int head_dim, int block_size,
                               int max_context_len, int64_t total_context_tokens, int dtype);
 
 /*

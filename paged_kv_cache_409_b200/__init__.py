@@ -6,6 +6,8 @@ the current CUDA stream into its C-ABI calls.  Importing the package does not
 load the library; the first call does, and fails loudly if it is missing.
 """
 from ._binding import (  # noqa: F401
+    FP8_E4M3,
+    FP8_POOL_DTYPES,
     PagedKVError,
     copy_blocks,
     decode_multi_partition_size,

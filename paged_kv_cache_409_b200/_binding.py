@@ -83,7 +83,7 @@ def load_library():
     lib.pkv_paged_attention_decode.argtypes = [P, P, P, P, P, P, F, I, I, I, I, I, I, I64, I, I, I, P, SZ, P]
     lib.pkv_decode_workspace_size.argtypes = [I, I, I, I, I]
     lib.pkv_decode_workspace_size.restype = SZ
-    lib.pkv_decode_partition_size.argtypes = [I, I, I, I, I, I64, I]
+    lib.pkv_decode_partition_size.argtypes = [I, I, I, I, I, I, I64, I]
     lib.pkv_paged_attention_prefill_chunk.argtypes = [P, P, P, P, P, P, P, I, I64, I, F, I, I, I, I, I, I64, I, P]
     lib.pkv_paged_attention_decode_multi.argtypes = [P, P, P, P, P, P, P, I, I64, I, I, F, I, I, I, I, I, I64, I, I,
                                                      P, SZ, P]
@@ -210,11 +210,11 @@ def decode_workspace_size(num_seqs, num_q_heads, head_dim, max_context_len, part
                                                          partition_size))
 
 
-def decode_partition_size(num_seqs, num_kv_heads, head_dim, block_size, max_context_len, dtype,
+def decode_partition_size(num_seqs, num_q_heads, num_kv_heads, head_dim, block_size, max_context_len, dtype,
                           total_context_tokens=0) -> int:
     code = DTYPE_CODE[dtype] if isinstance(dtype, torch.dtype) else int(dtype)
-    rc = load_library().pkv_decode_partition_size(num_seqs, num_kv_heads, head_dim, block_size, max_context_len,
-                                                  int(total_context_tokens), code)
+    rc = load_library().pkv_decode_partition_size(num_seqs, num_q_heads, num_kv_heads, head_dim, block_size,
+                                                  max_context_len, int(total_context_tokens), code)
     if rc < 0:
         raise PagedKVError("decode_partition_size", rc)
     return rc
@@ -235,7 +235,7 @@ def paged_attention_decode(out, query, key_cache, value_cache, block_tables, con
     if block_tables.dtype != torch.int32 or context_lens.dtype != torch.int32:
         raise ValueError("block_tables and context_lens must be int32")
     if partition_size is None:
-        partition_size = decode_partition_size(S, Hkv, D, B, max_context_len, query.dtype, total_context_tokens)
+        partition_size = decode_partition_size(S, Hq, Hkv, D, B, max_context_len, query.dtype, total_context_tokens)
     need = decode_workspace_size(S, Hq, D, max_context_len, partition_size) if partition_size else 0
     if need and (workspace is None or workspace.numel() * workspace.element_size() < need):
         workspace = torch.empty(need, dtype=torch.uint8, device=query.device)
@@ -262,7 +262,7 @@ def paged_attention_decode_fp8(out, query, key_cache, value_cache, block_tables,
     if block_tables.dtype != torch.int32 or context_lens.dtype != torch.int32:
         raise ValueError("block_tables and context_lens must be int32")
     if partition_size is None:
-        partition_size = decode_partition_size(S, Hkv, D, B, max_context_len, FP8_E4M3, total_context_tokens)
+        partition_size = decode_partition_size(S, Hq, Hkv, D, B, max_context_len, FP8_E4M3, total_context_tokens)
     need = decode_workspace_size(S, Hq, D, max_context_len, partition_size) if partition_size else 0
     if need and (workspace is None or workspace.numel() * workspace.element_size() < need):
         workspace = torch.empty(need, dtype=torch.uint8, device=query.device)

@@ -4,6 +4,7 @@ import os
 import re
 
 import pytest
+import torch
 
 import paged_kv_cache_409_b200 as pkv
 from paged_kv_cache_409_b200 import _binding
@@ -50,17 +51,40 @@ def test_workspace_size_arithmetic(lib):
 
 def test_partition_heuristic(lib):
     # large batches: one CTA per (sequence, KV head), no split
-    assert pkv.decode_partition_size(64, 32, 128, 16, 2048, 1) == 0
-    assert pkv.decode_partition_size(192, 8, 128, 32, 32768, 2) == 0
+    assert pkv.decode_partition_size(64, 32, 32, 128, 16, 2048, 1) == 0
+    assert pkv.decode_partition_size(192, 64, 8, 128, 32, 32768, 2) == 0
     # small batches: block-multiple partitions of at least 256 tokens, shorter than the context
     for B in (8, 16, 32):
-        p = pkv.decode_partition_size(2, 2, 128, B, 10000, 1)
+        p = pkv.decode_partition_size(2, 2, 2, 128, B, 10000, 1)
         assert p % B == 0 and 256 <= p < 10000
-    assert pkv.decode_partition_size(1, 1, 128, 16, 200, 1) == 0
+    assert pkv.decode_partition_size(1, 1, 1, 128, 16, 200, 1) == 0
     # a long tail (max far above the mean) is cut at 1.5x the mean
-    p = pkv.decode_partition_size(256, 8, 128, 16, 4096, 2, total_context_tokens=256 * 1436)
+    p = pkv.decode_partition_size(256, 64, 8, 128, 16, 4096, 2, total_context_tokens=256 * 1436)
     assert p == 2160
-    assert pkv.decode_partition_size(192, 8, 128, 32, 32768, 2, total_context_tokens=192 * 16500) == 0
+    assert pkv.decode_partition_size(192, 64, 8, 128, 32, 32768, 2, total_context_tokens=192 * 16500) == 0
+    # query heads must group evenly over KV heads
+    with pytest.raises(pkv.PagedKVError):
+        pkv.decode_partition_size(64, 12, 8, 128, 16, 2048, 1)
+
+
+def test_partition_heuristic_fp8_waves(lib):
+    """E4M3 pools, one query head per KV head: fewer pairs than ~22 CTAs per SM are cut into parts of
+    Hkv * total / (22 * SMs - pairs / 2) tokens (at least 512, block multiples); grouped heads, large
+    batches, an unknown total and 16-bit pools stay unsplit."""
+    sms = 148  # the library's SM count when no device is visible
+    total = 64 * 1039
+    p = pkv.decode_partition_size(64, 32, 32, 128, 16, 2029, pkv.FP8_E4M3, total_context_tokens=total)
+    want = -(-32 * total // (22 * sms - 64 * 32 // 2))
+    assert p == -(-want // 16) * 16 == 960
+    total = 32 * 2560
+    p = pkv.decode_partition_size(32, 32, 32, 128, 16, 4096, pkv.FP8_E4M3, total_context_tokens=total)
+    assert p == 960  # 32 x 81920 / (3256 - 512) = 955.4, rounded up to a block multiple
+    # short contexts: at least 512 tokens per part, and none when that covers the longest
+    assert pkv.decode_partition_size(64, 32, 32, 128, 16, 600, pkv.FP8_E4M3, total_context_tokens=64 * 300) == 512
+    assert pkv.decode_partition_size(64, 32, 32, 128, 16, 512, pkv.FP8_E4M3, total_context_tokens=64 * 300) == 0
+    for args, total in [((128, 32, 32), 128 * 1088), ((256, 64, 8), 256 * 1088), ((64, 32, 32), 0)]:
+        assert pkv.decode_partition_size(*args, 128, 16, 2048, pkv.FP8_E4M3, total_context_tokens=total) == 0
+    assert pkv.decode_partition_size(64, 32, 32, 128, 16, 2029, torch.float16, total_context_tokens=64 * 1039) == 0
 
 
 def test_host_rejections_before_launch(lib):

@@ -131,7 +131,8 @@ def test_llama7b_decode_fp8_full_sampled():
     eight sampled sequences against the oracle."""
     w = workloads.llama7b_decode_fp8(device="cuda", poison=True)
     pre_k, pre_v = w.key_caches[0].clone(), w.value_caches[0].clone()
-    part = pkv.decode_partition_size(w.num_seqs, w.num_kv_heads, w.head_dim, w.block_size, w.max_context_len, 3,
+    part = pkv.decode_partition_size(w.num_seqs, w.num_q_heads, w.num_kv_heads, w.head_dim, w.block_size,
+                                     w.max_context_len, 3,
                                      int(w.context_lens.sum()))
     out = gpu_decode_step(w, partition_size=part)
     torch.cuda.synchronize()
@@ -145,7 +146,8 @@ def test_gqa70b_decode_fp8_one_layer_sampled():
     """256 sequences, 64 q heads over 8 KV heads, lognormal contexts, bf16 query, FP8 pools (one layer)."""
     w = workloads.gqa70b_decode_fp8(device="cuda", num_layers=1, poison=True)
     pre_k, pre_v = w.key_caches[0].clone(), w.value_caches[0].clone()
-    part = pkv.decode_partition_size(w.num_seqs, w.num_kv_heads, w.head_dim, w.block_size, w.max_context_len, 3,
+    part = pkv.decode_partition_size(w.num_seqs, w.num_q_heads, w.num_kv_heads, w.head_dim, w.block_size,
+                                     w.max_context_len, 3,
                                      int(w.context_lens.sum()))
     out = gpu_decode_step(w, partition_size=part)
     torch.cuda.synchronize()
@@ -219,7 +221,8 @@ def test_mixed_step_fp8_sampled():
                                           torch.from_numpy(m.query_start_loc).cuda(), int(m.chunk_lens.max()),
                                           w.scale, ks, vs)
     bt, cl, _ = gpu_tables(w)
-    part = pkv.decode_partition_size(w.num_seqs, w.num_kv_heads, w.head_dim, w.block_size, w.max_context_len, 3,
+    part = pkv.decode_partition_size(w.num_seqs, w.num_q_heads, w.num_kv_heads, w.head_dim, w.block_size,
+                                     w.max_context_len, 3,
                                      int(w.context_lens.sum()))
     dout = torch.empty_like(w.queries[0])
     pkv.paged_attention_decode_fp8(dout, w.queries[0], kc, vc, bt, cl, w.scale, ks, vs, w.max_context_len,
