@@ -38,6 +38,7 @@ import torch
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
+L2_BYTES = 126e6  # B200 L2
 METRIC = "paged decode attention tokens/s and KV GB/s as % of B200 HBM peak (1 GPU)"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
@@ -79,6 +80,19 @@ class DecodeStep:
         # algorithmic bytes of one decode call: K/V once, q, out, block ids, lengths
         self.decode_bytes = self.kv_bytes + 2 * w.queries[0].numel() * t + 4 * nblocks + 4 * w.num_seqs
         self.tokens = w.num_seqs  # one generated token per sequence per step
+        # K/V bytes of the distinct physical blocks a step reads (shared blocks once)
+        used = [w.block_tables[s, :-(-int(c) // w.block_size)] for s, c in enumerate(w.context_lens)]
+        distinct = np.unique(np.concatenate(used)).size if used else 0
+        self.unique_kv_bytes = 2 * distinct * w.block_size * w.num_kv_heads * w.head_dim * tkv * self.layers
+
+    def l2_note(self):
+        """How the timed steps stand to the 126 MB L2."""
+        if self.unique_kv_bytes >= 2 * L2_BYTES:
+            return "inputs larger than L2 (K/V pools %.2f GB per layer)" % (
+                2 * self.w.key_caches[0].numel() * self.w.key_caches[0].element_size() / 1e9)
+        return ("distinct K/V blocks read per step %.3f GB, under twice the 126 MB L2: what one step reads "
+                "(the shared prefix above all) may stay cached for the next unless --flush-l2"
+                % (self.unique_kv_bytes / 1e9))
 
     def launches_per_step(self):
         return self.layers * (2 + (1 if self.parts > 1 else 0))
@@ -603,6 +617,9 @@ def main():
     ap.add_argument("--layers", type=int, default=None, help="cap on distinct layer pools (gqa70b_decode_bf16)")
     ap.add_argument("--no-graph", dest="graph", action="store_false",
                     help="launch every kernel of every step instead of replaying one captured CUDA graph")
+    ap.add_argument("--flush-l2", action="store_true",
+                    help="write a 512 MB buffer before every timed step (outside its events) so that no step "
+                         "finds the previous one's K/V in L2; the steps' own durations are summed")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
 
@@ -645,21 +662,33 @@ def main():
         graph.replay()
         torch.cuda.synchronize()
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    flush = torch.empty(512 << 20, dtype=torch.uint8, device=dev) if args.flush_l2 else None
+    per_step = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                for _ in range(args.steps)] if flush is not None else None
     h0 = time.perf_counter()
     torch.cuda.nvtx.range_push("timed")
     t0.record()
     for i in range(args.steps):
+        if flush is not None:
+            flush.fill_(i & 0xFF)
+            per_step[i][0].record()
         if graph is not None:
             graph.replay()
         else:
             step.run(timer=timer, step=i)
+        if flush is not None:
+            per_step[i][1].record()
     t1.record()
     torch.cuda.nvtx.range_pop()
     torch.cuda.synchronize()
     clocks.mark(h0, time.perf_counter())
     clk = clocks.stop()
     barrier(ws)
-    ms_total = max_over_ranks(t0.elapsed_time(t1), ws)
+    if flush is None:
+        ms_total = max_over_ranks(t0.elapsed_time(t1), ws)
+    else:
+        ms_total = max_over_ranks(sum(a.elapsed_time(b) for a, b in per_step), ws)
+        del flush
     ms_step = ms_total / args.steps
     if graph is not None:
         # the decode-call duration for the roofline, from a short plain loop
@@ -702,8 +731,10 @@ def main():
         "config": {"workload": cname, "num_seqs": w.num_seqs, "num_q_heads": w.num_q_heads,
                    "num_kv_heads": w.num_kv_heads, "head_dim": w.head_dim, "block_size": w.block_size,
                    "layers_per_step": step.layers, "partition_size": step.part, "cuda_graph": bool(args.graph),
-                   "l2": "inputs larger than L2 (K/V pools %.2f GB per layer)" % (
-                       2 * w.key_caches[0].numel() * w.key_caches[0].element_size() / 1e9),
+                   "l2": ("L2 flushed (512 MB written) before every step, outside the step's events; "
+                          if args.flush_l2 else "") + (step.l2_note() if hasattr(step, "l2_note") else
+                                                       "inputs larger than L2 (K/V pools %.2f GB per layer)" % (
+                       2 * w.key_caches[0].numel() * w.key_caches[0].element_size() / 1e9)),
                    "parallelism": f"replicas x{ws}"},
         "kv_gbs": step.kv_bytes * step.layers / (ms_step / 1e3) / 1e9,
         "roofline": {"bound": "hbm", "kernel": getattr(step, "kernel", "paged_attention_decode (decode + merge kernels)"),
@@ -721,6 +752,14 @@ def main():
         line["roofline"]["traffic"] = ratio * step.decode_bytes  # DRAM bytes per decode call
         line["roofline"]["traffic_unit"] = "bytes per launch"
         line["roofline"]["traffic_source"] = source + " (smaller case, scaled by algorithmic bytes)"
+    if getattr(step, "unique_kv_bytes", None) and 2 * step.unique_kv_bytes < step.kv_bytes * step.layers:
+        # shared blocks: most logical bytes come from L2, so the HBM fraction above exceeds 1 by design
+        uniq = step.unique_kv_bytes / step.layers
+        line["roofline"]["distinct_kv_bytes_per_launch"] = uniq
+        line["roofline"]["achieved_distinct_gbs"] = uniq / (unit_ms / 1e3) / 1e9
+        line["roofline"]["note"] = ("achieved counts logical K/V bytes (each sequence's blocks); %.0f%% of them are "
+                                    "shared blocks served from L2, so frac > 1 measures the reuse, not HBM"
+                                    % (100 * (1 - uniq / step.kv_bytes)))
     if isinstance(step, MixedStep):
         line["prefill_tokens_per_s"] = ws * step.prefill_tokens / (ms_step / 1e3)
         line["prefill_flops_per_step"] = step.prefill_flops
