@@ -10,9 +10,12 @@
 
 namespace pkv {
 
-// One CTA per token (grid-stride over tokens).  A token's K row and V row are
-// each contiguous (num_kv_heads * head_dim elements) in the source and, in the
-// [num_blocks, block_size, num_kv_heads, head_dim] pool, at row `slot`.
+// Grid (x, y): blockIdx.x picks a 128-vector slice of a row, y strides over
+// tokens, so a small batch (one new token per sequence) still spreads over
+// hundreds of CTAs with one vector of K and one of V per thread.  A token's K
+// row and V row are each contiguous (num_kv_heads * head_dim elements) in the
+// source and, in the [num_blocks, block_size, num_kv_heads, head_dim] pool, at
+// row `slot`.
 __global__ void __launch_bounds__(128) reshape_and_cache_kernel(const uint4* __restrict__ key,
                                                                 const uint4* __restrict__ value,
                                                                 uint4* __restrict__ key_cache,
@@ -20,22 +23,19 @@ __global__ void __launch_bounds__(128) reshape_and_cache_kernel(const uint4* __r
                                                                 const int64_t* __restrict__ slot_mapping,
                                                                 int64_t num_tokens, int row_vecs,
                                                                 int64_t num_slots) {
-    for (int64_t t = blockIdx.x; t < num_tokens; t += gridDim.x) {
+    const int i = blockIdx.x * blockDim.x + threadIdx.x;
+    for (int64_t t = blockIdx.y; t < num_tokens; t += gridDim.y) {
         const int64_t slot = slot_mapping[t];
         if (slot < 0) continue;  // padding token
         if (slot >= num_slots) {
-            if (threadIdx.x == 0) flag_error(PKV_DEVERR_SLOT);
+            if (i == 0) flag_error(PKV_DEVERR_SLOT);
             continue;
         }
-        const uint4* ks = key + t * row_vecs;
-        const uint4* vs = value + t * row_vecs;
-        uint4* kd = key_cache + slot * row_vecs;
-        uint4* vd = value_cache + slot * row_vecs;
-        for (int i = threadIdx.x; i < row_vecs; i += blockDim.x) {
-            const uint4 a = ks[i];
-            const uint4 b = vs[i];
-            kd[i] = a;
-            vd[i] = b;
+        if (i < row_vecs) {
+            const uint4 a = key[t * row_vecs + i];
+            const uint4 b = value[t * row_vecs + i];
+            key_cache[slot * row_vecs + i] = a;
+            value_cache[slot * row_vecs + i] = b;
         }
     }
 }
@@ -78,8 +78,9 @@ __device__ __forceinline__ uint2 quantise8(const float (&f)[8], float scale) {
     return make_uint2(w[0] | (w[1] << 16), w[2] | (w[3] << 16));
 }
 
-// One CTA per token (grid-stride); each thread quantises 8 consecutive
-// elements of the token's K row and of its V row.
+// Grid (x, y) as for reshape_and_cache_kernel: blockIdx.x picks 128 groups
+// of 8 consecutive elements of a row, y strides over tokens; each thread
+// quantises one group of the token's K row and the same group of its V row.
 template <typename TS>
 __global__ void __launch_bounds__(128) reshape_and_cache_fp8_kernel(const TS* __restrict__ key,
                                                                     const TS* __restrict__ value,
@@ -89,14 +90,15 @@ __global__ void __launch_bounds__(128) reshape_and_cache_fp8_kernel(const TS* __
                                                                     int64_t num_tokens, int row_elems,
                                                                     int64_t num_slots, float k_scale, float v_scale) {
     const int groups = row_elems / 8;
-    for (int64_t t = blockIdx.x; t < num_tokens; t += gridDim.x) {
+    const int i = blockIdx.x * blockDim.x + threadIdx.x;
+    for (int64_t t = blockIdx.y; t < num_tokens; t += gridDim.y) {
         const int64_t slot = slot_mapping[t];
         if (slot < 0) continue;
         if (slot >= num_slots) {
-            if (threadIdx.x == 0) flag_error(PKV_DEVERR_SLOT);
+            if (i == 0) flag_error(PKV_DEVERR_SLOT);
             continue;
         }
-        for (int i = threadIdx.x; i < groups; i += blockDim.x) {
+        if (i < groups) {
             float kf[8], vf[8];
             load8(key + t * row_elems + 8 * i, kf);
             load8(value + t * row_elems + 8 * i, vf);

@@ -531,7 +531,7 @@ int pkv_reshape_and_cache(const void* key, const void* value, void* key_cache, v
     if (num_tokens < 0 || num_kv_heads <= 0 || head_dim <= 0 || block_size <= 0 || num_blocks <= 0)
         return PKV_EINVAL;
     const int64_t row_bytes = (int64_t)num_kv_heads * head_dim * eb;
-    if (row_bytes % 16 != 0) return PKV_EUNSUPPORTED;
+    if (row_bytes % 16 != 0 || row_bytes / 16 > INT32_MAX) return PKV_EUNSUPPORTED;
     if (num_tokens == 0) return PKV_OK;
     if (!key || !value || !key_cache || !value_cache || !slot_mapping) return PKV_EINVAL;
     if (!aligned16(key) || !aligned16(value) || !aligned16(key_cache) || !aligned16(value_cache) ||
@@ -546,10 +546,11 @@ int pkv_reshape_and_cache(const void* key, const void* value, void* key_cache, v
         for (int64_t v : sm)
             if (v >= num_slots) return PKV_ERANGE;
     }
-    const int grid = (int)std::min<int64_t>(num_tokens, 65535);
+    const int row_vecs = (int)(row_bytes / 16);
+    const dim3 grid((unsigned)ceil_div(row_vecs, 128), (unsigned)std::min<int64_t>(num_tokens, 65535));
     pkv::reshape_and_cache_kernel<<<grid, 128, 0, s>>>(
         static_cast<const uint4*>(key), static_cast<const uint4*>(value), static_cast<uint4*>(key_cache),
-        static_cast<uint4*>(value_cache), slot_mapping, num_tokens, (int)(row_bytes / 16), num_slots);
+        static_cast<uint4*>(value_cache), slot_mapping, num_tokens, row_vecs, num_slots);
     PKV_CUDA(cudaGetLastError());
     return PKV_OK;
 }
@@ -578,7 +579,7 @@ int pkv_reshape_and_cache_fp8(const void* key, const void* value, void* key_cach
         for (int64_t v : sm)
             if (v >= num_slots) return PKV_ERANGE;
     }
-    const int grid = (int)std::min<int64_t>(num_tokens, 65535);
+    const dim3 grid((unsigned)ceil_div(row_elems / 8, 128), (unsigned)std::min<int64_t>(num_tokens, 65535));
     uint2* kc = static_cast<uint2*>(key_cache);
     uint2* vc = static_cast<uint2*>(value_cache);
     switch (src_dtype) {
