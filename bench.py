@@ -352,8 +352,8 @@ class MultiTokenStep:
 TRAFFIC_PER_ALGORITHMIC_BYTE = {
     "llama7b_decode_f16": ((287.471104 + 3.418624) / 285.38096,
                            "profiles/paged_decode_mma_kernel_llama7b_16seq_full.md"),
-    "llama7b_decode_fp8": ((305.048832 + 4.018688) / 303.293524,
-                           "profiles/paged_decode_fp8_kernel_llama7b_fp8_32seq.md"),
+    "llama7b_decode_fp8": ((305.044224 + 3.7632 + 1.388544 + 0.0) / 303.293524,
+                           "profiles/paged_decode_fp8_kernel_llama7b_fp8_launches.md (decode + merge)"),
 }
 
 
