@@ -1,9 +1,8 @@
 // index_kernels.cuh -- the two indexing kernels of the paged cache:
 //   reshape_and_cache (write new tokens' K/V into their physical slots) and
 //   copy_blocks (copy-on-write of shared blocks).
-// Both are pure data movement: 16-byte vector loads and stores, several in
-// flight per thread, bounded by HBM bandwidth (or by launch latency when the
-// token count is small).
+// Both are pure data movement in 16-byte vectors, bounded by HBM bandwidth
+// (or by launch latency when the token count is small).
 #pragma once
 
 #include "ptx.cuh"
