@@ -33,6 +33,19 @@
  *     with that hash is cached yet.
  *   - Freeing a sequence releases its blocks from the last to the first, so a
  *     cached prefix's deeper blocks enter the LRU list (and leave it) first.
+ *   - Swapping (case-study page, section 三: under memory pressure a request is
+ *     pre-empted by moving its KV to CPU memory, and resumed later; tutorial
+ *     page 4.3).  An optional host pool of num_host_blocks blocks has its own
+ *     free stack (block 0 on top).  Swapping a sequence out takes one host
+ *     block per device block, in logical order from the top of that stack,
+ *     reports the (device, host) pairs, and then releases the device blocks
+ *     like a free (last to first; cached ones stay cached).  Swapping it in
+ *     takes one device block per host block, in logical order (free stack,
+ *     else LRU eviction), reports the (host, device) pairs, and pushes the
+ *     host blocks back last to first.  Swapped-in blocks are private: they are
+ *     not re-entered in the prefix cache (the hash chain of later blocks
+ *     continues).  A swapped-out sequence can only be swapped in, freed or
+ *     asked for its token count.
  *
  * The manager is not thread-safe; one owner calls it.
  */
@@ -84,7 +97,9 @@ int pkv_bm_append_batch(pkv_block_manager* bm, const int64_t* seq_ids, const int
                         int64_t* slots_out, int64_t* cow_pairs_out, int64_t max_pairs, int64_t* num_pairs,
                         int64_t* num_done);
 
-/* child shares every block of parent (parallel sampling / beam search). */
+/* child shares every block of parent (parallel sampling / beam search).
+ * append, fork (as parent), slots and block_table reject a swapped-out
+ * sequence with PKV_BM_EINVAL. */
 int pkv_bm_fork(pkv_block_manager* bm, int64_t parent_id, int64_t child_id);
 
 /* Release seq_id's blocks (cached ones stay cached until evicted). */
@@ -103,8 +118,32 @@ int64_t pkv_bm_num_tokens(const pkv_block_manager* bm, int64_t seq_id);
 
 /* Counters: [0] free blocks, [1] evictable cached blocks, [2] cached blocks
  * in total, [3] cache-hit blocks so far, [4] evictions so far, [5] CoW copies
- * so far, [6] live sequences.  Returns the number written (<= n). */
+ * so far, [6] sequences (resident and swapped out), [7] free host blocks,
+ * [8] swapped-out sequences.  Returns the number written (<= n). */
 int pkv_bm_stats(const pkv_block_manager* bm, int64_t* out, int n);
+
+/* Size the host pool used by swapping (0 at creation).  Allowed only while no
+ * sequence is swapped out; the host free stack restarts as [0, ..., n-1]. */
+int pkv_bm_set_host_blocks(pkv_block_manager* bm, int64_t num_host_blocks);
+
+/* Pre-empt seq_id: pairs_out ([max_pairs][2] int64) receives one (device
+ * block, host block) pair per block of its table, in logical order, and
+ * *num_pairs their count.  Copy those blocks device -> host (pkv_swap_blocks)
+ * before any later call can hand the released device blocks out again, i.e.
+ * enqueue the copy before the K/V writes of the next step.  PKV_BM_ENOSPACE
+ * when the host pool has too few free blocks, PKV_BM_EBUFFER when max_pairs is
+ * too small; on failure nothing changes. */
+int pkv_bm_swap_out(pkv_block_manager* bm, int64_t seq_id, int64_t* pairs_out, int64_t max_pairs,
+                    int64_t* num_pairs);
+
+/* Resume a swapped-out seq_id: pairs_out receives one (host block, device
+ * block) pair per block, in logical order; copy them host -> device before the
+ * sequence's next attention.  The sequence's table then lists the new device
+ * blocks.  PKV_BM_ENOSPACE when the device pool has too few free or evictable
+ * blocks, PKV_BM_EBUFFER when max_pairs is too small; on failure nothing
+ * changes. */
+int pkv_bm_swap_in(pkv_block_manager* bm, int64_t seq_id, int64_t* pairs_out, int64_t max_pairs,
+                   int64_t* num_pairs);
 
 /* Reference count of a physical block (or a negative status). */
 int pkv_bm_ref_count(const pkv_block_manager* bm, int64_t block);

@@ -3,9 +3,10 @@
 It restates, with Python lists and dicts, the policy written in
 ``include/pagedkv_block_manager.h``: a free stack with block 0 on top, blocks
 taken on demand, reference counts, copy-on-write of a shared partial last
-block, and a prefix cache of full blocks keyed by their exact content chain
+block, a prefix cache of full blocks keyed by their exact content chain
 (parent block's key, token ids) -- no hashing -- whose unreferenced blocks sit
-in an LRU list, oldest evicted first.  The data model it follows is that of the
+in an LRU list, oldest evicted first, and swapping of whole sequences to a
+host pool with its own free stack.  The data model it follows is that of the
 vLLM case-study page ("vLLM 与 PagedAttention", sections 二 and 四) and the
 298.name page's ``PagedKVCache`` sketch.  The tests compare the C++ manager to
 this model operation by operation.
@@ -18,7 +19,7 @@ class NoSpace(Exception):
 
 
 class BlockManagerModel:
-    def __init__(self, num_blocks, block_size, prefix_caching=True):
+    def __init__(self, num_blocks, block_size, prefix_caching=True, num_host_blocks=0):
         self.B = block_size
         self.prefix_caching = prefix_caching
         self.free_stack = list(range(num_blocks - 1, -1, -1))  # block 0 on top (end of the list)
@@ -28,6 +29,7 @@ class BlockManagerModel:
         self.lru = []  # oldest first
         self.seqs = {}
         self.hits = self.evictions = self.cows = 0
+        self.host_free = list(range(num_host_blocks - 1, -1, -1))  # host block 0 on top
 
     # -- blocks
     def _take(self):
@@ -126,12 +128,42 @@ class BlockManagerModel:
             self.ref[b] += 1
 
     def free(self, sid):
-        for b in reversed(self.seqs.pop(sid)["blocks"]):
+        seq = self.seqs.pop(sid)
+        self.host_free += list(reversed(seq.get("host", [])))
+        for b in reversed(seq["blocks"]):
             self._release(b)
+
+    # -- swapping (a pre-empted sequence's blocks move to the host pool and back)
+    def swap_out(self, sid):
+        seq = self.seqs[sid]
+        assert "host" not in seq
+        if len(seq["blocks"]) > len(self.host_free):
+            raise NoSpace()
+        host = [self.host_free.pop() for _ in seq["blocks"]]
+        pairs = list(zip(seq["blocks"], host))
+        for b in reversed(seq["blocks"]):
+            self._release(b)
+        seq["blocks"], seq["host"] = [], host
+        return pairs
+
+    def swap_in(self, sid):
+        seq = self.seqs[sid]
+        host = seq["host"]
+        if len(host) > self._available():
+            raise NoSpace()
+        seq["blocks"] = [self._take() for _ in host]
+        pairs = list(zip(host, seq["blocks"]))
+        self.host_free += list(reversed(host))
+        del seq["host"]
+        return pairs
+
+    def swapped(self, sid):
+        return "host" in self.seqs[sid]
 
     def block_table(self, sid):
         return list(self.seqs[sid]["blocks"])
 
     def stats(self):
         return {"free": len(self.free_stack), "evictable": len(self.lru), "cached": len(self.cache),
-                "hits": self.hits, "evictions": self.evictions, "cow_copies": self.cows, "sequences": len(self.seqs)}
+                "hits": self.hits, "evictions": self.evictions, "cow_copies": self.cows, "sequences": len(self.seqs),
+                "free_host": len(self.host_free), "swapped": sum(1 for s in self.seqs.values() if "host" in s)}

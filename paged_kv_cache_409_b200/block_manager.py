@@ -50,8 +50,12 @@ def _lib():
         lib.pkv_bm_num_tokens.restype = I64
         lib.pkv_bm_stats.argtypes = [P, P, I]
         lib.pkv_bm_ref_count.argtypes = [P, I64]
-        for f in (lib.pkv_bm_add_sequence, lib.pkv_bm_append, lib.pkv_bm_append_batch, lib.pkv_bm_fork, lib.pkv_bm_free, lib.pkv_bm_slots,
-                  lib.pkv_bm_block_table, lib.pkv_bm_stats, lib.pkv_bm_ref_count):
+        lib.pkv_bm_set_host_blocks.argtypes = [P, I64]
+        lib.pkv_bm_swap_out.argtypes = [P, I64, P, I64, P]
+        lib.pkv_bm_swap_in.argtypes = [P, I64, P, I64, P]
+        for f in (lib.pkv_bm_add_sequence, lib.pkv_bm_append, lib.pkv_bm_append_batch, lib.pkv_bm_fork,
+                  lib.pkv_bm_free, lib.pkv_bm_slots, lib.pkv_bm_block_table, lib.pkv_bm_stats, lib.pkv_bm_ref_count,
+                  lib.pkv_bm_set_host_blocks, lib.pkv_bm_swap_out, lib.pkv_bm_swap_in):
             f.restype = I
         _bound = True
     return lib
@@ -70,16 +74,19 @@ def _ptr(a: np.ndarray):
 
 
 class BlockManager:
-    """One pool of ``num_blocks`` blocks of ``block_size`` tokens."""
+    """One pool of ``num_blocks`` blocks of ``block_size`` tokens (and, for
+    swapping, a host pool of ``num_host_blocks`` blocks)."""
 
-    STATS = ("free", "evictable", "cached", "hits", "evictions", "cow_copies", "sequences")
+    STATS = ("free", "evictable", "cached", "hits", "evictions", "cow_copies", "sequences", "free_host", "swapped")
 
-    def __init__(self, num_blocks: int, block_size: int, prefix_caching: bool = True):
+    def __init__(self, num_blocks: int, block_size: int, prefix_caching: bool = True, num_host_blocks: int = 0):
         self._l = _lib()
         self._h = self._l.pkv_bm_create(int(num_blocks), int(block_size), 1 if prefix_caching else 0)
         if not self._h:
             raise BlockManagerError("pkv_bm_create", EINVAL)
         self.num_blocks, self.block_size = int(num_blocks), int(block_size)
+        if num_host_blocks:
+            _check(self._l.pkv_bm_set_host_blocks(self._h, int(num_host_blocks)), "set_host_blocks")
 
     def close(self):
         if self._h:
@@ -128,6 +135,23 @@ class BlockManager:
 
     def free(self, seq_id: int):
         _check(self._l.pkv_bm_free(self._h, int(seq_id)), "free")
+
+    def _swap(self, fn, seq_id, what):
+        # a sequence of n tokens holds ceil(n / block_size) blocks, resident or not
+        tokens = _check(int(self._l.pkv_bm_num_tokens(self._h, int(seq_id))), what)
+        cap = max(-(-tokens // self.block_size), 1)
+        pairs = np.empty((cap, 2), dtype=np.int64)
+        k = ctypes.c_int64(0)
+        _check(fn(self._h, int(seq_id), _ptr(pairs), cap, ctypes.byref(k)), what)
+        return pairs[:k.value]
+
+    def swap_out(self, seq_id: int) -> np.ndarray:
+        """Pre-empt a sequence; returns its (device block, host block) pairs int64 [n, 2]."""
+        return self._swap(self._l.pkv_bm_swap_out, seq_id, "swap_out")
+
+    def swap_in(self, seq_id: int) -> np.ndarray:
+        """Resume a swapped-out sequence; returns its (host block, device block) pairs int64 [n, 2]."""
+        return self._swap(self._l.pkv_bm_swap_in, seq_id, "swap_in")
 
     def slots(self, seq_id: int, start: int, count: int) -> np.ndarray:
         out = np.empty(max(count, 1), dtype=np.int64)

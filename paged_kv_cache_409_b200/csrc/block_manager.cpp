@@ -1,6 +1,7 @@
 // block_manager.cpp -- host-side manager of the paged KV-cache pool: free
-// stack, reference counts, copy-on-write, and the hash-chain prefix cache with
-// LRU eviction declared in include/pagedkv_block_manager.h.  Pure host C++.
+// stack, reference counts, copy-on-write, the hash-chain prefix cache with
+// LRU eviction, and swapping of whole sequences to a host pool, declared in
+// include/pagedkv_block_manager.h.  Pure host C++.
 #include <cstdint>
 #include <cstring>
 #include <list>
@@ -36,10 +37,12 @@ struct CacheEntry {
 };
 
 struct Sequence {
-    std::vector<int32_t> blocks;
+    std::vector<int32_t> blocks;       // device blocks (empty while swapped out)
+    std::vector<int32_t> host_blocks;  // host blocks while swapped out
     std::vector<int32_t> tail;  // token ids of the last, partial block
     int64_t num_tokens = 0;
     uint64_t last_full_hash = 0;  // hash of the last full block (0 = none)
+    bool swapped = false;
 };
 
 }  // namespace
@@ -56,6 +59,9 @@ struct pkv_block_manager {
     std::vector<std::list<int32_t>::iterator> lru_pos;
     std::vector<char> in_lru;
     std::unordered_map<int64_t, Sequence> seqs;
+    std::vector<int32_t> host_free;    // host pool's free stack, top = back
+    int64_t num_host_blocks = 0;
+    int64_t swapped = 0;               // sequences swapped out
     int64_t hits = 0, evictions = 0, cows = 0;
 
     int32_t take_block() {
@@ -108,6 +114,22 @@ struct pkv_block_manager {
     }
 
     int64_t available() const { return static_cast<int64_t>(free_stack.size() + lru.size()); }
+
+    // Return a swapped-out sequence's host blocks, last to first (the first on top).
+    void release_host(Sequence& s) {
+        for (auto h = s.host_blocks.rbegin(); h != s.host_blocks.rend(); ++h) host_free.push_back(*h);
+        s.host_blocks.clear();
+    }
+
+    // A live (not swapped-out) sequence, or nullptr.
+    Sequence* resident(int64_t seq_id) {
+        auto it = seqs.find(seq_id);
+        return it == seqs.end() || it->second.swapped ? nullptr : &it->second;
+    }
+    const Sequence* resident(int64_t seq_id) const {
+        auto it = seqs.find(seq_id);
+        return it == seqs.end() || it->second.swapped ? nullptr : &it->second;
+    }
 };
 
 extern "C" {
@@ -180,9 +202,9 @@ int pkv_bm_add_sequence(pkv_block_manager* bm, int64_t seq_id, const int32_t* to
 int pkv_bm_append(pkv_block_manager* bm, int64_t seq_id, const int32_t* tokens, int64_t num_tokens,
                   int64_t* slots_out, int64_t* cow_pairs_out, int64_t max_pairs, int64_t* num_pairs) {
     if (!bm || num_tokens < 0 || (num_tokens > 0 && (!tokens || !slots_out))) return PKV_BM_EINVAL;
-    auto it = bm->seqs.find(seq_id);
-    if (it == bm->seqs.end()) return PKV_BM_EINVAL;
-    Sequence& s = it->second;
+    Sequence* sp = bm->resident(seq_id);
+    if (!sp) return PKV_BM_EINVAL;
+    Sequence& s = *sp;
     const int B = bm->block_size;
     // Blocks needed: one copy if the partial last block is shared, plus the new ones.
     const int64_t off0 = s.num_tokens % B;
@@ -237,9 +259,9 @@ int pkv_bm_append_batch(pkv_block_manager* bm, const int64_t* seq_ids, const int
 
 int pkv_bm_fork(pkv_block_manager* bm, int64_t parent_id, int64_t child_id) {
     if (!bm || parent_id == child_id) return PKV_BM_EINVAL;
-    auto it = bm->seqs.find(parent_id);
-    if (it == bm->seqs.end() || bm->seqs.count(child_id)) return PKV_BM_EINVAL;
-    Sequence child = it->second;
+    const Sequence* parent = bm->resident(parent_id);
+    if (!parent || bm->seqs.count(child_id)) return PKV_BM_EINVAL;
+    Sequence child = *parent;
     for (int32_t b : child.blocks) ++bm->ref[b];
     bm->seqs.emplace(child_id, std::move(child));
     return PKV_BM_OK;
@@ -249,6 +271,10 @@ int pkv_bm_free(pkv_block_manager* bm, int64_t seq_id) {
     if (!bm) return PKV_BM_EINVAL;
     auto it = bm->seqs.find(seq_id);
     if (it == bm->seqs.end()) return PKV_BM_EINVAL;
+    if (it->second.swapped) {
+        bm->release_host(it->second);
+        --bm->swapped;
+    }
     // release from the last block to the first, so that the LRU list keeps a
     // prefix's deeper blocks older than its shallower ones (evicted first)
     const std::vector<int32_t>& blocks = it->second.blocks;
@@ -257,14 +283,69 @@ int pkv_bm_free(pkv_block_manager* bm, int64_t seq_id) {
     return PKV_BM_OK;
 }
 
+int pkv_bm_set_host_blocks(pkv_block_manager* bm, int64_t num_host_blocks) {
+    if (!bm || num_host_blocks < 0 || num_host_blocks > INT32_MAX || bm->swapped) return PKV_BM_EINVAL;
+    bm->num_host_blocks = num_host_blocks;
+    bm->host_free.resize(num_host_blocks);
+    for (int64_t i = 0; i < num_host_blocks; ++i)
+        bm->host_free[i] = static_cast<int32_t>(num_host_blocks - 1 - i);
+    return PKV_BM_OK;
+}
+
+int pkv_bm_swap_out(pkv_block_manager* bm, int64_t seq_id, int64_t* pairs_out, int64_t max_pairs,
+                    int64_t* num_pairs) {
+    if (!bm || max_pairs < 0) return PKV_BM_EINVAL;
+    Sequence* sp = bm->resident(seq_id);
+    if (!sp) return PKV_BM_EINVAL;
+    Sequence& s = *sp;
+    const int64_t n = static_cast<int64_t>(s.blocks.size());
+    if (n > static_cast<int64_t>(bm->host_free.size())) return PKV_BM_ENOSPACE;
+    if (n > max_pairs || (n > 0 && !pairs_out)) return PKV_BM_EBUFFER;
+    for (int64_t i = 0; i < n; ++i) {
+        const int32_t h = bm->host_free.back();
+        bm->host_free.pop_back();
+        s.host_blocks.push_back(h);
+        pairs_out[2 * i] = s.blocks[i];
+        pairs_out[2 * i + 1] = h;
+    }
+    for (auto b = s.blocks.rbegin(); b != s.blocks.rend(); ++b) bm->release_block(*b);
+    s.blocks.clear();
+    s.swapped = true;
+    ++bm->swapped;
+    if (num_pairs) *num_pairs = n;
+    return PKV_BM_OK;
+}
+
+int pkv_bm_swap_in(pkv_block_manager* bm, int64_t seq_id, int64_t* pairs_out, int64_t max_pairs,
+                   int64_t* num_pairs) {
+    if (!bm || max_pairs < 0) return PKV_BM_EINVAL;
+    auto it = bm->seqs.find(seq_id);
+    if (it == bm->seqs.end() || !it->second.swapped) return PKV_BM_EINVAL;
+    Sequence& s = it->second;
+    const int64_t n = static_cast<int64_t>(s.host_blocks.size());
+    if (n > bm->available()) return PKV_BM_ENOSPACE;
+    if (n > max_pairs || (n > 0 && !pairs_out)) return PKV_BM_EBUFFER;
+    for (int64_t i = 0; i < n; ++i) {
+        const int32_t d = bm->take_block();
+        s.blocks.push_back(d);
+        pairs_out[2 * i] = s.host_blocks[i];
+        pairs_out[2 * i + 1] = d;
+    }
+    bm->release_host(s);
+    s.swapped = false;
+    --bm->swapped;
+    if (num_pairs) *num_pairs = n;
+    return PKV_BM_OK;
+}
+
 int pkv_bm_slots(const pkv_block_manager* bm, int64_t seq_id, int64_t start, int64_t count, int64_t* slots_out) {
     if (!bm || start < 0 || count < 0 || (count > 0 && !slots_out)) return PKV_BM_EINVAL;
-    auto it = bm->seqs.find(seq_id);
-    if (it == bm->seqs.end() || start + count > it->second.num_tokens) return PKV_BM_EINVAL;
+    const Sequence* s = bm->resident(seq_id);
+    if (!s || start + count > s->num_tokens) return PKV_BM_EINVAL;
     const int B = bm->block_size;
     for (int64_t i = 0; i < count; ++i) {
         const int64_t pos = start + i;
-        slots_out[i] = static_cast<int64_t>(it->second.blocks[pos / B]) * B + pos % B;
+        slots_out[i] = static_cast<int64_t>(s->blocks[pos / B]) * B + pos % B;
     }
     return PKV_BM_OK;
 }
@@ -272,9 +353,9 @@ int pkv_bm_slots(const pkv_block_manager* bm, int64_t seq_id, int64_t start, int
 int pkv_bm_block_table(const pkv_block_manager* bm, int64_t seq_id, int32_t* out, int64_t max_blocks,
                        int64_t* num_blocks) {
     if (!bm || max_blocks < 0 || (max_blocks > 0 && !out)) return PKV_BM_EINVAL;
-    auto it = bm->seqs.find(seq_id);
-    if (it == bm->seqs.end()) return PKV_BM_EINVAL;
-    const std::vector<int32_t>& b = it->second.blocks;
+    const Sequence* s = bm->resident(seq_id);
+    if (!s) return PKV_BM_EINVAL;
+    const std::vector<int32_t>& b = s->blocks;
     if (num_blocks) *num_blocks = static_cast<int64_t>(b.size());
     if (static_cast<int64_t>(b.size()) > max_blocks) return PKV_BM_EBUFFER;
     for (int64_t i = 0; i < max_blocks; ++i) out[i] = i < static_cast<int64_t>(b.size()) ? b[i] : -1;
@@ -289,10 +370,11 @@ int64_t pkv_bm_num_tokens(const pkv_block_manager* bm, int64_t seq_id) {
 
 int pkv_bm_stats(const pkv_block_manager* bm, int64_t* out, int n) {
     if (!bm || n < 0 || (n > 0 && !out)) return PKV_BM_EINVAL;
-    const int64_t v[7] = {static_cast<int64_t>(bm->free_stack.size()), static_cast<int64_t>(bm->lru.size()),
+    const int64_t v[9] = {static_cast<int64_t>(bm->free_stack.size()), static_cast<int64_t>(bm->lru.size()),
                           static_cast<int64_t>(bm->cache.size()), bm->hits, bm->evictions, bm->cows,
-                          static_cast<int64_t>(bm->seqs.size())};
-    const int m = n < 7 ? n : 7;
+                          static_cast<int64_t>(bm->seqs.size()), static_cast<int64_t>(bm->host_free.size()),
+                          bm->swapped};
+    const int m = n < 9 ? n : 9;
     for (int i = 0; i < m; ++i) out[i] = v[i];
     return m;
 }

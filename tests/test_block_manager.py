@@ -5,7 +5,7 @@ import pytest
 
 from oracle.block_manager_model import BlockManagerModel, NoSpace
 from oracle_pins import golden
-from paged_kv_cache_409_b200.block_manager import BlockManager, NoSpaceError
+from paged_kv_cache_409_b200.block_manager import BlockManager, BlockManagerError, NoSpaceError
 
 
 @pytest.fixture(autouse=True)
@@ -205,3 +205,190 @@ def test_append_batch_equals_one_by_one():
             pa += [tuple(x) for x in p1.tolist()]
         assert sb.tolist() == sa and [tuple(x) for x in pb.tolist()] == pa
     assert a.stats() == b.stats()
+
+
+# ----------------------------------------------------------------------------- swapping
+
+def test_swap_out_and_in_moves_the_table_through_the_host_pool():
+    bm = BlockManager(16, 4, num_host_blocks=8)
+    bm.add_sequence(1, range(10))                        # 3 blocks: 0, 1, 2
+    bm.add_sequence(2, range(100, 105))                  # 2 blocks: 3, 4
+    table = bm.block_table(1).tolist()
+    out = bm.swap_out(1)
+    assert out.tolist() == [[b, h] for b, h in zip(table, [0, 1, 2])]
+    st = bm.stats()
+    assert st["swapped"] == 1 and st["free_host"] == 5 and st["sequences"] == 2
+    assert bm.num_tokens(1) == 10
+    # the released device blocks are handed out again (the two cached full blocks wait in the LRU list)
+    bm.append(2, range(7))
+    back = bm.swap_in(1)
+    assert back[:, 0].tolist() == [0, 1, 2]
+    assert bm.block_table(1).tolist() == back[:, 1].tolist()
+    assert bm.stats()["free_host"] == 8 and bm.stats()["swapped"] == 0
+    slots, pairs = bm.append(1, [5, 6])                  # resident again: appends continue at position 10
+    assert slots.tolist() == [back[2, 1] * 4 + 2, back[2, 1] * 4 + 3] and len(pairs) == 0
+
+
+def test_swapped_sequence_only_swaps_in_frees_or_counts():
+    bm = BlockManager(16, 4, num_host_blocks=4)
+    bm.add_sequence(1, range(6))
+    bm.swap_out(1)
+    for call in (lambda: bm.append(1, [1]), lambda: bm.fork(1, 2), lambda: bm.slots(1, 0, 1),
+                 lambda: bm.block_table(1), lambda: bm.swap_out(1)):
+        with pytest.raises(BlockManagerError) as e:
+            call()
+        assert not isinstance(e.value, NoSpaceError)
+    assert bm._l.pkv_bm_set_host_blocks(bm._h, 8) < 0     # no resizing of the host pool while a sequence is out
+    assert bm.num_tokens(1) == 6
+    bm.free(1)                                            # returns its host blocks
+    assert bm.stats()["free_host"] == 4 and bm.stats()["sequences"] == 0
+    with pytest.raises(BlockManagerError):
+        bm.swap_in(1)
+
+
+def test_swap_without_room_changes_nothing():
+    bm = BlockManager(6, 4, num_host_blocks=2)
+    bm.add_sequence(1, range(12))                         # 3 blocks, host pool holds 2
+    before = (bm.stats(), bm.block_table(1).tolist())
+    with pytest.raises(NoSpaceError):
+        bm.swap_out(1)
+    assert (bm.stats(), bm.block_table(1).tolist()) == before
+    bm2 = BlockManager(4, 4, prefix_caching=False, num_host_blocks=4)
+    bm2.add_sequence(1, range(12))
+    bm2.swap_out(1)
+    bm2.add_sequence(2, range(100, 110))                  # 3 of the 4 device blocks
+    before = bm2.stats()
+    with pytest.raises(NoSpaceError):
+        bm2.swap_in(1)
+    assert bm2.stats() == before
+
+
+@pytest.mark.parametrize("seed", range(4))
+@pytest.mark.parametrize("caching", [True, False])
+def test_swap_matches_plain_model_on_random_operations(seed, caching):
+    """Random traces with pre-emption: every op is drawn valid for the model's current state, applied to both,
+    and the outputs (slots, CoW pairs, swap pairs), counters and resident tables compared after each."""
+    rng = np.random.default_rng(300 + seed)
+    B = int(rng.choice([4, 8]))
+    NB, NH = 64, 64
+    cpp, model = BlockManager(NB, B, caching, num_host_blocks=NH), BlockManagerModel(NB, B, caching, NH)
+    prefixes = [rng.integers(0, 30, int(rng.integers(0, 4 * B))).tolist() for _ in range(2)]
+    next_id = 0
+    swaps = 0
+    for _ in range(500):
+        resident = [s for s in model.seqs if not model.swapped(s)]
+        out = [s for s in model.seqs if model.swapped(s)]
+        r = rng.random()
+        if r < 0.2 or not model.seqs:
+            toks = prefixes[int(rng.integers(0, 2))] + rng.integers(0, 30, int(rng.integers(0, 2 * B))).tolist()
+            op = ("add", next_id, toks)
+            next_id += 1
+        elif r < 0.5 and resident:
+            op = ("append", resident[int(rng.integers(0, len(resident)))],
+                  rng.integers(0, 30, int(rng.integers(1, B + 2))).tolist())
+        elif r < 0.6 and resident:
+            op = ("fork", resident[int(rng.integers(0, len(resident)))], next_id)
+            next_id += 1
+        elif r < 0.72 and resident:
+            op = ("swap_out", resident[int(rng.integers(0, len(resident)))])
+        elif r < 0.84 and out:
+            op = ("swap_in", out[int(rng.integers(0, len(out)))])
+        else:
+            ids = list(model.seqs)
+            op = ("free", ids[int(rng.integers(0, len(ids)))])
+        results = []
+        for side in (cpp, model):
+            try:
+                if op[0] == "add":
+                    v = side.add_sequence(op[1], op[2])
+                elif op[0] == "append":
+                    s, p = side.append(op[1], op[2])
+                    v = (list(map(int, s)), [tuple(map(int, x)) for x in p])
+                elif op[0] == "fork":
+                    v = side.fork(op[1], op[2])
+                elif op[0] in ("swap_out", "swap_in"):
+                    v = [tuple(map(int, x)) for x in getattr(side, op[0])(op[1])]
+                else:
+                    v = side.free(op[1])
+            except (NoSpaceError, NoSpace):
+                v = "nospace"
+            results.append(v)
+        assert results[0] == results[1], (op, results)
+        swaps += op[0].startswith("swap") and results[0] != "nospace"
+        assert cpp.stats() == model.stats(), op
+        for sid in model.seqs:
+            assert cpp.num_tokens(sid) == model.seqs[sid]["n"]
+            if not model.swapped(sid):
+                assert cpp.block_table(sid).tolist() == model.block_table(sid), (op, sid)
+    assert swaps >= 30
+
+
+def test_swapped_kv_survives_reuse_of_its_device_blocks():
+    """A host mirror of the pools: every token's K row is a function of (position, token) written at its
+    slot; CoW pairs copy blocks, swap pairs move them to a host pool and back.  After every step each
+    resident sequence's rows, gathered through its table, must equal what was written -- across
+    pre-emptions whose device blocks other sequences took meanwhile."""
+    rng = np.random.default_rng(77)
+    B, NB, NH, W = 4, 24, 16, 3
+    bm = BlockManager(NB, B, num_host_blocks=NH)
+    dev = np.full((NB * B, W), -1.0)
+    host = np.full((NH * B, W), -1.0)
+    row = lambda pos, tok: np.array([pos, tok, 1000.0 * pos + tok])
+    tokens = {}
+
+    def write(slots, start, toks):
+        for i, (sl, t) in enumerate(zip(slots, toks)):
+            dev[sl] = row(start + i, t)
+
+    def move(src, dst, pairs):
+        for a, b in pairs:
+            dst[b * B:(b + 1) * B] = src[a * B:(a + 1) * B]
+
+    system = rng.integers(0, 20, 9).tolist()
+    next_id, preempted = 0, 0
+    swapped_set = set()
+    for step in range(400):
+        live = [s for s in tokens if s not in swapped_set]
+        r = rng.random()
+        try:
+            if r < 0.15 or not tokens:
+                toks = system + rng.integers(0, 20, int(rng.integers(0, 6))).tolist()
+                cached = bm.add_sequence(next_id, toks)
+                write(bm.slots(next_id, cached, len(toks) - cached), cached, toks[cached:])
+                tokens[next_id] = toks
+                next_id += 1
+            elif r < 0.55 and live:
+                sid = live[int(rng.integers(0, len(live)))]
+                t = int(rng.integers(0, 20))
+                slots, pairs = bm.append(sid, [t])
+                move(dev, dev, pairs)
+                write(slots, len(tokens[sid]), [t])
+                tokens[sid].append(t)
+            elif r < 0.65 and live:
+                sid = live[int(rng.integers(0, len(live)))]
+                bm.fork(sid, next_id)
+                tokens[next_id] = list(tokens[sid])
+                next_id += 1
+            elif r < 0.8 and live:
+                sid = live[int(rng.integers(0, len(live)))]
+                move(dev, host, bm.swap_out(sid))
+                swapped_set.add(sid)
+                preempted += 1
+            elif r < 0.92 and swapped_set:
+                sid = sorted(swapped_set)[int(rng.integers(0, len(swapped_set)))]
+                move(host, dev, bm.swap_in(sid))
+                swapped_set.discard(sid)
+            else:
+                sid = list(tokens)[int(rng.integers(0, len(tokens)))]
+                bm.free(sid)
+                del tokens[sid]
+                swapped_set.discard(sid)
+        except NoSpaceError:
+            pass
+        for sid, toks in tokens.items():
+            if sid in swapped_set:
+                continue
+            got = dev[bm.slots(sid, 0, len(toks))] if toks else np.zeros((0, W))
+            want = np.array([row(p, t) for p, t in enumerate(toks)]).reshape(-1, W)
+            assert np.array_equal(got, want), (step, sid)
+    assert preempted >= 20

@@ -101,3 +101,73 @@ def test_block_manager_drives_decode_steps(pools):
     assert cows == 1                                 # the fork's first append copied the shared partial block
     assert pkv.get_device_error() == 0
     assert np.array_equal(kc.cpu().numpy().view(np.uint8), kn.view(np.uint8))
+
+
+def test_preemption_by_swap_keeps_decode_exact():
+    """Sequence 1 is pre-empted at step 4: the block manager hands out host blocks, swap_blocks moves its
+    K/V to a page-locked host pool, and its device blocks go back to the free stack, where sequence 0's
+    next block comes from.  At step 10 it resumes into new device blocks.  Every step's decode of the
+    resident sequences, and the pools at the end, match the oracle's host mirror."""
+    NBs, NH = 16, 8
+    rng = np.random.default_rng(31)
+    g = torch.Generator().manual_seed(31)
+    ek = torch.randn(VOCAB, Hkv, D, generator=g)
+    ev = torch.randn(VOCAB, Hkv, D, generator=g)
+    bm = BlockManager(NBs, B, prefix_caching=False, num_host_blocks=NH)
+    kc = torch.zeros(NBs, B, Hkv, D, dtype=DT, device="cuda")
+    vc = torch.zeros_like(kc)
+    hk = torch.zeros(NH, B, Hkv, D, dtype=DT).pin_memory()
+    hv = torch.zeros(NH, B, Hkv, D, dtype=DT).pin_memory()
+    kn, vn = np.zeros((NBs, B, Hkv, D), np.float16), np.zeros((NBs, B, Hkv, D), np.float16)
+    hkn, hvn = np.zeros((NH, B, Hkv, D), np.float16), np.zeros((NH, B, Hkv, D), np.float16)
+    orc = oracle.get()
+    tokens = {}
+
+    def write(start, toks, slots):
+        pos = np.arange(start, start + len(toks))
+        k, v = kv_of(toks, pos, ek), kv_of(toks, pos, ev)
+        sl = torch.from_numpy(np.asarray(slots, dtype=np.int64))
+        pkv.reshape_and_cache(k.cuda(), v.cuda(), kc, vc, sl.cuda())
+        orc.reshape_and_cache(k.numpy(), v.numpy(), kn, vn, sl.numpy(), oracle.F16)
+
+    for sid, n in ((0, 40), (1, 30), (2, 50)):
+        pr = rng.integers(0, VOCAB, n).tolist()
+        bm.add_sequence(sid, pr)
+        write(0, pr, bm.slots(sid, 0, n))
+        tokens[sid] = pr
+    live = [0, 1, 2]
+    reused = False
+    for step in range(16):
+        if step == 4:
+            pairs = bm.swap_out(1)
+            freed = set(pairs[:, 0].tolist())
+            pkv.swap_blocks(kc, vc, hk, hv, torch.from_numpy(pairs).cuda())
+            hkn[pairs[:, 1]], hvn[pairs[:, 1]] = kn[pairs[:, 0]], vn[pairs[:, 0]]
+            live.remove(1)
+        if step == 10:
+            pairs = bm.swap_in(1)
+            pkv.swap_blocks(hk, hv, kc, vc, torch.from_numpy(pairs).pin_memory())
+            kn[pairs[:, 1]], vn[pairs[:, 1]] = hkn[pairs[:, 0]], hvn[pairs[:, 0]]
+            live = [0, 1, 2]
+        new = rng.integers(0, VOCAB, len(live))
+        slots, cow = bm.append_batch(live, new)
+        assert len(cow) == 0
+        for i, sid in enumerate(live):
+            write(len(tokens[sid]), [int(new[i])], [slots[i]])
+            tokens[sid].append(int(new[i]))
+        if 4 <= step < 10:
+            reused |= bool(freed & {int(b) for b in bm.block_table(0)})
+        lens = np.array([bm.num_tokens(s) for s in live], dtype=np.int32)
+        bt = bm.tables(live, int(-(-lens.max() // B)))
+        q = torch.randn(len(live), Hq, D, generator=g).to(DT)
+        out = torch.empty(len(live), Hq, D, dtype=DT, device="cuda")
+        scale = float(np.float32(D ** -0.5))
+        pkv.paged_attention_decode(out, q.cuda(), kc, vc, torch.from_numpy(bt).cuda(), torch.from_numpy(lens).cuda(),
+                                   scale, int(lens.max()))
+        ref = orc.paged_attention_decode(q.numpy(), kn, vn, bt, lens, scale, oracle.F16)
+        assert_close(out, ref, DT, f"step {step}")
+    assert reused                                     # sequence 0 wrote into a block sequence 1 had released
+    torch.cuda.synchronize()
+    assert pkv.get_device_error() == 0
+    assert np.array_equal(kc.cpu().numpy().view(np.uint16), kn.view(np.uint16))
+    assert np.array_equal(vc.cpu().numpy().view(np.uint16), vn.view(np.uint16))
