@@ -365,7 +365,7 @@ int pkv_bm_block_table(const pkv_block_manager* bm, int64_t seq_id, int32_t* out
 int64_t pkv_bm_num_tokens(const pkv_block_manager* bm, int64_t seq_id) {
     if (!bm) return PKV_BM_EINVAL;
     auto it = bm->seqs.find(seq_id);
-    return it == bm->seqs.end() ? PKV_BM_EINVAL : it->second.num_tokens;
+    return it == bm->seqs.end() ? static_cast<int64_t>(PKV_BM_EINVAL) : it->second.num_tokens;
 }
 
 int pkv_bm_stats(const pkv_block_manager* bm, int64_t* out, int n) {
