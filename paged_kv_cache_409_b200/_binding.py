@@ -96,9 +96,8 @@ def load_library():
     for name in ("pkv_reshape_and_cache", "pkv_reshape_and_cache_fp8", "pkv_paged_attention_decode_fp8",
                  "pkv_copy_blocks", "pkv_swap_blocks", "pkv_paged_attention_decode",
                  "pkv_decode_partition_size", "pkv_paged_attention_prefill_chunk", "pkv_get_device_error",
-                 "pkv_paged_attention_prefill_chunk_fp8",
-    "pkv_prefill_fp8_workspace_size",
-    "pkv_paged_attention_decode_multi", "pkv_decode_multi_partition_size"):
+                 "pkv_paged_attention_prefill_chunk_fp8", "pkv_paged_attention_decode_multi",
+                 "pkv_decode_multi_partition_size"):
         getattr(lib, name).restype = I
     _lib = lib
     return lib

@@ -145,3 +145,56 @@ def test_missing_library_fails_loudly(monkeypatch, tmp_path):
     monkeypatch.setattr(_binding, "LIB", str(tmp_path / "nope.so"))
     with pytest.raises(RuntimeError):
         _binding.load_library()
+
+
+def _prototypes():
+    """name -> (return type, [parameter types]) for every function both headers declare."""
+    protos = {}
+    for header in ("pagedkv.h", "pagedkv_block_manager.h"):
+        src = open(os.path.join(ROOT, "include", header)).read()
+        src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+        src = re.sub(r"//[^\n]*", "", src)
+        for ret, name, params in re.findall(r"([A-Za-z_][\w\s\*]*?)\s*\b(pkv_[a-z0-9_]+)\s*\(([^;{]*?)\)\s*;", src):
+            params = " ".join(params.split())
+            types = [] if params in ("", "void") else [re.sub(r"\s*\b\w+$", "", p.strip()) for p in params.split(",")]
+            protos[name] = (" ".join(ret.split()), types)
+    return protos
+
+
+def _kind(ctype_name):
+    """The ctypes type a C type marshals as."""
+    t = ctype_name.replace("const ", "").strip()
+    if "*" in t or t in ("pkv_stream_t",):
+        return "ptr"
+    return {"int": ctypes.c_int, "int64_t": ctypes.c_int64, "float": ctypes.c_float, "size_t": ctypes.c_size_t,
+            "uint32_t": ctypes.c_uint32, "void": None}[t]
+
+
+def _argkind(a):
+    if a in (ctypes.c_void_p, ctypes.c_char_p) or (isinstance(a, type) and issubclass(a, ctypes._Pointer)):
+        return "ptr"
+    return a
+
+
+def test_binding_argtypes_match_the_header_prototypes(lib):
+    """Every argtypes / restype the Python bindings set agrees with the header's prototype in count and
+    width (an int marshalled where the C side takes int64_t would pass garbage in the upper half)."""
+    from paged_kv_cache_409_b200 import block_manager
+    bm_lib = block_manager._lib()
+    protos = _prototypes()
+    assert "pkv_bm_swap_in" in protos and "pkv_paged_attention_decode_multi" in protos
+    checked = 0
+    for name, (ret, params) in protos.items():
+        fn = getattr(bm_lib if name.startswith("pkv_bm_") else lib, name)
+        if fn.argtypes is None:
+            continue
+        got = [_argkind(a) for a in fn.argtypes]
+        want = [_kind(p) for p in params]
+        assert got == want, f"{name}: binding {got} vs header {want}"
+        rk = _kind(ret)
+        if rk == "ptr":
+            assert fn.restype in (ctypes.c_void_p, ctypes.c_char_p), name
+        elif rk is not None:
+            assert fn.restype == rk, f"{name}: restype {fn.restype} vs header {ret}"
+        checked += 1
+    assert checked >= 25
