@@ -198,3 +198,22 @@ def test_binding_argtypes_match_the_header_prototypes(lib):
             assert fn.restype == rk, f"{name}: restype {fn.restype} vs header {ret}"
         checked += 1
     assert checked >= 25
+
+
+def test_python_constants_match_the_headers():
+    """dtype codes, status codes and device-error bits as the headers define them."""
+    from paged_kv_cache_409_b200 import block_manager
+    src = open(os.path.join(ROOT, "include", "pagedkv.h")).read() + \
+        open(os.path.join(ROOT, "include", "pagedkv_block_manager.h")).read()
+    enum = {k: int(v) for k, v in re.findall(r"\b(PKV_[A-Z0-9_]+)\s*=\s*(-?\d+)", src)}
+    bits = {k: int(v, 16) for k, v in re.findall(r"#define\s+(PKV_DEVERR_[A-Z_]+)\s+0x([0-9a-fA-F]+)u", src)}
+    assert _binding.DTYPE_CODE[torch.float32] == enum["PKV_F32"]
+    assert _binding.DTYPE_CODE[torch.float16] == enum["PKV_F16"]
+    assert _binding.DTYPE_CODE[torch.bfloat16] == enum["PKV_BF16"]
+    assert _binding.FP8_E4M3 == enum["PKV_FP8_E4M3"]
+    for name in ("BLOCK_ID", "SLOT", "LENGTH", "PAIR", "TIMEOUT"):
+        assert getattr(_binding, "DEVERR_" + name) == bits["PKV_DEVERR_" + name]
+    assert (block_manager.OK, block_manager.EINVAL, block_manager.ENOSPACE, block_manager.EBUFFER) == (
+        enum["PKV_BM_OK"], enum["PKV_BM_EINVAL"], enum["PKV_BM_ENOSPACE"], enum["PKV_BM_EBUFFER"])
+    for code in ("PKV_EINVAL", "PKV_EUNSUPPORTED", "PKV_ERANGE", "PKV_ECUDA", "PKV_EWORKSPACE"):
+        assert pkv.load_library().pkv_status_string(enum[code]) != b"ok"
