@@ -531,6 +531,49 @@ def weak_scaling_value(ws, units_per_rank, max_ms_per_step):
 
 # ----------------------------------------------------------------------------- CPU baseline (oracle)
 
+def disjoint_block_pairs(num_blocks, block_bytes, target_bytes=512 << 20, seed=7):
+    """(src, dst) pairs over distinct blocks, no dst among the srcs: about target_bytes of each pool's
+    blocks are copied per launch (capped at half the pool)."""
+    n = int(min(num_blocks // 2, max(1, target_bytes // block_bytes)))
+    perm = np.random.default_rng(seed).permutation(num_blocks)
+    return np.stack([perm[:n], perm[n:2 * n]], 1).astype(np.int64)
+
+
+def index_kernel_figures(step, hbm_gbs, launches=20):
+    """copy_blocks and reshape_and_cache timed alone with CUDA events, after every other measurement
+    (copy_blocks overwrites pool blocks).  copy_blocks moves ~0.5 GB of each of the K and V pools per
+    launch (inputs larger than L2); the append writes one step's new tokens (L2-sized, launch-bound)."""
+    pkv, w = step.pkv, step.w
+    kc, vc = w.key_caches[0], w.value_caches[0]
+    block_bytes = kc[0].numel() * kc.element_size()
+    pairs = torch.from_numpy(disjoint_block_pairs(kc.shape[0], block_bytes)).to(kc.device)
+    ev = lambda: torch.cuda.Event(enable_timing=True)
+
+    def timed(fn):
+        for _ in range(3):
+            fn()
+        torch.cuda.synchronize()
+        a, b = ev(), ev()
+        a.record()
+        for _ in range(launches):
+            fn()
+        b.record()
+        torch.cuda.synchronize()
+        return a.elapsed_time(b) / launches
+
+    ms = timed(lambda: pkv.copy_blocks([kc], [vc], pairs))
+    moved = 2 * 2 * pairs.shape[0] * block_bytes  # K and V, read and written
+    app_ms = timed(lambda: step.append(0))
+    nk = w.new_keys[0]
+    app_bytes = 2 * nk.numel() * (nk.element_size() + kc.element_size())  # K and V rows read, pool rows written
+    return {"copy_blocks": {"pairs": int(pairs.shape[0]), "bytes_per_launch": moved, "ms": ms,
+                            "achieved_gbs": moved / ms / 1e6, "frac": moved / ms / 1e6 / hbm_gbs},
+            "append": {"kernel": "reshape_and_cache_fp8" if w.fp8 else "reshape_and_cache",
+                       "tokens": int(nk.shape[0]), "bytes_per_launch": app_bytes, "us": app_ms * 1e3,
+                       "achieved_gbs": app_bytes / app_ms / 1e6,
+                       "note": "one step's append: launch-bound, its bytes fit in L2"}}
+
+
 def oracle_sample(step, budget_s, max_seqs=None):
     """Time the oracle (append + decode) on whole steps or a sequence sample, host cores."""
     import oracle
@@ -825,6 +868,11 @@ def main():
         line["cpu_baseline"] = {"value": v / 80.0, "unit": "tokens/s (80-layer steps)", "cores": 1,
                                 "kind": "oracle",
                                 "sample": f"{done} x one layer of {n} sequences, {el:.1f} s, 1 thread; /80 layers"}
+    if ws == 1 and type(step) is DecodeStep:
+        try:
+            line["index_kernels"] = index_kernel_figures(step, hbm)
+        except Exception as exc:  # an extra figure never costs the main line
+            line["index_kernels"] = {"error": f"{type(exc).__name__}: {exc}"}
     if rank == 0:
         print(json.dumps(line), flush=True)
     if ws > 1:

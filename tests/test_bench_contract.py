@@ -32,3 +32,19 @@ def test_reference_arm_multi_token_line():
     d = run_bench("--impl", "reference", "--config", "multi_token_decode_bf16", "--steps", "1", "--warmup", "3")
     assert d["impl"] == "reference" and d["unit"] == "tokens/s" and d["value"] > 0
     assert "draft tokens" in d["cpu_baseline"]["sample"]
+
+
+def test_copy_blocks_measurement_pairs_are_disjoint():
+    """The standalone copy_blocks figure copies distinct blocks onto distinct, unsourced blocks (the kernel's
+    precondition), about 0.5 GB of each pool per launch, at most half the pool."""
+    import importlib.util
+    import numpy as np
+    spec = importlib.util.spec_from_file_location("bench_module", os.path.join(ROOT, "bench.py"))
+    bench = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(bench)
+    for nb, bb in ((4188, 16 * 32 * 128 * 2), (100, 1 << 20), (3, 10), (1 << 16, 4096)):
+        p = bench.disjoint_block_pairs(nb, bb)
+        src, dst = set(p[:, 0].tolist()), set(p[:, 1].tolist())
+        assert len(src) == len(dst) == len(p) and not (src & dst)
+        assert p.min() >= 0 and p.max() < nb and p.dtype == np.int64
+        assert len(p) == min(nb // 2, max(1, (512 << 20) // bb))
