@@ -154,7 +154,7 @@ def _prototypes():
         src = open(os.path.join(ROOT, "include", header)).read()
         src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
         src = re.sub(r"//[^\n]*", "", src)
-        for ret, name, params in re.findall(r"([A-Za-z_][\w\s\*]*?)\s*\b(pkv_[a-z0-9_]+)\s*\(([^;{]*?)\)\s*;", src):
+        for ret, name, params in re.findall(r"^([A-Za-z_][\w \t\*]*?)\s*\b(pkv_[a-z0-9_]+)\s*\(([^;{]*?)\)\s*;", src, flags=re.M):
             params = " ".join(params.split())
             types = [] if params in ("", "void") else [re.sub(r"\s*\b\w+$", "", p.strip()) for p in params.split(",")]
             protos[name] = (" ".join(ret.split()), types)
