@@ -36,16 +36,24 @@
  *   - Swapping (case-study page, section 三: under memory pressure a request is
  *     pre-empted by moving its KV to CPU memory, and resumed later; tutorial
  *     page 4.3).  An optional host pool of num_host_blocks blocks has its own
- *     free stack (block 0 on top).  Swapping a sequence out takes one host
- *     block per device block, in logical order from the top of that stack,
- *     reports the (device, host) pairs, and then releases the device blocks
- *     like a free (last to first; cached ones stay cached).  Swapping it in
- *     takes one device block per host block, in logical order (free stack,
- *     else LRU eviction), reports the (host, device) pairs, and pushes the
- *     host blocks back last to first.  Swapped-in blocks are private: they are
- *     not re-entered in the prefix cache (the hash chain of later blocks
- *     continues).  A swapped-out sequence can only be swapped in, freed or
- *     asked for its token count.
+ *     free stack (block 0 on top) and a reference count per host block.
+ *     Swapping out a group of sequences (one, or e.g. the samples of one
+ *     request, which share blocks) takes one host block per DISTINCT device
+ *     block of the group's tables, in order of first appearance (sequences in
+ *     the given order, positions in logical order), from the top of that
+ *     stack; reports those (device, host) pairs; points every table entry at
+ *     its block's host copy; then releases each sequence's device blocks like
+ *     a free (sequences in order, each last to first; cached ones stay
+ *     cached).  Swapping a group in takes one device block per distinct host
+ *     block, in order of first appearance (free stack, else LRU eviction),
+ *     reports the (host, device) pairs, points the tables at them (a block
+ *     shared by k tables gets reference count k), and drops the sequences'
+ *     host references (sequences in order, each last to first); a host block
+ *     left with none goes back on top of the host stack.  Swapped-in blocks
+ *     are private to the group: they are not re-entered in the prefix cache
+ *     (the hash chain of later blocks continues).  A swapped-out sequence can
+ *     only be swapped in, freed (dropping its host references) or asked for
+ *     its token count.
  *
  * The manager is not thread-safe; one owner calls it.
  */
@@ -144,6 +152,16 @@ int pkv_bm_swap_out(pkv_block_manager* bm, int64_t seq_id, int64_t* pairs_out, i
  * changes. */
 int pkv_bm_swap_in(pkv_block_manager* bm, int64_t seq_id, int64_t* pairs_out, int64_t max_pairs,
                    int64_t* num_pairs);
+
+/* The same for n >= 1 distinct sequences at once: blocks they share cross to
+ * the host once and are shared again after swap-in (pairs: one per distinct
+ * block, see the policy above).  pkv_bm_swap_out / pkv_bm_swap_in are the
+ * one-sequence case.  PKV_BM_EINVAL if an id is unknown, repeated, or not
+ * resident (out) / not swapped out (in). */
+int pkv_bm_swap_out_group(pkv_block_manager* bm, const int64_t* seq_ids, int64_t n, int64_t* pairs_out,
+                          int64_t max_pairs, int64_t* num_pairs);
+int pkv_bm_swap_in_group(pkv_block_manager* bm, const int64_t* seq_ids, int64_t n, int64_t* pairs_out,
+                         int64_t max_pairs, int64_t* num_pairs);
 
 /* Reference count of a physical block (or a negative status). */
 int pkv_bm_ref_count(const pkv_block_manager* bm, int64_t block);

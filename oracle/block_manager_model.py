@@ -30,6 +30,7 @@ class BlockManagerModel:
         self.seqs = {}
         self.hits = self.evictions = self.cows = 0
         self.host_free = list(range(num_host_blocks - 1, -1, -1))  # host block 0 on top
+        self.host_ref = [0] * num_host_blocks
 
     # -- blocks
     def _take(self):
@@ -127,35 +128,70 @@ class BlockManagerModel:
         for b in p["blocks"]:
             self.ref[b] += 1
 
+    def _drop_host(self, seq):
+        for h in reversed(seq.pop("host")):
+            self.host_ref[h] -= 1
+            if self.host_ref[h] == 0:
+                self.host_free.append(h)
+
     def free(self, sid):
         seq = self.seqs.pop(sid)
-        self.host_free += list(reversed(seq.get("host", [])))
+        if "host" in seq:
+            self._drop_host(seq)
         for b in reversed(seq["blocks"]):
             self._release(b)
 
-    # -- swapping (a pre-empted sequence's blocks move to the host pool and back)
-    def swap_out(self, sid):
-        seq = self.seqs[sid]
-        assert "host" not in seq
-        if len(seq["blocks"]) > len(self.host_free):
-            raise NoSpace()
-        host = [self.host_free.pop() for _ in seq["blocks"]]
-        pairs = list(zip(seq["blocks"], host))
-        for b in reversed(seq["blocks"]):
-            self._release(b)
-        seq["blocks"], seq["host"] = [], host
-        return pairs
+    # -- swapping (pre-empted sequences' blocks move to the host pool and back; a group's shared blocks once)
+    @staticmethod
+    def _group(sids):
+        sids = [sids] if isinstance(sids, int) else [int(s) for s in sids]
+        assert sids and len(set(sids)) == len(sids)
+        return sids
 
-    def swap_in(self, sid):
-        seq = self.seqs[sid]
-        host = seq["host"]
-        if len(host) > self._available():
+    @staticmethod
+    def _distinct(lists):
+        out = []
+        for lst in lists:
+            for x in lst:
+                if x not in out:
+                    out.append(x)
+        return out
+
+    def swap_out(self, sids):
+        seqs = [self.seqs[s] for s in self._group(sids)]
+        assert all("host" not in q for q in seqs)
+        distinct = self._distinct(q["blocks"] for q in seqs)
+        if len(distinct) > len(self.host_free):
             raise NoSpace()
-        seq["blocks"] = [self._take() for _ in host]
-        pairs = list(zip(host, seq["blocks"]))
-        self.host_free += list(reversed(host))
-        del seq["host"]
-        return pairs
+        to_host = {}
+        for b in distinct:
+            to_host[b] = self.host_free.pop()
+        for q in seqs:
+            q["host"] = [to_host[b] for b in q["blocks"]]
+            for h in q["host"]:
+                self.host_ref[h] += 1
+            for b in reversed(q["blocks"]):
+                self._release(b)
+            q["blocks"] = []
+        return [(b, to_host[b]) for b in distinct]
+
+    def swap_in(self, sids):
+        seqs = [self.seqs[s] for s in self._group(sids)]
+        assert all("host" in q for q in seqs)
+        distinct = self._distinct(q["host"] for q in seqs)
+        if len(distinct) > self._available():
+            raise NoSpace()
+        to_dev = {}
+        for h in distinct:
+            d = self._take()
+            self.ref[d] = 0          # counted below, one per table entry
+            to_dev[h] = d
+        for q in seqs:
+            q["blocks"] = [to_dev[h] for h in q["host"]]
+            for d in q["blocks"]:
+                self.ref[d] += 1
+            self._drop_host(q)
+        return [(h, to_dev[h]) for h in distinct]
 
     def swapped(self, sid):
         return "host" in self.seqs[sid]

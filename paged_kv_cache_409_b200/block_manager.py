@@ -53,9 +53,12 @@ def _lib():
         lib.pkv_bm_set_host_blocks.argtypes = [P, I64]
         lib.pkv_bm_swap_out.argtypes = [P, I64, P, I64, P]
         lib.pkv_bm_swap_in.argtypes = [P, I64, P, I64, P]
+        lib.pkv_bm_swap_out_group.argtypes = [P, P, I64, P, I64, P]
+        lib.pkv_bm_swap_in_group.argtypes = [P, P, I64, P, I64, P]
         for f in (lib.pkv_bm_add_sequence, lib.pkv_bm_append, lib.pkv_bm_append_batch, lib.pkv_bm_fork,
                   lib.pkv_bm_free, lib.pkv_bm_slots, lib.pkv_bm_block_table, lib.pkv_bm_stats, lib.pkv_bm_ref_count,
-                  lib.pkv_bm_set_host_blocks, lib.pkv_bm_swap_out, lib.pkv_bm_swap_in):
+                  lib.pkv_bm_set_host_blocks, lib.pkv_bm_swap_out, lib.pkv_bm_swap_in, lib.pkv_bm_swap_out_group,
+                  lib.pkv_bm_swap_in_group):
             f.restype = I
         _bound = True
     return lib
@@ -136,22 +139,26 @@ class BlockManager:
     def free(self, seq_id: int):
         _check(self._l.pkv_bm_free(self._h, int(seq_id)), "free")
 
-    def _swap(self, fn, seq_id, what):
+    def _swap(self, fn, seq_ids, what):
+        ids = np.atleast_1d(np.asarray(seq_ids, dtype=np.int64))
         # a sequence of n tokens holds ceil(n / block_size) blocks, resident or not
-        tokens = _check(int(self._l.pkv_bm_num_tokens(self._h, int(seq_id))), what)
-        cap = max(-(-tokens // self.block_size), 1)
+        cap = 1
+        for s in ids.tolist():
+            cap += -(-_check(int(self._l.pkv_bm_num_tokens(self._h, int(s))), what) // self.block_size)
         pairs = np.empty((cap, 2), dtype=np.int64)
         k = ctypes.c_int64(0)
-        _check(fn(self._h, int(seq_id), _ptr(pairs), cap, ctypes.byref(k)), what)
+        _check(fn(self._h, _ptr(ids), ids.size, _ptr(pairs), cap, ctypes.byref(k)), what)
         return pairs[:k.value]
 
-    def swap_out(self, seq_id: int) -> np.ndarray:
-        """Pre-empt a sequence; returns its (device block, host block) pairs int64 [n, 2]."""
-        return self._swap(self._l.pkv_bm_swap_out, seq_id, "swap_out")
+    def swap_out(self, seq_ids) -> np.ndarray:
+        """Pre-empt one sequence, or several together (blocks they share cross once); returns the
+        (device block, host block) pairs int64 [k, 2], one per distinct block."""
+        return self._swap(self._l.pkv_bm_swap_out_group, seq_ids, "swap_out")
 
-    def swap_in(self, seq_id: int) -> np.ndarray:
-        """Resume a swapped-out sequence; returns its (host block, device block) pairs int64 [n, 2]."""
-        return self._swap(self._l.pkv_bm_swap_in, seq_id, "swap_in")
+    def swap_in(self, seq_ids) -> np.ndarray:
+        """Resume swapped-out sequences (shared blocks shared again); returns the (host block, device block)
+        pairs int64 [k, 2], one per distinct block."""
+        return self._swap(self._l.pkv_bm_swap_in_group, seq_ids, "swap_in")
 
     def slots(self, seq_id: int, start: int, count: int) -> np.ndarray:
         out = np.empty(max(count, 1), dtype=np.int64)

@@ -60,6 +60,7 @@ struct pkv_block_manager {
     std::vector<char> in_lru;
     std::unordered_map<int64_t, Sequence> seqs;
     std::vector<int32_t> host_free;    // host pool's free stack, top = back
+    std::vector<int32_t> host_ref;     // swapped-out table entries per host block
     int64_t num_host_blocks = 0;
     int64_t swapped = 0;               // sequences swapped out
     int64_t hits = 0, evictions = 0, cows = 0;
@@ -115,9 +116,12 @@ struct pkv_block_manager {
 
     int64_t available() const { return static_cast<int64_t>(free_stack.size() + lru.size()); }
 
-    // Return a swapped-out sequence's host blocks, last to first (the first on top).
+    // Drop a swapped-out sequence's references to its host blocks, last to
+    // first; a host block no sequence references any more goes back on top of
+    // the host free stack.
     void release_host(Sequence& s) {
-        for (auto h = s.host_blocks.rbegin(); h != s.host_blocks.rend(); ++h) host_free.push_back(*h);
+        for (auto h = s.host_blocks.rbegin(); h != s.host_blocks.rend(); ++h)
+            if (--host_ref[*h] == 0) host_free.push_back(*h);
         s.host_blocks.clear();
     }
 
@@ -286,56 +290,104 @@ int pkv_bm_free(pkv_block_manager* bm, int64_t seq_id) {
 int pkv_bm_set_host_blocks(pkv_block_manager* bm, int64_t num_host_blocks) {
     if (!bm || num_host_blocks < 0 || num_host_blocks > INT32_MAX || bm->swapped) return PKV_BM_EINVAL;
     bm->num_host_blocks = num_host_blocks;
+    bm->host_ref.assign(num_host_blocks, 0);
     bm->host_free.resize(num_host_blocks);
     for (int64_t i = 0; i < num_host_blocks; ++i)
         bm->host_free[i] = static_cast<int32_t>(num_host_blocks - 1 - i);
     return PKV_BM_OK;
 }
 
-int pkv_bm_swap_out(pkv_block_manager* bm, int64_t seq_id, int64_t* pairs_out, int64_t max_pairs,
-                    int64_t* num_pairs) {
-    if (!bm || max_pairs < 0) return PKV_BM_EINVAL;
-    Sequence* sp = bm->resident(seq_id);
-    if (!sp) return PKV_BM_EINVAL;
-    Sequence& s = *sp;
-    const int64_t n = static_cast<int64_t>(s.blocks.size());
-    if (n > static_cast<int64_t>(bm->host_free.size())) return PKV_BM_ENOSPACE;
-    if (n > max_pairs || (n > 0 && !pairs_out)) return PKV_BM_EBUFFER;
-    for (int64_t i = 0; i < n; ++i) {
+int pkv_bm_swap_out_group(pkv_block_manager* bm, const int64_t* seq_ids, int64_t n, int64_t* pairs_out,
+                          int64_t max_pairs, int64_t* num_pairs) {
+    if (!bm || n <= 0 || !seq_ids || max_pairs < 0) return PKV_BM_EINVAL;
+    std::vector<Sequence*> group;
+    for (int64_t g = 0; g < n; ++g) {
+        Sequence* sp = bm->resident(seq_ids[g]);
+        for (int64_t e = 0; e < g; ++e)
+            if (seq_ids[e] == seq_ids[g]) sp = nullptr;
+        if (!sp) return PKV_BM_EINVAL;
+        group.push_back(sp);
+    }
+    // distinct device blocks of the group, in order of first appearance
+    std::unordered_map<int32_t, int32_t> to_host;
+    std::vector<int32_t> distinct;
+    for (Sequence* sp : group)
+        for (int32_t b : sp->blocks)
+            if (to_host.emplace(b, -1).second) distinct.push_back(b);
+    const int64_t k = static_cast<int64_t>(distinct.size());
+    if (k > static_cast<int64_t>(bm->host_free.size())) return PKV_BM_ENOSPACE;
+    if (k > max_pairs || (k > 0 && !pairs_out)) return PKV_BM_EBUFFER;
+    for (int64_t i = 0; i < k; ++i) {
         const int32_t h = bm->host_free.back();
         bm->host_free.pop_back();
-        s.host_blocks.push_back(h);
-        pairs_out[2 * i] = s.blocks[i];
+        to_host[distinct[i]] = h;
+        pairs_out[2 * i] = distinct[i];
         pairs_out[2 * i + 1] = h;
     }
-    for (auto b = s.blocks.rbegin(); b != s.blocks.rend(); ++b) bm->release_block(*b);
-    s.blocks.clear();
-    s.swapped = true;
-    ++bm->swapped;
-    if (num_pairs) *num_pairs = n;
+    for (Sequence* sp : group) {
+        for (int32_t b : sp->blocks) {
+            const int32_t h = to_host[b];
+            sp->host_blocks.push_back(h);
+            ++bm->host_ref[h];
+        }
+        for (auto b = sp->blocks.rbegin(); b != sp->blocks.rend(); ++b) bm->release_block(*b);
+        sp->blocks.clear();
+        sp->swapped = true;
+        ++bm->swapped;
+    }
+    if (num_pairs) *num_pairs = k;
     return PKV_BM_OK;
+}
+
+int pkv_bm_swap_in_group(pkv_block_manager* bm, const int64_t* seq_ids, int64_t n, int64_t* pairs_out,
+                         int64_t max_pairs, int64_t* num_pairs) {
+    if (!bm || n <= 0 || !seq_ids || max_pairs < 0) return PKV_BM_EINVAL;
+    std::vector<Sequence*> group;
+    for (int64_t g = 0; g < n; ++g) {
+        auto it = bm->seqs.find(seq_ids[g]);
+        Sequence* sp = (it == bm->seqs.end() || !it->second.swapped) ? nullptr : &it->second;
+        for (int64_t e = 0; e < g; ++e)
+            if (seq_ids[e] == seq_ids[g]) sp = nullptr;
+        if (!sp) return PKV_BM_EINVAL;
+        group.push_back(sp);
+    }
+    std::unordered_map<int32_t, int32_t> to_dev;
+    std::vector<int32_t> distinct;
+    for (Sequence* sp : group)
+        for (int32_t h : sp->host_blocks)
+            if (to_dev.emplace(h, -1).second) distinct.push_back(h);
+    const int64_t k = static_cast<int64_t>(distinct.size());
+    if (k > bm->available()) return PKV_BM_ENOSPACE;
+    if (k > max_pairs || (k > 0 && !pairs_out)) return PKV_BM_EBUFFER;
+    for (int64_t i = 0; i < k; ++i) {
+        const int32_t d = bm->take_block();
+        bm->ref[d] = 0;  // counted below, one per table entry
+        to_dev[distinct[i]] = d;
+        pairs_out[2 * i] = distinct[i];
+        pairs_out[2 * i + 1] = d;
+    }
+    for (Sequence* sp : group) {
+        for (int32_t h : sp->host_blocks) {
+            const int32_t d = to_dev[h];
+            sp->blocks.push_back(d);
+            ++bm->ref[d];
+        }
+        bm->release_host(*sp);
+        sp->swapped = false;
+        --bm->swapped;
+    }
+    if (num_pairs) *num_pairs = k;
+    return PKV_BM_OK;
+}
+
+int pkv_bm_swap_out(pkv_block_manager* bm, int64_t seq_id, int64_t* pairs_out, int64_t max_pairs,
+                    int64_t* num_pairs) {
+    return pkv_bm_swap_out_group(bm, &seq_id, 1, pairs_out, max_pairs, num_pairs);
 }
 
 int pkv_bm_swap_in(pkv_block_manager* bm, int64_t seq_id, int64_t* pairs_out, int64_t max_pairs,
                    int64_t* num_pairs) {
-    if (!bm || max_pairs < 0) return PKV_BM_EINVAL;
-    auto it = bm->seqs.find(seq_id);
-    if (it == bm->seqs.end() || !it->second.swapped) return PKV_BM_EINVAL;
-    Sequence& s = it->second;
-    const int64_t n = static_cast<int64_t>(s.host_blocks.size());
-    if (n > bm->available()) return PKV_BM_ENOSPACE;
-    if (n > max_pairs || (n > 0 && !pairs_out)) return PKV_BM_EBUFFER;
-    for (int64_t i = 0; i < n; ++i) {
-        const int32_t d = bm->take_block();
-        s.blocks.push_back(d);
-        pairs_out[2 * i] = s.host_blocks[i];
-        pairs_out[2 * i + 1] = d;
-    }
-    bm->release_host(s);
-    s.swapped = false;
-    --bm->swapped;
-    if (num_pairs) *num_pairs = n;
-    return PKV_BM_OK;
+    return pkv_bm_swap_in_group(bm, &seq_id, 1, pairs_out, max_pairs, num_pairs);
 }
 
 int pkv_bm_slots(const pkv_block_manager* bm, int64_t seq_id, int64_t start, int64_t count, int64_t* slots_out) {

@@ -5,7 +5,8 @@
 // checks the pool's conservation laws after each operation:
 //   sum of reference counts == total length of the resident block tables,
 //   free + evictable + referenced blocks == num_blocks,
-//   free host blocks + host blocks held by swapped-out sequences == host pool.
+//   free host blocks + distinct host blocks of swapped-out tables == host pool
+// and that group swaps move each distinct block once and rebuild every table.
 #include <cstdio>
 #include <cstdlib>
 #include <map>
@@ -33,7 +34,7 @@ int main(int argc, char** argv) {
     CHECK(bm && pkv_bm_create(0, B, 1) == nullptr && pkv_bm_create(NB, 0, 1) == nullptr);
     CHECK(pkv_bm_set_host_blocks(bm, NH) == PKV_BM_OK && pkv_bm_set_host_blocks(bm, -1) == PKV_BM_EINVAL);
     std::map<int64_t, bool> seqs;  // id -> swapped out
-    std::map<int64_t, int64_t> host_held;
+    std::map<int64_t, std::vector<int64_t>> host_table;  // swapped-out sequence -> its host blocks
     int64_t next = 0, swapped_out = 0, swapped_in = 0, cow_pairs = 0;
     std::vector<int64_t> slots(512), pairs(2 * 512);
     std::vector<int32_t> table(512);
@@ -76,45 +77,73 @@ int main(int argc, char** argv) {
             CHECK(seqs[any] ? rc == PKV_BM_EINVAL : rc == PKV_BM_OK);
             if (rc == PKV_BM_OK) seqs[next] = false;
             ++next;
-        } else if (op == 6) {
-            rc = pkv_bm_swap_out(bm, any, pairs.data(), U(2) ? 512 : 1, &n);
-            CHECK(seqs[any] ? rc == PKV_BM_EINVAL : (rc == PKV_BM_OK || rc == PKV_BM_ENOSPACE || rc == PKV_BM_EBUFFER));
-            if (rc == PKV_BM_OK) {
-                ++swapped_out;
-                seqs[any] = true;
-                host_held[any] = n;
-                std::set<int64_t> hs;
-                for (int64_t i = 0; i < n; ++i) {
-                    CHECK(pairs[2 * i] >= 0 && pairs[2 * i] < NB && pairs[2 * i + 1] >= 0 && pairs[2 * i + 1] < NH);
-                    hs.insert(pairs[2 * i + 1]);
-                }
-                CHECK(static_cast<int64_t>(hs.size()) == n);
-            }
-        } else if (op == 7) {
-            std::vector<int64_t> out_ids;
+        } else if (op == 6 || op == 7) {
+            // a group of 1-3 sequences; mostly of the right state, sometimes any (invalid) id
+            const bool out = op == 6;
+            std::vector<int64_t> pool_ids;
             for (auto& kv : seqs)
-                if (kv.second) out_ids.push_back(kv.first);
-            const int64_t target = (!out_ids.empty() && U(4)) ? out_ids[U(static_cast<int>(out_ids.size()))] : any;
-            rc = pkv_bm_swap_in(bm, target, pairs.data(), U(4) ? 512 : 0, &n);
-            CHECK(!seqs[target] ? rc == PKV_BM_EINVAL
-                                : (rc == PKV_BM_OK || rc == PKV_BM_ENOSPACE || rc == PKV_BM_EBUFFER));
-            if (rc == PKV_BM_OK) {
-                ++swapped_in;
-                CHECK(n == host_held[target]);
-                std::set<int64_t> ds;
-                for (int64_t i = 0; i < n; ++i) {
-                    CHECK(pairs[2 * i + 1] >= 0 && pairs[2 * i + 1] < NB && pkv_bm_ref_count(bm, pairs[2 * i + 1]) == 1);
-                    ds.insert(pairs[2 * i + 1]);
+                if (kv.second != out) pool_ids.push_back(kv.first);
+            std::vector<int64_t> group;
+            const int want = 1 + U(3);
+            for (int g = 0; g < want && !pool_ids.empty(); ++g) {
+                const int j = U(static_cast<int>(pool_ids.size()));
+                group.push_back(pool_ids[j]);
+                pool_ids.erase(pool_ids.begin() + j);
+            }
+            if (group.empty() || U(8) == 0) group.push_back(any);  // possibly wrong state or a repeat
+            bool valid = true;
+            std::set<int64_t> uniq(group.begin(), group.end());
+            if (uniq.size() != group.size()) valid = false;
+            for (int64_t g : group)
+                if (!seqs.count(g) || seqs[g] != !out) valid = false;
+            std::map<int64_t, std::vector<int32_t>> before;
+            if (valid && out)
+                for (int64_t g : group) {
+                    int64_t nb = 0;
+                    CHECK(pkv_bm_block_table(bm, g, table.data(), 512, &nb) == PKV_BM_OK);
+                    before[g].assign(table.begin(), table.begin() + nb);
                 }
-                CHECK(static_cast<int64_t>(ds.size()) == n);
-                seqs[target] = false;
-                host_held.erase(target);
+            const int64_t cap = U(5) ? 512 : 1;
+            rc = out ? pkv_bm_swap_out_group(bm, group.data(), static_cast<int64_t>(group.size()), pairs.data(), cap, &n)
+                     : pkv_bm_swap_in_group(bm, group.data(), static_cast<int64_t>(group.size()), pairs.data(), cap, &n);
+            if (!valid) {
+                CHECK(rc == PKV_BM_EINVAL);
+            } else {
+                CHECK(rc == PKV_BM_OK || rc == PKV_BM_ENOSPACE || rc == PKV_BM_EBUFFER);
+            }
+            if (rc == PKV_BM_OK) {
+                std::map<int64_t, int64_t> m;  // pair source -> destination, each source once
+                std::set<int64_t> dsts;
+                for (int64_t i = 0; i < n; ++i) {
+                    CHECK(m.emplace(pairs[2 * i], pairs[2 * i + 1]).second && dsts.insert(pairs[2 * i + 1]).second);
+                    CHECK(pairs[2 * i + 1] >= 0 && pairs[2 * i + 1] < (out ? NH : NB));
+                }
+                for (int64_t g : group) {
+                    if (out) {
+                        std::vector<int64_t> ht;
+                        for (int32_t b : before[g]) {
+                            CHECK(m.count(b));
+                            ht.push_back(m[b]);
+                        }
+                        host_table[g] = ht;
+                        seqs[g] = true;
+                        ++swapped_out;
+                    } else {
+                        int64_t nb = 0;
+                        CHECK(pkv_bm_block_table(bm, g, table.data(), 512, &nb) == PKV_BM_OK);
+                        CHECK(nb == static_cast<int64_t>(host_table[g].size()));
+                        for (int64_t i = 0; i < nb; ++i) CHECK(m.count(host_table[g][i]) && table[i] == m[host_table[g][i]]);
+                        host_table.erase(g);
+                        seqs[g] = false;
+                        ++swapped_in;
+                    }
+                }
             }
         } else if (op == 8) {
             rc = pkv_bm_free(bm, any);
             CHECK(rc == PKV_BM_OK || ids.empty());
             seqs.erase(any);
-            host_held.erase(any);
+            host_table.erase(any);
         } else {
             // invalid and edge arguments: nothing may change
             CHECK(pkv_bm_append(nullptr, any, nullptr, 0, nullptr, nullptr, 0, nullptr) == PKV_BM_EINVAL);
@@ -136,11 +165,12 @@ int main(int argc, char** argv) {
             refs += r;
             referenced += r > 0;
         }
-        int64_t table_len = 0, held = 0;
+        int64_t table_len = 0;
+        std::set<int64_t> held_host;
         for (auto& kv : seqs) {
             CHECK(pkv_bm_num_tokens(bm, kv.first) >= 0);
             if (kv.second) {
-                held += host_held[kv.first];
+                held_host.insert(host_table[kv.first].begin(), host_table[kv.first].end());
                 continue;
             }
             int64_t nb = 0;
@@ -151,7 +181,7 @@ int main(int argc, char** argv) {
         }
         CHECK(refs == table_len);
         CHECK(st[0] + st[1] + referenced == NB);
-        CHECK(st[7] + held == NH);
+        CHECK(st[7] + static_cast<int64_t>(held_host.size()) == NH);
         CHECK(st[6] == static_cast<int64_t>(seqs.size()));
         int64_t out = 0;
         for (auto& kv : seqs) out += kv.second;

@@ -290,9 +290,11 @@ def test_swap_matches_plain_model_on_random_operations(seed, caching):
             op = ("fork", resident[int(rng.integers(0, len(resident)))], next_id)
             next_id += 1
         elif r < 0.72 and resident:
-            op = ("swap_out", resident[int(rng.integers(0, len(resident)))])
+            k = 1 if rng.random() < 0.5 else int(rng.integers(1, len(resident) + 1))
+            op = ("swap_out", [int(x) for x in rng.choice(resident, size=k, replace=False)])
         elif r < 0.84 and out:
-            op = ("swap_in", out[int(rng.integers(0, len(out)))])
+            k = 1 if rng.random() < 0.5 else int(rng.integers(1, len(out) + 1))
+            op = ("swap_in", [int(x) for x in rng.choice(out, size=k, replace=False)])
         else:
             ids = list(model.seqs)
             op = ("free", ids[int(rng.integers(0, len(ids)))])
@@ -370,14 +372,17 @@ def test_swapped_kv_survives_reuse_of_its_device_blocks():
                 tokens[next_id] = list(tokens[sid])
                 next_id += 1
             elif r < 0.8 and live:
-                sid = live[int(rng.integers(0, len(live)))]
-                move(dev, host, bm.swap_out(sid))
-                swapped_set.add(sid)
+                group = [int(x) for x in rng.choice(live, size=int(rng.integers(1, min(3, len(live)) + 1)),
+                                                    replace=False)]
+                move(dev, host, bm.swap_out(group))
+                swapped_set.update(group)
                 preempted += 1
             elif r < 0.92 and swapped_set:
-                sid = sorted(swapped_set)[int(rng.integers(0, len(swapped_set)))]
-                move(host, dev, bm.swap_in(sid))
-                swapped_set.discard(sid)
+                out = sorted(swapped_set)
+                group = [int(x) for x in rng.choice(out, size=int(rng.integers(1, min(3, len(out)) + 1)),
+                                                    replace=False)]
+                move(host, dev, bm.swap_in(group))
+                swapped_set.difference_update(group)
             else:
                 sid = list(tokens)[int(rng.integers(0, len(tokens)))]
                 bm.free(sid)
@@ -392,3 +397,43 @@ def test_swapped_kv_survives_reuse_of_its_device_blocks():
             want = np.array([row(p, t) for p, t in enumerate(toks)]).reshape(-1, W)
             assert np.array_equal(got, want), (step, sid)
     assert preempted >= 20
+
+
+def test_group_swap_keeps_shared_blocks_shared():
+    """Two samples of one request (a fork) share their prompt blocks: swapped out together, each shared block
+    crosses to the host once; swapped in together, both tables point at one device copy again, and the
+    shared partial last block is still copied on the first divergent append."""
+    bm = BlockManager(32, 4, prefix_caching=False, num_host_blocks=16)
+    bm.add_sequence(1, range(10))                          # blocks 0, 1 full, 2 partial
+    bm.fork(1, 2)
+    bm.append(2, [50, 51])                                 # CoW of block 2; sample 2 diverges
+    t1, t2 = bm.block_table(1).tolist(), bm.block_table(2).tolist()
+    assert t1[:2] == t2[:2] and t1[2] != t2[2]
+    out = bm.swap_out([1, 2])
+    assert out[:, 0].tolist() == [t1[0], t1[1], t1[2], t2[2]]      # distinct blocks, first appearance
+    assert bm.stats()["free_host"] == 12 and bm.stats()["swapped"] == 2
+    back = bm.swap_in([2, 1])
+    assert len(back) == 4 and set(back[:, 0].tolist()) == set(out[:, 1].tolist())
+    n1, n2 = bm.block_table(1).tolist(), bm.block_table(2).tolist()
+    assert n1[:2] == n2[:2] and n1[2] != n2[2]
+    assert bm.ref_count(n1[0]) == 2 and bm.ref_count(n1[2]) == 1 and bm.ref_count(n2[2]) == 1
+    assert bm.stats()["free_host"] == 16
+    bm.fork(1, 3)                                          # a new sample shares the restored partial block
+    slots, pairs = bm.append(3, [9])
+    assert len(pairs) == 1 and pairs[0, 0] == n1[2]
+
+
+def test_group_swap_in_part_of_a_group():
+    """Swapping in one sample of a swapped-out pair copies the shared blocks for it; the host copies stay
+    for the other sample until it is swapped in or freed."""
+    bm = BlockManager(32, 4, prefix_caching=False, num_host_blocks=8)
+    bm.add_sequence(1, range(8))                           # two full blocks
+    bm.fork(1, 2)
+    out = bm.swap_out([1, 2])
+    assert len(out) == 2 and bm.stats()["free_host"] == 6
+    a = bm.swap_in(1)
+    assert a[:, 0].tolist() == out[:, 1].tolist() and bm.stats()["free_host"] == 6
+    bm.free(2)                                             # drops the last host references
+    assert bm.stats()["free_host"] == 8
+    with pytest.raises(BlockManagerError):
+        bm.swap_out([1, 1])                                # repeated id
