@@ -14,7 +14,6 @@ CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libpagedkv.so")
 SOURCES = ["pagedkv.cu", "block_manager.cpp"]
-DEPENDS = ["pagedkv.cu", "block_manager.cpp", "ptx.cuh", "index_kernels.cuh", "decode.cuh", "decode_mma.cuh", "prefill.cuh"]
 
 
 def nvcc() -> str:
@@ -30,12 +29,19 @@ def command(out: str, extra=()) -> list:
             "-I", INCLUDE, "-I", CSRC, "-o", out, *extra, *[os.path.join(CSRC, s) for s in SOURCES]]
 
 
+def depends() -> list:
+    """Every file the library is built from: all sources and headers under csrc/ and include/."""
+    out = []
+    for d in (CSRC, INCLUDE):
+        out += [os.path.join(d, f) for f in sorted(os.listdir(d)) if f.endswith((".cu", ".cuh", ".cpp", ".h"))]
+    return out
+
+
 def stale() -> bool:
     if not os.path.exists(LIB):
         return True
     t = os.path.getmtime(LIB)
-    deps = [os.path.join(CSRC, d) for d in DEPENDS] + [os.path.join(INCLUDE, h) for h in ("pagedkv.h", "pagedkv_block_manager.h")]
-    return any(os.path.getmtime(d) > t for d in deps)
+    return any(os.path.getmtime(d) > t for d in depends())
 
 
 def build(force: bool = False, verbose: bool = False) -> str:

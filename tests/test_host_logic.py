@@ -135,3 +135,29 @@ def test_fp8_workload_codes():
     vals = torch.from_numpy(codes_live).view(torch.float8_e4m3fn).float() * 0.02
     assert abs(vals.std().item() - 1.0) < 0.1                     # N(0,1) after the scale
     assert w.kv_bytes() == 2 * int(w.context_lens.sum()) * 2 * 128  # one byte per element
+
+
+def test_build_tracks_every_included_file(tmp_path, monkeypatch):
+    """The library is rebuilt when any file it is compiled from changes: every local #include reachable
+    from the sources is among the build's dependencies, and a library older than one of them is stale."""
+    import os
+    import re
+    from paged_kv_cache_409_b200 import build
+    deps = {os.path.basename(d) for d in build.depends()}
+    todo, seen = list(build.SOURCES), set()
+    while todo:
+        f = todo.pop()
+        if f in seen:
+            continue
+        seen.add(f)
+        path = os.path.join(build.CSRC if os.path.exists(os.path.join(build.CSRC, f)) else build.INCLUDE, f)
+        todo += re.findall(r'#include\s+"([^"]+)"', open(path).read())
+    assert seen <= deps, seen - deps
+    newest = max(os.path.getmtime(d) for d in build.depends())
+    lib = tmp_path / "lib.so"
+    lib.write_bytes(b"")
+    monkeypatch.setattr(build, "LIB", str(lib))
+    os.utime(lib, (newest - 10, newest - 10))
+    assert build.stale()
+    os.utime(lib, (newest + 10, newest + 10))
+    assert not build.stale()
