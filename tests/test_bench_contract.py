@@ -48,3 +48,22 @@ def test_copy_blocks_measurement_pairs_are_disjoint():
         assert len(src) == len(dst) == len(p) and not (src & dst)
         assert p.min() >= 0 and p.max() < nb and p.dtype == np.int64
         assert len(p) == min(nb // 2, max(1, (512 << 20) // bb))
+
+
+def test_traffic_ratios_match_the_committed_profiles():
+    """roofline.traffic scales a committed ncu capture: each ratio's DRAM and algorithmic megabytes are the
+    ones its profile summary prints (to the summary's rounding), and the profile file exists."""
+    import importlib.util
+    import re
+    spec = importlib.util.spec_from_file_location("bench_module2", os.path.join(ROOT, "bench.py"))
+    bench = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(bench)
+    for cfg, (ratio, source) in bench.TRAFFIC_PER_ALGORITHMIC_BYTE.items():
+        path = os.path.join(ROOT, source.split(" ")[0])
+        assert os.path.exists(path), (cfg, source)
+        text = open(path).read()
+        mbs = [float(x) for x in re.findall(r"(\d+\.\d+) MB", text)]
+        assert 1.0 <= ratio < 1.1, cfg
+        # some read + write (+ merge) combination of the printed figures over a printed algorithmic figure
+        assert any(abs(ratio - t / a) < 2e-3 for a in mbs for t in mbs + [x + y for x in mbs for y in mbs]
+                   + [x + y + z for x in mbs for y in mbs for z in mbs] if a > 0), (cfg, ratio)
