@@ -217,3 +217,28 @@ def test_python_constants_match_the_headers():
         enum["PKV_BM_OK"], enum["PKV_BM_EINVAL"], enum["PKV_BM_ENOSPACE"], enum["PKV_BM_EBUFFER"])
     for code in ("PKV_EINVAL", "PKV_EUNSUPPORTED", "PKV_ERANGE", "PKV_ECUDA", "PKV_EWORKSPACE"):
         assert pkv.load_library().pkv_status_string(enum[code]) != b"ok"
+
+
+def test_partition_heuristics_properties(lib):
+    """Over random batches: a recommended partition is 0 (no split) or a block multiple of at least 256
+    tokens (512 for the E4M3 wave rule) shorter than the longest context, and the workspace it needs is
+    what pkv_decode_workspace_size reports for it."""
+    from hypothesis import given, settings, strategies as st
+
+    @settings(max_examples=300, deadline=None)
+    @given(st.integers(1, 512), st.sampled_from([1, 2, 4, 8]), st.sampled_from([1, 2, 4, 8, 32]),
+           st.sampled_from([8, 16, 32]), st.integers(1, 40000), st.floats(0.05, 1.0),
+           st.sampled_from([torch.float16, torch.bfloat16, torch.float32, pkv.FP8_E4M3]))
+    def check(S, G, Hkv, B, max_len, mean_frac, dt):
+        total = max(S, int(S * max_len * mean_frac))
+        p = pkv.decode_partition_size(S, Hkv * G, Hkv, 128, B, max_len, dt, total_context_tokens=total)
+        assert p == 0 or (p % B == 0 and 256 <= p < max_len)
+        if p:
+            parts = -(-max_len // p)
+            rows = S * Hkv * G * parts
+            assert pkv.decode_workspace_size(S, Hkv * G, 128, max_len, p) == 2 * (-(-rows * 4 // 16) * 16) + \
+                rows * 128 * 4
+        m = pkv.decode_multi_partition_size(S, Hkv, B, max_len)
+        assert m == 0 or (m % B == 0 and m >= 256 and m < max_len)
+
+    check()
