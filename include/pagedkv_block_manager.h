@@ -147,7 +147,11 @@ int pkv_bm_swap_out(pkv_block_manager* bm, int64_t seq_id, int64_t* pairs_out, i
 /* Resume a swapped-out seq_id: pairs_out receives one (host block, device
  * block) pair per block, in logical order; copy them host -> device before the
  * sequence's next attention.  The sequence's table then lists the new device
- * blocks.  PKV_BM_ENOSPACE when the device pool has too few free or evictable
+ * blocks.  The host blocks named as sources go back to the host free stack at
+ * once, so a later pkv_bm_swap_out (of this step or a later one) may name one
+ * of them as its copy target: enqueue this call's host -> device copies before
+ * the device -> host copies of any later swap-out, on the same stream (or with
+ * an event between the two streams).  PKV_BM_ENOSPACE when the device pool has too few free or evictable
  * blocks, PKV_BM_EBUFFER when max_pairs is too small; on failure nothing
  * changes. */
 int pkv_bm_swap_in(pkv_block_manager* bm, int64_t seq_id, int64_t* pairs_out, int64_t max_pairs,

@@ -437,3 +437,31 @@ def test_group_swap_in_part_of_a_group():
     assert bm.stats()["free_host"] == 8
     with pytest.raises(BlockManagerError):
         bm.swap_out([1, 1])                                # repeated id
+
+
+def test_swap_in_then_swap_out_in_one_step_reuses_a_host_block_in_call_order():
+    """Swap-in returns its host blocks to the host free stack at once, so a swap-out made right after it
+    may target one of them.  Applying each call's copies in the order of the calls (swap-in's host ->
+    device first) keeps both sequences' K/V intact; the reverse order would overwrite A's saved rows."""
+    B, NB, NH = 4, 8, 2
+    bm = BlockManager(NB, B, prefix_caching=False, num_host_blocks=NH)
+    dev = np.full((NB * B, 2), -1.0)
+    host = np.full((NH * B, 2), -1.0)
+
+    def move(src, dst, pairs):
+        for a, b in pairs:
+            dst[b * B:(b + 1) * B] = src[a * B:(a + 1) * B]
+
+    for sid in (1, 2):
+        bm.add_sequence(sid, [sid] * 6)                    # two blocks each, the second partial
+        for p, sl in enumerate(bm.slots(sid, 0, 6)):
+            dev[sl] = (sid, p)
+    move(dev, host, bm.swap_out(1))                        # A = 1 fills the whole host pool
+    pin = bm.swap_in(1)                                    # A's host blocks are free again ...
+    pout = bm.swap_out(2)                                  # ... and B = 2 is saved into them
+    assert set(pin[:, 0].tolist()) & set(pout[:, 1].tolist())
+    move(host, dev, pin)                                   # call order: A's copies in first
+    move(dev, host, pout)
+    assert np.array_equal(dev[bm.slots(1, 0, 6)], np.array([(1.0, p) for p in range(6)]))
+    move(host, dev, bm.swap_in(2))
+    assert np.array_equal(dev[bm.slots(2, 0, 6)], np.array([(2.0, p) for p in range(6)]))
