@@ -190,7 +190,11 @@ int pkv_swap_blocks(const void* src_key_pool, const void* src_value_pool, void* 
  *                   aligned; may be NULL when that size is 0.  Its contents
  *                   need no initialisation and are scratch after the call.
  * Supported: head_dim in {64, 128}; block_size in {8, 16, 32}; dtype in
- * {F32, F16, BF16}; num_q_heads / num_kv_heads in {1, 2, 4, 8}.
+ * {F32, F16, BF16}; num_q_heads / num_kv_heads in {1, 2, 4, 8}.  A partition
+ * holds at most 4096 blocks (a CTA keeps its block ids in shared memory): a
+ * partition_size above 4096 * block_size, or partition_size 0 with
+ * max_context_len above it, returns PKV_EUNSUPPORTED.
+ * pkv_decode_partition_size never recommends more.
  */
 int pkv_paged_attention_decode(void* out, const void* query, const void* key_cache,
                                const void* value_cache, const int32_t* block_tables,
@@ -234,9 +238,11 @@ size_t pkv_decode_workspace_size(int num_seqs, int num_q_heads, int head_dim, in
  * the GPU and no context is far longer than the mean, else a multiple of
  * block_size.  total_context_tokens (sum of context_lens, 0 = unknown) lets
  * it see a long tail and, for E4M3 pools (dtype PKV_FP8_E4M3) with one query
- * head per KV head, size parts so that the CTAs fill whole waves.
- * num_q_heads must be a multiple of num_kv_heads.  Returns a negative
- * pkv_status on bad input. */
+ * head per KV head, size parts so that the CTAs fill whole waves.  The result
+ * is at most 4096 * block_size, and a max_context_len above that is always
+ * split (into equal parts under the limit), so the decode accepts every
+ * recommendation.  num_q_heads must be a multiple of num_kv_heads.  Returns a
+ * negative pkv_status on bad input. */
 int pkv_decode_partition_size(int num_seqs, int num_q_heads, int num_kv_heads, int head_dim, int block_size,
                               int max_context_len, int64_t total_context_tokens, int dtype);
 
@@ -341,7 +347,9 @@ int pkv_paged_attention_decode_multi(void* out, const void* query, const void* k
 
 /* Partition size (tokens) recommended for pkv_paged_attention_decode_multi:
  * enough partitions for about eight CTAs per SM, at least 256 tokens each, a
- * multiple of block_size; 0 = no split.  Negative pkv_status on bad input. */
+ * multiple of block_size, at most 4096 blocks (the per-partition limit the
+ * call shares with pkv_paged_attention_decode); 0 = no split.  Negative
+ * pkv_status on bad input. */
 int pkv_decode_multi_partition_size(int num_chunks, int num_kv_heads, int block_size, int max_seq_len);
 
 /*
@@ -360,9 +368,14 @@ int pkv_decode_multi_partition_size(int num_chunks, int num_kv_heads, int block_
  *   - A request that needs more scratch than that (see
  *     pkv_decode_workspace_size) returns PKV_EWORKSPACE before any device work;
  *     partition_size == 0 needs none.
- *   - The first call on a device looks up the array's device address
- *     (cudaGetSymbolAddress) with that device current; make that first call
- *     before any stream capture.
+ *   - The first call in a CUDA context (the device's primary context, or a
+ *     context the caller made current through the driver API) looks up the
+ *     array's device address in that context (cudaGetSymbolAddress) with its
+ *     device current, and caches it per context; make that first call before
+ *     any stream capture.  A device reset (cudaDeviceReset) invalidates the
+ *     cached address: do not call this entry point after one.
+ *   - Bad arguments give the status pkv_paged_attention_decode gives; only
+ *     then is the scratch size checked.
  *   - All calls share the one array, which keeps the last call's contents.
  *     The decode writes every partial it later reads, so nothing needs to
  *     start at zero.  Calls whose executions overlap on the GPU (different

@@ -368,6 +368,10 @@ int launch_merge(int head_dim, const pkv::MergeParams& mp, cudaStream_t s) {
 
 bool supported_group(int g) { return g == 1 || g == 2 || g == 4 || g == 8; }
 
+// A decode CTA keeps its partition's block ids in shared memory: at most this
+// many blocks per partition.
+constexpr int64_t kMaxPartitionBlocks = 4096;
+
 int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
 
 // ------------------------------------------------------------ prefill dispatch
@@ -400,13 +404,13 @@ int prefill_by_group(int group, const pkv::PrefillParams& prm, const CUtensorMap
     }
 }
 
-// Decode with the query / output in `dtype` and the pools in `kv_dtype`
-// (the same 16/32-bit type, or FP8 E4M3 with its two scales).
-int decode_impl(void* out, const void* query, const void* key_cache, const void* value_cache,
-                const int32_t* block_tables, const int32_t* context_lens, float scale, int num_seqs, int num_q_heads,
-                int num_kv_heads, int head_dim, int block_size, int max_blocks_per_seq, int64_t num_blocks,
-                int max_context_len, int partition_size, int dtype, int kv_dtype, float k_scale, float v_scale,
-                void* workspace, size_t workspace_bytes, pkv_stream_t stream) {
+// Argument checks of the decode entry points that need no workspace: the
+// status the decode returns for these arguments, or PKV_OK (num_seqs == 0
+// passes: it launches nothing).
+int decode_check(const void* out, const void* query, const void* key_cache, const void* value_cache,
+                 const int32_t* block_tables, const int32_t* context_lens, float scale, int num_seqs,
+                 int num_q_heads, int num_kv_heads, int head_dim, int block_size, int max_blocks_per_seq,
+                 int64_t num_blocks, int max_context_len, int partition_size, int dtype, int kv_dtype) {
     const bool fp8 = kv_dtype == PKV_FP8_E4M3;
     if (!query_type(dtype) || (kv_dtype != dtype && !fp8)) return PKV_EUNSUPPORTED;
     if (fp8 && (dtype == PKV_F32 || head_dim != 128)) return PKV_EUNSUPPORTED;
@@ -425,13 +429,32 @@ int decode_impl(void* out, const void* query, const void* key_cache, const void*
     if (!aligned16(out) || !aligned16(query) || !aligned16(key_cache) || !aligned16(value_cache) ||
         (reinterpret_cast<uintptr_t>(block_tables) & 3) || (reinterpret_cast<uintptr_t>(context_lens) & 3))
         return PKV_EINVAL;
+    const int64_t max_blocks_needed = std::max<int64_t>(1, ceil_div(std::max(max_context_len, 1), block_size));
+    const int64_t pb = std::min<int64_t>(partition_size > 0 ? partition_size / block_size : max_blocks_needed,
+                                         max_blocks_needed);
+    if (pb > kMaxPartitionBlocks) return PKV_EUNSUPPORTED;
+    return PKV_OK;
+}
+
+// Decode with the query / output in `dtype` and the pools in `kv_dtype`
+// (the same 16/32-bit type, or FP8 E4M3 with its two scales).
+int decode_impl(void* out, const void* query, const void* key_cache, const void* value_cache,
+                const int32_t* block_tables, const int32_t* context_lens, float scale, int num_seqs, int num_q_heads,
+                int num_kv_heads, int head_dim, int block_size, int max_blocks_per_seq, int64_t num_blocks,
+                int max_context_len, int partition_size, int dtype, int kv_dtype, float k_scale, float v_scale,
+                void* workspace, size_t workspace_bytes, pkv_stream_t stream) {
+    const int check = decode_check(out, query, key_cache, value_cache, block_tables, context_lens, scale, num_seqs,
+                                   num_q_heads, num_kv_heads, head_dim, block_size, max_blocks_per_seq, num_blocks,
+                                   max_context_len, partition_size, dtype, kv_dtype);
+    if (check || num_seqs == 0) return check;
+    const bool fp8 = kv_dtype == PKV_FP8_E4M3;
+    const int group = num_q_heads / num_kv_heads;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
 
     const int64_t max_blocks_needed = std::max<int64_t>(1, ceil_div(std::max(max_context_len, 1), block_size));
     int64_t pb = partition_size > 0 ? partition_size / block_size : max_blocks_needed;
     pb = std::min(pb, max_blocks_needed);
     const int64_t parts = ceil_div(max_blocks_needed, pb);
-    if (pb > 4096) return PKV_EUNSUPPORTED;  // per-CTA block list lives in shared memory
     const size_t need = parts > 1 ? pkv_decode_workspace_size(num_seqs, num_q_heads, head_dim, max_context_len,
                                                               (int)(pb * block_size))
                                   : 0;
@@ -699,9 +722,14 @@ int pkv_decode_partition_size(int num_seqs, int num_q_heads, int num_kv_heads, i
     (void)head_dim;
     const int64_t pairs = (int64_t)num_seqs * num_kv_heads;
     if (max_context_len <= 0 || pairs == 0) return 0;
+    // A partition holds at most kMaxPartitionBlocks blocks; a longer context
+    // is always split, into equal parts under that cap.
+    const int64_t cap = kMaxPartitionBlocks * block_size;
+    const int64_t longest = ceil_div(max_context_len, ceil_div(max_context_len, cap));
     auto round_ps = [&](int64_t ps) -> int {
         ps = std::max<int64_t>(ps, 256);
         ps = ceil_div(ps, block_size) * block_size;
+        ps = std::min(ps, ceil_div(longest, block_size) * block_size);
         return ps >= max_context_len ? 0 : (int)ps;
     };
     const int64_t target = 4 * (int64_t)sm_count();
@@ -735,7 +763,7 @@ int pkv_decode_partition_size(int num_seqs, int num_q_heads, int num_kv_heads, i
             return round_ps(std::max<int64_t>((int64_t)std::ceil(per_part), 512));
         }
     }
-    return 0;
+    return round_ps(longest);  // 0 unless the longest context exceeds the cap
 }
 
 int pkv_paged_attention_decode(void* out, const void* query, const void* key_cache, const void* value_cache,
@@ -873,7 +901,7 @@ int pkv_paged_attention_decode_multi(void* out, const void* query, const void* k
     int64_t pb = partition_size > 0 ? partition_size / block_size : max_blocks_needed;
     pb = std::min(pb, max_blocks_needed);
     const int64_t parts = ceil_div(max_blocks_needed, pb);
-    if (pb > 4096) return PKV_EUNSUPPORTED;
+    if (pb > kMaxPartitionBlocks) return PKV_EUNSUPPORTED;
     const size_t need = parts > 1 ? pkv_decode_workspace_size((int)total_q_tokens, num_q_heads, head_dim,
                                                               max_seq_len, (int)(pb * block_size))
                                   : 0;
@@ -967,10 +995,12 @@ int pkv_decode_multi_partition_size(int num_chunks, int num_kv_heads, int block_
     if (max_seq_len <= 0 || pairs == 0) return 0;
     // About eight CTAs per SM over the whole launch, so that CTAs of uneven
     // length even out; partitions of at least 256 tokens.
+    // Never more than kMaxPartitionBlocks blocks per partition.
     const int64_t target = 8 * (int64_t)sm_count();
-    const int64_t parts = std::max<int64_t>(1, ceil_div(target, pairs));
+    const int64_t cap = kMaxPartitionBlocks * block_size;
+    const int64_t parts = std::max(std::max<int64_t>(1, ceil_div(target, pairs)), ceil_div(max_seq_len, cap));
     int64_t ps = std::max<int64_t>(256, ceil_div(max_seq_len, parts));
-    ps = ceil_div(ps, block_size) * block_size;
+    ps = std::min(ceil_div(ps, block_size) * block_size, cap);
     return ps >= max_seq_len ? 0 : (int)ps;
 }
 
@@ -1117,33 +1147,77 @@ static __device__ __align__(256) unsigned char g_static_decode_scratch[PKV_STATI
 
 namespace {
 
-// Device address of the scratch array on the current device, looked up once
-// per device (with that device current) and cached.
+// Device address of the scratch array in the current device's current
+// context, looked up once per context (with that device current) and cached.
+// A __device__ array has one address per CUDA context, so the cache is keyed
+// by the context, not by the device number: a caller on a context of its own
+// (driver API) gets that context's copy.
+using CtxGetCurrentFn = CUresult (*)(CUcontext*);
+
+CtxGetCurrentFn ctx_get_current_fn() {
+    static CtxGetCurrentFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<CtxGetCurrentFn>(p);
+    });
+    return fn;
+}
+
 void* static_scratch_address(int* rc) {
     static std::mutex mu;
-    static void* addr[64] = {};
-    int dev = 0;
-    cudaError_t e = cudaGetDevice(&dev);
-    if (e != cudaSuccess) {
-        *rc = cuda_fail(e, "cudaGetDevice");
+    constexpr int kSlots = 64;
+    static CUcontext ctx_of[kSlots] = {};
+    static void* addr_of[kSlots] = {};
+    CtxGetCurrentFn get_ctx = ctx_get_current_fn();
+    CUcontext ctx = nullptr;
+    void* looked = nullptr;
+    if (!get_ctx || get_ctx(&ctx) != CUDA_SUCCESS) {
+        snprintf(g_last_cuda_error, sizeof g_last_cuda_error, "cuCtxGetCurrent unavailable or failed");
+        *rc = PKV_ECUDA;
         return nullptr;
     }
-    if (dev < 0 || dev >= 64) {
-        *rc = PKV_EUNSUPPORTED;
-        return nullptr;
-    }
-    std::lock_guard<std::mutex> lock(mu);
-    if (!addr[dev]) {
-        void* p = nullptr;
-        e = cudaGetSymbolAddress(&p, g_static_decode_scratch);
-        if (e != cudaSuccess || !p) {
+    if (!ctx) {
+        // No context current on this host thread yet: the runtime's lookup
+        // makes the current device's primary context current.
+        cudaError_t e = cudaGetSymbolAddress(&looked, g_static_decode_scratch);
+        if (e != cudaSuccess || !looked) {
             *rc = cuda_fail(e != cudaSuccess ? e : cudaErrorInvalidSymbol, "cudaGetSymbolAddress(scratch)");
             return nullptr;
         }
-        addr[dev] = p;
+        if (get_ctx(&ctx) != CUDA_SUCCESS || !ctx) {
+            snprintf(g_last_cuda_error, sizeof g_last_cuda_error, "no current CUDA context");
+            *rc = PKV_ECUDA;
+            return nullptr;
+        }
     }
+    std::lock_guard<std::mutex> lock(mu);
+    int free_slot = -1;
+    for (int i = 0; i < kSlots; ++i) {
+        if (ctx_of[i] == ctx) {
+            *rc = PKV_OK;
+            return addr_of[i];
+        }
+        if (!ctx_of[i] && free_slot < 0) free_slot = i;
+    }
+    if (free_slot < 0) {
+        *rc = PKV_EUNSUPPORTED;
+        return nullptr;
+    }
+    if (!looked) {
+        cudaError_t e = cudaGetSymbolAddress(&looked, g_static_decode_scratch);
+        if (e != cudaSuccess || !looked) {
+            *rc = cuda_fail(e != cudaSuccess ? e : cudaErrorInvalidSymbol, "cudaGetSymbolAddress(scratch)");
+            return nullptr;
+        }
+    }
+    ctx_of[free_slot] = ctx;
+    addr_of[free_slot] = looked;
     *rc = PKV_OK;
-    return addr[dev];
+    return looked;
 }
 
 }  // namespace
@@ -1153,8 +1227,14 @@ extern "C" int pkv_paged_attention_decode_static_scratch(
     const int32_t* context_lens, float scale, int num_seqs, int num_q_heads, int num_kv_heads, int head_dim,
     int block_size, int max_blocks_per_seq, int64_t num_blocks, int max_context_len, int partition_size, int dtype,
     pkv_stream_t stream) {
-    // Size check first: a request that needs more scratch than the array holds
-    // is refused before any device work.
+    // The decode's own argument checks first, so that both entry points return
+    // the same status for the same bad input; then the size check: a request
+    // that needs more scratch than the array holds is refused before any
+    // device work.
+    const int check = decode_check(out, query, key_cache, value_cache, block_tables, context_lens, scale, num_seqs,
+                                   num_q_heads, num_kv_heads, head_dim, block_size, max_blocks_per_seq, num_blocks,
+                                   max_context_len, partition_size, dtype, dtype);
+    if (check) return check;
     int64_t ps = partition_size;
     if (ps > 0 && block_size > 0 && max_context_len > 0) {
         const int64_t max_blocks = ceil_div(max_context_len, block_size);

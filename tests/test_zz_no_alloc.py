@@ -6,8 +6,10 @@ loop that must not touch the allocator between steps) use
 ``pkv_paged_attention_decode_static_scratch``: the split-K scratch is the
 library's own device array instead of a caller workspace.  This test calls it
 through the C ABI and checks it against ``pkv_paged_attention_decode`` with an
-ordinary workspace, on two calls in a row with different inputs, and checks
-that an oversized request is refused.  The file is named to run last.
+ordinary workspace and against the CPU oracle, on two calls in a row with
+different inputs, checks that an oversized request is refused, and that a bad
+argument gets the status the workspace entry point gives.  The file is named
+to run last.
 """
 import ctypes
 
@@ -15,13 +17,14 @@ import numpy as np
 import pytest
 import torch
 
+import oracle
 import paged_kv_cache_409_b200 as pkv
 from paged_kv_cache_409_b200 import workloads
-from parity_helpers import TOL, gpu_tables, to_device
+from parity_helpers import TOL, assert_close, gpu_tables, to_device
 
 pytestmark = pytest.mark.gpu
 
-EWORKSPACE = -5
+EINVAL, EWORKSPACE = -1, -5
 SCRATCH_BYTES = 32 << 20
 
 
@@ -51,7 +54,10 @@ def _close(a, b, dtype):
 @pytest.mark.parametrize("dtype,Hq,Hkv", [(torch.float16, 8, 8), (torch.bfloat16, 16, 2)])
 def test_static_scratch_matches_workspace_decode_twice(dtype, Hq, Hkv):
     f = _entry()
-    w = to_device(workloads.decode_workload("ns", [700, 1, 129, 2000, 64, 1500], Hq, Hkv, 128, 16, dtype, seed=31))
+    w = workloads.decode_workload("ns", [700, 1, 129, 2000, 64, 1500], Hq, Hkv, 128, 16, dtype, seed=31)
+    kn, code = oracle.storage(w.key_caches[0].clone())  # host snapshots for the oracle, before any GPU work
+    vn, _ = oracle.storage(w.value_caches[0].clone())
+    w = to_device(w)
     bt, cl, _ = gpu_tables(w)
     part = 256  # several partitions per sequence: the scratch is used
     assert 0 < pkv.decode_workspace_size(w.num_seqs, Hq, 128, w.max_context_len, part) <= SCRATCH_BYTES
@@ -62,9 +68,13 @@ def test_static_scratch_matches_workspace_decode_twice(dtype, Hq, Hkv):
         pkv.paged_attention_decode(ref, q, w.key_caches[0], w.value_caches[0], bt, cl, w.scale, w.max_context_len,
                                    partition_size=part)
         out = torch.full_like(q, float("nan"))
+        qh = q.cpu()
         assert _call(f, out, w, q, bt, cl, part) == 0, f"call {call}"
         torch.cuda.synchronize()
         _close(out, ref, dtype)
+        want = oracle.get().paged_attention_decode(oracle.storage(qh)[0], kn, vn, w.block_tables, w.context_lens,
+                                                   w.scale, code)
+        assert_close(out, want, dtype, f"static-scratch call {call} vs oracle")
     assert pkv.get_device_error() == 0
 
 
@@ -88,3 +98,20 @@ def test_static_scratch_refuses_oversized_request():
                                w.max_context_len, partition_size=0)
     torch.cuda.synchronize()
     _close(out, ref, torch.bfloat16)
+
+
+def test_static_scratch_bad_argument_gets_the_workspace_calls_status():
+    """A partition_size that is not a multiple of block_size is an invalid argument for both decode entry
+    points, even when the request would also be too large for the library's array."""
+    f = _entry()
+    lib = pkv.load_library()
+    g = lib.pkv_paged_attention_decode
+    w = to_device(workloads.decode_workload("bad", [64] * 2, 64, 8, 128, 16, torch.bfloat16, seed=33))
+    bt, cl, _ = gpu_tables(w)
+    big = torch.empty(512, 64, 128, dtype=torch.bfloat16, device="cuda")
+    args = (big.data_ptr(), big.data_ptr(), w.key_caches[0].data_ptr(), w.value_caches[0].data_ptr(),
+            bt.data_ptr(), cl.data_ptr(), w.scale, 512, 64, 8, 128, 16, bt.shape[1], w.num_blocks, 4096, 24, 2)
+    assert pkv.decode_workspace_size(512, 64, 128, 4096, 24) > SCRATCH_BYTES
+    stream = torch.cuda.current_stream().cuda_stream
+    assert g(*args, None, 0, stream) == EINVAL
+    assert f(*args, stream) == EINVAL
