@@ -33,7 +33,7 @@ F32, F16, BF16, E4M3 = 0, 1, 2, 3
 def compile_source(src: str, out: str) -> str:
     """gcc -O2 one C source of the oracle into a shared library at ``out``."""
     tmp = out + f".tmp{os.getpid()}"
-    subprocess.check_call(["gcc", "-O2", "-std=c11", "-fPIC", "-shared", "-o", tmp, src, "-lm"])
+    subprocess.check_call(["gcc", "-O2", "-std=c11", "-fopenmp", "-fPIC", "-shared", "-o", tmp, src, "-lm"])
     os.replace(tmp, out)
     return out
 
@@ -77,6 +77,8 @@ class Oracle:
     def __init__(self, path: str):
         lib = ctypes.CDLL(path)
         P, I, L, D = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_double
+        lib.oracle_num_threads.argtypes = [I]
+        lib.oracle_num_threads.restype = I
         lib.oracle_to_double.argtypes = [P, P, L, I]
         lib.oracle_blocks_needed.argtypes = [L, I]
         lib.oracle_blocks_needed.restype = L
@@ -98,6 +100,10 @@ class Oracle:
             f.restype = ctypes.c_int
         self.lib = lib
         self.path = path
+
+    def num_threads(self, n: int = 0) -> int:
+        """Host threads the attention functions use (n > 0 sets it); 1 without OpenMP."""
+        return int(self.lib.oracle_num_threads(int(n)))
 
     def to_double(self, a: np.ndarray, dtype: int) -> np.ndarray:
         a = np.ascontiguousarray(a)

@@ -56,7 +56,23 @@
 #include <stdlib.h>
 #include <string.h>
 
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
 enum { ORC_F32 = 0, ORC_F16 = 1, ORC_BF16 = 2, ORC_E4M3 = 3 };
+
+/* Host threads the attention functions may use: n > 0 sets the number, any
+ * n returns the number now in force (1 in a build without OpenMP). */
+int oracle_num_threads(int n) {
+#ifdef _OPENMP
+    if (n > 0) omp_set_num_threads(n);
+    return omp_get_max_threads();
+#else
+    (void)n;
+    return 1;
+#endif
+}
 
 static int elem_bytes(int dtype) {
     switch (dtype) {
@@ -328,33 +344,40 @@ int oracle_paged_attention_decode_kv(double* out, const void* query, int q_dtype
         num_q_heads % num_kv_heads != 0 || head_dim <= 0 || block_size <= 0)
         return -1;
     int group = num_q_heads / num_kv_heads;
-    int rc = 0;
-    for (int64_t s = 0; s < num_seqs && rc == 0; ++s) {
+    for (int64_t s = 0; s < num_seqs; ++s) {
         int64_t n = context_lens[s];
         if (n < 0 || n > (int64_t)max_blocks_per_seq * block_size) return -1;
+    }
+    /* Each (sequence, KV head) pair is independent; with OpenMP the pairs are
+     * shared out over the host threads, each output row still computed by one
+     * thread in the same order (the result does not depend on the thread count). */
+    int64_t pairs = num_seqs * (int64_t)num_kv_heads;
+    int bad = 0;
+#pragma omp parallel for schedule(dynamic, 1) reduction(| : bad)
+    for (int64_t p = 0; p < pairs; ++p) {
+        int64_t s = p / num_kv_heads;
+        int g = (int)(p % num_kv_heads);
+        int64_t n = context_lens[s];
         int64_t cap = n > 0 ? n : 1;
         double* Kc = (double*)malloc(sizeof(double) * cap * head_dim);
         double* Vc = (double*)malloc(sizeof(double) * cap * head_dim);
         double* x = (double*)malloc(sizeof(double) * cap);
         double* qv = (double*)malloc(sizeof(double) * head_dim);
-        if (!Kc || !Vc || !x || !qv) {
-            free(Kc); free(Vc); free(x); free(qv);
-            return -1;
-        }
-        for (int g = 0; g < num_kv_heads && rc == 0; ++g) {
+        int rc = (!Kc || !Vc || !x || !qv) ? -1 : 0;
+        if (rc == 0)
             rc = gather_sequence(Kc, Vc, key_cache, value_cache, kv_dtype, k_scale, v_scale,
                                  block_tables + s * max_blocks_per_seq, n, g, num_kv_heads, head_dim,
                                  block_size, max_blocks_per_seq, num_blocks);
-            for (int hh = 0; hh < group && rc == 0; ++hh) {
-                int h = g * group + hh;
-                for (int d = 0; d < head_dim; ++d)
-                    qv[d] = load_elem(query, (s * num_q_heads + h) * (int64_t)head_dim + d, q_dtype);
-                attend(out + (s * num_q_heads + h) * (int64_t)head_dim, qv, Kc, Vc, n, head_dim, scale, x);
-            }
+        for (int hh = 0; hh < group && rc == 0; ++hh) {
+            int h = g * group + hh;
+            for (int d = 0; d < head_dim; ++d)
+                qv[d] = load_elem(query, (s * num_q_heads + h) * (int64_t)head_dim + d, q_dtype);
+            attend(out + (s * num_q_heads + h) * (int64_t)head_dim, qv, Kc, Vc, n, head_dim, scale, x);
         }
         free(Kc); free(Vc); free(x); free(qv);
+        bad |= rc != 0;
     }
-    return rc;
+    return bad ? -1 : 0;
 }
 
 /* Decode with query and pools of one type (no scaling). */
@@ -390,42 +413,49 @@ int oracle_paged_attention_prefill_chunk_kv(double* out, const void* query, int 
         num_q_heads % num_kv_heads != 0 || head_dim <= 0 || block_size <= 0)
         return -1;
     int group = num_q_heads / num_kv_heads;
-    int rc = 0;
-    for (int r = 0; r < num_chunks && rc == 0; ++r) {
+    for (int r = 0; r < num_chunks; ++r) {
+        int64_t nq = (int64_t)query_start_loc[r + 1] - query_start_loc[r];
+        int64_t len = seq_lens[r];
+        if (nq < 0 || len < nq || len > (int64_t)max_blocks_per_seq * block_size) return -1;
+    }
+    /* (chunk, KV head) pairs are independent: shared out over the host
+     * threads under OpenMP, each output row computed by one thread. */
+    int64_t pairs = (int64_t)num_chunks * num_kv_heads;
+    int bad = 0;
+#pragma omp parallel for schedule(dynamic, 1) reduction(| : bad)
+    for (int64_t p = 0; p < pairs; ++p) {
+        int r = (int)(p / num_kv_heads);
+        int g = (int)(p % num_kv_heads);
         int64_t q0 = query_start_loc[r];
         int64_t nq = (int64_t)query_start_loc[r + 1] - q0;
         int64_t len = seq_lens[r];
-        if (nq < 0 || len < nq || len > (int64_t)max_blocks_per_seq * block_size) return -1;
         int64_t c0 = len - nq;
         int64_t cap = len > 0 ? len : 1;
         double* Kc = (double*)malloc(sizeof(double) * cap * head_dim);
         double* Vc = (double*)malloc(sizeof(double) * cap * head_dim);
         double* x = (double*)malloc(sizeof(double) * cap);
         double* qv = (double*)malloc(sizeof(double) * head_dim);
-        if (!Kc || !Vc || !x || !qv) {
-            free(Kc); free(Vc); free(x); free(qv);
-            return -1;
-        }
-        for (int g = 0; g < num_kv_heads && rc == 0; ++g) {
+        int rc = (!Kc || !Vc || !x || !qv) ? -1 : 0;
+        if (rc == 0)
             rc = gather_sequence(Kc, Vc, key_cache, value_cache, kv_dtype, k_scale, v_scale,
                                  block_tables + (int64_t)r * max_blocks_per_seq, len, g, num_kv_heads,
                                  head_dim, block_size, max_blocks_per_seq, num_blocks);
-            for (int64_t i = 0; i < nq && rc == 0; ++i) {
-                int64_t row = q0 + i;
-                if (row_select && !row_select[row]) continue;
-                for (int hh = 0; hh < group; ++hh) {
-                    int h = g * group + hh;
-                    for (int d = 0; d < head_dim; ++d)
-                        qv[d] = load_elem(query, (row * num_q_heads + h) * (int64_t)head_dim + d, q_dtype);
-                    /* causal key set: positions 0 .. c0 + i inclusive */
-                    attend(out + (row * num_q_heads + h) * (int64_t)head_dim, qv, Kc, Vc, c0 + i + 1,
-                           head_dim, scale, x);
-                }
+        for (int64_t i = 0; i < nq && rc == 0; ++i) {
+            int64_t row = q0 + i;
+            if (row_select && !row_select[row]) continue;
+            for (int hh = 0; hh < group; ++hh) {
+                int h = g * group + hh;
+                for (int d = 0; d < head_dim; ++d)
+                    qv[d] = load_elem(query, (row * num_q_heads + h) * (int64_t)head_dim + d, q_dtype);
+                /* causal key set: positions 0 .. c0 + i inclusive */
+                attend(out + (row * num_q_heads + h) * (int64_t)head_dim, qv, Kc, Vc, c0 + i + 1,
+                       head_dim, scale, x);
             }
         }
         free(Kc); free(Vc); free(x); free(qv);
+        bad |= rc != 0;
     }
-    return rc;
+    return bad ? -1 : 0;
 }
 
 /* Prefill with query and pools of one type (no scaling). */

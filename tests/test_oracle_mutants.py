@@ -13,10 +13,10 @@ from oracle_pins import ALL_PINS
 
 MUTANTS = {
     "drop_scale": ("x[j] = scale * dot;", "x[j] = dot;"),
-    "group_head_mapping": ("int h = g * group + hh;\n                for (int d = 0; d < head_dim; ++d)\n"
-                           "                    qv[d] = load_elem(query, (s *",
-                           "int h = hh * num_kv_heads + g;\n                for (int d = 0; d < head_dim; ++d)\n"
-                           "                    qv[d] = load_elem(query, (s *"),
+    "group_head_mapping": ("int h = g * group + hh;\n            for (int d = 0; d < head_dim; ++d)\n"
+                           "                qv[d] = load_elem(query, (s *",
+                           "int h = hh * num_kv_heads + g;\n            for (int d = 0; d < head_dim; ++d)\n"
+                           "                qv[d] = load_elem(query, (s *"),
     "offset_in_block": ("int64_t offset = j % block_size;", "int64_t offset = 0;"),
     "causal_off_by_one": ("c0 + i + 1,", "c0 + i,"),
     "chunk_start_zero": ("int64_t c0 = len - nq;", "int64_t c0 = 0;"),
