@@ -228,6 +228,44 @@ int pkv_paged_attention_decode_fp8(void* out, const void* query, const void* key
                                    int max_context_len, int partition_size, int dtype, void* workspace,
                                    size_t workspace_bytes, pkv_stream_t stream);
 
+/*
+ * One decode step in one call: pkv_reshape_and_cache of the step's new tokens
+ * (new_keys / new_values [num_new_tokens, num_kv_heads, head_dim] in dtype, at
+ * slot_mapping), then pkv_paged_attention_decode over the same pools.  Source:
+ * case-study page section 二 (a new token's K/V go into its block, taken on
+ * demand, through the block table) and "注意力计算改造" (attention then reads
+ * the cache block by block); the guide page "KV Cache 是什么" (the new token
+ * attends to every cached token, itself included).
+ *
+ * The result equals the two calls made one after the other on `stream`.  The
+ * difference is in the launch: the decode kernel is launched as the append's
+ * programmatic dependent, so its CTAs load the query, the block tables and the
+ * lengths while the append drains, and read the pools only after the append's
+ * writes are complete.  The query, tables and lengths must therefore not be
+ * written by the append itself (they never are: it writes only pool slots).
+ * Arguments, workspace, supported shapes and errors are those of the two
+ * calls; every check of both runs before the first launch, so a refused step
+ * has changed nothing.
+ */
+int pkv_paged_attention_decode_step(const void* new_keys, const void* new_values, const int64_t* slot_mapping,
+                                    int64_t num_new_tokens, void* out, const void* query, void* key_cache,
+                                    void* value_cache, const int32_t* block_tables, const int32_t* context_lens,
+                                    float scale, int num_seqs, int num_q_heads, int num_kv_heads, int head_dim,
+                                    int block_size, int max_blocks_per_seq, int64_t num_blocks, int max_context_len,
+                                    int partition_size, int dtype, void* workspace, size_t workspace_bytes,
+                                    pkv_stream_t stream);
+
+/* The same step over FP8 (E4M3) pools: pkv_reshape_and_cache_fp8 (new tokens
+ * in dtype, quantised with k_scale / v_scale), then
+ * pkv_paged_attention_decode_fp8, launched as above. */
+int pkv_paged_attention_decode_step_fp8(const void* new_keys, const void* new_values, const int64_t* slot_mapping,
+                                        int64_t num_new_tokens, void* out, const void* query, void* key_cache,
+                                        void* value_cache, const int32_t* block_tables, const int32_t* context_lens,
+                                        float scale, float k_scale, float v_scale, int num_seqs, int num_q_heads,
+                                        int num_kv_heads, int head_dim, int block_size, int max_blocks_per_seq,
+                                        int64_t num_blocks, int max_context_len, int partition_size, int dtype,
+                                        void* workspace, size_t workspace_bytes, pkv_stream_t stream);
+
 /* Workspace bytes pkv_paged_attention_decode needs for these sizes (0 when
  * partition_size == 0 or max_context_len <= partition_size). */
 size_t pkv_decode_workspace_size(int num_seqs, int num_q_heads, int head_dim, int max_context_len,
@@ -388,6 +426,21 @@ int pkv_paged_attention_decode_static_scratch(void* out, const void* query, cons
                                               int num_q_heads, int num_kv_heads, int head_dim, int block_size,
                                               int max_blocks_per_seq, int64_t num_blocks, int max_context_len,
                                               int partition_size, int dtype, pkv_stream_t stream);
+
+/*
+ * Limit, in nanoseconds, of the bounded waits inside the kernels' main loops
+ * (decode, multi-token decode, chunked prefill) for launches made after this
+ * call on the current device; the vLLM pages have no counterpart (error
+ * handling).  PKV_DEFAULT_WAIT_LIMIT_NS (one second) is the default.  A wait
+ * that reaches its limit gives up: the kernel sets PKV_DEVERR_TIMEOUT, stops
+ * its main loop, waits (with the default limit) for its own bulk copies and
+ * tensor-core MMAs still in flight, releases its tensor memory and returns,
+ * leaving its outputs unspecified; the device stays usable.  0 makes every
+ * main-loop wait that would block give up at once: a test setting that runs
+ * that path on purpose.  Synchronises the device before and after the change.
+ */
+#define PKV_DEFAULT_WAIT_LIMIT_NS 1000000000ull
+int pkv_set_wait_limit_ns(uint64_t limit_ns);
 
 /* Read, and reset to 0, the current device's error word (PKV_DEVERR_* bits)
  * after all work queued on `stream` so far.  Synchronises `stream`. */

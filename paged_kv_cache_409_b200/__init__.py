@@ -19,10 +19,14 @@ from ._binding import (  # noqa: F401
     load_library,
     paged_attention_decode,
     paged_attention_decode_fp8,
+    paged_attention_decode_step,
+    paged_attention_decode_step_fp8,
     paged_attention_decode_multi,
     paged_attention_prefill_chunk,
     paged_attention_prefill_chunk_fp8,
     reshape_and_cache,
     reshape_and_cache_fp8,
+    set_wait_limit_ns,
+    DEFAULT_WAIT_LIMIT_NS,
     swap_blocks,
 )

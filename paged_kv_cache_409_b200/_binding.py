@@ -36,6 +36,8 @@ EXPORTED = (
     "pkv_swap_blocks",
     "pkv_paged_attention_decode",
     "pkv_paged_attention_decode_fp8",
+    "pkv_paged_attention_decode_step",
+    "pkv_paged_attention_decode_step_fp8",
     "pkv_paged_attention_decode_static_scratch",
     "pkv_decode_workspace_size",
     "pkv_decode_partition_size",
@@ -45,6 +47,7 @@ EXPORTED = (
     "pkv_paged_attention_decode_multi",
     "pkv_decode_multi_partition_size",
     "pkv_get_device_error",
+    "pkv_set_wait_limit_ns",
 )
 
 
@@ -93,11 +96,17 @@ def load_library():
     lib.pkv_prefill_fp8_workspace_size.argtypes = [I, I, I, I, I, I64, I, I]
     lib.pkv_prefill_fp8_workspace_size.restype = SZ
     lib.pkv_get_device_error.argtypes = [ctypes.POINTER(ctypes.c_uint32), P]
+    lib.pkv_paged_attention_decode_step.argtypes = [P, P, P, I64, P, P, P, P, P, P, F, I, I, I, I, I, I, I64, I, I,
+                                                    I, P, SZ, P]
+    lib.pkv_paged_attention_decode_step_fp8.argtypes = [P, P, P, I64, P, P, P, P, P, P, F, F, F, I, I, I, I, I, I,
+                                                        I64, I, I, I, P, SZ, P]
+    lib.pkv_set_wait_limit_ns.argtypes = [ctypes.c_uint64]
     for name in ("pkv_reshape_and_cache", "pkv_reshape_and_cache_fp8", "pkv_paged_attention_decode_fp8",
                  "pkv_copy_blocks", "pkv_swap_blocks", "pkv_paged_attention_decode",
                  "pkv_decode_partition_size", "pkv_paged_attention_prefill_chunk", "pkv_get_device_error",
                  "pkv_paged_attention_prefill_chunk_fp8", "pkv_paged_attention_decode_multi",
-                 "pkv_decode_multi_partition_size"):
+                 "pkv_decode_multi_partition_size", "pkv_paged_attention_decode_step",
+                 "pkv_paged_attention_decode_step_fp8", "pkv_set_wait_limit_ns"):
         getattr(lib, name).restype = I
     _lib = lib
     return lib
@@ -274,6 +283,82 @@ def paged_attention_decode_fp8(out, query, key_cache, value_cache, block_tables,
                                             int(partition_size), _code(query), ws_ptr, ws_bytes, _stream(stream))
     _ok(rc, "paged_attention_decode_fp8")
     return out
+
+
+def _decode_workspace(S, Hq, Hkv, D, B, max_context_len, dtype_code, partition_size, workspace, device,
+                      total_context_tokens):
+    """(partition_size, workspace pointer, workspace bytes) of a decode call; allocates a workspace when one
+    is needed and none (or too small a one) is given."""
+    if partition_size is None:
+        partition_size = decode_partition_size(S, Hq, Hkv, D, B, max_context_len, dtype_code, total_context_tokens)
+    need = decode_workspace_size(S, Hq, D, max_context_len, partition_size) if partition_size else 0
+    if need and (workspace is None or workspace.numel() * workspace.element_size() < need):
+        workspace = torch.empty(need, dtype=torch.uint8, device=device)
+    ws_ptr = _dev(workspace, "workspace") if (need and workspace is not None) else None
+    ws_bytes = workspace.numel() * workspace.element_size() if ws_ptr else 0
+    return int(partition_size), ws_ptr, ws_bytes
+
+
+def paged_attention_decode_step(new_keys, new_values, slot_mapping, out, query, key_cache, value_cache, block_tables,
+                                context_lens, scale, max_context_len, partition_size=None, workspace=None,
+                                stream=None, total_context_tokens=0):
+    """One decode step: ``reshape_and_cache(new_keys, new_values, ..., slot_mapping)`` then
+    ``paged_attention_decode`` in one call (the decode launched as the append's programmatic dependent)."""
+    lib = load_library()
+    S, Hq, D = query.shape
+    NB, B, Hkv, _ = key_cache.shape
+    MB = block_tables.shape[1] if block_tables.dim() == 2 else 1
+    if block_tables.dtype != torch.int32 or context_lens.dtype != torch.int32:
+        raise ValueError("block_tables and context_lens must be int32")
+    if slot_mapping.dtype != torch.int64:
+        raise ValueError("slot_mapping must be int64")
+    part, ws_ptr, ws_bytes = _decode_workspace(S, Hq, Hkv, D, B, max_context_len, _code(query), partition_size,
+                                               workspace, query.device, total_context_tokens)
+    rc = lib.pkv_paged_attention_decode_step(_dev(new_keys, "new_keys"), _dev(new_values, "new_values"),
+                                             _dev(slot_mapping, "slot_mapping"), new_keys.shape[0], _dev(out, "out"),
+                                             _dev(query, "query"), _dev(key_cache, "key_cache"),
+                                             _dev(value_cache, "value_cache"), _dev(block_tables, "block_tables"),
+                                             _dev(context_lens, "context_lens"), float(scale), S, Hq, Hkv, D, B, MB,
+                                             NB, int(max_context_len), part, _code(query), ws_ptr, ws_bytes,
+                                             _stream(stream))
+    _ok(rc, "paged_attention_decode_step")
+    return out
+
+
+def paged_attention_decode_step_fp8(new_keys, new_values, slot_mapping, out, query, key_cache, value_cache,
+                                    block_tables, context_lens, scale, k_scale, v_scale, max_context_len,
+                                    partition_size=None, workspace=None, stream=None, total_context_tokens=0):
+    """The decode step over E4M3 pools: ``reshape_and_cache_fp8`` then ``paged_attention_decode_fp8``."""
+    lib = load_library()
+    S, Hq, D = query.shape
+    NB, B, Hkv, _ = key_cache.shape
+    MB = block_tables.shape[1] if block_tables.dim() == 2 else 1
+    if block_tables.dtype != torch.int32 or context_lens.dtype != torch.int32:
+        raise ValueError("block_tables and context_lens must be int32")
+    if slot_mapping.dtype != torch.int64:
+        raise ValueError("slot_mapping must be int64")
+    part, ws_ptr, ws_bytes = _decode_workspace(S, Hq, Hkv, D, B, max_context_len, FP8_E4M3, partition_size,
+                                               workspace, query.device, total_context_tokens)
+    rc = lib.pkv_paged_attention_decode_step_fp8(_dev(new_keys, "new_keys"), _dev(new_values, "new_values"),
+                                                 _dev(slot_mapping, "slot_mapping"), new_keys.shape[0],
+                                                 _dev(out, "out"), _dev(query, "query"),
+                                                 _fp8_pool(key_cache, "key_cache"),
+                                                 _fp8_pool(value_cache, "value_cache"),
+                                                 _dev(block_tables, "block_tables"),
+                                                 _dev(context_lens, "context_lens"), float(scale), float(k_scale),
+                                                 float(v_scale), S, Hq, Hkv, D, B, MB, NB, int(max_context_len), part,
+                                                 _code(query), ws_ptr, ws_bytes, _stream(stream))
+    _ok(rc, "paged_attention_decode_step_fp8")
+    return out
+
+
+def set_wait_limit_ns(limit_ns: int):
+    """Limit of the kernels' main-loop waits for later launches (0 = give up at the first blocking wait; a
+    test setting).  The default is one second."""
+    _ok(load_library().pkv_set_wait_limit_ns(int(limit_ns)), "set_wait_limit_ns")
+
+
+DEFAULT_WAIT_LIMIT_NS = 1_000_000_000
 
 
 def paged_attention_prefill_chunk(out, query, key_cache, value_cache, block_tables, seq_lens, query_start_loc,

@@ -195,6 +195,10 @@ __global__ void __launch_bounds__(NW * 32) paged_decode_kernel(const DecodeParam
         }
     };
 
+    // Everything above reads only the query, the tables and the lengths; the
+    // pools may still be in the writes of a grid this one depends on (the
+    // append of a decode step), so their loads start after it completes.
+    griddep_wait();
     if (lane == 0) {
         for (int k = 0; k < NST && k < nw; ++k) issue(k);
     }
@@ -219,7 +223,7 @@ __global__ void __launch_bounds__(NW * 32) paged_decode_kernel(const DecodeParam
     int k = 0;
     for (; k < nw; ++k) {
         const int st = k % NST;
-        const bool ok = mbar_wait(&wbar[st], (k / NST) & 1);
+        const bool ok = mbar_wait_main(&wbar[st], (k / NST) & 1);
         if (!__all_sync(0xffffffffu, ok)) break;
         const int lb = b0 + warp + k * kDecodeWarps;
         const int valid = min(B, ctx - lb * B);
@@ -313,7 +317,8 @@ __global__ void __launch_bounds__(NW * 32) paged_decode_kernel(const DecodeParam
     if (k < nw && lane == 0) {
         // A wait gave up: wait (bounded) for the copies still in flight before
         // the stage buffers are reused, then drop this warp's partial state.
-        for (int kk = k + 1; kk < min(nw, k + NST); ++kk) mbar_wait(&wbar[kk % NST], (kk / NST) & 1);
+        // a wait gave up: wait (bounded) for this warp's copies still in flight, stage k's included
+        for (int kk = k; kk < min(nw, k + NST); ++kk) mbar_wait(&wbar[kk % NST], (kk / NST) & 1);
     }
     if (k < nw) {
 #pragma unroll
@@ -366,6 +371,7 @@ __global__ void __launch_bounds__(128) paged_decode_merge_kernel(const MergePara
                                        p.num_partitions * p.partition_blocks, false);
     const int nparts = nblk > 0 ? (nblk + p.partition_blocks - 1) / p.partition_blocks : 1;
     if (nparts <= 1) return;  // the decode kernel wrote this row itself
+    griddep_wait();           // the partials are the writes of the decode grid
     const float* pm = p.ws_max + static_cast<int64_t>(wid) * p.num_partitions;
     const float* pl = p.ws_sum + static_cast<int64_t>(wid) * p.num_partitions;
     const float* po = p.ws_out + static_cast<int64_t>(wid) * p.num_partitions * D;

@@ -123,6 +123,10 @@ __global__ void __launch_bounds__(NW * 32) paged_decode_fp8_kernel(const DecodeP
         tma_load_4d_hint(kd, &tm_k, 0, g, 0, coord, &wbar[st], policy);
         tma_load_4d_hint(kd + C::TILE, &tm_v, 0, g, 0, coord, &wbar[st], policy);
     };
+    // Everything above reads only the query, the tables and the lengths; the
+    // pools may still be in the writes of a grid this one depends on (the
+    // append of a decode step), so their loads start after it completes.
+    griddep_wait();
     if (lane == 0) {
         for (int k = 0; k < NST && k < nw; ++k) issue(k);
     }
@@ -139,7 +143,7 @@ __global__ void __launch_bounds__(NW * 32) paged_decode_fp8_kernel(const DecodeP
     int k = 0;
     for (; k < nw; ++k) {
         const int st = k % NST;
-        const bool ok = mbar_wait(&wbar[st], (k / NST) & 1);
+        const bool ok = mbar_wait_main(&wbar[st], (k / NST) & 1);
         if (!__all_sync(0xffffffffu, ok)) break;
         const int lb = b0 + warp + k * NW;
         const int valid = min(B, ctx - lb * B);
@@ -272,7 +276,8 @@ __global__ void __launch_bounds__(NW * 32) paged_decode_fp8_kernel(const DecodeP
         }
     }
     if (k < nw && lane == 0) {
-        for (int kk = k + 1; kk < min(nw, k + NST); ++kk) mbar_wait(&wbar[kk % NST], (kk / NST) & 1);
+        // a wait gave up: wait (bounded) for this warp's copies still in flight, stage k's included
+        for (int kk = k; kk < min(nw, k + NST); ++kk) mbar_wait(&wbar[kk % NST], (kk / NST) & 1);
     }
     if (k < nw) mA = mB = -INFINITY, lA = lB = 0.f;
 

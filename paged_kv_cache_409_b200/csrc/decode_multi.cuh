@@ -177,6 +177,7 @@ __global__ void __launch_bounds__(NW * 32) paged_decode_multi_kernel(const Multi
         }
     };
     int issued = 0;
+    griddep_wait();  // the pools may still be in the writes of a grid this one depends on
     if (lane == 0 && producer) {
         for (; issued < ring && issued < nw; ++issued) issue(issued);
     }
@@ -191,7 +192,7 @@ __global__ void __launch_bounds__(NW * 32) paged_decode_multi_kernel(const Multi
     int k = 0;
     for (; k < nw; ++k) {
         const int st = k % ring;
-        const bool ok = mbar_wait(&fbar[st], (k / ring) & 1);
+        const bool ok = mbar_wait_main(&fbar[st], (k / ring) & 1);
         if (!__all_sync(0xffffffffu, ok)) break;
         const int u = stream + k * nsw;
         const int pos0 = (b0 + u / C::UPB) * B + (u % C::UPB) * UT;  // key position of the unit's first token
@@ -323,7 +324,7 @@ __global__ void __launch_bounds__(NW * 32) paged_decode_multi_kernel(const Multi
             if (nrg > 1) mbar_arrive(&ebar[st]);
             if (producer && k + ring < nw) {
                 // the stage is refilled once every reader released unit k
-                go = nrg == 1 || mbar_wait(&ebar[st], (k / ring) & 1);
+                go = nrg == 1 || mbar_wait_main(&ebar[st], (k / ring) & 1);
                 if (go) {
                     fence_proxy_async();
                     issue(k + ring);
@@ -430,6 +431,7 @@ __global__ void __launch_bounds__(128) paged_decode_multi_merge_kernel(const Mul
                                        p.num_partitions * p.partition_blocks, false);
     const int nparts = nblk > 0 ? (nblk + p.partition_blocks - 1) / p.partition_blocks : 1;
     if (nparts <= 1) return;  // the attention kernel wrote this row itself
+    griddep_wait();           // the partials are the writes of the attention grid
     const float* pm = p.ws_max + wid * p.num_partitions;
     const float* pl = p.ws_sum + wid * p.num_partitions;
     const float* po = p.ws_out + wid * p.num_partitions * D;

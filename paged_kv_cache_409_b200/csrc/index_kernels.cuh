@@ -22,6 +22,9 @@ __global__ void __launch_bounds__(128) reshape_and_cache_kernel(const uint4* __r
                                                                 const int64_t* __restrict__ slot_mapping,
                                                                 int64_t num_tokens, int row_vecs,
                                                                 int64_t num_slots) {
+    // A decode launched as this grid's programmatic dependent may start its
+    // prologue now; it waits for this grid's writes before it reads the pools.
+    griddep_launch_dependents();
     const int i = blockIdx.x * blockDim.x + threadIdx.x;
     for (int64_t t = blockIdx.y; t < num_tokens; t += gridDim.y) {
         const int64_t slot = slot_mapping[t];
@@ -88,6 +91,7 @@ __global__ void __launch_bounds__(128) reshape_and_cache_fp8_kernel(const TS* __
                                                                     const int64_t* __restrict__ slot_mapping,
                                                                     int64_t num_tokens, int row_elems,
                                                                     int64_t num_slots, float k_scale, float v_scale) {
+    griddep_launch_dependents();  // as in reshape_and_cache_kernel
     const int groups = row_elems / 8;
     const int i = blockIdx.x * blockDim.x + threadIdx.x;
     for (int64_t t = blockIdx.y; t < num_tokens; t += gridDim.y) {

@@ -173,6 +173,33 @@ int check_tables(const int32_t* d_bt, const int32_t* d_lens, int num_seqs, int m
     return PKV_OK;
 }
 
+// ------------------------------------------------------------ launches
+// Stream of a launch and whether the kernel may start as a programmatic
+// dependent of the kernel before it in the stream (its prologue overlapping
+// that kernel's tail; the kernel waits with griddepcontrol.wait before it
+// touches what that kernel writes).
+struct Launch {
+    cudaStream_t s;
+    bool pdl;
+};
+
+template <typename... KArgs, typename... Args>
+int launch_kernel(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, const Launch& ln, Args&&... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = ln.s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = ln.pdl ? 1 : 0;
+    PKV_CUDA(cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...));
+    PKV_CUDA(cudaGetLastError());
+    return PKV_OK;
+}
+
 // ------------------------------------------------------------ decode dispatch
 // Launch shape of the decode kernels, from a sweep on B200 of warps per CTA x
 // stages per warp at equal shared memory: 8 KB stages (block 16, 16-bit,
@@ -193,7 +220,7 @@ constexpr int pick_stages(int stage_bytes, int warps) {
 
 template <typename Kern>
 int launch_decode_kernel(Kern kern, size_t smem, int threads, const pkv::DecodeParams& prm, const CUtensorMap& tk,
-                         const CUtensorMap& tv, int grid, cudaStream_t s, size_t* configured) {
+                         const CUtensorMap& tv, int grid, const Launch& ln, size_t* configured) {
     int dev = 0;
     PKV_CUDA(cudaGetDevice(&dev));
     size_t& have = configured[dev & 63];  // largest dynamic smem size set so far on this device
@@ -201,14 +228,12 @@ int launch_decode_kernel(Kern kern, size_t smem, int threads, const pkv::DecodeP
         PKV_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
         have = smem;
     }
-    kern<<<grid, threads, smem, s>>>(prm, tk, tv);
-    PKV_CUDA(cudaGetLastError());
-    return PKV_OK;
+    return launch_kernel(kern, dim3(grid), dim3(threads), smem, ln, prm, tk, tv);
 }
 
 template <typename T, int D, int B, int G>
 int launch_decode(const pkv::DecodeParams& prm, const CUtensorMap& tk, const CUtensorMap& tv, int grid,
-                  cudaStream_t s) {
+                  const Launch& ln) {
     constexpr int STAGE = 2 * B * D * pkv::Elem<T>::kBytes;
 #ifdef PKV_DECODE_WARPS
     constexpr int NW = PKV_DECODE_WARPS;
@@ -227,41 +252,41 @@ int launch_decode(const pkv::DecodeParams& prm, const CUtensorMap& tk, const CUt
 #endif
     if constexpr (sizeof(T) == 2 && G >= PKV_DECODE_MMA_MIN_G)
         return launch_decode_kernel(pkv::paged_decode_mma_kernel<T, D, B, G, NST, NW>, smem, NW * 32, prm, tk, tv,
-                                    grid, s, configured);
+                                    grid, ln, configured);
     else
         return launch_decode_kernel(pkv::paged_decode_kernel<T, D, B, G, NST, NW>, smem, NW * 32, prm, tk, tv,
-                                    grid, s, configured);
+                                    grid, ln, configured);
 }
 
 template <typename T, int D, int B>
 int decode_by_group(int group, const pkv::DecodeParams& prm, const CUtensorMap& tk, const CUtensorMap& tv,
-                    int grid, cudaStream_t s) {
+                    int grid, const Launch& ln) {
     switch (group) {
-        case 1: return launch_decode<T, D, B, 1>(prm, tk, tv, grid, s);
-        case 2: return launch_decode<T, D, B, 2>(prm, tk, tv, grid, s);
-        case 4: return launch_decode<T, D, B, 4>(prm, tk, tv, grid, s);
-        case 8: return launch_decode<T, D, B, 8>(prm, tk, tv, grid, s);
+        case 1: return launch_decode<T, D, B, 1>(prm, tk, tv, grid, ln);
+        case 2: return launch_decode<T, D, B, 2>(prm, tk, tv, grid, ln);
+        case 4: return launch_decode<T, D, B, 4>(prm, tk, tv, grid, ln);
+        case 8: return launch_decode<T, D, B, 8>(prm, tk, tv, grid, ln);
         default: return PKV_EUNSUPPORTED;
     }
 }
 
 template <typename T, int D>
 int decode_by_block(int block_size, int group, const pkv::DecodeParams& prm, const CUtensorMap& tk,
-                    const CUtensorMap& tv, int grid, cudaStream_t s) {
+                    const CUtensorMap& tv, int grid, const Launch& ln) {
     switch (block_size) {
-        case 8: return decode_by_group<T, D, 8>(group, prm, tk, tv, grid, s);
-        case 16: return decode_by_group<T, D, 16>(group, prm, tk, tv, grid, s);
-        case 32: return decode_by_group<T, D, 32>(group, prm, tk, tv, grid, s);
+        case 8: return decode_by_group<T, D, 8>(group, prm, tk, tv, grid, ln);
+        case 16: return decode_by_group<T, D, 16>(group, prm, tk, tv, grid, ln);
+        case 32: return decode_by_group<T, D, 32>(group, prm, tk, tv, grid, ln);
         default: return PKV_EUNSUPPORTED;
     }
 }
 
 template <typename T>
 int decode_by_dim(int head_dim, int block_size, int group, const pkv::DecodeParams& prm, const CUtensorMap& tk,
-                  const CUtensorMap& tv, int grid, cudaStream_t s) {
+                  const CUtensorMap& tv, int grid, const Launch& ln) {
     switch (head_dim) {
-        case 64: return decode_by_block<T, 64>(block_size, group, prm, tk, tv, grid, s);
-        case 128: return decode_by_block<T, 128>(block_size, group, prm, tk, tv, grid, s);
+        case 64: return decode_by_block<T, 64>(block_size, group, prm, tk, tv, grid, ln);
+        case 128: return decode_by_block<T, 128>(block_size, group, prm, tk, tv, grid, ln);
         default: return PKV_EUNSUPPORTED;
     }
 }
@@ -275,35 +300,35 @@ int decode_by_dim(int head_dim, int block_size, int group, const pkv::DecodePara
 
 template <typename T, int B, int G>
 int launch_decode_fp8(const pkv::DecodeParams& prm, const CUtensorMap& tk, const CUtensorMap& tv, int grid,
-                      cudaStream_t s) {
+                      const Launch& ln) {
     constexpr int STAGE = 2 * B * 128;
     constexpr int NW = PKV_FP8_WARPS;
     constexpr int NST = std::max(1, std::min(8, PKV_FP8_STAGE_BUDGET / (NW * STAGE)));
     using C = pkv::DecodeFp8Cfg<B, G, NST, NW>;
     static size_t configured[64] = {};
     return launch_decode_kernel(pkv::paged_decode_fp8_kernel<T, B, G, NST, NW>, C::smem_bytes(prm.partition_blocks),
-                                NW * 32, prm, tk, tv, grid, s, configured);
+                                NW * 32, prm, tk, tv, grid, ln, configured);
 }
 
 template <typename T, int B>
 int decode_fp8_by_group(int group, const pkv::DecodeParams& prm, const CUtensorMap& tk, const CUtensorMap& tv,
-                        int grid, cudaStream_t s) {
+                        int grid, const Launch& ln) {
     switch (group) {
-        case 1: return launch_decode_fp8<T, B, 1>(prm, tk, tv, grid, s);
-        case 2: return launch_decode_fp8<T, B, 2>(prm, tk, tv, grid, s);
-        case 4: return launch_decode_fp8<T, B, 4>(prm, tk, tv, grid, s);
-        case 8: return launch_decode_fp8<T, B, 8>(prm, tk, tv, grid, s);
+        case 1: return launch_decode_fp8<T, B, 1>(prm, tk, tv, grid, ln);
+        case 2: return launch_decode_fp8<T, B, 2>(prm, tk, tv, grid, ln);
+        case 4: return launch_decode_fp8<T, B, 4>(prm, tk, tv, grid, ln);
+        case 8: return launch_decode_fp8<T, B, 8>(prm, tk, tv, grid, ln);
         default: return PKV_EUNSUPPORTED;
     }
 }
 
 template <typename T>
 int decode_fp8_by_block(int block_size, int group, const pkv::DecodeParams& prm, const CUtensorMap& tk,
-                        const CUtensorMap& tv, int grid, cudaStream_t s) {
+                        const CUtensorMap& tv, int grid, const Launch& ln) {
     switch (block_size) {
-        case 8: return decode_fp8_by_group<T, 8>(group, prm, tk, tv, grid, s);
-        case 16: return decode_fp8_by_group<T, 16>(group, prm, tk, tv, grid, s);
-        case 32: return decode_fp8_by_group<T, 32>(group, prm, tk, tv, grid, s);
+        case 8: return decode_fp8_by_group<T, 8>(group, prm, tk, tv, grid, ln);
+        case 16: return decode_fp8_by_group<T, 16>(group, prm, tk, tv, grid, ln);
+        case 32: return decode_fp8_by_group<T, 32>(group, prm, tk, tv, grid, ln);
         default: return PKV_EUNSUPPORTED;
     }
 }
@@ -354,16 +379,16 @@ int multi_by_block(int block_size, int row_groups, const pkv::MultiParams& prm, 
     }
 }
 
+// The merge always follows this library's own decode kernel in the stream,
+// so it is launched as that kernel's programmatic dependent (it waits for the
+// partials before it reads them).
 template <typename T>
 int launch_merge(int head_dim, const pkv::MergeParams& mp, cudaStream_t s) {
     const int warps = mp.num_seqs * mp.num_q_heads;
     const int grid = (warps + 3) / 4;
-    if (head_dim == 64)
-        pkv::paged_decode_merge_kernel<T, 64><<<grid, 128, 0, s>>>(mp);
-    else
-        pkv::paged_decode_merge_kernel<T, 128><<<grid, 128, 0, s>>>(mp);
-    PKV_CUDA(cudaGetLastError());
-    return PKV_OK;
+    const Launch ln{s, true};
+    if (head_dim == 64) return launch_kernel(pkv::paged_decode_merge_kernel<T, 64>, dim3(grid), dim3(128), 0, ln, mp);
+    return launch_kernel(pkv::paged_decode_merge_kernel<T, 128>, dim3(grid), dim3(128), 0, ln, mp);
 }
 
 bool supported_group(int g) { return g == 1 || g == 2 || g == 4 || g == 8; }
@@ -436,13 +461,61 @@ int decode_check(const void* out, const void* query, const void* key_cache, cons
     return PKV_OK;
 }
 
+// The workspace and grid checks of the decode (arguments already passed
+// decode_check): PKV_EWORKSPACE when the split-K partials do not fit.
+int decode_workspace_check(int num_seqs, int num_q_heads, int num_kv_heads, int head_dim, int block_size,
+                           int max_context_len, int partition_size, const void* workspace, size_t workspace_bytes) {
+    if (num_seqs == 0) return PKV_OK;
+    const int64_t max_blocks_needed = std::max<int64_t>(1, ceil_div(std::max(max_context_len, 1), block_size));
+    const int64_t pb = std::min<int64_t>(partition_size > 0 ? partition_size / block_size : max_blocks_needed,
+                                         max_blocks_needed);
+    const int64_t parts = ceil_div(max_blocks_needed, pb);
+    const size_t need = parts > 1 ? pkv_decode_workspace_size(num_seqs, num_q_heads, head_dim, max_context_len,
+                                                              (int)(pb * block_size))
+                                  : 0;
+    if (need > 0 && (!workspace || workspace_bytes < need || !aligned16(workspace))) return PKV_EWORKSPACE;
+    if ((int64_t)num_seqs * parts * num_kv_heads > INT32_MAX) return PKV_EUNSUPPORTED;
+    return PKV_OK;
+}
+
+// Argument checks of the appends (16/32-bit pools, and E4M3 pools written
+// from `dtype`): the status the append returns, or PKV_OK (also for
+// num_tokens == 0, which launches nothing).
+int reshape_check(const void* key, const void* value, const void* key_cache, const void* value_cache,
+                  const int64_t* slot_mapping, int64_t num_tokens, int num_kv_heads, int head_dim, int block_size,
+                  int64_t num_blocks, int dtype, bool fp8) {
+    if (fp8 ? !query_type(dtype) : !elem_bytes(dtype)) return PKV_EUNSUPPORTED;
+    if (num_tokens < 0 || num_kv_heads <= 0 || head_dim <= 0 || block_size <= 0 || num_blocks <= 0)
+        return PKV_EINVAL;
+    const int64_t row_elems = (int64_t)num_kv_heads * head_dim;
+    if (fp8) {
+        if (row_elems % 16 != 0 || row_elems > INT32_MAX) return PKV_EUNSUPPORTED;
+    } else {
+        const int64_t row_bytes = row_elems * elem_bytes(dtype);
+        if (row_bytes % 16 != 0 || row_bytes / 16 > INT32_MAX) return PKV_EUNSUPPORTED;
+    }
+    if (num_tokens == 0) return PKV_OK;
+    if (!key || !value || !key_cache || !value_cache || !slot_mapping) return PKV_EINVAL;
+    if (!aligned16(key) || !aligned16(value) || !aligned16(key_cache) || !aligned16(value_cache) ||
+        (reinterpret_cast<uintptr_t>(slot_mapping) & 7))
+        return PKV_EINVAL;
+    return PKV_OK;
+}
+
+int reshape_fp8_check(const void* key, const void* value, const void* key_cache, const void* value_cache,
+                      const int64_t* slot_mapping, int64_t num_tokens, int num_kv_heads, int head_dim, int block_size,
+                      int64_t num_blocks, int src_dtype) {
+    return reshape_check(key, value, key_cache, value_cache, slot_mapping, num_tokens, num_kv_heads, head_dim,
+                         block_size, num_blocks, src_dtype, true);
+}
+
 // Decode with the query / output in `dtype` and the pools in `kv_dtype`
 // (the same 16/32-bit type, or FP8 E4M3 with its two scales).
 int decode_impl(void* out, const void* query, const void* key_cache, const void* value_cache,
                 const int32_t* block_tables, const int32_t* context_lens, float scale, int num_seqs, int num_q_heads,
                 int num_kv_heads, int head_dim, int block_size, int max_blocks_per_seq, int64_t num_blocks,
                 int max_context_len, int partition_size, int dtype, int kv_dtype, float k_scale, float v_scale,
-                void* workspace, size_t workspace_bytes, pkv_stream_t stream) {
+                void* workspace, size_t workspace_bytes, pkv_stream_t stream, bool pdl = false) {
     const int check = decode_check(out, query, key_cache, value_cache, block_tables, context_lens, scale, num_seqs,
                                    num_q_heads, num_kv_heads, head_dim, block_size, max_blocks_per_seq, num_blocks,
                                    max_context_len, partition_size, dtype, kv_dtype);
@@ -451,6 +524,9 @@ int decode_impl(void* out, const void* query, const void* key_cache, const void*
     const int group = num_q_heads / num_kv_heads;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
 
+    const int wcheck = decode_workspace_check(num_seqs, num_q_heads, num_kv_heads, head_dim, block_size,
+                                              max_context_len, partition_size, workspace, workspace_bytes);
+    if (wcheck) return wcheck;
     const int64_t max_blocks_needed = std::max<int64_t>(1, ceil_div(std::max(max_context_len, 1), block_size));
     int64_t pb = partition_size > 0 ? partition_size / block_size : max_blocks_needed;
     pb = std::min(pb, max_blocks_needed);
@@ -458,9 +534,7 @@ int decode_impl(void* out, const void* query, const void* key_cache, const void*
     const size_t need = parts > 1 ? pkv_decode_workspace_size(num_seqs, num_q_heads, head_dim, max_context_len,
                                                               (int)(pb * block_size))
                                   : 0;
-    if (need > 0 && (!workspace || workspace_bytes < need || !aligned16(workspace))) return PKV_EWORKSPACE;
     const int64_t grid = (int64_t)num_seqs * parts * num_kv_heads;
-    if (grid > INT32_MAX) return PKV_EUNSUPPORTED;
 
     if (checked_mode()) {
         int rc = check_tables(block_tables, context_lens, num_seqs, max_blocks_per_seq, block_size, num_blocks,
@@ -494,15 +568,16 @@ int decode_impl(void* out, const void* query, const void* key_cache, const void*
     prm.partition_blocks = (int)pb;
     prm.num_partitions = (int)parts;
 
+    const Launch ln{s, pdl};
     if (fp8) {
-        rc = dtype == PKV_F16 ? decode_fp8_by_block<__half>(block_size, group, prm, tk, tv, (int)grid, s)
-                              : decode_fp8_by_block<__nv_bfloat16>(block_size, group, prm, tk, tv, (int)grid, s);
+        rc = dtype == PKV_F16 ? decode_fp8_by_block<__half>(block_size, group, prm, tk, tv, (int)grid, ln)
+                              : decode_fp8_by_block<__nv_bfloat16>(block_size, group, prm, tk, tv, (int)grid, ln);
     } else {
         switch (dtype) {
-            case PKV_F32: rc = decode_by_dim<float>(head_dim, block_size, group, prm, tk, tv, (int)grid, s); break;
-            case PKV_F16: rc = decode_by_dim<__half>(head_dim, block_size, group, prm, tk, tv, (int)grid, s); break;
+            case PKV_F32: rc = decode_by_dim<float>(head_dim, block_size, group, prm, tk, tv, (int)grid, ln); break;
+            case PKV_F16: rc = decode_by_dim<__half>(head_dim, block_size, group, prm, tk, tv, (int)grid, ln); break;
             default:
-                rc = decode_by_dim<__nv_bfloat16>(head_dim, block_size, group, prm, tk, tv, (int)grid, s);
+                rc = decode_by_dim<__nv_bfloat16>(head_dim, block_size, group, prm, tk, tv, (int)grid, ln);
                 break;
         }
     }
@@ -549,17 +624,10 @@ const char* pkv_last_cuda_error(void) { return g_last_cuda_error; }
 int pkv_reshape_and_cache(const void* key, const void* value, void* key_cache, void* value_cache,
                           const int64_t* slot_mapping, int64_t num_tokens, int num_kv_heads, int head_dim,
                           int block_size, int64_t num_blocks, int dtype, pkv_stream_t stream) {
-    const int eb = elem_bytes(dtype);
-    if (!eb) return PKV_EUNSUPPORTED;
-    if (num_tokens < 0 || num_kv_heads <= 0 || head_dim <= 0 || block_size <= 0 || num_blocks <= 0)
-        return PKV_EINVAL;
-    const int64_t row_bytes = (int64_t)num_kv_heads * head_dim * eb;
-    if (row_bytes % 16 != 0 || row_bytes / 16 > INT32_MAX) return PKV_EUNSUPPORTED;
-    if (num_tokens == 0) return PKV_OK;
-    if (!key || !value || !key_cache || !value_cache || !slot_mapping) return PKV_EINVAL;
-    if (!aligned16(key) || !aligned16(value) || !aligned16(key_cache) || !aligned16(value_cache) ||
-        (reinterpret_cast<uintptr_t>(slot_mapping) & 7))
-        return PKV_EINVAL;
+    const int check = reshape_check(key, value, key_cache, value_cache, slot_mapping, num_tokens, num_kv_heads,
+                                    head_dim, block_size, num_blocks, dtype, false);
+    if (check || num_tokens == 0) return check;
+    const int64_t row_bytes = (int64_t)num_kv_heads * head_dim * elem_bytes(dtype);
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     const int64_t num_slots = num_blocks * block_size;
     if (checked_mode()) {
@@ -586,13 +654,10 @@ int pkv_reshape_and_cache_fp8(const void* key, const void* value, void* key_cach
     if (num_tokens < 0 || num_kv_heads <= 0 || head_dim <= 0 || block_size <= 0 || num_blocks <= 0)
         return PKV_EINVAL;
     if (!(std::isfinite(k_scale) && k_scale > 0.f && std::isfinite(v_scale) && v_scale > 0.f)) return PKV_EINVAL;
+    const int check = reshape_fp8_check(key, value, key_cache, value_cache, slot_mapping, num_tokens, num_kv_heads,
+                                        head_dim, block_size, num_blocks, src_dtype);
+    if (check || num_tokens == 0) return check;
     const int64_t row_elems = (int64_t)num_kv_heads * head_dim;
-    if (row_elems % 16 != 0 || row_elems > INT32_MAX) return PKV_EUNSUPPORTED;
-    if (num_tokens == 0) return PKV_OK;
-    if (!key || !value || !key_cache || !value_cache || !slot_mapping) return PKV_EINVAL;
-    if (!aligned16(key) || !aligned16(value) || !aligned16(key_cache) || !aligned16(value_cache) ||
-        (reinterpret_cast<uintptr_t>(slot_mapping) & 7))
-        return PKV_EINVAL;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     const int64_t num_slots = num_blocks * block_size;
     if (checked_mode()) {
@@ -788,6 +853,68 @@ int pkv_paged_attention_decode_fp8(void* out, const void* query, const void* key
                        partition_size, dtype, PKV_FP8_E4M3, k_scale, v_scale, workspace, workspace_bytes, stream);
 }
 
+int pkv_paged_attention_decode_step(const void* new_keys, const void* new_values, const int64_t* slot_mapping,
+                                    int64_t num_new_tokens, void* out, const void* query, void* key_cache,
+                                    void* value_cache, const int32_t* block_tables, const int32_t* context_lens,
+                                    float scale, int num_seqs, int num_q_heads, int num_kv_heads, int head_dim,
+                                    int block_size, int max_blocks_per_seq, int64_t num_blocks, int max_context_len,
+                                    int partition_size, int dtype, void* workspace, size_t workspace_bytes,
+                                    pkv_stream_t stream) {
+    // Every check of both calls before the first launch, so that a refused
+    // step has changed nothing.
+    int rc = decode_check(out, query, key_cache, value_cache, block_tables, context_lens, scale, num_seqs,
+                          num_q_heads, num_kv_heads, head_dim, block_size, max_blocks_per_seq, num_blocks,
+                          max_context_len, partition_size, dtype, dtype);
+    if (rc) return rc;
+    rc = decode_workspace_check(num_seqs, num_q_heads, num_kv_heads, head_dim, block_size, max_context_len,
+                                partition_size, workspace, workspace_bytes);
+    if (rc) return rc;
+    rc = reshape_check(new_keys, new_values, key_cache, value_cache, slot_mapping, num_new_tokens, num_kv_heads,
+                       head_dim, block_size, num_blocks, dtype, false);
+    if (rc) return rc;
+    rc = pkv_reshape_and_cache(new_keys, new_values, key_cache, value_cache, slot_mapping, num_new_tokens,
+                               num_kv_heads, head_dim, block_size, num_blocks, dtype, stream);
+    if (rc) return rc;
+    return decode_impl(out, query, key_cache, value_cache, block_tables, context_lens, scale, num_seqs, num_q_heads,
+                       num_kv_heads, head_dim, block_size, max_blocks_per_seq, num_blocks, max_context_len,
+                       partition_size, dtype, dtype, 1.f, 1.f, workspace, workspace_bytes, stream,
+                       /*pdl=*/num_new_tokens > 0);
+}
+
+int pkv_paged_attention_decode_step_fp8(const void* new_keys, const void* new_values, const int64_t* slot_mapping,
+                                        int64_t num_new_tokens, void* out, const void* query, void* key_cache,
+                                        void* value_cache, const int32_t* block_tables, const int32_t* context_lens,
+                                        float scale, float k_scale, float v_scale, int num_seqs, int num_q_heads,
+                                        int num_kv_heads, int head_dim, int block_size, int max_blocks_per_seq,
+                                        int64_t num_blocks, int max_context_len, int partition_size, int dtype,
+                                        void* workspace, size_t workspace_bytes, pkv_stream_t stream) {
+    if (!(std::isfinite(k_scale) && k_scale > 0.f && std::isfinite(v_scale) && v_scale > 0.f)) return PKV_EINVAL;
+    int rc = decode_check(out, query, key_cache, value_cache, block_tables, context_lens, scale, num_seqs,
+                          num_q_heads, num_kv_heads, head_dim, block_size, max_blocks_per_seq, num_blocks,
+                          max_context_len, partition_size, dtype, PKV_FP8_E4M3);
+    if (rc) return rc;
+    rc = decode_workspace_check(num_seqs, num_q_heads, num_kv_heads, head_dim, block_size, max_context_len,
+                                partition_size, workspace, workspace_bytes);
+    if (rc) return rc;
+    rc = reshape_fp8_check(new_keys, new_values, key_cache, value_cache, slot_mapping, num_new_tokens, num_kv_heads,
+                           head_dim, block_size, num_blocks, dtype);
+    if (rc) return rc;
+    rc = pkv_reshape_and_cache_fp8(new_keys, new_values, key_cache, value_cache, slot_mapping, num_new_tokens,
+                                   num_kv_heads, head_dim, block_size, num_blocks, dtype, k_scale, v_scale, stream);
+    if (rc) return rc;
+    return decode_impl(out, query, key_cache, value_cache, block_tables, context_lens, scale, num_seqs, num_q_heads,
+                       num_kv_heads, head_dim, block_size, max_blocks_per_seq, num_blocks, max_context_len,
+                       partition_size, dtype, PKV_FP8_E4M3, k_scale, v_scale, workspace, workspace_bytes, stream,
+                       /*pdl=*/num_new_tokens > 0);
+}
+
+int pkv_set_wait_limit_ns(uint64_t limit_ns) {
+    PKV_CUDA(cudaDeviceSynchronize());
+    PKV_CUDA(cudaMemcpyToSymbol(pkv::c_main_wait_limit_ns, &limit_ns, sizeof limit_ns));
+    PKV_CUDA(cudaDeviceSynchronize());
+    return PKV_OK;
+}
+
 int pkv_paged_attention_prefill_chunk(void* out, const void* query, const void* key_cache, const void* value_cache,
                                       const int32_t* block_tables, const int32_t* seq_lens,
                                       const int32_t* query_start_loc, int num_chunks, int64_t total_q_tokens,
@@ -977,16 +1104,13 @@ int pkv_paged_attention_decode_multi(void* out, const void* query, const void* k
     mp.partition_blocks = (int)pb;
     mp.num_partitions = (int)parts;
     const int64_t warps = total_q_tokens * num_q_heads;
-    const int mgrid = (int)ceil_div(warps, 4);
-    if (head_dim == 64) {
-        if (bf16) pkv::paged_decode_multi_merge_kernel<__nv_bfloat16, 64><<<mgrid, 128, 0, s>>>(mp);
-        else pkv::paged_decode_multi_merge_kernel<__half, 64><<<mgrid, 128, 0, s>>>(mp);
-    } else {
-        if (bf16) pkv::paged_decode_multi_merge_kernel<__nv_bfloat16, 128><<<mgrid, 128, 0, s>>>(mp);
-        else pkv::paged_decode_multi_merge_kernel<__half, 128><<<mgrid, 128, 0, s>>>(mp);
-    }
-    PKV_CUDA(cudaGetLastError());
-    return PKV_OK;
+    const dim3 mgrid((unsigned)ceil_div(warps, 4));
+    const Launch ln{s, true};  // follows this library's own attention kernel (see launch_merge)
+    if (head_dim == 64)
+        return bf16 ? launch_kernel(pkv::paged_decode_multi_merge_kernel<__nv_bfloat16, 64>, mgrid, dim3(128), 0, ln, mp)
+                    : launch_kernel(pkv::paged_decode_multi_merge_kernel<__half, 64>, mgrid, dim3(128), 0, ln, mp);
+    return bf16 ? launch_kernel(pkv::paged_decode_multi_merge_kernel<__nv_bfloat16, 128>, mgrid, dim3(128), 0, ln, mp)
+                : launch_kernel(pkv::paged_decode_multi_merge_kernel<__half, 128>, mgrid, dim3(128), 0, ln, mp);
 }
 
 int pkv_decode_multi_partition_size(int num_chunks, int num_kv_heads, int block_size, int max_seq_len) {

@@ -218,8 +218,12 @@ __global__ void __launch_bounds__(kPrefillThreads, 1) paged_prefill_kernel(const
             loaded_v = j + 1;
             ids = ids_next;
         }
-        if (leader && *abort_flag) {
-            // wait (bounded) for this warp's copies still in flight
+        if (leader) {
+            // Wait (bounded) for this warp's last copies.  On the normal path
+            // their consumers already waited for them; after an abort (another
+            // role's wait gave up, perhaps after this loop ended) they may
+            // still be in flight and must land before the CTA exits.
+            mbar_wait(q_full, 0);
             for (int t = max(0, loaded_k - 2); t < loaded_k; ++t) mbar_wait(&k_full[t & 1], (t >> 1) & 1);
             for (int t = max(0, loaded_v - 2); t < loaded_v; ++t) mbar_wait(&v_full[t & 1], (t >> 1) & 1);
         }
@@ -277,11 +281,11 @@ __global__ void __launch_bounds__(kPrefillThreads, 1) paged_prefill_kernel(const
                 if (t + 1 < nkt) ok = issue_s(t + 1);
                 if (ok) ok = issue_pv(t);
             }
-            if (*abort_flag) {
-                // wait (bounded) for the MMAs this thread issued before tensor memory is released
-                if (ns > 0) mbar_wait(&s_full[(ns - 1) & 1], ((ns - 1) >> 1) & 1);
-                if (npv > 0) mbar_wait(&o_full[(npv - 1) & 1], ((npv - 1) >> 1) & 1);
-            }
+            // Wait (bounded) for the MMAs this thread issued before tensor memory
+            // is released: complete already on the normal path, possibly in
+            // flight after an abort raised by another role.
+            if (ns > 0) mbar_wait(&s_full[(ns - 1) & 1], ((ns - 1) >> 1) & 1);
+            if (npv > 0) mbar_wait(&o_full[(npv - 1) & 1], ((npv - 1) >> 1) & 1);
         }
     } else {
         // ================================================================ softmax rows

@@ -19,7 +19,7 @@ __device__ unsigned int g_device_error;
 __device__ __forceinline__ void flag_error(unsigned int bits) { atomicOr(&g_device_error, bits); }
 
 // Bounded waits give up after this many nanoseconds of %globaltimer.
-constexpr uint64_t kWaitLimitNs = 1000000000ull;
+constexpr uint64_t kWaitLimitNs = PKV_DEFAULT_WAIT_LIMIT_NS;
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
     return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -72,6 +72,14 @@ __device__ __forceinline__ bool mbar_poll(uint64_t* bar, uint32_t parity) {
     return done != 0;
 }
 
+// Limit of the waits inside the kernels' main loops, in ns of %globaltimer.
+// The default is kWaitLimitNs; pkv_set_wait_limit_ns changes it for later
+// launches, and 0 makes a main-loop wait that would block give up at once (a
+// test setting that runs the give-up path).  The drain waits a CTA makes
+// before it exits (for its own bulk copies and tensor-core MMAs) always keep
+// kWaitLimitNs.
+__constant__ uint64_t c_main_wait_limit_ns = kWaitLimitNs;
+
 // Wait for the phase with the given parity to complete.  Gives up after
 // kWaitLimitNs, sets PKV_DEVERR_TIMEOUT and returns false.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
@@ -88,26 +96,63 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
     }
 }
 
+// The same wait under the main-loop limit (c_main_wait_limit_ns).
+__device__ __forceinline__ bool mbar_wait_main(uint64_t* bar, uint32_t parity) {
+    if (mbar_poll(bar, parity)) return true;
+    const uint64_t limit = c_main_wait_limit_ns;
+    if (limit == 0) {
+        flag_error(PKV_DEVERR_TIMEOUT);
+        return false;
+    }
+    const uint64_t t0 = global_timer_ns();
+    while (true) {
+#pragma unroll 1
+        for (int i = 0; i < 32; ++i)
+            if (mbar_test(bar, parity)) return true;
+        if (global_timer_ns() - t0 > limit) {
+            flag_error(PKV_DEVERR_TIMEOUT);
+            return false;
+        }
+    }
+}
+
 __device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
     asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
 }
 
-// Bounded wait that also returns false as soon as the CTA-wide abort flag is
-// set (by a thread whose own wait gave up); on expiry it sets the flag.
+// Bounded main-loop wait (c_main_wait_limit_ns) that also returns false as
+// soon as the CTA-wide abort flag is set (by a thread whose own wait gave
+// up); on expiry it sets the flag.
 __device__ __forceinline__ bool mbar_wait_or_abort(uint64_t* bar, uint32_t parity, volatile int* abort) {
-    if (mbar_test(bar, parity)) return true;
+    if (mbar_poll(bar, parity)) return true;
+    const uint64_t limit = c_main_wait_limit_ns;
+    if (limit == 0) {
+        flag_error(PKV_DEVERR_TIMEOUT);
+        *abort = 1;
+        return false;
+    }
     const uint64_t t0 = global_timer_ns();
     while (true) {
 #pragma unroll 1
         for (int i = 0; i < 32; ++i)
             if (mbar_test(bar, parity)) return true;
         if (*abort) return false;
-        if (global_timer_ns() - t0 > kWaitLimitNs) {
+        if (global_timer_ns() - t0 > limit) {
             flag_error(PKV_DEVERR_TIMEOUT);
             *abort = 1;
             return false;
         }
     }
+}
+
+// Programmatic dependent launch.  griddep_wait blocks until the grids this
+// one depends on have completed and their writes are visible (a no-op for a
+// grid launched without the programmatic-serialisation attribute);
+// griddep_launch_dependents lets a dependent grid start launching before this
+// one ends.
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void griddep_launch_dependents() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
 
 // 2^x, hardware approximation (flush-to-zero); 2^-inf = 0.

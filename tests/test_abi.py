@@ -167,7 +167,7 @@ def _kind(ctype_name):
     if "*" in t or t in ("pkv_stream_t",):
         return "ptr"
     return {"int": ctypes.c_int, "int64_t": ctypes.c_int64, "float": ctypes.c_float, "size_t": ctypes.c_size_t,
-            "uint32_t": ctypes.c_uint32, "void": None}[t]
+            "uint32_t": ctypes.c_uint32, "uint64_t": ctypes.c_uint64, "void": None}[t]
 
 
 def _argkind(a):

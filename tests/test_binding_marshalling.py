@@ -185,3 +185,31 @@ def test_size_queries_arguments(mock):
     assert name == "pkv_prefill_fp8_workspace_size" and a == {
         "num_chunks": 2, "max_blocks_per_seq": 6, "block_size": 16, "num_kv_heads": 2, "head_dim": 128,
         "total_q_tokens": 9, "num_q_heads": 8, "dtype": 2}
+
+
+def test_decode_step_arguments(mock):
+    S, Hq, Hkv, D, B, NB, MB = 5, 8, 8, 128, 16, 23, 4
+    q = torch.zeros(S, Hq, D, dtype=torch.float16)
+    out = torch.zeros_like(q)
+    kc, vc = torch.zeros(NB, B, Hkv, D, dtype=torch.float16), torch.zeros(NB, B, Hkv, D, dtype=torch.float16)
+    bt, cl = torch.zeros(S, MB, dtype=torch.int32), torch.zeros(S, dtype=torch.int32)
+    kn, vn = torch.zeros(S, Hkv, D, dtype=torch.float16), torch.zeros(S, Hkv, D, dtype=torch.float16)
+    sm = torch.zeros(S, dtype=torch.int64)
+    pkv.paged_attention_decode_step(kn, vn, sm, out, q, kc, vc, bt, cl, 0.4, 60, partition_size=0, stream=9)
+    name, a = mock.last()
+    assert name == "pkv_paged_attention_decode_step"
+    assert a == {"new_keys": kn.data_ptr(), "new_values": vn.data_ptr(), "slot_mapping": sm.data_ptr(),
+                 "num_new_tokens": S, "out": out.data_ptr(), "query": q.data_ptr(), "key_cache": kc.data_ptr(),
+                 "value_cache": vc.data_ptr(), "block_tables": bt.data_ptr(), "context_lens": cl.data_ptr(),
+                 "scale": f32(0.4), "num_seqs": S, "num_q_heads": Hq, "num_kv_heads": Hkv, "head_dim": D,
+                 "block_size": B, "max_blocks_per_seq": MB, "num_blocks": NB, "max_context_len": 60,
+                 "partition_size": 0, "dtype": 1, "workspace": 0, "workspace_bytes": 0, "stream": 9}
+    kc8, vc8 = torch.zeros(NB, B, Hkv, D, dtype=torch.uint8), torch.zeros(NB, B, Hkv, D, dtype=torch.uint8)
+    pkv.paged_attention_decode_step_fp8(kn, vn, sm, out, q, kc8, vc8, bt, cl, 0.4, 0.5, 0.25, 60, partition_size=0)
+    name, a = mock.last()
+    assert name == "pkv_paged_attention_decode_step_fp8"
+    assert (a["k_scale"], a["v_scale"], a["key_cache"], a["value_cache"], a["num_new_tokens"], a["dtype"]) == (
+        0.5, 0.25, kc8.data_ptr(), vc8.data_ptr(), S, 1)
+    pkv.set_wait_limit_ns(1234)
+    name, a = mock.last()
+    assert name == "pkv_set_wait_limit_ns" and a == {"limit_ns": 1234}
