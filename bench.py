@@ -8,18 +8,22 @@ sequences, 32 heads = 32 KV heads, head_dim 128, block 16, context U[128,
 paged decode attention (decode kernel + log-sum-exp merge) over all 64
 sequences, on inputs already resident in HBM (the pools, 1.25 GB each, are
 far larger than the 126 MB L2).  The step's launches are captured once in a
-CUDA graph and replayed (``--no-graph`` launches them one by one); the
-decode-call duration for the roofline comes from a plain launch loop.  ``value`` = decode tokens (sequences) per
-second over all ranks; multi-GPU runs are independent replicas (weak
-scaling, no collective on the data path).
+CUDA graph and replayed (``--no-graph`` launches them one by one).  The timed
+region of exactly ``--steps`` steps is repeated until at least
+``--min-timed-ms`` have been timed; ``ms_per_step`` is the median region's
+time per step.  The decode-call duration for the roofline comes from a second
+graph that holds only the step's decode calls, replayed the same way.
+``value`` = decode tokens (sequences) per second over all ranks; multi-GPU
+runs are independent replicas (weak scaling, no collective on the data path).
 
 Other ``--config`` values time the remaining named workloads for the
 report: gqa70b_decode_bf16 (80 layers per step), shared_prefix_decode_f16,
 mixed_step_bf16 (append + chunked prefill + decode).
 
-``--impl reference`` times the CPU oracle (double precision, one thread) on
-a bounded sample of the same workload: there is no runnable reference
-implementation of this path.
+``--impl reference`` times the CPU oracle (double precision, all host cores)
+on a bounded sample of the same workload: there is no runnable reference
+implementation of this path.  That arm loads only the oracle, never the CUDA
+library.
 """
 from __future__ import annotations
 
@@ -56,23 +60,30 @@ def peaks():
 # ----------------------------------------------------------------------------- workloads as timed steps
 
 class DecodeStep:
-    """reshape_and_cache + paged_attention_decode over every layer of a DecodeWorkload."""
+    """reshape_and_cache + paged_attention_decode over every layer of a DecodeWorkload.
 
-    def __init__(self, w, layers_per_step=None):
-        import paged_kv_cache_409_b200 as pkv
-        self.pkv, self.w = pkv, w
+    ``library=False`` (the oracle's arm) builds only the workload's figures and
+    never loads the CUDA library."""
+
+    def __init__(self, w, layers_per_step=None, library=True):
+        self.w = w
         dev = w.queries[0].device
         self.bt = torch.from_numpy(w.block_tables).to(dev)
         self.cl = torch.from_numpy(w.context_lens.astype(np.int32)).to(dev)
         self.sm = torch.from_numpy(w.slot_mapping.astype(np.int64)).to(dev)
         self.layers = layers_per_step or w.num_layers
+        self.units_per_step = self.layers  # decode calls per step
         self.outs = [torch.empty_like(q) for q in w.queries]
-        self.part = pkv.decode_partition_size(w.num_seqs, w.num_q_heads, w.num_kv_heads, w.head_dim, w.block_size,
-                                              w.max_context_len, 3 if w.fp8 else w.dtype,
-                                              int(w.context_lens.astype(np.int64).sum()))
-        need = pkv.decode_workspace_size(w.num_seqs, w.num_q_heads, w.head_dim, w.max_context_len, self.part)
-        self.ws = torch.empty(max(need, 16), dtype=torch.uint8, device=dev)
-        self.parts = -(-w.max_context_len // self.part) if self.part else 1
+        self.part, self.parts = 0, 1
+        if library:
+            import paged_kv_cache_409_b200 as pkv
+            self.pkv = pkv
+            self.part = pkv.decode_partition_size(w.num_seqs, w.num_q_heads, w.num_kv_heads, w.head_dim,
+                                                  w.block_size, w.max_context_len, 3 if w.fp8 else w.dtype,
+                                                  int(w.context_lens.astype(np.int64).sum()))
+            need = pkv.decode_workspace_size(w.num_seqs, w.num_q_heads, w.head_dim, w.max_context_len, self.part)
+            self.ws = torch.empty(max(need, 16), dtype=torch.uint8, device=dev)
+            self.parts = -(-w.max_context_len // self.part) if self.part else 1
         t = w.queries[0].element_size()
         tkv = w.key_caches[0].element_size()
         self.kv_bytes = 2 * int(w.context_lens.astype(np.int64).sum()) * w.num_kv_heads * w.head_dim * tkv
@@ -127,15 +138,36 @@ class DecodeStep:
                                             self.cl, w.scale, w.max_context_len, partition_size=self.part,
                                             workspace=self.ws)
 
+    def step_call(self, l):
+        """The layer's append + decode as one library call (the decode launched as the append's
+        programmatic dependent)."""
+        w = self.w
+        if w.fp8:
+            self.pkv.paged_attention_decode_step_fp8(w.new_keys[l], w.new_values[l], self.sm, self.outs[l],
+                                                     w.queries[l], w.key_caches[l], w.value_caches[l], self.bt,
+                                                     self.cl, w.scale, w.extra["k_scale"], w.extra["v_scale"],
+                                                     w.max_context_len, partition_size=self.part, workspace=self.ws)
+        else:
+            self.pkv.paged_attention_decode_step(w.new_keys[l], w.new_values[l], self.sm, self.outs[l],
+                                                 w.queries[l], w.key_caches[l], w.value_caches[l], self.bt, self.cl,
+                                                 w.scale, w.max_context_len, partition_size=self.part,
+                                                 workspace=self.ws)
+
     def run(self, timer=None, step=0):
         for i in range(self.layers):
             l = (step * self.layers + i) % self.w.num_layers
-            self.append(l)
-            if timer:
+            if timer:  # separate calls, so that events can bracket the decode
+                self.append(l)
                 timer.begin()
-            self.attend(l)
-            if timer:
+                self.attend(l)
                 timer.end()
+            else:
+                self.step_call(l)
+
+    def run_units(self, step=0):
+        """The step's decode calls alone (the roofline's unit), in the step's layer order."""
+        for i in range(self.layers):
+            self.attend((step * self.layers + i) % self.w.num_layers)
 
 
 class E2EPlan:
@@ -205,8 +237,8 @@ def pinned(t):
 class MixedStep(DecodeStep):
     """Continuous-batching step: append all tokens, chunked prefill, decode."""
 
-    def __init__(self, m):
-        super().__init__(m.decode)
+    def __init__(self, m, library=True):
+        super().__init__(m.decode, library=library)
         self.m = m
         dev = m.decode.queries[0].device
         self.aslots = torch.from_numpy(m.append_slots).to(dev)
@@ -219,7 +251,7 @@ class MixedStep(DecodeStep):
         n, c0 = m.chunk_lens.astype(np.int64), m.chunk_c0.astype(np.int64)
         self.prefill_flops = int(4 * D * Hq * np.sum(n * c0 + n * (n + 1) // 2))
         self.pws = None
-        if m.decode.fp8:
+        if m.decode.fp8 and library:
             w = m.decode
             need = self.pkv.prefill_fp8_workspace_size(len(n), m.chunk_tables.shape[1], w.block_size,
                                                        w.num_kv_heads, D, m.chunk_query.shape[0], Hq, w.dtype)
@@ -260,6 +292,9 @@ class MixedStep(DecodeStep):
         if timer:
             timer.end()
 
+    def run_units(self, step=0):
+        self.attend(0)
+
 
 class MultiTokenStep:
     """Multi-token decode (speculative verification): append each sequence's
@@ -267,10 +302,10 @@ class MultiTokenStep:
     (``paged_attention_decode_multi``; ``via_prefill`` times the chunked-prefill
     call on the same step instead)."""
 
-    def __init__(self, m, via_prefill=False):
-        import paged_kv_cache_409_b200 as pkv
-        self.pkv, self.m, self.w = pkv, m, m.decode
+    def __init__(self, m, via_prefill=False, library=True):
+        self.m, self.w = m, m.decode
         self.via_prefill = via_prefill
+        self.units_per_step = 1
         dev = m.chunk_query.device
         self.aslots = torch.from_numpy(m.append_slots).to(dev)
         self.cbt = torch.from_numpy(m.chunk_tables).to(dev)
@@ -282,11 +317,15 @@ class MultiTokenStep:
         w = m.decode
         R, Hkv, B = len(m.seq_lens), w.num_kv_heads, w.block_size
         self.layers = 1
-        self.part = 0 if via_prefill else pkv.decode_multi_partition_size(R, Hkv, B, self.max_len)
-        Tq, Hq, D = m.chunk_query.shape
-        need = pkv.decode_workspace_size(Tq, Hq, D, self.max_len, self.part) if self.part else 0
-        self.ws = torch.empty(max(need, 16), dtype=torch.uint8, device=dev)
-        self.parts = -(-self.max_len // self.part) if self.part else 1
+        self.part, self.parts = 0, 1
+        if library:
+            import paged_kv_cache_409_b200 as pkv
+            self.pkv = pkv
+            self.part = 0 if via_prefill else pkv.decode_multi_partition_size(R, Hkv, B, self.max_len)
+            Tq, Hq, D = m.chunk_query.shape
+            need = pkv.decode_workspace_size(Tq, Hq, D, self.max_len, self.part) if self.part else 0
+            self.ws = torch.empty(max(need, 16), dtype=torch.uint8, device=dev)
+            self.parts = -(-self.max_len // self.part) if self.part else 1
         t = m.chunk_query.element_size()
         self.kv_bytes = 2 * int(m.seq_lens.astype(np.int64).sum()) * w.num_kv_heads * w.head_dim * t
         nblocks = int(((m.seq_lens.astype(np.int64) + w.block_size - 1) // w.block_size).sum())
@@ -302,7 +341,7 @@ class MultiTokenStep:
                 "context_range": [int(m.chunk_c0.min()), int(m.chunk_c0.max())],
                 "partition_size": self.part, "call": "prefill_chunk" if self.via_prefill else "decode_multi"}
 
-    def oracle_sample(self, budget_s, max_seqs=8):
+    def oracle_sample(self, budget_s, max_seqs=64):
         """Oracle append + causal attention of the first sequences' drafts."""
         sys.path.insert(0, os.path.join(ROOT, "tests"))
         from parity_helpers import oracle_prefill_chunks
@@ -333,6 +372,12 @@ class MultiTokenStep:
         self.pkv.reshape_and_cache(m.append_keys, m.append_values, w.key_caches[0], w.value_caches[0], self.aslots)
         if timer:
             timer.begin()
+        self.run_units(step)
+        if timer:
+            timer.end()
+
+    def run_units(self, step=0):
+        m, w = self.m, self.w
         if self.via_prefill:
             self.pkv.paged_attention_prefill_chunk(self.out, m.chunk_query, w.key_caches[0], w.value_caches[0],
                                                    self.cbt, self.csl, self.qsl, self.max_q, w.scale)
@@ -340,64 +385,75 @@ class MultiTokenStep:
             self.pkv.paged_attention_decode_multi(self.out, m.chunk_query, w.key_caches[0], w.value_caches[0],
                                                   self.cbt, self.csl, self.qsl, self.max_q, self.max_len, w.scale,
                                                   partition_size=self.part, workspace=self.ws)
-        if timer:
-            timer.end()
 
 
-# DRAM bytes (read + write) per algorithmic byte of the decode call, from one
-# ncu capture of the same kernel on a smaller case of the workload (traffic
-# grows with the blocks read, so it scales to the full launch by the
-# algorithmic bytes).  A workload is listed only while its kernel is unchanged
-# since the capture.
-TRAFFIC_PER_ALGORITHMIC_BYTE = {
-    "llama7b_decode_f16": ((287.471104 + 3.418624) / 285.38096,
-                           "profiles/paged_decode_mma_kernel_llama7b_16seq_full.md"),
-    "llama7b_decode_fp8": ((305.044224 + 3.7632 + 1.388544 + 0.0) / 303.293524,
-                           "profiles/paged_decode_fp8_kernel_llama7b_fp8_launches.md (decode + merge)"),
+# DRAM traffic of the decode call per algorithmic byte, from one ncu capture
+# (dram__bytes_read.sum + dram__bytes_write.sum, --clock-control none) of the
+# same kernels on a smaller case of the workload: traffic grows with the blocks
+# read, so it scales to the full launch by the algorithmic bytes.  A workload
+# is listed only while its kernels are unchanged since the capture.  Figures in
+# MB (1e6 bytes): DRAM read, DRAM written, algorithmic bytes of the captured
+# launch(es).
+TRAFFIC_CAPTURES = {
+    "llama7b_decode_f16": {"case": "paged_decode_mma_kernel, the llama7b batch cut to 16 sequences",
+                           "read_mb": 287.471104, "write_mb": 3.418624, "algorithmic_mb": 285.38096},
+    "llama7b_decode_fp8": {"case": "paged_decode_fp8_kernel + merge, the 64-sequence llama7b batch on E4M3 pools",
+                           "read_mb": 305.044224 + 1.388544, "write_mb": 3.7632 + 0.0,
+                           "algorithmic_mb": 303.293524},
 }
 
 
-def make_step(name, device, rank, seqs=None, layers=None):
+def traffic_ratio(name):
+    c = TRAFFIC_CAPTURES[name]
+    return (c["read_mb"] + c["write_mb"]) / c["algorithmic_mb"]
+
+
+def make_step(name, device, rank, seqs=None, layers=None, library=True):
+    """The named workload as a timed step.  ``library=False`` (the oracle's arm) builds the same inputs
+    without loading the CUDA library; the shared-prefix setup (copy-on-write of the partial prefix block,
+    the private tokens' append) is then done with plain torch indexing."""
     from paged_kv_cache_409_b200 import workloads
     if name == "llama7b_decode_f16":
         w = workloads.llama7b_decode_f16(device=device, seed=1002 + rank, num_seqs=seqs or 64)
-        return DecodeStep(w), "llama7b_decode_f16" + (f" ({seqs} sequences)" if seqs else "")
+        return DecodeStep(w, library=library), "llama7b_decode_f16" + (f" ({seqs} sequences)" if seqs else "")
     if name == "llama7b_decode_fp8":
         w = workloads.llama7b_decode_fp8(device=device, seed=1002 + rank, num_seqs=seqs or 64)
-        return DecodeStep(w), "llama7b_decode_fp8" + (f" ({seqs} sequences)" if seqs else "")
-    if name == "gqa70b_decode_fp8":
-        free, _ = torch.cuda.mem_get_info()
-        per_layer = 0.9e9 * (seqs or 256) / 256  # FP8 pools of one layer (~0.81 GB at 256 sequences) plus headroom
+        return DecodeStep(w, library=library), "llama7b_decode_fp8" + (f" ({seqs} sequences)" if seqs else "")
+    if name in ("gqa70b_decode_fp8", "gqa70b_decode_bf16"):
+        fp8 = name.endswith("fp8")
+        per_layer = (0.9e9 if fp8 else 1.75e9) * (seqs or 256) / 256  # pools of one layer plus headroom
+        free = torch.cuda.mem_get_info()[0] if torch.cuda.is_available() else 16e9
         fit = int(max(1, min(80, (free - 8e9) // per_layer)))
         layers = min(fit, layers) if layers else fit
-        w = workloads.gqa70b_decode_fp8(device=device, num_layers=layers, seed=1003 + rank, num_seqs=seqs or 256)
+        if not library:
+            layers = 1  # the oracle reads one layer; its pools are the first layer's of the full workload
+        make = workloads.gqa70b_decode_fp8 if fp8 else workloads.gqa70b_decode_bf16
+        w = make(device=device, num_layers=layers, seed=1003 + rank, num_seqs=seqs or 256)
         note = "" if layers == 80 else f", {layers} distinct layer pools cycled"
-        return DecodeStep(w, layers_per_step=80), f"gqa70b_decode_fp8 (80 layers per step{note})"
+        return DecodeStep(w, layers_per_step=80, library=library), f"{name} (80 layers per step{note})"
     if name == "tiny_decode_f32":
-        return DecodeStep(workloads.tiny_decode_f32(device=device)), name
-    if name == "gqa70b_decode_bf16":
-        free, _ = torch.cuda.mem_get_info()
-        per_layer = 1.75e9 * (seqs or 256) / 256  # pools of one layer (~1.62 GB at 256 sequences) plus headroom
-        fit = int(max(1, min(80, (free - 8e9) // per_layer)))
-        layers = min(fit, layers) if layers else fit
-        w = workloads.gqa70b_decode_bf16(device=device, num_layers=layers, seed=1003 + rank, num_seqs=seqs or 256)
-        note = "" if layers == 80 else f", {layers} distinct layer pools cycled"
-        return DecodeStep(w, layers_per_step=80), f"gqa70b_decode_bf16 (80 layers per step{note})"
+        return DecodeStep(workloads.tiny_decode_f32(device=device), library=library), name
     if name == "shared_prefix_decode_f16":
         sp = workloads.shared_prefix_decode_f16(device=device, seed=1004 + rank)
-        st = DecodeStep(sp.step)
+        st = DecodeStep(sp.step, library=library)
         kc, vc = sp.step.key_caches[0], sp.step.value_caches[0]
-        st.pkv.copy_blocks([kc], [vc], torch.from_numpy(sp.cow_pairs).to(device))
-        st.pkv.reshape_and_cache(sp.private_keys, sp.private_values, kc, vc,
-                                 torch.from_numpy(sp.private_slots).to(device))
+        pairs = torch.from_numpy(sp.cow_pairs).to(device)
+        slots = torch.from_numpy(sp.private_slots).to(device)
+        if library:
+            st.pkv.copy_blocks([kc], [vc], pairs)
+            st.pkv.reshape_and_cache(sp.private_keys, sp.private_values, kc, vc, slots)
+        else:
+            for c, new in ((kc, sp.private_keys), (vc, sp.private_values)):
+                c[pairs[:, 1]] = c[pairs[:, 0]]
+                c.view(-1, *c.shape[2:])[slots] = new
         return st, name
     if name in ("mixed_step_bf16", "mixed_step_fp8"):
         make = workloads.mixed_step_bf16 if name == "mixed_step_bf16" else workloads.mixed_step_fp8
         m = make(device=device, seed=1005 + rank, num_decode=seqs or 192)
-        return MixedStep(m), name + (f" ({seqs} decode sequences)" if seqs else "")
+        return MixedStep(m, library=library), name + (f" ({seqs} decode sequences)" if seqs else "")
     if name in ("multi_token_decode_bf16", "multi_token_decode_bf16_via_prefill"):
         m = workloads.multi_token_decode_bf16(device=device, seed=1006 + rank, num_seqs=seqs or 64)
-        return MultiTokenStep(m, via_prefill=name.endswith("via_prefill")), name + (
+        return MultiTokenStep(m, via_prefill=name.endswith("via_prefill"), library=library), name + (
             f" ({seqs} sequences)" if seqs else "")
     raise SystemExit(f"unknown config {name}")
 
@@ -574,6 +630,20 @@ def index_kernel_figures(step, hbm_gbs, launches=20):
                        "note": "one step's append: launch-bound, its bytes fit in L2"}}
 
 
+def host_cores():
+    """Host cores this process may run on."""
+    try:
+        return len(os.sched_getaffinity(0))
+    except (AttributeError, OSError):
+        return os.cpu_count() or 1
+
+
+def oracle_threads(n):
+    """Set the oracle's host threads; returns the number in force."""
+    import oracle
+    return oracle.get().num_threads(n)
+
+
 def oracle_sample(step, budget_s, max_seqs=None):
     """Time the oracle (append + decode) on whole steps or a sequence sample, host cores."""
     import oracle
@@ -611,15 +681,41 @@ def oracle_sample(step, budget_s, max_seqs=None):
     return len(seqs) * done / el, done, len(seqs), el
 
 
+def cpu_baselines(step, args):
+    """The oracle timed on all host cores (the reported cpu_baseline) and on one thread, each on about half
+    of --cpu-budget seconds of the same workload (whole steps, or a sequence sample of large ones)."""
+    w = step.w
+    out = []
+    for n in (host_cores(), 1):
+        cores = oracle_threads(n)
+        if hasattr(step, "oracle_sample"):
+            v, done, what, el = step.oracle_sample(args.cpu_budget / 2)
+            out.append({"value": v, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                        "sample": f"{done} x (append + causal attention of {what}), {el:.1f} s, {cores} threads"})
+        elif step.layers == 1:
+            v, done, k, el = oracle_sample(step, args.cpu_budget / 2, max_seqs=None if w.num_seqs <= 64 else 16)
+            out.append({"value": v, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                        "sample": f"{done} x (append + decode of {k} sequences), {el:.1f} s, {cores} threads"})
+        else:
+            v, done, k, el = oracle_sample(step, args.cpu_budget / 2, max_seqs=16)
+            out.append({"value": v / step.layers, "unit": f"tokens/s ({step.layers}-layer steps)", "cores": cores,
+                        "kind": "oracle", "sample": f"{done} x one layer of {k} sequences, {el:.1f} s, {cores} "
+                                                    f"threads; /{step.layers} layers"})
+    oracle_threads(host_cores())
+    return out[0], out[1]
+
+
 # ----------------------------------------------------------------------------- main
 
 def run_reference(args, ws, rank):
-    """The oracle as it stands, on the host cores, on a bounded sample of the workload."""
+    """The oracle as it stands, on all host cores, on a bounded sample of the workload.  Only the oracle
+    is loaded: the inputs are the same seeded workload, built with torch alone."""
     if rank != 0:
         return
     dev = "cuda" if torch.cuda.is_available() else "cpu"
-    step, cname = make_step(args.config, dev, 0)
+    step, cname = make_step(args.config, dev, 0, library=False)
     w = step.w
+    cores = oracle_threads(host_cores())
     times = []
     if hasattr(step, "oracle_sample"):
         for i in range(args.warmup + args.steps):
@@ -627,22 +723,28 @@ def run_reference(args, ws, rank):
             if i >= args.warmup:
                 times.append(el)
         per = statistics.fmean(times)
-        value, sample_text = v * el / per, f"append + causal attention of {what} per step"
+        value = v * el / per
+        sample_text = f"append + causal attention of {what} per step"
         sample = what
     else:
-        sample = min(w.num_seqs, 8)
+        sample = w.num_seqs if w.num_seqs <= 64 else 16
         for i in range(args.warmup + args.steps):
             v, done, n, el = oracle_sample(step, 0.0, max_seqs=sample)
             if i >= args.warmup:
                 times.append(el)
         per = statistics.fmean(times)
         value = sample / per
-        sample_text = f"append + decode of the first {sample} of {w.num_seqs} sequences per step"
+        sample_text = (f"append + decode of {'all' if sample == w.num_seqs else 'the first'} {sample} of "
+                       f"{w.num_seqs} sequences per step")
+        if step.layers > 1:
+            value /= step.layers
+            sample_text += f" (one layer; tokens/s of {step.layers}-layer steps)"
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": args.gpus,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": per * 1e3, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "config": {"workload": cname, "sample": sample},
-            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": 1, "kind": "oracle", "sample": sample_text},
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                             "sample": f"{sample_text}, {cores} threads"},
             "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
 
@@ -690,6 +792,21 @@ def run_swap(args, ws, rank):
         print(json.dumps(line), flush=True)
 
 
+def capture(fn):
+    """fn's launches captured once in a CUDA graph (after one run on a side stream), replayed once."""
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        fn()
+    torch.cuda.current_stream().wait_stream(side)
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        fn()
+    g.replay()
+    torch.cuda.synchronize()
+    return g
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -703,6 +820,9 @@ def main():
     ap.add_argument("--layers", type=int, default=None, help="cap on distinct layer pools (gqa70b_decode_bf16)")
     ap.add_argument("--no-graph", dest="graph", action="store_false",
                     help="launch every kernel of every step instead of replaying one captured CUDA graph")
+    ap.add_argument("--min-timed-ms", type=float, default=1000.0,
+                    help="repeat the timed region of --steps steps until at least this much has been timed")
+    ap.add_argument("--max-regions", type=int, default=1000, help="cap on the number of timed regions")
     ap.add_argument("--flush-l2", action="store_true",
                     help="write a 512 MB buffer before every timed step (outside its events) so that no step "
                          "finds the previous one's K/V in L2; the steps' own durations are summed")
@@ -726,7 +846,7 @@ def main():
     step, cname = make_step(args.config, dev, rank, args.seqs, args.layers)
     torch.cuda.synchronize()
 
-    # warm-up, then exactly K timed steps between barriers
+    # warm-up, then timed regions of exactly K steps between barriers, repeated until enough time is timed
     clocks = ClockSampler(torch.cuda.current_device())
     clocks.start()
     for i in range(args.warmup):
@@ -734,55 +854,55 @@ def main():
     torch.cuda.synchronize()
     barrier(ws)
     timer = EventTimer()
-    graph = None
+    graph = unit_graph = None
     if args.graph:
-        # one whole step (every layer) per graph; layers cycle within it
-        side = torch.cuda.Stream()
-        side.wait_stream(torch.cuda.current_stream())
-        with torch.cuda.stream(side):
-            step.run(step=0)
-        torch.cuda.current_stream().wait_stream(side)
-        graph = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(graph):
-            step.run(step=0)
-        graph.replay()
-        torch.cuda.synchronize()
-    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        graph = capture(lambda: step.run(step=0))
+        unit_graph = capture(lambda: step.run_units(step=0))
     flush = torch.empty(512 << 20, dtype=torch.uint8, device=dev) if args.flush_l2 else None
-    per_step = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-                for _ in range(args.steps)] if flush is not None else None
+
+    def region(fn):
+        """K steps of fn between a barrier and a synchronize on both sides; the max over ranks."""
+        barrier(ws)
+        torch.cuda.synchronize()
+        t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        per = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(args.steps)] if flush is not None else None
+        t0.record()
+        for i in range(args.steps):
+            if flush is not None:
+                flush.fill_(i & 0xFF)
+                per[i][0].record()
+            fn(i)
+            if flush is not None:
+                per[i][1].record()
+        t1.record()
+        torch.cuda.synchronize()
+        ms = sum(a.elapsed_time(b) for a, b in per) if flush is not None else t0.elapsed_time(t1)
+        return max_over_ranks(ms, ws)  # every rank gets the same value, so every rank decides alike
+
+    def repeat(fn, min_ms):
+        out = []
+        while not out or (sum(out) < min_ms and len(out) < args.max_regions):
+            out.append(region(fn))
+        return out
+
     h0 = time.perf_counter()
     torch.cuda.nvtx.range_push("timed")
-    t0.record()
-    for i in range(args.steps):
-        if flush is not None:
-            flush.fill_(i & 0xFF)
-            per_step[i][0].record()
-        if graph is not None:
-            graph.replay()
-        else:
-            step.run(timer=timer, step=i)
-        if flush is not None:
-            per_step[i][1].record()
-    t1.record()
+    regions = repeat((lambda i: graph.replay()) if graph is not None else (lambda i: step.run(timer=timer, step=i)),
+                     args.min_timed_ms)
     torch.cuda.nvtx.range_pop()
-    torch.cuda.synchronize()
     clocks.mark(h0, time.perf_counter())
     clk = clocks.stop()
-    barrier(ws)
-    if flush is None:
-        ms_total = max_over_ranks(t0.elapsed_time(t1), ws)
+    ms_step = statistics.median(regions) / args.steps
+    if unit_graph is not None:
+        # the decode calls of the step alone, replayed as captured: the roofline's unit
+        unit_regions = repeat(lambda i: unit_graph.replay(), args.min_timed_ms / 4)
+        unit_ms = statistics.median(unit_regions) / (args.steps * step.units_per_step)
+        unit_how = "CUDA graph of the step's decode calls alone, replayed (median region)"
     else:
-        ms_total = max_over_ranks(sum(a.elapsed_time(b) for a, b in per_step), ws)
-        del flush
-    ms_step = ms_total / args.steps
-    if graph is not None:
-        # the decode-call duration for the roofline, from a short plain loop
-        for i in range(min(args.steps, 50)):
-            step.run(timer=timer, step=i)
-        torch.cuda.synchronize()
-        del graph
-    unit_ms = max_over_ranks(timer.mean_ms(), ws)
+        unit_ms = max_over_ranks(timer.mean_ms(), ws)
+        unit_how = "CUDA events around each decode call of the timed steps (mean)"
+    del graph, unit_graph, flush
     assert pkv.get_device_error() == 0, "device error word set during the run"
 
     # end to end through the public API: pinned host inputs in, result out, every step
@@ -835,15 +955,18 @@ def main():
                 "copies": "on two side streams, overlapping the neighbouring steps' kernels (two device sets)",
                 "result_matches_device_run": e2e.matches()},
         "gpu_launches": step.launches_per_step() * args.steps,
+        "timed_regions": len(regions), "timed_ms": sum(regions),
         "clocks": clk,
     }
+    line["roofline"]["unit_ms"] = unit_ms
+    line["roofline"]["unit_timing"] = unit_how
     if hasattr(step, "config"):
         line["config"].update(step.config())
-    if args.config in TRAFFIC_PER_ALGORITHMIC_BYTE and not args.seqs:
-        ratio, source = TRAFFIC_PER_ALGORITHMIC_BYTE[args.config]
-        line["roofline"]["traffic"] = ratio * step.decode_bytes  # DRAM bytes per decode call
+    if args.config in TRAFFIC_CAPTURES and not args.seqs:
+        line["roofline"]["traffic"] = traffic_ratio(args.config) * step.decode_bytes  # DRAM bytes per decode call
         line["roofline"]["traffic_unit"] = "bytes per launch"
-        line["roofline"]["traffic_source"] = source + " (smaller case, scaled by algorithmic bytes)"
+        line["roofline"]["traffic_source"] = ("ncu DRAM bytes of " + TRAFFIC_CAPTURES[args.config]["case"] +
+                                              ", scaled by algorithmic bytes")
     if getattr(step, "unique_kv_bytes", None) and 2 * step.unique_kv_bytes < step.kv_bytes * step.layers:
         # shared blocks: most logical bytes come from L2, so the HBM fraction above exceeds 1 by design
         uniq = step.unique_kv_bytes / step.layers
@@ -855,19 +978,8 @@ def main():
     if isinstance(step, MixedStep):
         line["prefill_tokens_per_s"] = ws * step.prefill_tokens / (ms_step / 1e3)
         line["prefill_flops_per_step"] = step.prefill_flops
-    if rank == 0 and ws == 1 and args.cpu_budget > 0 and hasattr(step, "oracle_sample"):
-        v, done, what, el = step.oracle_sample(args.cpu_budget)
-        line["cpu_baseline"] = {"value": v, "unit": "tokens/s", "cores": 1, "kind": "oracle",
-                                "sample": f"{done} x (append + causal attention of {what}), {el:.1f} s, 1 thread"}
-    elif rank == 0 and ws == 1 and args.cpu_budget > 0 and not args.config.startswith("gqa70b"):
-        v, done, n, el = oracle_sample(step, args.cpu_budget, max_seqs=None if w.num_seqs <= 64 else 16)
-        line["cpu_baseline"] = {"value": v, "unit": "tokens/s", "cores": 1, "kind": "oracle",
-                                "sample": f"{done} x (append + decode of {n} sequences), {el:.1f} s, 1 thread"}
-    elif rank == 0 and ws == 1 and args.cpu_budget > 0:
-        v, done, n, el = oracle_sample(step, args.cpu_budget, max_seqs=16)
-        line["cpu_baseline"] = {"value": v / 80.0, "unit": "tokens/s (80-layer steps)", "cores": 1,
-                                "kind": "oracle",
-                                "sample": f"{done} x one layer of {n} sequences, {el:.1f} s, 1 thread; /80 layers"}
+    if rank == 0 and ws == 1 and args.cpu_budget > 0:
+        line["cpu_baseline"], line["cpu_baseline_1_thread"] = cpu_baselines(step, args)
     if ws == 1 and type(step) is DecodeStep:
         try:
             line["index_kernels"] = index_kernel_figures(step, hbm)

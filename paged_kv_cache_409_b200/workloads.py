@@ -399,14 +399,23 @@ def mixed_workload(name, decode_lens, chunk_c0, chunk_lens, num_q_heads, num_kv_
                          np.concatenate([dslots, cslots]).astype(np.int64))
 
 
+def _mixed_lengths(seed, num_decode, num_chunks, decode_lo, decode_hi, c0_hi, full_decode=192):
+    """Decode context lengths, then the chunks' prior contexts c0, from one
+    stream.  The lengths are drawn for at least the full 192-sequence batch and
+    cut to num_decode, so a smaller decode batch (a profiling case) keeps the
+    same chunks."""
+    rng = np.random.default_rng(seed)
+    dl = rng.integers(decode_lo, decode_hi + 1, size=max(num_decode, full_decode))[:num_decode]
+    c0 = rng.integers(0, c0_hi + 1, size=num_chunks)
+    return dl, c0
+
+
 def mixed_step_bf16(device="cpu", num_decode=192, num_chunks=4, chunk_len=512, poison=False, seed=1005,
                     decode_lo=256, decode_hi=32768, c0_hi=8192):
     """192 decode sequences (context U[256, 32768]) plus 4 prefill chunks of 512
     tokens over prior context U[0, 8192]; 32 q heads over 8 KV heads, d 128,
     block 32, bf16."""
-    rng = np.random.default_rng(seed)
-    dl = rng.integers(decode_lo, decode_hi + 1, size=num_decode)
-    c0 = rng.integers(0, c0_hi + 1, size=num_chunks)
+    dl, c0 = _mixed_lengths(seed, num_decode, num_chunks, decode_lo, decode_hi, c0_hi)
     n = np.full(num_chunks, chunk_len)
     return mixed_workload("mixed_step_bf16", dl, c0, n, 32, 8, 128, 32, torch.bfloat16, seed=seed, device=device,
                           poison=poison)
@@ -416,9 +425,7 @@ def mixed_step_fp8(device="cpu", num_decode=192, num_chunks=4, chunk_len=512, po
                    decode_lo=256, decode_hi=32768, c0_hi=8192):
     """The mixed step (192 decode sequences + 4 prefill chunks of 512, 32 q
     heads over 8 KV heads, d 128, block 32, bf16 queries) on E4M3 pools."""
-    rng = np.random.default_rng(seed)
-    dl = rng.integers(decode_lo, decode_hi + 1, size=num_decode)
-    c0 = rng.integers(0, c0_hi + 1, size=num_chunks)
+    dl, c0 = _mixed_lengths(seed, num_decode, num_chunks, decode_lo, decode_hi, c0_hi)
     n = np.full(num_chunks, chunk_len)
     return mixed_workload("mixed_step_fp8", dl, c0, n, 32, 8, 128, 32, torch.bfloat16, seed=seed, device=device,
                           poison=poison, fp8_scales=(FP8_K_SCALE, FP8_V_SCALE))
