@@ -967,8 +967,8 @@ int pkv_paged_attention_prefill_chunk(void* out, const void* query, const void* 
     if (rc) return rc;
 
     const int tile_tokens = 128 / group;
-    const int64_t q_tiles = ceil_div(max_q_len, tile_tokens);
-    const int64_t grid = (int64_t)num_chunks * q_tiles * num_kv_heads;
+    const int64_t tile_pairs = ceil_div(ceil_div(max_q_len, tile_tokens), 2);
+    const int64_t grid = (int64_t)num_chunks * tile_pairs * num_kv_heads;
     if (grid > INT32_MAX) return PKV_EUNSUPPORTED;
 
     pkv::PrefillParams prm;
@@ -983,7 +983,7 @@ int pkv_paged_attention_prefill_chunk(void* out, const void* query, const void* 
     prm.max_blocks_per_seq = max_blocks_per_seq;
     prm.block_size = block_size;
     prm.num_blocks = num_blocks;
-    prm.q_tiles = (int)q_tiles;
+    prm.tile_pairs = (int)tile_pairs;
     prm.out_scale = 1.f;
     const bool bf16 = dtype == PKV_BF16;
     if (head_dim == 64)
@@ -1220,8 +1220,8 @@ int pkv_paged_attention_prefill_chunk_fp8(void* out, const void* query, const vo
     if (rc) return rc;
 
     const int tile_tokens = 128 / group;
-    const int64_t q_tiles = ceil_div(max_q_len, tile_tokens);
-    const int64_t grid = (int64_t)num_chunks * q_tiles * num_kv_heads;
+    const int64_t tile_pairs = ceil_div(ceil_div(max_q_len, tile_tokens), 2);
+    const int64_t grid = (int64_t)num_chunks * tile_pairs * num_kv_heads;
     if (grid > INT32_MAX) return PKV_EUNSUPPORTED;
     pkv::PrefillParams prm;
     prm.out = out;
@@ -1236,7 +1236,7 @@ int pkv_paged_attention_prefill_chunk_fp8(void* out, const void* query, const vo
     prm.max_blocks_per_seq = max_blocks_per_seq;
     prm.block_size = block_size;
     prm.num_blocks = entries;
-    prm.q_tiles = (int)q_tiles;
+    prm.tile_pairs = (int)tile_pairs;
     const bool bf16 = dtype == PKV_BF16;
     if (head_dim == 64)
         return bf16 ? prefill_by_group<__half, 64, __nv_bfloat16>(group, prm, tq, tk, tv, (int)grid, s)

@@ -52,6 +52,12 @@ CASES = [
     (torch.float16, 64, 16, 4, 2, [17], [300]),
     (torch.bfloat16, 128, 16, 16, 2, [255, 64], [200, 16]),
     (torch.float16, 128, 32, 8, 4, [0], [1]),
+    # the first tile of a pair needs one key tile fewer than the second (c0 = 90: rows up to 121 and 153)
+    (torch.bfloat16, 128, 32, 32, 8, [90, 7], [64, 100]),
+    # more chunks than the longest-first ordering handles: the plain launch order
+    (torch.float16, 64, 16, 8, 1, [7 * i for i in range(70)], [1 + i % 3 for i in range(70)]),
+    # chunks of equal length (ties in the longest-first order)
+    (torch.bfloat16, 128, 16, 16, 4, [200, 200, 200], [40, 40, 40]),
 ]
 
 
