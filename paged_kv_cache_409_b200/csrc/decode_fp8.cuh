@@ -197,15 +197,22 @@ __global__ void __launch_bounds__(NW * 32) paged_decode_fp8_kernel(const DecodeP
                 bmA = fmaxf(bmA, __shfl_xor_sync(0xffffffffu, bmA, off));
                 bmB = fmaxf(bmB, __shfl_xor_sync(0xffffffffu, bmB, off));
             }
-            const float mnA = fmaxf(mA, bmA), mnB = fmaxf(mB, bmB);
-            const float alA = exp2f(mA - mnA), alB = exp2f(mB - mnB);
+            // Lazy rescaling: the exponent base (mA, mB) moves, and O and the
+            // sums are rescaled, only when a block's max exceeds it by more than
+            // 2^8; the weights exp2(s - m) then stay below 256, inside f16.
+            const bool rsA = bmA > mA + 8.f || (mA == -INFINITY && bmA != -INFINITY);
+            const bool rsB = bmB > mB + 8.f || (mB == -INFINITY && bmB != -INFINITY);
+            float alA = 1.f, alB = 1.f;
+            if (rsA) alA = ex2_approx(mA - bmA), mA = bmA;  // 0 when mA was -inf
+            if (rsB) alB = ex2_approx(mB - bmB), mB = bmB;
+            const float eA = mA == -INFINITY ? 0.f : mA, eB = mB == -INFINITY ? 0.f : mB;
             float sA = 0.f, sB = 0.f;
 #pragma unroll
             for (int mt = 0; mt < MT; ++mt) {
-                sc[mt][0] = exp2f(sc[mt][0] - mnA);
-                sc[mt][1] = exp2f(sc[mt][1] - mnB);
-                sc[mt][2] = exp2f(sc[mt][2] - mnA);
-                sc[mt][3] = exp2f(sc[mt][3] - mnB);
+                sc[mt][0] = ex2_approx(sc[mt][0] - eA);
+                sc[mt][1] = ex2_approx(sc[mt][1] - eB);
+                sc[mt][2] = ex2_approx(sc[mt][2] - eA);
+                sc[mt][3] = ex2_approx(sc[mt][3] - eB);
                 sA += sc[mt][0] + sc[mt][2];
                 sB += sc[mt][1] + sc[mt][3];
             }
@@ -216,14 +223,14 @@ __global__ void __launch_bounds__(NW * 32) paged_decode_fp8_kernel(const DecodeP
             }
             lA = lA * alA + sA;
             lB = lB * alB + sB;
-            mA = mnA;
-            mB = mnB;
+            if (__any_sync(0xffffffffu, rsA || rsB)) {
 #pragma unroll
-            for (int t = 0; t < KS; ++t) {
-                o[t][0] *= alA;
-                o[t][1] *= alB;
-                o[t][2] *= alA;
-                o[t][3] *= alB;
+                for (int t = 0; t < KS; ++t) {
+                    o[t][0] *= alA;
+                    o[t][1] *= alB;
+                    o[t][2] *= alA;
+                    o[t][3] *= alB;
+                }
             }
             // ---- O^T += V^T . P^T
 #pragma unroll

@@ -244,33 +244,41 @@ __global__ void __launch_bounds__(NW * 32) paged_decode_multi_kernel(const Multi
                     bm[h] = fmaxf(bm[h], s[nt][e]);
                 }
             }
-            float alpha[2], msafe[2];
+            // Lazy rescaling: a row's exponent base m moves, and its O and sum
+            // are rescaled, only when a unit's max exceeds it by more than 2^8;
+            // the weights exp2(s - m) then stay below 256 (bf16 / f16 P).
+            float alpha[2] = {1.f, 1.f}, msafe[2];
+            bool rs = false;
 #pragma unroll
             for (int h = 0; h < 2; ++h) {
                 bm[h] = fmaxf(bm[h], __shfl_xor_sync(0xffffffffu, bm[h], 1));
                 bm[h] = fmaxf(bm[h], __shfl_xor_sync(0xffffffffu, bm[h], 2));
-                const float mn = fmaxf(m[h], bm[h]);
-                msafe[h] = mn == -INFINITY ? 0.f : mn;  // a row with no key yet stays empty
-                alpha[h] = exp2f(m[h] - msafe[h]);
-                m[h] = mn;
+                if (bm[h] > m[h] + 8.f || (m[h] == -INFINITY && bm[h] != -INFINITY)) {
+                    alpha[h] = ex2_approx(m[h] - bm[h]);  // 0 when m was -inf
+                    m[h] = bm[h];
+                    rs = true;
+                }
+                msafe[h] = m[h] == -INFINITY ? 0.f : m[h];  // a row with no key yet stays empty
             }
             float ps[2] = {0.f, 0.f};
 #pragma unroll
             for (int nt = 0; nt < 2; ++nt) {
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
-                    s[nt][e] = exp2f(s[nt][e] - msafe[e >> 1]);
+                    s[nt][e] = ex2_approx(s[nt][e] - msafe[e >> 1]);
                     ps[e >> 1] += s[nt][e];
                 }
             }
             l[0] = l[0] * alpha[0] + ps[0];  // per-lane partial row sums; the quad is summed at the end
             l[1] = l[1] * alpha[1] + ps[1];
+            if (__any_sync(0xffffffffu, rs)) {
 #pragma unroll
-            for (int j = 0; j < DT; ++j) {
-                o[j][0] *= alpha[0];
-                o[j][1] *= alpha[0];
-                o[j][2] *= alpha[1];
-                o[j][3] *= alpha[1];
+                for (int j = 0; j < DT; ++j) {
+                    o[j][0] *= alpha[0];
+                    o[j][1] *= alpha[0];
+                    o[j][2] *= alpha[1];
+                    o[j][3] *= alpha[1];
+                }
             }
             // ---- O += P . V  (P: the S accumulators in the A layout; bf16 as hi + lo)
             uint32_t pa[4], pl[4] = {0u, 0u, 0u, 0u};
