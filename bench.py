@@ -396,10 +396,15 @@ class MultiTokenStep:
 # launch(es).
 TRAFFIC_CAPTURES = {
     "llama7b_decode_f16": {"case": "paged_decode_mma_kernel, the llama7b batch cut to 16 sequences",
-                           "read_mb": 287.471104, "write_mb": 3.418624, "algorithmic_mb": 285.38096},
-    "llama7b_decode_fp8": {"case": "paged_decode_fp8_kernel + merge, the 64-sequence llama7b batch on E4M3 pools",
-                           "read_mb": 305.044224 + 1.388544, "write_mb": 3.7632 + 0.0,
-                           "algorithmic_mb": 303.293524},
+                           "read_mb": 287.470592, "write_mb": 3.234304, "algorithmic_mb": 285.38096},
+    "mixed_step_bf16": {"case": "paged_decode_mma_kernel, the mixed step's decode cut to 8 sequences",
+                        "read_mb": 575.334656, "write_mb": 3.36512, "algorithmic_mb": 574.8748},
+    "multi_token_decode_bf16": {"case": "paged_decode_multi_kernel, the multi-token batch cut to 32 sequences",
+                                "read_mb": 281.808896, "write_mb": 6.08384, "algorithmic_mb": 281.830028},
+    # the whole workload was captured (its distinct blocks fit the capture size rule): not scaled
+    "shared_prefix_decode_f16": {"case": "paged_decode_mma_kernel, the whole shared-prefix workload",
+                                 "read_mb": 155.911168, "write_mb": 3.894784, "algorithmic_mb": 3227.190064,
+                                 "whole": True},
 }
 
 
@@ -963,10 +968,13 @@ def main():
     if hasattr(step, "config"):
         line["config"].update(step.config())
     if args.config in TRAFFIC_CAPTURES and not args.seqs:
-        line["roofline"]["traffic"] = traffic_ratio(args.config) * step.decode_bytes  # DRAM bytes per decode call
+        cap = TRAFFIC_CAPTURES[args.config]
+        # DRAM bytes per decode call
+        line["roofline"]["traffic"] = ((cap["read_mb"] + cap["write_mb"]) * 1e6 if cap.get("whole") else
+                                       traffic_ratio(args.config) * step.decode_bytes)
         line["roofline"]["traffic_unit"] = "bytes per launch"
-        line["roofline"]["traffic_source"] = ("ncu DRAM bytes of " + TRAFFIC_CAPTURES[args.config]["case"] +
-                                              ", scaled by algorithmic bytes")
+        line["roofline"]["traffic_source"] = "ncu DRAM bytes of " + cap["case"] + (
+            "" if cap.get("whole") else ", scaled by algorithmic bytes")
     if getattr(step, "unique_kv_bytes", None) and 2 * step.unique_kv_bytes < step.kv_bytes * step.layers:
         # shared blocks: most logical bytes come from L2, so the HBM fraction above exceeds 1 by design
         uniq = step.unique_kv_bytes / step.layers

@@ -60,8 +60,11 @@ def test_traffic_ratios_are_the_captured_dram_bytes_over_algorithmic_bytes():
     for cfg, cap in bench.TRAFFIC_CAPTURES.items():
         ratio = bench.traffic_ratio(cfg)
         assert ratio == (cap["read_mb"] + cap["write_mb"]) / cap["algorithmic_mb"]
-        assert 1.0 <= ratio < 1.1, cfg
         assert cap["case"] and "profiles" not in cap["case"]
+        if cap.get("whole"):  # shared blocks: DRAM sees the distinct bytes once, far below the logical bytes
+            assert ratio < 0.1, cfg
+        else:
+            assert 1.0 <= ratio < 1.1, cfg
 
 
 def test_reference_arm_loads_only_the_oracle():
