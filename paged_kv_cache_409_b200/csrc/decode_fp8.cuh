@@ -41,8 +41,13 @@ struct DecodeFp8Cfg {
     static size_t smem_bytes(int pb) { return 1024 + BT_OFF + static_cast<size_t>(pb) * 4 + 16 + NW * NST * 8; }
 };
 
+// Resident CTAs per SM the register allocation must allow (launch bounds).
+#ifndef PKV_FP8_MIN_CTAS
+#define PKV_FP8_MIN_CTAS 1
+#endif
+
 template <typename T, int B, int G, int NST, int NW>
-__global__ void __launch_bounds__(NW * 32) paged_decode_fp8_kernel(const DecodeParams p,
+__global__ void __launch_bounds__(NW * 32, PKV_FP8_MIN_CTAS) paged_decode_fp8_kernel(const DecodeParams p,
                                                                    const __grid_constant__ CUtensorMap tm_k,
                                                                    const __grid_constant__ CUtensorMap tm_v) {
     using C = DecodeFp8Cfg<B, G, NST, NW>;

@@ -65,8 +65,13 @@ struct MultiCfg {
     static size_t smem_bytes(int pb) { return 1024 + BT_OFF + static_cast<size_t>(pb) * 4 + 16 + 2 * NW * NST * 8; }
 };
 
+// Resident CTAs per SM the register allocation must allow (launch bounds).
+#ifndef PKV_MULTI_MIN_CTAS
+#define PKV_MULTI_MIN_CTAS 1
+#endif
+
 template <typename T, int D, int B, int NST, int NW, int RG>
-__global__ void __launch_bounds__(NW * 32) paged_decode_multi_kernel(const MultiParams p, const int G,
+__global__ void __launch_bounds__(NW * 32, PKV_MULTI_MIN_CTAS) paged_decode_multi_kernel(const MultiParams p, const int G,
                                                                      const __grid_constant__ CUtensorMap tm_k,
                                                                      const __grid_constant__ CUtensorMap tm_v) {
     using C = MultiCfg<T, D, B, NST, NW, RG>;

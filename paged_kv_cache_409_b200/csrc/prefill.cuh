@@ -162,6 +162,17 @@ __device__ __forceinline__ bool prefill_item(const int32_t* seq_lens, const int3
     return true;
 }
 
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+    float d;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+    return d;
+}
+__device__ __forceinline__ float fmin3(float a, float b, float c) {
+    float d;
+    asm("min.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+    return d;
+}
+
 // T: the type of the query and the K/V tiles the MMAs read; TO: the output's.
 template <typename T, int D, int G, typename TO = T>
 __global__ void __launch_bounds__(kPrefillThreads, 1) paged_prefill_kernel(const PrefillParams p,
@@ -422,18 +433,19 @@ __global__ void __launch_bounds__(kPrefillThreads, 1) paged_prefill_kernel(const
             // into the exponent's FMA), scaled scores with -inf masks otherwise
             float mrow;
             if (all_vis) {
+                // four independent chains of 3-input max (min for a negative scale)
                 float r0 = sv[0], r1 = sv[1], r2 = sv[2], r3 = sv[3];
                 if (sl2 >= 0.f) {
 #pragma unroll
-                    for (int i = 4; i < C::BN; i += 4)
-                        r0 = fmaxf(r0, sv[i]), r1 = fmaxf(r1, sv[i + 1]), r2 = fmaxf(r2, sv[i + 2]),
-                        r3 = fmaxf(r3, sv[i + 3]);
+                    for (int i = 4; i < C::BN; i += 8)
+                        r0 = fmax3(r0, sv[i], sv[i + 4]), r1 = fmax3(r1, sv[i + 1], sv[i + 5]),
+                        r2 = fmax3(r2, sv[i + 2], sv[i + 6]), r3 = fmax3(r3, sv[i + 3], sv[i + 7]);
                     mrow = fmaxf(fmaxf(r0, r1), fmaxf(r2, r3)) * sl2;
                 } else {
 #pragma unroll
-                    for (int i = 4; i < C::BN; i += 4)
-                        r0 = fminf(r0, sv[i]), r1 = fminf(r1, sv[i + 1]), r2 = fminf(r2, sv[i + 2]),
-                        r3 = fminf(r3, sv[i + 3]);
+                    for (int i = 4; i < C::BN; i += 8)
+                        r0 = fmin3(r0, sv[i], sv[i + 4]), r1 = fmin3(r1, sv[i + 1], sv[i + 5]),
+                        r2 = fmin3(r2, sv[i + 2], sv[i + 6]), r3 = fmin3(r3, sv[i + 3], sv[i + 7]);
                     mrow = fminf(fminf(r0, r1), fminf(r2, r3)) * sl2;
                 }
             } else {
@@ -456,15 +468,17 @@ __global__ void __launch_bounds__(kPrefillThreads, 1) paged_prefill_kernel(const
             const float mexp = m_used == -INFINITY ? 0.f : m_used;
             const float smul = all_vis ? sl2 : 1.f;  // the exponent is sv * smul - m
             // ---- P = exp2(S - m_used) over the S columns, 32 keys at a time
-            float ts4[4] = {0.f, 0.f, 0.f, 0.f};
+            // (packed f32x2 arithmetic: the exponent arguments and the row sum)
+            float2 acc[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+            const float2 smul2 = make_float2(smul, smul), nm2 = make_float2(-mexp, -mexp);
 #pragma unroll
             for (int c = 0; c < C::BN / 32; ++c) {
                 uint32_t hi[16], lo[16];
 #pragma unroll
                 for (int i = 0; i < 32; i += 2) {
-                    const float p0 = ex2_approx(fmaf(sv[c * 32 + i], smul, -mexp));
-                    const float p1 = ex2_approx(fmaf(sv[c * 32 + i + 1], smul, -mexp));
-                    ts4[(i / 2) & 3] += p0 + p1;
+                    const float2 arg = __ffma2_rn(make_float2(sv[c * 32 + i], sv[c * 32 + i + 1]), smul2, nm2);
+                    const float p0 = ex2_approx(arg.x), p1 = ex2_approx(arg.y);
+                    acc[(i / 2) & 1] = __fadd2_rn(acc[(i / 2) & 1], make_float2(p0, p1));
                     if constexpr (C::SPLIT_P) {
                         // hi = p truncated to bf16 (its top 16 bits); lo = the exact
                         // remainder rounded to bf16, |lo| < 2^-7 |p|
@@ -479,7 +493,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1) paged_prefill_kernel(const
                 tmem_st16_nowait(ts + c * 16, hi);
                 if constexpr (C::SPLIT_P) tmem_st16_nowait(ts + C::PLO + c * 16, lo);
             }
-            lsum = lsum * alpha + ((ts4[0] + ts4[1]) + (ts4[2] + ts4[3]));
+            lsum = lsum * alpha + ((acc[0].x + acc[0].y) + (acc[1].x + acc[1].y));
             // ---- O *= alpha once P.V of the previous tile is done (the next
             // P.V accumulates on top of it)
             if (j >= 1 && __any_sync(0xffffffffu, rescale && alpha != 1.f)) {
