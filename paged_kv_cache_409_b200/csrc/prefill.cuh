@@ -325,28 +325,37 @@ __global__ void __launch_bounds__(kPrefillThreads, 1) paged_prefill_kernel(const
         if ((tid & 31) == 0) {
             constexpr uint32_t IDESC_S = umma_idesc_f16(128, C::BN, kBf16, false, false);
             constexpr uint32_t IDESC_O = umma_idesc_f16(128, D, kBf16, false, true);
+            // Shared-memory descriptors of every operand tile, made once: a
+            // 16-element k slice is the tile's descriptor plus its byte offset / 16
+            // (the start-address field), so issuing an MMA costs a few
+            // instructions -- one thread issues fast enough for the tensor pipe
+            // only without per-MMA descriptor arithmetic.
+            uint64_t qdesc[2], kdesc[2], vdesc[2];
+#pragma unroll
+            for (int i = 0; i < 2; ++i) {
+                qdesc[i] = smem_desc_sw128(smem_u32(smem + C::Q_OFF + i * C::Q_BYTES), 16, 1024);
+                kdesc[i] = smem_desc_sw128(smem_u32(smem + C::K_OFF + i * C::KT_BYTES), 16, 1024);
+                vdesc[i] = smem_desc_sw128(smem_u32(smem + C::V_OFF + i * C::KT_BYTES), C::BN * 128, 1024);
+            }
             auto issue_s = [&](int x, int t) {  // S_x(t) = Q_x . K_t^T
-                const uint32_t q_addr = smem_u32(smem + C::Q_OFF + x * C::Q_BYTES);
-                const uint32_t k_addr = smem_u32(smem + C::K_OFF + (t & 1) * C::KT_BYTES);
+                const uint64_t qd = qdesc[x], kd = kdesc[t & 1];
                 const uint32_t s_col = C::S_COL0 + 128 * x;
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {
-                    const uint32_t qoff = (kk / 4) * (C::BM * 128) + (kk % 4) * 32;
-                    const uint32_t koff = (kk / 4) * (C::BN * 128) + (kk % 4) * 32;
-                    umma_f16_ss(tmem + s_col, smem_desc_sw128(q_addr + qoff, 16, 1024),
-                                smem_desc_sw128(k_addr + koff, 16, 1024), IDESC_S, kk > 0);
+                    constexpr int kQ = C::BM * 128 / 16, kK = C::BN * 128 / 16;  // panel strides / 16
+                    umma_f16_ss(tmem + s_col, qd + (kk / 4) * kQ + (kk % 4) * 2, kd + (kk / 4) * kK + (kk % 4) * 2,
+                                IDESC_S, kk > 0);
                 }
                 umma_commit(&s_full[x]);
             };
             auto issue_pv = [&](int x, int t) {  // O_x += P_x(t) . V_t, P from tensor memory
-                const uint32_t v_addr = smem_u32(smem + C::V_OFF + (t & 1) * C::KT_BYTES);
+                const uint64_t vd = vdesc[t & 1];
                 const uint32_t p_col = C::S_COL0 + 128 * x, o_col = C::O_COL0 + D * x;
 #pragma unroll
                 for (int kk = 0; kk < C::BN / 16; ++kk) {
-                    const uint64_t vdesc = smem_desc_sw128(v_addr + kk * 16 * 128, C::BN * 128, 1024);
-                    umma_f16_ts(tmem + o_col, tmem + p_col + kk * 8, vdesc, IDESC_O, t > 0 || kk > 0);
-                    if constexpr (C::SPLIT_P)
-                        umma_f16_ts(tmem + o_col, tmem + p_col + C::PLO + kk * 8, vdesc, IDESC_O, 1);
+                    const uint64_t v = vd + kk * (16 * 128 / 16);  // 16 key rows of 128 bytes
+                    umma_f16_ts(tmem + o_col, tmem + p_col + kk * 8, v, IDESC_O, t > 0 || kk > 0);
+                    if constexpr (C::SPLIT_P) umma_f16_ts(tmem + o_col, tmem + p_col + C::PLO + kk * 8, v, IDESC_O, 1);
                 }
                 umma_commit(&o_full[x]);
             };
