@@ -191,7 +191,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1) paged_prefill_kernel(const
     uint64_t* v_free = bars + 7;   // [2]  the P.V MMAs that read the stage are done
     uint64_t* s_full = bars + 9;   // [2]  per tile: S_x(j) done
     uint64_t* p_full = bars + 11;  // [2]  per tile: P_x(j) written (128 arrivals)
-    uint64_t* o_full = bars + 13;  // [2]  per tile: PV_x(j) done
+    uint64_t* o_full = bars + 13;  // [2]  per tile: the tile's last P.V done
     uint64_t* mma_done = bars + 15;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 16);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + 17);
@@ -348,7 +348,11 @@ __global__ void __launch_bounds__(kPrefillThreads, 1) paged_prefill_kernel(const
                 }
                 umma_commit(&s_full[x]);
             };
-            auto issue_pv = [&](int x, int t) {  // O_x += P_x(t) . V_t, P from tensor memory
+            // O_x += P_x(t) . V_t, P from tensor memory.  Only the tile's last
+            // P.V is committed on its own (for the epilogue): the commit of
+            // S_x(t + 1), issued after PV_x(t), also tells the softmax that O_x
+            // holds every P.V before it.
+            auto issue_pv = [&](int x, int t, bool last) {
                 const uint64_t vd = vdesc[t & 1];
                 const uint32_t p_col = C::S_COL0 + 128 * x, o_col = C::O_COL0 + D * x;
 #pragma unroll
@@ -357,7 +361,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1) paged_prefill_kernel(const
                     umma_f16_ts(tmem + o_col, tmem + p_col + kk * 8, v, IDESC_O, t > 0 || kk > 0);
                     if constexpr (C::SPLIT_P) umma_f16_ts(tmem + o_col, tmem + p_col + C::PLO + kk * 8, v, IDESC_O, 1);
                 }
-                umma_commit(&o_full[x]);
+                if (last) umma_commit(&o_full[x]);
             };
             bool ok = mbar_wait_or_abort(q_full, 0, abort_flag) && mbar_wait_or_abort(&k_full[0], 0, abort_flag);
             if (ok) {
@@ -376,7 +380,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1) paged_prefill_kernel(const
                     ok = mbar_wait_or_abort(&p_full[x], t & 1, abort_flag);
                     if (!ok) break;
                     tc_fence_after();
-                    issue_pv(x, t);
+                    issue_pv(x, t, t + 1 == nk);
                     if (t + 1 < nk) {
                         if (!k_next) {
                             ok = k_next = mbar_wait_or_abort(&k_full[(t + 1) & 1], ((t + 1) >> 1) & 1, abort_flag);
@@ -503,14 +507,9 @@ __global__ void __launch_bounds__(kPrefillThreads, 1) paged_prefill_kernel(const
                 if constexpr (C::SPLIT_P) tmem_st16_nowait(ts + C::PLO + c * 16, lo);
             }
             lsum = lsum * alpha + ((acc[0].x + acc[0].y) + (acc[1].x + acc[1].y));
-            // ---- O *= alpha once P.V of the previous tile is done (the next
-            // P.V accumulates on top of it)
+            // ---- O *= alpha: P.V of the previous tile is done (S_j, committed
+            // after it, was), and the next P.V accumulates on top of it
             if (j >= 1 && __any_sync(0xffffffffu, rescale && alpha != 1.f)) {
-                if (!__all_sync(0xffffffffu, mbar_wait_or_abort(&o_full[x], (j - 1) & 1, abort_flag))) {
-                    ok = false;
-                    break;
-                }
-                tc_fence_after();
 #pragma unroll
                 for (int c = 0; c < D / 32; ++c) {  // warp-collective: lanes without a rescale store O back as is
                     float v[32];
@@ -545,8 +544,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1) paged_prefill_kernel(const
             mbar_arrive(&p_full[x]);
         }
         if (ok && nk > 0) {
-            const int jl = nk - 1;
-            if (__all_sync(0xffffffffu, mbar_wait_or_abort(&o_full[x], jl & 1, abort_flag))) {
+            if (__all_sync(0xffffffffu, mbar_wait_or_abort(&o_full[x], 0, abort_flag))) {
                 tc_fence_after();
                 const bool live = tok < n && !*abort_flag;
                 const float inv = p.out_scale / lsum;
