@@ -94,7 +94,32 @@ __global__ void __launch_bounds__(NW * 32, PKV_FP8_MIN_CTAS) paged_decode_fp8_ke
         fence_mbar_init();
     }
 
-    // Q^T fragments (B operand, f16): head lane/4, dims 16 ks + 4 (lane%4) + {0,1} | {2,3}.
+    __syncthreads();
+
+    const int nw = nb > warp ? (nb - warp + NW - 1) / NW : 0;
+    uint8_t* wstage = smem + warp * NST * C::STAGE;
+    uint64_t* wbar = bars + warp * NST;
+    const uint64_t policy = l2_policy_evict_first();
+
+    auto issue = [&](int k) {  // lane 0 only
+        const int st = k % NST;
+        const int id = bt_s[warp + k * NW];
+        const int coord = id >= 0 ? id : static_cast<int>(p.num_blocks);  // out of range: zero fill
+        uint8_t* kd = wstage + st * C::STAGE;
+        mbar_arrive_expect_tx(&wbar[st], C::STAGE);
+        tma_load_4d_hint(kd, &tm_k, 0, g, 0, coord, &wbar[st], policy);
+        tma_load_4d_hint(kd + C::TILE, &tm_v, 0, g, 0, coord, &wbar[st], policy);
+    };
+    // Everything above reads only the tables and the lengths; the
+    // pools may still be in the writes of a grid this one depends on (the
+    // append of a decode step), so their loads start after it completes.
+    griddep_wait();
+    if (lane == 0) {
+        for (int k = 0; k < NST && k < nw; ++k) issue(k);
+    }
+    __syncwarp();
+    // Q^T fragments (B operand, f16), loaded while the first stages are in
+    // flight: head lane/4, dims 16 ks + 4 (lane%4) + {0,1} | {2,3}.
     uint32_t qf[KS][2];
     {
         const int hq = lane >> 2, k4 = 4 * (lane & 3);
@@ -112,30 +137,6 @@ __global__ void __launch_bounds__(NW * 32, PKV_FP8_MIN_CTAS) paged_decode_fp8_ke
             }
         }
     }
-    __syncthreads();
-
-    const int nw = nb > warp ? (nb - warp + NW - 1) / NW : 0;
-    uint8_t* wstage = smem + warp * NST * C::STAGE;
-    uint64_t* wbar = bars + warp * NST;
-    const uint64_t policy = l2_policy_evict_first();
-
-    auto issue = [&](int k) {  // lane 0 only
-        const int st = k % NST;
-        const int id = bt_s[warp + k * NW];
-        const int coord = id >= 0 ? id : static_cast<int>(p.num_blocks);  // out of range: zero fill
-        uint8_t* kd = wstage + st * C::STAGE;
-        mbar_arrive_expect_tx(&wbar[st], C::STAGE);
-        tma_load_4d_hint(kd, &tm_k, 0, g, 0, coord, &wbar[st], policy);
-        tma_load_4d_hint(kd + C::TILE, &tm_v, 0, g, 0, coord, &wbar[st], policy);
-    };
-    // Everything above reads only the query, the tables and the lengths; the
-    // pools may still be in the writes of a grid this one depends on (the
-    // append of a decode step), so their loads start after it completes.
-    griddep_wait();
-    if (lane == 0) {
-        for (int k = 0; k < NST && k < nw; ++k) issue(k);
-    }
-    __syncwarp();
 
     float mA = -INFINITY, mB = -INFINITY, lA = 0.f, lB = 0.f;
     // O^T: [chunk t][c0: (dim 16t + 2(lane/4), hA), c1: (same dim, hB), c2: (dim + 1, hA), c3: (dim + 1, hB)]

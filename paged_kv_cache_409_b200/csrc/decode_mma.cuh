@@ -72,18 +72,6 @@ __global__ void __launch_bounds__(NW * 32) paged_decode_mma_kernel(const DecodeP
         fence_mbar_init();
     }
 
-    // Q^T fragments (B operand): this lane holds head lane/4, dims 2(lane%4)+{0,1} (+8) of every 16-dim step.
-    uint32_t qf[KS][2];
-    {
-        const int hq = lane >> 2, kq = 2 * (lane & 3);
-        const T* qrow = reinterpret_cast<const T*>(p.query) +
-                        (static_cast<int64_t>(s) * p.num_q_heads + static_cast<int64_t>(g) * G + hq) * D;
-#pragma unroll
-        for (int ks = 0; ks < KS; ++ks) {
-            qf[ks][0] = hq < G ? *reinterpret_cast<const uint32_t*>(qrow + 16 * ks + kq) : 0u;
-            qf[ks][1] = hq < G ? *reinterpret_cast<const uint32_t*>(qrow + 16 * ks + 8 + kq) : 0u;
-        }
-    }
     __syncthreads();
 
     const int nw = nb > warp ? (nb - warp + kDecodeWarps - 1) / kDecodeWarps : 0;
@@ -104,7 +92,7 @@ __global__ void __launch_bounds__(NW * 32) paged_decode_mma_kernel(const DecodeP
             tma_load_4d_hint(vd + pn * B * 128, &tm_v, pn * C::PANEL, g, 0, coord, &wbar[st], policy);
         }
     };
-    // Everything above reads only the query, the tables and the lengths; the
+    // Everything above reads only the tables and the lengths; the
     // pools may still be in the writes of a grid this one depends on (the
     // append of a decode step), so their loads start after it completes.
     griddep_wait();
@@ -112,6 +100,19 @@ __global__ void __launch_bounds__(NW * 32) paged_decode_mma_kernel(const DecodeP
         for (int k = 0; k < NST && k < nw; ++k) issue(k);
     }
     __syncwarp();
+    // Q^T fragments (B operand), loaded while the first stages are in flight:
+    // this lane holds head lane/4, dims 2(lane%4)+{0,1} (+8) of every 16-dim step.
+    uint32_t qf[KS][2];
+    {
+        const int hq = lane >> 2, kq = 2 * (lane & 3);
+        const T* qrow = reinterpret_cast<const T*>(p.query) +
+                        (static_cast<int64_t>(s) * p.num_q_heads + static_cast<int64_t>(g) * G + hq) * D;
+#pragma unroll
+        for (int ks = 0; ks < KS; ++ks) {
+            qf[ks][0] = hq < G ? *reinterpret_cast<const uint32_t*>(qrow + 16 * ks + kq) : 0u;
+            qf[ks][1] = hq < G ? *reinterpret_cast<const uint32_t*>(qrow + 16 * ks + 8 + kq) : 0u;
+        }
+    }
 
     // Columns of S^T held by this lane: heads hA = 2(lane%4) and hB = hA + 1.
     float mA = -INFINITY, mB = -INFINITY, lA = 0.f, lB = 0.f;

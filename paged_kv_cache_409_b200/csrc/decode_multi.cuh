@@ -65,9 +65,12 @@ struct MultiCfg {
     static size_t smem_bytes(int pb) { return 1024 + BT_OFF + static_cast<size_t>(pb) * 4 + 16 + 2 * NW * NST * 8; }
 };
 
-// Resident CTAs per SM the register allocation must allow (launch bounds).
+// Resident CTAs per SM the register allocation must allow (launch bounds):
+// three 4-warp CTAs (168 registers) -- left free, the compiler takes 203 and
+// two CTAs fit, 10 % slower on the multi-token batch; a fourth CTA (128
+// registers) spills and is slower still.
 #ifndef PKV_MULTI_MIN_CTAS
-#define PKV_MULTI_MIN_CTAS 1
+#define PKV_MULTI_MIN_CTAS 3
 #endif
 
 template <typename T, int D, int B, int NST, int NW, int RG>
@@ -138,24 +141,6 @@ __global__ void __launch_bounds__(NW * 32, PKV_MULTI_MIN_CTAS) paged_decode_mult
         }
         fence_mbar_init();
     }
-    const int gq = lane >> 2, cq = lane & 3;
-    int lim[2];  // last key position each of the lane's two rows may see
-    uint32_t qa[KS][4];
-#pragma unroll
-    for (int h = 0; h < 2; ++h) {
-        const int row = 16 * rg + gq + 8 * h;
-        const int i = row / G, hh = row - (row / G) * G;
-        lim[h] = c0 + min(i, n - 1);
-        const bool live = i < n;
-        const T* qrow = reinterpret_cast<const T*>(p.query) +
-                        ((static_cast<int64_t>(q0) + (live ? i : 0)) * p.num_q_heads + static_cast<int64_t>(g) * G +
-                         hh) * D;
-#pragma unroll
-        for (int ks = 0; ks < KS; ++ks) {
-            qa[ks][h] = live ? *reinterpret_cast<const uint32_t*>(qrow + 16 * ks + 2 * cq) : 0u;
-            qa[ks][h + 2] = live ? *reinterpret_cast<const uint32_t*>(qrow + 16 * ks + 8 + 2 * cq) : 0u;
-        }
-    }
     __syncthreads();
 
     // units (16-token sub-blocks) holding positions [b0 * B, min(len, (b0 + nb) * B))
@@ -187,6 +172,25 @@ __global__ void __launch_bounds__(NW * 32, PKV_MULTI_MIN_CTAS) paged_decode_mult
         for (; issued < ring && issued < nw; ++issued) issue(issued);
     }
     __syncwarp();
+    // The query fragments load while the first stages are in flight.
+    const int gq = lane >> 2, cq = lane & 3;
+    int lim[2];  // last key position each of the lane's two rows may see
+    uint32_t qa[KS][4];
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+        const int row = 16 * rg + gq + 8 * h;
+        const int i = row / G, hh = row - (row / G) * G;
+        lim[h] = c0 + min(i, n - 1);
+        const bool live = i < n;
+        const T* qrow = reinterpret_cast<const T*>(p.query) +
+                        ((static_cast<int64_t>(q0) + (live ? i : 0)) * p.num_q_heads + static_cast<int64_t>(g) * G +
+                         hh) * D;
+#pragma unroll
+        for (int ks = 0; ks < KS; ++ks) {
+            qa[ks][h] = live ? *reinterpret_cast<const uint32_t*>(qrow + 16 * ks + 2 * cq) : 0u;
+            qa[ks][h + 2] = live ? *reinterpret_cast<const uint32_t*>(qrow + 16 * ks + 8 + 2 * cq) : 0u;
+        }
+    }
 
     float m[2] = {-INFINITY, -INFINITY}, l[2] = {0.f, 0.f};
     float o[DT][4];  // [dim tile j][c0: (row rq, dim 8j + 2cq), c1: +1, c2: (row rq + 8, dim 8j + 2cq), c3: +1]
