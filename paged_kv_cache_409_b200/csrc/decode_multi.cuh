@@ -5,23 +5,50 @@
 // chunk with c0 = seq_len - n prior tokens attends causally to keys
 // j <= c0 + i -- the chunked-prefill definition, for chunks of a few tokens.
 //
-// With n * G query rows per KV head (G query heads share one), the work per
-// K/V byte is 4 * n * G flops: too little for tcgen05's 128-row tiles (the
-// prefill kernel spends its time in the per-tile softmax of 128 rows of which
-// n * G are live) and too much for the CUDA cores.  The rows therefore go to
-// the M side of warp MMAs (mma.sync m16n8k16, fp32 accumulation), 16 rows per
-// warp, in the usual register layout of attention kernels on warp MMAs:
-//   S [16 rows x 16 keys]  = Q [16 x D] . K^T       (B: ldmatrix of the K tile)
-//   O [16 rows x D]       += P [16 x 16 keys] . V   (A: S accumulators reused,
-//                                                     B: ldmatrix.trans of V)
-// Rows are (token, head) pairs, token-major: row r = i * G + hh.  A CTA serves
-// one (chunk, partition, KV head); its warps form one row group of 16 rows per
-// 16 live rows (at most RG) and NW / groups streams, each warp with its own
-// TMA pipeline over the 16-token units (sub-blocks) of its stream, and its own
-// online-softmax state.  Warps of
-// one row group merge in shared memory; the CTA writes output rows (one
-// partition) or partials for the merge kernel, which combines partitions as
-// the decode merge does.
+// A KV head serves R = n * G query rows (token-major: row r = i * G + hh),
+// at most 32.  That is far below the 128-row M of a tcgen05 MMA, so the keys
+// go on M and the rows on N, on the 5th-generation tensor cores:
+//   S^T [128 keys x 32 rows] = K [128 keys x D] . Q^T        (A: the K tile,
+//                                                             B: the Q rows)
+//   O^T [D x 32 rows]       += V^T [D x 128 keys] . P^T      (A: the V tile read
+//                                                             MN-major, B: P^T)
+// S^T and O^T live in tensor memory (lane = key, resp. lane = head_dim
+// element; column = query row).  The tensor cores then do 4 flops per K/V
+// element per row in 24 (bf16: 40) instructions per 128-key tile, and the
+// kernel is bound by streaming K/V from HBM.
+//
+// Persistent grid: one CTA per SM takes work items (chunk, partition, KV
+// head) by rank blockIdx.x, blockIdx.x + gridDim.x, ...; its loader streams
+// the K/V tiles of consecutive items through one ring, so an item's epilogue
+// overlaps the next item's loads.  With at most kMultiLptChunks chunks the
+// ranks go longest first (every full partition, then the chunks' shorter
+// last partitions by key tiles, descending); else partition-major.
+//
+// Roles, by warp (kMultiRowGroups = 2: 16 warps, 512 threads):
+//  * softmax warps (4 per row group) -- TMEM lane t (key t of a tile for
+//    S^T) belongs to warp t / 32 of each row group; a row group takes
+//    32 / kMultiRowGroups of the 32 rows.  For key tile j: read the key's
+//    scores, mask them (causal limit, context end), and vote: when any score
+//    exceeds its row's exponent base by more than 2^8 (lazy rescaling; always
+//    on an item's first tile), the tile's row maxima are reduced across the
+//    128 keys (warp shuffles + shared memory), the bases move and O^T is
+//    rescaled in tensor memory.  Then P = exp2(s - m) goes to shared memory
+//    as P^T (bf16: hi + lo terms), and per-thread partial row sums accumulate.
+//    After the item's last tile the row sums are reduced the same way and
+//    handed, with the rows' exponent bases, to the epilogue warps.
+//  * K loader -- per item the Q rows (one TMA box per 64 dims), then the K
+//    tiles (one box per physical block and 64 dims) into three stages;
+//    V loader (the last warp) -- the V tiles into two.
+//  * S issuer, P.V issuer (lane 0 each) -- the S^T MMAs of each tile as soon
+//    as its K stage and S buffer are ready; the P.V MMAs as soon as P^T and
+//    the V stage are.  The softmax of tile j runs while S(j+1) and PV(j-1) run.
+//  * 4 epilogue warps, thread t = O^T lane t -- after the item's last P.V,
+//    element t of every row (or of the partition's partial, for the merge
+//    kernel), while the softmax goes on with the next item.
+// Every wait is bounded; a wait that gives up raises a CTA-wide abort flag,
+// the softmax warps leave their loop together (their named barriers stay
+// matched), and every role waits (bounded) for the copies / MMAs it issued
+// before tensor memory is released.
 #pragma once
 
 #include "decode.cuh"
@@ -30,7 +57,6 @@ namespace pkv {
 
 struct MultiParams {
     void* out;                       // [total_q_tokens, Hq, D]
-    const void* query;               // [total_q_tokens, Hq, D]
     const int32_t* block_tables;     // [num_chunks, max_blocks_per_seq]
     const int32_t* seq_lens;         // [num_chunks]
     const int32_t* query_start_loc;  // [num_chunks + 1]
@@ -41,6 +67,8 @@ struct MultiParams {
     int num_chunks;
     int num_q_heads;
     int num_kv_heads;
+    int group;  // G = num_q_heads / num_kv_heads; n * G <= 32 rows per chunk
+    int block_size;
     int max_blocks_per_seq;
     int64_t num_blocks;
     int partition_blocks;
@@ -48,369 +76,794 @@ struct MultiParams {
     int64_t total_q_tokens;
 };
 
-template <typename T, int D, int B, int NST, int NW, int RG>
+// Softmax warps per TMEM lane quadrant, each with 32 / kMultiRowGroups of the 32 rows.
+#ifndef PKV_MULTI_ROW_GROUPS
+#define PKV_MULTI_ROW_GROUPS 4
+#endif
+constexpr int kMultiRowGroups = PKV_MULTI_ROW_GROUPS;
+constexpr int kMultiRPT = 32 / kMultiRowGroups;  // rows per softmax thread
+constexpr int kMultiSoftmaxWarps = 4 * kMultiRowGroups;
+constexpr int kMultiSoftmaxThreads = kMultiSoftmaxWarps * 32;
+static_assert(kMultiRowGroups == 2 || kMultiRowGroups == 4, "row groups");
+constexpr int kMultiLoadWarp = kMultiSoftmaxWarps;
+constexpr int kMultiMmaSWarp = kMultiSoftmaxWarps + 1;   // issues the S^T MMAs
+constexpr int kMultiMmaPVWarp = kMultiSoftmaxWarps + 2;  // issues the P.V MMAs
+constexpr int kMultiEpiWarp0 = kMultiSoftmaxWarps + 3;   // 4 epilogue warps (one per TMEM lane quadrant)
+constexpr int kMultiLoadVWarp = kMultiSoftmaxWarps + 7;  // loads the V tiles (kMultiLoadWarp: the Q rows and K tiles)
+constexpr int kMultiThreads = (kMultiSoftmaxWarps + 8) * 32;
+constexpr int kMultiLptChunks = 128;  // up to this many chunks the items go longest first
+constexpr int kMultiKT = 128;         // keys per tile
+
+template <int D>
 struct MultiCfg {
-    static constexpr int TB = 2;
-    static constexpr int UT = B < 16 ? B : 16;        // tokens per unit (one TMA stage)
-    static constexpr int UPB = B / UT;                // units per block
-    static constexpr int NP = D * TB / 128;           // 128-byte panels per row
-    static constexpr int TILE = UT * D * TB;          // one unit of K (or V) for one KV head
-    static constexpr int STAGE = 2 * TILE;
-    static constexpr int STAGES_BYTES = NW * NST * STAGE;
-    static constexpr int RED_BYTES = NW * 16 * (D + 2) * 4;
-    static constexpr int BT_OFF = STAGES_BYTES > RED_BYTES ? STAGES_BYTES : RED_BYTES;
-    static_assert(TILE % 1024 == 0, "tiles must keep 1024-byte alignment for the 128-byte swizzle");
-    static_assert(NW % RG == 0, "warps must split evenly into row groups");
-    // per warp: NST full barriers, then NST empty barriers (used when two row groups share a stream's stages)
-    static size_t smem_bytes(int pb) { return 1024 + BT_OFF + static_cast<size_t>(pb) * 4 + 16 + 2 * NW * NST * 8; }
+    static constexpr int KT = kMultiKT;        // keys per tile (M of S^T)
+    static constexpr int NR = 32;              // query rows per KV head (N of both products)
+    static constexpr int NP = D / 64;          // 128-byte panels of a 16-bit row
+    static constexpr int TILE = NP * KT * 128;  // one K (or V) tile
+    static constexpr int NSK = 3;              // stages of K: refilled once S(t) is done, 3 tiles ahead
+    static constexpr int NSV = 2;              // stages of V: refilled once PV(t) is done
+    static constexpr int QBYTES = NP * NR * 128;
+    static constexpr int PBYTES = 2 * NR * 128;  // one P^T term: 32 rows x 128 keys, two 64-key panels
+    static constexpr int K_OFF = 0;
+    static constexpr int V_OFF = K_OFF + NSK * TILE;
+    static constexpr int Q_OFF = V_OFF + NSV * TILE;  // [2] query tiles
+    static constexpr int P_OFF = Q_OFF + 2 * QBYTES;  // [2] buffers x (hi, lo)
+    static constexpr int RED_OFF = P_OFF + 2 * 2 * PBYTES;
+    static constexpr int STAT_OFF = RED_OFF + kMultiSoftmaxWarps * kMultiRPT * 4;  // [2 items][max, sum][32 rows]
+    static constexpr int TAB_OFF = STAT_OFF + 2 * 2 * 32 * 4;
+    // schedule tables: full-partition prefix [R + 1], remainder tiles [R], remainder order [R], counts [2],
+    // then the chunks' q0, n, len, partitions [R] each
+    static constexpr int TAB_INTS = 7 * kMultiLptChunks + 3;
+    static constexpr int BAR_OFF = (TAB_OFF + TAB_INTS * 4 + 7) & ~7;
+    static constexpr int NBAR = 2 * NSK + 2 * NSV + 8 * 2 + 2 + 2;
+    static constexpr int SMEM = 1024 + BAR_OFF + (NBAR + 2) * 8;
+    static constexpr uint32_t TMEM_COLS = 128;
+    static constexpr uint32_t S_COL = 0;   // S^T of tile t at S_COL + 32 (t & 1)
+    static constexpr uint32_t O_COL = 64;  // O^T of item k at O_COL + 32 (k & 1)
+    static_assert(D == 64 || D == 128, "head_dim");
+    static_assert(SMEM <= 227 * 1024, "shared memory");
 };
 
-// Resident CTAs per SM the register allocation must allow (launch bounds):
-// three 4-warp CTAs (168 registers) -- left free, the compiler takes 203 and
-// two CTAs fit, 10 % slower on the multi-token batch; a fourth CTA (128
-// registers) spills and is slower still.
-#ifndef PKV_MULTI_MIN_CTAS
-#define PKV_MULTI_MIN_CTAS 3
-#endif
+// A chunk's rows and key range as the kernel sees them: n query tokens after
+// c0 = len - n prior ones; len clamped to the block table / the launch's
+// partitions (flagged, as in the decode kernels).  ok = false: nothing to do
+// (n <= 0 silently; an inconsistent chunk flagged when `report`).
+struct MultiChunk {
+    int q0, n, len, nblk, nparts;
+    bool ok;
+};
 
-template <typename T, int D, int B, int NST, int NW, int RG>
-__global__ void __launch_bounds__(NW * 32, PKV_MULTI_MIN_CTAS) paged_decode_multi_kernel(const MultiParams p, const int G,
-                                                                     const __grid_constant__ CUtensorMap tm_k,
-                                                                     const __grid_constant__ CUtensorMap tm_v) {
-    using C = MultiCfg<T, D, B, NST, NW, RG>;
+__device__ __forceinline__ MultiChunk multi_chunk(const MultiParams& p, int r, bool report) {
+    MultiChunk c;
+    c.q0 = p.query_start_loc[r];
+    c.n = p.query_start_loc[r + 1] - c.q0;
+    const int len_raw = p.seq_lens[r];
+    c.ok = c.n > 0;
+    if (c.ok && (c.n * p.group > 32 || len_raw < c.n || c.q0 < 0 || c.q0 + c.n > p.total_q_tokens)) {
+        if (report) flag_error(PKV_DEVERR_LENGTH);
+        c.ok = false;
+    }
+    c.nblk = c.ok ? decode_seq_blocks(len_raw, p.block_size, p.max_blocks_per_seq,
+                                      p.num_partitions * p.partition_blocks, report)
+                  : 0;
+    c.len = min(len_raw, c.nblk * p.block_size);
+    c.ok = c.ok && c.len >= c.n;  // a table too short for the new tokens themselves: nothing sensible to attend
+    c.nparts = c.ok ? (c.nblk + p.partition_blocks - 1) / p.partition_blocks : 0;
+    return c;
+}
+
+// One work item: chunk r's partition `part` for KV head g.
+struct MultiWork {
+    int r, part, g;
+    int q0, n, c0, len;
+    int kb, ke;  // keys [kb, ke)
+    int nt;      // key tiles (0: nothing to do)
+    bool direct;  // the chunk has one partition: write rows, not partials
+};
+
+// Schedule tables (longest first), built once per CTA; every thread of the
+// CTA calls it (block-wide barriers), threads below num_chunks do the work.
+// The chunks' geometry stays in shared memory for the items' lookups.
+constexpr int kTabChunk = 3 * kMultiLptChunks + 3;  // q0, n, len, nparts: [4][kMultiLptChunks]
+
+__device__ __forceinline__ void multi_build_schedule(const MultiParams& p, int* tab, bool report) {
+    const int R = p.num_chunks;
+    int* prefix = tab;                              // [R + 1]
+    int* rem_tiles = tab + kMultiLptChunks + 1;     // [R]
+    int* rem_order = tab + 2 * kMultiLptChunks + 1; // [R]
+    int* counts = tab + 3 * kMultiLptChunks + 1;    // full items per KV head, partial chunks
+    int* geo = tab + kTabChunk;
+    const int t = threadIdx.x;
+    const int part_tokens = p.partition_blocks * p.block_size;
+    int full = 0, remt = 0;
+    if (t < R) {
+        const MultiChunk c = multi_chunk(p, t, report);
+        if (c.ok) {
+            full = c.len / part_tokens;
+            const int rem = c.len - full * part_tokens;
+            remt = (rem + kMultiKT - 1) / kMultiKT;
+        }
+        rem_tiles[t] = remt;
+        prefix[t + 1] = full;
+        geo[t] = c.q0;
+        geo[kMultiLptChunks + t] = c.n;
+        geo[2 * kMultiLptChunks + t] = c.len;
+        geo[3 * kMultiLptChunks + t] = c.ok ? c.nparts : 0;
+    }
+    __syncthreads();
+    if (t < 32) {  // inclusive scan of the full-partition counts, 32 chunks per round
+        int carry = 0;
+        for (int base = 0; base < R; base += 32) {
+            int v = base + t < R ? prefix[base + t + 1] : 0;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int u = __shfl_up_sync(0xffffffffu, v, o);
+                if (t >= o) v += u;
+            }
+            if (base + t < R) prefix[base + t + 1] = carry + v;
+            carry += __shfl_sync(0xffffffffu, v, 31);
+        }
+        if (t == 0) {
+            prefix[0] = 0;
+            counts[0] = carry;
+        }
+    }
+    if (t < R && remt > 0) {  // rank among the partial partitions: more tiles first, then chunk order
+        int rank = 0;
+        for (int q = 0; q < R; ++q) {
+            const int tq = rem_tiles[q];
+            rank += tq > remt || (tq == remt && q < t);
+        }
+        rem_order[rank] = t;
+    }
+    const int has = __syncthreads_count(t < R && remt > 0);  // every thread of the CTA takes part
+    if (t == 0) counts[1] = has;
+}
+
+// The CTA's k-th item (rank blockIdx.x + k * gridDim.x); false past the last.
+__device__ __forceinline__ bool multi_item(const MultiParams& p, const int* tab, bool lpt, int k, MultiWork& w) {
+    // 32-bit ranks: the launch keeps chunks x partitions x KV heads below 2^30
+    const int H = p.num_kv_heads;
+    const int rank = static_cast<int>(blockIdx.x) + k * static_cast<int>(gridDim.x);
+    int r, part, g;
+    if (lpt) {
+        const int R = p.num_chunks;
+        const int* prefix = tab;
+        const int* rem_order = tab + 2 * kMultiLptChunks + 1;
+        const int nfull = tab[3 * kMultiLptChunks + 1] * H;
+        const int nrem = tab[3 * kMultiLptChunks + 2] * H;
+        if (rank < nfull) {
+            const int fi = rank / H;
+            g = rank - fi * H;
+            int lo = 0, hi = R;  // the last chunk whose full partitions start at or before fi
+            while (hi - lo > 1) {
+                const int mid = (lo + hi) >> 1;
+                if (prefix[mid] <= fi) lo = mid; else hi = mid;
+            }
+            r = lo;
+            part = fi - prefix[r];
+        } else if (rank < nfull + nrem) {
+            const int qi = (rank - nfull) / H;
+            g = (rank - nfull) - qi * H;
+            r = rem_order[qi];
+            part = prefix[r + 1] - prefix[r];
+        } else {
+            return false;
+        }
+    } else {
+        const int per_part = p.num_chunks * H;
+        if (rank >= per_part * p.num_partitions) return false;
+        part = rank / per_part;
+        const int rem = rank - part * per_part;
+        r = rem / H;
+        g = rem - r * H;
+    }
+    w.r = r, w.part = part, w.g = g;
+    MultiChunk c;
+    if (lpt) {  // the schedule reported the chunks' errors and kept their geometry
+        const int* geo = tab + kTabChunk;
+        c.q0 = geo[r];
+        c.n = geo[kMultiLptChunks + r];
+        c.len = geo[2 * kMultiLptChunks + r];
+        c.nparts = geo[3 * kMultiLptChunks + r];
+        c.ok = c.nparts > 0;
+    } else {  // errors reported by item (0, 0)'s loader lane 0
+        c = multi_chunk(p, r, part == 0 && g == 0 && threadIdx.x == kMultiLoadWarp * 32);
+    }
+    w.nt = 0;
+    if (!c.ok || part >= c.nparts) return true;
+    w.q0 = c.q0, w.n = c.n, w.len = c.len, w.c0 = c.len - c.n;
+    w.kb = part * p.partition_blocks * p.block_size;
+    w.ke = min(c.len, w.kb + p.partition_blocks * p.block_size);
+    w.nt = (w.ke - w.kb + kMultiKT - 1) / kMultiKT;
+    w.direct = c.nparts == 1;
+    return true;
+}
+
+// OR of a predicate over the softmax threads (named barrier 1).
+__device__ __forceinline__ bool multi_vote_any(bool v) {
+    uint32_t r;
+    asm volatile(
+        "{\n\t.reg .pred q, p;\n\t"
+        "setp.ne.u32 q, %1, 0;\n\t"
+        "barrier.cta.red.or.pred p, 1, %2, q;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(r)
+        : "r"(static_cast<uint32_t>(v)), "n"(kMultiSoftmaxThreads)
+        : "memory");
+    return r != 0;
+}
+
+__device__ __forceinline__ void multi_sync_softmax() {
+    asm volatile("barrier.cta.sync 1, %0;" ::"n"(kMultiSoftmaxThreads) : "memory");
+}
+
+// v[c] (c < N) holds this lane's value of column c; returns the max (kMax)
+// or sum over the warp's 32 lanes of column lane % N.  Each step halves the
+// columns a lane keeps (N/2 + ... + 1 shuffles); the last steps join the
+// lanes that kept the same column.
+template <bool kMax, int N>
+__device__ __forceinline__ float multi_reduce_scatter(float (&v)[N], int lane) {
+#pragma unroll
+    for (int o = N / 2; o >= 1; o >>= 1) {
+        const bool upper = (lane & o) != 0;
+#pragma unroll
+        for (int j = 0; j < o; ++j) {
+            const float send = upper ? v[j] : v[j + o];
+            const float keep = upper ? v[j + o] : v[j];
+            const float recv = __shfl_xor_sync(0xffffffffu, send, o);
+            v[j] = kMax ? fmaxf(keep, recv) : keep + recv;
+        }
+    }
+    float x = v[0];
+#pragma unroll
+    for (int o = N; o < 32; o <<= 1) {
+        const float other = __shfl_xor_sync(0xffffffffu, x, o);
+        x = kMax ? fmaxf(x, other) : x + other;
+    }
+    return x;
+}
+
+// N (8 or 16) consecutive 32-bit columns of this thread's TMEM lane (32x32b shape).
+template <int N>
+__device__ __forceinline__ void multi_tmem_ld(uint32_t taddr, float (&v)[N]) {
+    uint32_t r[N];
+    if constexpr (N == 16) {
+        asm volatile(
+            "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+            "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15}, [%16];"
+            : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+              "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+            : "r"(taddr));
+    } else {
+        static_assert(N == 8, "columns");
+        asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
+                     : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7])
+                     : "r"(taddr));
+    }
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+    for (int i = 0; i < N; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+template <int N>
+__device__ __forceinline__ void multi_tmem_st(uint32_t taddr, const float (&v)[N]) {
+    if constexpr (N == 16) {
+        asm volatile(
+            "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
+            "{%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16};" ::"r"(taddr),
+            "r"(__float_as_uint(v[0])), "r"(__float_as_uint(v[1])), "r"(__float_as_uint(v[2])),
+            "r"(__float_as_uint(v[3])), "r"(__float_as_uint(v[4])), "r"(__float_as_uint(v[5])),
+            "r"(__float_as_uint(v[6])), "r"(__float_as_uint(v[7])), "r"(__float_as_uint(v[8])),
+            "r"(__float_as_uint(v[9])), "r"(__float_as_uint(v[10])), "r"(__float_as_uint(v[11])),
+            "r"(__float_as_uint(v[12])), "r"(__float_as_uint(v[13])), "r"(__float_as_uint(v[14])),
+            "r"(__float_as_uint(v[15]))
+            : "memory");
+    } else {
+        static_assert(N == 8, "columns");
+        asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"r"(taddr),
+                     "r"(__float_as_uint(v[0])), "r"(__float_as_uint(v[1])), "r"(__float_as_uint(v[2])),
+                     "r"(__float_as_uint(v[3])), "r"(__float_as_uint(v[4])), "r"(__float_as_uint(v[5])),
+                     "r"(__float_as_uint(v[6])), "r"(__float_as_uint(v[7]))
+                     : "memory");
+    }
+    asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+}
+
+template <typename T, int D>
+__global__ void __launch_bounds__(kMultiThreads, 1) paged_decode_multi_kernel(const MultiParams p, const int lpt,
+                                                                            const __grid_constant__ CUtensorMap tm_q,
+                                                                            const __grid_constant__ CUtensorMap tm_k,
+                                                                            const __grid_constant__ CUtensorMap tm_v) {
+    using C = MultiCfg<D>;
     constexpr bool kBf16 = Elem<T>::kCuType == CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
-    constexpr int KS = D / 16;  // 16-dim steps of Q.K^T
-    constexpr int DT = D / 8;   // 8-dim output tiles
-    constexpr int UT = C::UT;
+    constexpr int NSK = C::NSK, NSV = C::NSV;
+    constexpr int KT = kMultiKT;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = align_1024(smem_raw);
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::BAR_OFF);
+    uint64_t* k_full = bars;                     // [NSK] the K tile landed
+    uint64_t* k_free = bars + NSK;               // [NSK] the S MMAs that read the stage are done
+    uint64_t* v_full = bars + 2 * NSK;           // [NSV]
+    uint64_t* v_free = bars + 2 * NSK + NSV;     // [NSV] the P.V MMAs that read the stage are done
+    uint64_t* q_full = bars + 2 * NSK + 2 * NSV; // [2] per item: the Q rows landed
+    uint64_t* q_free = q_full + 2;     // [2] per item: its S MMAs are done
+    uint64_t* s_full = q_full + 4;     // [2] per tile: S^T(t) done
+    uint64_t* s_free = q_full + 6;     // [2] per tile: the softmax read S^T(t) (256 arrivals)
+    uint64_t* p_full = q_full + 8;     // [2] per tile: P^T(t) written (256 arrivals)
+    uint64_t* p_free = q_full + 10;    // [2] per tile: PV(t) done
+    uint64_t* o_full = q_full + 12;    // [2] per item: its last PV done
+    uint64_t* o_free = q_full + 14;    // [2] per item: the epilogue read O^T and the row stats (128 arrivals)
+    uint64_t* mma_done = q_full + 16;  // [2] the S / P.V issuer's MMAs are all done (exit drain)
+    uint64_t* stat_full = q_full + 18; // [2] per item: the softmax wrote its rows' max and sum (256 arrivals)
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(q_full + 20);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(q_full + 21);
+    int* tab = reinterpret_cast<int*>(smem + C::TAB_OFF);
+    float* red = reinterpret_cast<float*>(smem + C::RED_OFF);
+    float* stat = reinterpret_cast<float*>(smem + C::STAT_OFF);
 
-    const int per_chunk = p.num_partitions * p.num_kv_heads;
-    const int r = blockIdx.x / per_chunk;
-    const int rem = blockIdx.x - r * per_chunk;
-    const int part = rem / p.num_kv_heads;
-    const int g = rem - part * p.num_kv_heads;
-    const int warp = threadIdx.x >> 5;
-    const int lane = threadIdx.x & 31;
+    const int tid = threadIdx.x;
+    const int warp = tid >> 5;
+    const int lane = tid & 31;
+    const bool lpt_order = lpt != 0;
 
-    const int q0 = p.query_start_loc[r];
-    const int n = p.query_start_loc[r + 1] - q0;
-    const int len_raw = p.seq_lens[r];
-    if (n <= 0) return;
-    if (n * G > 16 * RG || len_raw < n || q0 < 0 || q0 + n > p.total_q_tokens) {
-        if (threadIdx.x == 0 && part == 0 && g == 0) flag_error(PKV_DEVERR_LENGTH);
-        return;
+    if (warp == 0) {
+        tmem_alloc(tmem_slot, C::TMEM_COLS);
+        tmem_relinquish();
     }
-    const int nblk = decode_seq_blocks(len_raw, B, p.max_blocks_per_seq, p.num_partitions * p.partition_blocks,
-                                       threadIdx.x == 0 && part == 0 && g == 0);
-    const int len = min(len_raw, nblk * B);
-    const int c0 = len - n;  // a clamped sequence keeps its last rows' limits inside the table
-    const int nparts = nblk > 0 ? (nblk + p.partition_blocks - 1) / p.partition_blocks : 1;
-    if (part >= nparts) return;
-    const int b0 = part * p.partition_blocks;
-    const int nb = max(0, min(nblk - b0, p.partition_blocks));
-    const bool direct = nparts == 1;
-
-    int* bt_s = reinterpret_cast<int*>(smem + C::BT_OFF);
-    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + ((C::BT_OFF + p.partition_blocks * 4 + 15) & ~15));
-    const int32_t* bt_row = p.block_tables + static_cast<int64_t>(r) * p.max_blocks_per_seq + b0;
-    for (int i = threadIdx.x; i < nb; i += NW * 32) {
-        int id = bt_row[i];
-        if (id < 0 || id >= p.num_blocks) {
-            flag_error(PKV_DEVERR_BLOCK_ID);
-            id = -1;
+    if (tid == 32) {
+        for (int i = 0; i < NSK; ++i) {
+            mbar_init(&k_full[i], 1);
+            mbar_init(&k_free[i], 1);
         }
-        bt_s[i] = id;
-    }
-    // ---- this warp's 16 rows: the lane holds rows rq and rq + 8 (rq = lane / 4).
-    // A chunk with at most 16 rows uses one row group: every warp is a stream.
-    // With two row groups the two warps of a stream share its stages: the
-    // first issues each unit's copy once into a ring of 2 * NST stages, both
-    // read it, and each releases it on the stage's empty barrier.
-    const int nrg = n * G > 16 ? RG : 1;
-    const int nsw = NW / nrg;
-    const int rg = warp % nrg, stream = warp / nrg;
-    const int ring = nrg * NST;
-    uint64_t* fbar = bars + stream * ring;            // full: the unit's bytes arrived
-    uint64_t* ebar = bars + NW * NST + stream * ring;  // empty: every reader of the stage is done
-    if (lane == 0) {
-#pragma unroll
-        for (int st = 0; st < NST; ++st) {
-            mbar_init(&bars[warp * NST + st], 1);
-            mbar_init(&bars[NW * NST + warp * NST + st], nrg);
+        for (int i = 0; i < NSV; ++i) {
+            mbar_init(&v_full[i], 1);
+            mbar_init(&v_free[i], 1);
         }
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&q_full[i], 1);
+            mbar_init(&q_free[i], 1);
+            mbar_init(&s_full[i], 1);
+            mbar_init(&s_free[i], kMultiSoftmaxThreads);
+            mbar_init(&p_full[i], kMultiSoftmaxThreads);
+            mbar_init(&p_free[i], 1);
+            mbar_init(&o_full[i], 1);
+            mbar_init(&o_free[i], 128);
+            mbar_init(&stat_full[i], kMultiSoftmaxThreads);
+        }
+        mbar_init(&mma_done[0], 1);
+        mbar_init(&mma_done[1], 1);
+        *abort_flag = 0;
         fence_mbar_init();
     }
+    if (lpt_order) multi_build_schedule(p, tab, blockIdx.x == 0);
+    tc_fence_before();
     __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
 
-    // units (16-token sub-blocks) holding positions [b0 * B, min(len, (b0 + nb) * B))
-    const int span = max(0, min(len, (b0 + nb) * B) - b0 * B);
-    const int units = (span + UT - 1) / UT;
-    const int nw = units > stream ? (units - stream + nsw - 1) / nsw : 0;
-    uint8_t* wstage = smem + stream * ring * C::STAGE;  // the stream's ring of stages
-    const bool producer = rg == 0;
-    const uint64_t policy = l2_policy_evict_first();
-
-    auto issue = [&](int k) {  // lane 0 of the producer only
-        const int st = k % ring;
-        const int u = stream + k * nsw;
-        const int id = bt_s[u / C::UPB];
-        const int coord = id >= 0 ? id : static_cast<int>(p.num_blocks);  // out of range: zero fill
-        const int row0 = (u % C::UPB) * UT;
-        uint8_t* kd = wstage + st * C::STAGE;
-        uint8_t* vd = kd + C::TILE;
-        mbar_arrive_expect_tx(&fbar[st], C::STAGE);
+    if (warp == kMultiLoadWarp || warp == kMultiLoadVWarp) {
+        // ================================================================ loaders (whole warps)
+        // kMultiLoadWarp: per item the Q rows, then the K tiles; kMultiLoadVWarp: the V tiles.
+        // A stage is refilled as soon as the MMAs that read it are done; the
+        // block ids of the next tile (across items too) are loaded one tile
+        // ahead, one per lane.
+        const bool k_role = warp == kMultiLoadWarp;
+        const int NSR = k_role ? NSK : NSV;
+        uint64_t* full = k_role ? k_full : v_full;
+        uint64_t* freed = k_role ? k_free : v_free;
+        const CUtensorMap* map = k_role ? &tm_k : &tm_v;
+        uint8_t* ring = smem + (k_role ? C::K_OFF : C::V_OFF);
+        const bool leader = lane == 0;
+        const int B = p.block_size;
+        const int per_tile = KT / B;  // blocks per key tile (4, 8 or 16), one lane each
+        const uint64_t policy = l2_policy_evict_first();
+        // a wait by lane 0, its outcome for the whole warp
+        auto wait_all = [&](uint64_t* bar, int parity) -> bool {
+            const int got = leader ? static_cast<int>(mbar_wait_or_abort_idle(bar, parity, abort_flag)) : 0;
+            return __shfl_sync(0xffffffffu, got, 0) != 0;
+        };
+        auto next_work = [&](int& k, MultiWork& w) -> bool {
+            while (multi_item(p, tab, lpt_order, k++, w))
+                if (w.nt > 0) return true;
+            return false;
+        };
+        auto fetch = [&](const MultiWork& w, int j) -> int {
+            const int lb = w.kb / B + j * per_tile + lane;
+            return (lane < per_tile && lb < (w.ke + B - 1) / B)
+                       ? p.block_tables[static_cast<int64_t>(w.r) * p.max_blocks_per_seq + lb]
+                       : -1;
+        };
+        griddep_wait();  // the pools may still be in the writes of a grid this one depends on
+        int n = 0, nq = 0;  // tiles, Q tiles issued
+        bool ok = true;
+        int k = 0;
+        MultiWork w;
+        bool have = next_work(k, w);
+        int ids = have ? fetch(w, 0) : -1;
+        while (have && ok) {
+            if (k_role) {
+                const int qb = nq & 1;
+                if (nq >= 2) ok = wait_all(&q_free[qb], ((nq - 2) >> 1) & 1);
+                if (!ok) break;
+                if (leader) {
+                    // 32 / G tokens x G heads = 32 rows, token-major; rows past the
+                    // chunk belong to other tokens (or are zero filled) and are masked
+                    mbar_arrive_expect_tx(&q_full[qb], C::QBYTES);
 #pragma unroll
-        for (int pn = 0; pn < C::NP; ++pn) {
-            tma_load_4d_hint(kd + pn * UT * 128, &tm_k, pn * 64, g, row0, coord, &fbar[st], policy);
-            tma_load_4d_hint(vd + pn * UT * 128, &tm_v, pn * 64, g, row0, coord, &fbar[st], policy);
-        }
-    };
-    int issued = 0;
-    griddep_wait();  // the pools may still be in the writes of a grid this one depends on
-    if (lane == 0 && producer) {
-        for (; issued < ring && issued < nw; ++issued) issue(issued);
-    }
-    __syncwarp();
-    // The query fragments load while the first stages are in flight.
-    const int gq = lane >> 2, cq = lane & 3;
-    int lim[2];  // last key position each of the lane's two rows may see
-    uint32_t qa[KS][4];
-#pragma unroll
-    for (int h = 0; h < 2; ++h) {
-        const int row = 16 * rg + gq + 8 * h;
-        const int i = row / G, hh = row - (row / G) * G;
-        lim[h] = c0 + min(i, n - 1);
-        const bool live = i < n;
-        const T* qrow = reinterpret_cast<const T*>(p.query) +
-                        ((static_cast<int64_t>(q0) + (live ? i : 0)) * p.num_q_heads + static_cast<int64_t>(g) * G +
-                         hh) * D;
-#pragma unroll
-        for (int ks = 0; ks < KS; ++ks) {
-            qa[ks][h] = live ? *reinterpret_cast<const uint32_t*>(qrow + 16 * ks + 2 * cq) : 0u;
-            qa[ks][h + 2] = live ? *reinterpret_cast<const uint32_t*>(qrow + 16 * ks + 8 + 2 * cq) : 0u;
-        }
-    }
-
-    float m[2] = {-INFINITY, -INFINITY}, l[2] = {0.f, 0.f};
-    float o[DT][4];  // [dim tile j][c0: (row rq, dim 8j + 2cq), c1: +1, c2: (row rq + 8, dim 8j + 2cq), c3: +1]
-#pragma unroll
-    for (int j = 0; j < DT; ++j) o[j][0] = o[j][1] = o[j][2] = o[j][3] = 0.f;
-    const int lr = lane & 7, lm = lane >> 3;
-
-    int k = 0;
-    for (; k < nw; ++k) {
-        const int st = k % ring;
-        const bool ok = mbar_wait_main(&fbar[st], (k / ring) & 1);
-        if (!__all_sync(0xffffffffu, ok)) break;
-        const int u = stream + k * nsw;
-        const int pos0 = (b0 + u / C::UPB) * B + (u % C::UPB) * UT;  // key position of the unit's first token
-        const int valid = min(UT, len - pos0);
-        if (bt_s[u / C::UPB] >= 0) {
-            const uint8_t* Ks = wstage + st * C::STAGE;
-            const uint8_t* Vs = Ks + C::TILE;
-            // ---- S = Q . K^T: s[nt] covers keys 8 nt .. 8 nt + 7 of the unit
-            // two accumulator sets (even / odd dim steps) halve the dependent MMA chain
-            float s[2][4], s2[2][4];
-#pragma unroll
-            for (int nt = 0; nt < 2; ++nt) {
-                s[nt][0] = s[nt][1] = s[nt][2] = s[nt][3] = 0.f;
-                s2[nt][0] = s2[nt][1] = s2[nt][2] = s2[nt][3] = 0.f;
+                    for (int pn = 0; pn < C::NP; ++pn)
+                        tma_load_3d(smem + C::Q_OFF + qb * C::QBYTES + pn * C::NR * 128, &tm_q, pn * 64,
+                                    w.g * p.group, w.q0, &q_full[qb]);
+                }
+                ++nq;
             }
-#pragma unroll
-            for (int ks = 0; ks < KS; ++ks) {
-                float (&acc)[2][4] = (ks & 1) ? s2 : s;
-                if constexpr (UT == 16) {
-                    // matrices: (keys 0-7, chunk 2ks), (keys 0-7, chunk 2ks+1), (keys 8-15, ...), (keys 8-15, ...)
-                    const int key = lr + 8 * (lm >> 1);
-                    const int ch = 2 * ks + (lm & 1);
-                    uint32_t b[4];
-                    ldsm_x4(b, Ks + (ch / 8) * UT * 128 + key * 128 + (((ch % 8) ^ (key & 7)) << 4));
-                    mma_16816<kBf16>(acc[0], qa[ks], b[0], b[1]);
-                    mma_16816<kBf16>(acc[1], qa[ks], b[2], b[3]);
+            MultiWork nw;
+            bool have_next = false;
+            for (int j = 0; j < w.nt; ++j) {
+                int ids_next;
+                if (j + 1 < w.nt) {
+                    ids_next = fetch(w, j + 1);
                 } else {
-                    const int key = lr;
-                    const int ch = 2 * ks + (lm & 1);
-                    uint32_t b0r, b1r;
-                    ldsm_x2(b0r, b1r, Ks + (ch / 8) * UT * 128 + key * 128 + (((ch % 8) ^ (key & 7)) << 4));
-                    mma_16816<kBf16>(acc[0], qa[ks], b0r, b1r);
+                    have_next = next_work(k, nw);
+                    ids_next = have_next ? fetch(nw, 0) : -1;
                 }
+                const int lb = w.kb / B + j * per_tile + lane;
+                int id = ids;
+                if (lane < per_tile && lb < (w.ke + B - 1) / B && (id < 0 || id >= p.num_blocks)) {
+                    flag_error(PKV_DEVERR_BLOCK_ID);
+                    id = -1;
+                }
+                const int coord = id >= 0 ? id : static_cast<int>(p.num_blocks);  // out of range: zero fill
+                const int st = n % NSR;
+                if (n >= NSR) ok = wait_all(&freed[st], ((n - NSR) / NSR) & 1);
+                if (!ok) break;
+                if (leader) mbar_arrive_expect_tx(&full[st], C::TILE);
+                __syncwarp();
+                if (lane < per_tile) {
+#pragma unroll
+                    for (int pn = 0; pn < C::NP; ++pn)
+                        tma_load_4d_hint(ring + st * C::TILE + pn * KT * 128 + lane * B * 128, map, pn * 64, w.g, 0,
+                                         coord, &full[st], policy);
+                }
+                ++n;
+                ids = ids_next;
             }
-#pragma unroll
-            for (int nt = 0; nt < 2; ++nt)
-#pragma unroll
-                for (int e = 0; e < 4; ++e) s[nt][e] += s2[nt][e];
-            // ---- causal mask and online softmax of the lane's two rows (log2 domain)
-            float bm[2] = {-INFINITY, -INFINITY};
-#pragma unroll
-            for (int nt = 0; nt < 2; ++nt) {
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const int key = 8 * nt + 2 * cq + (e & 1);
-                    const int h = e >> 1;
-                    const bool ok_key = (UT == 16 || nt == 0) && key < valid && pos0 + key <= lim[h];
-                    s[nt][e] = ok_key ? s[nt][e] * p.scale_log2 : -INFINITY;
-                    bm[h] = fmaxf(bm[h], s[nt][e]);
-                }
-            }
-            // Lazy rescaling: a row's exponent base m moves, and its O and sum
-            // are rescaled, only when a unit's max exceeds it by more than 2^8;
-            // the weights exp2(s - m) then stay below 256 (bf16 / f16 P).
-            float alpha[2] = {1.f, 1.f}, msafe[2];
-            bool rs = false;
-#pragma unroll
-            for (int h = 0; h < 2; ++h) {
-                bm[h] = fmaxf(bm[h], __shfl_xor_sync(0xffffffffu, bm[h], 1));
-                bm[h] = fmaxf(bm[h], __shfl_xor_sync(0xffffffffu, bm[h], 2));
-                if (bm[h] > m[h] + 8.f || (m[h] == -INFINITY && bm[h] != -INFINITY)) {
-                    alpha[h] = ex2_approx(m[h] - bm[h]);  // 0 when m was -inf
-                    m[h] = bm[h];
-                    rs = true;
-                }
-                msafe[h] = m[h] == -INFINITY ? 0.f : m[h];  // a row with no key yet stays empty
-            }
-            float ps[2] = {0.f, 0.f};
-#pragma unroll
-            for (int nt = 0; nt < 2; ++nt) {
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    s[nt][e] = ex2_approx(s[nt][e] - msafe[e >> 1]);
-                    ps[e >> 1] += s[nt][e];
-                }
-            }
-            l[0] = l[0] * alpha[0] + ps[0];  // per-lane partial row sums; the quad is summed at the end
-            l[1] = l[1] * alpha[1] + ps[1];
-            if (__any_sync(0xffffffffu, rs)) {
-#pragma unroll
-                for (int j = 0; j < DT; ++j) {
-                    o[j][0] *= alpha[0];
-                    o[j][1] *= alpha[0];
-                    o[j][2] *= alpha[1];
-                    o[j][3] *= alpha[1];
-                }
-            }
-            // ---- O += P . V  (P: the S accumulators in the A layout; bf16 as hi + lo)
-            uint32_t pa[4], pl[4] = {0u, 0u, 0u, 0u};
-            pa[0] = Elem<T>::pack(s[0][0], s[0][1]);
-            pa[1] = Elem<T>::pack(s[0][2], s[0][3]);
-            pa[2] = Elem<T>::pack(s[1][0], s[1][1]);
-            pa[3] = Elem<T>::pack(s[1][2], s[1][3]);
-            if constexpr (kBf16) {
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const float2 f = Elem<T>::pair(pa[e]);
-                    pl[e] = Elem<T>::pack(s[e >> 1][2 * (e & 1)] - f.x, s[e >> 1][2 * (e & 1) + 1] - f.y);
-                }
-            }
-            // keys of this lane's B fragment halves, for masking rows past the context
-            const bool partial = valid < 16;
-            const int t0 = 2 * cq;
-            const uint32_t mk0 = (t0 < valid ? 0x0000FFFFu : 0u) | (t0 + 1 < valid ? 0xFFFF0000u : 0u);
-            const uint32_t mk1 = (t0 + 8 < valid ? 0x0000FFFFu : 0u) | (t0 + 9 < valid ? 0xFFFF0000u : 0u);
-#pragma unroll
-            for (int jp = 0; jp < DT / 2; ++jp) {
-                uint32_t b[4];
-                if constexpr (UT == 16) {
-                    // matrices: (keys 0-7, chunk 2jp), (keys 8-15, chunk 2jp), (keys 0-7, 2jp+1), (keys 8-15, 2jp+1)
-                    const int key = lr + 8 * (lm & 1);
-                    const int ch = 2 * jp + (lm >> 1);
-                    ldsm_x4_trans(b, Vs + (ch / 8) * UT * 128 + key * 128 + (((ch % 8) ^ (key & 7)) << 4));
-                } else {
-                    const int key = lr;
-                    const int ch = 2 * jp + (lm & 1);
-                    ldsm_x2_trans(b[0], b[2], Vs + (ch / 8) * UT * 128 + key * 128 + (((ch % 8) ^ (key & 7)) << 4));
-                    b[1] = b[3] = 0u;
-                }
-                if (partial) {  // rows past the context may hold anything: 0 * NaN must not reach O
-                    b[0] &= mk0;
-                    b[2] &= mk0;
-                    b[1] &= mk1;
-                    b[3] &= mk1;
-                }
-                mma_16816<kBf16>(o[2 * jp], pa, b[0], b[1]);
-                mma_16816<kBf16>(o[2 * jp + 1], pa, b[2], b[3]);
-                if constexpr (kBf16) {
-                    mma_16816<kBf16>(o[2 * jp], pl, b[0], b[1]);
-                    mma_16816<kBf16>(o[2 * jp + 1], pl, b[2], b[3]);
-                }
-            }
+            w = nw;
+            have = have_next;
         }
-        __syncwarp();
-        bool go = true;
+        if (leader) {
+            // Wait (bounded) for this warp's last copies: on the normal path
+            // their consumers waited for them already; after an abort they may
+            // still be in flight and must land before the CTA exits.
+            for (int t = max(0, nq - 2); t < nq; ++t) mbar_wait(&q_full[t & 1], (t >> 1) & 1);
+            for (int t = max(0, n - NSR); t < n; ++t) mbar_wait(&full[t % NSR], (t / NSR) & 1);
+        }
+    } else if (warp == kMultiMmaSWarp || warp == kMultiMmaPVWarp) {
+        // ================================================================ MMA issue (lane 0 of two warps)
+        // The S^T and P.V streams share no accumulator or operand buffer, so
+        // two threads issue them: the tensor cores take an N = 32 MMA in a
+        // fraction of the time one thread needs to issue the next.
         if (lane == 0) {
-            if (nrg > 1) mbar_arrive(&ebar[st]);
-            if (producer && k + ring < nw) {
-                // the stage is refilled once every reader released unit k
-                go = nrg == 1 || mbar_wait_main(&ebar[st], (k / ring) & 1);
-                if (go) {
-                    fence_proxy_async();
-                    issue(k + ring);
-                    issued = k + ring + 1;
+            const bool s_role = warp == kMultiMmaSWarp;
+            constexpr uint32_t IDESC_S = umma_idesc_f16(128, C::NR, kBf16, false, false);
+            constexpr uint32_t IDESC_O = umma_idesc_f16(128, C::NR, kBf16, true, false);  // A (V^T) MN-major
+            constexpr int kKP = KT * 128 / 16;    // panel stride of a K tile (16-byte units)
+            constexpr int kQP = C::NR * 128 / 16;  // panel stride of the Q rows and of P^T
+            // Descriptors made once; a 16-element k slice adds its byte offset / 16.
+            // V^T: M = head_dim in 64-element atoms (the tile's panels, LBO apart;
+            // one panel at head_dim 64, read twice: lanes 64-127 of O^T repeat 0-63),
+            // K = keys, 8 key rows per 1024-byte swizzle atom (SBO).
+            const uint64_t kdesc0 = smem_desc_sw128(smem_u32(smem + C::K_OFF), 16, 1024);
+            const uint64_t vdesc0 = smem_desc_sw128(smem_u32(smem + C::V_OFF), C::NP > 1 ? KT * 128 : 0, 1024);
+            const uint64_t qdesc0 = smem_desc_sw128(smem_u32(smem + C::Q_OFF), 16, 1024);
+            const uint64_t pdesc0 = smem_desc_sw128(smem_u32(smem + C::P_OFF), 16, 1024);
+            int it = 0, tb = 0;  // items and key tiles of this CTA so far
+            bool ok = true;
+            for (int k = 0; ok; ++k) {
+                MultiWork w;
+                if (!multi_item(p, tab, lpt_order, k, w)) break;
+                if (w.nt == 0) continue;
+                if (s_role) {
+                    // S^T(t) = K_t . Q^T into S buffer t & 1
+                    const int qb = it & 1;
+                    ok = mbar_wait_or_abort_idle(&q_full[qb], (it >> 1) & 1, abort_flag);
+                    const uint64_t qd = qdesc0 + qb * (C::QBYTES / 16);
+                    for (int j = 0; ok && j < w.nt; ++j) {
+                        const int t = tb + j;
+                        ok = mbar_wait_or_abort_idle(&k_full[t % NSK], (t / NSK) & 1, abort_flag) &&
+                             (t < 2 || mbar_wait_or_abort_idle(&s_free[t & 1], ((t - 2) >> 1) & 1, abort_flag));
+                        if (!ok) break;
+                        tc_fence_after();
+                        const uint64_t kd = kdesc0 + (t % NSK) * (C::TILE / 16);
+                        const uint32_t s_col = tmem + C::S_COL + 32 * (t & 1);
+#pragma unroll
+                        for (int kk = 0; kk < D / 16; ++kk)
+                            umma_f16_ss(s_col, kd + (kk / 4) * kKP + (kk % 4) * 2, qd + (kk / 4) * kQP + (kk % 4) * 2,
+                                        IDESC_S, kk > 0 ? 1u : 0u);
+                        umma_commit(&s_full[t & 1]);
+                        umma_commit(&k_free[t % NSK]);
+                        if (j == w.nt - 1) umma_commit(&q_free[qb]);
+                    }
+                } else {
+                    // O^T(item) += V_t^T . P_t^T; the item's first tile starts the accumulator
+                    const int ob = it & 1;
+                    const uint32_t o_col = tmem + C::O_COL + 32 * ob;
+                    for (int j = 0; ok && j < w.nt; ++j) {
+                        const int t = tb + j;
+                        ok = mbar_wait_or_abort_idle(&v_full[t % NSV], (t / NSV) & 1, abort_flag) &&
+                             mbar_wait_or_abort_idle(&p_full[t & 1], (t >> 1) & 1, abort_flag) &&
+                             (j > 0 || it < 2 || mbar_wait_or_abort_idle(&o_free[ob], ((it - 2) >> 1) & 1, abort_flag));
+                        if (!ok) break;
+                        tc_fence_after();
+                        const uint64_t vd = vdesc0 + (t % NSV) * (C::TILE / 16);
+                        const uint64_t pd = pdesc0 + (t & 1) * (2 * C::PBYTES / 16);
+#pragma unroll
+                        for (int kk = 0; kk < KT / 16; ++kk) {
+                            const uint64_t a = vd + kk * (16 * 128 / 16);  // 16 key rows of 128 bytes
+                            const uint64_t b = pd + (kk / 4) * kQP + (kk % 4) * 2;
+                            umma_f16_ss(o_col, a, b, IDESC_O, (j == 0 && kk == 0) ? 0u : 1u);
+                            if constexpr (kBf16) umma_f16_ss(o_col, a, b + C::PBYTES / 16, IDESC_O, 1u);
+                        }
+                        umma_commit(&p_free[t & 1]);
+                        umma_commit(&v_free[t % NSV]);
+                        if (j == w.nt - 1) umma_commit(&o_full[ob]);
+                    }
+                }
+                tb += w.nt;
+                ++it;
+            }
+            // Wait (bounded) for every MMA this thread issued before tensor
+            // memory is released: complete already on the normal path, possibly
+            // in flight after an abort.
+            uint64_t* done = &mma_done[s_role ? 0 : 1];
+            umma_commit(done);
+            mbar_wait(done, 0);
+        }
+    } else if (warp >= kMultiEpiWarp0) {
+        // ================================================================ epilogue: thread t = O^T lane t
+        // Once the item's last P.V is done and the softmax handed over the
+        // row statistics: O^T's lane t (head_dim element t of every row) to
+        // registers, O^T and the stats released, then element t of each row
+        // (or of the partition's fp32 partial, and the row's max / sum).
+        const int q4 = warp & 3;
+        const int t = q4 * 32 + lane;
+        const uint32_t lane_base = static_cast<uint32_t>(q4 * 32) << 16;
+        const int G = p.group;
+        int it = 0;
+        bool ok = true;
+        for (int k = 0; ok; ++k) {
+            MultiWork w;
+            if (!multi_item(p, tab, lpt_order, k, w)) break;
+            if (w.nt == 0) continue;
+            const int ob = it & 1;
+            const int got = lane == 0 ? (mbar_wait_or_abort_idle(&o_full[ob], (it >> 1) & 1, abort_flag) &&
+                                         mbar_wait_or_abort_idle(&stat_full[ob], (it >> 1) & 1, abort_flag))
+                                      : 0;
+            ok = __shfl_sync(0xffffffffu, got, 0) != 0;
+            if (!ok) break;
+            tc_fence_after();
+            float o[32];
+            if (q4 * 32 < D) tmem_ld32(tmem + lane_base + C::O_COL + 32 * ob, o);  // lanes past head_dim 64 repeat 0-63
+            const float mrow = stat[ob * 64 + lane];       // row `lane`
+            const float lsum = stat[ob * 64 + 32 + lane];
+            tc_fence_before();
+            mbar_arrive(&o_free[ob]);
+            const float inv = lsum > 0.f ? 1.f / lsum : 0.f;  // a row without keys writes 0
+            const int R = w.n * G;
+            if (!w.direct && q4 == 0 && lane < R) {
+                const int64_t pi = (static_cast<int64_t>(w.q0 + lane / G) * p.num_q_heads +
+                                    static_cast<int64_t>(w.g) * G + lane % G) * p.num_partitions + w.part;
+                p.ws_max[pi] = mrow;
+                p.ws_sum[pi] = lsum;
+            }
+            if (q4 * 32 < D) {
+                int i = 0, hh = 0;
+#pragma unroll
+                for (int r = 0; r < 32; ++r) {
+                    const float val = o[r] * __shfl_sync(0xffffffffu, inv, r);
+                    if (r < R) {
+                        const int64_t orow = static_cast<int64_t>(w.q0 + i) * p.num_q_heads +
+                                             static_cast<int64_t>(w.g) * G + hh;
+                        if (w.direct)
+                            reinterpret_cast<T*>(p.out)[orow * D + t] = Elem<T>::from_f(val);
+                        else
+                            p.ws_out[(orow * p.num_partitions + w.part) * D + t] = val;
+                    }
+                    if (++hh == G) hh = 0, ++i;
                 }
             }
+            ++it;
         }
-        if (!__shfl_sync(0xffffffffu, go, 0)) {
-            ++k;
-            break;
-        }
-    }
-    if (k < nw && lane == 0 && producer) {
-        // a wait gave up: wait (bounded) for this warp's copies still in flight
-        for (int kk = k; kk < issued; ++kk) mbar_wait(&fbar[kk % ring], (kk / ring) & 1);
-    }
-    if (k < nw) m[0] = m[1] = -INFINITY, l[0] = l[1] = 0.f;
+    } else {
+        // ================================================================ softmax
+        // Thread (quadrant q = warp % 4, lane): TMEM lane t = 32 q + lane, i.e.
+        // key t of the tile for S^T and head_dim element t for O^T; the warp
+        // group h = warp / 4 takes rows (columns) RPT h .. RPT h + RPT - 1.
+        constexpr int RPT = kMultiRPT;
+        const int q4 = warp & 3, h = warp >> 2;
+        const int t = q4 * 32 + lane;
+        const int c0r = RPT * h;  // first row of this thread
+        const uint32_t lane_base = static_cast<uint32_t>(q4 * 32) << 16;
+        const int G = p.group;
+        const int B = p.block_size;
+        const float sl2 = p.scale_log2;
+        // Lazy rescaling: a row's exponent base m moves (and O^T and the sums
+        // are rescaled) only when some score exceeds it by more than 2^8; the
+        // weights exp2(s - m) then stay below 256, inside the 16-bit P range.
+        constexpr float kRescaleLog2 = 8.f;
+        const int pn_t = t >> 6, ch_t = (t & 63) >> 3;  // this key's panel and 16-byte chunk in a P^T row
+        int it = 0, tb = 0;
+        bool ok = true;
+        for (int k = 0;; ++k) {
+            MultiWork w;
+            if (!multi_item(p, tab, lpt_order, k, w)) break;
+            if (w.nt == 0) continue;
+            const int R = w.n * G;
+            const bool active = c0r < R;  // this row group holds rows of the chunk
+            const uint32_t to = tmem + lane_base + C::O_COL + 32 * (it & 1) + c0r;
+            // m: the rows' exponent bases; mexp: the same with -inf as 0 (the
+            // exponent's offset); l: this thread's partial row sums
+            float m[RPT], mexp[RPT], l[RPT];
 #pragma unroll
-    for (int h = 0; h < 2; ++h) {
-        l[h] += __shfl_xor_sync(0xffffffffu, l[h], 1);
-        l[h] += __shfl_xor_sync(0xffffffffu, l[h], 2);
-    }
-
-    // ---- merge the streams of each row group, write rows or partials
-    __syncthreads();
-    float* red_m = reinterpret_cast<float*>(smem);  // [NW][16]
-    float* red_l = red_m + NW * 16;                 // [NW][16]
-    float* red_o = red_l + NW * 16;                 // [NW][16][D]
-    if (cq == 0) {
-        red_m[warp * 16 + gq] = m[0], red_l[warp * 16 + gq] = l[0];
-        red_m[warp * 16 + gq + 8] = m[1], red_l[warp * 16 + gq + 8] = l[1];
-    }
+            for (int c = 0; c < RPT; ++c) m[c] = -INFINITY, mexp[c] = 0.f, l[c] = 0.f;
+            // keys past the context in its last block (the chunk's last
+            // partition only): their V rows may hold anything, and 0 * NaN must
+            // not reach O^T, so they are zeroed before P.V
+            const int dead_lo = w.len;
+            const int dead_hi = w.ke == w.len ? ((w.len + B - 1) / B) * B : w.len;
+            for (int j = 0; j < w.nt; ++j) {
+                const int tt = tb + j;
+                const int sb = tt & 1;
+                ok = ok && mbar_wait_or_abort(&s_full[sb], (tt >> 1) & 1, abort_flag);
+                tc_fence_after();
+                float s[RPT];
+                if (active) multi_tmem_ld<RPT>(tmem + lane_base + C::S_COL + 32 * sb + c0r, s);
+                tc_fence_before();
+                mbar_arrive(&s_free[sb]);
+                // ---- mask: row r = i G + hh sees key pos iff pos <= c0 + i, i < n, pos < ke
+                const int pos = w.kb + j * KT + t;
+                const int rlo = (pos >= w.ke ? C::NR : (pos <= w.c0 ? 0 : (pos - w.c0) * G)) - c0r;
+                const int rhi = R - c0r;
+                bool exceed = false;
+                if (active) {
 #pragma unroll
-    for (int j = 0; j < DT; ++j) {
-        const int d = 8 * j + 2 * cq;
-        *reinterpret_cast<float2*>(&red_o[(warp * 16 + gq) * D + d]) = make_float2(o[j][0], o[j][1]);
-        *reinterpret_cast<float2*>(&red_o[(warp * 16 + gq + 8) * D + d]) = make_float2(o[j][2], o[j][3]);
-    }
-    __syncthreads();
-    const int rows = n * G;
-    for (int idx = threadIdx.x; idx < rows * D; idx += NW * 32) {
-        const int row = idx / D, d = idx - row * D;
-        const int rgr = row / 16, rr = row - rgr * 16;
-        float mx = -INFINITY;
-        for (int w = rgr; w < NW; w += nrg) mx = fmaxf(mx, red_m[w * 16 + rr]);
-        float sum = 0.f, acc = 0.f;
-        if (mx != -INFINITY) {
-            for (int w = rgr; w < NW; w += nrg) {
-                const float mw = red_m[w * 16 + rr];
-                if (mw != -INFINITY) {
-                    const float f = exp2f(mw - mx);
-                    sum += red_l[w * 16 + rr] * f;
-                    acc += red_o[(w * 16 + rr) * D + d] * f;
+                    for (int c = 0; c < RPT; ++c) {
+                        s[c] = (c >= rlo && c < rhi) ? s[c] * sl2 : -INFINITY;
+                        exceed |= s[c] > m[c] + kRescaleLog2;
+                    }
                 }
+                // ---- one vote per tile: a wait gave up, or a row's base must move.
+                // Then every softmax thread leaves together, or the tile's row
+                // maxima over its 128 keys become the new bases.
+                if (multi_vote_any(exceed || !ok)) {
+                    if (multi_vote_any(!ok)) {
+                        ok = false;
+                        break;
+                    }
+                    if (active) {
+                        float v[RPT];
+#pragma unroll
+                        for (int c = 0; c < RPT; ++c) v[c] = s[c];
+                        const float wm = multi_reduce_scatter<true, RPT>(v, lane);  // column lane % RPT over this warp's keys
+                        if (lane < RPT) red[warp * RPT + lane] = wm;
+                    }
+                    multi_sync_softmax();
+                    if (active) {
+                        const int cc = lane % RPT;
+                        const float cm = fmaxf(fmaxf(red[(4 * h + 0) * RPT + cc], red[(4 * h + 1) * RPT + cc]),
+                                               fmaxf(red[(4 * h + 2) * RPT + cc], red[(4 * h + 3) * RPT + cc]));
+                        bool moved = false;  // the same on the threads of a row group: m and cm are
+#pragma unroll
+                        for (int c = 0; c < RPT; ++c) moved |= __shfl_sync(0xffffffffu, cm, c) > m[c];
+                        // O^T *= alpha once the previous P.V is done (the next one waits
+                        // for this tile's P); on an item's first tile O^T is not started
+                        const bool rescale_o = j > 0 && moved;
+                        if (rescale_o)
+                            ok = __all_sync(0xffffffffu,
+                                            ok && mbar_wait_or_abort(&p_free[(tt - 1) & 1], ((tt - 1) >> 1) & 1, abort_flag));
+                        float o[RPT];
+                        if (rescale_o && ok) {
+                            tc_fence_after();
+                            multi_tmem_ld<RPT>(to, o);
+                        }
+#pragma unroll
+                        for (int c = 0; c < RPT; ++c) {
+                            const float mn = fmaxf(m[c], __shfl_sync(0xffffffffu, cm, c));
+                            const float alpha = mn == m[c] ? 1.f : ex2_approx(m[c] - mn);  // 0 when m was -inf
+                            m[c] = mn;
+                            mexp[c] = mn == -INFINITY ? 0.f : mn;
+                            l[c] *= alpha;
+                            o[c] *= alpha;
+                        }
+                        if (rescale_o && ok) multi_tmem_st<RPT>(to, o);
+                    }
+                }
+                // ---- P^T(r, key t) = exp2(s - m), bf16 as hi + lo (hi: the top 16
+                // bits of P; lo: the exact remainder rounded, |lo| < 2^-7 |P|).  A
+                // row group past the chunk's rows skips it: P.V then mixes stale
+                // P^T rows into O^T columns that are never read.
+                float pv[RPT];
+                if (active) {
+#pragma unroll
+                    for (int c = 0; c < RPT; ++c) {
+                        pv[c] = ex2_approx(s[c] - mexp[c]);
+                        l[c] += pv[c];
+                    }
+                }
+                if (active && tt >= 2)
+                    ok = __all_sync(0xffffffffu, ok && mbar_wait_or_abort(&p_free[sb], ((tt - 2) >> 1) & 1, abort_flag));
+                if (active && ok) {
+                    uint8_t* col = smem + C::P_OFF + sb * 2 * C::PBYTES + pn_t * (C::NR * 128) + (t & 7) * 2;
+#pragma unroll
+                    for (int c = 0; c < RPT; ++c) {
+                        const int r = c0r + c;
+                        uint8_t* dst = col + r * 128 + ((ch_t ^ (r & 7)) << 4);
+                        if constexpr (kBf16) {
+                            const uint32_t bits = __float_as_uint(pv[c]);
+                            *reinterpret_cast<uint16_t*>(dst) = static_cast<uint16_t>(bits >> 16);
+                            *reinterpret_cast<uint16_t*>(dst + C::PBYTES) =
+                                __bfloat16_as_ushort(__float2bfloat16_rn(pv[c] - __uint_as_float(bits & 0xFFFF0000u)));
+                        } else {
+                            *reinterpret_cast<uint16_t*>(dst) = __half_as_ushort(__float2half_rn(pv[c]));
+                        }
+                    }
+                }
+                // ---- dead V rows of this tile (the row group h = 0 threads zero them)
+                const int tk0 = w.kb + j * KT;
+                if (h == 0 && dead_lo < dead_hi && dead_hi > tk0 && dead_lo < tk0 + KT) {
+                    ok = __all_sync(0xffffffffu, ok && mbar_wait_or_abort(&v_full[tt % NSV], (tt / NSV) & 1, abort_flag));
+                    if (ok && pos >= dead_lo && pos < dead_hi) {
+                        uint8_t* vrow = smem + C::V_OFF + (tt % NSV) * C::TILE + t * 128;
+#pragma unroll
+                        for (int pn = 0; pn < C::NP; ++pn)
+#pragma unroll
+                            for (int cq = 0; cq < 8; ++cq)
+                                *reinterpret_cast<uint4*>(vrow + pn * KT * 128 + cq * 16) = make_uint4(0, 0, 0, 0);
+                    }
+                }
+                if (active) fence_proxy_async();  // P^T and zeroed V rows -> the tensor cores' (async) proxy
+                tc_fence_before();
+                mbar_arrive(&p_full[sb]);
             }
-        }
-        const float val = mx != -INFINITY ? acc / sum : 0.f;
-        const int i = row / G, hh = row - (row / G) * G;
-        const int64_t orow = (static_cast<int64_t>(q0) + i) * p.num_q_heads + static_cast<int64_t>(g) * G + hh;
-        if (direct) {
-            reinterpret_cast<T*>(p.out)[orow * D + d] = Elem<T>::from_f(val);
-        } else {
-            const int64_t pi = orow * p.num_partitions + part;
-            p.ws_out[pi * D + d] = val;
-            if (d == 0) {
-                p.ws_max[pi] = mx;
-                p.ws_sum[pi] = sum;
+            // ---- hand the item over to the epilogue warps: each row's exponent
+            // base and sum (the rows themselves stay in O^T)
+            if (multi_vote_any(!ok)) {
+                ok = false;
+                break;
             }
+            {
+                float v[RPT];
+#pragma unroll
+                for (int c = 0; c < RPT; ++c) v[c] = l[c];
+                const float ws = multi_reduce_scatter<false, RPT>(v, lane);
+                if (lane < RPT) red[warp * RPT + lane] = ws;
+            }
+            multi_sync_softmax();
+            {
+                const int cc = lane % RPT;
+                const float cl = (red[(4 * h + 0) * RPT + cc] + red[(4 * h + 1) * RPT + cc]) +
+                                 (red[(4 * h + 2) * RPT + cc] + red[(4 * h + 3) * RPT + cc]);
+                // the slot of item it - 2 is free once its epilogue read it
+                if (it >= 2) ok = ok && mbar_wait_or_abort(&o_free[it & 1], ((it - 2) >> 1) & 1, abort_flag);
+                float* st_m = stat + (it & 1) * 64;
+                if (q4 == 0 && ok) {
+                    if (lane < RPT) st_m[32 + c0r + lane] = cl;
+                    if (lane == 0) {
+#pragma unroll
+                        for (int c = 0; c < RPT; ++c) st_m[c0r + c] = m[c];
+                    }
+                }
+                mbar_arrive(&stat_full[it & 1]);
+            }
+            tb += w.nt;
+            ++it;
         }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        tc_fence_after();
+        tmem_dealloc(tmem, C::TMEM_COLS);
     }
 }
 
@@ -475,5 +928,6 @@ __global__ void __launch_bounds__(128) paged_decode_multi_merge_kernel(const Mul
 #pragma unroll
     for (int j = 0; j < DPL; ++j) dst[j] = Elem<T>::from_f(o[j] * inv);
 }
+
 
 }  // namespace pkv

@@ -114,9 +114,9 @@ int make_pool_map(CUtensorMap* map, const void* pool, int dtype, int64_t num_blo
 }
 
 // Packed query [tokens, num_q_heads, head_dim] as a 3-D tensor; one box =
-// 128 / group tokens x group heads x 128 bytes of head_dim.
+// box_tokens (default 128 / group) tokens x group heads x 128 bytes of head_dim.
 int make_query_map(CUtensorMap* map, const void* q, int dtype, int64_t tokens, int num_q_heads, int head_dim,
-                   int group) {
+                   int group, int box_tokens = 0) {
     auto fn = encode_fn();
     if (!fn) {
         snprintf(g_last_cuda_error, sizeof g_last_cuda_error, "cuTensorMapEncodeTiled unavailable");
@@ -125,7 +125,8 @@ int make_query_map(CUtensorMap* map, const void* q, int dtype, int64_t tokens, i
     const int eb = elem_bytes(dtype);
     cuuint64_t dims[3] = {(cuuint64_t)head_dim, (cuuint64_t)num_q_heads, (cuuint64_t)tokens};
     cuuint64_t strides[2] = {(cuuint64_t)head_dim * eb, (cuuint64_t)num_q_heads * head_dim * eb};
-    cuuint32_t box[3] = {(cuuint32_t)(128 / eb), (cuuint32_t)group, (cuuint32_t)(128 / group)};
+    cuuint32_t box[3] = {(cuuint32_t)(128 / eb), (cuuint32_t)group,
+                         (cuuint32_t)(box_tokens > 0 ? box_tokens : 128 / group)};
     cuuint32_t estr[3] = {1, 1, 1};
     CUresult r = fn(map, cu_type(dtype), 3, const_cast<void*>(q), dims, strides, box, estr,
                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -334,49 +335,28 @@ int decode_fp8_by_block(int block_size, int group, const pkv::DecodeParams& prm,
 }
 
 // ------------------------------------------------------------ multi-token decode dispatch
-constexpr int kMultiWarps = 4;
-#ifndef PKV_MULTI_STAGE_BUDGET
-#define PKV_MULTI_STAGE_BUDGET 65536
-#endif
-
-template <typename T, int D, int B, int RG>
-int launch_multi(const pkv::MultiParams& prm, int group, const CUtensorMap& tk, const CUtensorMap& tv, int grid,
-                 cudaStream_t s) {
-    constexpr int UT = B < 16 ? B : 16;
-    constexpr int STAGE = 2 * UT * D * 2;
-    constexpr int NST = std::max(1, std::min(4, PKV_MULTI_STAGE_BUDGET / (kMultiWarps * STAGE)));
-    using C = pkv::MultiCfg<T, D, B, NST, kMultiWarps, RG>;
-    auto kern = pkv::paged_decode_multi_kernel<T, D, B, NST, kMultiWarps, RG>;
-    const size_t smem = C::smem_bytes(prm.partition_blocks);
+// Persistent: as many CTAs as fit on the device at once (one per SM at
+// head_dim 128), at most one per item.
+template <typename T, int D>
+int launch_multi(const pkv::MultiParams& prm, int lpt, const CUtensorMap& tq, const CUtensorMap& tk,
+                 const CUtensorMap& tv, int64_t items, cudaStream_t s) {
+    using C = pkv::MultiCfg<D>;
+    auto kern = pkv::paged_decode_multi_kernel<T, D>;
     int dev = 0;
     PKV_CUDA(cudaGetDevice(&dev));
-    static size_t configured[64] = {};
-    size_t& have = configured[dev & 63];
-    if (smem > have) {
-        PKV_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
-        have = smem;
+    static int resident[64] = {};  // CTAs per SM, per device (0: not configured yet)
+    int& per_sm = resident[dev & 63];
+    if (per_sm == 0) {
+        PKV_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM));
+        int n = 0;
+        PKV_CUDA(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kern, pkv::kMultiThreads, C::SMEM));
+        if (n <= 0) return PKV_EUNSUPPORTED;
+        per_sm = n;
     }
-    kern<<<grid, kMultiWarps * 32, smem, s>>>(prm, group, tk, tv);
+    const int grid = (int)std::min<int64_t>(items, (int64_t)sm_count() * per_sm);
+    kern<<<grid, pkv::kMultiThreads, C::SMEM, s>>>(prm, lpt, tq, tk, tv);
     PKV_CUDA(cudaGetLastError());
     return PKV_OK;
-}
-
-template <typename T, int D, int B>
-int multi_by_rows(int row_groups, const pkv::MultiParams& prm, int group, const CUtensorMap& tk,
-                  const CUtensorMap& tv, int grid, cudaStream_t s) {
-    return row_groups == 1 ? launch_multi<T, D, B, 1>(prm, group, tk, tv, grid, s)
-                           : launch_multi<T, D, B, 2>(prm, group, tk, tv, grid, s);
-}
-
-template <typename T, int D>
-int multi_by_block(int block_size, int row_groups, const pkv::MultiParams& prm, int group, const CUtensorMap& tk,
-                   const CUtensorMap& tv, int grid, cudaStream_t s) {
-    switch (block_size) {
-        case 8: return multi_by_rows<T, D, 8>(row_groups, prm, group, tk, tv, grid, s);
-        case 16: return multi_by_rows<T, D, 16>(row_groups, prm, group, tk, tv, grid, s);
-        case 32: return multi_by_rows<T, D, 32>(row_groups, prm, group, tk, tv, grid, s);
-        default: return PKV_EUNSUPPORTED;
-    }
 }
 
 // The merge always follows this library's own decode kernel in the stream,
@@ -1033,8 +1013,8 @@ int pkv_paged_attention_decode_multi(void* out, const void* query, const void* k
                                                               max_seq_len, (int)(pb * block_size))
                                   : 0;
     if (need > 0 && (!workspace || workspace_bytes < need || !aligned16(workspace))) return PKV_EWORKSPACE;
-    const int64_t grid = (int64_t)num_chunks * parts * num_kv_heads;
-    if (grid > INT32_MAX) return PKV_EUNSUPPORTED;
+    const int64_t items = (int64_t)num_chunks * parts * num_kv_heads;  // (chunk, partition, KV head)
+    if (items >= (int64_t(1) << 30)) return PKV_EUNSUPPORTED;  // the kernel ranks items in 32 bits
 
     if (checked_mode()) {
         std::vector<int32_t> qsl, lens;
@@ -1052,16 +1032,17 @@ int pkv_paged_attention_decode_multi(void* out, const void* query, const void* k
         if (rc) return rc;
     }
 
-    const int unit_rows = block_size < 16 ? block_size : 16;
-    CUtensorMap tk, tv;
-    int rc = make_pool_map(&tk, key_cache, dtype, num_blocks, block_size, num_kv_heads, head_dim, unit_rows);
+    CUtensorMap tq, tk, tv;
+    // Q: 32 / G tokens x G heads = the 32 rows of a KV head; K/V: one box per block
+    int rc = make_query_map(&tq, query, dtype, total_q_tokens, num_q_heads, head_dim, group, 32 / group);
     if (rc) return rc;
-    rc = make_pool_map(&tv, value_cache, dtype, num_blocks, block_size, num_kv_heads, head_dim, unit_rows);
+    rc = make_pool_map(&tk, key_cache, dtype, num_blocks, block_size, num_kv_heads, head_dim);
+    if (rc) return rc;
+    rc = make_pool_map(&tv, value_cache, dtype, num_blocks, block_size, num_kv_heads, head_dim);
     if (rc) return rc;
 
     pkv::MultiParams prm;
     prm.out = out;
-    prm.query = query;
     prm.block_tables = block_tables;
     prm.seq_lens = seq_lens;
     prm.query_start_loc = query_start_loc;
@@ -1074,19 +1055,21 @@ int pkv_paged_attention_decode_multi(void* out, const void* query, const void* k
     prm.num_chunks = num_chunks;
     prm.num_q_heads = num_q_heads;
     prm.num_kv_heads = num_kv_heads;
+    prm.group = group;
+    prm.block_size = block_size;
     prm.max_blocks_per_seq = max_blocks_per_seq;
     prm.num_blocks = num_blocks;
     prm.partition_blocks = (int)pb;
     prm.num_partitions = (int)parts;
     prm.total_q_tokens = total_q_tokens;
-    const int row_groups = max_q_len * group > 16 ? 2 : 1;
+    const int lpt = num_chunks <= pkv::kMultiLptChunks ? 1 : 0;
     const bool bf16 = dtype == PKV_BF16;
     if (head_dim == 64)
-        rc = bf16 ? multi_by_block<__nv_bfloat16, 64>(block_size, row_groups, prm, group, tk, tv, (int)grid, s)
-                  : multi_by_block<__half, 64>(block_size, row_groups, prm, group, tk, tv, (int)grid, s);
+        rc = bf16 ? launch_multi<__nv_bfloat16, 64>(prm, lpt, tq, tk, tv, items, s)
+                  : launch_multi<__half, 64>(prm, lpt, tq, tk, tv, items, s);
     else
-        rc = bf16 ? multi_by_block<__nv_bfloat16, 128>(block_size, row_groups, prm, group, tk, tv, (int)grid, s)
-                  : multi_by_block<__half, 128>(block_size, row_groups, prm, group, tk, tv, (int)grid, s);
+        rc = bf16 ? launch_multi<__nv_bfloat16, 128>(prm, lpt, tq, tk, tv, items, s)
+                  : launch_multi<__half, 128>(prm, lpt, tq, tk, tv, items, s);
     if (rc || parts <= 1) return rc;
 
     pkv::MultiMergeParams mp;
@@ -1117,14 +1100,15 @@ int pkv_decode_multi_partition_size(int num_chunks, int num_kv_heads, int block_
     if (num_chunks < 0 || num_kv_heads <= 0 || block_size <= 0 || max_seq_len < 0) return PKV_EINVAL;
     const int64_t pairs = (int64_t)num_chunks * num_kv_heads;
     if (max_seq_len <= 0 || pairs == 0) return 0;
-    // About eight CTAs per SM over the whole launch, so that CTAs of uneven
-    // length even out; partitions of at least 256 tokens.
-    // Never more than kMaxPartitionBlocks blocks per partition.
+    // About eight work items per SM over the whole launch, so that the
+    // persistent CTAs' loads even out; partitions of at least 256 tokens, in
+    // whole 128-key tiles.  Never more than kMaxPartitionBlocks blocks.
     const int64_t target = 8 * (int64_t)sm_count();
     const int64_t cap = kMaxPartitionBlocks * block_size;
     const int64_t parts = std::max(std::max<int64_t>(1, ceil_div(target, pairs)), ceil_div(max_seq_len, cap));
     int64_t ps = std::max<int64_t>(256, ceil_div(max_seq_len, parts));
-    ps = std::min(ceil_div(ps, block_size) * block_size, cap);
+    const int64_t unit = 128 % block_size == 0 ? 128 : block_size;
+    ps = std::min(ceil_div(ps, unit) * unit, cap);
     return ps >= max_seq_len ? 0 : (int)ps;
 }
 

@@ -145,6 +145,43 @@ __device__ __forceinline__ bool mbar_wait_or_abort(uint64_t* bar, uint32_t parit
     }
 }
 
+// try_wait with a suspend-time hint: a thread whose phase is not complete
+// sleeps until it completes (or the hint's time passes) instead of spinning,
+// leaving the issue slots to the warps that compute.
+__device__ __forceinline__ bool mbar_test_suspend(uint64_t* bar, uint32_t parity) {
+    uint32_t done;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(done)
+        : "r"(smem_u32(bar)), "r"(parity), "r"(100000u)
+        : "memory");
+    return done != 0;
+}
+
+// mbar_wait_or_abort for roles that only wait (loaders, MMA issuers, an
+// epilogue): the same limit and abort flag, the thread suspended between polls.
+__device__ __forceinline__ bool mbar_wait_or_abort_idle(uint64_t* bar, uint32_t parity, volatile int* abort) {
+    if (mbar_poll(bar, parity)) return true;
+    const uint64_t limit = c_main_wait_limit_ns;
+    if (limit == 0) {
+        flag_error(PKV_DEVERR_TIMEOUT);
+        *abort = 1;
+        return false;
+    }
+    const uint64_t t0 = global_timer_ns();
+    while (true) {
+        if (mbar_test_suspend(bar, parity)) return true;
+        if (*abort) return false;
+        if (global_timer_ns() - t0 > limit) {
+            flag_error(PKV_DEVERR_TIMEOUT);
+            *abort = 1;
+            return false;
+        }
+    }
+}
+
 // Programmatic dependent launch.  griddep_wait blocks until the grids this
 // one depends on have completed and their writes are visible (a no-op for a
 // grid launched without the programmatic-serialisation attribute);

@@ -1,7 +1,8 @@
 """Multi-token decode (speculative verification): every sequence appends a few
 draft tokens and each of them attends causally over the whole cache.  Both
-calls that compute it are checked: the chunked-prefill call (tcgen05) and the
-multi-token decode call (warp MMAs, split-K partitions)."""
+calls that compute it are checked: the chunked-prefill call and the multi-token
+decode call (keys on the M side of the tcgen05 MMAs, persistent CTAs, split-K
+partitions merged by a second kernel)."""
 import numpy as np
 import pytest
 import torch
@@ -53,7 +54,7 @@ def test_multi_token_matches_oracle(case, call):
         assert_close(out, ref, dtype, f"multi-token {call} {case} partition {part}")
 
 
-# more rows than one warp's 16: two row groups (n * G up to 32), and one head per KV head with 16-token drafts
+# up to 32 rows per KV head (n * G): G 4 and 8 with long drafts, and one head per KV head with 16-token drafts
 ROW_CASES = [
     (torch.bfloat16, 128, 16, 32, 8, [40, 1000, 3], [8, 5, 7]),
     (torch.float16, 64, 32, 16, 16, [100, 31], [16, 9]),
@@ -72,6 +73,41 @@ def test_multi_token_row_groups(case):
         torch.cuda.synchronize()
         assert pkv.get_device_error() == 0
         assert_close(out, ref, dtype, f"multi-token rows {case} partition {part}")
+
+
+def test_multi_token_many_chunks_and_partitions():
+    """More chunks than the longest-first schedule takes (partition-major item
+    order), and partitions of one, two and three 128-key tiles and of a
+    size that leaves a partial tile at every partition end."""
+    R = 150
+    rng = np.random.default_rng(11)
+    c0s = rng.integers(0, 700, size=R).tolist()
+    ns = rng.integers(1, 9, size=R).tolist()
+    m = workloads.mixed_workload("mtm", [], c0s, ns, 16, 4, 128, 16, torch.float16, seed=12, poison=True)
+    pre_k, pre_v = m.decode.key_caches[0].clone(), m.decode.value_caches[0].clone()
+    ref = oracle_prefill_chunks(m, pre_k, pre_v)
+    for part in (None, 0, 128, 256, 384, 80):
+        out, _, _ = run_gpu(m, call="multi", partition_size=part)
+        torch.cuda.synchronize()
+        assert pkv.get_device_error() == 0
+        assert_close(out, ref, torch.float16, f"{R} chunks, partition {part}")
+
+
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float16])
+def test_multi_token_rescales_mid_partition(dtype):
+    """Queries scaled up 24x: scores spread over tens of units in the log2
+    domain, so a row's running maximum keeps growing by more than 2^8 after
+    the first key tile and the accumulated O is rescaled in tensor memory."""
+    m = workloads.mixed_workload("mts", [], [900, 2500, 130, 1700], [4, 2, 6, 3], 32, 8, 128, 32, dtype, seed=21,
+                                 poison=True)
+    m.chunk_query.mul_(24.0)
+    pre_k, pre_v = m.decode.key_caches[0].clone(), m.decode.value_caches[0].clone()
+    ref = oracle_prefill_chunks(m, pre_k, pre_v)
+    for part in (0, 512, None):
+        out, _, _ = run_gpu(m, call="multi", partition_size=part)
+        torch.cuda.synchronize()
+        assert pkv.get_device_error() == 0
+        assert_close(out, ref, dtype, f"large scores, partition {part}")
 
 
 def test_multi_token_call_rejects_too_many_rows():
