@@ -103,7 +103,7 @@ struct MultiCfg {
     static constexpr int NSK = 3;              // stages of K: refilled once S(t) is done, 3 tiles ahead
     static constexpr int NSV = 2;              // stages of V: refilled once PV(t) is done
     static constexpr int QBYTES = NP * NR * 128;
-    static constexpr int PBYTES = 2 * NR * 128;  // one P^T term: 32 rows x 128 keys, two 64-key panels
+    static constexpr int PBYTES = KT * NR * 2;  // one P^T term: 128 keys x 32 rows, 64 bytes per key
     static constexpr int K_OFF = 0;
     static constexpr int V_OFF = K_OFF + NSK * TILE;
     static constexpr int Q_OFF = V_OFF + NSV * TILE;  // [2] query tiles
@@ -546,9 +546,9 @@ __global__ void __launch_bounds__(kMultiThreads, 1) paged_decode_multi_kernel(co
         if (lane == 0) {
             const bool s_role = warp == kMultiMmaSWarp;
             constexpr uint32_t IDESC_S = umma_idesc_f16(128, C::NR, kBf16, false, false);
-            constexpr uint32_t IDESC_O = umma_idesc_f16(128, C::NR, kBf16, true, false);  // A (V^T) MN-major
+            constexpr uint32_t IDESC_O = umma_idesc_f16(128, C::NR, kBf16, true, true);  // A (V^T), B (P^T) MN-major
             constexpr int kKP = KT * 128 / 16;    // panel stride of a K tile (16-byte units)
-            constexpr int kQP = C::NR * 128 / 16;  // panel stride of the Q rows and of P^T
+            constexpr int kQP = C::NR * 128 / 16;  // panel stride of the Q rows
             // Descriptors made once; a 16-element k slice adds its byte offset / 16.
             // V^T: M = head_dim in 64-element atoms (the tile's panels, LBO apart;
             // one panel at head_dim 64, read twice: lanes 64-127 of O^T repeat 0-63),
@@ -556,7 +556,9 @@ __global__ void __launch_bounds__(kMultiThreads, 1) paged_decode_multi_kernel(co
             const uint64_t kdesc0 = smem_desc_sw128(smem_u32(smem + C::K_OFF), 16, 1024);
             const uint64_t vdesc0 = smem_desc_sw128(smem_u32(smem + C::V_OFF), C::NP > 1 ? KT * 128 : 0, 1024);
             const uint64_t qdesc0 = smem_desc_sw128(smem_u32(smem + C::Q_OFF), 16, 1024);
-            const uint64_t pdesc0 = smem_desc_sw128(smem_u32(smem + C::P_OFF), 16, 1024);
+            // P^T: N = 32 rows = one 64-byte swizzle atom wide (MN-major), K = keys,
+            // 8 keys per 512-byte atom (SBO)
+            const uint64_t pdesc0 = smem_desc_sw64(smem_u32(smem + C::P_OFF), C::PBYTES, 512);
             int it = 0, tb = 0;  // items and key tiles of this CTA so far
             bool ok = true;
             for (int k = 0; ok; ++k) {
@@ -600,7 +602,7 @@ __global__ void __launch_bounds__(kMultiThreads, 1) paged_decode_multi_kernel(co
 #pragma unroll
                         for (int kk = 0; kk < KT / 16; ++kk) {
                             const uint64_t a = vd + kk * (16 * 128 / 16);  // 16 key rows of 128 bytes
-                            const uint64_t b = pd + (kk / 4) * kQP + (kk % 4) * 2;
+                            const uint64_t b = pd + kk * (2 * 512 / 16);  // 16 keys: two 512-byte atoms
                             umma_f16_ss(o_col, a, b, IDESC_O, (j == 0 && kk == 0) ? 0u : 1u);
                             if constexpr (kBf16) umma_f16_ss(o_col, a, b + C::PBYTES / 16, IDESC_O, 1u);
                         }
@@ -691,7 +693,6 @@ __global__ void __launch_bounds__(kMultiThreads, 1) paged_decode_multi_kernel(co
         // are rescaled) only when some score exceeds it by more than 2^8; the
         // weights exp2(s - m) then stay below 256, inside the 16-bit P range.
         constexpr float kRescaleLog2 = 8.f;
-        const int pn_t = t >> 6, ch_t = (t & 63) >> 3;  // this key's panel and 16-byte chunk in a P^T row
         int it = 0, tb = 0;
         bool ok = true;
         for (int k = 0;; ++k) {
@@ -702,10 +703,18 @@ __global__ void __launch_bounds__(kMultiThreads, 1) paged_decode_multi_kernel(co
             const bool active = c0r < R;  // this row group holds rows of the chunk
             const uint32_t to = tmem + lane_base + C::O_COL + 32 * (it & 1) + c0r;
             // m: the rows' exponent bases; mexp: the same with -inf as 0 (the
-            // exponent's offset); l: this thread's partial row sums
-            float m[RPT], mexp[RPT], l[RPT];
+            // exponent's offset); mth: m + 2^8 in the log2 domain, the rescale
+            // threshold; l: this thread's partial row sums.  A row past the
+            // chunk's rows gets m = +inf: its weights are 0 and it never votes.
+            float m[RPT], mexp[RPT], mth[RPT], l[RPT];
 #pragma unroll
-            for (int c = 0; c < RPT; ++c) m[c] = -INFINITY, mexp[c] = 0.f, l[c] = 0.f;
+            for (int c = 0; c < RPT; ++c) {
+                const bool live = c0r + c < R;
+                m[c] = live ? -INFINITY : INFINITY;
+                mexp[c] = live ? 0.f : INFINITY;
+                mth[c] = m[c];
+                l[c] = 0.f;
+            }
             // keys past the context in its last block (the chunk's last
             // partition only): their V rows may hold anything, and 0 * NaN must
             // not reach O^T, so they are zeroed before P.V
@@ -720,16 +729,26 @@ __global__ void __launch_bounds__(kMultiThreads, 1) paged_decode_multi_kernel(co
                 if (active) multi_tmem_ld<RPT>(tmem + lane_base + C::S_COL + 32 * sb + c0r, s);
                 tc_fence_before();
                 mbar_arrive(&s_free[sb]);
-                // ---- mask: row r = i G + hh sees key pos iff pos <= c0 + i, i < n, pos < ke
+                // ---- mask: row r = i G + hh sees key pos iff pos <= c0 + i, i < n, pos < ke;
+                // a tile whose keys all lie before the chunk's first new token and
+                // inside the partition needs none
                 const int pos = w.kb + j * KT + t;
-                const int rlo = (pos >= w.ke ? C::NR : (pos <= w.c0 ? 0 : (pos - w.c0) * G)) - c0r;
-                const int rhi = R - c0r;
+                const int tk0 = w.kb + j * KT;
                 bool exceed = false;
                 if (active) {
+                    if (tk0 + KT - 1 <= min(w.c0, w.ke - 1)) {
 #pragma unroll
-                    for (int c = 0; c < RPT; ++c) {
-                        s[c] = (c >= rlo && c < rhi) ? s[c] * sl2 : -INFINITY;
-                        exceed |= s[c] > m[c] + kRescaleLog2;
+                        for (int c = 0; c < RPT; ++c) {
+                            s[c] *= sl2;
+                            exceed |= s[c] > mth[c];
+                        }
+                    } else {
+                        const int rlo = (pos >= w.ke ? C::NR : (pos <= w.c0 ? 0 : (pos - w.c0) * G)) - c0r;
+#pragma unroll
+                        for (int c = 0; c < RPT; ++c) {
+                            s[c] = c >= rlo ? s[c] * sl2 : -INFINITY;
+                            exceed |= s[c] > mth[c];
+                        }
                     }
                 }
                 // ---- one vote per tile: a wait gave up, or a row's base must move.
@@ -772,6 +791,7 @@ __global__ void __launch_bounds__(kMultiThreads, 1) paged_decode_multi_kernel(co
                             const float alpha = mn == m[c] ? 1.f : ex2_approx(m[c] - mn);  // 0 when m was -inf
                             m[c] = mn;
                             mexp[c] = mn == -INFINITY ? 0.f : mn;
+                            mth[c] = mn + kRescaleLog2;
                             l[c] *= alpha;
                             o[c] *= alpha;
                         }
@@ -793,23 +813,34 @@ __global__ void __launch_bounds__(kMultiThreads, 1) paged_decode_multi_kernel(co
                 if (active && tt >= 2)
                     ok = __all_sync(0xffffffffu, ok && mbar_wait_or_abort(&p_free[sb], ((tt - 2) >> 1) & 1, abort_flag));
                 if (active && ok) {
-                    uint8_t* col = smem + C::P_OFF + sb * 2 * C::PBYTES + pn_t * (C::NR * 128) + (t & 7) * 2;
+                    // P^T is the B operand in the MN-major, 64-byte-swizzled layout:
+                    // key k's 32 row weights are 64 contiguous bytes (k % 8 of an
+                    // 8-key, 512-byte atom; 16-byte piece q at q ^ ((k >> 1) & 3)),
+                    // so this thread's rows are 16-byte pieces of one line.
+                    uint8_t* line = smem + C::P_OFF + sb * 2 * C::PBYTES + (t >> 3) * 512 + (t & 7) * 64;
+                    const int sw = (t >> 1) & 3;
 #pragma unroll
-                    for (int c = 0; c < RPT; ++c) {
-                        const int r = c0r + c;
-                        uint8_t* dst = col + r * 128 + ((ch_t ^ (r & 7)) << 4);
-                        if constexpr (kBf16) {
-                            const uint32_t bits = __float_as_uint(pv[c]);
-                            *reinterpret_cast<uint16_t*>(dst) = static_cast<uint16_t>(bits >> 16);
-                            *reinterpret_cast<uint16_t*>(dst + C::PBYTES) =
-                                __bfloat16_as_ushort(__float2bfloat16_rn(pv[c] - __uint_as_float(bits & 0xFFFF0000u)));
-                        } else {
-                            *reinterpret_cast<uint16_t*>(dst) = __half_as_ushort(__float2half_rn(pv[c]));
+                    for (int q = 0; q < RPT / 8; ++q) {
+                        uint8_t* dst = line + ((((c0r >> 3) + q) ^ sw) << 4);
+                        uint32_t hw[4], lw[4];
+#pragma unroll
+                        for (int i = 0; i < 4; ++i) {
+                            const float a = pv[8 * q + 2 * i], b = pv[8 * q + 2 * i + 1];
+                            if constexpr (kBf16) {
+                                const uint32_t ba = __float_as_uint(a), bb = __float_as_uint(b);
+                                hw[i] = __byte_perm(ba, bb, 0x7632);  // the top 16 bits of each
+                                lw[i] = Elem<T>::pack(a - __uint_as_float(ba & 0xFFFF0000u),
+                                                      b - __uint_as_float(bb & 0xFFFF0000u));
+                            } else {
+                                hw[i] = Elem<T>::pack(a, b);
+                            }
                         }
+                        *reinterpret_cast<uint4*>(dst) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+                        if constexpr (kBf16)
+                            *reinterpret_cast<uint4*>(dst + C::PBYTES) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
                     }
                 }
                 // ---- dead V rows of this tile (the row group h = 0 threads zero them)
-                const int tk0 = w.kb + j * KT;
                 if (h == 0 && dead_lo < dead_hi && dead_hi > tk0 && dead_lo < tk0 + KT) {
                     ok = __all_sync(0xffffffffu, ok && mbar_wait_or_abort(&v_full[tt % NSV], (tt / NSV) & 1, abort_flag));
                     if (ok && pos >= dead_lo && pos < dead_hi) {
