@@ -37,8 +37,8 @@
 //    After the item's last tile the row sums are reduced the same way and
 //    handed, with the rows' exponent bases, to the epilogue warps.
 //  * K loader -- per item the Q rows (one TMA box per 64 dims), then the K
-//    tiles (one box per physical block and 64 dims) into three stages;
-//    V loader (the last warp) -- the V tiles into two.
+//    tiles (one box per physical block and 64 dims) into two stages;
+//    V loader (the last warp) -- the V tiles into three.
 //  * S issuer, P.V issuer (lane 0 each) -- the S^T MMAs of each tile as soon
 //    as its K stage and S buffer are ready; the P.V MMAs as soon as P^T and
 //    the V stage are.  The softmax of tile j runs while S(j+1) and PV(j-1) run.
@@ -100,8 +100,11 @@ struct MultiCfg {
     static constexpr int NR = 32;              // query rows per KV head (N of both products)
     static constexpr int NP = D / 64;          // 128-byte panels of a 16-bit row
     static constexpr int TILE = NP * KT * 128;  // one K (or V) tile
-    static constexpr int NSK = 3;              // stages of K: refilled once S(t) is done, 3 tiles ahead
-    static constexpr int NSV = 2;              // stages of V: refilled once PV(t) is done
+    // Stages of K (refilled once S(t) is done; the S MMAs run well ahead of
+    // the softmax) and of V (refilled once PV(t) is done, which waits for the
+    // softmax of tile t: three stages cover the load latency).
+    static constexpr int NSK = 2;
+    static constexpr int NSV = 3;
     static constexpr int QBYTES = NP * NR * 128;
     static constexpr int PBYTES = KT * NR * 2;  // one P^T term: 128 keys x 32 rows, 64 bytes per key
     static constexpr int K_OFF = 0;
