@@ -93,6 +93,7 @@ constexpr int kMultiLoadVWarp = kMultiSoftmaxWarps + 7;  // loads the V tiles (k
 constexpr int kMultiThreads = (kMultiSoftmaxWarps + 8) * 32;
 constexpr int kMultiLptChunks = 128;  // up to this many chunks the items go longest first
 constexpr int kMultiKT = 128;         // keys per tile
+constexpr int kMultiItemCache = 32;   // items a CTA decodes once, at its start
 
 template <int D>
 struct MultiCfg {
@@ -117,7 +118,8 @@ struct MultiCfg {
     // schedule tables: full-partition prefix [R + 1], remainder tiles [R], remainder order [R], counts [2],
     // then the chunks' q0, n, len, partitions [R] each
     static constexpr int TAB_INTS = 7 * kMultiLptChunks + 3;
-    static constexpr int BAR_OFF = (TAB_OFF + TAB_INTS * 4 + 7) & ~7;
+    static constexpr int ITEM_OFF = (TAB_OFF + TAB_INTS * 4 + 15) & ~15;  // the CTA's first items, decoded
+    static constexpr int BAR_OFF = ITEM_OFF + kMultiItemCache * 48;
     static constexpr int NBAR = 2 * NSK + 2 * NSV + 8 * 2 + 2 + 2;
     static constexpr int SMEM = 1024 + BAR_OFF + (NBAR + 2) * 8;
     static constexpr uint32_t TMEM_COLS = 128;
@@ -156,13 +158,14 @@ __device__ __forceinline__ MultiChunk multi_chunk(const MultiParams& p, int r, b
 }
 
 // One work item: chunk r's partition `part` for KV head g.
-struct MultiWork {
+struct alignas(16) MultiWork {
     int r, part, g;
     int q0, n, c0, len;
     int kb, ke;  // keys [kb, ke)
     int nt;      // key tiles (0: nothing to do)
     bool direct;  // the chunk has one partition: write rows, not partials
 };
+static_assert(sizeof(MultiWork) == 48, "item cache entries");
 
 // Schedule tables (longest first), built once per CTA; every thread of the
 // CTA calls it (block-wide barriers), threads below num_chunks do the work.
@@ -224,7 +227,8 @@ __device__ __forceinline__ void multi_build_schedule(const MultiParams& p, int* 
 }
 
 // The CTA's k-th item (rank blockIdx.x + k * gridDim.x); false past the last.
-__device__ __forceinline__ bool multi_item(const MultiParams& p, const int* tab, bool lpt, int k, MultiWork& w) {
+__device__ __forceinline__ bool multi_item(const MultiParams& p, const int* tab, bool lpt, int k, MultiWork& w,
+                                           bool report) {
     // 32-bit ranks: the launch keeps chunks x partitions x KV heads below 2^30
     const int H = p.num_kv_heads;
     const int rank = static_cast<int>(blockIdx.x) + k * static_cast<int>(gridDim.x);
@@ -270,8 +274,8 @@ __device__ __forceinline__ bool multi_item(const MultiParams& p, const int* tab,
         c.len = geo[2 * kMultiLptChunks + r];
         c.nparts = geo[3 * kMultiLptChunks + r];
         c.ok = c.nparts > 0;
-    } else {  // errors reported by item (0, 0)'s loader lane 0
-        c = multi_chunk(p, r, part == 0 && g == 0 && threadIdx.x == kMultiLoadWarp * 32);
+    } else {  // errors reported by the decoding of item (0, 0)
+        c = multi_chunk(p, r, report && part == 0 && g == 0);
     }
     w.nt = 0;
     if (!c.ok || part >= c.nparts) return true;
@@ -440,10 +444,26 @@ __global__ void __launch_bounds__(kMultiThreads, 1) paged_decode_multi_kernel(co
         fence_mbar_init();
     }
     if (lpt_order) multi_build_schedule(p, tab, blockIdx.x == 0);
+    // The CTA's first items, decoded once for every role (nt = -1: past the last)
+    MultiWork* items = reinterpret_cast<MultiWork*>(smem + C::ITEM_OFF);
+    if (lpt_order) __syncthreads();  // the schedule tables
+    if (tid < kMultiItemCache) {
+        MultiWork w;
+        if (!multi_item(p, tab, lpt_order, tid, w, true)) w.nt = -1;
+        items[tid] = w;
+    }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
+    // item k of this CTA: false past the last one
+    auto next_item = [&](int k, MultiWork& w) -> bool {
+        if (k < kMultiItemCache) {
+            w = items[k];
+            return w.nt >= 0;
+        }
+        return multi_item(p, tab, lpt_order, k, w, false);
+    };
 
     if (warp == kMultiLoadWarp || warp == kMultiLoadVWarp) {
         // ================================================================ loaders (whole warps)
@@ -467,7 +487,7 @@ __global__ void __launch_bounds__(kMultiThreads, 1) paged_decode_multi_kernel(co
             return __shfl_sync(0xffffffffu, got, 0) != 0;
         };
         auto next_work = [&](int& k, MultiWork& w) -> bool {
-            while (multi_item(p, tab, lpt_order, k++, w))
+            while (next_item(k++, w))
                 if (w.nt > 0) return true;
             return false;
         };
@@ -566,7 +586,7 @@ __global__ void __launch_bounds__(kMultiThreads, 1) paged_decode_multi_kernel(co
             bool ok = true;
             for (int k = 0; ok; ++k) {
                 MultiWork w;
-                if (!multi_item(p, tab, lpt_order, k, w)) break;
+                if (!next_item(k, w)) break;
                 if (w.nt == 0) continue;
                 if (s_role) {
                     // S^T(t) = K_t . Q^T into S buffer t & 1
@@ -638,7 +658,7 @@ __global__ void __launch_bounds__(kMultiThreads, 1) paged_decode_multi_kernel(co
         bool ok = true;
         for (int k = 0; ok; ++k) {
             MultiWork w;
-            if (!multi_item(p, tab, lpt_order, k, w)) break;
+            if (!next_item(k, w)) break;
             if (w.nt == 0) continue;
             const int ob = it & 1;
             const int got = lane == 0 ? (mbar_wait_or_abort_idle(&o_full[ob], (it >> 1) & 1, abort_flag) &&
@@ -700,7 +720,7 @@ __global__ void __launch_bounds__(kMultiThreads, 1) paged_decode_multi_kernel(co
         bool ok = true;
         for (int k = 0;; ++k) {
             MultiWork w;
-            if (!multi_item(p, tab, lpt_order, k, w)) break;
+            if (!next_item(k, w)) break;
             if (w.nt == 0) continue;
             const int R = w.n * G;
             const bool active = c0r < R;  // this row group holds rows of the chunk
