@@ -1100,10 +1100,12 @@ int pkv_decode_multi_partition_size(int num_chunks, int num_kv_heads, int block_
     if (num_chunks < 0 || num_kv_heads <= 0 || block_size <= 0 || max_seq_len < 0) return PKV_EINVAL;
     const int64_t pairs = (int64_t)num_chunks * num_kv_heads;
     if (max_seq_len <= 0 || pairs == 0) return 0;
-    // About eight work items per SM over the whole launch, so that the
-    // persistent CTAs' loads even out; partitions of at least 256 tokens, in
-    // whole 128-key tiles.  Never more than kMaxPartitionBlocks blocks.
-    const int64_t target = 8 * (int64_t)sm_count();
+    // At least two work items per SM over the whole launch: the persistent
+    // CTAs take them longest first, and an item boundary costs about two key
+    // tiles, so (chunk, KV head) pairs are split only when there are fewer;
+    // partitions of at least 256 tokens, in whole 128-key tiles.  Never more
+    // than kMaxPartitionBlocks blocks.
+    const int64_t target = 2 * (int64_t)sm_count();
     const int64_t cap = kMaxPartitionBlocks * block_size;
     const int64_t parts = std::max(std::max<int64_t>(1, ceil_div(target, pairs)), ceil_div(max_seq_len, cap));
     int64_t ps = std::max<int64_t>(256, ceil_div(max_seq_len, parts));
