@@ -667,12 +667,8 @@ __global__ void __launch_bounds__(kMultiThreads, 1) paged_decode_multi_kernel(co
             ok = __shfl_sync(0xffffffffu, got, 0) != 0;
             if (!ok) break;
             tc_fence_after();
-            float o[32];
-            if (q4 * 32 < D) tmem_ld32(tmem + lane_base + C::O_COL + 32 * ob, o);  // lanes past head_dim 64 repeat 0-63
-            const float mrow = stat[ob * 64 + lane];       // row `lane`
+            const float mrow = stat[ob * 64 + lane];  // row `lane`
             const float lsum = stat[ob * 64 + 32 + lane];
-            tc_fence_before();
-            mbar_arrive(&o_free[ob]);
             const float inv = lsum > 0.f ? 1.f / lsum : 0.f;  // a row without keys writes 0
             const int R = w.n * G;
             if (!w.direct && q4 == 0 && lane < R) {
@@ -681,22 +677,39 @@ __global__ void __launch_bounds__(kMultiThreads, 1) paged_decode_multi_kernel(co
                 p.ws_max[pi] = mrow;
                 p.ws_sum[pi] = lsum;
             }
+            // O^T's lane t in two halves of 16 rows (lanes past head_dim 64 repeat
+            // 0-63); O^T and the stats are released once both are out: the next
+            // item on this O^T buffer is two items away
             if (q4 * 32 < D) {
-                int i = 0, hh = 0;
+                // row r = i G + hh: element t sits (i Hq + hh) rows (times the
+                // partitions for partials) after the item's first row
+                const int64_t row0 = static_cast<int64_t>(w.q0) * p.num_q_heads + static_cast<int64_t>(w.g) * G;
+                T* out_t = reinterpret_cast<T*>(p.out) + row0 * D + t;
+                float* part_t = w.direct ? nullptr : p.ws_out + (row0 * p.num_partitions + w.part) * D + t;
+                const int row_step = w.direct ? D : p.num_partitions * D;   // next head
+                const int tok_step = (p.num_q_heads - G) * row_step;        // next token, after G heads
+                int off = 0, hh = 0;
 #pragma unroll
-                for (int r = 0; r < 32; ++r) {
-                    const float val = o[r] * __shfl_sync(0xffffffffu, inv, r);
-                    if (r < R) {
-                        const int64_t orow = static_cast<int64_t>(w.q0 + i) * p.num_q_heads +
-                                             static_cast<int64_t>(w.g) * G + hh;
-                        if (w.direct)
-                            reinterpret_cast<T*>(p.out)[orow * D + t] = Elem<T>::from_f(val);
-                        else
-                            p.ws_out[(orow * p.num_partitions + w.part) * D + t] = val;
+                for (int half = 0; half < 2; ++half) {
+                    float o[16];
+                    multi_tmem_ld<16>(tmem + lane_base + C::O_COL + 32 * ob + 16 * half, o);
+#pragma unroll
+                    for (int c = 0; c < 16; ++c) {
+                        const int r = 16 * half + c;
+                        const float val = o[c] * __shfl_sync(0xffffffffu, inv, r);
+                        if (r < R) {
+                            if (w.direct)
+                                out_t[off] = Elem<T>::from_f(val);
+                            else
+                                part_t[off] = val;
+                        }
+                        off += row_step;
+                        if (++hh == G) hh = 0, off += tok_step;
                     }
-                    if (++hh == G) hh = 0, ++i;
                 }
             }
+            tc_fence_before();
+            mbar_arrive(&o_free[ob]);
             ++it;
         }
     } else {
@@ -725,17 +738,15 @@ __global__ void __launch_bounds__(kMultiThreads, 1) paged_decode_multi_kernel(co
             const int R = w.n * G;
             const bool active = c0r < R;  // this row group holds rows of the chunk
             const uint32_t to = tmem + lane_base + C::O_COL + 32 * (it & 1) + c0r;
-            // m: the rows' exponent bases; mexp: the same with -inf as 0 (the
-            // exponent's offset); mth: m + 2^8 in the log2 domain, the rescale
-            // threshold; l: this thread's partial row sums.  A row past the
-            // chunk's rows gets m = +inf: its weights are 0 and it never votes.
-            float m[RPT], mexp[RPT], mth[RPT], l[RPT];
+            // mb: the rows' exponent bases (log2 domain), set by the item's first
+            // tile (which always votes for new bases); l: this thread's partial
+            // row sums.  A row past the chunk's rows keeps mb = +inf: its
+            // weights are 0 and it never votes.  A row without a key yet keeps
+            // base 0 (its sum and O^T column are 0).
+            float mb[RPT], l[RPT];
 #pragma unroll
             for (int c = 0; c < RPT; ++c) {
-                const bool live = c0r + c < R;
-                m[c] = live ? -INFINITY : INFINITY;
-                mexp[c] = live ? 0.f : INFINITY;
-                mth[c] = m[c];
+                mb[c] = c0r + c < R ? 0.f : INFINITY;
                 l[c] = 0.f;
             }
             // keys past the context in its last block (the chunk's last
@@ -763,21 +774,21 @@ __global__ void __launch_bounds__(kMultiThreads, 1) paged_decode_multi_kernel(co
 #pragma unroll
                         for (int c = 0; c < RPT; ++c) {
                             s[c] *= sl2;
-                            exceed |= s[c] > mth[c];
+                            exceed |= s[c] > mb[c] + kRescaleLog2;
                         }
                     } else {
                         const int rlo = (pos >= w.ke ? C::NR : (pos <= w.c0 ? 0 : (pos - w.c0) * G)) - c0r;
 #pragma unroll
                         for (int c = 0; c < RPT; ++c) {
                             s[c] = c >= rlo ? s[c] * sl2 : -INFINITY;
-                            exceed |= s[c] > mth[c];
+                            exceed |= s[c] > mb[c] + kRescaleLog2;
                         }
                     }
                 }
                 // ---- one vote per tile: a wait gave up, or a row's base must move.
                 // Then every softmax thread leaves together, or the tile's row
                 // maxima over its 128 keys become the new bases.
-                if (multi_vote_any(exceed || !ok)) {
+                if (multi_vote_any(exceed || j == 0 || !ok)) {
                     if (multi_vote_any(!ok)) {
                         ok = false;
                         break;
@@ -796,7 +807,7 @@ __global__ void __launch_bounds__(kMultiThreads, 1) paged_decode_multi_kernel(co
                                                fmaxf(red[(4 * h + 2) * RPT + cc], red[(4 * h + 3) * RPT + cc]));
                         bool moved = false;  // the same on the threads of a row group: m and cm are
 #pragma unroll
-                        for (int c = 0; c < RPT; ++c) moved |= __shfl_sync(0xffffffffu, cm, c) > m[c];
+                        for (int c = 0; c < RPT; ++c) moved |= __shfl_sync(0xffffffffu, cm, c) > mb[c];
                         // O^T *= alpha once the previous P.V is done (the next one waits
                         // for this tile's P); on an item's first tile O^T is not started
                         const bool rescale_o = j > 0 && moved;
@@ -810,11 +821,12 @@ __global__ void __launch_bounds__(kMultiThreads, 1) paged_decode_multi_kernel(co
                         }
 #pragma unroll
                         for (int c = 0; c < RPT; ++c) {
-                            const float mn = fmaxf(m[c], __shfl_sync(0xffffffffu, cm, c));
-                            const float alpha = mn == m[c] ? 1.f : ex2_approx(m[c] - mn);  // 0 when m was -inf
-                            m[c] = mn;
-                            mexp[c] = mn == -INFINITY ? 0.f : mn;
-                            mth[c] = mn + kRescaleLog2;
+                            // the first tile starts the bases; a row past the chunk stays at +inf
+                            const float old = j == 0 && mb[c] != INFINITY ? -INFINITY : mb[c];
+                            float mn = fmaxf(old, __shfl_sync(0xffffffffu, cm, c));
+                            mn = mn == -INFINITY ? 0.f : mn;  // no key yet
+                            const float alpha = j == 0 || mn == mb[c] ? 1.f : ex2_approx(mb[c] - mn);
+                            mb[c] = mn;
                             l[c] *= alpha;
                             o[c] *= alpha;
                         }
@@ -825,12 +837,11 @@ __global__ void __launch_bounds__(kMultiThreads, 1) paged_decode_multi_kernel(co
                 // bits of P; lo: the exact remainder rounded, |lo| < 2^-7 |P|).  A
                 // row group past the chunk's rows skips it: P.V then mixes stale
                 // P^T rows into O^T columns that are never read.
-                float pv[RPT];
                 if (active) {
 #pragma unroll
                     for (int c = 0; c < RPT; ++c) {
-                        pv[c] = ex2_approx(s[c] - mexp[c]);
-                        l[c] += pv[c];
+                        s[c] = ex2_approx(s[c] - mb[c]);  // the weights, in place
+                        l[c] += s[c];
                     }
                 }
                 if (active && tt >= 2)
@@ -848,7 +859,7 @@ __global__ void __launch_bounds__(kMultiThreads, 1) paged_decode_multi_kernel(co
                         uint32_t hw[4], lw[4];
 #pragma unroll
                         for (int i = 0; i < 4; ++i) {
-                            const float a = pv[8 * q + 2 * i], b = pv[8 * q + 2 * i + 1];
+                            const float a = s[8 * q + 2 * i], b = s[8 * q + 2 * i + 1];
                             if constexpr (kBf16) {
                                 const uint32_t ba = __float_as_uint(a), bb = __float_as_uint(b);
                                 hw[i] = __byte_perm(ba, bb, 0x7632);  // the top 16 bits of each
@@ -904,7 +915,7 @@ __global__ void __launch_bounds__(kMultiThreads, 1) paged_decode_multi_kernel(co
                     if (lane < RPT) st_m[32 + c0r + lane] = cl;
                     if (lane == 0) {
 #pragma unroll
-                        for (int c = 0; c < RPT; ++c) st_m[c0r + c] = m[c];
+                        for (int c = 0; c < RPT; ++c) st_m[c0r + c] = mb[c];
                     }
                 }
                 mbar_arrive(&stat_full[it & 1]);
