@@ -357,9 +357,10 @@ size_t pkv_prefill_fp8_workspace_size(int num_chunks, int max_blocks_per_seq, in
  * Row i of chunk r (its n_r tokens are the last of its seq_lens[r] cached
  * tokens, written beforehand) attends causally to positions
  * j <= seq_lens[r] - n_r + i, exactly as pkv_paged_attention_prefill_chunk.
- * The n_r * G query rows that share a KV head go to the M side of warp
- * tensor-core MMAs (16 rows per warp) and the K/V stream in 16-token units,
- * split into partitions like decode (partials merged by a log-sum-exp kernel).
+ * On the tcgen05 tensor cores with the keys on the MMA's M side (128-key
+ * tiles) and the n_r * G <= 32 query rows that share a KV head on N; one
+ * persistent CTA per SM takes the (chunk, partition, KV head) items longest
+ * first; partials of split chunks are merged by a log-sum-exp kernel.
  *
  *   out, query, block_tables, seq_lens, query_start_loc   as for prefill_chunk
  *   max_q_len       host bound on n_r; max_q_len * (num_q_heads / num_kv_heads)
@@ -384,10 +385,11 @@ int pkv_paged_attention_decode_multi(void* out, const void* query, const void* k
                                      pkv_stream_t stream);
 
 /* Partition size (tokens) recommended for pkv_paged_attention_decode_multi:
- * enough partitions for about eight CTAs per SM, at least 256 tokens each, a
- * multiple of block_size, at most 4096 blocks (the per-partition limit the
- * call shares with pkv_paged_attention_decode); 0 = no split.  Negative
- * pkv_status on bad input. */
+ * 0 (no split) when there are at least two (chunk, KV head) items per SM,
+ * else enough partitions for that, at least 256 tokens each, in whole
+ * 128-key tiles (a multiple of block_size), at most 4096 blocks (the
+ * per-partition limit the call shares with pkv_paged_attention_decode).
+ * Negative pkv_status on bad input. */
 int pkv_decode_multi_partition_size(int num_chunks, int num_kv_heads, int block_size, int max_seq_len);
 
 /*
