@@ -66,21 +66,25 @@ struct PrefillCfg {
     static constexpr int PANEL = 64;
     static constexpr int Q_BYTES = NP * BM * 128;   // one query tile
     static constexpr int KT_BYTES = NP * BN * 128;  // one K (or V) tile
-    // bf16 keeps only 8 significant bits: P goes to the tensor cores as two
-    // bf16 terms (P = hi + lo: hi the top 16 bits of P, lo the remainder
-    // rounded, |lo| < 2^-7 |P|), which brings the rounding of the attention
-    // weights far below the output tolerance.  fp16 P is one term.
-    static constexpr bool SPLIT_P = Elem<T>::kCuType == CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+    // P.V runs in f16: P (below 2^8 under lazy rescaling) keeps 11
+    // significant bits, far below the output tolerance.  bf16 V tiles are
+    // widened in shared memory first, scaled by 2^-8 (exact for |v| in
+    // [2^-6, 1.6e7]; below, f16 subnormals keep an absolute error under
+    // 2^-25 * 2^8 = 7.6e-6; above 1.6e7 a value becomes inf); the epilogue
+    // scales O back by 2^8.  Q.K^T stays in the input type.
+    static constexpr bool WIDEN_V = Elem<T>::kCuType == CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+    // V stages: a stage is refilled once the P.V MMAs of its tile are done;
+    // widened tiles need a third stage to cover the conversion as well
+    static constexpr int NV = WIDEN_V ? 3 : 2;
     static constexpr int Q_OFF = 0;                       // [2] query tiles
     static constexpr int K_OFF = Q_OFF + 2 * Q_BYTES;     // [2] stages
-    static constexpr int V_OFF = K_OFF + 2 * KT_BYTES;    // [2] stages
-    static constexpr int BAR_OFF = V_OFF + 2 * KT_BYTES;
-    static constexpr int NBAR = 20;
+    static constexpr int V_OFF = K_OFF + 2 * KT_BYTES;    // [NV] stages
+    static constexpr int BAR_OFF = V_OFF + NV * KT_BYTES;
+    static constexpr int NBAR = 24;
     static constexpr int SMEM = 1024 + BAR_OFF + NBAR * 8;
     static constexpr uint32_t TMEM_COLS = 512;
     static constexpr uint32_t S_COL0 = 0;        // S (then P) of tile x at S_COL0 + 128 x
     static constexpr uint32_t O_COL0 = 256;      // O of tile x at O_COL0 + D x
-    static constexpr uint32_t PLO = BN / 2;      // P's lo term after the hi term (64 columns)
     static_assert(D == 64 || D == 128, "head_dim");
     static_assert(SMEM <= 227 * 1024, "shared memory");
 };
@@ -162,6 +166,14 @@ __device__ __forceinline__ bool prefill_item(const int32_t* seq_lens, const int3
     return true;
 }
 
+// Two bf16 values -> two f16 values times 2^-8 (the scaling is exact; f16
+// rounds the values below 2^-6 to its subnormal grid).
+__device__ __forceinline__ uint32_t widen_bf16x2_scaled(uint32_t u) {
+    const float lo = __uint_as_float(u << 16) * 0.00390625f;
+    const float hi = __uint_as_float(u & 0xFFFF0000u) * 0.00390625f;
+    return pack_half2(lo, hi);
+}
+
 __device__ __forceinline__ float fmax3(float a, float b, float c) {
     float d;
     asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
@@ -184,17 +196,19 @@ __global__ void __launch_bounds__(kPrefillThreads, 1) paged_prefill_kernel(const
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = align_1024(smem_raw);
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::BAR_OFF);
+    constexpr int NV = C::NV;
     uint64_t* q_full = bars + 0;
-    uint64_t* k_full = bars + 1;   // [2]  TMA landed
-    uint64_t* v_full = bars + 3;   // [2]
-    uint64_t* k_free = bars + 5;   // [2]  the S MMAs that read the stage are done (tcgen05.commit)
-    uint64_t* v_free = bars + 7;   // [2]  the P.V MMAs that read the stage are done
-    uint64_t* s_full = bars + 9;   // [2]  per tile: S_x(j) done
-    uint64_t* p_full = bars + 11;  // [2]  per tile: P_x(j) written (128 arrivals)
-    uint64_t* o_full = bars + 13;  // [2]  per tile: the tile's last P.V done
-    uint64_t* mma_done = bars + 15;
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 16);
-    volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + 17);
+    uint64_t* k_full = bars + 1;    // [2]  TMA landed
+    uint64_t* k_free = bars + 3;    // [2]  the S MMAs that read the stage are done (tcgen05.commit)
+    uint64_t* v_full = bars + 5;    // [NV]
+    uint64_t* v_free = bars + 8;    // [NV] the P.V MMAs that read the stage are done
+    uint64_t* v_ready = bars + 11;  // [NV] the V tile widened to f16 (256 arrivals; bf16 inputs)
+    uint64_t* s_full = bars + 14;   // [2]  per tile: S_x(j) done
+    uint64_t* p_full = bars + 16;   // [2]  per tile: P_x(j) written (128 arrivals)
+    uint64_t* o_full = bars + 18;   // [2]  per tile: the tile's last P.V done
+    uint64_t* mma_done = bars + 20;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 21);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + 22);
 
     // The CTA's (chunk, tile pair): KV head fastest; items longest first (see
     // prefill_item), or with many chunks, tile pair outermost, last pair first.
@@ -236,12 +250,15 @@ __global__ void __launch_bounds__(kPrefillThreads, 1) paged_prefill_kernel(const
         mbar_init(q_full, 1);
         for (int i = 0; i < 2; ++i) {
             mbar_init(&k_full[i], 1);
-            mbar_init(&v_full[i], 1);
             mbar_init(&k_free[i], 1);
-            mbar_init(&v_free[i], 1);
             mbar_init(&s_full[i], 1);
             mbar_init(&p_full[i], 128);
             mbar_init(&o_full[i], 1);
+        }
+        for (int i = 0; i < NV; ++i) {
+            mbar_init(&v_full[i], 1);
+            mbar_init(&v_free[i], 1);
+            mbar_init(&v_ready[i], 256);
         }
         mbar_init(mma_done, 1);
         *abort_flag = 0;
@@ -265,8 +282,8 @@ __global__ void __launch_bounds__(kPrefillThreads, 1) paged_prefill_kernel(const
             const int lb = j * per_tile + lane;
             return (lane < per_tile && lb < nblk) ? bt_row[lb] : -1;
         };
-        auto load_tile = [&](const CUtensorMap* map, int off, uint64_t* full, int j, int ids) {
-            const int st = j & 1;
+        auto load_tile = [&](const CUtensorMap* map, int off, uint64_t* full, int j, int ids, int nst) {
+            const int st = j % nst;
             uint8_t* dst = smem + off + st * C::KT_BYTES;
             const int lb = j * per_tile + lane;
             if (lane < per_tile && lb < nblk && (ids < 0 || ids >= p.num_blocks)) {
@@ -296,20 +313,29 @@ __global__ void __launch_bounds__(kPrefillThreads, 1) paged_prefill_kernel(const
         int ids = fetch_ids(0);
         int j = 0;
         for (; j < min(nkt, 2); ++j) {
-            load_tile(&tm_k, C::K_OFF, k_full, j, ids);
-            load_tile(&tm_v, C::V_OFF, v_full, j, ids);
+            load_tile(&tm_k, C::K_OFF, k_full, j, ids, 2);
+            load_tile(&tm_v, C::V_OFF, v_full, j, ids, NV);
             ids = fetch_ids(j + 1);
         }
-        // K of tile j once the S MMAs of tile j - 2 freed its stage; V once the P.V MMAs did.
         int loaded_k = j, loaded_v = j;
+        if (NV == 3 && j < nkt) {  // V runs one tile ahead of K
+            load_tile(&tm_v, C::V_OFF, v_full, j, ids, NV);
+            loaded_v = j + 1;
+        }
+        // K of tile j once the S MMAs of tile j - 2 freed its stage; V of tile
+        // j + NV - 2 once the P.V MMAs of tile j - 2 did.
         for (; j < nkt; ++j) {
             const int ids_next = fetch_ids(j + 1);
             if (!__all_sync(0xffffffffu, mbar_wait_or_abort(&k_free[j & 1], ((j - 2) >> 1) & 1, abort_flag))) break;
-            load_tile(&tm_k, C::K_OFF, k_full, j, ids);
+            load_tile(&tm_k, C::K_OFF, k_full, j, ids, 2);
             loaded_k = j + 1;
-            if (!__all_sync(0xffffffffu, mbar_wait_or_abort(&v_free[j & 1], ((j - 2) >> 1) & 1, abort_flag))) break;
-            load_tile(&tm_v, C::V_OFF, v_full, j, ids);
-            loaded_v = j + 1;
+            const int jv = j + NV - 2;
+            if (jv < nkt) {
+                if (!__all_sync(0xffffffffu, mbar_wait_or_abort(&v_free[jv % NV], ((jv - NV) / NV) & 1, abort_flag)))
+                    break;
+                load_tile(&tm_v, C::V_OFF, v_full, jv, NV == 2 ? ids : ids_next, NV);
+                loaded_v = jv + 1;
+            }
             ids = ids_next;
         }
         if (leader) {
@@ -318,25 +344,27 @@ __global__ void __launch_bounds__(kPrefillThreads, 1) paged_prefill_kernel(const
             // still be in flight and must land before the CTA exits.
             mbar_wait(q_full, 0);
             for (int t = max(0, loaded_k - 2); t < loaded_k; ++t) mbar_wait(&k_full[t & 1], (t >> 1) & 1);
-            for (int t = max(0, loaded_v - 2); t < loaded_v; ++t) mbar_wait(&v_full[t & 1], (t >> 1) & 1);
+            for (int t = max(0, loaded_v - NV); t < loaded_v; ++t) mbar_wait(&v_full[t % NV], (t / NV) & 1);
         }
     } else if (warp == kPrefillMmaWarp) {
         // ================================================================ MMA issue (lane 0)
         if ((tid & 31) == 0) {
             constexpr uint32_t IDESC_S = umma_idesc_f16(128, C::BN, kBf16, false, false);
-            constexpr uint32_t IDESC_O = umma_idesc_f16(128, D, kBf16, false, true);
+            constexpr uint32_t IDESC_O = umma_idesc_f16(128, D, false, false, true);  // f16 P and V
             // Shared-memory descriptors of every operand tile, made once: a
             // 16-element k slice is the tile's descriptor plus its byte offset / 16
             // (the start-address field), so issuing an MMA costs a few
             // instructions -- one thread issues fast enough for the tensor pipe
             // only without per-MMA descriptor arithmetic.
-            uint64_t qdesc[2], kdesc[2], vdesc[2];
+            uint64_t qdesc[2], kdesc[2], vdesc[NV];
 #pragma unroll
             for (int i = 0; i < 2; ++i) {
                 qdesc[i] = smem_desc_sw128(smem_u32(smem + C::Q_OFF + i * C::Q_BYTES), 16, 1024);
                 kdesc[i] = smem_desc_sw128(smem_u32(smem + C::K_OFF + i * C::KT_BYTES), 16, 1024);
-                vdesc[i] = smem_desc_sw128(smem_u32(smem + C::V_OFF + i * C::KT_BYTES), C::BN * 128, 1024);
             }
+#pragma unroll
+            for (int i = 0; i < NV; ++i)
+                vdesc[i] = smem_desc_sw128(smem_u32(smem + C::V_OFF + i * C::KT_BYTES), C::BN * 128, 1024);
             auto issue_s = [&](int x, int t) {  // S_x(t) = Q_x . K_t^T
                 const uint64_t qd = qdesc[x], kd = kdesc[t & 1];
                 const uint32_t s_col = C::S_COL0 + 128 * x;
@@ -353,13 +381,12 @@ __global__ void __launch_bounds__(kPrefillThreads, 1) paged_prefill_kernel(const
             // S_x(t + 1), issued after PV_x(t), also tells the softmax that O_x
             // holds every P.V before it.
             auto issue_pv = [&](int x, int t, bool last) {
-                const uint64_t vd = vdesc[t & 1];
+                const uint64_t vd = vdesc[t % NV];
                 const uint32_t p_col = C::S_COL0 + 128 * x, o_col = C::O_COL0 + D * x;
 #pragma unroll
                 for (int kk = 0; kk < C::BN / 16; ++kk) {
                     const uint64_t v = vd + kk * (16 * 128 / 16);  // 16 key rows of 128 bytes
                     umma_f16_ts(tmem + o_col, tmem + p_col + kk * 8, v, IDESC_O, t > 0 || kk > 0);
-                    if constexpr (C::SPLIT_P) umma_f16_ts(tmem + o_col, tmem + p_col + C::PLO + kk * 8, v, IDESC_O, 1);
                 }
                 if (last) umma_commit(&o_full[x]);
             };
@@ -373,7 +400,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1) paged_prefill_kernel(const
             for (int t = 0; ok && t < nkt; ++t) {
                 const bool next = t + 1 < nkt;
                 bool k_next = false;  // K_{t+1} landed (waited for once, when first needed)
-                ok = mbar_wait_or_abort(&v_full[t & 1], (t >> 1) & 1, abort_flag);
+                ok = mbar_wait_or_abort(C::WIDEN_V ? &v_ready[t % NV] : &v_full[t % NV], (t / NV) & 1, abort_flag);
                 for (int x = 0; ok && x < 2; ++x) {
                     const int nk = x == 0 ? nkt_a : nkt_b;
                     if (t >= nk) continue;
@@ -391,7 +418,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1) paged_prefill_kernel(const
                     }
                 }
                 if (ok) {
-                    umma_commit(&v_free[t & 1]);
+                    umma_commit(&v_free[t % NV]);
                     if (next) umma_commit(&k_free[(t + 1) & 1]);
                 }
             }
@@ -424,7 +451,40 @@ __global__ void __launch_bounds__(kPrefillThreads, 1) paged_prefill_kernel(const
         // reach O): tile a's, unless tile a stops one key tile earlier.
         const int jz = nkt - 1;
         const bool zeroes = (x == 0) == (jz < nkt_a);
-        for (int j = 0; j < nk; ++j) {
+        // bf16 inputs: this warpgroup's half of V tile jt's bytes (at head_dim
+        // 128, one of its two panels) to f16 times 2^-8, in place; the rows past
+        // the sequence end of the CTA's last key tile are zeroed instead.  Each
+        // warpgroup widens V(0) first and V(j + 1) after its P(j), while the
+        // tensor cores run P.V(j) and S(j + 1); P.V(j) waits for both halves.
+        auto widen_half = [&](int jt) -> bool {
+            if (!__all_sync(0xffffffffu, mbar_wait_or_abort(&v_full[jt % NV], (jt / NV) & 1, abort_flag)))
+                return false;
+            uint8_t* vs = smem + C::V_OFF + (jt % NV) * C::KT_BYTES;
+            const int tk0 = jt * C::BN;
+            const bool last = jt == nkt - 1;
+            const int dead_lo = last ? max(L, tk0) - tk0 : C::BN;  // tile rows [dead_lo, dead_hi)
+            const int dead_hi = last ? min(nblk * B, tk0 + C::BN) - tk0 : C::BN;
+            constexpr int HALF = C::KT_BYTES / 2;
+#pragma unroll 4
+            for (int off = x * HALF + row * 16; off < (x + 1) * HALF; off += 128 * 16) {
+                const int vrow = (off % (C::BN * 128)) / 128;
+                uint4 v = *reinterpret_cast<const uint4*>(vs + off);
+                if (vrow >= dead_lo && vrow < dead_hi) {
+                    v = make_uint4(0, 0, 0, 0);
+                } else {
+                    v.x = widen_bf16x2_scaled(v.x);
+                    v.y = widen_bf16x2_scaled(v.y);
+                    v.z = widen_bf16x2_scaled(v.z);
+                    v.w = widen_bf16x2_scaled(v.w);
+                }
+                *reinterpret_cast<uint4*>(vs + off) = v;
+            }
+            fence_proxy_async();  // the widened half -> the tensor cores' (async) proxy
+            mbar_arrive(&v_ready[jt % NV]);
+            return true;
+        };
+        if constexpr (C::WIDEN_V) ok = nkt > 0 && widen_half(0);
+        for (int j = 0; ok && j < nk; ++j) {
             if (!__all_sync(0xffffffffu, mbar_wait_or_abort(&s_full[x], j & 1, abort_flag))) {
                 ok = false;
                 break;
@@ -486,25 +546,15 @@ __global__ void __launch_bounds__(kPrefillThreads, 1) paged_prefill_kernel(const
             const float2 smul2 = make_float2(smul, smul), nm2 = make_float2(-mexp, -mexp);
 #pragma unroll
             for (int c = 0; c < C::BN / 32; ++c) {
-                uint32_t hi[16], lo[16];
+                uint32_t pw[16];  // f16 pairs
 #pragma unroll
                 for (int i = 0; i < 32; i += 2) {
                     const float2 arg = __ffma2_rn(make_float2(sv[c * 32 + i], sv[c * 32 + i + 1]), smul2, nm2);
                     const float p0 = ex2_approx(arg.x), p1 = ex2_approx(arg.y);
                     acc[(i / 2) & 1] = __fadd2_rn(acc[(i / 2) & 1], make_float2(p0, p1));
-                    if constexpr (C::SPLIT_P) {
-                        // hi = p truncated to bf16 (its top 16 bits); lo = the exact
-                        // remainder rounded to bf16, |lo| < 2^-7 |p|
-                        const uint32_t b0 = __float_as_uint(p0), b1 = __float_as_uint(p1);
-                        hi[i / 2] = __byte_perm(b0, b1, 0x7632);
-                        lo[i / 2] = Elem<T>::pack(p0 - __uint_as_float(b0 & 0xFFFF0000u),
-                                                  p1 - __uint_as_float(b1 & 0xFFFF0000u));
-                    } else {
-                        hi[i / 2] = Elem<T>::pack(p0, p1);
-                    }
+                    pw[i / 2] = pack_half2(p0, p1);
                 }
-                tmem_st16_nowait(ts + c * 16, hi);
-                if constexpr (C::SPLIT_P) tmem_st16_nowait(ts + C::PLO + c * 16, lo);
+                tmem_st16_nowait(ts + c * 16, pw);
             }
             lsum = lsum * alpha + ((acc[0].x + acc[0].y) + (acc[1].x + acc[1].y));
             // ---- O *= alpha: P.V of the previous tile is done (S_j, committed
@@ -520,15 +570,15 @@ __global__ void __launch_bounds__(kPrefillThreads, 1) paged_prefill_kernel(const
                 }
             }
             // ---- dead V rows of the last key tile
-            if (j == jz && zeroes) {
+            if (!C::WIDEN_V && j == jz && zeroes) {
                 const int tk0 = j * C::BN;
                 const int dead_lo = max(L, tk0), dead_hi = min(nblk * B, tk0 + C::BN);
                 if (dead_lo < dead_hi) {
-                    if (!__all_sync(0xffffffffu, mbar_wait_or_abort(&v_full[j & 1], (j >> 1) & 1, abort_flag))) {
+                    if (!__all_sync(0xffffffffu, mbar_wait_or_abort(&v_full[j % NV], (j / NV) & 1, abort_flag))) {
                         ok = false;
                         break;
                     }
-                    uint8_t* vs = smem + C::V_OFF + (j & 1) * C::KT_BYTES;
+                    uint8_t* vs = smem + C::V_OFF + (j % NV) * C::KT_BYTES;
                     const int rows = dead_hi - dead_lo;
                     for (int i = row; i < rows * C::NP * 8; i += 128) {
                         const int rr = (dead_lo - tk0) + i / (C::NP * 8);
@@ -542,12 +592,21 @@ __global__ void __launch_bounds__(kPrefillThreads, 1) paged_prefill_kernel(const
             tmem_wait_st();
             tc_fence_before();
             mbar_arrive(&p_full[x]);
+            if constexpr (C::WIDEN_V) {
+                if (j + 1 < nkt && !widen_half(j + 1)) {
+                    ok = false;
+                    break;
+                }
+            }
+        }
+        if constexpr (C::WIDEN_V) {  // tiles past this warpgroup's last (its query tile needs fewer)
+            for (int jt = max(nk + 1, 1); ok && jt < nkt; ++jt) ok = widen_half(jt);
         }
         if (ok && nk > 0) {
             if (__all_sync(0xffffffffu, mbar_wait_or_abort(&o_full[x], 0, abort_flag))) {
                 tc_fence_after();
                 const bool live = tok < n && !*abort_flag;
-                const float inv = p.out_scale / lsum;
+                const float inv = p.out_scale * (C::WIDEN_V ? 256.f : 1.f) / lsum;
                 TO* dst = reinterpret_cast<TO*>(p.out) +
                           (static_cast<int64_t>(q0 + tok) * p.num_q_heads + static_cast<int64_t>(g) * G + row % G) * D;
 #pragma unroll
