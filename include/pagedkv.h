@@ -295,7 +295,10 @@ int pkv_decode_partition_size(int num_seqs, int num_q_heads, int num_kv_heads, i
  * attends causally to positions j <= c0 + i:
  *     out[row][h] = sum_{j <= c0 + i} softmax_j(scale * q[row][h] . K_j) V_j.
  * The Q.K^T and P.V products run on the tcgen05 tensor cores (fp32
- * accumulation in tensor memory).
+ * accumulation in tensor memory).  P.V runs in f16: with bf16 inputs each V
+ * tile is widened in shared memory to f16 times 2^-8 (the output is scaled
+ * back), exact for |v| in [2^-6, 1.6e7], within 7.6e-6 absolute below that;
+ * a V element above 1.6e7 in magnitude becomes inf.
  *
  *   out, query      device [total_q_tokens, num_q_heads, head_dim], dtype
  *   block_tables    device int32 [num_chunks, max_blocks_per_seq]
