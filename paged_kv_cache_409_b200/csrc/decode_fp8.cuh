@@ -160,6 +160,9 @@ __global__ void __launch_bounds__(NW * 32, PKV_FP8_MIN_CTAS) paged_decode_fp8_ke
             float sc[MT][4];
 #pragma unroll
             for (int mt = 0; mt < MT; ++mt) {
+                // two accumulator chains (the h = 0 and h = 1 halves of each
+                // 32-dim step) halve the dependent MMA chain
+                float sc2[4] = {0.f, 0.f, 0.f, 0.f};
                 sc[mt][0] = sc[mt][1] = sc[mt][2] = sc[mt][3] = 0.f;
 #pragma unroll
                 for (int kp = 0; kp < KS / 2; ++kp) {
@@ -182,9 +185,14 @@ __global__ void __launch_bounds__(NW * 32, PKV_FP8_MIN_CTAS) paged_decode_fp8_ke
                                                f16x2_from_e4m3x2(static_cast<uint16_t>(bot)),
                                                f16x2_from_e4m3x2(static_cast<uint16_t>(top >> 16)),
                                                f16x2_from_e4m3x2(static_cast<uint16_t>(bot >> 16))};
-                        mma_16816<false>(sc[mt], a, qf[2 * kp + h][0], qf[2 * kp + h][1]);
+                        if (h == 0)
+                            mma_16816<false>(sc[mt], a, qf[2 * kp + h][0], qf[2 * kp + h][1]);
+                        else
+                            mma_16816<false>(sc2, a, qf[2 * kp + h][0], qf[2 * kp + h][1]);
                     }
                 }
+#pragma unroll
+                for (int e = 0; e < 4; ++e) sc[mt][e] += sc2[e];
             }
             // ---- online softmax per head column (log2 domain)
             float bmA = -INFINITY, bmB = -INFINITY;

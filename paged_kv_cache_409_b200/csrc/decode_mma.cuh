@@ -137,6 +137,9 @@ __global__ void __launch_bounds__(NW * 32) paged_decode_mma_kernel(const DecodeP
             float sc[MT][4];
 #pragma unroll
             for (int mt = 0; mt < MT; ++mt) {
+                // two accumulator chains (even / odd 16-dim steps) halve the
+                // dependent MMA chain
+                float sc2[4] = {0.f, 0.f, 0.f, 0.f};
                 sc[mt][0] = sc[mt][1] = sc[mt][2] = sc[mt][3] = 0.f;
 #pragma unroll
                 for (int ks = 0; ks < KS; ++ks) {
@@ -151,8 +154,13 @@ __global__ void __launch_bounds__(NW * 32) paged_decode_mma_kernel(const DecodeP
                         ldsm_x2(a[0], a[2], Ks + (ch / 8) * B * 128 + tok * 128 + (((ch % 8) ^ (tok & 7)) << 4));
                         a[1] = a[3] = 0u;
                     }
-                    mma_16816<kBf16>(sc[mt], a, qf[ks][0], qf[ks][1]);
+                    if (ks & 1)
+                        mma_16816<kBf16>(sc2, a, qf[ks][0], qf[ks][1]);
+                    else
+                        mma_16816<kBf16>(sc[mt], a, qf[ks][0], qf[ks][1]);
                 }
+#pragma unroll
+                for (int e = 0; e < 4; ++e) sc[mt][e] += sc2[e];
             }
             // ---- online softmax per head column (log2 domain)
             float bmA = -INFINITY, bmB = -INFINITY;
