@@ -396,14 +396,14 @@ class MultiTokenStep:
 # launch(es).
 TRAFFIC_CAPTURES = {
     "llama7b_decode_f16": {"case": "paged_decode_mma_kernel, the llama7b batch cut to 16 sequences",
-                           "read_mb": 287.470592, "write_mb": 3.234304, "algorithmic_mb": 285.38096},
+                           "read_mb": 287.47136, "write_mb": 3.24992, "algorithmic_mb": 285.38096},
     "mixed_step_bf16": {"case": "paged_decode_mma_kernel, the mixed step's decode cut to 8 sequences",
-                        "read_mb": 575.334656, "write_mb": 3.36512, "algorithmic_mb": 574.8748},
+                        "read_mb": 575.264768, "write_mb": 3.259648, "algorithmic_mb": 574.8748},
     "multi_token_decode_bf16": {"case": "paged_decode_multi_kernel (tcgen05, persistent), the 64-sequence batch",
                                 "read_mb": 588.89472, "write_mb": 4.645376, "algorithmic_mb": 586.926064},
     # the whole workload was captured (its distinct blocks fit the capture size rule): not scaled
     "shared_prefix_decode_f16": {"case": "paged_decode_mma_kernel, the whole shared-prefix workload",
-                                 "read_mb": 155.911168, "write_mb": 3.894784, "algorithmic_mb": 3227.190064,
+                                 "read_mb": 155.9552, "write_mb": 4.007168, "algorithmic_mb": 3227.190064,
                                  "whole": True},
 }
 
