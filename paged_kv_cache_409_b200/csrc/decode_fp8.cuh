@@ -29,10 +29,14 @@
 
 namespace pkv {
 
-template <int B, int G, int NST, int NW>
+// U consecutive blocks of a sequence form one unit (one stage, one softmax
+// step): at block 16 with 4 or 8 heads per KV head, 32-token units give every
+// step two independent 16-token S tiles and halve the per-block reductions,
+// shuffles and waits.
+template <int B, int G, int NST, int NW, int U>
 struct DecodeFp8Cfg {
     static constexpr int D = 128;
-    static constexpr int TILE = B * D;       // one block-head of K (or V): B rows of 128 bytes
+    static constexpr int TILE = B * U * D;   // one unit-head of K (or V): B * U rows of 128 bytes
     static constexpr int STAGE = 2 * TILE;
     static constexpr int STAGES_BYTES = NW * NST * STAGE;
     static constexpr int RED_BYTES = NW * G * (D + 2) * 4;  // the merge reuses the stage buffers
@@ -46,15 +50,16 @@ struct DecodeFp8Cfg {
 #define PKV_FP8_MIN_CTAS 1
 #endif
 
-template <typename T, int B, int G, int NST, int NW>
+template <typename T, int B, int G, int NST, int NW, int U>
 __global__ void __launch_bounds__(NW * 32, PKV_FP8_MIN_CTAS) paged_decode_fp8_kernel(const DecodeParams p,
                                                                    const __grid_constant__ CUtensorMap tm_k,
                                                                    const __grid_constant__ CUtensorMap tm_v) {
-    using C = DecodeFp8Cfg<B, G, NST, NW>;
+    using C = DecodeFp8Cfg<B, G, NST, NW, U>;
     constexpr int D = C::D;
     constexpr int kThreads = NW * 32;
-    constexpr int KS = D / 16;         // 16-dim chunks
-    constexpr int MT = (B + 15) / 16;  // 16-token tiles per block
+    constexpr int KS = D / 16;          // 16-dim chunks
+    constexpr int BU = B * U;           // tokens per unit
+    constexpr int MT = (BU + 15) / 16;  // 16-token tiles per unit
     static_assert(sizeof(T) == 2 && G >= 1 && G <= 8, "FP8 decode takes a 16-bit query and 1..8 heads");
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = align_1024(smem_raw);
@@ -96,19 +101,24 @@ __global__ void __launch_bounds__(NW * 32, PKV_FP8_MIN_CTAS) paged_decode_fp8_ke
 
     __syncthreads();
 
-    const int nw = nb > warp ? (nb - warp + NW - 1) / NW : 0;
+    const int nu = (nb + U - 1) / U;  // units of the partition
+    const int nw = nu > warp ? (nu - warp + NW - 1) / NW : 0;
     uint8_t* wstage = smem + warp * NST * C::STAGE;
     uint64_t* wbar = bars + warp * NST;
     const uint64_t policy = l2_policy_evict_first();
 
     auto issue = [&](int k) {  // lane 0 only
         const int st = k % NST;
-        const int id = bt_s[warp + k * NW];
-        const int coord = id >= 0 ? id : static_cast<int>(p.num_blocks);  // out of range: zero fill
         uint8_t* kd = wstage + st * C::STAGE;
         mbar_arrive_expect_tx(&wbar[st], C::STAGE);
-        tma_load_4d_hint(kd, &tm_k, 0, g, 0, coord, &wbar[st], policy);
-        tma_load_4d_hint(kd + C::TILE, &tm_v, 0, g, 0, coord, &wbar[st], policy);
+#pragma unroll
+        for (int i = 0; i < U; ++i) {
+            const int bi = (warp + k * NW) * U + i;
+            const int id = bi < nb ? bt_s[bi] : -1;
+            const int coord = id >= 0 ? id : static_cast<int>(p.num_blocks);  // out of range: zero fill
+            tma_load_4d_hint(kd + i * B * 128, &tm_k, 0, g, 0, coord, &wbar[st], policy);
+            tma_load_4d_hint(kd + C::TILE + i * B * 128, &tm_v, 0, g, 0, coord, &wbar[st], policy);
+        }
     };
     // Everything above reads only the tables and the lengths; the
     // pools may still be in the writes of a grid this one depends on (the
@@ -151,9 +161,15 @@ __global__ void __launch_bounds__(NW * 32, PKV_FP8_MIN_CTAS) paged_decode_fp8_ke
         const int st = k % NST;
         const bool ok = mbar_wait_main(&wbar[st], (k / NST) & 1);
         if (!__all_sync(0xffffffffu, ok)) break;
-        const int lb = b0 + warp + k * NW;
-        const int valid = min(B, ctx - lb * B);
-        if (bt_s[warp + k * NW] >= 0) {
+        const int u0 = (warp + k * NW) * U;  // the unit's first block in the partition
+        const int lb = b0 + u0;
+        // the unit's keys end at the partition's end or at a bad block id
+        // (flagged when the table was staged); the rest was loaded as zeros
+        int valid = min(BU, ctx - lb * B);
+#pragma unroll
+        for (int i = 1; i < U; ++i)
+            if (u0 + i >= nb || bt_s[u0 + i] < 0) valid = min(valid, i * B);
+        if (bt_s[u0] >= 0) {
             const uint8_t* Ks = wstage + st * C::STAGE;
             const uint8_t* Vs = Ks + C::TILE;
             // ---- S^T = K . Q^T
@@ -168,7 +184,7 @@ __global__ void __launch_bounds__(NW * 32, PKV_FP8_MIN_CTAS) paged_decode_fp8_ke
                 for (int kp = 0; kp < KS / 2; ++kp) {
                     // r[0]: token g, chunk 2kp; r[1]: token g + 8, chunk 2kp; r[2], r[3]: chunk 2kp + 1
                     uint32_t r[4];
-                    if constexpr (B >= 16) {
+                    if constexpr (BU >= 16) {
                         const int tok = 16 * mt + lr + 8 * (lm & 1);
                         const int ch = 2 * kp + (lm >> 1);
                         ldsm_x4(r, Ks + tok * 128 + ((ch ^ (tok & 7)) << 4));
@@ -259,7 +275,7 @@ __global__ void __launch_bounds__(NW * 32, PKV_FP8_MIN_CTAS) paged_decode_fp8_ke
                 for (int jp = 0; jp < KS / 2; ++jp) {
                     // r[0]: tokens 2c, 2c+1 x dims 2g, 2g+1 of chunk 2jp; r[1]: tokens + 8; r[2], r[3]: chunk 2jp + 1
                     uint32_t r[4];
-                    if constexpr (B >= 16) {
+                    if constexpr (BU >= 16) {
                         const int tok = 16 * kt + lr + 8 * (lm & 1);
                         const int ch = 2 * jp + (lm >> 1);
                         ldsm_x4_trans(r, Vs + tok * 128 + ((ch ^ (tok & 7)) << 4));

@@ -295,6 +295,9 @@ int decode_by_dim(int head_dim, int block_size, int group, const pkv::DecodePara
 #ifndef PKV_FP8_WARPS
 #define PKV_FP8_WARPS 4
 #endif
+#ifndef PKV_FP8_UNIT_TOKENS
+#define PKV_FP8_UNIT_TOKENS 32  // tokens per softmax step of the E4M3 decode with grouped heads
+#endif
 #ifndef PKV_FP8_STAGE_BUDGET
 #define PKV_FP8_STAGE_BUDGET 32768  // bytes of K/V stages per FP8 decode CTA
 #endif
@@ -302,12 +305,16 @@ int decode_by_dim(int head_dim, int block_size, int group, const pkv::DecodePara
 template <typename T, int B, int G>
 int launch_decode_fp8(const pkv::DecodeParams& prm, const CUtensorMap& tk, const CUtensorMap& tv, int grid,
                       const Launch& ln) {
-    constexpr int STAGE = 2 * B * 128;
+    // Blocks of 8 or 16 tokens are grouped into 32-token units for 4 or 8
+    // heads per KV head (+3 % on the gqa70b-shaped E4M3 batch, with twice the
+    // stage budget to keep two stages per warp; no gain with one head).
+    constexpr int U = (G >= 4 && B < PKV_FP8_UNIT_TOKENS) ? PKV_FP8_UNIT_TOKENS / B : 1;  // blocks per unit
+    constexpr int STAGE = 2 * B * U * 128;
     constexpr int NW = PKV_FP8_WARPS;
-    constexpr int NST = std::max(1, std::min(8, PKV_FP8_STAGE_BUDGET / (NW * STAGE)));
-    using C = pkv::DecodeFp8Cfg<B, G, NST, NW>;
+    constexpr int NST = std::max(1, std::min(8, (U > 1 ? 2 : 1) * PKV_FP8_STAGE_BUDGET / (NW * STAGE)));
+    using C = pkv::DecodeFp8Cfg<B, G, NST, NW, U>;
     static size_t configured[64] = {};
-    return launch_decode_kernel(pkv::paged_decode_fp8_kernel<T, B, G, NST, NW>, C::smem_bytes(prm.partition_blocks),
+    return launch_decode_kernel(pkv::paged_decode_fp8_kernel<T, B, G, NST, NW, U>, C::smem_bytes(prm.partition_blocks),
                                 NW * 32, prm, tk, tv, grid, ln, configured);
 }
 

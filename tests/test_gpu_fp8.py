@@ -82,7 +82,8 @@ def test_fp8_decode_matches_oracle(q, B, G):
     pre_k, pre_v = w.key_caches[0].clone(), w.value_caches[0].clone()
     ref, k_after, v_after, used = oracle_decode_step(w, pre_k=pre_k, pre_v=pre_v)
     to_device(w)
-    for part in (0, B, 4 * B):
+    # partitions of 1 and 3 blocks end inside a 32-token unit of grouped blocks
+    for part in (0, B, 3 * B, 4 * B):
         w.key_caches[0], w.value_caches[0] = pre_k.cuda(), pre_v.cuda()
         out = gpu_decode_step(w, partition_size=part)
         torch.cuda.synchronize()
