@@ -332,7 +332,8 @@ class MultiTokenStep:
         self.decode_bytes = self.kv_bytes + 2 * m.chunk_query.numel() * t + 4 * nblocks + 8 * len(m.seq_lens)
         self.tokens = int(m.chunk_lens.sum())
         self.kernel = ("paged_attention_prefill_chunk (tcgen05)" if via_prefill else
-                       "paged_attention_decode_multi (multi-token decode + merge kernels)")
+                       "paged_attention_decode_multi_step (append, then the multi-token decode as its "
+                       "programmatic dependent, + merge kernel)")
 
     def config(self):
         m = self.m
@@ -369,8 +370,14 @@ class MultiTokenStep:
 
     def run(self, timer=None, step=0):
         m, w = self.m, self.w
+        if timer is None and not self.via_prefill:  # append + attention as one library call
+            self.pkv.paged_attention_decode_multi_step(
+                m.append_keys, m.append_values, self.aslots, self.out, m.chunk_query, w.key_caches[0],
+                w.value_caches[0], self.cbt, self.csl, self.qsl, self.max_q, self.max_len, w.scale,
+                partition_size=self.part, workspace=self.ws)
+            return
         self.pkv.reshape_and_cache(m.append_keys, m.append_values, w.key_caches[0], w.value_caches[0], self.aslots)
-        if timer:
+        if timer:  # separate calls, so that events can bracket the attention
             timer.begin()
         self.run_units(step)
         if timer:

@@ -387,6 +387,23 @@ int pkv_paged_attention_decode_multi(void* out, const void* query, const void* k
                                      int partition_size, int dtype, void* workspace, size_t workspace_bytes,
                                      pkv_stream_t stream);
 
+/* One verification step in one call: pkv_reshape_and_cache of the step's
+ * num_new_tokens draft K/V rows (new_keys, new_values, slot_mapping as there;
+ * normally every chunk's n_r rows), then pkv_paged_attention_decode_multi.
+ * The attention grid is launched as the append's programmatic dependent: it
+ * reads the tables and lengths and sets up while the append drains, and
+ * reads the pools only after the append has completed.  Every check of both
+ * calls runs before the first launch, so a refused step (same statuses as
+ * the two calls) has changed nothing. */
+int pkv_paged_attention_decode_multi_step(const void* new_keys, const void* new_values, const int64_t* slot_mapping,
+                                          int64_t num_new_tokens, void* out, const void* query, void* key_cache,
+                                          void* value_cache, const int32_t* block_tables, const int32_t* seq_lens,
+                                          const int32_t* query_start_loc, int num_chunks, int64_t total_q_tokens,
+                                          int max_q_len, int max_seq_len, float scale, int num_q_heads,
+                                          int num_kv_heads, int head_dim, int block_size, int max_blocks_per_seq,
+                                          int64_t num_blocks, int partition_size, int dtype, void* workspace,
+                                          size_t workspace_bytes, pkv_stream_t stream);
+
 /* Partition size (tokens) recommended for pkv_paged_attention_decode_multi:
  * 0 (no split) when there are at least two (chunk, KV head) items per SM,
  * else enough partitions for that, at least 256 tokens each, in whole

@@ -22,6 +22,7 @@ from ._binding import (  # noqa: F401
     paged_attention_decode_step,
     paged_attention_decode_step_fp8,
     paged_attention_decode_multi,
+    paged_attention_decode_multi_step,
     paged_attention_prefill_chunk,
     paged_attention_prefill_chunk_fp8,
     reshape_and_cache,

@@ -45,6 +45,7 @@ EXPORTED = (
     "pkv_paged_attention_prefill_chunk_fp8",
     "pkv_prefill_fp8_workspace_size",
     "pkv_paged_attention_decode_multi",
+    "pkv_paged_attention_decode_multi_step",
     "pkv_decode_multi_partition_size",
     "pkv_get_device_error",
     "pkv_set_wait_limit_ns",
@@ -90,6 +91,8 @@ def load_library():
     lib.pkv_paged_attention_prefill_chunk.argtypes = [P, P, P, P, P, P, P, I, I64, I, F, I, I, I, I, I, I64, I, P]
     lib.pkv_paged_attention_decode_multi.argtypes = [P, P, P, P, P, P, P, I, I64, I, I, F, I, I, I, I, I, I64, I, I,
                                                      P, SZ, P]
+    lib.pkv_paged_attention_decode_multi_step.argtypes = [P, P, P, I64, P, P, P, P, P, P, P, I, I64, I, I, F, I, I,
+                                                          I, I, I, I64, I, I, P, SZ, P]
     lib.pkv_decode_multi_partition_size.argtypes = [I, I, I, I]
     lib.pkv_paged_attention_prefill_chunk_fp8.argtypes = [P, P, P, P, P, P, P, I, I64, I, F, F, F, I, I, I, I, I,
                                                           I64, I, P, SZ, P]
@@ -105,6 +108,7 @@ def load_library():
                  "pkv_copy_blocks", "pkv_swap_blocks", "pkv_paged_attention_decode",
                  "pkv_decode_partition_size", "pkv_paged_attention_prefill_chunk", "pkv_get_device_error",
                  "pkv_paged_attention_prefill_chunk_fp8", "pkv_paged_attention_decode_multi",
+                 "pkv_paged_attention_decode_multi_step",
                  "pkv_decode_multi_partition_size", "pkv_paged_attention_decode_step",
                  "pkv_paged_attention_decode_step_fp8", "pkv_set_wait_limit_ns"):
         getattr(lib, name).restype = I
@@ -446,6 +450,39 @@ def paged_attention_decode_multi(out, query, key_cache, value_cache, block_table
                                               MB, NB, int(partition_size), _code(query), ws_ptr, ws_bytes,
                                               _stream(stream))
     _ok(rc, "paged_attention_decode_multi")
+    return out
+
+
+def paged_attention_decode_multi_step(new_keys, new_values, slot_mapping, out, query, key_cache, value_cache,
+                                      block_tables, seq_lens, query_start_loc, max_q_len, max_seq_len, scale,
+                                      partition_size=None, workspace=None, stream=None):
+    """One verification step: ``reshape_and_cache(new_keys, new_values, ..., slot_mapping)`` then
+    ``paged_attention_decode_multi`` in one call (the attention launched as the append's
+    programmatic dependent)."""
+    lib = load_library()
+    Tq, Hq, D = query.shape
+    NB, B, Hkv, _ = key_cache.shape
+    R = seq_lens.numel()
+    MB = block_tables.shape[1]
+    for t, name in ((block_tables, "block_tables"), (seq_lens, "seq_lens"), (query_start_loc, "query_start_loc")):
+        if t.dtype != torch.int32:
+            raise ValueError(f"{name} must be int32")
+    if slot_mapping.dtype != torch.int64:
+        raise ValueError("slot_mapping must be int64")
+    if partition_size is None:
+        partition_size = decode_multi_partition_size(R, Hkv, B, max_seq_len)
+    need = decode_workspace_size(Tq, Hq, D, max_seq_len, partition_size) if partition_size else 0
+    if need and (workspace is None or workspace.numel() * workspace.element_size() < need):
+        workspace = torch.empty(need, dtype=torch.uint8, device=query.device)
+    ws_ptr = _dev(workspace, "workspace") if (need and workspace is not None) else None
+    ws_bytes = workspace.numel() * workspace.element_size() if ws_ptr else 0
+    rc = lib.pkv_paged_attention_decode_multi_step(
+        _dev(new_keys, "new_keys"), _dev(new_values, "new_values"), _dev(slot_mapping, "slot_mapping"),
+        new_keys.shape[0], _dev(out, "out"), _dev(query, "query"), _dev(key_cache, "key_cache"),
+        _dev(value_cache, "value_cache"), _dev(block_tables, "block_tables"), _dev(seq_lens, "seq_lens"),
+        _dev(query_start_loc, "query_start_loc"), R, Tq, int(max_q_len), int(max_seq_len), float(scale), Hq, Hkv, D,
+        B, MB, NB, int(partition_size), _code(query), ws_ptr, ws_bytes, _stream(stream))
+    _ok(rc, "paged_attention_decode_multi_step")
     return out
 
 

@@ -346,7 +346,7 @@ int decode_fp8_by_block(int block_size, int group, const pkv::DecodeParams& prm,
 // head_dim 128), at most one per item.
 template <typename T, int D>
 int launch_multi(const pkv::MultiParams& prm, int lpt, const CUtensorMap& tq, const CUtensorMap& tk,
-                 const CUtensorMap& tv, int64_t items, cudaStream_t s) {
+                 const CUtensorMap& tv, int64_t items, const Launch& ln) {
     using C = pkv::MultiCfg<D>;
     auto kern = pkv::paged_decode_multi_kernel<T, D>;
     int dev = 0;
@@ -361,9 +361,7 @@ int launch_multi(const pkv::MultiParams& prm, int lpt, const CUtensorMap& tq, co
         per_sm = n;
     }
     const int grid = (int)std::min<int64_t>(items, (int64_t)sm_count() * per_sm);
-    kern<<<grid, pkv::kMultiThreads, C::SMEM, s>>>(prm, lpt, tq, tk, tv);
-    PKV_CUDA(cudaGetLastError());
-    return PKV_OK;
+    return launch_kernel(kern, dim3(grid), dim3(pkv::kMultiThreads), C::SMEM, ln, prm, lpt, tq, tk, tv);
 }
 
 // The merge always follows this library's own decode kernel in the stream,
@@ -980,13 +978,19 @@ int pkv_paged_attention_prefill_chunk(void* out, const void* query, const void* 
                 : prefill_by_group<__half, 128>(group, prm, tq, tk, tv, (int)grid, s);
 }
 
-int pkv_paged_attention_decode_multi(void* out, const void* query, const void* key_cache, const void* value_cache,
-                                     const int32_t* block_tables, const int32_t* seq_lens,
-                                     const int32_t* query_start_loc, int num_chunks, int64_t total_q_tokens,
-                                     int max_q_len, int max_seq_len, float scale, int num_q_heads, int num_kv_heads,
-                                     int head_dim, int block_size, int max_blocks_per_seq, int64_t num_blocks,
-                                     int partition_size, int dtype, void* workspace, size_t workspace_bytes,
-                                     pkv_stream_t stream) {
+}  // extern "C"
+
+namespace {
+
+// The multi-token decode: every host check, then (unless check_only) the
+// launches; pdl launches the attention grid as the programmatic dependent of
+// the kernel before it on the stream (this library's append, in the step call).
+int decode_multi_impl(void* out, const void* query, const void* key_cache, const void* value_cache,
+                      const int32_t* block_tables, const int32_t* seq_lens, const int32_t* query_start_loc,
+                      int num_chunks, int64_t total_q_tokens, int max_q_len, int max_seq_len, float scale,
+                      int num_q_heads, int num_kv_heads, int head_dim, int block_size, int max_blocks_per_seq,
+                      int64_t num_blocks, int partition_size, int dtype, void* workspace, size_t workspace_bytes,
+                      pkv_stream_t stream, bool check_only, bool pdl) {
     if (dtype != PKV_F16 && dtype != PKV_BF16) return PKV_EUNSUPPORTED;
     if (num_chunks < 0 || total_q_tokens < 0 || max_q_len < 0 || max_seq_len < 0 || num_q_heads <= 0 ||
         num_kv_heads <= 0 || max_blocks_per_seq <= 0 || num_blocks <= 0 || partition_size < 0 ||
@@ -1038,6 +1042,7 @@ int pkv_paged_attention_decode_multi(void* out, const void* query, const void* k
                           max_seq_len, s);
         if (rc) return rc;
     }
+    if (check_only) return PKV_OK;
 
     CUtensorMap tq, tk, tv;
     // Q: 32 / G tokens x G heads = the 32 rows of a KV head; K/V: one box per block
@@ -1071,12 +1076,13 @@ int pkv_paged_attention_decode_multi(void* out, const void* query, const void* k
     prm.total_q_tokens = total_q_tokens;
     const int lpt = num_chunks <= pkv::kMultiLptChunks ? 1 : 0;
     const bool bf16 = dtype == PKV_BF16;
+    const Launch la{s, pdl};
     if (head_dim == 64)
-        rc = bf16 ? launch_multi<__nv_bfloat16, 64>(prm, lpt, tq, tk, tv, items, s)
-                  : launch_multi<__half, 64>(prm, lpt, tq, tk, tv, items, s);
+        rc = bf16 ? launch_multi<__nv_bfloat16, 64>(prm, lpt, tq, tk, tv, items, la)
+                  : launch_multi<__half, 64>(prm, lpt, tq, tk, tv, items, la);
     else
-        rc = bf16 ? launch_multi<__nv_bfloat16, 128>(prm, lpt, tq, tk, tv, items, s)
-                  : launch_multi<__half, 128>(prm, lpt, tq, tk, tv, items, s);
+        rc = bf16 ? launch_multi<__nv_bfloat16, 128>(prm, lpt, tq, tk, tv, items, la)
+                  : launch_multi<__half, 128>(prm, lpt, tq, tk, tv, items, la);
     if (rc || parts <= 1) return rc;
 
     pkv::MultiMergeParams mp;
@@ -1101,6 +1107,50 @@ int pkv_paged_attention_decode_multi(void* out, const void* query, const void* k
                     : launch_kernel(pkv::paged_decode_multi_merge_kernel<__half, 64>, mgrid, dim3(128), 0, ln, mp);
     return bf16 ? launch_kernel(pkv::paged_decode_multi_merge_kernel<__nv_bfloat16, 128>, mgrid, dim3(128), 0, ln, mp)
                 : launch_kernel(pkv::paged_decode_multi_merge_kernel<__half, 128>, mgrid, dim3(128), 0, ln, mp);
+}
+
+}  // namespace
+
+extern "C" {
+
+int pkv_paged_attention_decode_multi(void* out, const void* query, const void* key_cache, const void* value_cache,
+                                     const int32_t* block_tables, const int32_t* seq_lens,
+                                     const int32_t* query_start_loc, int num_chunks, int64_t total_q_tokens,
+                                     int max_q_len, int max_seq_len, float scale, int num_q_heads, int num_kv_heads,
+                                     int head_dim, int block_size, int max_blocks_per_seq, int64_t num_blocks,
+                                     int partition_size, int dtype, void* workspace, size_t workspace_bytes,
+                                     pkv_stream_t stream) {
+    return decode_multi_impl(out, query, key_cache, value_cache, block_tables, seq_lens, query_start_loc, num_chunks,
+                             total_q_tokens, max_q_len, max_seq_len, scale, num_q_heads, num_kv_heads, head_dim,
+                             block_size, max_blocks_per_seq, num_blocks, partition_size, dtype, workspace,
+                             workspace_bytes, stream, false, false);
+}
+
+int pkv_paged_attention_decode_multi_step(const void* new_keys, const void* new_values, const int64_t* slot_mapping,
+                                          int64_t num_new_tokens, void* out, const void* query, void* key_cache,
+                                          void* value_cache, const int32_t* block_tables, const int32_t* seq_lens,
+                                          const int32_t* query_start_loc, int num_chunks, int64_t total_q_tokens,
+                                          int max_q_len, int max_seq_len, float scale, int num_q_heads,
+                                          int num_kv_heads, int head_dim, int block_size, int max_blocks_per_seq,
+                                          int64_t num_blocks, int partition_size, int dtype, void* workspace,
+                                          size_t workspace_bytes, pkv_stream_t stream) {
+    // Every check of both calls before the first launch, so that a refused
+    // step has changed nothing.
+    int rc = decode_multi_impl(out, query, key_cache, value_cache, block_tables, seq_lens, query_start_loc,
+                               num_chunks, total_q_tokens, max_q_len, max_seq_len, scale, num_q_heads, num_kv_heads,
+                               head_dim, block_size, max_blocks_per_seq, num_blocks, partition_size, dtype, workspace,
+                               workspace_bytes, stream, true, false);
+    if (rc) return rc;
+    rc = reshape_check(new_keys, new_values, key_cache, value_cache, slot_mapping, num_new_tokens, num_kv_heads,
+                       head_dim, block_size, num_blocks, dtype, false);
+    if (rc) return rc;
+    rc = pkv_reshape_and_cache(new_keys, new_values, key_cache, value_cache, slot_mapping, num_new_tokens,
+                               num_kv_heads, head_dim, block_size, num_blocks, dtype, stream);
+    if (rc) return rc;
+    return decode_multi_impl(out, query, key_cache, value_cache, block_tables, seq_lens, query_start_loc, num_chunks,
+                             total_q_tokens, max_q_len, max_seq_len, scale, num_q_heads, num_kv_heads, head_dim,
+                             block_size, max_blocks_per_seq, num_blocks, partition_size, dtype, workspace,
+                             workspace_bytes, stream, false, /*pdl=*/num_new_tokens > 0);
 }
 
 int pkv_decode_multi_partition_size(int num_chunks, int num_kv_heads, int block_size, int max_seq_len) {

@@ -110,6 +110,35 @@ def test_multi_token_rescales_mid_partition(dtype):
         assert_close(out, ref, dtype, f"large scores, partition {part}")
 
 
+@pytest.mark.parametrize("case", [CASES[0], CASES[3], ROW_CASES[0]], ids=["case0", "case3", "rows0"])
+def test_multi_token_step_call(case):
+    """The one-call step (append, then the attention launched as its programmatic
+    dependent) writes the same pools and the same rows as the two calls, and
+    matches the oracle, with and without partitions."""
+    dtype, D, B, Hq, Hkv, c0s, ns = case
+    m = workloads.mixed_workload("mtst", [], c0s, ns, Hq, Hkv, D, B, dtype, seed=31 + sum(ns), poison=True)
+    pre_k, pre_v = m.decode.key_caches[0].clone(), m.decode.value_caches[0].clone()
+    ref = oracle_prefill_chunks(m, pre_k, pre_v)
+    dev = "cuda"
+    for part in (0, 2 * B):
+        two, k2, v2 = run_gpu(m, call="multi", partition_size=part)
+        kc, vc = pre_k.to(dev), pre_v.to(dev)
+        one = torch.empty_like(m.chunk_query, device=dev)
+        pkv.paged_attention_decode_multi_step(
+            m.append_keys.to(dev), m.append_values.to(dev), torch.from_numpy(m.append_slots).to(dev), one,
+            m.chunk_query.to(dev), kc, vc, torch.from_numpy(m.chunk_tables).to(dev),
+            torch.from_numpy(m.seq_lens).to(dev), torch.from_numpy(m.query_start_loc).to(dev),
+            int(m.chunk_lens.max()), int(m.seq_lens.max()), m.decode.scale, partition_size=part)
+        torch.cuda.synchronize()
+        assert pkv.get_device_error() == 0
+        # bit patterns: the poisoned free slots hold NaNs
+        assert torch.equal(kc.view(torch.int16), k2.view(torch.int16))
+        assert torch.equal(vc.view(torch.int16), v2.view(torch.int16))
+        assert torch.equal(one.view(torch.int16), two.view(torch.int16)), \
+            f"step call differs from the two calls, partition {part}"
+        assert_close(one, ref, dtype, f"multi-token step call {case} partition {part}")
+
+
 def test_multi_token_call_rejects_too_many_rows():
     q = torch.zeros(9, 32, 128, device="cuda", dtype=torch.float16)  # 9 tokens x G 4 = 36 rows > 32
     kc = torch.zeros(4, 16, 8, 128, device="cuda", dtype=torch.float16)
