@@ -408,6 +408,15 @@ TRAFFIC_CAPTURES = {
                         "read_mb": 575.264768, "write_mb": 3.259648, "algorithmic_mb": 574.8748},
     "multi_token_decode_bf16": {"case": "paged_decode_multi_kernel (tcgen05, persistent), the 64-sequence batch",
                                 "read_mb": 588.89472, "write_mb": 4.645376, "algorithmic_mb": 586.926064},
+    "llama7b_decode_fp8": {"case": "paged_decode_fp8_kernel, the llama7b batch on E4M3 pools cut to 32 sequences",
+                           "read_mb": 305.044736, "write_mb": 3.660288, "algorithmic_mb": 303.293652},
+    "gqa70b_decode_fp8": {"case": "paged_decode_fp8_kernel (32-token units), one gqa70b layer on E4M3 pools cut to "
+                                  "64 sequences",
+                          "read_mb": 171.1424, "write_mb": 3.097856, "algorithmic_mb": 171.248148},
+    "gqa70b_decode_bf16": {"case": "paged_decode_mma_kernel, one gqa70b layer cut to 64 sequences",
+                           "read_mb": 341.175808, "write_mb": 3.977472, "algorithmic_mb": 340.378132},
+    "mixed_step_fp8": {"case": "paged_decode_fp8_kernel, the E4M3 mixed step's decode cut to 8 sequences",
+                       "read_mb": 287.688448, "write_mb": 3.3216, "algorithmic_mb": 287.511728},
     # the whole workload was captured (its distinct blocks fit the capture size rule): not scaled
     "shared_prefix_decode_f16": {"case": "paged_decode_mma_kernel, the whole shared-prefix workload",
                                  "read_mb": 155.9552, "write_mb": 4.007168, "algorithmic_mb": 3227.190064,
