@@ -139,6 +139,43 @@ def test_multi_token_step_call(case):
         assert_close(one, ref, dtype, f"multi-token step call {case} partition {part}")
 
 
+def test_multi_token_step_refused_changes_nothing():
+    """A step the attention call refuses (9 tokens x 4 heads = 36 rows per KV head) returns before the
+    append: the pools keep their bytes."""
+    dev = "cuda"
+    q = torch.zeros(9, 32, 128, device=dev, dtype=torch.float16)
+    kc = torch.zeros(4, 16, 8, 128, device=dev, dtype=torch.float16)
+    vc = torch.zeros_like(kc)
+    nk = torch.ones(9, 8, 128, device=dev, dtype=torch.float16)
+    slots = torch.arange(9, dtype=torch.int64, device=dev)
+    bt = torch.zeros(1, 4, dtype=torch.int32, device=dev)
+    sl = torch.tensor([20], dtype=torch.int32, device=dev)
+    qsl = torch.tensor([0, 9], dtype=torch.int32, device=dev)
+    with pytest.raises(pkv.PagedKVError) as e:
+        pkv.paged_attention_decode_multi_step(nk, nk, slots, torch.empty_like(q), q, kc, vc, bt, sl, qsl, 9, 20, 0.1)
+    assert e.value.status == -2
+    torch.cuda.synchronize()
+    assert not kc.any() and not vc.any()
+
+
+def test_multi_token_step_without_new_tokens_is_the_attention_call():
+    """No draft rows to append: the step is the attention call alone (launched without the dependency)."""
+    dtype, D, B, Hq, Hkv, c0s, ns = CASES[1]
+    m = workloads.mixed_workload("mt0", [], c0s, ns, Hq, Hkv, D, B, dtype, seed=41, poison=True)
+    dev = "cuda"
+    two, kc, vc = run_gpu(m, call="multi", partition_size=0)  # appends, then attends
+    one = torch.empty_like(two)
+    empty_kv = torch.empty(0, Hkv, D, dtype=dtype, device=dev)
+    pkv.paged_attention_decode_multi_step(
+        empty_kv, empty_kv, torch.empty(0, dtype=torch.int64, device=dev), one, m.chunk_query.to(dev), kc, vc,
+        torch.from_numpy(m.chunk_tables).to(dev), torch.from_numpy(m.seq_lens).to(dev),
+        torch.from_numpy(m.query_start_loc).to(dev), int(m.chunk_lens.max()), int(m.seq_lens.max()),
+        m.decode.scale, partition_size=0)
+    torch.cuda.synchronize()
+    assert pkv.get_device_error() == 0
+    assert torch.equal(one.view(torch.int16), two.view(torch.int16))
+
+
 def test_multi_token_call_rejects_too_many_rows():
     q = torch.zeros(9, 32, 128, device="cuda", dtype=torch.float16)  # 9 tokens x G 4 = 36 rows > 32
     kc = torch.zeros(4, 16, 8, 128, device="cuda", dtype=torch.float16)
