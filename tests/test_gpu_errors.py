@@ -61,6 +61,29 @@ def test_bad_block_id_is_flagged_not_faulted():
     assert pkv.get_device_error() == 0  # reading clears it
 
 
+@pytest.mark.parametrize("B", [8, 16])
+def test_bad_block_id_in_an_e4m3_unit_is_flagged_not_faulted(B):
+    """E4M3 pools with 8 heads per KV head group blocks into 32-token steps: a bad id in the first
+    block of a step or inside one is skipped and flagged, and the other sequences' rows are unchanged."""
+    w = to_device(workloads.decode_workload("e8", [100, 200, 90], 16, 2, 128, B, torch.float16, seed=4,
+                                            fp8_scales=(0.05, 0.05)))
+    bt, cl, _ = gpu_tables(w)
+    ks, vs = w.extra["k_scale"], w.extra["v_scale"]
+    ref = torch.empty_like(w.queries[0])
+    pkv.paged_attention_decode_fp8(ref, w.queries[0], w.key_caches[0], w.value_caches[0], bt, cl, w.scale, ks, vs,
+                                   200, partition_size=0)
+    torch.cuda.synchronize()
+    assert pkv.get_device_error() == 0
+    for col in (0, 1, 3):  # first block of a unit, inside one, inside a later one
+        bad = bt.clone()
+        bad[1, col] = w.num_blocks + 77
+        out = torch.empty_like(ref)
+        pkv.paged_attention_decode_fp8(out, w.queries[0], w.key_caches[0], w.value_caches[0], bad, cl, w.scale, ks,
+                                       vs, 200, partition_size=0)
+        assert pkv.get_device_error() & pkv._binding.DEVERR_BLOCK_ID
+        assert torch.equal(out[0], ref[0]) and torch.equal(out[2], ref[2])
+
+
 def test_context_beyond_table_is_flagged():
     w, bt, cl, _ = small()
     cl[0] = bt.shape[1] * 16 + 5
