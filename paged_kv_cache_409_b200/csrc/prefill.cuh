@@ -16,12 +16,15 @@
 // Roles (320 threads):
 //  * warps 0-3 / 4-7 -- softmax of tile a / tile b, one thread per row (TMEM
 //    lane = row).  For key tile j: read the row of S_j (128 columns), take its
-//    max, write P_j = exp2(S_j * scale * log2 e - m) over the S columns (bf16:
-//    P = hi + lo, two terms), rescale O when the row max grew by more than
-//    2^8 (lazy rescaling), and signal the MMA warp.
-//  * warp 8 -- loader: the two Q tiles once, then K_j and V_j (two stages
-//    each) as soon as the MMAs that read the stage's previous tile are done.
-//    Its lanes prefetch the next tile's block ids, one per lane.
+//    max, write P_j = exp2(S_j * scale * log2 e - m) over the S columns as
+//    f16, rescale O when the row max grew by more than 2^8 (lazy rescaling),
+//    and signal the MMA warp.  With bf16 inputs each warpgroup then widens
+//    its half of the next V tile to f16 (times 2^-8) in shared memory, so
+//    that P.V runs as one f16 product.
+//  * warp 8 -- loader: the two Q tiles once, then K_j (two stages) and V_j
+//    (three stages for bf16, running one tile ahead of K) as soon as the MMAs
+//    that read the stage's previous tile are done.  Its lanes prefetch the
+//    next tile's block ids, one per lane.
 //  * warp 9 -- MMA issue (lane 0), in the order
 //        S_a(0) S_b(0) | PV_a(0) S_a(1) PV_b(0) S_b(1) | PV_a(1) S_a(2) ...
 //    so that while one tile's softmax runs, the tensor cores work on the
